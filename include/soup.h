@@ -1,0 +1,130 @@
+/*
+ * soup.h - C ABI of the B200 (sm_100a) layer-streamed LoRA training library.
+ *
+ * What the library computes (the method of the Soup "layer streaming" pages):
+ * LoRA fine-tuning over a frozen base model whose weights live in pinned host
+ * RAM as per-layer NF4 (or bf16) shards and are fed one decoder layer at a
+ * time into a small ring of preallocated device slots by a separate copy
+ * stream.  Each adapted projection computes  y = W x + (alpha/r) B A x;  the
+ * backward pass re-reads and recomputes the layer and produces
+ * dL/dx = W^T dL/dy plus the adapter terms, and dA, dB, while W stays frozen.
+ *
+ * Conventions for every entry point
+ *  - Every function returns a soup_status; SOUP_OK (0) on success.  On failure
+ *    soup_last_error() returns a message for the calling thread.  Nothing
+ *    aborts the process and no argument is silently clamped: an argument that
+ *    is out of range is refused.
+ *  - Pointers named *_dev, and all tensor pointers unless stated otherwise,
+ *    are CUDA device pointers owned by the caller.  The library allocates no
+ *    device memory except the slot arena of soup_stream_plan.
+ *  - "bf16" tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ *  - Matrices are row-major.  [R, C] means R rows of C contiguous elements.
+ *  - `stream` is a cudaStream_t passed as void*; work is enqueued on it and
+ *    the call returns without waiting, except where a function says it
+ *    synchronises.
+ *  - A kernel whose internal wait exceeds its time limit records a code in a
+ *    device error word instead of hanging; soup_device_error() reads it.
+ */
+#ifndef SOUP_H_
+#define SOUP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t soup_status;
+#define SOUP_OK 0
+#define SOUP_ERR_INVALID_ARG 1 /* null pointer, value out of range */
+#define SOUP_ERR_SHAPE 2       /* dimensions the kernels do not support */
+#define SOUP_ERR_ALIGN 3       /* pointer or stride misaligned */
+#define SOUP_ERR_NONFINITE 4   /* NaN or Inf in an input that must be finite */
+#define SOUP_ERR_OOM_PLAN 5    /* a stream plan does not fit the device cap */
+#define SOUP_ERR_TIMEOUT 6     /* a host wait or a kernel's bounded wait expired */
+#define SOUP_ERR_CUDA 7        /* a CUDA runtime call failed */
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char* soup_last_error(void);
+
+/* Reads and clears the device error word of the current device (synchronises
+ * the device).  *code_out = 0 when no kernel reported a problem; otherwise a
+ * nonzero code (1 = a bounded wait on an mbarrier expired in a GEMM).
+ * Returns SOUP_OK, or SOUP_ERR_CUDA if the read itself failed. */
+soup_status soup_device_error(int32_t* code_out);
+
+/* ------------------------------------------------------------------ NF4 ---
+ * NF4 block quantisation of the frozen base (the pages' `quantization: 4bit`
+ * storage of the streamed base; Soup pages, "configuration and training" and
+ * the published-numbers table).  Data type: QLoRA's 16-level NormalFloat
+ * codebook.  Blocks of 64 consecutive elements along the input dimension of a
+ * row share one fp32 absmax (no double quantisation).  A weight w in a block
+ * with absmax a gets the code of the codebook value nearest to fl32(w / a)
+ * (ties to the lower code); an all-zero block gets code 7 (exact zero).
+ * Packing: byte j of a row holds element 2j in bits 7..4 and 2j+1 in bits 3..0.
+ */
+
+/* W [out, in] fp32 -> codes [out, in/2] u8, absmax [out, in/64] fp32.
+ * in must be a positive multiple of 64.  flag_dev: caller-owned device int32
+ * used as scratch (the call zeroes it, the kernel sets it when it meets a
+ * non-finite weight).  This call SYNCHRONISES `stream` and returns
+ * SOUP_ERR_NONFINITE if any weight was NaN/Inf (codes/absmax are then
+ * unspecified). */
+soup_status soup_nf4_quantize(const float* W, int64_t out, int64_t in, uint8_t* codes,
+                              float* absmax, int32_t* flag_dev, void* stream);
+
+/* codes [out, in/2], absmax [out, in/64] -> W [out, in] bf16 where each value
+ * is round-to-nearest-even-to-bf16 of the fp32 product codebook[code]*absmax. */
+soup_status soup_nf4_dequant(const uint8_t* codes, const float* absmax, int64_t out,
+                             int64_t in, uint16_t* W_bf16, void* stream);
+
+/* ----------------------------------------------------------- LoRA linear ---
+ * One adapted projection, y = x W^T + s (x A^T) B^T with s = alpha/r
+ * (row-vector form of y = W x + (alpha/r) B A x), W frozen.
+ *
+ * Precision contract: bf16 operands, fp32 accumulation on tensor cores.  The
+ * down-projection result is stored as u_save = bf16(s * A x), transposed
+ * [r, ldT] with ldT = round_up(T, 8); the up-projection consumes that bf16
+ * value.  y is rounded once to bf16 from the fp32 sum.
+ */
+#define SOUP_WEIGHT_NF4 0
+#define SOUP_WEIGHT_BF16 1
+
+typedef struct soup_weight {
+  int32_t kind;          /* SOUP_WEIGHT_NF4 or SOUP_WEIGHT_BF16 */
+  int64_t out_features;  /* rows of W (N) */
+  int64_t in_features;   /* columns of W (K); a multiple of 64 */
+  const uint8_t* codes;  /* NF4: [out, in/2] */
+  const float* absmax;   /* NF4: [out, in/64] */
+  const uint16_t* w;     /* BF16: [out, in] */
+} soup_weight;
+
+/* Forward.  A [r, in] bf16, B [out, r] bf16 (r a multiple of 8, 8 <= r <= 64),
+ * x [T, in] bf16, y [T, out] bf16, u_save [r, round_up(T, 8)] bf16.
+ * T >= 1; out a multiple of 16; in a multiple of 64; all pointers 16-byte
+ * aligned. */
+soup_status soup_lora_linear_fwd(const soup_weight* W, const uint16_t* A, const uint16_t* B,
+                                 int32_t r, float scale, const uint16_t* x, int64_t T,
+                                 uint16_t* y, uint16_t* u_save, void* stream);
+
+/* Workspace bytes soup_lora_linear_bwd needs for (T, r, out). */
+size_t soup_lora_linear_bwd_workspace(int64_t T, int32_t r, int64_t out_features);
+
+/* Backward.  dy [T, out] bf16 -> dx [T, in] bf16, dA [r, in] fp32 and
+ * dB [out, r] fp32 (overwritten, not accumulated):
+ *   g' = bf16(s * dy B)        (stored transposed in the workspace)
+ *   dx = dy W + g' A,   dA = g'^T x,   dB = dy^T u_save^T
+ * u_save is the tensor soup_lora_linear_fwd wrote for the same x.
+ * workspace: device memory of at least soup_lora_linear_bwd_workspace() bytes,
+ * 256-byte aligned. */
+soup_status soup_lora_linear_bwd(const soup_weight* W, const uint16_t* A, const uint16_t* B,
+                                 int32_t r, float scale, const uint16_t* x,
+                                 const uint16_t* u_save, const uint16_t* dy, int64_t T,
+                                 uint16_t* dx, float* dA, float* dB, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SOUP_H_ */

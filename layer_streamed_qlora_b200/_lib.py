@@ -1,0 +1,123 @@
+"""ctypes binding of ``libsoup.so`` (the C ABI in ``include/soup.h``).
+
+Argument marshalling only: every function takes PyTorch tensors (device
+memory and streams come from PyTorch), passes their raw pointers and sizes to
+the C entry point of the same name, and raises ``SoupError`` on a nonzero
+status.  There is no fallback: if the library is missing, importing a function
+raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsoup.so")
+
+c_void_p, c_int32, c_int64, c_float, c_size_t = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                                  ctypes.c_float, ctypes.c_size_t)
+
+SOUP_WEIGHT_NF4 = 0
+SOUP_WEIGHT_BF16 = 1
+
+
+class SoupError(RuntimeError):
+    def __init__(self, fn, status, msg):
+        super().__init__(f"{fn} failed with status {status}: {msg}")
+        self.status = status
+
+
+class SoupWeight(ctypes.Structure):
+    _fields_ = [("kind", c_int32), ("out_features", c_int64), ("in_features", c_int64),
+                ("codes", c_void_p), ("absmax", c_void_p), ("w", c_void_p)]
+
+
+# name -> (restype, argtypes)
+_SIGS = {
+    "soup_last_error": (ctypes.c_char_p, []),
+    "soup_device_error": (c_int32, [ctypes.POINTER(c_int32)]),
+    "soup_nf4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "soup_nf4_dequant": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
+    "soup_lora_linear_fwd": (c_int32, [ctypes.POINTER(SoupWeight), c_void_p, c_void_p, c_int32, c_float,
+                                       c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
+    "soup_lora_linear_bwd_workspace": (c_size_t, [c_int64, c_int32, c_int64]),
+    "soup_lora_linear_bwd": (c_int32, [ctypes.POINTER(SoupWeight), c_void_p, c_void_p, c_int32, c_float,
+                                       c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_size_t, c_void_p]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m layer_streamed_qlora_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn, st):
+    if st != 0:
+        msg = lib().soup_last_error()
+        raise SoupError(fn, st, msg.decode() if msg else "")
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def device_error() -> int:
+    v = c_int32(0)
+    _check("soup_device_error", lib().soup_device_error(ctypes.byref(v)))
+    return v.value
+
+
+# ---------------------------------------------------------------- NF4
+def soup_nf4_quantize(W, codes, absmax, flag, stream=None):
+    out_f, in_f = W.shape
+    _check("soup_nf4_quantize", lib().soup_nf4_quantize(_p(W), out_f, in_f, _p(codes), _p(absmax), _p(flag),
+                                                        _stream(stream)))
+
+
+def soup_nf4_dequant(codes, absmax, out_f, in_f, W_bf16, stream=None):
+    _check("soup_nf4_dequant", lib().soup_nf4_dequant(_p(codes), _p(absmax), out_f, in_f, _p(W_bf16),
+                                                      _stream(stream)))
+
+
+# ---------------------------------------------------------------- weights
+def weight_nf4(codes, absmax, out_f, in_f) -> SoupWeight:
+    return SoupWeight(SOUP_WEIGHT_NF4, out_f, in_f, codes.data_ptr(), absmax.data_ptr(), None)
+
+
+def weight_bf16(w) -> SoupWeight:
+    return SoupWeight(SOUP_WEIGHT_BF16, w.shape[0], w.shape[1], None, None, w.data_ptr())
+
+
+# ---------------------------------------------------------------- LoRA linear
+def soup_lora_linear_fwd(W: SoupWeight, A, B, r, scale, x, T, y, u_save, stream=None):
+    _check("soup_lora_linear_fwd", lib().soup_lora_linear_fwd(ctypes.byref(W), _p(A), _p(B), r, scale, _p(x), T,
+                                                              _p(y), _p(u_save), _stream(stream)))
+
+
+def soup_lora_linear_bwd_workspace(T, r, out_f) -> int:
+    return int(lib().soup_lora_linear_bwd_workspace(T, r, out_f))
+
+
+def soup_lora_linear_bwd(W: SoupWeight, A, B, r, scale, x, u_save, dy, T, dx, dA, dB, workspace, stream=None):
+    _check("soup_lora_linear_bwd", lib().soup_lora_linear_bwd(
+        ctypes.byref(W), _p(A), _p(B), r, scale, _p(x), _p(u_save), _p(dy), T, _p(dx), _p(dA), _p(dB),
+        _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))

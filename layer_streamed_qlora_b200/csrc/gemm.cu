@@ -1,0 +1,544 @@
+// tcgen05 GEMM engine for sm_100a.
+//
+// D[M, N] (fp32, tensor memory) = A[M, K] * B[N, K]^T  (+ tailA * tailB^T)
+//
+// * 128 x BN x 64 CTA tiles, one CTA per SM (shared memory ~196 KB), a ring of
+//   STAGES shared-memory stages, warp-specialised:
+//     warp 0      one elected thread issues TMA loads (A, bf16 B, tail tiles)
+//     warp 1      allocates tensor memory; one elected thread issues
+//                 tcgen05.mma (M=128, N=BN, K=16) and tcgen05.commit
+//     warps 2..   NF4 modes: 8 warps decode the packed 4-bit weights straight
+//                 into the 128-byte-swizzled B stage (the "NF4 dequant
+//                 prologue"), then all of them run the epilogue;
+//                 bf16 modes: 4 epilogue warps.
+// * The LoRA up-projection is folded in as one extra K-block ("tail"): after
+//   the main loop the same accumulator receives u[M, r] * B_lora[N, r]^T
+//   (forward) or g'[M, r] * A_lora[r, N] (backward), so the adapter term costs
+//   at most one more 64-wide k-stage and no extra pass over y.
+// * Every mbarrier wait is bounded in time; on expiry the CTA records an error
+//   in the device error word and winds down (no hang).
+//
+// Operand layouts in shared memory (128-byte swizzle, 1024-byte atoms):
+//   K-major tile [rows, 64]: row i at i*128 bytes, 16-byte unit u stored at
+//     unit position u ^ (i % 8); descriptor SBO = 1024, k-step advance 32 B.
+//   MN-major tile [64 k-rows, 64*c MN]: chunk c (64 MN elements) at c*8192,
+//     k-row j at j*128, unit u at u ^ (j % 8); descriptor LBO = 8192 (chunk
+//     stride), SBO = 1024, k-step advance 2048 B.
+#include <cuda.h>
+
+#include "gemm.h"
+#include "nf4_codebook.cuh"
+#include "ptx.cuh"
+
+namespace soup {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
+
+template <int BN>
+struct Cfg {
+  static constexpr int B_STAGE = BN * BK * 2;
+  static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+  static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int LUT_BYTES = 16 * 32 * 4;
+  static constexpr int SMEM = 1024 + STAGES * (A_STAGE_BYTES + B_STAGE) + BAR_BYTES + LUT_BYTES;
+};
+
+struct KArgs {
+  int M, N, K, num_kb;
+  const uint8_t* codes;
+  const float* absmax;
+  int tail_ksteps, nseg;
+  int seg_end[4], seg_row[4];
+  int out_kind;
+  void* out;
+  long long ldo;
+  const uint16_t* resid;
+  long long ldr;
+  float alpha;
+  int vec_ok;
+  int* err;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// 8 NF4 codes (one 32-bit word: byte p holds element 2p high, 2p+1 low) ->
+// 8 bf16 values RNE(fp32(c * absmax)) packed in a uint4.
+__device__ __forceinline__ uint4 decode8(uint32_t w, const float* lut_lane, float am) {
+  uint32_t o[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t c0 = (w >> (8 * p + 4)) & 15u;
+    const uint32_t c1 = (w >> (8 * p)) & 15u;
+    const float f0 = lut_lane[c0 * 32] * am;
+    const float f1 = lut_lane[c1 * 32] * am;
+    o[p] = pack_bf16x2(f0, f1);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void st_shared_v4(void* p, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ptx::smem_u32(p)), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+template <int NWORDS>
+__device__ __forceinline__ void load_codes(const uint8_t* src, uint32_t (&w)[NWORDS]) {
+  if constexpr (NWORDS == 8) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else if constexpr (NWORDS == 4) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+  } else {
+    const uint2 a = __ldg(reinterpret_cast<const uint2*>(src));
+    w[0] = a.x; w[1] = a.y;
+  }
+}
+
+template <int BN, int AMJ, int BMD>
+__global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmTA,
+                const __grid_constant__ CUtensorMap tmTB, const KArgs args) {
+  using C = Cfg<BN>;
+  constexpr bool NF4 = BMD >= B_NF4_K;
+  constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
+  constexpr int STAGES = C::STAGES;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* lut = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * BM;
+  const int n0 = blockIdx.y * BN;
+  const int num_kb = args.num_kb;
+  const int n_iters = num_kb + (args.tail_ksteps > 0 ? 1 : 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1 + (NF4 ? 8 : 0));
+      ptx::mbar_init(&empty[s], 1);
+    }
+    ptx::mbar_init(accf, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmA);
+    if (!NF4) ptx::prefetch_tmap(&tmB);
+    if (args.tail_ksteps > 0) {
+      ptx::prefetch_tmap(&tmTA);
+      ptx::prefetch_tmap(&tmTB);
+    }
+  }
+  if (NF4 && threadIdx.x >= 64) {
+    for (int i = threadIdx.x - 64; i < 16 * 32; i += 256) lut[i] = __uint_as_float(nf4_code_bits(i >> 5));
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // tail row offset of this tile's N segment (no dynamic indexing of the
+  // parameter arrays, which would spill them to local memory)
+  int tail_row = args.seg_row[0];
+  if (args.nseg > 1 && n0 >= args.seg_end[0]) tail_row = args.seg_row[1];
+  if (args.nseg > 2 && n0 >= args.seg_end[1]) tail_row = args.seg_row[2];
+  if (args.nseg > 3 && n0 >= args.seg_end[2]) tail_row = args.seg_row[3];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+          atomicOr(args.err, 1);
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* a = sA + s * A_STAGE_BYTES;
+        uint8_t* b = sB + s * C::B_STAGE;
+        const bool tail = it >= num_kb;
+        const uint32_t bytes = A_STAGE_BYTES + ((!NF4 || tail) ? C::B_STAGE : 0);
+        ptx::mbar_arrive_expect_tx(&full[s], bytes);
+        if (!tail) {
+          const int k0 = it * BK;
+          if (AMJ == A_K) {
+            ptx::tma_load_2d(a, &tmA, &full[s], k0, m0);
+          } else {
+            ptx::tma_load_2d(a, &tmA, &full[s], m0, k0);
+            ptx::tma_load_2d(a + 8192, &tmA, &full[s], m0 + 64, k0);
+          }
+          if (!NF4) {
+            if (!B_MN) {
+              ptx::tma_load_2d(b, &tmB, &full[s], k0, n0);
+            } else {
+#pragma unroll
+              for (int c = 0; c < BN / 64; ++c) ptx::tma_load_2d(b + c * 8192, &tmB, &full[s], n0 + 64 * c, k0);
+            }
+          }
+        } else {
+          ptx::tma_load_2d(a, &tmTA, &full[s], m0, tail_row);
+          ptx::tma_load_2d(a + 8192, &tmTA, &full[s], m0 + 64, tail_row);
+          if (!B_MN) {
+            ptx::tma_load_2d(b, &tmTB, &full[s], 0, n0);
+          } else {
+#pragma unroll
+            for (int c = 0; c < (BN >= 64 ? BN / 64 : 1); ++c)
+              ptx::tma_load_2d(b + c * 8192, &tmTB, &full[s], n0 + 64 * c, 0);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_main = ptx::idesc_bf16(BM, BN, AMJ, B_MN ? 1 : 0);
+      constexpr uint32_t idesc_tail = ptx::idesc_bf16(BM, BN, 1, B_MN ? 1 : 0);
+      bool ok = true;
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!ptx::mbar_wait_bounded(&full[s], ph, abort_flag)) {
+          atomicOr(args.err, 1);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t a_base = ptx::smem_u32(sA + s * A_STAGE_BYTES);
+        const uint32_t b_base = ptx::smem_u32(sB + s * C::B_STAGE);
+        const bool tail = it >= num_kb;
+        const int nk = tail ? args.tail_ksteps : BK / 16;
+        const bool a_mn = tail || AMJ == A_MN;
+        for (int k = 0; k < nk; ++k) {
+          const uint64_t ad = a_mn ? ptx::smem_desc_sw128(a_base + k * 2048, 8192, 1024)
+                                   : ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
+          const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k * 2048, 8192, 1024)
+                                   : ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
+          ptx::mma_bf16(tmem, ad, bd, tail ? idesc_tail : idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(&empty[s]);
+      }
+      if (ok) ptx::mma_commit(accf);
+    }
+  } else {
+    const int t = threadIdx.x - 64;  // 0 .. (NF4 ? 255 : 127)
+    if constexpr (NF4) {
+      // ----------------------------------------------------- NF4 decode warps
+      const float* lut_lane = lut + lane;
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+          atomicOr(args.err, 1);
+          *abort_flag = 1;
+          break;
+        }
+        if (it < num_kb) {
+          uint8_t* b = sB + s * C::B_STAGE;
+          if constexpr (BMD == B_NF4_K) {
+            // B tile [BN rows n, 64 k]: codes [N, K/2], one absmax per row per stage
+            constexpr int TPR = 256 / BN;      // threads per row
+            constexpr int EPT = 64 / TPR;      // elements per thread
+            constexpr int NW = EPT / 8;        // 32-bit code words per thread
+            const int row = t / TPR, h = t % TPR;
+            const int n = n0 + row;
+            uint32_t w[NW];
+            float am = 0.f;
+            if (n < args.N) {
+              load_codes(args.codes + (size_t)n * (args.K / 2) + (size_t)it * 32 + h * (EPT / 2), w);
+              am = __ldg(args.absmax + (size_t)n * (args.K / 64) + it);
+            }
+#pragma unroll
+            for (int u = 0; u < NW; ++u) {
+              const int unit = h * NW + u;
+              const uint4 v = (n < args.N) ? decode8(w[u], lut_lane, am) : make_uint4(0, 0, 0, 0);
+              st_shared_v4(b + row * 128 + ((unit ^ (row & 7)) << 4), v);
+            }
+          } else {
+            // B tile [64 k-rows, BN cols]: codes [K, N/2], absmax [K, N/64]
+            constexpr int CPT = BN / 4;        // columns per thread
+            constexpr int NW = CPT / 8;
+            const int kr = t & 63, q = t >> 6;
+            const int k = it * BK + kr;
+            const int c0 = q * CPT;
+            uint32_t w[NW];
+            float am = 0.f;
+            if (k < args.K) {
+              load_codes(args.codes + (size_t)k * (args.N / 2) + (n0 + c0) / 2, w);
+              am = __ldg(args.absmax + (size_t)k * (args.N / 64) + (n0 + c0) / 64);
+            }
+#pragma unroll
+            for (int u = 0; u < NW; ++u) {
+              const int col = c0 + 8 * u;
+              const int chunk = col >> 6, unit = (col >> 3) & 7;
+              const uint4 v = (k < args.K) ? decode8(w[u], lut_lane, am) : make_uint4(0, 0, 0, 0);
+              st_shared_v4(b + chunk * 8192 + kr * 128 + ((unit ^ (kr & 7)) << 4), v);
+            }
+          }
+          ptx::fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&full[s]);
+      }
+    }
+    // ------------------------------------------------------------ epilogue
+    constexpr int NEPI = NF4 ? 8 : 4;
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const bool got = ptx::mbar_wait_bounded(accf, 0, abort_flag);
+    if (!got) {
+      atomicOr(args.err, 1);
+      *abort_flag = 1;
+    } else {
+      ptx::tc_fence_after();
+      const int row = m0 + q * 32 + lane;
+      const bool row_ok = row < args.M;
+      constexpr int NCH = BN / 16;
+      for (int ch = (NEPI == 8 ? ew / 4 : 0); ch < NCH; ch += (NEPI == 8 ? 2 : 1)) {
+        uint32_t v[16];
+        ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + ch * 16, v);
+        ptx::tmem_ld_wait();
+        const int n = n0 + ch * 16;
+        if (!row_ok || n >= args.N) continue;
+        float f[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * args.alpha;
+        const bool full16 = (n + 16 <= args.N);
+        if (args.out_kind == OUT_BF16) {
+          uint16_t* o = static_cast<uint16_t*>(args.out) + (size_t)row * args.ldo + n;
+          if (args.resid) {
+            const uint16_t* r = args.resid + (size_t)row * args.ldr + n;
+            if (args.vec_ok && full16) {
+              const uint4 r0 = *reinterpret_cast<const uint4*>(r);
+              const uint4 r1 = *reinterpret_cast<const uint4*>(r + 8);
+              const uint32_t rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                f[2 * i] += bf16_to_f32(rr[i] & 0xFFFF);
+                f[2 * i + 1] += bf16_to_f32(rr[i] >> 16);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (n + i < args.N) f[i] += bf16_to_f32(r[i]);
+            }
+          }
+          if (args.vec_ok && full16) {
+            uint32_t p[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) p[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+            reinterpret_cast<uint4*>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
+            reinterpret_cast<uint4*>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (n + i < args.N) {
+                __nv_bfloat16 h = __float2bfloat16_rn(f[i]);
+                o[i] = *reinterpret_cast<uint16_t*>(&h);
+              }
+          }
+        } else if (args.out_kind == OUT_F32) {
+          float* o = static_cast<float*>(args.out) + (size_t)row * args.ldo + n;
+          if (args.vec_ok && full16) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              reinterpret_cast<float4*>(o)[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (n + i < args.N) o[i] = f[i];
+          }
+        } else if (args.out_kind == OUT_BF16_T) {
+          uint16_t* o = static_cast<uint16_t*>(args.out);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (n + i < args.N) {
+              __nv_bfloat16 h = __float2bfloat16_rn(f[i]);
+              o[(size_t)(n + i) * args.ldo + row] = *reinterpret_cast<uint16_t*>(&h);
+            }
+        } else {
+          float* o = static_cast<float*>(args.out);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (n + i < args.N) o[(size_t)(n + i) * args.ldo + row] = f[i];
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    // let copies and MMAs already in flight land before the CTA releases its
+    // shared and tensor memory (bounded: ~1 ms)
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000LL) {
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------- host side
+constexpr int CU_DT_BF16 = 9;       // CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+constexpr int CU_SWIZZLE_128B = 3;  // CU_TENSOR_MAP_SWIZZLE_128B
+constexpr int CU_L2_256B = 3;       // CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+
+soup_status make_map(CUtensorMap* m, const Mat& mat, uint32_t box0, uint32_t box1, const char* what) {
+  SOUP_CHECK(mat.ptr && mat.rows > 0 && mat.cols > 0, SOUP_ERR_INVALID_ARG, "gemm: %s is empty", what);
+  SOUP_CHECK(soup_aligned(mat.ptr, 16), SOUP_ERR_ALIGN, "gemm: %s base not 16-byte aligned", what);
+  SOUP_CHECK((mat.ld * 2) % 16 == 0 && mat.ld >= mat.cols, SOUP_ERR_ALIGN,
+             "gemm: %s row stride %lld elements is not a multiple of 8 (or < cols)", what,
+             (long long)mat.ld);
+  EncodeTiledFn enc = encode_tiled();
+  SOUP_CHECK(enc != nullptr, SOUP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const uint64_t gdim[2] = {(uint64_t)mat.cols, (uint64_t)mat.rows};
+  const uint64_t gstride[1] = {(uint64_t)mat.ld * 2};
+  const uint32_t box[2] = {box0, box1};
+  const uint32_t estr[2] = {1, 1};
+  int r = enc(m, CU_DT_BF16, 2, const_cast<void*>(mat.ptr), gdim, gstride, box, estr, 0,
+              CU_SWIZZLE_128B, CU_L2_256B, 0);
+  SOUP_CHECK(r == 0, SOUP_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, r);
+  return SOUP_OK;
+}
+
+template <int BN, int AMJ, int BMD>
+soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
+  using C = Cfg<BN>;
+  CUtensorMap mA, mB, mTA, mTB;
+  memset(&mA, 0, sizeof(mA));
+  memset(&mB, 0, sizeof(mB));
+  memset(&mTA, 0, sizeof(mTA));
+  memset(&mTB, 0, sizeof(mTB));
+  if (AMJ == A_K) SOUP_TRY(make_map(&mA, d.A, 64, 128, "A"));
+  else SOUP_TRY(make_map(&mA, d.A, 64, 64, "A (MN-major)"));
+  constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
+  if (BMD == B_TMA_K) SOUP_TRY(make_map(&mB, d.B, 64, BN, "B"));
+  if (BMD == B_TMA_MN) SOUP_TRY(make_map(&mB, d.B, 64, 64, "B (MN-major)"));
+  if (d.tail_ksteps > 0) {
+    SOUP_TRY(make_map(&mTA, d.tailA, 64, 64, "tail A"));
+    if (!B_MN) SOUP_TRY(make_map(&mTB, d.tailB, 64, BN, "tail B"));
+    else SOUP_TRY(make_map(&mTB, d.tailB, 64, 64, "tail B (MN-major)"));
+  }
+  auto kern = gemm_kernel<BN, AMJ, BMD>;
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    SOUP_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    attr_set = true;
+  }
+  constexpr int NT = 32 * (2 + (BMD >= B_NF4_K ? 8 : 4));
+  dim3 grid((d.M + BM - 1) / BM, (d.N + BN - 1) / BN);
+  kern<<<grid, NT, C::SMEM, st>>>(mA, mB, mTA, mTB, ka);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+int pick_bn(const GemmDesc& d) {
+  if (d.bn) return d.bn;
+  const bool nf4 = d.b_mode >= B_NF4_K;
+  const bool mn = d.b_mode == B_TMA_MN || d.b_mode == B_NF4_MN;
+  auto fits = [&](int bn) {
+    for (int i = 0; i < d.nseg - 1; ++i)
+      if (d.seg_end[i] % bn) return false;
+    return true;
+  };
+  if (!nf4 && !mn && d.N <= 64) return ((d.N + 15) / 16) * 16 == 64 ? 64 : ((d.N + 15) / 16) * 16;
+  if (d.N >= 256 && (d.N % 256 == 0 || d.N >= 1024) && fits(256)) return 256;
+  if (d.N >= 128 && fits(128)) return 128;
+  return 64;
+}
+
+}  // namespace
+
+soup_status gemm(const GemmDesc& d, cudaStream_t st) {
+  SOUP_CHECK(d.M > 0 && d.N > 0 && d.K > 0, SOUP_ERR_SHAPE, "gemm: empty problem %dx%dx%d", d.M, d.N, d.K);
+  SOUP_CHECK(d.out != nullptr, SOUP_ERR_INVALID_ARG, "gemm: null output");
+  SOUP_CHECK(d.tail_ksteps >= 0 && d.tail_ksteps <= 4, SOUP_ERR_SHAPE, "gemm: tail_ksteps %d", d.tail_ksteps);
+  SOUP_CHECK(d.nseg >= 1 && d.nseg <= 4, SOUP_ERR_SHAPE, "gemm: nseg %d", d.nseg);
+  const bool nf4 = d.b_mode >= B_NF4_K;
+  if (nf4) {
+    SOUP_CHECK(d.codes && d.absmax, SOUP_ERR_INVALID_ARG, "gemm: NF4 operand missing");
+    SOUP_CHECK(d.a_major == A_K, SOUP_ERR_SHAPE, "gemm: NF4 B needs a K-major A");
+    SOUP_CHECK(d.K % 64 == 0, SOUP_ERR_SHAPE, "gemm: NF4 needs K %% 64 == 0 (K=%d)", d.K);
+    if (d.b_mode == B_NF4_MN)
+      SOUP_CHECK(d.N % 64 == 0, SOUP_ERR_SHAPE, "gemm: NF4 (transposed) needs N %% 64 == 0");
+    const size_t need = d.b_mode == B_NF4_K ? 32 : 16;
+    SOUP_CHECK(soup_aligned(d.codes, need), SOUP_ERR_ALIGN, "gemm: NF4 codes misaligned");
+  }
+  const int bn = pick_bn(d);
+  for (int i = 0; i < d.nseg - 1; ++i)
+    SOUP_CHECK(d.seg_end[i] % bn == 0, SOUP_ERR_SHAPE, "gemm: segment end %d not a multiple of the tile %d",
+               d.seg_end[i], bn);
+  KArgs ka;
+  memset(&ka, 0, sizeof(ka));
+  ka.M = d.M; ka.N = d.N; ka.K = d.K;
+  ka.num_kb = (d.K + BK - 1) / BK;
+  ka.codes = d.codes; ka.absmax = d.absmax;
+  ka.tail_ksteps = d.tail_ksteps; ka.nseg = d.nseg;
+  for (int i = 0; i < 4; ++i) { ka.seg_end[i] = d.seg_end[i]; ka.seg_row[i] = d.seg_row[i]; }
+  ka.out_kind = d.out_kind; ka.out = d.out; ka.ldo = d.ldo;
+  ka.resid = d.resid; ka.ldr = d.ldr; ka.alpha = d.alpha;
+  const int esz = (d.out_kind == OUT_BF16 || d.out_kind == OUT_BF16_T) ? 2 : 4;
+  ka.vec_ok = soup_aligned(d.out, 16) && ((d.ldo * esz) % 16 == 0) &&
+              (!d.resid || (soup_aligned(d.resid, 16) && (d.ldr * 2) % 16 == 0));
+  ka.err = device_error_word();
+  SOUP_CHECK(ka.err != nullptr, SOUP_ERR_CUDA, "device error word unavailable");
+
+#define SOUP_GEMM_CASE(BN_, AM_, BMD_) \
+  if (bn == BN_ && d.a_major == AM_ && d.b_mode == BMD_) return launch<BN_, AM_, BMD_>(d, ka, st);
+  SOUP_GEMM_CASE(256, A_K, B_NF4_K)
+  SOUP_GEMM_CASE(128, A_K, B_NF4_K)
+  SOUP_GEMM_CASE(64, A_K, B_NF4_K)
+  SOUP_GEMM_CASE(256, A_K, B_NF4_MN)
+  SOUP_GEMM_CASE(128, A_K, B_NF4_MN)
+  SOUP_GEMM_CASE(64, A_K, B_NF4_MN)
+  SOUP_GEMM_CASE(256, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(128, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(64, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(48, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(32, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(16, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(256, A_K, B_TMA_MN)
+  SOUP_GEMM_CASE(128, A_K, B_TMA_MN)
+  SOUP_GEMM_CASE(64, A_K, B_TMA_MN)
+  SOUP_GEMM_CASE(64, A_MN, B_TMA_K)
+  SOUP_GEMM_CASE(48, A_MN, B_TMA_K)
+  SOUP_GEMM_CASE(32, A_MN, B_TMA_K)
+  SOUP_GEMM_CASE(16, A_MN, B_TMA_K)
+#undef SOUP_GEMM_CASE
+  return fail(SOUP_ERR_SHAPE, "gemm: no kernel for BN=%d a_major=%d b_mode=%d (M=%d N=%d K=%d)", bn,
+              d.a_major, d.b_mode, d.M, d.N, d.K);
+}
+
+}  // namespace soup

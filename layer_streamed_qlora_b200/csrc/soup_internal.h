@@ -1,0 +1,62 @@
+// Internal host-side helpers shared by the library's translation units:
+// status codes, the thread-local last-error string, argument checks and the
+// device error word that bounded waits in kernels report into.
+#pragma once
+
+#include <cstdint>
+#include <cstdio>
+#include <cuda_runtime.h>
+
+#include "../../include/soup.h"
+
+namespace soup {
+
+// Records a formatted message as the calling thread's last error and returns `st`.
+soup_status fail(soup_status st, const char* fmt, ...);
+void clear_error();
+
+// Device-side error word for the current device (set by kernels whose bounded
+// waits expired; read by soup_device_error()).
+int* device_error_word();
+
+// cuTensorMapEncodeTiled resolved through the runtime's driver entry point.
+typedef int (*EncodeTiledFn)(void* tmap, int dtype, uint32_t rank, void* gaddr,
+                             const uint64_t* gdim, const uint64_t* gstride,
+                             const uint32_t* box, const uint32_t* estride, int interleave,
+                             int swizzle, int l2promo, int oobfill);
+EncodeTiledFn encode_tiled();
+
+int sm_count();
+
+}  // namespace soup
+
+#define SOUP_CUDA_TRY(expr)                                                            \
+  do {                                                                                 \
+    cudaError_t e__ = (expr);                                                          \
+    if (e__ != cudaSuccess)                                                            \
+      return ::soup::fail(SOUP_ERR_CUDA, "%s: %s (%s:%d)", #expr, cudaGetErrorString(e__), \
+                          __FILE__, __LINE__);                                         \
+  } while (0)
+
+#define SOUP_CHECK(cond, st, ...)                  \
+  do {                                             \
+    if (!(cond)) return ::soup::fail((st), __VA_ARGS__); \
+  } while (0)
+
+#define SOUP_TRY(expr)                   \
+  do {                                   \
+    soup_status s__ = (expr);            \
+    if (s__ != SOUP_OK) return s__;      \
+  } while (0)
+
+#define SOUP_LAUNCH_CHECK()                                                            \
+  do {                                                                                 \
+    cudaError_t e__ = cudaGetLastError();                                              \
+    if (e__ != cudaSuccess)                                                            \
+      return ::soup::fail(SOUP_ERR_CUDA, "kernel launch: %s (%s:%d)", cudaGetErrorString(e__), \
+                          __FILE__, __LINE__);                                         \
+  } while (0)
+
+static inline bool soup_aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}

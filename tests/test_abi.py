@@ -1,0 +1,59 @@
+"""CPU checks of the C ABI: the library builds for sm_100a, loads, and exports
+every function that include/*.h declares.  No compute call is made (there is
+no GPU here)."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        names |= set(re.findall(r"\b(soup_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def libpath():
+    from layer_streamed_qlora_b200 import build
+    return build.build()
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for n in ("soup_nf4_quantize", "soup_nf4_dequant", "soup_lora_linear_fwd", "soup_lora_linear_bwd"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(libpath):
+    out = subprocess.run(["nm", "-D", "--defined-only", libpath], capture_output=True, text=True, check=True).stdout
+    syms = {l.split()[-1] for l in out.splitlines() if l.strip()}
+    missing = [n for n in _declared() if n not in syms]
+    assert not missing, missing
+
+
+def test_library_loads_and_binds(libpath):
+    from layer_streamed_qlora_b200 import _lib
+    L = _lib.lib()
+    for n in _declared():
+        assert hasattr(L, n)
+    # pure host queries work without a GPU
+    assert _lib.soup_lora_linear_bwd_workspace(64, 8, 512) > 0
+    assert L.soup_last_error() is not None
+
+
+def test_library_is_sm100a_only(libpath):
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", libpath], capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    arches = set(re.findall(r"sm_(\d+a?)", out.stdout))
+    assert arches == {"100a"}, arches
