@@ -124,6 +124,74 @@ soup_status soup_lora_linear_bwd(const soup_weight* W, const uint16_t* A, const 
                                  uint16_t* dx, float* dA, float* dB, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* --------------------------------------------------------- decoder layer ---
+ * One Llama-style decoder layer with LoRA on all seven projections (the unit
+ * the pages stream "one decoder layer at a time"; Soup pages, "layer
+ * streaming" and "how layer streaming works"):
+ *   x1 = RMSNorm(h; norm1); q,k,v = LoRA projections of x1; RoPE(q, k);
+ *   h2 = h + LoRA_o(causal GQA attention(q, k, v));
+ *   x2 = RMSNorm(h2; norm2); h_out = h2 + LoRA_down(silu(LoRA_gate(x2)) * LoRA_up(x2)).
+ * RMSNorm y = x / sqrt(mean(x^2) + eps) * w (w frozen); RoPE rotates pairs
+ * (i, i + d/2) by pos * theta^(-2i/d), positions restarting in every sequence;
+ * attention scale 1/sqrt(d), kv head = q_head / (Hq / Hkv); no biases.
+ * Activations are [T, features] bf16 with T = batch * seq (batch-major).
+ */
+typedef struct soup_layer_cfg {
+  int32_t hidden;        /* H: a multiple of 256 */
+  int32_t n_q_heads;     /* Hq */
+  int32_t n_kv_heads;    /* Hkv: divides Hq */
+  int32_t head_dim;      /* d: must be 128 */
+  int32_t intermediate;  /* I: a multiple of 128 */
+  int32_t rank;          /* r: must be 16 */
+  float alpha;           /* LoRA scale s = alpha / r */
+  float eps;             /* RMSNorm epsilon */
+  float theta;           /* RoPE base */
+} soup_layer_cfg;
+
+/* The frozen base of one layer (all NF4 or all bf16), as it sits in a device
+ * slot.  Fused row layouts: qkv = [q; k; v] rows ([(Hq + 2 Hkv) d, H]),
+ * gate_up = [gate; up] rows ([2 I, H]); o [H, Hq d]; down [H, I]. */
+typedef struct soup_layer_weights {
+  soup_weight qkv, o, gate_up, down;
+  const uint16_t* norm1; /* [H] bf16 */
+  const uint16_t* norm2; /* [H] bf16 */
+} soup_layer_weights;
+
+/* LoRA factors (bf16), concatenated in the same row order as the base:
+ * A_qkv [3r, H] = [A_q; A_k; A_v], B_qkv [(Hq + 2 Hkv) d, r] = [B_q; B_k; B_v],
+ * A_o [r, Hq d], B_o [H, r], A_gu [2r, H] = [A_gate; A_up],
+ * B_gu [2I, r] = [B_gate; B_up], A_down [r, I], B_down [H, r]. */
+typedef struct soup_layer_lora {
+  const uint16_t *A_qkv, *B_qkv, *A_o, *B_o, *A_gu, *B_gu, *A_down, *B_down;
+} soup_layer_lora;
+
+/* fp32 gradients of the LoRA factors, same shapes as soup_layer_lora
+ * (overwritten by soup_decoder_layer_bwd). */
+typedef struct soup_layer_grads {
+  float *dA_qkv, *dB_qkv, *dA_o, *dB_o, *dA_gu, *dB_gu, *dA_down, *dB_down;
+} soup_layer_grads;
+
+/* Workspace bytes the layer calls need for (batch, seq). */
+size_t soup_decoder_layer_workspace(const soup_layer_cfg* cfg, int64_t batch, int64_t seq);
+
+/* Forward: h_in [T, H] bf16 -> h_out [T, H] bf16.  adapters_on = 0 drops
+ * every LoRA term (the adapters-off reference model used for DPO).
+ * workspace: >= soup_decoder_layer_workspace bytes, 256-byte aligned. */
+soup_status soup_decoder_layer_fwd(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                   const soup_layer_cfg* cfg, const uint16_t* h_in, int64_t batch,
+                                   int64_t seq, uint16_t* h_out, int32_t adapters_on, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/* Recompute-backward: re-runs the forward from h_in (keeping intermediates),
+ * then back-propagates dh_out [T, H] fp32 (gradient w.r.t. h_out) to
+ * dh_in [T, H] fp32 and fills the LoRA gradients.  W gets no gradient.
+ * dh_in may alias dh_out.  With adapters_on = 0 the grads are not written. */
+soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                   const soup_layer_cfg* cfg, const uint16_t* h_in,
+                                   const float* dh_out, int64_t batch, int64_t seq, float* dh_in,
+                                   const soup_layer_grads* grads, int32_t adapters_on,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -34,6 +34,26 @@ class SoupWeight(ctypes.Structure):
                 ("codes", c_void_p), ("absmax", c_void_p), ("w", c_void_p)]
 
 
+class LayerCfg(ctypes.Structure):
+    _fields_ = [("hidden", c_int32), ("n_q_heads", c_int32), ("n_kv_heads", c_int32), ("head_dim", c_int32),
+                ("intermediate", c_int32), ("rank", c_int32), ("alpha", c_float), ("eps", c_float),
+                ("theta", c_float)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("qkv", SoupWeight), ("o", SoupWeight), ("gate_up", SoupWeight), ("down", SoupWeight),
+                ("norm1", c_void_p), ("norm2", c_void_p)]
+
+
+class LayerLora(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in ("A_qkv", "B_qkv", "A_o", "B_o", "A_gu", "B_gu", "A_down", "B_down")]
+
+
+class LayerGrads(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in ("dA_qkv", "dB_qkv", "dA_o", "dB_o", "dA_gu", "dB_gu", "dA_down",
+                                        "dB_down")]
+
+
 # name -> (restype, argtypes)
 _SIGS = {
     "soup_last_error": (ctypes.c_char_p, []),
@@ -46,6 +66,13 @@ _SIGS = {
     "soup_lora_linear_bwd": (c_int32, [ctypes.POINTER(SoupWeight), c_void_p, c_void_p, c_int32, c_float,
                                        c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_size_t, c_void_p]),
+    "soup_decoder_layer_workspace": (c_size_t, [ctypes.POINTER(LayerCfg), c_int64, c_int64]),
+    "soup_decoder_layer_fwd": (c_int32, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerLora),
+                                         ctypes.POINTER(LayerCfg), c_void_p, c_int64, c_int64, c_void_p, c_int32,
+                                         c_void_p, c_size_t, c_void_p]),
+    "soup_decoder_layer_bwd": (c_int32, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerLora),
+                                         ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_int64, c_int64, c_void_p,
+                                         ctypes.POINTER(LayerGrads), c_int32, c_void_p, c_size_t, c_void_p]),
 }
 
 _lib = None
@@ -120,4 +147,41 @@ def soup_lora_linear_bwd_workspace(T, r, out_f) -> int:
 def soup_lora_linear_bwd(W: SoupWeight, A, B, r, scale, x, u_save, dy, T, dx, dA, dB, workspace, stream=None):
     _check("soup_lora_linear_bwd", lib().soup_lora_linear_bwd(
         ctypes.byref(W), _p(A), _p(B), r, scale, _p(x), _p(u_save), _p(dy), T, _p(dx), _p(dA), _p(dB),
+        _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- decoder layer
+def layer_cfg(shape) -> LayerCfg:
+    return LayerCfg(shape.hidden, shape.n_q_heads, shape.n_kv_heads, shape.head_dim, shape.intermediate,
+                    shape.rank, float(shape.alpha), float(shape.eps), float(shape.theta))
+
+
+def layer_lora(t: dict) -> LayerLora:
+    return LayerLora(*[t[n].data_ptr() for n in ("A_qkv", "B_qkv", "A_o", "B_o", "A_gu", "B_gu", "A_down",
+                                                 "B_down")])
+
+
+def layer_grads(t: dict) -> LayerGrads:
+    return LayerGrads(*[t[n].data_ptr() for n in ("dA_qkv", "dB_qkv", "dA_o", "dB_o", "dA_gu", "dB_gu",
+                                                  "dA_down", "dB_down")])
+
+
+def soup_decoder_layer_workspace(cfg: LayerCfg, batch, seq) -> int:
+    return int(lib().soup_decoder_layer_workspace(ctypes.byref(cfg), batch, seq))
+
+
+def soup_decoder_layer_fwd(W: LayerWeights, lora, cfg: LayerCfg, h_in, batch, seq, h_out, adapters_on, workspace,
+                           stream=None):
+    lp = ctypes.byref(lora) if lora is not None else None
+    _check("soup_decoder_layer_fwd", lib().soup_decoder_layer_fwd(
+        ctypes.byref(W), lp, ctypes.byref(cfg), _p(h_in), batch, seq, _p(h_out), int(adapters_on), _p(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def soup_decoder_layer_bwd(W: LayerWeights, lora, cfg: LayerCfg, h_in, dh_out, batch, seq, dh_in, grads,
+                           adapters_on, workspace, stream=None):
+    lp = ctypes.byref(lora) if lora is not None else None
+    gp = ctypes.byref(grads) if grads is not None else None
+    _check("soup_decoder_layer_bwd", lib().soup_decoder_layer_bwd(
+        ctypes.byref(W), lp, ctypes.byref(cfg), _p(h_in), _p(dh_out), batch, seq, _p(dh_in), gp, int(adapters_on),
         _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))

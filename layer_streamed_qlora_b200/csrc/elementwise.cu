@@ -1,0 +1,226 @@
+// Memory-bound kernels of the decoder layer: RMSNorm forward/backward, the
+// RoPE angle table, the attention-backward row dot D = rowsum(dO * O), and
+// dtype conversions.  (RoPE itself is applied in the QKV GEMM epilogue and in
+// the attention-backward epilogues; SwiGLU in the gate|up and down GEMM
+// epilogues.)  All accesses are 16-byte
+// vectorised and coalesced; row reductions use warp shuffles.  Layouts are
+// token-major: [T, features] with T = batch * seq.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "elementwise.h"
+
+namespace soup {
+namespace {
+
+__device__ __forceinline__ float b2f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+__device__ __forceinline__ uint16_t f2b(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+__device__ __forceinline__ void unpack8(const uint4 v, float* f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Loads 8 consecutive elements of row `row` (chunk c8) from bf16 or fp32 storage.
+__device__ __forceinline__ void load8(const uint16_t* xb, const float* xf, size_t off, float* f) {
+  if (xf) {
+    const float4 a = reinterpret_cast<const float4*>(xf + off)[0];
+    const float4 b = reinterpret_cast<const float4*>(xf + off)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  } else {
+    unpack8(*reinterpret_cast<const uint4*>(xb + off), f);
+  }
+}
+
+// One warp per row; H % 256 == 0 so every lane owns H/256 chunks of 8.
+__global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ xf,
+                                   const uint16_t* __restrict__ w, int T, int H, float eps, uint16_t* __restrict__ y,
+                                   float* __restrict__ rinv) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= T) return;
+  const size_t rb = (size_t)row * H;
+  float ss = 0.f;
+  const int nch = H / 256;
+  for (int c = 0; c < nch; ++c) {
+    float f[8];
+    load8(x, xf, rb + (size_t)(c * 32 + lane) * 8, f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss += f[i] * f[i];
+  }
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / (float)H + eps);
+  if (lane == 0 && rinv) rinv[row] = r;
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  uint4* yr = reinterpret_cast<uint4*>(y + rb);
+  for (int c = 0; c < nch; ++c) {
+    float f[8], g[8];
+    load8(x, xf, rb + (size_t)(c * 32 + lane) * 8, f);
+    unpack8(wr[c * 32 + lane], g);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = (f[i] * r) * g[i];
+    yr[c * 32 + lane] = pack8(f);
+  }
+}
+
+// dh = dres + rinv * (dy*w - xh * mean(dy*w*xh)),  xh = x * rinv
+__global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ xf,
+                                   const uint16_t* __restrict__ w, const float* __restrict__ rinv,
+                                   const uint16_t* __restrict__ dy, const float* __restrict__ dres, int T, int H,
+                                   float* __restrict__ dh, uint16_t* __restrict__ dh_bf16) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= T) return;
+  const float r = rinv[row];
+  const size_t rb = (size_t)row * H;
+  const uint4* dyr = reinterpret_cast<const uint4*>(dy + rb);
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  const int nch = H / 256;
+  float dot = 0.f;
+  for (int c = 0; c < nch; ++c) {
+    float a[8], b[8], g[8];
+    load8(x, xf, rb + (size_t)(c * 32 + lane) * 8, a);
+    unpack8(dyr[c * 32 + lane], b);
+    unpack8(wr[c * 32 + lane], g);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dot += (b[i] * g[i]) * (a[i] * r);
+  }
+  dot = warp_sum(dot) / (float)H;
+  for (int c = 0; c < nch; ++c) {
+    float a[8], b[8], g[8], o[8];
+    load8(x, xf, rb + (size_t)(c * 32 + lane) * 8, a);
+    unpack8(dyr[c * 32 + lane], b);
+    unpack8(wr[c * 32 + lane], g);
+    const size_t base = rb + (size_t)(c * 32 + lane) * 8;
+    const float4 d0 = dres ? reinterpret_cast<const float4*>(dres + base)[0] : make_float4(0, 0, 0, 0);
+    const float4 d1 = dres ? reinterpret_cast<const float4*>(dres + base)[1] : make_float4(0, 0, 0, 0);
+    const float dr[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = dr[i] + r * (b[i] * g[i] - (a[i] * r) * dot);
+    reinterpret_cast<float4*>(dh + base)[0] = make_float4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<float4*>(dh + base)[1] = make_float4(o[4], o[5], o[6], o[7]);
+    if (dh_bf16) reinterpret_cast<uint4*>(dh_bf16 + base)[0] = pack8(o);
+  }
+}
+
+// cos/sin of pos * theta^(-2i/d), computed in fp64 and rounded to fp32.
+__global__ void rope_table_kernel(int S, int half, double theta, float* __restrict__ cosb, float* __restrict__ sinb) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= S * half) return;
+  const int pos = i / half, j = i % half;
+  const double inv = pow(theta, -(2.0 * j) / (2.0 * half));
+  const double a = (double)pos * inv;
+  cosb[i] = (float)cos(a);
+  sinb[i] = (float)sin(a);
+}
+
+// D[h, t] = sum_d dO[t, h*128 + d] * O[t, h*128 + d]; one warp per (t, h).
+__global__ void attn_rowdot_kernel(const uint16_t* __restrict__ dO, const uint16_t* __restrict__ O, int T, int Hq,
+                                   float* __restrict__ D) {
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= T * Hq) return;
+  const int t = gw / Hq, h = gw % Hq;
+  const size_t off = (size_t)t * Hq * 128 + h * 128 + lane * 4;
+  const uint2 a = *reinterpret_cast<const uint2*>(dO + off);
+  const uint2 b = *reinterpret_cast<const uint2*>(O + off);
+  // dO is fp16, O is bf16
+  const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&a.x));
+  const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&a.y));
+  float s = d01.x * __uint_as_float(b.x << 16) + d01.y * __uint_as_float(b.x & 0xFFFF0000u) +
+            d23.x * __uint_as_float(b.y << 16) + d23.y * __uint_as_float(b.y & 0xFFFF0000u);
+  s = warp_sum(s);
+  if (lane == 0) D[(size_t)h * T + t] = s;
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ in, size_t n, uint16_t* __restrict__ out) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n / 8; i += (size_t)gridDim.x * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(in)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(in)[2 * i + 1];
+    const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    reinterpret_cast<uint4*>(out)[i] = pack8(f);
+  }
+}
+
+__global__ void bf16_to_f32_kernel(const uint16_t* __restrict__ in, size_t n, float* __restrict__ out) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n / 8; i += (size_t)gridDim.x * blockDim.x) {
+    float f[8];
+    unpack8(reinterpret_cast<const uint4*>(in)[i], f);
+    reinterpret_cast<float4*>(out)[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(out)[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+}
+
+unsigned grid_for(size_t work, int threads) {
+  size_t g = (work + threads - 1) / threads;
+  const size_t cap = (size_t)sm_count() * 16;
+  return (unsigned)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+}  // namespace
+
+soup_status rmsnorm_fwd(const uint16_t* x, const float* x_f32, const uint16_t* w, int T, int H, float eps,
+                        uint16_t* y, float* rinv, cudaStream_t st) {
+  SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
+  rmsnorm_fwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, T, H, eps, y, rinv);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+soup_status rmsnorm_bwd(const uint16_t* x, const float* x_f32, const uint16_t* w, const float* rinv,
+                        const uint16_t* dy, const float* dres, int T, int H, float* dh, uint16_t* dh_bf16,
+                        cudaStream_t st) {
+  SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
+  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, rinv, dy, dres, T, H, dh, dh_bf16);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+soup_status rope_table(int S, int head_dim, double theta, float* cosb, float* sinb, cudaStream_t st) {
+  const int n = S * head_dim / 2;
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(S, head_dim / 2, theta, cosb, sinb);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+soup_status attn_rowdot(const uint16_t* dO, const uint16_t* O, int T, int Hq, float* D, cudaStream_t st) {
+  attn_rowdot_kernel<<<(T * Hq + 7) / 8, 256, 0, st>>>(dO, O, T, Hq, D);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t st) {
+  SOUP_CHECK(n % 8 == 0, SOUP_ERR_SHAPE, "f32_to_bf16: n %% 8");
+  f32_to_bf16_kernel<<<grid_for(n / 8, 256), 256, 0, st>>>(in, n, out);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+soup_status bf16_to_f32(const uint16_t* in, size_t n, float* out, cudaStream_t st) {
+  SOUP_CHECK(n % 8 == 0, SOUP_ERR_SHAPE, "bf16_to_f32: n %% 8");
+  bf16_to_f32_kernel<<<grid_for(n / 8, 256), 256, 0, st>>>(in, n, out);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+}  // namespace soup

@@ -1,0 +1,36 @@
+// Internal launchers of the memory-bound decoder-layer kernels.
+#pragma once
+
+#include "soup_internal.h"
+
+namespace soup {
+
+// RMSNorm over rows of x (bf16 when x_f32 is null, else fp32 x_f32).
+soup_status rmsnorm_fwd(const uint16_t* x, const float* x_f32, const uint16_t* w, int T, int H, float eps,
+                        uint16_t* y, float* rinv, cudaStream_t st);
+soup_status rmsnorm_bwd(const uint16_t* x, const float* x_f32, const uint16_t* w, const float* rinv,
+                        const uint16_t* dy, const float* dres, int T, int H, float* dh, uint16_t* dh_bf16,
+                        cudaStream_t st);
+soup_status rope_table(int S, int head_dim, double theta, float* cosb, float* sinb, cudaStream_t st);
+soup_status rope_apply(uint16_t* buf, int T, int S, int ld, int col0, int nh, const float* cosb, const float* sinb,
+                       bool inverse, cudaStream_t st);
+// D[h, t] = sum_d dO (fp16) * O (bf16)
+soup_status attn_rowdot(const uint16_t* dO, const uint16_t* O, int T, int Hq, float* D, cudaStream_t st);
+soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t st);
+soup_status bf16_to_f32(const uint16_t* in, size_t n, float* out, cudaStream_t st);
+
+// Causal GQA flash attention, head_dim 128.  qkv [T, ld] (fp16) holds q heads
+// at columns [0, Hq*128), k heads at [Hq*128, (Hq+Hkv)*128), v after them;
+// T = Bsz * S tokens, batch-major.  out [T, Hq*128] bf16; lse [Hq, T] (log2
+// units).
+soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, uint16_t* out,
+                          float* lse, cudaStream_t st);
+// Backward: dout [T, Hq*128] fp16; D [Hq, T] = rowsum(dout * out); dqkv bf16; writes dq, dk,
+// dv into dqkv [T, ld] at the same column layout as qkv.  q and k in qkv are
+// post-RoPE; when rope_cos/rope_sin ([S, 64]) are given, dq and dk are
+// rotated back (gradient w.r.t. the pre-RoPE q, k) before they are stored.
+soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, const uint16_t* dout,
+                          const float* lse, const float* D, uint16_t* dqkv, const float* rope_cos,
+                          const float* rope_sin, cudaStream_t st);
+
+}  // namespace soup

@@ -29,6 +29,7 @@
 #include "gemm.h"
 #include "nf4_codebook.cuh"
 #include "ptx.cuh"
+#include <cuda_fp16.h>
 
 namespace soup {
 namespace {
@@ -53,13 +54,21 @@ struct KArgs {
   const float* absmax;
   int tail_ksteps, nseg;
   int seg_end[4], seg_row[4];
-  int out_kind;
+  int pair_off;
+  int epi, out_kind;
   void* out;
   long long ldo;
   const uint16_t* resid;
+  const float* resid_f32;
   long long ldr;
   float alpha;
+  uint16_t* aux16;
+  long long ld_aux;
+  int swiglu_I;
   int vec_ok;
+  int rope_cols, rope_S;
+  const float* rope_cos;
+  const float* rope_sin;
   int* err;
 };
 
@@ -67,9 +76,65 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }
+__device__ __forceinline__ float f16_to_f32(uint16_t b) {
+  return __half2float(__ushort_as_half(b));
+}
+
+// Stores 16 consecutive values of one row (row-major 16-bit or fp32 output),
+// vectorised when the whole chunk is in range and aligned.
+__device__ __forceinline__ void store_row16(void* out, int out_kind, long long ldo, int row, int n, int N,
+                                            const float (&f)[16], bool vec) {
+  const bool full = vec && (n + 16 <= N);
+  if (out_kind == OUT_F32) {
+    float* o = static_cast<float*>(out) + (size_t)row * ldo + n;
+    if (full) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        reinterpret_cast<float4*>(o)[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (n + i < N) o[i] = f[i];
+    }
+    return;
+  }
+  uint16_t* o = static_cast<uint16_t*>(out) + (size_t)row * ldo + n;
+  const bool h = out_kind == OUT_F16;
+  if (full) {
+    uint32_t p[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = h ? pack_f16x2(f[2 * i], f[2 * i + 1]) : pack_bf16x2(f[2 * i], f[2 * i + 1]);
+    reinterpret_cast<uint4*>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
+    reinterpret_cast<uint4*>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (n + i < N) {
+        const uint32_t w = h ? pack_f16x2(f[i], 0.f) : pack_bf16x2(f[i], 0.f);
+        o[i] = static_cast<uint16_t>(w & 0xFFFF);
+      }
+  }
+}
+
+__device__ __forceinline__ void load16_u16(const uint16_t* p, uint16_t (&v)[16]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(p);
+  const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = static_cast<uint16_t>(w[i] & 0xFFFF);
+    v[2 * i + 1] = static_cast<uint16_t>(w[i] >> 16);
+  }
+}
+
+__device__ __forceinline__ float sigmoid_f(float g) { return 1.0f / (1.0f + expf(-g)); }
 
 // 8 NF4 codes (one 32-bit word: byte p holds element 2p high, 2p+1 low) ->
 // 8 bf16 values RNE(fp32(c * absmax)) packed in a uint4.
@@ -117,6 +182,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
   constexpr bool NF4 = BMD >= B_NF4_K;
   constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
   constexpr int STAGES = C::STAGES;
+  constexpr int NEPI = NF4 ? 8 : 4;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -133,7 +199,10 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * BM;
-  const int n0 = blockIdx.y * BN;
+  const bool paired = args.pair_off > 0;
+  // paired: the tile covers columns [nb, nb + BN/2) of both halves
+  const int nb = paired ? blockIdx.y * (BN / 2) : blockIdx.y * BN;
+  const int n0 = nb;  // first B row / output column of the tile (first half when paired)
   const int num_kb = args.num_kb;
   const int n_iters = num_kb + (args.tail_ksteps > 0 ? 1 : 0);
 
@@ -170,6 +239,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
   if (args.nseg > 1 && n0 >= args.seg_end[0]) tail_row = args.seg_row[1];
   if (args.nseg > 2 && n0 >= args.seg_end[1]) tail_row = args.seg_row[2];
   if (args.nseg > 3 && n0 >= args.seg_end[2]) tail_row = args.seg_row[3];
+  if (paired) tail_row = 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -197,7 +267,12 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
           }
           if (!NF4) {
             if (!B_MN) {
-              ptx::tma_load_2d(b, &tmB, &full[s], k0, n0);
+              if (paired) {
+                ptx::tma_load_2d(b, &tmB, &full[s], k0, nb);
+                ptx::tma_load_2d(b + (BN / 2) * 128, &tmB, &full[s], k0, args.pair_off + nb);
+              } else {
+                ptx::tma_load_2d(b, &tmB, &full[s], k0, n0);
+              }
             } else {
 #pragma unroll
               for (int c = 0; c < BN / 64; ++c) ptx::tma_load_2d(b + c * 8192, &tmB, &full[s], n0 + 64 * c, k0);
@@ -207,7 +282,12 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
           ptx::tma_load_2d(a, &tmTA, &full[s], m0, tail_row);
           ptx::tma_load_2d(a + 8192, &tmTA, &full[s], m0 + 64, tail_row);
           if (!B_MN) {
-            ptx::tma_load_2d(b, &tmTB, &full[s], 0, n0);
+            if (paired) {
+              ptx::tma_load_2d(b, &tmTB, &full[s], 0, nb);
+              ptx::tma_load_2d(b + (BN / 2) * 128, &tmTB, &full[s], 0, args.pair_off + nb);
+            } else {
+              ptx::tma_load_2d(b, &tmTB, &full[s], 0, n0);
+            }
           } else {
 #pragma unroll
             for (int c = 0; c < (BN >= 64 ? BN / 64 : 1); ++c)
@@ -221,6 +301,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     if (lane == 0) {
       constexpr uint32_t idesc_main = ptx::idesc_bf16(BM, BN, AMJ, B_MN ? 1 : 0);
       constexpr uint32_t idesc_tail = ptx::idesc_bf16(BM, BN, 1, B_MN ? 1 : 0);
+      constexpr uint32_t idesc_half = ptx::idesc_bf16(BM, BN >= 32 ? BN / 2 : BN, 1, B_MN ? 1 : 0);
       bool ok = true;
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % STAGES;
@@ -235,14 +316,25 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
         const uint32_t a_base = ptx::smem_u32(sA + s * A_STAGE_BYTES);
         const uint32_t b_base = ptx::smem_u32(sB + s * C::B_STAGE);
         const bool tail = it >= num_kb;
-        const int nk = tail ? args.tail_ksteps : BK / 16;
-        const bool a_mn = tail || AMJ == A_MN;
-        for (int k = 0; k < nk; ++k) {
-          const uint64_t ad = a_mn ? ptx::smem_desc_sw128(a_base + k * 2048, 8192, 1024)
-                                   : ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
-          const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k * 2048, 8192, 1024)
-                                   : ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
-          ptx::mma_bf16(tmem, ad, bd, tail ? idesc_tail : idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+        if (tail && paired) {
+          // two half-width MMAs: adapter rows [0,16) for the first half of
+          // the tile, [16,32) for the second
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint64_t ad = ptx::smem_desc_sw128(a_base + hf * 2048, 8192, 1024);
+            const uint64_t bd = ptx::smem_desc_sw128(b_base + hf * (BN / 2) * 128, 16, 1024);
+            ptx::mma_bf16(tmem + hf * (BN / 2), ad, bd, idesc_half, 1u);
+          }
+        } else {
+          const int nk = tail ? args.tail_ksteps : BK / 16;
+          const bool a_mn = tail || AMJ == A_MN;
+          for (int k = 0; k < nk; ++k) {
+            const uint64_t ad = a_mn ? ptx::smem_desc_sw128(a_base + k * 2048, 8192, 1024)
+                                     : ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k * 2048, 8192, 1024)
+                                     : ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
+            ptx::mma_bf16(tmem, ad, bd, tail ? idesc_tail : idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+          }
         }
         ptx::mma_commit(&empty[s]);
       }
@@ -252,65 +344,103 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     const int t = threadIdx.x - 64;  // 0 .. (NF4 ? 255 : 127)
     if constexpr (NF4) {
       // ----------------------------------------------------- NF4 decode warps
+      // Each thread decodes one row-segment of the B tile per stage; the
+      // codes of stage it+1 are loaded into registers while stage it is
+      // decoded, so the global-load latency overlaps the decode.
       const float* lut_lane = lut + lane;
-      for (int it = 0; it < n_iters; ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
-          atomicOr(args.err, 1);
-          *abort_flag = 1;
-          break;
+      if constexpr (BMD == B_NF4_K) {
+        constexpr int TPR = 256 / BN;      // threads per row
+        constexpr int EPT = 64 / TPR;      // elements per thread
+        constexpr int NW = EPT / 8;        // 32-bit code words per thread
+        const int row = t / TPR, h = t % TPR;
+        const int n = paired ? (row < BN / 2 ? nb + row : args.pair_off + nb + row - BN / 2) : n0 + row;
+        const bool nvalid = n < args.N;
+        const uint8_t* src = args.codes + (size_t)(nvalid ? n : 0) * (args.K / 2) + h * (EPT / 2);
+        const float* amp = args.absmax + (size_t)(nvalid ? n : 0) * (args.K / 64);
+        uint32_t wn[NW];
+        float amn = 0.f;
+        if (nvalid && num_kb > 0) {
+          load_codes(src, wn);
+          amn = __ldg(amp);
         }
-        if (it < num_kb) {
-          uint8_t* b = sB + s * C::B_STAGE;
-          if constexpr (BMD == B_NF4_K) {
-            // B tile [BN rows n, 64 k]: codes [N, K/2], one absmax per row per stage
-            constexpr int TPR = 256 / BN;      // threads per row
-            constexpr int EPT = 64 / TPR;      // elements per thread
-            constexpr int NW = EPT / 8;        // 32-bit code words per thread
-            const int row = t / TPR, h = t % TPR;
-            const int n = n0 + row;
-            uint32_t w[NW];
-            float am = 0.f;
-            if (n < args.N) {
-              load_codes(args.codes + (size_t)n * (args.K / 2) + (size_t)it * 32 + h * (EPT / 2), w);
-              am = __ldg(args.absmax + (size_t)n * (args.K / 64) + it);
-            }
+        for (int it = 0; it < n_iters; ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          uint32_t w[NW];
+#pragma unroll
+          for (int u = 0; u < NW; ++u) w[u] = wn[u];
+          const float am = amn;
+          if (nvalid && it + 1 < num_kb) {
+            load_codes(src + (size_t)(it + 1) * 32, wn);
+            amn = __ldg(amp + it + 1);
+          }
+          if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+            atomicOr(args.err, 1);
+            *abort_flag = 1;
+            break;
+          }
+          if (it < num_kb) {
+            uint8_t* b = sB + s * C::B_STAGE;
 #pragma unroll
             for (int u = 0; u < NW; ++u) {
               const int unit = h * NW + u;
-              const uint4 v = (n < args.N) ? decode8(w[u], lut_lane, am) : make_uint4(0, 0, 0, 0);
+              const uint4 v = nvalid ? decode8(w[u], lut_lane, am) : make_uint4(0, 0, 0, 0);
               st_shared_v4(b + row * 128 + ((unit ^ (row & 7)) << 4), v);
             }
-          } else {
-            // B tile [64 k-rows, BN cols]: codes [K, N/2], absmax [K, N/64]
-            constexpr int CPT = BN / 4;        // columns per thread
-            constexpr int NW = CPT / 8;
-            const int kr = t & 63, q = t >> 6;
-            const int k = it * BK + kr;
-            const int c0 = q * CPT;
-            uint32_t w[NW];
-            float am = 0.f;
-            if (k < args.K) {
-              load_codes(args.codes + (size_t)k * (args.N / 2) + (n0 + c0) / 2, w);
-              am = __ldg(args.absmax + (size_t)k * (args.N / 64) + (n0 + c0) / 64);
-            }
+            ptx::fence_proxy_async_smem();
+          }
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&full[s]);
+        }
+      } else {
+        // B tile [64 k-rows, BN cols]: codes [K, N/2], absmax [K, N/64]
+        constexpr int CPT = BN / 4;        // columns per thread
+        constexpr int NW = CPT / 8;
+        const int kr = t & 63, q = t >> 6;
+        const int c0 = q * CPT;
+        const uint8_t* src = args.codes + (size_t)kr * (args.N / 2) + (n0 + c0) / 2;
+        const float* amp = args.absmax + (size_t)kr * (args.N / 64) + (n0 + c0) / 64;
+        const size_t cstep = (size_t)BK * (args.N / 2), astep = (size_t)BK * (args.N / 64);
+        uint32_t wn[NW];
+        float amn = 0.f;
+        if (kr < args.K && num_kb > 0) {
+          load_codes(src, wn);
+          amn = __ldg(amp);
+        }
+        for (int it = 0; it < n_iters; ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          uint32_t w[NW];
+#pragma unroll
+          for (int u = 0; u < NW; ++u) w[u] = wn[u];
+          const float am = amn;
+          const bool kvalid = it * BK + kr < args.K;
+          if (it + 1 < num_kb && (it + 1) * BK + kr < args.K) {
+            load_codes(src + (size_t)(it + 1) * cstep, wn);
+            amn = __ldg(amp + (size_t)(it + 1) * astep);
+          }
+          if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+            atomicOr(args.err, 1);
+            *abort_flag = 1;
+            break;
+          }
+          if (it < num_kb) {
+            uint8_t* b = sB + s * C::B_STAGE;
 #pragma unroll
             for (int u = 0; u < NW; ++u) {
               const int col = c0 + 8 * u;
               const int chunk = col >> 6, unit = (col >> 3) & 7;
-              const uint4 v = (k < args.K) ? decode8(w[u], lut_lane, am) : make_uint4(0, 0, 0, 0);
+              const uint4 v = kvalid ? decode8(w[u], lut_lane, am) : make_uint4(0, 0, 0, 0);
               st_shared_v4(b + chunk * 8192 + kr * 128 + ((unit ^ (kr & 7)) << 4), v);
             }
+            ptx::fence_proxy_async_smem();
           }
-          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&full[s]);
         }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&full[s]);
       }
     }
     // ------------------------------------------------------------ epilogue
-    constexpr int NEPI = NF4 ? 8 : 4;
     const int ew = warp - 2;
     const int q = warp & 3;
     const bool got = ptx::mbar_wait_bounded(accf, 0, abort_flag);
@@ -322,73 +452,139 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
       const int row = m0 + q * 32 + lane;
       const bool row_ok = row < args.M;
       constexpr int NCH = BN / 16;
-      for (int ch = (NEPI == 8 ? ew / 4 : 0); ch < NCH; ch += (NEPI == 8 ? 2 : 1)) {
-        uint32_t v[16];
-        ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + ch * 16, v);
-        ptx::tmem_ld_wait();
-        const int n = n0 + ch * 16;
-        if (!row_ok || n >= args.N) continue;
-        float f[16];
+      const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+      const int ch0 = NEPI == 8 ? ew / 4 : 0, chs = NEPI == 8 ? 2 : 1;
+      const bool vec = args.vec_ok != 0;
+      if (args.epi == EPI_SWIGLU) {
+        // paired gate|up tile: chunk c (gate) pairs with c + NCH/2 (up); both
+        // owned by this warp (NCH/2 is even)
+        const int I = args.swiglu_I;
+        for (int ch = ch0; ch < NCH / 2; ch += chs) {
+          uint32_t vg[16], vu[16];
+          ptx::tmem_ld16(trow + ch * 16, vg);
+          ptx::tmem_ld16(trow + (ch + NCH / 2) * 16, vu);
+          ptx::tmem_ld_wait();
+          const int n = nb + ch * 16;
+          if (!row_ok || n >= I) continue;
+          float a[16], gg[16], uu[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * args.alpha;
-        const bool full16 = (n + 16 <= args.N);
-        if (args.out_kind == OUT_BF16) {
-          uint16_t* o = static_cast<uint16_t*>(args.out) + (size_t)row * args.ldo + n;
+          for (int i = 0; i < 16; ++i) {
+            gg[i] = __uint_as_float(vg[i]) * args.alpha;
+            uu[i] = __uint_as_float(vu[i]) * args.alpha;
+            a[i] = gg[i] * sigmoid_f(gg[i]) * uu[i];
+          }
+          store_row16(args.out, OUT_BF16, args.ldo, row, n, I, a, vec);
+          if (args.aux16) {
+            store_row16(args.aux16, OUT_F16, args.ld_aux, row, n, I, gg, vec);
+            store_row16(args.aux16 + I, OUT_F16, args.ld_aux, row, n, I, uu, vec);
+          }
+        }
+      } else if ((BN >= 128) && args.rope_cols > 0 && n0 < args.rope_cols) {
+        // RoPE (q/k heads of the fused QKV projection): the pair (i, i + 64)
+        // of a 128-wide head lives in chunks c and c + 4 of the head, which
+        // the same warp owns; rotate the fp32 accumulators, then round once.
+        for (int ch = ch0; ch < NCH; ch += chs) {
+          if ((ch & 7) >= 4) continue;
+          uint32_t v0[16], v1[16];
+          ptx::tmem_ld16(trow + ch * 16, v0);
+          ptx::tmem_ld16(trow + (ch + 4) * 16, v1);
+          ptx::tmem_ld_wait();
+          const int n = n0 + ch * 16;
+          if (!row_ok || n >= args.N) continue;
+          const int pos = row % args.rope_S;
+          const float* cs = args.rope_cos + (size_t)pos * 64 + (ch & 7) * 16;
+          const float* sn = args.rope_sin + (size_t)pos * 64 + (ch & 7) * 16;
+          float a[16], b[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float x0 = __uint_as_float(v0[i]) * args.alpha, x1 = __uint_as_float(v1[i]) * args.alpha;
+            const float c = __ldg(cs + i), sv = __ldg(sn + i);
+            a[i] = x0 * c - x1 * sv;
+            b[i] = x1 * c + x0 * sv;
+          }
+          store_row16(args.out, args.out_kind, args.ldo, row, n, args.N, a, vec);
+          store_row16(args.out, args.out_kind, args.ldo, row, n + 64, args.N, b, vec);
+        }
+      } else {
+        for (int ch = ch0; ch < NCH; ch += chs) {
+          uint32_t v[16];
+          ptx::tmem_ld16(trow + ch * 16, v);
+          ptx::tmem_ld_wait();
+          const int n = n0 + ch * 16;
+          if (!row_ok || n >= args.N) continue;
+          float f[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * args.alpha;
+          const bool full16 = vec && (n + 16 <= args.N);
+          if (args.epi == EPI_SWIGLU_BWD) {
+            // f = dL/d(act); g, u from the forward (fp16); out = [dL/dg | dL/du] bf16
+            const int I = args.swiglu_I;
+            uint16_t gb[16], ub[16];
+            const uint16_t* gp = args.aux16 + (size_t)row * args.ld_aux + n;
+            if (full16) {
+              load16_u16(gp, gb);
+              load16_u16(gp + I, ub);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                gb[i] = (n + i < args.N) ? gp[i] : 0;
+                ub[i] = (n + i < args.N) ? gp[I + i] : 0;
+              }
+            }
+            float dg[16], du[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g = f16_to_f32(gb[i]), u = f16_to_f32(ub[i]);
+              const float sg = sigmoid_f(g);
+              dg[i] = f[i] * u * sg * (1.0f + g * (1.0f - sg));
+              du[i] = f[i] * g * sg;
+            }
+            store_row16(args.out, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
+            store_row16(static_cast<uint16_t*>(args.out) + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
+            continue;
+          }
+          if (args.out_kind == OUT_BF16_T || args.out_kind == OUT_F32_T) {
+            if (args.out_kind == OUT_BF16_T) {
+              uint16_t* o = static_cast<uint16_t*>(args.out);
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (n + i < args.N)
+                  o[(size_t)(n + i) * args.ldo + row] = static_cast<uint16_t>(pack_bf16x2(f[i], 0.f) & 0xFFFF);
+            } else {
+              float* o = static_cast<float*>(args.out);
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (n + i < args.N) o[(size_t)(n + i) * args.ldo + row] = f[i];
+            }
+            continue;
+          }
           if (args.resid) {
             const uint16_t* r = args.resid + (size_t)row * args.ldr + n;
-            if (args.vec_ok && full16) {
-              const uint4 r0 = *reinterpret_cast<const uint4*>(r);
-              const uint4 r1 = *reinterpret_cast<const uint4*>(r + 8);
-              const uint32_t rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+            if (full16) {
+              uint16_t rb[16];
+              load16_u16(r, rb);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                f[2 * i] += bf16_to_f32(rr[i] & 0xFFFF);
-                f[2 * i + 1] += bf16_to_f32(rr[i] >> 16);
-              }
+              for (int i = 0; i < 16; ++i) f[i] += bf16_to_f32(rb[i]);
             } else {
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 if (n + i < args.N) f[i] += bf16_to_f32(r[i]);
             }
-          }
-          if (args.vec_ok && full16) {
-            uint32_t p[8];
+          } else if (args.resid_f32) {
+            const float* r = args.resid_f32 + (size_t)row * args.ldr + n;
+            if (full16) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) p[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
-            reinterpret_cast<uint4*>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
-            reinterpret_cast<uint4*>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (n + i < args.N) {
-                __nv_bfloat16 h = __float2bfloat16_rn(f[i]);
-                o[i] = *reinterpret_cast<uint16_t*>(&h);
+              for (int i = 0; i < 4; ++i) {
+                const float4 x = reinterpret_cast<const float4*>(r)[i];
+                f[4 * i] += x.x; f[4 * i + 1] += x.y; f[4 * i + 2] += x.z; f[4 * i + 3] += x.w;
               }
-          }
-        } else if (args.out_kind == OUT_F32) {
-          float* o = static_cast<float*>(args.out) + (size_t)row * args.ldo + n;
-          if (args.vec_ok && full16) {
+            } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              reinterpret_cast<float4*>(o)[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (n + i < args.N) o[i] = f[i];
-          }
-        } else if (args.out_kind == OUT_BF16_T) {
-          uint16_t* o = static_cast<uint16_t*>(args.out);
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (n + i < args.N) {
-              __nv_bfloat16 h = __float2bfloat16_rn(f[i]);
-              o[(size_t)(n + i) * args.ldo + row] = *reinterpret_cast<uint16_t*>(&h);
+              for (int i = 0; i < 16; ++i)
+                if (n + i < args.N) f[i] += r[i];
             }
-        } else {
-          float* o = static_cast<float*>(args.out);
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (n + i < args.N) o[(size_t)(n + i) * args.ldo + row] = f[i];
+          }
+          store_row16(args.out, args.out_kind, args.ldo, row, n, args.N, f, vec);
         }
       }
     }
@@ -441,14 +637,15 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
   memset(&mB, 0, sizeof(mB));
   memset(&mTA, 0, sizeof(mTA));
   memset(&mTB, 0, sizeof(mTB));
+  const bool paired = d.pair_off > 0;
   if (AMJ == A_K) SOUP_TRY(make_map(&mA, d.A, 64, 128, "A"));
   else SOUP_TRY(make_map(&mA, d.A, 64, 64, "A (MN-major)"));
   constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
-  if (BMD == B_TMA_K) SOUP_TRY(make_map(&mB, d.B, 64, BN, "B"));
+  if (BMD == B_TMA_K) SOUP_TRY(make_map(&mB, d.B, 64, paired ? BN / 2 : BN, "B"));
   if (BMD == B_TMA_MN) SOUP_TRY(make_map(&mB, d.B, 64, 64, "B (MN-major)"));
   if (d.tail_ksteps > 0) {
     SOUP_TRY(make_map(&mTA, d.tailA, 64, 64, "tail A"));
-    if (!B_MN) SOUP_TRY(make_map(&mTB, d.tailB, 64, BN, "tail B"));
+    if (!B_MN) SOUP_TRY(make_map(&mTB, d.tailB, 64, paired ? BN / 2 : BN, "tail B"));
     else SOUP_TRY(make_map(&mTB, d.tailB, 64, 64, "tail B (MN-major)"));
   }
   auto kern = gemm_kernel<BN, AMJ, BMD>;
@@ -458,7 +655,8 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
     attr_set = true;
   }
   constexpr int NT = 32 * (2 + (BMD >= B_NF4_K ? 8 : 4));
-  dim3 grid((d.M + BM - 1) / BM, (d.N + BN - 1) / BN);
+  const int ntiles = paired ? (d.pair_off + BN / 2 - 1) / (BN / 2) : (d.N + BN - 1) / BN;
+  dim3 grid((d.M + BM - 1) / BM, ntiles);
   kern<<<grid, NT, C::SMEM, st>>>(mA, mB, mTA, mTB, ka);
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
@@ -473,7 +671,8 @@ int pick_bn(const GemmDesc& d) {
       if (d.seg_end[i] % bn) return false;
     return true;
   };
-  if (!nf4 && !mn && d.N <= 64) return ((d.N + 15) / 16) * 16 == 64 ? 64 : ((d.N + 15) / 16) * 16;
+  if (d.pair_off > 0) return 256;
+  if (!nf4 && !mn && d.N <= 64) return ((d.N + 15) / 16) * 16;
   if (d.N >= 256 && (d.N % 256 == 0 || d.N >= 1024) && fits(256)) return 256;
   if (d.N >= 128 && fits(128)) return 128;
   return 64;
@@ -493,13 +692,25 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
     SOUP_CHECK(d.K % 64 == 0, SOUP_ERR_SHAPE, "gemm: NF4 needs K %% 64 == 0 (K=%d)", d.K);
     if (d.b_mode == B_NF4_MN)
       SOUP_CHECK(d.N % 64 == 0, SOUP_ERR_SHAPE, "gemm: NF4 (transposed) needs N %% 64 == 0");
-    const size_t need = d.b_mode == B_NF4_K ? 32 : 16;
-    SOUP_CHECK(soup_aligned(d.codes, need), SOUP_ERR_ALIGN, "gemm: NF4 codes misaligned");
+    SOUP_CHECK(soup_aligned(d.codes, 16), SOUP_ERR_ALIGN, "gemm: NF4 codes misaligned");
   }
   const int bn = pick_bn(d);
   for (int i = 0; i < d.nseg - 1; ++i)
     SOUP_CHECK(d.seg_end[i] % bn == 0, SOUP_ERR_SHAPE, "gemm: segment end %d not a multiple of the tile %d",
                d.seg_end[i], bn);
+  if (d.pair_off > 0) {
+    SOUP_CHECK(d.N == 2 * d.pair_off && d.pair_off % 128 == 0 && bn == 256 &&
+                   (d.b_mode == B_NF4_K || d.b_mode == B_TMA_K) && d.a_major == A_K,
+               SOUP_ERR_SHAPE, "gemm: paired tiles need N = 2*pair_off, pair_off %% 128 == 0, K-major B");
+    SOUP_CHECK(d.tail_ksteps == 0 || d.tail_ksteps == 1, SOUP_ERR_SHAPE, "gemm: paired tiles take one tail step per half");
+  }
+  if (d.epi == EPI_SWIGLU) {
+    SOUP_CHECK(d.pair_off > 0 && d.swiglu_I == d.pair_off, SOUP_ERR_SHAPE, "gemm: SwiGLU epilogue needs paired tiles");
+  }
+  if (d.epi == EPI_SWIGLU_BWD) {
+    SOUP_CHECK(d.aux16 && d.swiglu_I == d.N && d.out_kind == OUT_BF16, SOUP_ERR_INVALID_ARG,
+               "gemm: SwiGLU backward epilogue needs g|u and a bf16 [M, 2N] output");
+  }
   KArgs ka;
   memset(&ka, 0, sizeof(ka));
   ka.M = d.M; ka.N = d.N; ka.K = d.K;
@@ -507,11 +718,23 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
   ka.codes = d.codes; ka.absmax = d.absmax;
   ka.tail_ksteps = d.tail_ksteps; ka.nseg = d.nseg;
   for (int i = 0; i < 4; ++i) { ka.seg_end[i] = d.seg_end[i]; ka.seg_row[i] = d.seg_row[i]; }
+  ka.pair_off = d.pair_off;
+  ka.epi = d.epi;
   ka.out_kind = d.out_kind; ka.out = d.out; ka.ldo = d.ldo;
-  ka.resid = d.resid; ka.ldr = d.ldr; ka.alpha = d.alpha;
-  const int esz = (d.out_kind == OUT_BF16 || d.out_kind == OUT_BF16_T) ? 2 : 4;
+  ka.resid = d.resid; ka.resid_f32 = d.resid_f32; ka.ldr = d.ldr; ka.alpha = d.alpha;
+  ka.aux16 = d.aux16; ka.ld_aux = d.ld_aux; ka.swiglu_I = d.swiglu_I;
+  const int esz = (d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T) ? 4 : 2;
   ka.vec_ok = soup_aligned(d.out, 16) && ((d.ldo * esz) % 16 == 0) &&
-              (!d.resid || (soup_aligned(d.resid, 16) && (d.ldr * 2) % 16 == 0));
+              (!d.resid || (soup_aligned(d.resid, 16) && (d.ldr * 2) % 16 == 0)) &&
+              (!d.resid_f32 || (soup_aligned(d.resid_f32, 16) && (d.ldr * 4) % 16 == 0)) &&
+              (!d.aux16 || (soup_aligned(d.aux16, 16) && (d.ld_aux * 2) % 16 == 0 && (d.swiglu_I % 8) == 0));
+  ka.rope_cols = d.rope_cols; ka.rope_S = d.rope_S;
+  ka.rope_cos = d.rope_cos; ka.rope_sin = d.rope_sin;
+  if (d.rope_cols > 0) {
+    SOUP_CHECK((d.out_kind == OUT_BF16 || d.out_kind == OUT_F16) && !d.resid && !d.resid_f32 && d.rope_cos &&
+                   d.rope_sin && d.rope_S > 0 && d.rope_cols % 128 == 0 && bn >= 128,
+               SOUP_ERR_SHAPE, "gemm: RoPE epilogue needs a plain 16-bit output, 128-aligned heads and BN >= 128");
+  }
   ka.err = device_error_word();
   SOUP_CHECK(ka.err != nullptr, SOUP_ERR_CUDA, "device error word unavailable");
 

@@ -1,6 +1,7 @@
 // Internal interface of the tcgen05 GEMM engine used by every contraction of
 // the training step: D[M, N] = A[M, K] * B[N, K]^T (+ tail) with bf16
-// operands and fp32 accumulation in tensor memory.
+// operands and fp32 accumulation in tensor memory, followed by a fused
+// epilogue.
 #pragma once
 
 #include <cstdint>
@@ -24,7 +25,13 @@ enum BMode : int {
   B_NF4_K = 2,   // B = dequant(codes [N, K/2], absmax [N, K/64])      (forward W)
   B_NF4_MN = 3,  // B = dequant(codes [K, N/2], absmax [K, N/64])^T    (backward W^T)
 };
-enum OutKind : int { OUT_BF16 = 0, OUT_BF16_T = 1, OUT_F32 = 2, OUT_F32_T = 3 };
+// Output element type and layout: row-major [M, N] or transposed [N, M].
+enum OutKind : int { OUT_BF16 = 0, OUT_BF16_T = 1, OUT_F32 = 2, OUT_F32_T = 3, OUT_F16 = 4 };
+enum Epi : int {
+  EPI_STORE = 0,       // out = alpha * acc (+ resid), one rounding
+  EPI_SWIGLU = 1,      // paired gate|up tile: out = bf16(silu(g) * u), aux16 <- fp16 g | u
+  EPI_SWIGLU_BWD = 2,  // acc = dL/d(act): reads fp16 g | u from aux16, out <- bf16 dL/dg | dL/du
+};
 
 struct GemmDesc {
   int M = 0, N = 0, K = 0;
@@ -43,13 +50,30 @@ struct GemmDesc {
   int nseg = 1;             // N segments (tiles never straddle a segment end)
   int seg_end[4] = {0, 0, 0, 0};
   int seg_row[4] = {0, 0, 0, 0};
-  // Epilogue: out = alpha * acc (+ resid), rounded once.
+  // Paired tiles (gate|up): when pair_off > 0, B has 2*pair_off rows and the
+  // CTA of N-tile j computes columns [j*BN/2, (j+1)*BN/2) of both halves
+  // (rows of B at j*BN/2 and pair_off + j*BN/2) into one BN-wide
+  // accumulator; the tail then uses tailA rows [0, 16) for the first half and
+  // [16, 32) for the second.  N must equal 2*pair_off.
+  int pair_off = 0;
+  // Epilogue.
+  int epi = EPI_STORE;
   int out_kind = OUT_BF16;
   void* out = nullptr;
   int64_t ldo = 0;
-  const uint16_t* resid = nullptr;  // bf16 [M, N] row stride ldr (OUT_BF16 only)
+  const uint16_t* resid = nullptr;  // bf16 [M, N] row stride ldr (row-major outputs)
+  const float* resid_f32 = nullptr; // fp32 [M, N] row stride ldr (row-major outputs)
   int64_t ldr = 0;
   float alpha = 1.f;
+  uint16_t* aux16 = nullptr;        // fp16 [M, 2*I] g | u (SwiGLU modes), row stride ld_aux
+  int64_t ld_aux = 0;
+  int swiglu_I = 0;                 // I: offset of u within aux16 / of dL/du within out
+  // Optional RoPE on output columns [0, rope_cols) (128-wide heads): pairs
+  // (i, i+64) of each head rotated by the angle of position row % rope_S,
+  // cos/sin tables [rope_S, 64] fp32, applied to the fp32 accumulator.
+  int rope_cols = 0, rope_S = 0;
+  const float* rope_cos = nullptr;
+  const float* rope_sin = nullptr;
   int bn = 0;               // N tile (0 = pick)
 };
 

@@ -1,0 +1,394 @@
+// One decoder layer, forward and recompute-backward, as a sequence of the
+// library's kernels on one stream:
+//
+// forward:  RMSNorm -> [u_qkv] -> QKV GEMM (NF4 decode + 3-segment LoRA tail,
+//           RoPE on q/k in the epilogue, fp16 out) -> attention -> [u_o]
+//           -> O GEMM (+ residual, fp32 out) -> RMSNorm -> [u_gu]
+//           -> gate|up GEMM on paired tiles with SwiGLU in the epilogue
+//           -> [u_d] -> down GEMM (+ fp32 residual, bf16 out)
+// backward: the forward again from the saved layer input (the layer was read
+//           a second time for this; the down GEMM's output is not needed and
+//           is skipped), then in reverse: g = dy B (per adapter), dx = dy W +
+//           g' A (NF4 decode of W^T + tail; the down projection's epilogue
+//           applies the SwiGLU backward), dB = dy^T u, dA = g'^T x for each
+//           projection group, with RMSNorm / attention backward in between
+//           (inverse RoPE in the attention-backward epilogues).  The
+//           residual-stream gradient and the mid-layer residual h2 stay fp32.
+#include <cuda_bf16.h>
+
+#include "elementwise.h"
+#include "lora_internal.h"
+
+namespace soup {
+namespace {
+
+struct Dims {
+  int T, S, B, H, Hq, Hkv, d, I, r, qkv_w, o_in;
+  int64_t ldT;
+  float s;
+};
+
+// Workspace layout (byte offsets, each 256-aligned).
+struct WS {
+  size_t x1, rinv1, qkv, attn, lse, h2, x2, rinv2, gu16, act, u_qkv, u_o, u_gu, u_d, cosb, sinb;
+  size_t dh_b, g_d, g_gu, g_o, g_qkv, Bt, d_gu, dx2, dh2, dh2_b, d_attn, D, d_qkv, dx1;
+  size_t total;
+};
+
+WS layout(const Dims& m) {
+  WS w;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o += align256(bytes);
+    return at;
+  };
+  const size_t T = m.T, H = m.H, I = m.I, r = m.r, ldT = m.ldT;
+  w.x1 = take(T * H * 2);
+  w.rinv1 = take(T * 4);
+  w.qkv = take(T * m.qkv_w * 2);  // fp16
+  w.attn = take(T * m.o_in * 2);
+  w.lse = take((size_t)m.Hq * T * 4);
+  w.h2 = take(T * H * 4);  // fp32
+  w.x2 = take(T * H * 2);
+  w.rinv2 = take(T * 4);
+  w.gu16 = take(T * 2 * I * 2);  // fp16 g | u saved for the SwiGLU backward
+  w.act = take(T * I * 2);
+  w.u_qkv = take(3 * r * ldT * 2);
+  w.u_o = take(r * ldT * 2);
+  w.u_gu = take(2 * r * ldT * 2);
+  w.u_d = take(r * ldT * 2);
+  w.cosb = take((size_t)m.S * (m.d / 2) * 4);
+  w.sinb = take((size_t)m.S * (m.d / 2) * 4);
+  w.dh_b = take(T * H * 2);
+  w.g_d = take(r * ldT * 2);
+  w.g_gu = take(2 * r * ldT * 2);
+  w.g_o = take(r * ldT * 2);
+  w.g_qkv = take(3 * r * ldT * 2);
+  size_t max_out = std::max<size_t>(std::max<size_t>(H, I), (size_t)m.qkv_w);
+  w.Bt = take(max_out * r * 2);
+  w.d_gu = take(T * 2 * I * 2);
+  w.dx2 = take(T * H * 2);
+  w.dh2 = take(T * H * 4);
+  w.dh2_b = take(T * H * 2);
+  w.d_attn = take(T * m.o_in * 2);  // fp16
+  w.D = take((size_t)m.Hq * T * 4);
+  w.d_qkv = take(T * m.qkv_w * 2);
+  w.dx1 = take(T * H * 2);
+  w.total = o;
+  return w;
+}
+
+soup_status make_dims(const soup_layer_cfg* c, int64_t batch, int64_t seq, Dims* m) {
+  SOUP_CHECK(c, SOUP_ERR_INVALID_ARG, "decoder layer: null cfg");
+  SOUP_CHECK(c->head_dim == 128, SOUP_ERR_SHAPE, "decoder layer: head_dim must be 128 (got %d)", c->head_dim);
+  SOUP_CHECK(c->rank == 16, SOUP_ERR_SHAPE, "decoder layer: rank must be 16 (got %d)", c->rank);
+  SOUP_CHECK(c->hidden > 0 && c->hidden % 256 == 0, SOUP_ERR_SHAPE, "decoder layer: hidden %% 256");
+  SOUP_CHECK(c->n_q_heads > 0 && c->n_kv_heads > 0 && c->n_q_heads % c->n_kv_heads == 0, SOUP_ERR_SHAPE,
+             "decoder layer: heads %d/%d", c->n_q_heads, c->n_kv_heads);
+  SOUP_CHECK(c->intermediate > 0 && c->intermediate % 128 == 0, SOUP_ERR_SHAPE,
+             "decoder layer: intermediate must be a multiple of 128");
+  SOUP_CHECK(batch >= 1 && seq >= 1 && batch * seq < (1 << 24), SOUP_ERR_SHAPE, "decoder layer: batch/seq");
+  SOUP_CHECK(c->eps >= 0.f && c->theta > 0.f, SOUP_ERR_INVALID_ARG, "decoder layer: eps/theta");
+  m->B = (int)batch; m->S = (int)seq; m->T = (int)(batch * seq);
+  m->H = c->hidden; m->Hq = c->n_q_heads; m->Hkv = c->n_kv_heads; m->d = c->head_dim;
+  m->I = c->intermediate; m->r = c->rank;
+  m->qkv_w = (m->Hq + 2 * m->Hkv) * m->d;
+  m->o_in = m->Hq * m->d;
+  m->ldT = round_up8(m->T);
+  m->s = c->alpha / (float)c->rank;
+  return SOUP_OK;
+}
+
+soup_status check_weights(const soup_layer_weights* W, const Dims& m) {
+  SOUP_CHECK(W && W->norm1 && W->norm2, SOUP_ERR_INVALID_ARG, "decoder layer: null weights");
+  SOUP_TRY(check_weight(&W->qkv, "decoder layer qkv"));
+  SOUP_TRY(check_weight(&W->o, "decoder layer o"));
+  SOUP_TRY(check_weight(&W->gate_up, "decoder layer gate_up"));
+  SOUP_TRY(check_weight(&W->down, "decoder layer down"));
+  SOUP_CHECK(W->qkv.out_features == m.qkv_w && W->qkv.in_features == m.H, SOUP_ERR_SHAPE, "qkv shape");
+  SOUP_CHECK(W->o.out_features == m.H && W->o.in_features == m.o_in, SOUP_ERR_SHAPE, "o shape");
+  SOUP_CHECK(W->gate_up.out_features == 2 * m.I && W->gate_up.in_features == m.H, SOUP_ERR_SHAPE, "gate_up shape");
+  SOUP_CHECK(W->down.out_features == m.H && W->down.in_features == m.I, SOUP_ERR_SHAPE, "down shape");
+  return SOUP_OK;
+}
+
+#define P(off) (reinterpret_cast<uint16_t*>(base + ws.off))
+#define PF(off) (reinterpret_cast<float*>(base + ws.off))
+
+// y = x W^T (+ tail u B^T) (+ resid) into out [T, N]
+struct ProjOpts {
+  int out_kind = OUT_BF16;
+  const uint16_t* resid = nullptr;
+  const float* resid_f32 = nullptr;
+  int rope_cols = 0, rope_S = 0;
+  const float* rope_cos = nullptr;
+  const float* rope_sin = nullptr;
+  int swiglu_I = 0;          // > 0: paired gate|up tiles with the SwiGLU epilogue
+  uint16_t* aux16 = nullptr; // SwiGLU: fp16 g | u output (may be null)
+};
+
+soup_status proj_fwd(const soup_weight* W, const uint16_t* x, int T, const uint16_t* u, int64_t ldT, int u_rows,
+                     const uint16_t* Bl, int r, int nseg, const int* seg_end, const int* seg_row, bool on,
+                     uint16_t* out, cudaStream_t st, const ProjOpts& o = ProjOpts()) {
+  GemmDesc g;
+  g.M = T; g.N = (int)W->out_features; g.K = (int)W->in_features;
+  g.A = Mat{x, T, W->in_features, W->in_features};
+  set_weight_fwd(g, W);
+  if (on) {
+    g.tail_ksteps = r / 16;
+    g.tailA = Mat{u, u_rows, T, ldT};
+    g.tailB = Mat{Bl, W->out_features, r, r};
+    g.nseg = nseg;
+    for (int i = 0; i < nseg; ++i) { g.seg_end[i] = seg_end[i]; g.seg_row[i] = seg_row[i]; }
+  }
+  g.out_kind = o.out_kind; g.out = out; g.ldo = W->out_features;
+  g.resid = o.resid; g.resid_f32 = o.resid_f32; g.ldr = W->out_features;
+  g.rope_cols = o.rope_cols; g.rope_S = o.rope_S; g.rope_cos = o.rope_cos; g.rope_sin = o.rope_sin;
+  if (o.swiglu_I > 0) {
+    g.pair_off = o.swiglu_I;
+    g.nseg = 1;
+    g.epi = EPI_SWIGLU;
+    g.swiglu_I = o.swiglu_I;
+    g.ldo = o.swiglu_I;
+    g.aux16 = o.aux16;
+    g.ld_aux = 2 * (int64_t)o.swiglu_I;
+  }
+  return gemm(g, st);
+}
+
+// u' = bf16(s * x A^T), transposed [rows, ldT]
+soup_status lora_down(const uint16_t* x, int T, int K, const uint16_t* A, int rows, float s, uint16_t* u,
+                      int64_t ldT, cudaStream_t st) {
+  GemmDesc g;
+  g.M = T; g.N = rows; g.K = K;
+  g.A = Mat{x, T, K, K};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{A, rows, K, K};
+  g.out_kind = OUT_BF16_T; g.out = u; g.ldo = ldT; g.alpha = s;
+  return gemm(g, st);
+}
+
+// g' = bf16(s * dy B) for one adapter segment: dy = columns [c0, c0+n) of a
+// [T, ld] buffer, B [n, r]; writes rows of a transposed [*, ldT] buffer.
+soup_status lora_g(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t* Bl, int r, float s, uint16_t* Bt,
+                   uint16_t* gout, int64_t ldT, cudaStream_t st) {
+  SOUP_TRY(transpose_bf16(Bl, n, r, Bt, st));
+  GemmDesc g;
+  g.M = T; g.N = r; g.K = n;
+  g.A = Mat{dy, T, n, ld};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{Bt, r, n, n};
+  g.out_kind = OUT_BF16_T; g.out = gout; g.ldo = ldT; g.alpha = s;
+  return gemm(g, st);
+}
+
+// dB [n, r] = dy_seg^T u_seg^T : dy = columns of a [T, ld] buffer.
+soup_status lora_dB(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t* u, int r, int64_t ldT, float* dB,
+                    cudaStream_t st) {
+  GemmDesc g;
+  g.M = n; g.N = r; g.K = T;
+  g.a_major = A_MN;
+  g.A = Mat{dy, T, n, ld};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{u, r, T, ldT};
+  g.out_kind = OUT_F32; g.out = dB; g.ldo = r;
+  return gemm(g, st);
+}
+
+// dA [rows, K] = g'^T x  (computed transposed: M = K, N = rows)
+soup_status lora_dA(const uint16_t* x, int T, int K, const uint16_t* gt, int rows, int64_t ldT, float* dA,
+                    cudaStream_t st) {
+  GemmDesc g;
+  g.M = K; g.N = rows; g.K = T;
+  g.a_major = A_MN;
+  g.A = Mat{x, T, K, K};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{gt, rows, T, ldT};
+  g.out_kind = OUT_F32_T; g.out = dA; g.ldo = K;
+  return gemm(g, st);
+}
+
+// dx = dy W (+ g' A); with swiglu_I > 0 the epilogue turns dL/d(act) into
+// [dL/dg | dL/du] (bf16, [T, 2I]) using the fp16 g | u saved by the forward.
+soup_status proj_bwd(const soup_weight* W, const uint16_t* dy, int T, const uint16_t* gt, int64_t ldT, int g_rows,
+                     const uint16_t* Al, bool on, uint16_t* dx, cudaStream_t st, int out_kind = OUT_BF16,
+                     int swiglu_I = 0, uint16_t* aux16 = nullptr) {
+  GemmDesc g;
+  g.M = T; g.N = (int)W->in_features; g.K = (int)W->out_features;
+  g.A = Mat{dy, T, W->out_features, W->out_features};
+  set_weight_bwd(g, W);
+  if (on) {
+    g.tail_ksteps = g_rows / 16;
+    g.tailA = Mat{gt, g_rows, T, ldT};
+    g.tailB = Mat{Al, g_rows, W->in_features, W->in_features};
+  }
+  g.out_kind = out_kind; g.out = dx; g.ldo = W->in_features;
+  if (swiglu_I > 0) {
+    g.epi = EPI_SWIGLU_BWD;
+    g.swiglu_I = swiglu_I;
+    g.aux16 = aux16;
+    g.ld_aux = 2 * (int64_t)swiglu_I;
+    g.ldo = 2 * (int64_t)swiglu_I;
+  }
+  return gemm(g, st);
+}
+
+// Forward through the layer; with `keep_down_out` false the final down GEMM
+// (whose output the backward pass does not need) is skipped.
+soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const soup_layer_cfg* c, const Dims& m,
+                    const WS& ws, char* base, const uint16_t* h_in, uint16_t* h_out, bool on, bool recompute,
+                    cudaStream_t st) {
+  const int T = m.T, r = m.r;
+  SOUP_TRY(rope_table(m.S, m.d, (double)c->theta, PF(cosb), PF(sinb), st));
+  SOUP_TRY(rmsnorm_fwd(h_in, nullptr, W->norm1, T, m.H, c->eps, P(x1), PF(rinv1), st));
+  if (on) SOUP_TRY(lora_down(P(x1), T, m.H, L->A_qkv, 3 * r, m.s, P(u_qkv), m.ldT, st));
+  {
+    const int se[3] = {m.Hq * m.d, (m.Hq + m.Hkv) * m.d, m.qkv_w};
+    const int sr[3] = {0, r, 2 * r};
+    ProjOpts o;
+    o.out_kind = OUT_F16;  // q, k, v feed only the attention kernels
+    o.rope_cols = (m.Hq + m.Hkv) * m.d;
+    o.rope_S = m.S; o.rope_cos = PF(cosb); o.rope_sin = PF(sinb);
+    SOUP_TRY(proj_fwd(&W->qkv, P(x1), T, P(u_qkv), m.ldT, 3 * r, L ? L->B_qkv : nullptr, r, 3, se, sr, on, P(qkv),
+                      st, o));
+  }
+  SOUP_TRY(attention_fwd(P(qkv), m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(attn), PF(lse), st));
+  if (on) SOUP_TRY(lora_down(P(attn), T, m.o_in, L->A_o, r, m.s, P(u_o), m.ldT, st));
+  {
+    const int se[1] = {m.H};
+    const int sr[1] = {0};
+    ProjOpts o;
+    o.out_kind = OUT_F32;  // h2 = h + o kept in fp32
+    o.resid = h_in;
+    SOUP_TRY(proj_fwd(&W->o, P(attn), T, P(u_o), m.ldT, r, L ? L->B_o : nullptr, r, 1, se, sr, on,
+                      reinterpret_cast<uint16_t*>(PF(h2)), st, o));
+  }
+  SOUP_TRY(rmsnorm_fwd(nullptr, PF(h2), W->norm2, T, m.H, c->eps, P(x2), PF(rinv2), st));
+  if (on) SOUP_TRY(lora_down(P(x2), T, m.H, L->A_gu, 2 * r, m.s, P(u_gu), m.ldT, st));
+  {
+    const int se[1] = {2 * m.I};
+    const int sr[1] = {0};
+    ProjOpts o;
+    o.swiglu_I = m.I;
+    o.aux16 = recompute ? P(gu16) : nullptr;  // g | u are needed only by the backward
+    SOUP_TRY(proj_fwd(&W->gate_up, P(x2), T, P(u_gu), m.ldT, 2 * r, L ? L->B_gu : nullptr, r, 1, se, sr, on,
+                      P(act), st, o));
+  }
+  if (on) SOUP_TRY(lora_down(P(act), T, m.I, L->A_down, r, m.s, P(u_d), m.ldT, st));
+  if (!recompute) {
+    const int se[1] = {m.H};
+    const int sr[1] = {0};
+    ProjOpts o;
+    o.resid_f32 = PF(h2);
+    SOUP_TRY(proj_fwd(&W->down, P(act), T, P(u_d), m.ldT, r, L ? L->B_down : nullptr, r, 1, se, sr, on, h_out, st,
+                      o));
+  }
+  return SOUP_OK;
+}
+
+}  // namespace
+}  // namespace soup
+
+using namespace soup;
+
+extern "C" size_t soup_decoder_layer_workspace(const soup_layer_cfg* cfg, int64_t batch, int64_t seq) {
+  Dims m;
+  if (make_dims(cfg, batch, seq, &m) != SOUP_OK) return 0;
+  return layout(m).total;
+}
+
+extern "C" soup_status soup_decoder_layer_fwd(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                              const soup_layer_cfg* cfg, const uint16_t* h_in, int64_t batch,
+                                              int64_t seq, uint16_t* h_out, int32_t adapters_on, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  Dims m;
+  SOUP_TRY(make_dims(cfg, batch, seq, &m));
+  SOUP_TRY(check_weights(W, m));
+  SOUP_CHECK(h_in && h_out && workspace, SOUP_ERR_INVALID_ARG, "soup_decoder_layer_fwd: null pointer");
+  SOUP_CHECK(!adapters_on || (lora && lora->A_qkv && lora->B_qkv && lora->A_o && lora->B_o && lora->A_gu &&
+                              lora->B_gu && lora->A_down && lora->B_down),
+             SOUP_ERR_INVALID_ARG, "soup_decoder_layer_fwd: adapters on but LoRA factors missing");
+  const WS ws = layout(m);
+  SOUP_CHECK(workspace_bytes >= ws.total && soup_aligned(workspace, 256), SOUP_ERR_INVALID_ARG,
+             "soup_decoder_layer_fwd: workspace %zu < %zu bytes or misaligned", workspace_bytes, ws.total);
+  return forward(W, lora, cfg, m, ws, static_cast<char*>(workspace), h_in, h_out, adapters_on != 0, false,
+                 static_cast<cudaStream_t>(stream));
+}
+
+extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const soup_layer_lora* L,
+                                              const soup_layer_cfg* cfg, const uint16_t* h_in, const float* dh_out,
+                                              int64_t batch, int64_t seq, float* dh_in,
+                                              const soup_layer_grads* G, int32_t adapters_on, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  Dims m;
+  SOUP_TRY(make_dims(cfg, batch, seq, &m));
+  SOUP_TRY(check_weights(W, m));
+  SOUP_CHECK(h_in && dh_out && dh_in && workspace, SOUP_ERR_INVALID_ARG, "soup_decoder_layer_bwd: null pointer");
+  const bool on = adapters_on != 0;
+  SOUP_CHECK(!on || (L && G && G->dA_qkv && G->dB_qkv && G->dA_o && G->dB_o && G->dA_gu && G->dB_gu && G->dA_down &&
+                     G->dB_down),
+             SOUP_ERR_INVALID_ARG, "soup_decoder_layer_bwd: adapters on but LoRA factors/grads missing");
+  const WS ws = layout(m);
+  SOUP_CHECK(workspace_bytes >= ws.total && soup_aligned(workspace, 256), SOUP_ERR_INVALID_ARG,
+             "soup_decoder_layer_bwd: workspace %zu < %zu bytes or misaligned", workspace_bytes, ws.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(workspace);
+  const int T = m.T, r = m.r, H = m.H, I = m.I;
+  const int64_t ldT = m.ldT;
+
+  SOUP_TRY(forward(W, L, cfg, m, ws, base, h_in, nullptr, on, true, st));
+
+  // ---- MLP block
+  SOUP_TRY(f32_to_bf16(dh_out, (size_t)T * H, P(dh_b), st));
+  if (on) SOUP_TRY(lora_g(P(dh_b), H, T, H, L->B_down, r, m.s, P(Bt), P(g_d), ldT, st));
+  // d_gu = SwiGLU backward of (dh W_down + g' A_down), fused in the epilogue
+  SOUP_TRY(proj_bwd(&W->down, P(dh_b), T, P(g_d), ldT, r, on ? L->A_down : nullptr, on, P(d_gu), st, OUT_BF16, I,
+                    P(gu16)));
+  if (on) {
+    SOUP_TRY(lora_dB(P(dh_b), H, T, H, P(u_d), r, ldT, G->dB_down, st));
+    SOUP_TRY(lora_dA(P(act), T, I, P(g_d), r, ldT, G->dA_down, st));
+  }
+  uint16_t* d_gu = P(d_gu);
+  if (on) {
+    for (int sg = 0; sg < 2; ++sg)
+      SOUP_TRY(lora_g(d_gu + (size_t)sg * I, 2 * I, T, I, L->B_gu + (size_t)sg * I * r, r, m.s, P(Bt),
+                      P(g_gu) + (size_t)sg * r * ldT, ldT, st));
+  }
+  SOUP_TRY(proj_bwd(&W->gate_up, d_gu, T, P(g_gu), ldT, 2 * r, on ? L->A_gu : nullptr, on, P(dx2), st));
+  if (on) {
+    for (int sg = 0; sg < 2; ++sg)
+      SOUP_TRY(lora_dB(d_gu + (size_t)sg * I, 2 * I, T, I, P(u_gu) + (size_t)sg * r * ldT, r, ldT,
+                       G->dB_gu + (size_t)sg * I * r, st));
+    SOUP_TRY(lora_dA(P(x2), T, H, P(g_gu), 2 * r, ldT, G->dA_gu, st));
+  }
+  SOUP_TRY(rmsnorm_bwd(nullptr, PF(h2), W->norm2, PF(rinv2), P(dx2), dh_out, T, H, PF(dh2), P(dh2_b), st));
+
+  // ---- attention block
+  if (on) SOUP_TRY(lora_g(P(dh2_b), H, T, H, L->B_o, r, m.s, P(Bt), P(g_o), ldT, st));
+  SOUP_TRY(proj_bwd(&W->o, P(dh2_b), T, P(g_o), ldT, r, on ? L->A_o : nullptr, on, P(d_attn), st, OUT_F16));
+  if (on) {
+    SOUP_TRY(lora_dB(P(dh2_b), H, T, H, P(u_o), r, ldT, G->dB_o, st));
+    SOUP_TRY(lora_dA(P(attn), T, m.o_in, P(g_o), r, ldT, G->dA_o, st));
+  }
+  SOUP_TRY(attn_rowdot(P(d_attn), P(attn), T, m.Hq, PF(D), st));
+  // dq and dk leave the attention backward already rotated back (inverse RoPE in its epilogues)
+  SOUP_TRY(attention_bwd(P(qkv), m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(d_attn), PF(lse), PF(D), P(d_qkv), PF(cosb),
+                         PF(sinb), st));
+  const int seg_n[3] = {m.Hq * m.d, m.Hkv * m.d, m.Hkv * m.d};
+  const int seg_c[3] = {0, m.Hq * m.d, (m.Hq + m.Hkv) * m.d};
+  if (on) {
+    for (int sg = 0; sg < 3; ++sg)
+      SOUP_TRY(lora_g(P(d_qkv) + seg_c[sg], m.qkv_w, T, seg_n[sg], L->B_qkv + (size_t)seg_c[sg] * r, r, m.s, P(Bt),
+                      P(g_qkv) + (size_t)sg * r * ldT, ldT, st));
+  }
+  SOUP_TRY(proj_bwd(&W->qkv, P(d_qkv), T, P(g_qkv), ldT, 3 * r, on ? L->A_qkv : nullptr, on, P(dx1), st));
+  if (on) {
+    for (int sg = 0; sg < 3; ++sg)
+      SOUP_TRY(lora_dB(P(d_qkv) + seg_c[sg], m.qkv_w, T, seg_n[sg], P(u_qkv) + (size_t)sg * r * ldT, r, ldT,
+                       G->dB_qkv + (size_t)seg_c[sg] * r, st));
+    SOUP_TRY(lora_dA(P(x1), T, H, P(g_qkv), 3 * r, ldT, G->dA_qkv, st));
+  }
+  SOUP_TRY(rmsnorm_bwd(h_in, nullptr, W->norm1, PF(rinv1), P(dx1), PF(dh2), T, H, dh_in, nullptr, st));
+  return SOUP_OK;
+}
