@@ -1,0 +1,362 @@
+#!/usr/bin/env python
+"""Benchmark of the layer-streamed NF4 LoRA training step on B200.
+
+Default workload: a Llama-3.1-8B-shaped stack (32 decoder layers, hidden
+4096, 32 q / 8 kv heads of 128, SwiGLU 14336, vocab 128256, untied lm_head),
+all seven projections NF4 (64-blocks) with LoRA r=16 alpha=32, streamed from
+pinned host RAM through stream_buffers=2 device slots under a 4 GB device cap;
+batch 4 x seq 512 uniform-random token ids; one SFT step = forward through the
+streamed stack, chunked next-token CE, recompute-backward through the stream
+producing every LoRA gradient.  Synthetic random-init weights of that
+architecture (no checkpoints, no datasets).
+
+Prints one JSON line (rank 0).  `value` is train tokens/s measured on the
+device (CUDA events on the compute stream, max over ranks) with the step's
+inputs already in HBM; `e2e` is the same metric through the public API with
+the token ids copied from pinned host memory and the loss read back every
+step.  `roofline` reports the dominant kernel (the fused NF4-dequant GEMM)
+against the measured bf16 tensor peak.
+
+Multi-GPU (torchrun): data parallel, one micro-batch per rank (weak scaling),
+each rank streaming its own copy of the base over its own host link, LoRA
+gradients all-reduced with NCCL after the backward pass.
+
+--impl reference times the CPU oracle (plain fp64 numpy) on this host's
+cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # Llama-3.1-8B-shaped NF4 stack, batch 4 x seq 512, stream_buffers=2, 4 GB cap
+    "llama8b-nf4-stream-sft": dict(hidden=4096, n_q_heads=32, n_kv_heads=8, head_dim=128, intermediate=14336,
+                                   rank=16, alpha=32.0, vocab=128256, n_layers=32, kind="nf4", tied=False,
+                                   batch=4, seq=512, buffers=2, cap_gb=4.0, task="sft"),
+    # Qwen2.5-3B-shaped un-quantised bf16 stack, batch 2 x seq 1024, tied embeddings
+    "qwen3b-bf16-stream-sft": dict(hidden=2048, n_q_heads=16, n_kv_heads=2, head_dim=128, intermediate=11008,
+                                   rank=16, alpha=32.0, vocab=151936, n_layers=36, kind="bf16", tied=True,
+                                   batch=2, seq=1024, buffers=2, cap_gb=0.0, task="sft"),
+    # DPO on the 8B NF4 stream: 4 pairs, 256-token shared prompt + 256-token continuations
+    "llama8b-nf4-stream-dpo": dict(hidden=4096, n_q_heads=32, n_kv_heads=8, head_dim=128, intermediate=14336,
+                                   rank=16, alpha=32.0, vocab=128256, n_layers=32, kind="nf4", tied=False,
+                                   batch=8, seq=512, buffers=2, cap_gb=0.0, task="dpo", prompt=256, beta=0.1),
+}
+DEFAULT = "llama8b-nf4-stream-sft"
+METRIC = "train tokens/s, 8B-shape NF4 streamed LoRA, 1 B200; fused GEMM % bf16 peak"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def gemm_traffic():
+    """Per-launch DRAM bytes of the dominant kernel from a committed ncu
+    summary, if it was taken on the current GEMM source (else None)."""
+    p = os.path.join(ROOT, "profiles", "gemm_nf4_traffic.json")
+    src = os.path.join(ROOT, "layer_streamed_qlora_b200", "csrc", "gemm.cu")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()
+    if d.get("gemm_cu_sha256") != h:
+        return None
+    return d
+
+
+class ClockSampler:
+    def __init__(self, dev):
+        self.dev = dev
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{dev}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,"
+                 "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample_seconds(w, tokens=256, reps=1):
+    """Times the CPU oracle (fp64 numpy) on one decoder layer of the workload's
+    shape: forward + backward for `tokens` tokens of one sequence.  Weights are
+    random fp64 (their preparation is not timed)."""
+    import numpy as np
+
+    import soup_synth as ss
+    from oracle.layer import layer_bwd, layer_fwd
+    shape = ss.LayerShape(hidden=w["hidden"], n_q_heads=w["n_q_heads"], n_kv_heads=w["n_kv_heads"],
+                          head_dim=w["head_dim"], intermediate=w["intermediate"], rank=w["rank"], alpha=w["alpha"])
+    g = np.random.default_rng(0)
+    W = {p: g.standard_normal(shape.proj_shape(p)) * 0.02 for p in ss.PROJ_NAMES}
+    W["norm1"] = 1 + 0.02 * g.standard_normal(shape.hidden)
+    W["norm2"] = 1 + 0.02 * g.standard_normal(shape.hidden)
+    lora = {}
+    for p in ss.PROJ_NAMES:
+        o, i = shape.proj_shape(p)
+        lora[p] = (g.standard_normal((shape.rank, i)) * 0.02, g.standard_normal((o, shape.rank)) * 0.02)
+    h = g.standard_normal((1, tokens, shape.hidden))
+    dh = g.standard_normal(h.shape)
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        _, cache = layer_fwd(h, W, lora, shape)
+        layer_bwd(cache, W, lora, shape, dh)
+        times.append(time.perf_counter() - t0)
+    return min(times)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, tokens=256):
+    t = oracle_sample_seconds(w, tokens)
+    per_token_stack = t * w["n_layers"] / tokens
+    return {"value": 1.0 / per_token_stack, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"one {w['hidden']}-hidden decoder layer, fwd+bwd on 1x{tokens} tokens in fp64 numpy "
+                      f"({t:.2f} s), projected to the {w['n_layers']}-layer stack (head excluded)"}
+
+
+def run_reference(args, w, name):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup and 1):
+        pass
+    per = []
+    tokens = 256
+    for _ in range(args.steps):
+        per.append(oracle_sample_seconds(w, tokens))
+    t = statistics.median(per)
+    value = tokens / (t * w["n_layers"])
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t * w["n_layers"] * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": name, "global_batch": w["batch"], "seq_len": w["seq"], "layers": w["n_layers"]},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"per step: one decoder layer fwd+bwd on 1x{tokens} tokens, fp64 numpy, "
+                                       f"projected to {w['n_layers']} layers"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
+    ap.add_argument("--buffers", type=int, default=0, help="override stream_buffers (2..8)")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (diagnostics only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = dict(WORKLOADS[args.workload])
+    if args.buffers:
+        w["buffers"] = args.buffers
+    if args.layers:
+        w["n_layers"] = args.layers
+    if args.impl == "reference":
+        return run_reference(args, w, args.workload)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from layer_streamed_qlora_b200 import _lib as L
+    from layer_streamed_qlora_b200.model import ModelConfig, StreamedLoRAModel
+
+    cfg = ModelConfig(hidden=w["hidden"], n_q_heads=w["n_q_heads"], n_kv_heads=w["n_kv_heads"],
+                      head_dim=w["head_dim"], intermediate=w["intermediate"], rank=w["rank"], alpha=w["alpha"],
+                      vocab=w["vocab"], n_layers=w["n_layers"], kind=w["kind"], tied=w["tied"])
+    B, S = w["batch"], w["seq"]
+    cap = int(w["cap_gb"] * (1 << 30))
+    torch.cuda.reset_peak_memory_stats()
+    t_build = time.time()
+    model = StreamedLoRAModel(cfg, B, S, n_buffers=w["buffers"], device_cap_bytes=cap, seed=0)
+    t_build = time.time() - t_build
+    g = torch.Generator().manual_seed(1000 + rank)
+    ids_host = torch.randint(0, cfg.vocab, (B, S), generator=g, dtype=torch.int32).pin_memory()
+    loss_host = torch.zeros(1, dtype=torch.float32).pin_memory()
+    model.set_ids(ids_host)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    flat = None
+    if world > 1:
+        flat_numel = sum(v.numel() for gd in model.grads for v in gd.values())
+        flat = torch.empty(flat_numel, dtype=torch.float32, device="cuda")
+
+    def step():
+        loss = model.sft_step() if w["task"] == "sft" else model.dpo_step(w["prompt"], w["beta"])
+        if world > 1:
+            # data parallel: the one exchange of the step, the LoRA gradients
+            torch.cat([v.reshape(-1) for gd in model.grads for v in gd.values()], out=flat)
+            dist.all_reduce(flat)
+        return loss
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    model.plan.reset_stats()
+    clocks = ClockSampler(local)
+    clocks.start()
+    L.profile_enable(True)
+    n0 = L.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    launches = (L.launch_count() - n0) // args.steps
+    prof = L.profile_read()
+    L.profile_enable(False)
+    sstats = model.plan.stats()
+    clk = clocks.stop()
+
+    # end-to-end through the public API: host ids in, loss out, every step
+    torch.cuda.synchronize()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(st)
+    for _ in range(args.steps):
+        model.set_ids(ids_host)
+        loss = step()
+        loss_host.copy_(loss, non_blocking=True)
+        st.synchronize()
+    e3.record(st)
+    torch.cuda.synchronize()
+    ms_e2e = e2.elapsed_time(e3) / args.steps
+    if world > 1:
+        t = torch.tensor([ms, ms_e2e], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_e2e = float(t[0]), float(t[1])
+    tokens = B * S * world
+    value = tokens / (ms / 1e3)
+    pk, pk_kind = peaks()
+    # dominant kernel: the GEMM class with the most device time
+    dom_name, dom = max(prof.items(), key=lambda kv: kv[1]["total_ms"])
+    achieved = dom["flops"] / (dom["total_ms"] / 1e3) / 1e12 if dom["total_ms"] > 0 else 0.0
+    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    tr = gemm_traffic()
+    roofline = {"bound": "tensor", "kernel": f"gemm {dom_name}", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak if peak else None,
+                "traffic": tr.get("bytes_per_launch") if tr else None,
+                "peak_kind": f"{pk_kind} sustained bf16 (kernel timed inside a long step)",
+                "launches_per_step": dom["launches"] // args.steps,
+                "algorithmic_flops_per_launch": dom["flops"] / max(1, dom["launches"]),
+                "avg_launch_ms": dom["total_ms"] / max(1, dom["launches"])}
+    gemm_summary = {k: {"launches_per_step": v["launches"] // args.steps, "ms_per_step": v["total_ms"] / args.steps,
+                        "TFLOP/s": (v["flops"] / (v["total_ms"] / 1e3) / 1e12) if v["total_ms"] > 0 else None}
+                    for k, v in prof.items()}
+    h2d_bytes = sstats["bytes_copied"] / args.steps
+    copy_ms = sstats["copy_ms"] / args.steps
+    step_flops = sum(v["flops"] for v in prof.values()) / args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "global_batch": B * world, "seq_len": S, "layers": cfg.n_layers,
+                   "base": cfg.kind, "stream_buffers": w["buffers"], "device_cap_gb": w["cap_gb"],
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (the streamed base, >4 GB per step)"},
+        "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": ids_host.numel() * 4,
+                "d2h_bytes_per_step": 4},
+        "gpu_launches": launches,
+        "roofline": roofline,
+        "gemm_classes": gemm_summary,
+        "stream": {"h2d_gb_per_step": h2d_bytes / 1e9, "copies_per_step": sstats["copies"] / args.steps,
+                   "reused_per_step": sstats["reuses"] / args.steps,
+                   "h2d_gbs": (h2d_bytes / 1e9) / (copy_ms / 1e3) if copy_ms > 0 else None,
+                   "copy_ms_per_step": copy_ms, "stall_ms_per_step": sstats["stall_ms"] / args.steps,
+                   "stall_frac": (sstats["stall_ms"] / args.steps) / ms},
+        "gemm_tflops_per_step": step_flops / (ms / 1e3) / 1e12,
+        "peak_device_bytes": torch.cuda.max_memory_allocated() + sstats["arena_bytes"],
+        "build_s": t_build,
+        "loss": float(loss_host.item()),
+    }
+    if clk:
+        line["clocks"] = clk
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    model.close()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -54,6 +54,24 @@ const char* soup_last_error(void);
  * Returns SOUP_OK, or SOUP_ERR_CUDA if the read itself failed. */
 soup_status soup_device_error(int32_t* code_out);
 
+/* Number of kernels this library has launched in this process. */
+int64_t soup_launch_count(void);
+
+/* Optional timing of the tensor-core GEMM launches: when enabled, every GEMM
+ * launch is bracketed by CUDA events recorded on its own stream and tagged
+ * with its class and algorithmic work.  soup_profile_read synchronises those
+ * events and sums them per class: 0 = fused NF4-decode GEMM (forward, W),
+ * 1 = fused NF4-decode GEMM (backward, W^T), 2 = other bf16 GEMMs with
+ * N > 64, 3 = skinny LoRA GEMMs (N <= 64).  Enabling resets the records. */
+typedef struct soup_gemm_profile {
+  int64_t launches;
+  double total_ms;
+  double flops;  /* 2 M N (K + r_tail) summed over launches */
+  double bytes;  /* A read once + B (NF4 packed or bf16) + output written once */
+} soup_gemm_profile;
+soup_status soup_profile_enable(int32_t on);
+soup_status soup_profile_read(soup_gemm_profile* out, int32_t n_classes);
+
 /* ------------------------------------------------------------------ NF4 ---
  * NF4 block quantisation of the frozen base (the pages' `quantization: 4bit`
  * storage of the streamed base; Soup pages, "configuration and training" and
@@ -191,6 +209,133 @@ soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const soup_layer
                                    const float* dh_out, int64_t batch, int64_t seq, float* dh_in,
                                    const soup_layer_grads* grads, int32_t adapters_on,
                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------- layer streaming ---
+ * The frozen base lives in pinned host RAM as one blob per decoder layer
+ * (Soup pages, "how layer streaming works": per-layer shards in page-locked
+ * host memory; `stream_buffers` preallocated device buffers, 2..8, default 2;
+ * a dedicated CUDA stream copies the next layer while the current one
+ * computes; the vocab-sized embed_tokens and an untied lm_head share one
+ * slot).  A plan owns the only device memory this library allocates: an
+ * arena of n_buffers layer slots plus one vocab slot, a copy stream and
+ * events.  Slots are reused least-recently-released first; prefetching an
+ * item that is still resident in a released slot makes no copy.
+ */
+#define SOUP_ITEM_NONE (-100)
+#define SOUP_ITEM_EMBED (-1) /* the embed_tokens matrix, into the vocab slot */
+#define SOUP_ITEM_HEAD (-2)  /* the lm_head matrix, into the vocab slot */
+
+typedef struct soup_plan soup_plan; /* opaque */
+
+typedef struct soup_stream_desc {
+  int32_t n_layers;
+  size_t layer_bytes;              /* bytes of one layer blob (multiple of 256) */
+  const void* const* host_layers;  /* n_layers pinned host blobs */
+  size_t vocab_bytes;              /* bytes of the vocab slot (0: none; multiple of 256) */
+  const void* host_embed;          /* pinned host embed_tokens blob (vocab_bytes) or NULL */
+  const void* host_head;           /* pinned host lm_head blob or NULL (tied: same as embed) */
+  int32_t n_buffers;               /* stream_buffers: 2..8 */
+  size_t device_cap_bytes;         /* 0: no cap; else refuse plans that exceed it */
+  size_t reserve_bytes;            /* device bytes the caller holds besides the plan */
+} soup_stream_desc;
+
+typedef struct soup_stream_stats_t {
+  int64_t copies;      /* H2D copies issued */
+  int64_t reuses;      /* prefetches served by a still-resident slot */
+  size_t bytes_copied;
+  size_t arena_bytes;
+  int64_t waits;       /* soup_stream_wait calls */
+  double stall_ms;     /* total time the compute stream spent inside those waits */
+  double copy_ms;      /* total duration of the copies on the copy stream */
+} soup_stream_stats_t;
+
+/* Allocates the slot arena and the copy stream.  Refuses (no allocation)
+ * with SOUP_ERR_INVALID_ARG when n_buffers is outside [2, 8], and with
+ * SOUP_ERR_OOM_PLAN when n_buffers * layer_bytes + vocab_bytes +
+ * reserve_bytes exceeds a nonzero device_cap_bytes. */
+soup_status soup_stream_plan(const soup_stream_desc* desc, soup_plan** plan_out);
+soup_status soup_stream_plan_free(soup_plan* plan);
+
+/* Enqueues the copy of `item` (a layer index, SOUP_ITEM_EMBED or
+ * SOUP_ITEM_HEAD) into a free slot on the plan's copy stream; the copy first
+ * waits (on the device) until the compute stream released the slot's
+ * previous item.  Refuses when every slot of the kind holds an unreleased
+ * item or the item is already held. */
+soup_status soup_stream_prefetch(soup_plan* plan, int32_t item);
+
+/* Makes `compute_stream` wait (on the device) until the item's copy is done
+ * and returns the slot's device address in *slot_dev. */
+soup_status soup_stream_wait(soup_plan* plan, int32_t item, void* compute_stream, void** slot_dev);
+
+/* Host-side wait for the item's copy, at most timeout_ms; SOUP_ERR_TIMEOUT
+ * when it does not finish in time (the copy is left in flight). */
+soup_status soup_stream_wait_host(soup_plan* plan, int32_t item, int32_t timeout_ms);
+
+/* Marks the item's slot reusable once `compute_stream` reaches this point. */
+soup_status soup_stream_release(soup_plan* plan, int32_t item, void* compute_stream);
+
+/* Copy/stall statistics since the plan was made or last reset (synchronises
+ * the copy stream and the recorded events). */
+soup_status soup_stream_stats(soup_plan* plan, soup_stream_stats_t* out);
+soup_status soup_stream_stats_reset(soup_plan* plan);
+
+/* The plan's copy stream (cudaStream_t as void*). */
+void* soup_stream_copy_stream(soup_plan* plan);
+
+/* Fault-injection hooks for tests (host side only): the next prefetch fails
+ * with SOUP_ERR_CUDA without copying; or the next copy first waits on
+ * `event` (a cudaEvent_t). */
+soup_status soup_stream_debug_fail_next_copy(soup_plan* plan);
+soup_status soup_stream_debug_gate_next_copy(soup_plan* plan, void* event);
+
+/* Layer blob layout (host arithmetic, no device access).  NF4 blob: qkv
+ * codes | qkv absmax | o codes | o absmax | gate_up codes | gate_up absmax |
+ * down codes | down absmax | norm1 | norm2; bf16 blob: qkv | o | gate_up |
+ * down | norm1 | norm2; every part 256-byte aligned.  soup_layer_blob_views
+ * fills *out with pointers into a blob at `base`. */
+size_t soup_layer_blob_bytes(const soup_layer_cfg* cfg, int32_t kind);
+soup_status soup_layer_blob_views(const soup_layer_cfg* cfg, int32_t kind, const void* base,
+                                  soup_layer_weights* out);
+
+/* ------------------------------------------------------- embedding, head ---
+ * Token embedding gather: h[t] = E[ids[t]] (E [V, H] bf16 in the vocab slot,
+ * ids [T] int32).  An id outside [0, V) writes a zero row and sets code 2 in
+ * the device error word. */
+soup_status soup_embed(const uint16_t* E, int64_t V, int64_t H, const int32_t* ids, int64_t T,
+                       uint16_t* h, void* stream);
+
+/* Final RMSNorm + lm_head + next-token log-probabilities, `chunk` tokens at a
+ * time (the pages' stream_loss_chunk):  x = RMSNorm(h; w_final),
+ * logp[b, s] = log softmax(x_t E^T)[ids[b, s+1]] for t = b*seq + s, s < seq-1.
+ * h [batch*seq, H] bf16, E [V, H] bf16 (lm_head), ids [batch, seq] int32,
+ * logp [batch, seq-1] fp32.  When coef [batch, seq-1] (= dL/dlogp) is given,
+ * also dh [batch*seq, H] fp32 = dL/dh.  Logits are fp32; dL/dlogits enter the
+ * backward GEMM in bf16. */
+size_t soup_head_workspace(int64_t V, int64_t H, int64_t batch, int64_t seq, int32_t chunk);
+soup_status soup_head_fwd_bwd(const uint16_t* h, const uint16_t* w_final, const uint16_t* E, int64_t V,
+                              int64_t H, const int32_t* ids, int64_t batch, int64_t seq, float eps,
+                              int32_t chunk, const float* coef, float* logp, float* dh, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Mean next-token cross-entropy over batch*(seq-1) targets into *loss (a
+ * device float; optional, then logp may be NULL); coef (optional) <-
+ * dL/dlogp = -1/(batch*(seq-1)), which does not depend on logp and so can be
+ * produced before the head runs. */
+soup_status soup_ce_loss(const float* logp, int64_t batch, int64_t seq, float* loss, float* coef,
+                         void* stream);
+
+/* DPO loss (Rafailov et al. 2023) over `pairs` preference pairs; rows 2p /
+ * 2p+1 of the [2*pairs, seq-1] log-prob arrays are the chosen / rejected
+ * sequence of pair p, sharing a prompt of prompt_len tokens.  Sequence
+ * log-probs sum the targets at positions >= prompt_len (continuation tokens).
+ *   L = -(1/P) sum_p log sigmoid(beta [(pi_c - ref_c) - (pi_r - ref_r)])
+ * logp_policy: adapters on; logp_ref: the same streamed base with adapters
+ * off (the pages' memory-free reference model).  *loss (device) <- L;
+ * seq_sums (optional, [4*pairs]) <- policy sums then reference sums;
+ * coef [2*pairs, seq-1] <- dL/dlogp_policy (zero on prompt positions). */
+soup_status soup_dpo_loss(const float* logp_policy, const float* logp_ref, int64_t pairs, int64_t seq,
+                          int64_t prompt_len, float beta, float* loss, float* seq_sums, float* coef,
+                          void* stream);
 
 #ifdef __cplusplus
 }

@@ -54,10 +54,34 @@ class LayerGrads(ctypes.Structure):
                                         "dB_down")]
 
 
+class StreamDesc(ctypes.Structure):
+    _fields_ = [("n_layers", c_int32), ("layer_bytes", c_size_t), ("host_layers", ctypes.POINTER(c_void_p)),
+                ("vocab_bytes", c_size_t), ("host_embed", c_void_p), ("host_head", c_void_p),
+                ("n_buffers", c_int32), ("device_cap_bytes", c_size_t), ("reserve_bytes", c_size_t)]
+
+
+class StreamStats(ctypes.Structure):
+    _fields_ = [("copies", c_int64), ("reuses", c_int64), ("bytes_copied", c_size_t), ("arena_bytes", c_size_t),
+                ("waits", c_int64), ("stall_ms", ctypes.c_double), ("copy_ms", ctypes.c_double)]
+
+
+class GemmProfile(ctypes.Structure):
+    _fields_ = [("launches", c_int64), ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double)]
+
+
+GEMM_CLASSES = ("nf4_fwd", "nf4_bwd", "bf16", "lora_skinny")
+
+SOUP_ITEM_EMBED = -1
+SOUP_ITEM_HEAD = -2
+
 # name -> (restype, argtypes)
 _SIGS = {
     "soup_last_error": (ctypes.c_char_p, []),
     "soup_device_error": (c_int32, [ctypes.POINTER(c_int32)]),
+    "soup_launch_count": (c_int64, []),
+    "soup_profile_enable": (c_int32, [c_int32]),
+    "soup_profile_read": (c_int32, [ctypes.POINTER(GemmProfile), c_int32]),
     "soup_nf4_quantize": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_void_p]),
     "soup_nf4_dequant": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
     "soup_lora_linear_fwd": (c_int32, [ctypes.POINTER(SoupWeight), c_void_p, c_void_p, c_int32, c_float,
@@ -73,6 +97,26 @@ _SIGS = {
     "soup_decoder_layer_bwd": (c_int32, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerLora),
                                          ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_int64, c_int64, c_void_p,
                                          ctypes.POINTER(LayerGrads), c_int32, c_void_p, c_size_t, c_void_p]),
+    "soup_stream_plan": (c_int32, [ctypes.POINTER(StreamDesc), ctypes.POINTER(c_void_p)]),
+    "soup_stream_plan_free": (c_int32, [c_void_p]),
+    "soup_stream_prefetch": (c_int32, [c_void_p, c_int32]),
+    "soup_stream_wait": (c_int32, [c_void_p, c_int32, c_void_p, ctypes.POINTER(c_void_p)]),
+    "soup_stream_wait_host": (c_int32, [c_void_p, c_int32, c_int32]),
+    "soup_stream_release": (c_int32, [c_void_p, c_int32, c_void_p]),
+    "soup_stream_stats": (c_int32, [c_void_p, ctypes.POINTER(StreamStats)]),
+    "soup_stream_stats_reset": (c_int32, [c_void_p]),
+    "soup_stream_copy_stream": (c_void_p, [c_void_p]),
+    "soup_stream_debug_fail_next_copy": (c_int32, [c_void_p]),
+    "soup_stream_debug_gate_next_copy": (c_int32, [c_void_p, c_void_p]),
+    "soup_layer_blob_bytes": (c_size_t, [ctypes.POINTER(LayerCfg), c_int32]),
+    "soup_layer_blob_views": (c_int32, [ctypes.POINTER(LayerCfg), c_int32, c_void_p, ctypes.POINTER(LayerWeights)]),
+    "soup_embed": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_void_p]),
+    "soup_head_workspace": (c_size_t, [c_int64, c_int64, c_int64, c_int64, c_int32]),
+    "soup_head_fwd_bwd": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_int64, c_int64,
+                                    c_float, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "soup_ce_loss": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
+    "soup_dpo_loss": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_float, c_void_p, c_void_p,
+                                c_void_p, c_void_p]),
 }
 
 _lib = None
@@ -111,6 +155,20 @@ def device_error() -> int:
     v = c_int32(0)
     _check("soup_device_error", lib().soup_device_error(ctypes.byref(v)))
     return v.value
+
+
+def launch_count() -> int:
+    return int(lib().soup_launch_count())
+
+
+def profile_enable(on: bool):
+    _check("soup_profile_enable", lib().soup_profile_enable(1 if on else 0))
+
+
+def profile_read() -> dict:
+    arr = (GemmProfile * len(GEMM_CLASSES))()
+    _check("soup_profile_read", lib().soup_profile_read(arr, len(GEMM_CLASSES)))
+    return {name: {k: getattr(arr[i], k) for k, _ in GemmProfile._fields_} for i, name in enumerate(GEMM_CLASSES)}
 
 
 # ---------------------------------------------------------------- NF4
@@ -185,3 +243,98 @@ def soup_decoder_layer_bwd(W: LayerWeights, lora, cfg: LayerCfg, h_in, dh_out, b
     _check("soup_decoder_layer_bwd", lib().soup_decoder_layer_bwd(
         ctypes.byref(W), lp, ctypes.byref(cfg), _p(h_in), _p(dh_out), batch, seq, _p(dh_in), gp, int(adapters_on),
         _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- streaming
+class Plan:
+    """Owns a soup_plan (slot arena + copy stream)."""
+
+    def __init__(self, host_layers, layer_bytes, n_buffers, vocab_bytes=0, host_embed=None, host_head=None,
+                 device_cap_bytes=0, reserve_bytes=0):
+        self._arr = (c_void_p * len(host_layers))(*[t.data_ptr() for t in host_layers])
+        self._keep = (host_layers, host_embed, host_head)
+        d = StreamDesc(len(host_layers), layer_bytes, ctypes.cast(self._arr, ctypes.POINTER(c_void_p)), vocab_bytes,
+                       host_embed.data_ptr() if host_embed is not None else None,
+                       host_head.data_ptr() if host_head is not None else None, n_buffers, device_cap_bytes,
+                       reserve_bytes)
+        h = c_void_p()
+        _check("soup_stream_plan", lib().soup_stream_plan(ctypes.byref(d), ctypes.byref(h)))
+        self.h = h
+
+    def free(self):
+        if self.h:
+            lib().soup_stream_plan_free(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+    def prefetch(self, item):
+        _check("soup_stream_prefetch", lib().soup_stream_prefetch(self.h, item))
+
+    def wait(self, item, stream=None) -> int:
+        p = c_void_p()
+        _check("soup_stream_wait", lib().soup_stream_wait(self.h, item, _stream(stream), ctypes.byref(p)))
+        return p.value
+
+    def wait_host(self, item, timeout_ms):
+        _check("soup_stream_wait_host", lib().soup_stream_wait_host(self.h, item, timeout_ms))
+
+    def release(self, item, stream=None):
+        _check("soup_stream_release", lib().soup_stream_release(self.h, item, _stream(stream)))
+
+    def stats(self) -> dict:
+        s = StreamStats()
+        _check("soup_stream_stats", lib().soup_stream_stats(self.h, ctypes.byref(s)))
+        return {k: getattr(s, k) for k, _ in StreamStats._fields_}
+
+    def reset_stats(self):
+        _check("soup_stream_stats_reset", lib().soup_stream_stats_reset(self.h))
+
+    def copy_stream_handle(self) -> int:
+        return lib().soup_stream_copy_stream(self.h)
+
+    def debug_fail_next_copy(self):
+        _check("soup_stream_debug_fail_next_copy", lib().soup_stream_debug_fail_next_copy(self.h))
+
+    def debug_gate_next_copy(self, event_handle):
+        _check("soup_stream_debug_gate_next_copy", lib().soup_stream_debug_gate_next_copy(self.h, c_void_p(event_handle)))
+
+
+def soup_layer_blob_bytes(cfg: LayerCfg, kind) -> int:
+    return int(lib().soup_layer_blob_bytes(ctypes.byref(cfg), kind))
+
+
+def soup_layer_blob_views(cfg: LayerCfg, kind, base_ptr: int) -> LayerWeights:
+    w = LayerWeights()
+    _check("soup_layer_blob_views", lib().soup_layer_blob_views(ctypes.byref(cfg), kind, c_void_p(base_ptr),
+                                                                ctypes.byref(w)))
+    return w
+
+
+# ---------------------------------------------------------------- embedding / head / losses
+def soup_embed(E_ptr: int, V, H, ids, T, h, stream=None):
+    _check("soup_embed", lib().soup_embed(c_void_p(E_ptr), V, H, _p(ids), T, _p(h), _stream(stream)))
+
+
+def soup_head_workspace(V, H, batch, seq, chunk) -> int:
+    return int(lib().soup_head_workspace(V, H, batch, seq, chunk))
+
+
+def soup_head_fwd_bwd(h, w_final, E_ptr: int, V, H, ids, batch, seq, eps, chunk, coef, logp, dh, workspace,
+                      stream=None):
+    _check("soup_head_fwd_bwd", lib().soup_head_fwd_bwd(
+        _p(h), _p(w_final), c_void_p(E_ptr), V, H, _p(ids), batch, seq, eps, chunk, _p(coef), _p(logp), _p(dh),
+        _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def soup_ce_loss(logp, batch, seq, loss, coef, stream=None):
+    _check("soup_ce_loss", lib().soup_ce_loss(_p(logp), batch, seq, _p(loss), _p(coef), _stream(stream)))
+
+
+def soup_dpo_loss(logp_policy, logp_ref, pairs, seq, prompt_len, beta, loss, seq_sums, coef, stream=None):
+    _check("soup_dpo_loss", lib().soup_dpo_loss(_p(logp_policy), _p(logp_ref), pairs, seq, prompt_len, beta,
+                                                _p(loss), _p(seq_sums), _p(coef), _stream(stream)))

@@ -86,21 +86,21 @@ __global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const float* 
 // dh = dres + rinv * (dy*w - xh * mean(dy*w*xh)),  xh = x * rinv
 __global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ xf,
                                    const uint16_t* __restrict__ w, const float* __restrict__ rinv,
-                                   const uint16_t* __restrict__ dy, const float* __restrict__ dres, int T, int H,
-                                   float* __restrict__ dh, uint16_t* __restrict__ dh_bf16) {
+                                   const uint16_t* __restrict__ dy, const float* __restrict__ dyf,
+                                   const float* __restrict__ dres, int T, int H, float* __restrict__ dh,
+                                   uint16_t* __restrict__ dh_bf16) {
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= T) return;
   const float r = rinv[row];
   const size_t rb = (size_t)row * H;
-  const uint4* dyr = reinterpret_cast<const uint4*>(dy + rb);
   const uint4* wr = reinterpret_cast<const uint4*>(w);
   const int nch = H / 256;
   float dot = 0.f;
   for (int c = 0; c < nch; ++c) {
     float a[8], b[8], g[8];
     load8(x, xf, rb + (size_t)(c * 32 + lane) * 8, a);
-    unpack8(dyr[c * 32 + lane], b);
+    load8(dy, dyf, rb + (size_t)(c * 32 + lane) * 8, b);
     unpack8(wr[c * 32 + lane], g);
 #pragma unroll
     for (int i = 0; i < 8; ++i) dot += (b[i] * g[i]) * (a[i] * r);
@@ -109,7 +109,7 @@ __global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ x, const float* 
   for (int c = 0; c < nch; ++c) {
     float a[8], b[8], g[8], o[8];
     load8(x, xf, rb + (size_t)(c * 32 + lane) * 8, a);
-    unpack8(dyr[c * 32 + lane], b);
+    load8(dy, dyf, rb + (size_t)(c * 32 + lane) * 8, b);
     unpack8(wr[c * 32 + lane], g);
     const size_t base = rb + (size_t)(c * 32 + lane) * 8;
     const float4 d0 = dres ? reinterpret_cast<const float4*>(dres + base)[0] : make_float4(0, 0, 0, 0);
@@ -191,7 +191,15 @@ soup_status rmsnorm_bwd(const uint16_t* x, const float* x_f32, const uint16_t* w
                         const uint16_t* dy, const float* dres, int T, int H, float* dh, uint16_t* dh_bf16,
                         cudaStream_t st) {
   SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
-  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, rinv, dy, dres, T, H, dh, dh_bf16);
+  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, rinv, dy, nullptr, dres, T, H, dh, dh_bf16);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+soup_status rmsnorm_bwd_f32dy(const uint16_t* x, const uint16_t* w, const float* rinv, const float* dy, int T, int H,
+                              float* dh, cudaStream_t st) {
+  SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
+  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, nullptr, w, rinv, nullptr, dy, nullptr, T, H, dh, nullptr);
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
 }

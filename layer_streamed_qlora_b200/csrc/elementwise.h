@@ -11,6 +11,9 @@ soup_status rmsnorm_fwd(const uint16_t* x, const float* x_f32, const uint16_t* w
 soup_status rmsnorm_bwd(const uint16_t* x, const float* x_f32, const uint16_t* w, const float* rinv,
                         const uint16_t* dy, const float* dres, int T, int H, float* dh, uint16_t* dh_bf16,
                         cudaStream_t st);
+// Same with an fp32 upstream gradient and no residual (the final norm).
+soup_status rmsnorm_bwd_f32dy(const uint16_t* x, const uint16_t* w, const float* rinv, const float* dy, int T, int H,
+                              float* dh, cudaStream_t st);
 soup_status rope_table(int S, int head_dim, double theta, float* cosb, float* sinb, cudaStream_t st);
 soup_status rope_apply(uint16_t* buf, int T, int S, int ld, int col0, int nh, const float* cosb, const float* sinb,
                        bool inverse, cudaStream_t st);

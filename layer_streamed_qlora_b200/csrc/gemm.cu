@@ -657,8 +657,20 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
   constexpr int NT = 32 * (2 + (BMD >= B_NF4_K ? 8 : 4));
   const int ntiles = paired ? (d.pair_off + BN / 2 - 1) / (BN / 2) : (d.N + BN - 1) / BN;
   dim3 grid((d.M + BM - 1) / BM, ntiles);
+  if (profiling()) {
+    // algorithmic work: 2 M N K (+ 2 M N r for the LoRA tail); bytes: the
+    // operands read once and the output written once
+    const int cls = BMD == B_NF4_K ? GC_NF4_FWD : (BMD == B_NF4_MN ? GC_NF4_BWD : (d.N <= 64 ? GC_SKINNY : GC_BF16));
+    const double tail_k = d.tail_ksteps > 0 ? (double)d.tailA.rows : 0.0;
+    const double flops = 2.0 * d.M * d.N * ((double)d.K + (paired ? 16.0 : tail_k));
+    const double wbytes = (BMD >= B_NF4_K) ? (double)d.N * d.K * (0.5 + 4.0 / 64) : (double)d.N * d.K * 2;
+    const int oes = (d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T) ? 4 : 2;
+    const double bytes = (double)d.M * d.K * 2 + wbytes + (double)d.M * d.N * oes;
+    profile_begin(st, cls, flops, bytes);
+  }
   kern<<<grid, NT, C::SMEM, st>>>(mA, mB, mTA, mTB, ka);
   SOUP_LAUNCH_CHECK();
+  profile_end(st);
   return SOUP_OK;
 }
 

@@ -16,6 +16,9 @@
 //           residual-stream gradient and the mid-layer residual h2 stay fp32.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <cstring>
+
 #include "elementwise.h"
 #include "lora_internal.h"
 
@@ -390,5 +393,52 @@ extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const
     SOUP_TRY(lora_dA(P(x1), T, H, P(g_qkv), 3 * r, ldT, G->dA_qkv, st));
   }
   SOUP_TRY(rmsnorm_bwd(h_in, nullptr, W->norm1, PF(rinv1), P(dx1), PF(dh2), T, H, dh_in, nullptr, st));
+  return SOUP_OK;
+}
+
+namespace {
+struct BlobPart {
+  int64_t out, in;
+};
+}  // namespace
+
+extern "C" size_t soup_layer_blob_bytes(const soup_layer_cfg* cfg, int32_t kind) {
+  soup_layer_weights w;
+  if (soup_layer_blob_views(cfg, kind, nullptr, &w) != SOUP_OK) return 0;
+  // the last part is norm2 of `hidden` bf16 values
+  return reinterpret_cast<size_t>(w.norm2) + align256((size_t)cfg->hidden * 2);
+}
+
+extern "C" soup_status soup_layer_blob_views(const soup_layer_cfg* cfg, int32_t kind, const void* base,
+                                             soup_layer_weights* out) {
+  Dims m;
+  SOUP_TRY(make_dims(cfg, 1, 1, &m));
+  SOUP_CHECK(out, SOUP_ERR_INVALID_ARG, "soup_layer_blob_views: null out");
+  SOUP_CHECK(kind == SOUP_WEIGHT_NF4 || kind == SOUP_WEIGHT_BF16, SOUP_ERR_INVALID_ARG, "bad weight kind %d", kind);
+  SOUP_CHECK(soup_aligned(base, 256), SOUP_ERR_ALIGN, "soup_layer_blob_views: base not 256-byte aligned");
+  const char* b = static_cast<const char*>(base);
+  size_t o = 0;
+  const BlobPart parts[4] = {{m.qkv_w, m.H}, {m.H, m.o_in}, {2 * (int64_t)m.I, m.H}, {m.H, m.I}};
+  soup_weight* dst[4] = {&out->qkv, &out->o, &out->gate_up, &out->down};
+  for (int i = 0; i < 4; ++i) {
+    soup_weight& w = *dst[i];
+    memset(&w, 0, sizeof(w));
+    w.kind = kind;
+    w.out_features = parts[i].out;
+    w.in_features = parts[i].in;
+    const size_t n = (size_t)parts[i].out * parts[i].in;
+    if (kind == SOUP_WEIGHT_NF4) {
+      w.codes = reinterpret_cast<const uint8_t*>(b + o);
+      o += align256(n / 2);
+      w.absmax = reinterpret_cast<const float*>(b + o);
+      o += align256(n / 64 * 4);
+    } else {
+      w.w = reinterpret_cast<const uint16_t*>(b + o);
+      o += align256(n * 2);
+    }
+  }
+  out->norm1 = reinterpret_cast<const uint16_t*>(b + o);
+  o += align256((size_t)m.H * 2);
+  out->norm2 = reinterpret_cast<const uint16_t*>(b + o);
   return SOUP_OK;
 }

@@ -1,9 +1,11 @@
 // Library-wide runtime pieces: last-error strings, the device error word that
 // bounded kernel waits report into, and the driver entry point used to build
 // TMA tensor maps.
+#include <atomic>
 #include <cstdarg>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "soup_internal.h"
 
@@ -17,6 +19,17 @@ int* g_err_ptr[64] = {nullptr};
 std::mutex g_mu;
 soup::EncodeTiledFn g_encode = nullptr;
 bool g_encode_tried = false;
+std::atomic<long long> g_launches{0};
+
+struct ProfRec {
+  cudaEvent_t a, b;
+  int cls;
+  double flops, bytes;
+};
+bool g_prof = false;
+std::vector<ProfRec> g_prof_recs;
+size_t g_prof_used = 0;
+int g_prof_open = -1;
 }  // namespace
 
 namespace soup {
@@ -56,6 +69,36 @@ EncodeTiledFn encode_tiled() {
   return g_encode;
 }
 
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+bool profiling() { return g_prof; }
+
+void profile_begin(cudaStream_t st, int cls, double flops, double bytes) {
+  if (!g_prof) return;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_prof_used == g_prof_recs.size()) {
+    ProfRec r;
+    cudaEventCreate(&r.a);
+    cudaEventCreate(&r.b);
+    g_prof_recs.push_back(r);
+  }
+  ProfRec& r = g_prof_recs[g_prof_used];
+  r.cls = cls;
+  r.flops = flops;
+  r.bytes = bytes;
+  cudaEventRecord(r.a, st);
+  g_prof_open = (int)g_prof_used;
+}
+
+void profile_end(cudaStream_t st) {
+  if (!g_prof) return;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_prof_open < 0) return;
+  cudaEventRecord(g_prof_recs[g_prof_open].b, st);
+  g_prof_open = -1;
+  ++g_prof_used;
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -77,5 +120,34 @@ extern "C" soup_status soup_device_error(int32_t* code_out) {
   const int zero = 0;
   SOUP_CUDA_TRY(cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice));
   *code_out = v;
+  return SOUP_OK;
+}
+
+extern "C" int64_t soup_launch_count(void) { return g_launches.load(); }
+
+extern "C" soup_status soup_profile_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_prof = on != 0;
+  g_prof_used = 0;
+  g_prof_open = -1;
+  return SOUP_OK;
+}
+
+extern "C" soup_status soup_profile_read(soup_gemm_profile* out, int32_t n_classes) {
+  SOUP_CHECK(out && n_classes >= 1, SOUP_ERR_INVALID_ARG, "soup_profile_read: bad argument");
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int c = 0; c < n_classes; ++c) memset(&out[c], 0, sizeof(out[c]));
+  for (size_t i = 0; i < g_prof_used; ++i) {
+    const ProfRec& r = g_prof_recs[i];
+    SOUP_CUDA_TRY(cudaEventSynchronize(r.b));
+    float ms = 0;
+    SOUP_CUDA_TRY(cudaEventElapsedTime(&ms, r.a, r.b));
+    if (r.cls < n_classes) {
+      out[r.cls].launches += 1;
+      out[r.cls].total_ms += ms;
+      out[r.cls].flops += r.flops;
+      out[r.cls].bytes += r.bytes;
+    }
+  }
   return SOUP_OK;
 }

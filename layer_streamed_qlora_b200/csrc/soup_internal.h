@@ -28,6 +28,17 @@ EncodeTiledFn encode_tiled();
 
 int sm_count();
 
+// Counts kernel launches made by this library (every launch site goes
+// through SOUP_LAUNCH_CHECK).
+void count_launch();
+
+// Optional CUDA-event timing of GEMM launches, by class, on the launching
+// stream (enabled through soup_profile_enable).
+enum GemmClass : int { GC_NF4_FWD = 0, GC_NF4_BWD = 1, GC_BF16 = 2, GC_SKINNY = 3, GC_N = 4 };
+bool profiling();
+void profile_begin(cudaStream_t st, int cls, double flops, double bytes);
+void profile_end(cudaStream_t st);
+
 }  // namespace soup
 
 #define SOUP_CUDA_TRY(expr)                                                            \
@@ -51,6 +62,7 @@ int sm_count();
 
 #define SOUP_LAUNCH_CHECK()                                                            \
   do {                                                                                 \
+    ::soup::count_launch();                                                            \
     cudaError_t e__ = cudaGetLastError();                                              \
     if (e__ != cudaSuccess)                                                            \
       return ::soup::fail(SOUP_ERR_CUDA, "kernel launch: %s (%s:%d)", cudaGetErrorString(e__), \

@@ -1,0 +1,306 @@
+"""Layer-streamed LoRA training step over a frozen NF4 (or bf16) base.
+
+The Soup pages' method ("how layer streaming works"): the frozen base is cut
+into per-layer shards held in pinned host RAM; a ring of `stream_buffers`
+(2..8) device slots is filled by a dedicated copy stream while the compute
+stream works on the previous layer; the vocab-sized embed_tokens / lm_head
+share one slot; every layer is read once for the forward pass and once more
+for the checkpoint-recompute backward (layers still resident in the ring at
+the turn-around are not copied again); only the LoRA adapters (and their
+gradients) live in VRAM permanently.
+
+This module is host-side orchestration only: device memory comes from
+PyTorch, and every operation of the step (NF4 quantisation of the shards,
+embedding, the decoder layers forward and backward, the chunked output head
+and the losses) runs in the CUDA library through its C ABI (``_lib``).
+"""
+from __future__ import annotations
+
+import zlib
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib as L
+
+ITEM_EMBED, ITEM_HEAD = L.SOUP_ITEM_EMBED, L.SOUP_ITEM_HEAD
+PROJS = ("q", "k", "v", "o", "gate", "up", "down")
+
+
+@dataclass(frozen=True)
+class ModelConfig:
+    hidden: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    intermediate: int
+    rank: int
+    alpha: float
+    vocab: int
+    n_layers: int
+    eps: float = 1e-5
+    theta: float = 5e5
+    kind: str = "nf4"      # "nf4" or "bf16" frozen base
+    tied: bool = False     # lm_head == embed_tokens
+
+    @property
+    def qkv_out(self):
+        return (self.n_q_heads + 2 * self.n_kv_heads) * self.head_dim
+
+    @property
+    def o_in(self):
+        return self.n_q_heads * self.head_dim
+
+    def layer_cfg(self) -> L.LayerCfg:
+        return L.LayerCfg(self.hidden, self.n_q_heads, self.n_kv_heads, self.head_dim, self.intermediate,
+                          self.rank, float(self.alpha), float(self.eps), float(self.theta))
+
+    @property
+    def weight_kind(self):
+        return L.SOUP_WEIGHT_NF4 if self.kind == "nf4" else L.SOUP_WEIGHT_BF16
+
+
+def _seed(*parts) -> int:
+    return zlib.crc32("/".join(str(p) for p in parts).encode()) & 0x7FFFFFFF
+
+
+def _randn(shape, seed, std=1.0, mean=0.0):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    t = torch.randn(shape, generator=g, device="cuda", dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    if mean != 0.0:
+        t.add_(mean)
+    return t
+
+
+class SyntheticWeights:
+    """Seeded synthetic frozen base drawn on the device: projections N(0, 0.02),
+    RMSNorm weights 1 + 0.02 N(0, 1), embeddings N(0, 0.02)."""
+
+    def __init__(self, cfg: ModelConfig, seed: int = 0, std: float = 0.02):
+        self.cfg, self.seed, self.std = cfg, seed, std
+
+    def layer(self, l):
+        c = self.cfg
+        shapes = {"qkv": (c.qkv_out, c.hidden), "o": (c.hidden, c.o_in), "gate_up": (2 * c.intermediate, c.hidden),
+                  "down": (c.hidden, c.intermediate)}
+        out = {k: _randn(s, _seed(self.seed, l, k), self.std) for k, s in shapes.items()}
+        out["norm1"] = _randn((c.hidden,), _seed(self.seed, l, "norm1"), 0.02, 1.0).to(torch.bfloat16)
+        out["norm2"] = _randn((c.hidden,), _seed(self.seed, l, "norm2"), 0.02, 1.0).to(torch.bfloat16)
+        return out
+
+    def vocab(self, which):
+        c = self.cfg
+        return _randn((c.vocab, c.hidden), _seed(self.seed, which), self.std).to(torch.bfloat16)
+
+    def final_norm(self):
+        return _randn((self.cfg.hidden,), _seed(self.seed, "final_norm"), 0.02, 1.0).to(torch.bfloat16)
+
+    def lora(self, l):
+        c = self.cfg
+        r = c.rank
+        shapes = {"A_qkv": (3 * r, c.hidden), "B_qkv": (c.qkv_out, r), "A_o": (r, c.o_in), "B_o": (c.hidden, r),
+                  "A_gu": (2 * r, c.hidden), "B_gu": (2 * c.intermediate, r), "A_down": (r, c.intermediate),
+                  "B_down": (c.hidden, r)}
+        return {k: _randn(s, _seed(self.seed, l, k), 0.02).to(torch.bfloat16) for k, s in shapes.items()}
+
+
+class StreamedLoRAModel:
+    """Frozen base in pinned host blobs + a soup_plan slot ring + resident LoRA.
+
+    weights: an object with ``layer(l)`` (fused fp32 device matrices qkv, o,
+    gate_up, down and bf16 norm1/norm2), ``vocab(name)`` (bf16 [V, H]),
+    ``final_norm()`` and ``lora(l)`` (bf16 fused LoRA factors).
+    """
+
+    def __init__(self, cfg: ModelConfig, batch: int, seq: int, n_buffers: int = 2, device_cap_bytes: int = 0,
+                 head_chunk: int = 256, weights=None, seed: int = 0):
+        self.cfg, self.batch, self.seq, self.n_buffers = cfg, batch, seq, n_buffers
+        self.T = batch * seq
+        self.head_chunk = head_chunk
+        self.lcfg = cfg.layer_cfg()
+        weights = weights or SyntheticWeights(cfg, seed)
+        self._build_blobs(weights)
+        self._alloc(weights)
+        self.plan = L.Plan(self.host_layers, self.blob_bytes, n_buffers, self.vocab_bytes, self.host_embed,
+                           self.host_head, device_cap_bytes, self.reserve_bytes)
+        self._views = {}
+        # When set to a dict, the backward pass stores dL/d(layer input) of
+        # every layer in it (index l = input of layer l, n_layers = head output).
+        self.capture_dh = None
+
+    # ------------------------------------------------------------ shard build
+    def _build_blobs(self, weights):
+        cfg = self.cfg
+        kind = cfg.weight_kind
+        self.blob_bytes = L.soup_layer_blob_bytes(self.lcfg, kind)
+        staging = torch.empty(self.blob_bytes, dtype=torch.uint8, device="cuda")
+        base = staging.data_ptr()
+        v = L.soup_layer_blob_views(self.lcfg, kind, base)
+        flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+        st = torch.cuda.current_stream()
+
+        def region(ptr, nbytes):
+            off = ptr - base
+            return staging[off:off + nbytes]
+
+        self.host_layers = []
+        for l in range(cfg.n_layers):
+            w = weights.layer(l)
+            for name in ("qkv", "o", "gate_up", "down"):
+                sw = getattr(v, name)
+                W = w[name].contiguous()
+                assert tuple(W.shape) == (sw.out_features, sw.in_features), (name, W.shape)
+                n = W.numel()
+                if kind == L.SOUP_WEIGHT_NF4:
+                    st_ = L.lib().soup_nf4_quantize(L.c_void_p(W.data_ptr()), sw.out_features, sw.in_features,
+                                                    L.c_void_p(sw.codes), L.c_void_p(sw.absmax),
+                                                    L.c_void_p(flag.data_ptr()), L.c_void_p(st.cuda_stream))
+                    L._check("soup_nf4_quantize", st_)
+                else:
+                    region(sw.w, n * 2).view(torch.bfloat16).copy_(W.reshape(-1).to(torch.bfloat16))
+            region(v.norm1, cfg.hidden * 2).view(torch.bfloat16).copy_(w["norm1"].reshape(-1))
+            region(v.norm2, cfg.hidden * 2).view(torch.bfloat16).copy_(w["norm2"].reshape(-1))
+            hb = torch.empty(self.blob_bytes, dtype=torch.uint8, pin_memory=True)
+            hb.copy_(staging)
+            self.host_layers.append(hb)
+            del w
+        del staging
+        V, H = cfg.vocab, cfg.hidden
+        self.vocab_bytes = (V * H * 2 + 255) // 256 * 256
+
+        def pin_vocab(t):
+            hb = torch.zeros(self.vocab_bytes, dtype=torch.uint8, pin_memory=True)
+            hb[:V * H * 2].copy_(t.reshape(-1).view(torch.uint8))
+            return hb
+
+        self.host_embed = pin_vocab(weights.vocab("embed"))
+        self.host_head = self.host_embed if cfg.tied else pin_vocab(weights.vocab("lm_head"))
+        torch.cuda.synchronize()
+
+    # ------------------------------------------------------------ device state
+    def _alloc(self, weights):
+        cfg, T = self.cfg, self.T
+        before = torch.cuda.memory_allocated()
+        self.final_norm = weights.final_norm().contiguous()
+        self.lora = [{k: v.contiguous() for k, v in weights.lora(l).items()} for l in range(cfg.n_layers)]
+        self.grads = [{"d" + k: torch.zeros(v.shape, dtype=torch.float32, device="cuda") for k, v in lo.items()}
+                      for lo in self.lora]
+        self.lora_s = [L.layer_lora(lo) for lo in self.lora]
+        self.grads_s = [L.layer_grads(g) for g in self.grads]
+        self.ckpt = torch.empty((cfg.n_layers + 1, T, cfg.hidden), dtype=torch.bfloat16, device="cuda")
+        self.dh = torch.empty((T, cfg.hidden), dtype=torch.float32, device="cuda")
+        self.ws = torch.empty(L.soup_decoder_layer_workspace(self.lcfg, self.batch, self.seq), dtype=torch.uint8,
+                              device="cuda")
+        self.head_ws = torch.empty(L.soup_head_workspace(cfg.vocab, cfg.hidden, self.batch, self.seq,
+                                                         self.head_chunk), dtype=torch.uint8, device="cuda")
+        self.logp = torch.empty((self.batch, self.seq - 1), dtype=torch.float32, device="cuda")
+        self.logp_ref = torch.empty_like(self.logp)
+        self.coef = torch.empty_like(self.logp)
+        self.loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+        self.seq_sums = torch.zeros(4 * max(1, self.batch // 2), dtype=torch.float32, device="cuda")
+        self.ids = torch.empty((self.batch, self.seq), dtype=torch.int32, device="cuda")
+        self.reserve_bytes = torch.cuda.memory_allocated() - before
+
+    def views(self, base: int) -> L.LayerWeights:
+        w = self._views.get(base)
+        if w is None:
+            w = L.soup_layer_blob_views(self.lcfg, self.cfg.weight_kind, base)
+            self._views[base] = w
+        return w
+
+    @property
+    def head_item(self):
+        return ITEM_EMBED if self.cfg.tied else ITEM_HEAD
+
+    # ------------------------------------------------------------ passes
+    def _embed(self):
+        """ckpt[0] = embed_tokens[ids].  The gather reads its rows straight
+        from the pinned host matrix (mapped into the device address space), so
+        only the batch's rows cross the host link, not the whole vocab matrix;
+        the vocab slot is left to the lm_head."""
+        L.soup_embed(self.host_embed.data_ptr(), self.cfg.vocab, self.cfg.hidden, self.ids, self.T, self.ckpt[0])
+
+    def _forward_layers(self, adapters_on: bool):
+        """ckpt[0] -> ckpt[L], saving every layer input (the checkpoints)."""
+        P, N, nl = self.plan, self.n_buffers, self.cfg.n_layers
+        for l in range(min(N, nl)):
+            P.prefetch(l)
+        for l in range(nl):
+            base = P.wait(l)
+            L.soup_decoder_layer_fwd(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.batch, self.seq,
+                                     self.ckpt[l + 1], adapters_on, self.ws)
+            P.release(l)
+            if l + N < nl:
+                P.prefetch(l + N)
+
+    def _head(self, coef, logp, dh):
+        P = self.plan
+        P.prefetch(self.head_item)
+        E = P.wait(self.head_item)
+        L.soup_head_fwd_bwd(self.ckpt[self.cfg.n_layers], self.final_norm, E, self.cfg.vocab, self.cfg.hidden,
+                            self.ids, self.batch, self.seq, self.cfg.eps, self.head_chunk, coef, logp, dh,
+                            self.head_ws)
+        P.release(self.head_item)
+
+    def _backward_layers(self):
+        P, N, nl = self.plan, self.n_buffers, self.cfg.n_layers
+        for l in range(nl - 1, max(nl - 1 - N, -1), -1):
+            P.prefetch(l)  # the layers still resident from the forward pass are reused, not copied
+        for l in range(nl - 1, -1, -1):
+            if self.capture_dh is not None:  # inspection hook for layer-by-layer checks
+                self.capture_dh[l + 1] = self.dh.clone()
+            base = P.wait(l)
+            L.soup_decoder_layer_bwd(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.dh, self.batch,
+                                     self.seq, self.dh, self.grads_s[l], 1, self.ws)
+            P.release(l)
+            if l - N >= 0:
+                P.prefetch(l - N)
+        if self.capture_dh is not None:
+            self.capture_dh[0] = self.dh.clone()
+
+    # ------------------------------------------------------------ steps
+    def set_ids(self, ids_host):
+        """Copies a step's token ids [batch, seq] (pinned int32 host tensor) to the device."""
+        self.ids.copy_(ids_host, non_blocking=True)
+
+    def sft_step(self):
+        """One SFT step on self.ids: next-token CE; leaves LoRA grads in self.grads
+        and the loss in self.loss (device)."""
+        self._embed()
+        self._forward_layers(True)
+        L.soup_ce_loss(None, self.batch, self.seq, None, self.coef)
+        self._head(self.coef, self.logp, self.dh)
+        L.soup_ce_loss(self.logp, self.batch, self.seq, self.loss, None)
+        self._backward_layers()
+        return self.loss
+
+    def dpo_step(self, prompt_len: int, beta: float):
+        """One DPO step on self.ids ([2P, seq]: rows 2p chosen, 2p+1 rejected):
+        reference pass with adapters off over the same streamed base, policy
+        pass with adapters on, DPO loss, backward through the policy."""
+        pairs = self.batch // 2
+        self._embed()
+        self._forward_layers(False)
+        self._head(None, self.logp_ref, None)
+        self._forward_layers(True)
+        self._head(None, self.logp, None)
+        L.soup_dpo_loss(self.logp, self.logp_ref, pairs, self.seq, prompt_len, beta, self.loss, self.seq_sums,
+                        self.coef)
+        self._head(self.coef, self.logp, self.dh)
+        self._backward_layers()
+        return self.loss
+
+    def forward_logprobs(self, adapters_on=True):
+        """Forward only (no grads): per-token log-probs into self.logp."""
+        self._embed()
+        self._forward_layers(adapters_on)
+        self._head(None, self.logp, None)
+        return self.logp
+
+    def close(self):
+        if getattr(self, "plan", None) is not None:
+            self.plan.free()
+            self.plan = None

@@ -1,0 +1,109 @@
+"""GPU checks of the slot ring: bytes arrive intact, resident items are reused
+without a copy, the host wait times out instead of hanging, an injected copy
+failure surfaces as a status, and a full ring refuses another prefetch.
+Nothing here faults or hangs the GPU: the delayed copy waits on an event
+recorded on another stream after a short, bounded spin (torch.cuda._sleep)."""
+import time
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+L = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    global L
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from layer_streamed_qlora_b200 import _lib as lib
+    lib.lib()
+    L = lib
+    yield
+
+
+def _blobs(n, nbytes):
+    out = []
+    for i in range(n):
+        t = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+        t.copy_(torch.randint(0, 256, (nbytes,), dtype=torch.uint8, generator=torch.Generator().manual_seed(i)))
+        out.append(t)
+    return out
+
+
+def test_round_trip_reuse_and_refusal():
+    nb = 1 << 20
+    blobs = _blobs(5, nb)
+    plan = L.Plan(blobs, nb, 2)
+    seen = {}
+    for item in range(5):
+        if item >= 2:
+            plan.release(item - 2)
+        plan.prefetch(item)
+        ptr = plan.wait(item)
+        seen[item] = ptr
+    torch.cuda.synchronize()
+    s = plan.stats()
+    assert s["copies"] == 5 and s["reuses"] == 0 and s["bytes_copied"] == 5 * nb
+    # both slots hold unreleased items: a third prefetch is refused
+    with pytest.raises(L.SoupError):
+        plan.prefetch(0)
+    plan.release(3)
+    plan.release(4)
+    plan.prefetch(4)  # still resident: reused, no copy
+    assert plan.stats()["reuses"] == 1
+    plan.release(4)
+    plan.free()
+
+
+def test_slot_contents_are_the_host_bytes():
+    nb = 1 << 16
+    blobs = _blobs(3, nb)
+    plan = L.Plan(blobs, nb, 2)
+    # read the slot back with the embedding gather: the slot viewed as
+    # [nb/16, 8] bf16 rows (16 bytes each), ids = every row
+    rows = nb // 16
+    ids = torch.arange(rows, dtype=torch.int32, device="cuda")
+    out = torch.empty((rows, 8), dtype=torch.bfloat16, device="cuda")
+    for item in range(3):
+        if item >= 2:
+            plan.release(item - 2)
+        plan.prefetch(item)
+        ptr = plan.wait(item)
+        L.soup_embed(ptr, rows, 8, ids, rows, out)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.uint8).reshape(-1).cpu(), blobs[item])
+    plan.free()
+
+
+def test_host_wait_times_out_then_completes():
+    nb = 1 << 20
+    blobs = _blobs(2, nb)
+    plan = L.Plan(blobs, nb, 2)
+    gate_stream = torch.cuda.Stream()
+    ev = torch.cuda.Event()
+    with torch.cuda.stream(gate_stream):
+        torch.cuda._sleep(int(4e8))  # ~0.2 s of bounded device-side spinning on the gate stream only
+        ev.record()
+    plan.debug_gate_next_copy(ev.cuda_event)
+    plan.prefetch(0)
+    t0 = time.time()
+    with pytest.raises(L.SoupError) as e:
+        plan.wait_host(0, 10)
+    assert e.value.status == 6  # SOUP_ERR_TIMEOUT
+    assert time.time() - t0 < 0.15
+    plan.wait_host(0, 30000)  # the copy does finish once the gate opens
+    plan.free()
+
+
+def test_injected_copy_failure_is_a_status():
+    nb = 1 << 16
+    plan = L.Plan(_blobs(2, nb), nb, 2)
+    plan.debug_fail_next_copy()
+    with pytest.raises(L.SoupError) as e:
+        plan.prefetch(0)
+    assert e.value.status == 7
+    plan.prefetch(0)  # the next one works
+    plan.wait_host(0, 10000)
+    plan.free()

@@ -1,0 +1,65 @@
+"""CPU checks of the stream planner's refusals (they happen before any CUDA
+call): stream_buffers outside [2, 8], a plan that does not fit the device cap,
+misaligned sizes, missing host blobs.  Refuse, never clamp."""
+import ctypes
+
+import pytest
+
+from layer_streamed_qlora_b200 import _lib as L
+
+
+def _desc(n_layers=4, layer_bytes=1 << 20, n_buffers=2, cap=0, reserve=0, vocab=0, null_layer=False):
+    ptrs = (ctypes.c_void_p * n_layers)(*[0x1000 * (i + 1) for i in range(n_layers)])
+    if null_layer:
+        ptrs[1] = None
+    d = L.StreamDesc(n_layers, layer_bytes, ctypes.cast(ptrs, ctypes.POINTER(ctypes.c_void_p)), vocab, None, None,
+                     n_buffers, cap, reserve)
+    return d, ptrs
+
+
+def _plan_status(d):
+    h = ctypes.c_void_p()
+    st = L.lib().soup_stream_plan(ctypes.byref(d), ctypes.byref(h))
+    return st, h
+
+
+@pytest.mark.parametrize("nb", [0, 1, 9, 16])
+def test_buffers_out_of_range_refused(nb):
+    d, keep = _desc(n_buffers=nb)
+    st, h = _plan_status(d)
+    assert st == 1 and not h.value
+    assert b"[2, 8]" in L.lib().soup_last_error()
+
+
+def test_cap_too_small_refused():
+    # 2 slots x 100 MiB + 50 MiB reserve > 200 MiB cap
+    d, keep = _desc(layer_bytes=100 << 20, n_buffers=2, cap=200 << 20, reserve=50 << 20)
+    st, h = _plan_status(d)
+    assert st == 5 and not h.value  # SOUP_ERR_OOM_PLAN
+    assert b"cap" in L.lib().soup_last_error()
+
+
+def test_misaligned_and_missing_refused():
+    d, keep = _desc(layer_bytes=1000)
+    assert _plan_status(d)[0] == 3  # SOUP_ERR_ALIGN
+    d, keep = _desc(null_layer=True)
+    assert _plan_status(d)[0] == 1
+    d, keep = _desc(vocab=100)
+    assert _plan_status(d)[0] == 3
+
+
+def test_blob_layout_sizes_match_the_shapes():
+    import soup_synth as ss
+    c = L.layer_cfg(ss.LLAMA8B_LAYER)
+    nf4 = L.soup_layer_blob_bytes(c, L.SOUP_WEIGHT_NF4)
+    bf = L.soup_layer_blob_bytes(c, L.SOUP_WEIGHT_BF16)
+    params = 6144 * 4096 + 4096 * 4096 + 2 * 14336 * 4096 + 4096 * 14336
+    assert params == 218_103_808
+    # codes (1/2 byte) + absmax (4 bytes / 64) + two norms, each part 256-aligned
+    assert abs(nf4 - (params // 2 + params // 16 + 2 * 4096 * 2)) < 10 * 256
+    assert abs(bf - (params * 2 + 2 * 4096 * 2)) < 10 * 256
+    v = L.soup_layer_blob_views(c, L.SOUP_WEIGHT_NF4, 0)
+    assert v.qkv.out_features == 6144 and v.down.in_features == 14336
+    assert v.norm2 + 4096 * 2 <= nf4
+    cq = L.layer_cfg(ss.QWEN3B_LAYER)
+    assert abs(L.soup_layer_blob_bytes(cq, L.SOUP_WEIGHT_BF16) - 154_148_864) < 10 * 256
