@@ -142,6 +142,31 @@ soup_status soup_lora_linear_bwd(const soup_weight* W, const uint16_t* A, const 
                                  uint16_t* dx, float* dA, float* dB, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* Allocation-free variant of soup_lora_linear_bwd (the pages have no
+ * counterpart: this is an integration convenience).  For callers that cannot
+ * allocate device memory when they run the backward, e.g. an integration
+ * whose device memory is entirely owned by another allocator's pool, or a
+ * latency-critical path where cudaMalloc (which may synchronise the device)
+ * is not allowed.  Same arguments and results as soup_lora_linear_bwd minus
+ * the workspace: the scratch lives in a static device array of
+ * soup_lora_linear_bwd_noalloc_max_scratch() bytes (8 MiB) that every GPU
+ * loading the library holds until the process exits.
+ *  - Sizes whose scratch, soup_lora_linear_bwd_workspace(T, r, out), exceeds
+ *    that maximum are refused with SOUP_ERR_SHAPE and a message (nothing runs).
+ *  - The first call on each device does a one-time set-up (it looks up the
+ *    array's device address with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array and it keeps the last call's contents:
+ *    calls that overlap on the GPU (different streams, or different host
+ *    threads on one device) race and corrupt each other's results; serialise
+ *    them.  No part of the scratch has to start at zero.
+ *  - Never calls cudaMalloc, cudaFree or any allocating routine. */
+size_t soup_lora_linear_bwd_noalloc_max_scratch(void);
+soup_status soup_lora_linear_bwd_noalloc(const soup_weight* W, const uint16_t* A, const uint16_t* B,
+                                         int32_t r, float scale, const uint16_t* x,
+                                         const uint16_t* u_save, const uint16_t* dy, int64_t T,
+                                         uint16_t* dx, float* dA, float* dB, void* stream);
+
 /* --------------------------------------------------------- decoder layer ---
  * One Llama-style decoder layer with LoRA on all seven projections (the unit
  * the pages stream "one decoder layer at a time"; Soup pages, "layer

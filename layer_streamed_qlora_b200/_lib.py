@@ -90,6 +90,10 @@ _SIGS = {
     "soup_lora_linear_bwd": (c_int32, [ctypes.POINTER(SoupWeight), c_void_p, c_void_p, c_int32, c_float,
                                        c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
                                        c_void_p, c_size_t, c_void_p]),
+    "soup_lora_linear_bwd_noalloc_max_scratch": (c_size_t, []),
+    "soup_lora_linear_bwd_noalloc": (c_int32, [ctypes.POINTER(SoupWeight), c_void_p, c_void_p, c_int32, c_float,
+                                               c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
+                                               c_void_p]),
     "soup_decoder_layer_workspace": (c_size_t, [ctypes.POINTER(LayerCfg), c_int64, c_int64]),
     "soup_decoder_layer_fwd": (c_int32, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerLora),
                                          ctypes.POINTER(LayerCfg), c_void_p, c_int64, c_int64, c_void_p, c_int32,
@@ -206,6 +210,17 @@ def soup_lora_linear_bwd(W: SoupWeight, A, B, r, scale, x, u_save, dy, T, dx, dA
     _check("soup_lora_linear_bwd", lib().soup_lora_linear_bwd(
         ctypes.byref(W), _p(A), _p(B), r, scale, _p(x), _p(u_save), _p(dy), T, _p(dx), _p(dA), _p(dB),
         _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def soup_lora_linear_bwd_noalloc_max_scratch() -> int:
+    return int(lib().soup_lora_linear_bwd_noalloc_max_scratch())
+
+
+def soup_lora_linear_bwd_noalloc(W: SoupWeight, A, B, r, scale, x, u_save, dy, T, dx, dA, dB, stream=None):
+    """soup_lora_linear_bwd without a workspace (static scratch; see soup.h)."""
+    _check("soup_lora_linear_bwd_noalloc", lib().soup_lora_linear_bwd_noalloc(
+        ctypes.byref(W), _p(A), _p(B), r, scale, _p(x), _p(u_save), _p(dy), T, _p(dx), _p(dA), _p(dB),
+        _stream(stream)))
 
 
 # ---------------------------------------------------------------- decoder layer

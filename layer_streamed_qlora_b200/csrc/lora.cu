@@ -12,6 +12,8 @@
 // works").
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "gemm.h"
 #include "lora_internal.h"
 
@@ -176,4 +178,64 @@ extern "C" soup_status soup_lora_linear_bwd(const soup_weight* W, const uint16_t
   g4.B = Mat{gt, r, T, ldT};
   g4.out_kind = OUT_F32_T; g4.out = dA; g4.ldo = in;
   return gemm(g4, st);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the LoRA linear backward.
+//
+// For callers that cannot allocate device memory when they run the backward
+// (for example an integration whose device memory is entirely owned by
+// another allocator's pool, or a latency-critical path where cudaMalloc,
+// which may synchronise the device, is not allowed).  Its scratch (the
+// transposed B and the g' = bf16(s dy B) buffer) lives in this file-scope
+// array instead of a caller-provided workspace.  Every GPU that loads the
+// library holds the array until the process exits.
+#define SOUP_NOALLOC_SCRATCH_BYTES (8u << 20)
+static __device__ __align__(256) uint8_t g_lora_noalloc_scratch[SOUP_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of the scratch array on the current device.  Host code may
+// not pass the array's name to a kernel (that is a host-side stand-in, not a
+// device address), so it is looked up once per device, with that device
+// current, and cached.
+soup_status noalloc_scratch(void** out) {
+  int dev = 0;
+  SOUP_CUDA_TRY(cudaGetDevice(&dev));
+  SOUP_CHECK(dev >= 0 && dev < 64, SOUP_ERR_INVALID_ARG, "soup_lora_linear_bwd_noalloc: device %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    SOUP_CUDA_TRY(cudaGetSymbolAddress(&p, g_lora_noalloc_scratch));
+    SOUP_CHECK(p != nullptr && soup_aligned(p, 256), SOUP_ERR_CUDA, "soup_lora_linear_bwd_noalloc: bad scratch address");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SOUP_OK;
+}
+}  // namespace
+
+extern "C" size_t soup_lora_linear_bwd_noalloc_max_scratch(void) { return SOUP_NOALLOC_SCRATCH_BYTES; }
+
+extern "C" soup_status soup_lora_linear_bwd_noalloc(const soup_weight* W, const uint16_t* A, const uint16_t* B,
+                                                    int32_t r, float scale, const uint16_t* x,
+                                                    const uint16_t* u_save, const uint16_t* dy, int64_t T,
+                                                    uint16_t* dx, float* dA, float* dB, void* stream) {
+  SOUP_CHECK(W, SOUP_ERR_INVALID_ARG, "soup_lora_linear_bwd_noalloc: null weight");
+  const size_t need = soup_lora_linear_bwd_workspace(T, r, W->out_features);
+  SOUP_CHECK(need > 0, SOUP_ERR_SHAPE, "soup_lora_linear_bwd_noalloc: bad sizes (T=%lld r=%d out=%lld)",
+             (long long)T, r, (long long)W->out_features);
+  SOUP_CHECK(need <= SOUP_NOALLOC_SCRATCH_BYTES, SOUP_ERR_SHAPE,
+             "soup_lora_linear_bwd_noalloc: T=%lld, r=%d, out=%lld need %zu bytes of scratch, more than the "
+             "static maximum of %u bytes; use soup_lora_linear_bwd with a workspace",
+             (long long)T, r, (long long)W->out_features, need, SOUP_NOALLOC_SCRATCH_BYTES);
+  void* ws = nullptr;
+  SOUP_TRY(noalloc_scratch(&ws));
+  // Every byte of the scratch that this call reads it first writes (the
+  // transpose fills B^T, the GEMM fills g' for columns [0, T), the only ones
+  // read), so nothing left by an earlier call needs clearing.
+  return soup_lora_linear_bwd(W, A, B, r, scale, x, u_save, dy, T, dx, dA, dB, ws, SOUP_NOALLOC_SCRATCH_BYTES,
+                              stream);
 }
