@@ -14,6 +14,7 @@
 #include <cuda_fp16.h>
 
 #include "elementwise.h"
+#include "gscale.cuh"
 
 namespace soup {
 namespace {
@@ -91,7 +92,7 @@ __device__ __forceinline__ const uint16_t* bk_addr(const uint16_t* tile, int k0,
 // `scale`, rotating pairs (i, i+64) back by the position's angle when tables
 // are given: (a, b) -> (a c + b s, b c - a s).
 __device__ __forceinline__ void store_row_rot(uint16_t* p, const float (&acc)[16][4], int e0, float scale,
-                                              const float* cosr, const float* sinr, int t4) {
+                                              const float* cosr, const float* sinr, int t4, float* p32 = nullptr) {
 #pragma unroll
   for (int dt = 0; dt < 8; ++dt) {
     float a0 = acc[dt][e0] * scale, a1 = acc[dt][e0 + 1] * scale;
@@ -105,13 +106,18 @@ __device__ __forceinline__ void store_row_rot(uint16_t* p, const float (&acc)[16
     }
     *reinterpret_cast<uint32_t*>(p + dt * 8 + 2 * t4) = packbf(a0, a1);
     *reinterpret_cast<uint32_t*>(p + 64 + dt * 8 + 2 * t4) = packbf(b0, b1);
+    if (p32) {
+      *reinterpret_cast<float2*>(p32 + dt * 8 + 2 * t4) = make_float2(a0, a1);
+      *reinterpret_cast<float2*>(p32 + 64 + dt * 8 + 2 * t4) = make_float2(b0, b1);
+    }
   }
 }
 
 // ------------------------------------------------------------------ forward
 __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restrict__ qkv, int ld, int S, int Hq,
                                                         int Hkv, uint16_t* __restrict__ out,
-                                                        float* __restrict__ lse, float scale_log2) {
+                                                        float* __restrict__ lse, float scale_log2,
+                                                        uint16_t* __restrict__ out16, float* __restrict__ out32) {
   extern __shared__ __align__(16) uint16_t sm[];
   uint16_t* Qs = sm;
   uint16_t* Ks = Qs + 64 * LDS;   // 2 buffers
@@ -224,17 +230,23 @@ __global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restric
   const float i0 = 1.f / l0, i1 = 1.f / l1;
   const int ldo = Hq * HD;
   if (qr0 < S) {
-    uint16_t* op = out + (size_t)(row0 + qr0) * ldo + h * HD;
+    const size_t off = (size_t)(row0 + qr0) * ldo + h * HD;
 #pragma unroll
-    for (int dt = 0; dt < 16; ++dt)
-      *reinterpret_cast<uint32_t*>(op + dt * 8 + 2 * t4) = packbf(o[dt][0] * i0, o[dt][1] * i0);
+    for (int dt = 0; dt < 16; ++dt) {
+      *reinterpret_cast<uint32_t*>(out + off + dt * 8 + 2 * t4) = packbf(o[dt][0] * i0, o[dt][1] * i0);
+      if (out16) *reinterpret_cast<uint32_t*>(out16 + off + dt * 8 + 2 * t4) = packh(o[dt][0] * i0, o[dt][1] * i0);
+      if (out32) *reinterpret_cast<float2*>(out32 + off + dt * 8 + 2 * t4) = make_float2(o[dt][0] * i0, o[dt][1] * i0);
+    }
     if (t4 == 0) lse[(size_t)h * T + row0 + qr0] = m0 + log2f(l0);
   }
   if (qr1 < S) {
-    uint16_t* op = out + (size_t)(row0 + qr1) * ldo + h * HD;
+    const size_t off = (size_t)(row0 + qr1) * ldo + h * HD;
 #pragma unroll
-    for (int dt = 0; dt < 16; ++dt)
-      *reinterpret_cast<uint32_t*>(op + dt * 8 + 2 * t4) = packbf(o[dt][2] * i1, o[dt][3] * i1);
+    for (int dt = 0; dt < 16; ++dt) {
+      *reinterpret_cast<uint32_t*>(out + off + dt * 8 + 2 * t4) = packbf(o[dt][2] * i1, o[dt][3] * i1);
+      if (out16) *reinterpret_cast<uint32_t*>(out16 + off + dt * 8 + 2 * t4) = packh(o[dt][2] * i1, o[dt][3] * i1);
+      if (out32) *reinterpret_cast<float2*>(out32 + off + dt * 8 + 2 * t4) = make_float2(o[dt][2] * i1, o[dt][3] * i1);
+    }
     if (t4 == 0) lse[(size_t)h * T + row0 + qr1] = m1 + log2f(l1);
   }
 }
@@ -248,7 +260,9 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const uint16_t* __re
                                                              const float* __restrict__ Dd,
                                                              uint16_t* __restrict__ dqkv, float scale_log2,
                                                              float scale, const float* __restrict__ rcos,
-                                                             const float* __restrict__ rsin) {
+                                                             const float* __restrict__ rsin,
+                                                             const unsigned int* __restrict__ amax,
+                                                             float* __restrict__ dqkv32) {
   extern __shared__ __align__(16) uint16_t sm[];
   uint16_t* Ks = sm;
   uint16_t* Vs = Ks + 64 * LDS;
@@ -363,15 +377,19 @@ __global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const uint16_t* __re
       }
     }
   }
+  // dO carried the power-of-two gradient scale: undo it (exact)
+  const float unscale = amax ? 1.f / grad_scale_from_amax(__uint_as_float(*amax)) : 1.f;
   if (key0 < S) {
-    store_row_rot(dqkv + (size_t)(row0 + key0) * ld + kcol, dk, 0, scale, rcos ? rcos + (size_t)key0 * 64 : nullptr,
-                  rsin ? rsin + (size_t)key0 * 64 : nullptr, t4);
-    store_row_rot(dqkv + (size_t)(row0 + key0) * ld + vcol, dv, 0, 1.f, nullptr, nullptr, t4);
+    const size_t r = (size_t)(row0 + key0) * ld;
+    store_row_rot(dqkv + r + kcol, dk, 0, scale * unscale, rcos ? rcos + (size_t)key0 * 64 : nullptr,
+                  rsin ? rsin + (size_t)key0 * 64 : nullptr, t4, dqkv32 ? dqkv32 + r + kcol : nullptr);
+    store_row_rot(dqkv + r + vcol, dv, 0, unscale, nullptr, nullptr, t4, dqkv32 ? dqkv32 + r + vcol : nullptr);
   }
   if (key1 < S) {
-    store_row_rot(dqkv + (size_t)(row0 + key1) * ld + kcol, dk, 2, scale, rcos ? rcos + (size_t)key1 * 64 : nullptr,
-                  rsin ? rsin + (size_t)key1 * 64 : nullptr, t4);
-    store_row_rot(dqkv + (size_t)(row0 + key1) * ld + vcol, dv, 2, 1.f, nullptr, nullptr, t4);
+    const size_t r = (size_t)(row0 + key1) * ld;
+    store_row_rot(dqkv + r + kcol, dk, 2, scale * unscale, rcos ? rcos + (size_t)key1 * 64 : nullptr,
+                  rsin ? rsin + (size_t)key1 * 64 : nullptr, t4, dqkv32 ? dqkv32 + r + kcol : nullptr);
+    store_row_rot(dqkv + r + vcol, dv, 2, unscale, nullptr, nullptr, t4, dqkv32 ? dqkv32 + r + vcol : nullptr);
   }
 }
 
@@ -382,7 +400,9 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const uint16_t* __rest
                                                            const float* __restrict__ Dd,
                                                            uint16_t* __restrict__ dqkv, float scale_log2,
                                                            float scale, const float* __restrict__ rcos,
-                                                           const float* __restrict__ rsin) {
+                                                           const float* __restrict__ rsin,
+                                                           const unsigned int* __restrict__ amax,
+                                                           float* __restrict__ dqkv32) {
   extern __shared__ __align__(16) uint16_t sm[];
   uint16_t* Qs = sm;
   uint16_t* Os = Qs + 64 * LDS;
@@ -471,12 +491,17 @@ __global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const uint16_t* __rest
     }
     __syncthreads();
   }
-  if (qr0 < S)
-    store_row_rot(dqkv + (size_t)(row0 + qr0) * ld + h * HD, dq, 0, scale, rcos ? rcos + (size_t)qr0 * 64 : nullptr,
-                  rsin ? rsin + (size_t)qr0 * 64 : nullptr, t4);
-  if (qr1 < S)
-    store_row_rot(dqkv + (size_t)(row0 + qr1) * ld + h * HD, dq, 2, scale, rcos ? rcos + (size_t)qr1 * 64 : nullptr,
-                  rsin ? rsin + (size_t)qr1 * 64 : nullptr, t4);
+  const float unscale = amax ? 1.f / grad_scale_from_amax(__uint_as_float(*amax)) : 1.f;
+  if (qr0 < S) {
+    const size_t r = (size_t)(row0 + qr0) * ld + h * HD;
+    store_row_rot(dqkv + r, dq, 0, scale * unscale, rcos ? rcos + (size_t)qr0 * 64 : nullptr,
+                  rsin ? rsin + (size_t)qr0 * 64 : nullptr, t4, dqkv32 ? dqkv32 + r : nullptr);
+  }
+  if (qr1 < S) {
+    const size_t r = (size_t)(row0 + qr1) * ld + h * HD;
+    store_row_rot(dqkv + r, dq, 2, scale * unscale, rcos ? rcos + (size_t)qr1 * 64 : nullptr,
+                  rsin ? rsin + (size_t)qr1 * 64 : nullptr, t4, dqkv32 ? dqkv32 + r : nullptr);
+  }
 }
 
 constexpr int FWD_SMEM = 5 * 64 * LDS * 2;
@@ -497,31 +522,31 @@ soup_status attn_init() {
 }  // namespace
 
 soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, uint16_t* out, float* lse,
-                          cudaStream_t st) {
+                          cudaStream_t st, uint16_t* out16, float* out32) {
   SOUP_CHECK(Hq % Hkv == 0 && S > 0 && Bsz > 0, SOUP_ERR_SHAPE, "attention: bad heads/shape");
   SOUP_CHECK(ld % 8 == 0 && soup_aligned(qkv, 16) && soup_aligned(out, 16), SOUP_ERR_ALIGN, "attention: alignment");
   SOUP_TRY(attn_init());
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   dim3 grid((S + 63) / 64, Hq, Bsz);
-  attn_fwd_kernel<<<grid, 128, FWD_SMEM, st>>>(qkv, ld, S, Hq, Hkv, out, lse, scale_log2);
+  attn_fwd_kernel<<<grid, 128, FWD_SMEM, st>>>(qkv, ld, S, Hq, Hkv, out, lse, scale_log2, out16, out32);
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
 }
 
 soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, const uint16_t* dout,
                           const float* lse, const float* D, uint16_t* dqkv, const float* rope_cos,
-                          const float* rope_sin, cudaStream_t st) {
+                          const float* rope_sin, const unsigned int* amax, cudaStream_t st, float* dqkv32) {
   SOUP_CHECK(Hq % Hkv == 0 && S > 0 && Bsz > 0, SOUP_ERR_SHAPE, "attention: bad heads/shape");
   SOUP_TRY(attn_init());
   const float scale = 1.0f / sqrtf((float)HD);
   const float scale_log2 = 1.4426950408889634f * scale;
   dim3 g1((S + 63) / 64, Hkv, Bsz);
   attn_bwd_dkdv_kernel<<<g1, 128, DKDV_SMEM, st>>>(qkv, ld, S, Hq, Hkv, dout, lse, D, dqkv, scale_log2, scale,
-                                                   rope_cos, rope_sin);
+                                                   rope_cos, rope_sin, amax, dqkv32);
   SOUP_LAUNCH_CHECK();
   dim3 g2((S + 63) / 64, Hq, Bsz);
   attn_bwd_dq_kernel<<<g2, 128, DQ_SMEM, st>>>(qkv, ld, S, Hq, Hkv, dout, lse, D, dqkv, scale_log2, scale,
-                                               rope_cos, rope_sin);
+                                               rope_cos, rope_sin, amax, dqkv32);
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
 }

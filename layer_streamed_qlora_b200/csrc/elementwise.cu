@@ -55,7 +55,7 @@ __device__ __forceinline__ void load8(const uint16_t* xb, const float* xf, size_
 // One warp per row; H % 256 == 0 so every lane owns H/256 chunks of 8.
 __global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const float* __restrict__ xf,
                                    const uint16_t* __restrict__ w, int T, int H, float eps, uint16_t* __restrict__ y,
-                                   float* __restrict__ rinv) {
+                                   float* __restrict__ rinv, float* __restrict__ y32, uint16_t* __restrict__ ylo) {
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= T) return;
@@ -79,7 +79,20 @@ __global__ void rmsnorm_fwd_kernel(const uint16_t* __restrict__ x, const float* 
     unpack8(wr[c * 32 + lane], g);
 #pragma unroll
     for (int i = 0; i < 8; ++i) f[i] = (f[i] * r) * g[i];
-    yr[c * 32 + lane] = pack8(f);
+    const uint4 hi = pack8(f);
+    yr[c * 32 + lane] = hi;
+    if (ylo) {  // rounding residual: y = hi + lo to ~16 significant bits
+      float fh[8], fl[8];
+      unpack8(hi, fh);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) fl[i] = f[i] - fh[i];
+      reinterpret_cast<uint4*>(ylo + rb)[c * 32 + lane] = pack8(fl);
+    }
+    if (y32) {
+      float4* o = reinterpret_cast<float4*>(y32 + rb + (size_t)(c * 32 + lane) * 8);
+      o[0] = make_float4(f[0], f[1], f[2], f[3]);
+      o[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
   }
 }
 
@@ -88,7 +101,8 @@ __global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ x, const float* 
                                    const uint16_t* __restrict__ w, const float* __restrict__ rinv,
                                    const uint16_t* __restrict__ dy, const float* __restrict__ dyf,
                                    const float* __restrict__ dres, int T, int H, float* __restrict__ dh,
-                                   uint16_t* __restrict__ dh_bf16) {
+                                   uint16_t* __restrict__ dh_bf16, unsigned int* __restrict__ amax,
+                                   uint16_t* __restrict__ dh_lo) {
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= T) return;
@@ -106,6 +120,7 @@ __global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ x, const float* 
     for (int i = 0; i < 8; ++i) dot += (b[i] * g[i]) * (a[i] * r);
   }
   dot = warp_sum(dot) / (float)H;
+  float mx = 0.f;
   for (int c = 0; c < nch; ++c) {
     float a[8], b[8], g[8], o[8];
     load8(x, xf, rb + (size_t)(c * 32 + lane) * 8, a);
@@ -119,7 +134,25 @@ __global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ x, const float* 
     for (int i = 0; i < 8; ++i) o[i] = dr[i] + r * (b[i] * g[i] - (a[i] * r) * dot);
     reinterpret_cast<float4*>(dh + base)[0] = make_float4(o[0], o[1], o[2], o[3]);
     reinterpret_cast<float4*>(dh + base)[1] = make_float4(o[4], o[5], o[6], o[7]);
-    if (dh_bf16) reinterpret_cast<uint4*>(dh_bf16 + base)[0] = pack8(o);
+    if (dh_bf16) {
+      const uint4 hi = pack8(o);
+      reinterpret_cast<uint4*>(dh_bf16 + base)[0] = hi;
+      if (dh_lo) {
+        float oh[8], ol[8];
+        unpack8(hi, oh);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ol[i] = o[i] - oh[i];
+        reinterpret_cast<uint4*>(dh_lo + base)[0] = pack8(ol);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(o[i]));
+  }
+  if (amax) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    // non-negative floats order like their bit patterns: an integer max is exact and order-independent
+    if (lane == 0) atomicMax(amax, __float_as_uint(mx));
   }
 }
 
@@ -144,11 +177,12 @@ __global__ void attn_rowdot_kernel(const uint16_t* __restrict__ dO, const uint16
   const size_t off = (size_t)t * Hq * 128 + h * 128 + lane * 4;
   const uint2 a = *reinterpret_cast<const uint2*>(dO + off);
   const uint2 b = *reinterpret_cast<const uint2*>(O + off);
-  // dO is fp16, O is bf16
+  // dO and O are both fp16 here (O: the attention forward's fp16 copy)
   const float2 d01 = __half22float2(*reinterpret_cast<const __half2*>(&a.x));
   const float2 d23 = __half22float2(*reinterpret_cast<const __half2*>(&a.y));
-  float s = d01.x * __uint_as_float(b.x << 16) + d01.y * __uint_as_float(b.x & 0xFFFF0000u) +
-            d23.x * __uint_as_float(b.y << 16) + d23.y * __uint_as_float(b.y & 0xFFFF0000u);
+  const float2 o01 = __half22float2(*reinterpret_cast<const __half2*>(&b.x));
+  const float2 o23 = __half22float2(*reinterpret_cast<const __half2*>(&b.y));
+  float s = d01.x * o01.x + d01.y * o01.y + d23.x * o23.x + d23.y * o23.y;
   s = warp_sum(s);
   if (lane == 0) D[(size_t)h * T + t] = s;
 }
@@ -171,6 +205,22 @@ __global__ void bf16_to_f32_kernel(const uint16_t* __restrict__ in, size_t n, fl
   }
 }
 
+// in [rows, cols] bf16 -> out [cols, rows] fp32 (exact)
+__global__ void transpose_bf16_f32_kernel(const uint16_t* __restrict__ in, int rows, int cols,
+                                          float* __restrict__ out) {
+  __shared__ float tile[32][33];
+  const int bx = blockIdx.x * 32, by = blockIdx.y * 32;
+  for (int j = threadIdx.y; j < 32; j += blockDim.y) {
+    const int r = by + j, c = bx + threadIdx.x;
+    if (r < rows && c < cols) tile[j][threadIdx.x] = b2f(in[(size_t)r * cols + c]);
+  }
+  __syncthreads();
+  for (int j = threadIdx.y; j < 32; j += blockDim.y) {
+    const int c = bx + j, r = by + threadIdx.x;
+    if (r < rows && c < cols) out[(size_t)c * rows + r] = tile[threadIdx.x][j];
+  }
+}
+
 unsigned grid_for(size_t work, int threads) {
   size_t g = (work + threads - 1) / threads;
   const size_t cap = (size_t)sm_count() * 16;
@@ -180,18 +230,19 @@ unsigned grid_for(size_t work, int threads) {
 }  // namespace
 
 soup_status rmsnorm_fwd(const uint16_t* x, const float* x_f32, const uint16_t* w, int T, int H, float eps,
-                        uint16_t* y, float* rinv, cudaStream_t st) {
+                        uint16_t* y, float* rinv, cudaStream_t st, float* y32, uint16_t* ylo) {
   SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
-  rmsnorm_fwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, T, H, eps, y, rinv);
+  rmsnorm_fwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, T, H, eps, y, rinv, y32, ylo);
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
 }
 
 soup_status rmsnorm_bwd(const uint16_t* x, const float* x_f32, const uint16_t* w, const float* rinv,
                         const uint16_t* dy, const float* dres, int T, int H, float* dh, uint16_t* dh_bf16,
-                        cudaStream_t st) {
+                        cudaStream_t st, unsigned int* amax, uint16_t* dh_lo) {
   SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
-  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, rinv, dy, nullptr, dres, T, H, dh, dh_bf16);
+  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, rinv, dy, nullptr, dres, T, H, dh, dh_bf16, amax,
+                                                  dh_lo);
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
 }
@@ -199,7 +250,15 @@ soup_status rmsnorm_bwd(const uint16_t* x, const float* x_f32, const uint16_t* w
 soup_status rmsnorm_bwd_f32dy(const uint16_t* x, const uint16_t* w, const float* rinv, const float* dy, int T, int H,
                               float* dh, cudaStream_t st) {
   SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
-  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, nullptr, w, rinv, nullptr, dy, nullptr, T, H, dh, nullptr);
+  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, nullptr, w, rinv, nullptr, dy, nullptr, T, H, dh, nullptr,
+                                                  nullptr, nullptr);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+soup_status transpose_bf16_f32(const uint16_t* in, int rows, int cols, float* out, cudaStream_t st) {
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32);
+  transpose_bf16_f32_kernel<<<grid, dim3(32, 8), 0, st>>>(in, rows, cols, out);
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
 }

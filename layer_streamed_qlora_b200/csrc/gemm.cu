@@ -29,6 +29,7 @@
 #include "gemm.h"
 #include "nf4_codebook.cuh"
 #include "ptx.cuh"
+#include "gscale.cuh"
 #include <cuda_fp16.h>
 
 namespace soup {
@@ -38,14 +39,17 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
 
-template <int BN>
+template <int BN, bool DUAL = false>
 struct Cfg {
+  // DUAL: each stage holds two A tiles (the hi and lo bf16 parts of a more
+  // precise A), multiplied against the same B tile
+  static constexpr int A_STAGE = A_STAGE_BYTES * (DUAL ? 2 : 1);
   static constexpr int B_STAGE = BN * BK * 2;
-  static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+  static constexpr int STAGES = (196608 / (A_STAGE + B_STAGE)) > 8 ? 8 : (196608 / (A_STAGE + B_STAGE));
   static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   static constexpr int BAR_BYTES = 256;
   static constexpr int LUT_BYTES = 16 * 32 * 4;
-  static constexpr int SMEM = 1024 + STAGES * (A_STAGE_BYTES + B_STAGE) + BAR_BYTES + LUT_BYTES;
+  static constexpr int SMEM = 1024 + STAGES * (A_STAGE + B_STAGE) + BAR_BYTES + LUT_BYTES;
 };
 
 struct KArgs {
@@ -57,11 +61,13 @@ struct KArgs {
   int pair_off;
   int epi, out_kind;
   void* out;
+  float* out2;
   long long ldo;
   const uint16_t* resid;
   const float* resid_f32;
   long long ldr;
   float alpha;
+  const unsigned int* scale_amax;
   uint16_t* aux16;
   long long ld_aux;
   int swiglu_I;
@@ -173,22 +179,33 @@ __device__ __forceinline__ void load_codes(const uint8_t* src, uint32_t (&w)[NWO
   }
 }
 
-template <int BN, int AMJ, int BMD>
+template <int BN, int AMJ, int BMD, bool TF, bool DUAL>
 __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmTA,
-                const __grid_constant__ CUtensorMap tmTB, const KArgs args) {
-  using C = Cfg<BN>;
+                const __grid_constant__ CUtensorMap tmTB, const __grid_constant__ CUtensorMap tmA2,
+                const KArgs args) {
+  using C = Cfg<BN, DUAL>;
+  static_assert(!DUAL || (AMJ == A_K && !TF), "dual-A: K-major bf16 A only");
   constexpr bool NF4 = BMD >= B_NF4_K;
   constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
   constexpr int STAGES = C::STAGES;
   constexpr int NEPI = NF4 ? 8 : 4;
+  // Element geometry: every stage row is one 128-byte swizzle row.  bf16:
+  // 64 K-elements per stage, K = 16 per MMA, 64-wide MN-major chunks; tf32
+  // (fp32 operands): 32 K-elements per stage, K = 8 per MMA, 32-wide chunks.
+  constexpr int BKE = TF ? 32 : 64;          // K elements per stage
+  constexpr int KI = TF ? 8 : 16;            // K per MMA instruction
+  constexpr int CW = TF ? 32 : 64;           // MN-major chunk width (elements)
+  constexpr int CHUNK_BYTES = BKE * 128;     // one MN-major chunk of a stage
+  constexpr int KSTEP_MN = KI * 128;         // MN-major descriptor advance per MMA
+  static_assert(!TF || (BMD == B_TMA_K), "tf32 mode: TMA-fed K-major B only");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint8_t* sB = smem + STAGES * C::A_STAGE;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_STAGE);
   uint64_t* empty = full + STAGES;
   uint64_t* accf = empty + STAGES;
@@ -215,6 +232,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmA);
+    if (DUAL) ptx::prefetch_tmap(&tmA2);
     if (!NF4) ptx::prefetch_tmap(&tmB);
     if (args.tail_ksteps > 0) {
       ptx::prefetch_tmap(&tmTA);
@@ -252,18 +270,19 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
           *abort_flag = 1;
           break;
         }
-        uint8_t* a = sA + s * A_STAGE_BYTES;
+        uint8_t* a = sA + s * C::A_STAGE;
         uint8_t* b = sB + s * C::B_STAGE;
         const bool tail = it >= num_kb;
-        const uint32_t bytes = A_STAGE_BYTES + ((!NF4 || tail) ? C::B_STAGE : 0);
+        const uint32_t bytes = ((DUAL && !tail) ? C::A_STAGE : A_STAGE_BYTES) + ((!NF4 || tail) ? C::B_STAGE : 0);
         ptx::mbar_arrive_expect_tx(&full[s], bytes);
         if (!tail) {
-          const int k0 = it * BK;
+          const int k0 = it * BKE;
           if (AMJ == A_K) {
             ptx::tma_load_2d(a, &tmA, &full[s], k0, m0);
+            if (DUAL) ptx::tma_load_2d(a + A_STAGE_BYTES, &tmA2, &full[s], k0, m0);
           } else {
-            ptx::tma_load_2d(a, &tmA, &full[s], m0, k0);
-            ptx::tma_load_2d(a + 8192, &tmA, &full[s], m0 + 64, k0);
+#pragma unroll
+            for (int c = 0; c < BM / CW; ++c) ptx::tma_load_2d(a + c * CHUNK_BYTES, &tmA, &full[s], m0 + c * CW, k0);
           }
           if (!NF4) {
             if (!B_MN) {
@@ -299,7 +318,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_main = ptx::idesc_bf16(BM, BN, AMJ, B_MN ? 1 : 0);
+      constexpr uint32_t idesc_main = ptx::idesc_fmt(BM, BN, AMJ, B_MN ? 1 : 0, TF ? 2u : 1u);
       constexpr uint32_t idesc_tail = ptx::idesc_bf16(BM, BN, 1, B_MN ? 1 : 0);
       constexpr uint32_t idesc_half = ptx::idesc_bf16(BM, BN >= 32 ? BN / 2 : BN, 1, B_MN ? 1 : 0);
       bool ok = true;
@@ -313,7 +332,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t a_base = ptx::smem_u32(sA + s * A_STAGE_BYTES);
+        const uint32_t a_base = ptx::smem_u32(sA + s * C::A_STAGE);
         const uint32_t b_base = ptx::smem_u32(sB + s * C::B_STAGE);
         const bool tail = it >= num_kb;
         if (tail && paired) {
@@ -326,14 +345,28 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
             ptx::mma_bf16(tmem + hf * (BN / 2), ad, bd, idesc_half, 1u);
           }
         } else {
-          const int nk = tail ? args.tail_ksteps : BK / 16;
+          const int nk = tail ? args.tail_ksteps : BKE / KI;
           const bool a_mn = tail || AMJ == A_MN;
           for (int k = 0; k < nk; ++k) {
-            const uint64_t ad = a_mn ? ptx::smem_desc_sw128(a_base + k * 2048, 8192, 1024)
-                                     : ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k * 2048, 8192, 1024)
+            uint64_t ad;
+            if constexpr (TF)  // MN-major tf32: 32-byte-atom swizzle, 4-row period (SBO 512 B)
+              ad = a_mn ? ptx::smem_desc_sw128_32b(a_base + k * KSTEP_MN, CHUNK_BYTES, 512)
+                        : ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
+            else
+              ad = a_mn ? ptx::smem_desc_sw128(a_base + k * KSTEP_MN, CHUNK_BYTES, 1024)
+                        : ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k * KSTEP_MN, CHUNK_BYTES, 1024)
                                      : ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
-            ptx::mma_bf16(tmem, ad, bd, tail ? idesc_tail : idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+            if constexpr (TF)
+              ptx::mma_tf32(tmem, ad, bd, idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+            else
+              ptx::mma_bf16(tmem, ad, bd, tail ? idesc_tail : idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+            if constexpr (DUAL) {
+              if (!tail) {  // lo part of A against the same B tile
+                const uint64_t ad2 = ptx::smem_desc_sw128(a_base + A_STAGE_BYTES + k * 32, 16, 1024);
+                ptx::mma_bf16(tmem, ad2, bd, idesc_main, 1u);
+              }
+            }
           }
         }
         ptx::mma_commit(&empty[s]);
@@ -452,6 +485,8 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
       const int row = m0 + q * 32 + lane;
       const bool row_ok = row < args.M;
       constexpr int NCH = BN / 16;
+      const float alpha =
+          args.scale_amax ? args.alpha * grad_scale_from_amax(__uint_as_float(*args.scale_amax)) : args.alpha;
       const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
       const int ch0 = NEPI == 8 ? ew / 4 : 0, chs = NEPI == 8 ? 2 : 1;
       const bool vec = args.vec_ok != 0;
@@ -469,8 +504,8 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
           float a[16], gg[16], uu[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            gg[i] = __uint_as_float(vg[i]) * args.alpha;
-            uu[i] = __uint_as_float(vu[i]) * args.alpha;
+            gg[i] = __uint_as_float(vg[i]) * alpha;
+            uu[i] = __uint_as_float(vu[i]) * alpha;
             a[i] = gg[i] * sigmoid_f(gg[i]) * uu[i];
           }
           store_row16(args.out, OUT_BF16, args.ldo, row, n, I, a, vec);
@@ -497,7 +532,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
           float a[16], b[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float x0 = __uint_as_float(v0[i]) * args.alpha, x1 = __uint_as_float(v1[i]) * args.alpha;
+            const float x0 = __uint_as_float(v0[i]) * alpha, x1 = __uint_as_float(v1[i]) * alpha;
             const float c = __ldg(cs + i), sv = __ldg(sn + i);
             a[i] = x0 * c - x1 * sv;
             b[i] = x1 * c + x0 * sv;
@@ -514,7 +549,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
           if (!row_ok || n >= args.N) continue;
           float f[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * args.alpha;
+          for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * alpha;
           const bool full16 = vec && (n + 16 <= args.N);
           if (args.epi == EPI_SWIGLU_BWD) {
             // f = dL/d(act); g, u from the forward (fp16); out = [dL/dg | dL/du] bf16
@@ -550,6 +585,11 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
               for (int i = 0; i < 16; ++i)
                 if (n + i < args.N)
                   o[(size_t)(n + i) * args.ldo + row] = static_cast<uint16_t>(pack_bf16x2(f[i], 0.f) & 0xFFFF);
+              if (args.out2) {  // the same values unrounded, fp32, same layout
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  if (n + i < args.N) args.out2[(size_t)(n + i) * args.ldo + row] = f[i];
+              }
             } else {
               float* o = static_cast<float*>(args.out);
 #pragma unroll
@@ -611,44 +651,52 @@ constexpr int CU_DT_BF16 = 9;       // CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
 constexpr int CU_SWIZZLE_128B = 3;  // CU_TENSOR_MAP_SWIZZLE_128B
 constexpr int CU_L2_256B = 3;       // CU_TENSOR_MAP_L2_PROMOTION_L2_256B
 
-soup_status make_map(CUtensorMap* m, const Mat& mat, uint32_t box0, uint32_t box1, const char* what) {
+constexpr int CU_DT_F32 = 7;        // CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+constexpr int CU_SWIZZLE_128B_ATOM_32B = 4;  // 32-byte chunks within a 128-byte span
+
+soup_status make_map(CUtensorMap* m, const Mat& mat, uint32_t box0, uint32_t box1, const char* what,
+                     bool f32 = false, int swizzle = CU_SWIZZLE_128B) {
+  const int es = f32 ? 4 : 2;
   SOUP_CHECK(mat.ptr && mat.rows > 0 && mat.cols > 0, SOUP_ERR_INVALID_ARG, "gemm: %s is empty", what);
   SOUP_CHECK(soup_aligned(mat.ptr, 16), SOUP_ERR_ALIGN, "gemm: %s base not 16-byte aligned", what);
-  SOUP_CHECK((mat.ld * 2) % 16 == 0 && mat.ld >= mat.cols, SOUP_ERR_ALIGN,
-             "gemm: %s row stride %lld elements is not a multiple of 8 (or < cols)", what,
+  SOUP_CHECK((mat.ld * es) % 16 == 0 && mat.ld >= mat.cols, SOUP_ERR_ALIGN,
+             "gemm: %s row stride %lld elements is not a multiple of 16 bytes (or < cols)", what,
              (long long)mat.ld);
   EncodeTiledFn enc = encode_tiled();
   SOUP_CHECK(enc != nullptr, SOUP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const uint64_t gdim[2] = {(uint64_t)mat.cols, (uint64_t)mat.rows};
-  const uint64_t gstride[1] = {(uint64_t)mat.ld * 2};
+  const uint64_t gstride[1] = {(uint64_t)mat.ld * es};
   const uint32_t box[2] = {box0, box1};
   const uint32_t estr[2] = {1, 1};
-  int r = enc(m, CU_DT_BF16, 2, const_cast<void*>(mat.ptr), gdim, gstride, box, estr, 0,
-              CU_SWIZZLE_128B, CU_L2_256B, 0);
+  int r = enc(m, f32 ? CU_DT_F32 : CU_DT_BF16, 2, const_cast<void*>(mat.ptr), gdim, gstride, box, estr, 0,
+              swizzle, CU_L2_256B, 0);
   SOUP_CHECK(r == 0, SOUP_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, r);
   return SOUP_OK;
 }
 
-template <int BN, int AMJ, int BMD>
+template <int BN, int AMJ, int BMD, bool TF = false, bool DUAL = false>
 soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
-  using C = Cfg<BN>;
-  CUtensorMap mA, mB, mTA, mTB;
+  using C = Cfg<BN, DUAL>;
+  CUtensorMap mA, mB, mTA, mTB, mA2;
+  memset(&mA2, 0, sizeof(mA2));
+  if (DUAL) SOUP_TRY(make_map(&mA2, d.A_lo, 64, 128, "A (lo part)"));
   memset(&mA, 0, sizeof(mA));
   memset(&mB, 0, sizeof(mB));
   memset(&mTA, 0, sizeof(mTA));
   memset(&mTB, 0, sizeof(mTB));
   const bool paired = d.pair_off > 0;
-  if (AMJ == A_K) SOUP_TRY(make_map(&mA, d.A, 64, 128, "A"));
-  else SOUP_TRY(make_map(&mA, d.A, 64, 64, "A (MN-major)"));
+  constexpr uint32_t EW = TF ? 32 : 64;  // elements per 128-byte row
+  if (AMJ == A_K) SOUP_TRY(make_map(&mA, d.A, EW, 128, "A", TF));
+  else SOUP_TRY(make_map(&mA, d.A, EW, EW, "A (MN-major)", TF, TF ? CU_SWIZZLE_128B_ATOM_32B : CU_SWIZZLE_128B));
   constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
-  if (BMD == B_TMA_K) SOUP_TRY(make_map(&mB, d.B, 64, paired ? BN / 2 : BN, "B"));
+  if (BMD == B_TMA_K) SOUP_TRY(make_map(&mB, d.B, EW, paired ? BN / 2 : BN, "B", TF));
   if (BMD == B_TMA_MN) SOUP_TRY(make_map(&mB, d.B, 64, 64, "B (MN-major)"));
   if (d.tail_ksteps > 0) {
     SOUP_TRY(make_map(&mTA, d.tailA, 64, 64, "tail A"));
     if (!B_MN) SOUP_TRY(make_map(&mTB, d.tailB, 64, paired ? BN / 2 : BN, "tail B"));
     else SOUP_TRY(make_map(&mTB, d.tailB, 64, 64, "tail B (MN-major)"));
   }
-  auto kern = gemm_kernel<BN, AMJ, BMD>;
+  auto kern = gemm_kernel<BN, AMJ, BMD, TF, DUAL>;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     SOUP_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
@@ -662,13 +710,13 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
     // operands read once and the output written once
     const int cls = BMD == B_NF4_K ? GC_NF4_FWD : (BMD == B_NF4_MN ? GC_NF4_BWD : (d.N <= 64 ? GC_SKINNY : GC_BF16));
     const double tail_k = d.tail_ksteps > 0 ? (double)d.tailA.rows : 0.0;
-    const double flops = 2.0 * d.M * d.N * ((double)d.K + (paired ? 16.0 : tail_k));
+    const double flops = 2.0 * d.M * d.N * ((double)d.K * (DUAL ? 2 : 1) + (paired ? 16.0 : tail_k));
     const double wbytes = (BMD >= B_NF4_K) ? (double)d.N * d.K * (0.5 + 4.0 / 64) : (double)d.N * d.K * 2;
     const int oes = (d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T) ? 4 : 2;
     const double bytes = (double)d.M * d.K * 2 + wbytes + (double)d.M * d.N * oes;
     profile_begin(st, cls, flops, bytes);
   }
-  kern<<<grid, NT, C::SMEM, st>>>(mA, mB, mTA, mTB, ka);
+  kern<<<grid, NT, C::SMEM, st>>>(mA, mB, mTA, mTB, mA2, ka);
   SOUP_LAUNCH_CHECK();
   profile_end(st);
   return SOUP_OK;
@@ -726,14 +774,15 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
   KArgs ka;
   memset(&ka, 0, sizeof(ka));
   ka.M = d.M; ka.N = d.N; ka.K = d.K;
-  ka.num_kb = (d.K + BK - 1) / BK;
+  ka.num_kb = d.tf32 ? (d.K + 31) / 32 : (d.K + BK - 1) / BK;
   ka.codes = d.codes; ka.absmax = d.absmax;
   ka.tail_ksteps = d.tail_ksteps; ka.nseg = d.nseg;
   for (int i = 0; i < 4; ++i) { ka.seg_end[i] = d.seg_end[i]; ka.seg_row[i] = d.seg_row[i]; }
   ka.pair_off = d.pair_off;
   ka.epi = d.epi;
-  ka.out_kind = d.out_kind; ka.out = d.out; ka.ldo = d.ldo;
+  ka.out_kind = d.out_kind; ka.out = d.out; ka.ldo = d.ldo; ka.out2 = d.out2;
   ka.resid = d.resid; ka.resid_f32 = d.resid_f32; ka.ldr = d.ldr; ka.alpha = d.alpha;
+  ka.scale_amax = d.scale_amax;
   ka.aux16 = d.aux16; ka.ld_aux = d.ld_aux; ka.swiglu_I = d.swiglu_I;
   const int esz = (d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T) ? 4 : 2;
   ka.vec_ok = soup_aligned(d.out, 16) && ((d.ldo * esz) % 16 == 0) &&
@@ -750,6 +799,28 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
   ka.err = device_error_word();
   SOUP_CHECK(ka.err != nullptr, SOUP_ERR_CUDA, "device error word unavailable");
 
+  if (d.tf32) {
+    SOUP_CHECK(d.b_mode == B_TMA_K && d.tail_ksteps == 0 && d.pair_off == 0 && d.epi == EPI_STORE && bn <= 64,
+               SOUP_ERR_SHAPE, "gemm: tf32 mode supports skinny (N <= 64) K-major-B GEMMs without tail");
+#define SOUP_GEMM_TF(BN_, AM_) \
+  if (bn == BN_ && d.a_major == AM_) return launch<BN_, AM_, B_TMA_K, true>(d, ka, st);
+    SOUP_GEMM_TF(64, A_K) SOUP_GEMM_TF(48, A_K) SOUP_GEMM_TF(32, A_K) SOUP_GEMM_TF(16, A_K)
+    SOUP_GEMM_TF(64, A_MN) SOUP_GEMM_TF(48, A_MN) SOUP_GEMM_TF(32, A_MN) SOUP_GEMM_TF(16, A_MN)
+#undef SOUP_GEMM_TF
+    return fail(SOUP_ERR_SHAPE, "gemm: no tf32 kernel for BN=%d", bn);
+  }
+  if (d.A_lo.ptr) {
+    SOUP_CHECK(d.a_major == A_K && !d.tf32 && (bn == 256 || bn == 128) && d.A_lo.rows == d.A.rows &&
+                   d.A_lo.cols == d.A.cols,
+               SOUP_ERR_SHAPE, "gemm: dual-A needs a K-major bf16 A, N tile 128/256 and matching hi/lo shapes");
+#define SOUP_GEMM_DUAL(BN_, BMD_) \
+  if (bn == BN_ && d.b_mode == BMD_) return launch<BN_, A_K, BMD_, false, true>(d, ka, st);
+    SOUP_GEMM_DUAL(256, B_NF4_K) SOUP_GEMM_DUAL(128, B_NF4_K) SOUP_GEMM_DUAL(256, B_NF4_MN)
+    SOUP_GEMM_DUAL(128, B_NF4_MN) SOUP_GEMM_DUAL(256, B_TMA_K) SOUP_GEMM_DUAL(128, B_TMA_K)
+    SOUP_GEMM_DUAL(256, B_TMA_MN) SOUP_GEMM_DUAL(128, B_TMA_MN)
+#undef SOUP_GEMM_DUAL
+    return fail(SOUP_ERR_SHAPE, "gemm: no dual-A kernel for BN=%d b_mode=%d", bn, d.b_mode);
+  }
 #define SOUP_GEMM_CASE(BN_, AM_, BMD_) \
   if (bn == BN_ && d.a_major == AM_ && d.b_mode == BMD_) return launch<BN_, AM_, BMD_>(d, ka, st);
   SOUP_GEMM_CASE(256, A_K, B_NF4_K)

@@ -35,8 +35,16 @@ enum Epi : int {
 
 struct GemmDesc {
   int M = 0, N = 0, K = 0;
+  // tf32 mode: every TMA operand is fp32 (Mat sizes in fp32 elements) and the
+  // MMA is kind::tf32 (skinny K-major-B GEMMs only, no tail).
+  bool tf32 = false;
   int a_major = A_K;
   Mat A;                    // [M, K] (A_K) or [K, M] (A_MN)
+  // Dual-A (when A_lo.ptr is set): A is the sum of two bf16 tensors, the
+  // rounded value (A) and its rounding residual (A_lo); each k-step issues
+  // both MMAs against the same B tile, so an fp32-accurate A costs no extra
+  // B traffic or NF4 decoding.
+  Mat A_lo;
   int b_mode = B_TMA_K;
   Mat B;                    // bf16 B for TMA modes
   const uint8_t* codes = nullptr;
@@ -60,11 +68,15 @@ struct GemmDesc {
   int epi = EPI_STORE;
   int out_kind = OUT_BF16;
   void* out = nullptr;
+  float* out2 = nullptr;            // OUT_BF16_T only: also the unrounded fp32 values, same layout
   int64_t ldo = 0;
   const uint16_t* resid = nullptr;  // bf16 [M, N] row stride ldr (row-major outputs)
   const float* resid_f32 = nullptr; // fp32 [M, N] row stride ldr (row-major outputs)
   int64_t ldr = 0;
   float alpha = 1.f;
+  // Optional power-of-two gradient scale (gscale.cuh) multiplied into alpha,
+  // derived on the device from the bit pattern of an amax value.
+  const unsigned int* scale_amax = nullptr;
   uint16_t* aux16 = nullptr;        // fp16 [M, 2*I] g | u (SwiGLU modes), row stride ld_aux
   int64_t ld_aux = 0;
   int swiglu_I = 0;                 // I: offset of u within aux16 / of dL/du within out

@@ -34,7 +34,10 @@ struct Dims {
 // Workspace layout (byte offsets, each 256-aligned).
 struct WS {
   size_t x1, rinv1, qkv, attn, lse, h2, x2, rinv2, gu16, act, u_qkv, u_o, u_gu, u_d, cosb, sinb;
-  size_t dh_b, g_d, g_gu, g_o, g_qkv, Bt, d_gu, dx2, dh2, dh2_b, d_attn, D, d_qkv, dx1;
+  size_t dh_b, g_d, g_gu, g_o, g_qkv, Bt, d_gu, dx2, dh2, dh2_b, d_attn, D, d_qkv, dx1, attn16, gamax;
+  size_t x1_32, dqkv32, u32, g32, A32, Bt32;  // fp32 operands of the q/k/v LoRA-gradient GEMMs (tf32)
+  size_t x1_lo, dh2_lo;                       // bf16 rounding residuals (dual-A GEMM inputs)
+  size_t attn32, uo32, go32, Ao32;            // fp32 operands of the o LoRA-gradient GEMMs (tf32)
   size_t total;
 };
 
@@ -78,6 +81,20 @@ WS layout(const Dims& m) {
   w.D = take((size_t)m.Hq * T * 4);
   w.d_qkv = take(T * m.qkv_w * 2);
   w.dx1 = take(T * H * 2);
+  w.attn16 = take(T * m.o_in * 2);  // fp16 copy of the attention output (for D = rowsum(dO * O))
+  w.gamax = take(4);                // max |dh2| bit pattern (gradient scale of dO)
+  w.x1_32 = take(T * H * 4);
+  w.dqkv32 = take(T * m.qkv_w * 4);
+  w.u32 = take(3 * r * ldT * 4);
+  w.g32 = take(3 * r * ldT * 4);
+  w.A32 = take(3 * r * H * 4);
+  w.Bt32 = take(max_out * r * 4);
+  w.x1_lo = take(T * H * 2);
+  w.dh2_lo = take(T * H * 2);
+  w.attn32 = take(T * m.o_in * 4);
+  w.uo32 = take(r * ldT * 4);
+  w.go32 = take(r * ldT * 4);
+  w.Ao32 = take(r * (size_t)m.o_in * 4);
   w.total = o;
   return w;
 }
@@ -129,6 +146,7 @@ struct ProjOpts {
   const float* rope_sin = nullptr;
   int swiglu_I = 0;          // > 0: paired gate|up tiles with the SwiGLU epilogue
   uint16_t* aux16 = nullptr; // SwiGLU: fp16 g | u output (may be null)
+  const uint16_t* x_lo = nullptr;  // dual-A: bf16 rounding residual of x
 };
 
 soup_status proj_fwd(const soup_weight* W, const uint16_t* x, int T, const uint16_t* u, int64_t ldT, int u_rows,
@@ -137,6 +155,7 @@ soup_status proj_fwd(const soup_weight* W, const uint16_t* x, int T, const uint1
   GemmDesc g;
   g.M = T; g.N = (int)W->out_features; g.K = (int)W->in_features;
   g.A = Mat{x, T, W->in_features, W->in_features};
+  if (o.x_lo) g.A_lo = Mat{o.x_lo, T, W->in_features, W->in_features};
   set_weight_fwd(g, W);
   if (on) {
     g.tail_ksteps = r / 16;
@@ -212,12 +231,69 @@ soup_status lora_dA(const uint16_t* x, int T, int K, const uint16_t* gt, int row
   return gemm(g, st);
 }
 
+// tf32 variants of the LoRA GEMMs of the q/k/v group, on fp32 operands:
+// u = s x A^T (bf16 copy u' for the tail, fp32 copy for dB), g = s dy B
+// (bf16 copy g' for the tail, fp32 copy for dA), dA = g^T x, dB = dy^T u.
+soup_status lora_down_tf32(const float* x, int T, int K, const float* A32, int rows, float s, uint16_t* u,
+                           float* u32, int64_t ldT, cudaStream_t st) {
+  GemmDesc g;
+  g.tf32 = true;
+  g.M = T; g.N = rows; g.K = K;
+  g.A = Mat{x, T, K, K};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{A32, rows, K, K};
+  g.out_kind = OUT_BF16_T; g.out = u; g.out2 = u32; g.ldo = ldT; g.alpha = s;
+  return gemm(g, st);
+}
+
+soup_status lora_g_tf32(const float* dy, int64_t ld, int T, int n, const uint16_t* Bl, int r, float s, float* Bt32,
+                        uint16_t* gout, float* g32, int64_t ldT, cudaStream_t st) {
+  SOUP_TRY(transpose_bf16_f32(Bl, n, r, Bt32, st));
+  GemmDesc g;
+  g.tf32 = true;
+  g.M = T; g.N = r; g.K = n;
+  g.A = Mat{dy, T, n, ld};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{Bt32, r, n, n};
+  g.out_kind = OUT_BF16_T; g.out = gout; g.out2 = g32; g.ldo = ldT; g.alpha = s;
+  return gemm(g, st);
+}
+
+soup_status lora_dB_tf32(const float* dy, int64_t ld, int T, int n, const float* u32, int r, int64_t ldT, float* dB,
+                         cudaStream_t st) {
+  GemmDesc g;
+  g.tf32 = true;
+  g.M = n; g.N = r; g.K = T;
+  g.a_major = A_MN;
+  g.A = Mat{dy, T, n, ld};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{u32, r, T, ldT};
+  g.out_kind = OUT_F32; g.out = dB; g.ldo = r;
+  return gemm(g, st);
+}
+
+soup_status lora_dA_tf32(const float* x, int T, int K, const float* g32, int rows, int64_t ldT, float* dA,
+                         cudaStream_t st) {
+  GemmDesc g;
+  g.tf32 = true;
+  g.M = K; g.N = rows; g.K = T;
+  g.a_major = A_MN;
+  g.A = Mat{x, T, K, K};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{g32, rows, T, ldT};
+  g.out_kind = OUT_F32_T; g.out = dA; g.ldo = K;
+  return gemm(g, st);
+}
+
 // dx = dy W (+ g' A); with swiglu_I > 0 the epilogue turns dL/d(act) into
 // [dL/dg | dL/du] (bf16, [T, 2I]) using the fp16 g | u saved by the forward.
 soup_status proj_bwd(const soup_weight* W, const uint16_t* dy, int T, const uint16_t* gt, int64_t ldT, int g_rows,
                      const uint16_t* Al, bool on, uint16_t* dx, cudaStream_t st, int out_kind = OUT_BF16,
-                     int swiglu_I = 0, uint16_t* aux16 = nullptr) {
+                     int swiglu_I = 0, uint16_t* aux16 = nullptr, const unsigned int* scale_amax = nullptr,
+                     const uint16_t* dy_lo = nullptr) {
   GemmDesc g;
+  g.scale_amax = scale_amax;
+  if (dy_lo) g.A_lo = Mat{dy_lo, T, W->out_features, W->out_features};
   g.M = T; g.N = (int)W->in_features; g.K = (int)W->out_features;
   g.A = Mat{dy, T, W->out_features, W->out_features};
   set_weight_bwd(g, W);
@@ -244,8 +320,14 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
                     cudaStream_t st) {
   const int T = m.T, r = m.r;
   SOUP_TRY(rope_table(m.S, m.d, (double)c->theta, PF(cosb), PF(sinb), st));
-  SOUP_TRY(rmsnorm_fwd(h_in, nullptr, W->norm1, T, m.H, c->eps, P(x1), PF(rinv1), st));
-  if (on) SOUP_TRY(lora_down(P(x1), T, m.H, L->A_qkv, 3 * r, m.s, P(u_qkv), m.ldT, st));
+  SOUP_TRY(rmsnorm_fwd(h_in, nullptr, W->norm1, T, m.H, c->eps, P(x1), PF(rinv1), st, on ? PF(x1_32) : nullptr,
+                       recompute ? P(x1_lo) : nullptr));
+  if (on) {
+    // q/k/v adapters: u from the fp32 normalised input (tf32 tensor cores); the
+    // tail consumes its bf16 copy, the dB GEMM its fp32 copy
+    SOUP_TRY(bf16_to_f32(L->A_qkv, (size_t)3 * r * m.H, PF(A32), st));
+    SOUP_TRY(lora_down_tf32(PF(x1_32), T, m.H, PF(A32), 3 * r, m.s, P(u_qkv), PF(u32), m.ldT, st));
+  }
   {
     const int se[3] = {m.Hq * m.d, (m.Hq + m.Hkv) * m.d, m.qkv_w};
     const int sr[3] = {0, r, 2 * r};
@@ -253,11 +335,19 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     o.out_kind = OUT_F16;  // q, k, v feed only the attention kernels
     o.rope_cols = (m.Hq + m.Hkv) * m.d;
     o.rope_S = m.S; o.rope_cos = PF(cosb); o.rope_sin = PF(sinb);
+    // for the backward, q/k/v from an fp32-accurate x1 (hi + lo parts): the
+    // attention backward amplifies the bf16 rounding of x1 into the q/k/v
+    // adapter gradients
+    if (recompute) o.x_lo = P(x1_lo);
     SOUP_TRY(proj_fwd(&W->qkv, P(x1), T, P(u_qkv), m.ldT, 3 * r, L ? L->B_qkv : nullptr, r, 3, se, sr, on, P(qkv),
                       st, o));
   }
-  SOUP_TRY(attention_fwd(P(qkv), m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(attn), PF(lse), st));
-  if (on) SOUP_TRY(lora_down(P(attn), T, m.o_in, L->A_o, r, m.s, P(u_o), m.ldT, st));
+  SOUP_TRY(attention_fwd(P(qkv), m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(attn), PF(lse), st,
+                         recompute ? P(attn16) : nullptr, on ? PF(attn32) : nullptr));
+  if (on) {
+    SOUP_TRY(bf16_to_f32(L->A_o, (size_t)r * m.o_in, PF(Ao32), st));
+    SOUP_TRY(lora_down_tf32(PF(attn32), T, m.o_in, PF(Ao32), r, m.s, P(u_o), PF(uo32), m.ldT, st));
+  }
   {
     const int se[1] = {m.H};
     const int sr[1] = {0};
@@ -365,32 +455,38 @@ extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const
                        G->dB_gu + (size_t)sg * I * r, st));
     SOUP_TRY(lora_dA(P(x2), T, H, P(g_gu), 2 * r, ldT, G->dA_gu, st));
   }
-  SOUP_TRY(rmsnorm_bwd(nullptr, PF(h2), W->norm2, PF(rinv2), P(dx2), dh_out, T, H, PF(dh2), P(dh2_b), st));
+  unsigned int* gamax = reinterpret_cast<unsigned int*>(base + ws.gamax);
+  SOUP_CUDA_TRY(cudaMemsetAsync(gamax, 0, sizeof(unsigned int), st));
+  SOUP_TRY(rmsnorm_bwd(nullptr, PF(h2), W->norm2, PF(rinv2), P(dx2), dh_out, T, H, PF(dh2), P(dh2_b), st, gamax,
+                       P(dh2_lo)));
 
   // ---- attention block
-  if (on) SOUP_TRY(lora_g(P(dh2_b), H, T, H, L->B_o, r, m.s, P(Bt), P(g_o), ldT, st));
-  SOUP_TRY(proj_bwd(&W->o, P(dh2_b), T, P(g_o), ldT, r, on ? L->A_o : nullptr, on, P(d_attn), st, OUT_F16));
+  if (on) SOUP_TRY(lora_g_tf32(PF(dh2), H, T, H, L->B_o, r, m.s, PF(Bt32), P(g_o), PF(go32), ldT, st));
+  // dO for the attention backward: from the fp32-accurate dh2 (hi + lo parts),
+  // stored fp16 scaled by a power of two derived from max |dh2|
+  SOUP_TRY(proj_bwd(&W->o, P(dh2_b), T, P(g_o), ldT, r, on ? L->A_o : nullptr, on, P(d_attn), st, OUT_F16, 0,
+                    nullptr, gamax, P(dh2_lo)));
   if (on) {
-    SOUP_TRY(lora_dB(P(dh2_b), H, T, H, P(u_o), r, ldT, G->dB_o, st));
-    SOUP_TRY(lora_dA(P(attn), T, m.o_in, P(g_o), r, ldT, G->dA_o, st));
+    SOUP_TRY(lora_dB_tf32(PF(dh2), H, T, H, PF(uo32), r, ldT, G->dB_o, st));
+    SOUP_TRY(lora_dA_tf32(PF(attn32), T, m.o_in, PF(go32), r, ldT, G->dA_o, st));
   }
-  SOUP_TRY(attn_rowdot(P(d_attn), P(attn), T, m.Hq, PF(D), st));
+  SOUP_TRY(attn_rowdot(P(d_attn), P(attn16), T, m.Hq, PF(D), st));
   // dq and dk leave the attention backward already rotated back (inverse RoPE in its epilogues)
   SOUP_TRY(attention_bwd(P(qkv), m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(d_attn), PF(lse), PF(D), P(d_qkv), PF(cosb),
-                         PF(sinb), st));
+                         PF(sinb), gamax, st, on ? PF(dqkv32) : nullptr));
   const int seg_n[3] = {m.Hq * m.d, m.Hkv * m.d, m.Hkv * m.d};
   const int seg_c[3] = {0, m.Hq * m.d, (m.Hq + m.Hkv) * m.d};
   if (on) {
     for (int sg = 0; sg < 3; ++sg)
-      SOUP_TRY(lora_g(P(d_qkv) + seg_c[sg], m.qkv_w, T, seg_n[sg], L->B_qkv + (size_t)seg_c[sg] * r, r, m.s, P(Bt),
-                      P(g_qkv) + (size_t)sg * r * ldT, ldT, st));
+      SOUP_TRY(lora_g_tf32(PF(dqkv32) + seg_c[sg], m.qkv_w, T, seg_n[sg], L->B_qkv + (size_t)seg_c[sg] * r, r, m.s,
+                           PF(Bt32), P(g_qkv) + (size_t)sg * r * ldT, PF(g32) + (size_t)sg * r * ldT, ldT, st));
   }
   SOUP_TRY(proj_bwd(&W->qkv, P(d_qkv), T, P(g_qkv), ldT, 3 * r, on ? L->A_qkv : nullptr, on, P(dx1), st));
   if (on) {
     for (int sg = 0; sg < 3; ++sg)
-      SOUP_TRY(lora_dB(P(d_qkv) + seg_c[sg], m.qkv_w, T, seg_n[sg], P(u_qkv) + (size_t)sg * r * ldT, r, ldT,
-                       G->dB_qkv + (size_t)seg_c[sg] * r, st));
-    SOUP_TRY(lora_dA(P(x1), T, H, P(g_qkv), 3 * r, ldT, G->dA_qkv, st));
+      SOUP_TRY(lora_dB_tf32(PF(dqkv32) + seg_c[sg], m.qkv_w, T, seg_n[sg], PF(u32) + (size_t)sg * r * ldT, r, ldT,
+                            G->dB_qkv + (size_t)seg_c[sg] * r, st));
+    SOUP_TRY(lora_dA_tf32(PF(x1_32), T, H, PF(g32), 3 * r, ldT, G->dA_qkv, st));
   }
   SOUP_TRY(rmsnorm_bwd(h_in, nullptr, W->norm1, PF(rinv1), P(dx1), PF(dh2), T, H, dh_in, nullptr, st));
   return SOUP_OK;

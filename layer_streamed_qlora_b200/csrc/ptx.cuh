@@ -109,6 +109,16 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D(tmem) (+)= A * B^T, kind::tf32 (fp32 operands read as tf32, fp32 accumulate)
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive on an mbarrier once all previously issued tcgen05 ops of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
@@ -142,6 +152,32 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// Same with layout type 1 (128-byte swizzle with 32-byte atoms): the only
+// shared-memory layout tcgen05 accepts for MN-major 32-bit (tf32) operands;
+// 32-byte chunks of each 128-byte row are XOR-ed with (row % 4).
+__device__ __forceinline__ uint64_t smem_desc_sw128_32b(uint32_t saddr, uint32_t lbo_bytes,
+                                                        uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)1 << 61;
+  return d;
+}
+
+// Instruction descriptor for kind::f16 (bf16 A/B) or kind::tf32 (tf32 A/B),
+// fp32 D.  Operand format field: 1 = bf16, 2 = tf32.
+__host__ __device__ constexpr uint32_t idesc_fmt(int M, int N, int a_mn, int b_mn, uint32_t fmt) {
+  return (1u << 4)                       // D format: f32
+         | (fmt << 7)                    // A format
+         | (fmt << 10)                   // B format
+         | ((uint32_t)a_mn << 15)        // A major (0 = K, 1 = MN)
+         | ((uint32_t)b_mn << 16)        // B major
+         | ((uint32_t)(N >> 3) << 17)    // N >> 3
+         | ((uint32_t)(M >> 4) << 24);   // M >> 4
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.

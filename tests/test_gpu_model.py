@@ -38,7 +38,8 @@ def _mods():
 
 
 def small_cfg(kind="nf4", tied=False, n_layers=3):
-    return M.ModelConfig(hidden=256, n_q_heads=2, n_kv_heads=1, head_dim=128, intermediate=512, rank=16,
+    # reduced Llama-style shape: 4 q / 2 kv heads of 128 (GQA group 2), SwiGLU 1024
+    return M.ModelConfig(hidden=512, n_q_heads=4, n_kv_heads=2, head_dim=128, intermediate=1024, rank=16,
                          alpha=32.0, vocab=512, n_layers=n_layers, kind=kind, tied=tied)
 
 
