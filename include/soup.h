@@ -57,19 +57,20 @@ soup_status soup_device_error(int32_t* code_out);
 /* Number of kernels this library has launched in this process. */
 int64_t soup_launch_count(void);
 
-/* Optional timing of the tensor-core GEMM launches: when enabled, every GEMM
- * launch is bracketed by CUDA events recorded on its own stream and tagged
- * with its class and algorithmic work.  soup_profile_read synchronises those
- * events and sums them per class: 0 = fused NF4-decode GEMM (forward, W),
- * 1 = fused NF4-decode GEMM (backward, W^T), 2 = other bf16 GEMMs with
- * N > 64, 3 = skinny LoRA GEMMs (N <= 64).  Enabling resets the records. */
+/* Optional timing of the tensor-core GEMM launches: while enabled, every GEMM
+ * launch of a class in class_mask (bit c = class c) is bracketed by CUDA
+ * events recorded on its own stream and tagged with its algorithmic work.
+ * soup_profile_read synchronises those events and sums them per class:
+ * 0 = fused NF4-decode GEMM (forward, W), 1 = fused NF4-decode GEMM
+ * (backward, W^T), 2 = other GEMMs with N > 64, 3 = skinny LoRA GEMMs
+ * (N <= 64).  Enabling resets the records; class_mask 0 disables. */
 typedef struct soup_gemm_profile {
   int64_t launches;
   double total_ms;
   double flops;  /* 2 M N (K + r_tail) summed over launches */
   double bytes;  /* A read once + B (NF4 packed or bf16) + output written once */
 } soup_gemm_profile;
-soup_status soup_profile_enable(int32_t on);
+soup_status soup_profile_enable(int32_t class_mask);
 soup_status soup_profile_read(soup_gemm_profile* out, int32_t n_classes);
 
 /* ------------------------------------------------------------------ NF4 ---

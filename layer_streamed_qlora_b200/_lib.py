@@ -165,8 +165,9 @@ def launch_count() -> int:
     return int(lib().soup_launch_count())
 
 
-def profile_enable(on: bool):
-    _check("soup_profile_enable", lib().soup_profile_enable(1 if on else 0))
+def profile_enable(class_mask: int):
+    """class_mask bit c enables timing of GEMM class c (GEMM_CLASSES order); 0 disables."""
+    _check("soup_profile_enable", lib().soup_profile_enable(int(class_mask)))
 
 
 def profile_read() -> dict:

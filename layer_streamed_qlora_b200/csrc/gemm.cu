@@ -26,6 +26,8 @@
 //     stride), SBO = 1024, k-step advance 2048 B.
 #include <cuda.h>
 
+#include <algorithm>
+
 #include "gemm.h"
 #include "nf4_codebook.cuh"
 #include "ptx.cuh"
@@ -39,21 +41,31 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
 
-template <int BN, bool DUAL = false>
+template <int BN, bool DUAL = false, int CG = 1>
 struct Cfg {
   // DUAL: each stage holds two A tiles (the hi and lo bf16 parts of a more
-  // precise A), multiplied against the same B tile
+  // precise A), multiplied against the same B tile.  CG = 2: the tile is
+  // shared by a CTA pair (M = 256 over the pair, each CTA holds half of B).
   static constexpr int A_STAGE = A_STAGE_BYTES * (DUAL ? 2 : 1);
-  static constexpr int B_STAGE = BN * BK * 2;
-  static constexpr int STAGES = (196608 / (A_STAGE + B_STAGE)) > 8 ? 8 : (196608 / (A_STAGE + B_STAGE));
+  static constexpr int B_STAGE = (BN / CG) * BK * 2;
+  // CTA pairs also stage the packed codes (128 rows x 32 bytes, or 64 k-rows
+  // x 64 bytes) and a 4-block-wide absmax box per stage through TMA
+  static constexpr int C_STAGE = CG == 2 ? 4096 : 0;
+  static constexpr int S_STAGE = CG == 2 ? 2048 : 0;
   static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   static constexpr int BAR_BYTES = 256;
-  static constexpr int LUT_BYTES = 16 * 32 * 4;
-  static constexpr int SMEM = 1024 + STAGES * (A_STAGE + B_STAGE) + BAR_BYTES + LUT_BYTES;
+  // CTA pairs: byte-indexed NF4 table (256 code pairs x 32 lanes x float2)
+  // at the start of shared memory; single CTAs: nibble table after the barriers
+  static constexpr int LUT_BYTES = CG == 2 ? 65536 : 16 * 32 * 4;
+  static constexpr int STAGE_BYTES = A_STAGE + B_STAGE + C_STAGE + S_STAGE;
+  static constexpr int STAGE_BUDGET = CG == 2 ? (232448 - 1024 - BAR_BYTES - LUT_BYTES) : 196608;
+  static constexpr int STAGES = (STAGE_BUDGET / STAGE_BYTES) > 8 ? 8 : (STAGE_BUDGET / STAGE_BYTES);
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + LUT_BYTES;
 };
 
 struct KArgs {
   int M, N, K, num_kb;
+  int kb_split;  // split-K: k-blocks per slice (blockIdx.z = slice), 0 = no split
   const uint8_t* codes;
   const float* absmax;
   int tail_ksteps, nseg;
@@ -62,6 +74,7 @@ struct KArgs {
   int epi, out_kind;
   void* out;
   float* out2;
+  uint16_t* out_lo;
   long long ldo;
   const uint16_t* resid;
   const float* resid_f32;
@@ -157,6 +170,23 @@ __device__ __forceinline__ uint4 decode8(uint32_t w, const float* lut_lane, floa
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Same result from the byte-indexed table of the pair kernels: entry b of
+// lane l (byte offset b*256 + l*8) holds the codebook values of the two
+// codes packed in byte b (high nibble first); one byte permute forms the
+// offset, one 8-byte shared load fetches both values, one packed multiply
+// scales them, and the products are rounded exactly as above.
+__device__ __forceinline__ uint4 decode8_pairs(uint32_t w, const uint8_t* lut_bytes, uint32_t lane8, float am) {
+  uint32_t o[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t off = __byte_perm(w, lane8, 0x5504u | ((uint32_t)p << 4));
+    const float2 c = *reinterpret_cast<const float2*>(lut_bytes + off);
+    const float2 f = ptx::mul_f32x2(c, am);
+    o[p] = pack_bf16x2(f.x, f.y);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 __device__ __forceinline__ void st_shared_v4(void* p, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ptx::smem_u32(p)), "r"(v.x),
                "r"(v.y), "r"(v.z), "r"(v.w)
@@ -179,14 +209,16 @@ __device__ __forceinline__ void load_codes(const uint8_t* src, uint32_t (&w)[NWO
   }
 }
 
-template <int BN, int AMJ, int BMD, bool TF, bool DUAL>
+template <int BN, int AMJ, int BMD, bool TF, bool DUAL, int CG>
 __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmTA,
                 const __grid_constant__ CUtensorMap tmTB, const __grid_constant__ CUtensorMap tmA2,
                 const KArgs args) {
-  using C = Cfg<BN, DUAL>;
+  using C = Cfg<BN, DUAL, CG>;
   static_assert(!DUAL || (AMJ == A_K && !TF), "dual-A: K-major bf16 A only");
+  static_assert(CG == 1 || (BN == 256 && AMJ == A_K && BMD >= B_NF4_K && !TF && !DUAL),
+                "CTA pairs: NF4 B, K-major bf16 A, 256-wide tiles");
   constexpr bool NF4 = BMD >= B_NF4_K;
   constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
   constexpr int STAGES = C::STAGES;
@@ -201,53 +233,80 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
   constexpr int KSTEP_MN = KI * 128;         // MN-major descriptor advance per MMA
   static_assert(!TF || (BMD == B_TMA_K), "tf32 mode: TMA-fed K-major B only");
 
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  constexpr int LUT_FRONT = CG == 2 ? C::LUT_BYTES : 0;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+      (reinterpret_cast<uintptr_t>(smem_raw + LUT_FRONT) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * C::A_STAGE;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_STAGE);
+  uint8_t* sC = sB + STAGES * C::B_STAGE;     // CTA pairs: packed codes per stage
+  uint8_t* sS = sC + STAGES * C::C_STAGE;     // CTA pairs: absmax box per stage
+  uint64_t* full = reinterpret_cast<uint64_t*>(sS + STAGES * C::S_STAGE);
   uint64_t* empty = full + STAGES;
-  uint64_t* accf = empty + STAGES;
+  uint64_t* cfull = empty + STAGES;           // CTA pairs: codes + absmax of the stage landed
+  uint64_t* accf = cfull + (CG == 2 ? STAGES : 0);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* lut = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pairs: blockIdx.x = 2 * (pair M tile) + rank; this CTA owns rows
+  // [m0, m0 + 128) of A and of the accumulator either way
+  const uint32_t rank = CG == 2 ? ptx::cluster_ctarank() : 0u;
   const int m0 = blockIdx.x * BM;
   const bool paired = args.pair_off > 0;
   // paired: the tile covers columns [nb, nb + BN/2) of both halves
   const int nb = paired ? blockIdx.y * (BN / 2) : blockIdx.y * BN;
   const int n0 = nb;  // first B row / output column of the tile (first half when paired)
-  const int num_kb = args.num_kb;
+  // split-K: this CTA's slice of k-blocks and its fp32 partial-product plane
+  const int kz = args.kb_split > 0 ? (int)blockIdx.z * args.kb_split : 0;
+  const int num_kb = args.kb_split > 0 ? min(args.kb_split, args.num_kb - kz) : args.num_kb;
   const int n_iters = num_kb + (args.tail_ksteps > 0 ? 1 : 0);
+  void* const outp = args.kb_split > 0 ? static_cast<void*>(static_cast<float*>(args.out) +
+                                                           (size_t)blockIdx.z * args.M * args.ldo)
+                                       : args.out;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&full[s], 1 + (NF4 ? 8 : 0));
+      ptx::mbar_init(&full[s], CG == 2 ? 1 + 16 : 1 + (NF4 ? 8 : 0));
       ptx::mbar_init(&empty[s], 1);
+      if (CG == 2) ptx::mbar_init(&cfull[s], 1);
     }
     ptx::mbar_init(accf, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmA);
-    if (DUAL) ptx::prefetch_tmap(&tmA2);
-    if (!NF4) ptx::prefetch_tmap(&tmB);
+    if (DUAL || CG == 2) ptx::prefetch_tmap(&tmA2);
+    if (!NF4 || CG == 2) ptx::prefetch_tmap(&tmB);
     if (args.tail_ksteps > 0) {
       ptx::prefetch_tmap(&tmTA);
       ptx::prefetch_tmap(&tmTB);
     }
   }
   if (NF4 && threadIdx.x >= 64) {
-    for (int i = threadIdx.x - 64; i < 16 * 32; i += 256) lut[i] = __uint_as_float(nf4_code_bits(i >> 5));
+    if constexpr (CG == 2) {
+      float2* lut2 = reinterpret_cast<float2*>(smem_raw);
+      for (int i = threadIdx.x - 64; i < 256 * 32; i += 256) {
+        const int b = i >> 5;
+        lut2[i] = make_float2(__uint_as_float(nf4_code_bits(b >> 4)), __uint_as_float(nf4_code_bits(b & 15)));
+      }
+    } else {
+      for (int i = threadIdx.x - 64; i < 16 * 32; i += 256) lut[i] = __uint_as_float(nf4_code_bits(i >> 5));
+    }
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
-    ptx::tmem_relinquish();
+    if constexpr (CG == 2) {
+      ptx::tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
+      ptx::tmem_relinquish();
+    }
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) ptx::cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
+  else __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -259,7 +318,101 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
   if (args.nseg > 3 && n0 >= args.seg_end[2]) tail_row = args.seg_row[3];
   if (paired) tail_row = 0;
 
-  if (warp == 0) {
+  if (CG == 2 && warp == 0) {
+    // ------------------------------------------- TMA producer (CTA pair)
+    // Each CTA loads its own A rows (and its half of the tail B); the
+    // transaction bytes of both land on the even CTA's full barrier.
+    if (lane == 0) {
+      const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(full), 0);
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+          atomicOr(args.err, 1);
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* a = sA + s * C::A_STAGE;
+        uint8_t* b = sB + s * C::B_STAGE;
+        const bool tail = it >= num_kb;
+        const uint32_t bytes = tail ? (uint32_t)(A_STAGE_BYTES + C::B_STAGE) : (uint32_t)A_STAGE_BYTES;
+        if (rank == 0) ptx::mbar_arrive_expect_tx(&full[s], 2 * bytes);
+        const uint32_t bar = full0 + s * 8;
+        if (!tail) {
+          ptx::tma_load_2d_pair(a, &tmA, bar, it * BKE, m0);
+          // this CTA's codes and absmax for the stage (tmB: codes bytes,
+          // tmA2: absmax fp32; boxes out of range read as zeros)
+          uint8_t* c = sC + s * C::C_STAGE;
+          uint8_t* sc = sS + s * C::S_STAGE;
+          ptx::mbar_arrive_expect_tx(&cfull[s], (uint32_t)(C::C_STAGE + (B_MN ? 1024 : 2048)));
+          if (!B_MN) {
+            const int r0 = paired ? (rank == 0 ? nb : args.pair_off + nb) : n0 + (int)rank * 128;
+            ptx::tma_load_2d(c, &tmB, &cfull[s], it * 32, r0);
+            ptx::tma_load_2d(sc, &tmA2, &cfull[s], it & ~3, r0);
+          } else {
+            const int c0 = n0 + (int)rank * 128;
+            ptx::tma_load_2d(c, &tmB, &cfull[s], c0 / 2, it * BK);
+            ptx::tma_load_2d(sc, &tmA2, &cfull[s], (c0 / 64) & ~3, it * BK);
+          }
+        } else {
+          ptx::tma_load_2d_pair(a, &tmTA, bar, m0, tail_row);
+          ptx::tma_load_2d_pair(a + 8192, &tmTA, bar, m0 + 64, tail_row);
+          if (!B_MN) {
+            if (paired) {  // 64 rows of each half per CTA
+              ptx::tma_load_2d_pair(b, &tmTB, bar, 0, nb + (int)rank * 64);
+              ptx::tma_load_2d_pair(b + 8192, &tmTB, bar, 0, args.pair_off + nb + (int)rank * 64);
+            } else {
+              ptx::tma_load_2d_pair(b, &tmTB, bar, 0, n0 + (int)rank * 128);
+            }
+          } else {
+            ptx::tma_load_2d_pair(b, &tmTB, bar, n0 + (int)rank * 128, 0);
+            ptx::tma_load_2d_pair(b + 8192, &tmTB, bar, n0 + (int)rank * 128 + 64, 0);
+          }
+        }
+      }
+    }
+  } else if (CG == 2 && warp == 1) {
+    // ------------------------------------- MMA issuer (even CTA of the pair)
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc_main = ptx::idesc_bf16(2 * BM, BN, 0, B_MN ? 1 : 0);
+      constexpr uint32_t idesc_tail = ptx::idesc_bf16(2 * BM, BN, 1, B_MN ? 1 : 0);
+      constexpr uint32_t idesc_half = ptx::idesc_bf16(2 * BM, BN / 2, 1, B_MN ? 1 : 0);
+      bool ok = true;
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!ptx::mbar_wait_bounded(&full[s], ph, abort_flag)) {
+          atomicOr(args.err, 1);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t a_base = ptx::smem_u32(sA + s * C::A_STAGE);
+        const uint32_t b_base = ptx::smem_u32(sB + s * C::B_STAGE);
+        const bool tail = it >= num_kb;
+        if (tail && paired) {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint64_t ad = ptx::smem_desc_sw128(a_base + hf * 2048, 8192, 1024);
+            const uint64_t bd = ptx::smem_desc_sw128(b_base + hf * 8192, 16, 1024);
+            ptx::mma_bf16_pair(tmem + hf * (BN / 2), ad, bd, idesc_half, 1u);
+          }
+        } else {
+          const int nk = tail ? args.tail_ksteps : BKE / KI;
+          for (int k = 0; k < nk; ++k) {
+            const uint64_t ad = tail ? ptx::smem_desc_sw128(a_base + k * KSTEP_MN, CHUNK_BYTES, 1024)
+                                     : ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k * KSTEP_MN, CHUNK_BYTES, 1024)
+                                     : ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
+            ptx::mma_bf16_pair(tmem, ad, bd, tail ? idesc_tail : idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+          }
+        }
+        ptx::mma_commit_pair(&empty[s], 3);
+      }
+      if (ok) ptx::mma_commit_pair(accf, 3);
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       for (int it = 0; it < n_iters; ++it) {
@@ -276,7 +429,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
         const uint32_t bytes = ((DUAL && !tail) ? C::A_STAGE : A_STAGE_BYTES) + ((!NF4 || tail) ? C::B_STAGE : 0);
         ptx::mbar_arrive_expect_tx(&full[s], bytes);
         if (!tail) {
-          const int k0 = it * BKE;
+          const int k0 = (kz + it) * BKE;
           if (AMJ == A_K) {
             ptx::tma_load_2d(a, &tmA, &full[s], k0, m0);
             if (DUAL) ptx::tma_load_2d(a + A_STAGE_BYTES, &tmA2, &full[s], k0, m0);
@@ -375,7 +528,70 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     }
   } else {
     const int t = threadIdx.x - 64;  // 0 .. (NF4 ? 255 : 127)
-    if constexpr (NF4) {
+    if constexpr (NF4 && CG == 2) {
+      // ------------------------------------------ NF4 decode warps (CTA pair)
+      // This CTA decodes its 128 of the tile's 256 B rows (K-major: weight
+      // rows; transposed: weight columns); each thread one 32-element run
+      // per stage (one absmax), codes of stage it+1 prefetched in registers.
+      // Arrivals go to the even CTA's full barrier.
+      const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(full), 0);
+      const uint32_t lane8 = (uint32_t)lane * 8u;
+      const uint8_t* lutb = smem_raw;
+      // thread -> (shared row of the B stage, first 16-byte unit, chunk),
+      // its 16 code bytes within the staged codes tile, and its absmax
+      // within the staged absmax box (fp32 index)
+      int srow, unit0, chunk, coff, soff;
+      bool valid;
+      if constexpr (BMD == B_NF4_K) {
+        const int row = t >> 1, h = t & 1;
+        const int n = paired ? (rank == 0 ? nb + row : args.pair_off + nb + row) : n0 + (int)rank * 128 + row;
+        valid = n < args.N;
+        srow = row;
+        unit0 = h * 4;
+        chunk = 0;
+        coff = row * 32 + h * 16;
+        soff = row * 4;  // + (it & 3)
+      } else {
+        const int q = t & 3, kr = t >> 2;
+        const int col = n0 + (int)rank * 128 + q * 32;
+        valid = col < args.N;
+        srow = kr;
+        unit0 = (q & 1) * 4;
+        chunk = q >> 1;
+        coff = kr * 64 + q * 16;
+        soff = kr * 4 + ((n0 + (int)rank * 128) / 64 & 3) + (q >> 1);
+      }
+      uint8_t* const drow = sB + chunk * 8192 + srow * 128;
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+          atomicOr(args.err, 1);
+          *abort_flag = 1;
+          break;
+        }
+        if (it < num_kb) {
+          if (!ptx::mbar_wait_bounded(&cfull[s], ph, abort_flag)) {
+            atomicOr(args.err, 1);
+            *abort_flag = 1;
+            break;
+          }
+          const uint4 w = *reinterpret_cast<const uint4*>(sC + s * C::C_STAGE + coff);
+          const float am =
+              reinterpret_cast<const float*>(sS + s * C::S_STAGE)[soff + (BMD == B_NF4_K ? (it & 3) : 0)];
+          uint8_t* b = drow + s * C::B_STAGE;
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 v = valid ? decode8_pairs(ws[u], lutb, lane8, am) : make_uint4(0, 0, 0, 0);
+            st_shared_v4(b + (((unit0 + u) ^ (srow & 7)) << 4), v);
+          }
+          ptx::fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(full0 + s * 8);
+      }
+    } else if constexpr (NF4) {
       // ----------------------------------------------------- NF4 decode warps
       // Each thread decodes one row-segment of the B tile per stage; the
       // codes of stage it+1 are loaded into registers while stage it is
@@ -508,7 +724,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
             uu[i] = __uint_as_float(vu[i]) * alpha;
             a[i] = gg[i] * sigmoid_f(gg[i]) * uu[i];
           }
-          store_row16(args.out, OUT_BF16, args.ldo, row, n, I, a, vec);
+          store_row16(outp, OUT_BF16, args.ldo, row, n, I, a, vec);
           if (args.aux16) {
             store_row16(args.aux16, OUT_F16, args.ld_aux, row, n, I, gg, vec);
             store_row16(args.aux16 + I, OUT_F16, args.ld_aux, row, n, I, uu, vec);
@@ -537,8 +753,8 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
             a[i] = x0 * c - x1 * sv;
             b[i] = x1 * c + x0 * sv;
           }
-          store_row16(args.out, args.out_kind, args.ldo, row, n, args.N, a, vec);
-          store_row16(args.out, args.out_kind, args.ldo, row, n + 64, args.N, b, vec);
+          store_row16(outp, args.out_kind, args.ldo, row, n, args.N, a, vec);
+          store_row16(outp, args.out_kind, args.ldo, row, n + 64, args.N, b, vec);
         }
       } else {
         for (int ch = ch0; ch < NCH; ch += chs) {
@@ -574,13 +790,22 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
               dg[i] = f[i] * u * sg * (1.0f + g * (1.0f - sg));
               du[i] = f[i] * g * sg;
             }
-            store_row16(args.out, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
-            store_row16(static_cast<uint16_t*>(args.out) + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
+            store_row16(outp, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
+            store_row16(static_cast<uint16_t*>(outp) + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
+            if (args.out_lo) {  // rounding residuals of both halves, same layout
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                dg[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(dg[i], 0.f) & 0xFFFF));
+                du[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(du[i], 0.f) & 0xFFFF));
+              }
+              store_row16(args.out_lo, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
+              store_row16(args.out_lo + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
+            }
             continue;
           }
           if (args.out_kind == OUT_BF16_T || args.out_kind == OUT_F32_T) {
             if (args.out_kind == OUT_BF16_T) {
-              uint16_t* o = static_cast<uint16_t*>(args.out);
+              uint16_t* o = static_cast<uint16_t*>(outp);
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 if (n + i < args.N)
@@ -590,8 +815,17 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
                 for (int i = 0; i < 16; ++i)
                   if (n + i < args.N) args.out2[(size_t)(n + i) * args.ldo + row] = f[i];
               }
+              if (args.out_lo) {  // rounding residual: hi + lo carries ~16 significant bits
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                  if (n + i < args.N) {
+                    const uint16_t hb = static_cast<uint16_t>(pack_bf16x2(f[i], 0.f) & 0xFFFF);
+                    args.out_lo[(size_t)(n + i) * args.ldo + row] =
+                        static_cast<uint16_t>(pack_bf16x2(f[i] - bf16_to_f32(hb), 0.f) & 0xFFFF);
+                  }
+              }
             } else {
-              float* o = static_cast<float*>(args.out);
+              float* o = static_cast<float*>(outp);
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 if (n + i < args.N) o[(size_t)(n + i) * args.ldo + row] = f[i];
@@ -624,7 +858,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
                 if (n + i < args.N) f[i] += r[i];
             }
           }
-          store_row16(args.out, args.out_kind, args.ldo, row, n, args.N, f, vec);
+          store_row16(outp, args.out_kind, args.ldo, row, n, args.N, f, vec);
         }
       }
     }
@@ -640,9 +874,39 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     }
     __syncthreads();
   }
+  if constexpr (CG == 2) ptx::cluster_sync();  // no CTA leaves while its pair may still signal it
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+    if constexpr (CG == 2) ptx::tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Split-K epilogue: out = alpha * sum over slices (in slice order) of the
+// fp32 partial products ws[z, M, N], stored as the GEMM's own epilogue would.
+__global__ void splitk_reduce_kernel(const float* __restrict__ ws, int splits, int M, int N, int out_kind,
+                                     void* out, float* out2, uint16_t* out_lo, long long ldo, float alpha,
+                                     const unsigned int* scale_amax) {
+  const float a = scale_amax ? alpha * grad_scale_from_amax(__uint_as_float(*scale_amax)) : alpha;
+  const bool tr = out_kind == OUT_BF16_T || out_kind == OUT_F32_T;
+  const size_t total = (size_t)M * N, plane = (size_t)M * N;
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += (size_t)gridDim.x * blockDim.x) {
+    // transposed outputs: consecutive threads take consecutive rows m
+    const int m = tr ? (int)(idx % M) : (int)(idx / N);
+    const int n = tr ? (int)(idx / M) : (int)(idx % N);
+    float acc = 0.f;
+    for (int z = 0; z < splits; ++z) acc += ws[z * plane + (size_t)m * N + n];
+    const float v = acc * a;
+    const size_t o = tr ? (size_t)n * ldo + m : (size_t)m * ldo + n;
+    if (out_kind == OUT_F32 || out_kind == OUT_F32_T) {
+      static_cast<float*>(out)[o] = v;
+    } else {
+      const uint32_t w = out_kind == OUT_F16 ? pack_f16x2(v, 0.f) : pack_bf16x2(v, 0.f);
+      static_cast<uint16_t*>(out)[o] = static_cast<uint16_t>(w & 0xFFFF);
+      if (out2 && out_kind == OUT_BF16_T) out2[o] = v;
+      if (out_lo && out_kind == OUT_BF16_T)
+        out_lo[o] = static_cast<uint16_t>(pack_bf16x2(v - bf16_to_f32(static_cast<uint16_t>(w & 0xFFFF)), 0.f) & 0xFFFF);
+    }
   }
 }
 
@@ -674,9 +938,29 @@ soup_status make_map(CUtensorMap* m, const Mat& mat, uint32_t box0, uint32_t box
   return SOUP_OK;
 }
 
-template <int BN, int AMJ, int BMD, bool TF = false, bool DUAL = false>
+// Un-swizzled tensor map over a row-major [rows, cols] array of 1- or 4-byte
+// elements (the NF4 codes / absmax staging of the pair kernels).
+soup_status make_plain_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int es, int dtype,
+                           uint32_t box0, uint32_t box1, const char* what) {
+  SOUP_CHECK(ptr && rows > 0 && cols > 0, SOUP_ERR_INVALID_ARG, "gemm: %s is empty", what);
+  SOUP_CHECK(soup_aligned(ptr, 16), SOUP_ERR_ALIGN, "gemm: %s base not 16-byte aligned", what);
+  SOUP_CHECK((cols * es) % 16 == 0, SOUP_ERR_ALIGN, "gemm: %s row of %lld bytes is not a multiple of 16", what,
+             (long long)(cols * es));
+  EncodeTiledFn enc = encode_tiled();
+  SOUP_CHECK(enc != nullptr, SOUP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const uint64_t gdim[2] = {(uint64_t)cols, (uint64_t)rows};
+  const uint64_t gstride[1] = {(uint64_t)(cols * es)};
+  const uint32_t box[2] = {box0, box1};
+  const uint32_t estr[2] = {1, 1};
+  int r = enc(m, dtype, 2, const_cast<void*>(ptr), gdim, gstride, box, estr, 0, 0 /* no swizzle */, CU_L2_256B, 0);
+  SOUP_CHECK(r == 0, SOUP_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, r);
+  return SOUP_OK;
+}
+constexpr int CU_DT_U8 = 0;  // CU_TENSOR_MAP_DATA_TYPE_UINT8
+
+template <int BN, int AMJ, int BMD, bool TF = false, bool DUAL = false, int CG = 1>
 soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
-  using C = Cfg<BN, DUAL>;
+  using C = Cfg<BN, DUAL, CG>;
   CUtensorMap mA, mB, mTA, mTB, mA2;
   memset(&mA2, 0, sizeof(mA2));
   if (DUAL) SOUP_TRY(make_map(&mA2, d.A_lo, 64, 128, "A (lo part)"));
@@ -691,12 +975,25 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
   constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
   if (BMD == B_TMA_K) SOUP_TRY(make_map(&mB, d.B, EW, paired ? BN / 2 : BN, "B", TF));
   if (BMD == B_TMA_MN) SOUP_TRY(make_map(&mB, d.B, 64, 64, "B (MN-major)"));
+  if (CG == 2) {
+    // codes and absmax staged per stage: K-major 128 rows x 32 bytes and a
+    // 128 x 4 absmax box; transposed 64 k-rows x 64 bytes and a 64 x 4 box
+    if (BMD == B_NF4_K) {
+      SOUP_TRY(make_plain_map(&mB, d.codes, d.N, d.K / 2, 1, CU_DT_U8, 32, 128, "NF4 codes"));
+      SOUP_TRY(make_plain_map(&mA2, d.absmax, d.N, d.K / 64, 4, CU_DT_F32, 4, 128, "NF4 absmax"));
+    } else {
+      SOUP_TRY(make_plain_map(&mB, d.codes, d.K, d.N / 2, 1, CU_DT_U8, 64, 64, "NF4 codes (transposed)"));
+      SOUP_TRY(make_plain_map(&mA2, d.absmax, d.K, d.N / 64, 4, CU_DT_F32, 4, 64, "NF4 absmax (transposed)"));
+    }
+  }
   if (d.tail_ksteps > 0) {
     SOUP_TRY(make_map(&mTA, d.tailA, 64, 64, "tail A"));
-    if (!B_MN) SOUP_TRY(make_map(&mTB, d.tailB, 64, paired ? BN / 2 : BN, "tail B"));
+    // K-major tail B rows per box: the tile's (CTA pairs: this CTA's half of
+    // it; paired gate|up tiles: one half of the pair's half)
+    if (!B_MN) SOUP_TRY(make_map(&mTB, d.tailB, 64, (paired ? BN / 2 : BN) / CG, "tail B"));
     else SOUP_TRY(make_map(&mTB, d.tailB, 64, 64, "tail B (MN-major)"));
   }
-  auto kern = gemm_kernel<BN, AMJ, BMD, TF, DUAL>;
+  auto kern = gemm_kernel<BN, AMJ, BMD, TF, DUAL, CG>;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
     SOUP_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
@@ -704,7 +1001,8 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
   }
   constexpr int NT = 32 * (2 + (BMD >= B_NF4_K ? 8 : 4));
   const int ntiles = paired ? (d.pair_off + BN / 2 - 1) / (BN / 2) : (d.N + BN - 1) / BN;
-  dim3 grid((d.M + BM - 1) / BM, ntiles);
+  const int nz = ka.kb_split > 0 ? (ka.num_kb + ka.kb_split - 1) / ka.kb_split : 1;
+  dim3 grid(CG == 2 ? 2 * ((d.M + 2 * BM - 1) / (2 * BM)) : (d.M + BM - 1) / BM, ntiles, nz);
   if (profiling()) {
     // algorithmic work: 2 M N K (+ 2 M N r for the LoRA tail); bytes: the
     // operands read once and the output written once
@@ -716,7 +1014,24 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
     const double bytes = (double)d.M * d.K * 2 + wbytes + (double)d.M * d.N * oes;
     profile_begin(st, cls, flops, bytes);
   }
-  kern<<<grid, NT, C::SMEM, st>>>(mA, mB, mTA, mTB, mA2, ka);
+  if constexpr (CG == 2) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    SOUP_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, mA, mB, mTA, mTB, mA2, ka));
+  } else {
+    kern<<<grid, NT, C::SMEM, st>>>(mA, mB, mTA, mTB, mA2, ka);
+  }
   SOUP_LAUNCH_CHECK();
   profile_end(st);
   return SOUP_OK;
@@ -736,6 +1051,67 @@ int pick_bn(const GemmDesc& d) {
   if (d.N >= 256 && (d.N % 256 == 0 || d.N >= 1024) && fits(256)) return 256;
   if (d.N >= 128 && fits(128)) return 128;
   return 64;
+}
+
+// Kernel selection for one launch (after the descriptor checks).
+soup_status dispatch(const GemmDesc& d, const KArgs& ka, int bn, cudaStream_t st) {
+  const bool nf4 = d.b_mode >= B_NF4_K;
+  if (d.tf32) {
+    SOUP_CHECK(d.b_mode == B_TMA_K && d.tail_ksteps == 0 && d.pair_off == 0 && d.epi == EPI_STORE && bn <= 64,
+               SOUP_ERR_SHAPE, "gemm: tf32 mode supports skinny (N <= 64) K-major-B GEMMs without tail");
+#define SOUP_GEMM_TF(BN_, AM_) \
+  if (bn == BN_ && d.a_major == AM_) return launch<BN_, AM_, B_TMA_K, true>(d, ka, st);
+    SOUP_GEMM_TF(64, A_K) SOUP_GEMM_TF(48, A_K) SOUP_GEMM_TF(32, A_K) SOUP_GEMM_TF(16, A_K)
+    SOUP_GEMM_TF(64, A_MN) SOUP_GEMM_TF(48, A_MN) SOUP_GEMM_TF(32, A_MN) SOUP_GEMM_TF(16, A_MN)
+#undef SOUP_GEMM_TF
+    return fail(SOUP_ERR_SHAPE, "gemm: no tf32 kernel for BN=%d", bn);
+  }
+  if (d.A_lo.ptr) {
+    SOUP_CHECK(d.a_major == A_K && !d.tf32 && (bn == 256 || bn == 128 || (bn <= 32 && d.b_mode == B_TMA_K)) &&
+                   d.A_lo.rows == d.A.rows &&
+                   d.A_lo.cols == d.A.cols,
+               SOUP_ERR_SHAPE, "gemm: dual-A needs a K-major bf16 A, N tile 128/256 (16/32 for skinny K-major B) "
+               "and matching hi/lo shapes");
+#define SOUP_GEMM_DUAL(BN_, BMD_) \
+  if (bn == BN_ && d.b_mode == BMD_) return launch<BN_, A_K, BMD_, false, true>(d, ka, st);
+    SOUP_GEMM_DUAL(256, B_NF4_K) SOUP_GEMM_DUAL(128, B_NF4_K) SOUP_GEMM_DUAL(256, B_NF4_MN)
+    SOUP_GEMM_DUAL(128, B_NF4_MN) SOUP_GEMM_DUAL(256, B_TMA_K) SOUP_GEMM_DUAL(128, B_TMA_K)
+    SOUP_GEMM_DUAL(256, B_TMA_MN) SOUP_GEMM_DUAL(128, B_TMA_MN)
+    SOUP_GEMM_DUAL(32, B_TMA_K) SOUP_GEMM_DUAL(16, B_TMA_K)
+#undef SOUP_GEMM_DUAL
+    return fail(SOUP_ERR_SHAPE, "gemm: no dual-A kernel for BN=%d b_mode=%d", bn, d.b_mode);
+  }
+  // NF4 B with 256-wide tiles: CTA pairs (half the decode per CTA)
+  const bool pair_ok = nf4 && bn == 256 && d.a_major == A_K && soup_aligned(d.absmax, 16) &&
+                       (d.b_mode == B_NF4_K ? d.K % 256 == 0 : d.N % 256 == 0);
+  if (pair_ok) {
+    if (d.b_mode == B_NF4_K) return launch<256, A_K, B_NF4_K, false, false, 2>(d, ka, st);
+    return launch<256, A_K, B_NF4_MN, false, false, 2>(d, ka, st);
+  }
+#define SOUP_GEMM_CASE(BN_, AM_, BMD_) \
+  if (bn == BN_ && d.a_major == AM_ && d.b_mode == BMD_) return launch<BN_, AM_, BMD_>(d, ka, st);
+  SOUP_GEMM_CASE(256, A_K, B_NF4_K)
+  SOUP_GEMM_CASE(128, A_K, B_NF4_K)
+  SOUP_GEMM_CASE(64, A_K, B_NF4_K)
+  SOUP_GEMM_CASE(256, A_K, B_NF4_MN)
+  SOUP_GEMM_CASE(128, A_K, B_NF4_MN)
+  SOUP_GEMM_CASE(64, A_K, B_NF4_MN)
+  SOUP_GEMM_CASE(256, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(128, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(64, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(48, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(32, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(16, A_K, B_TMA_K)
+  SOUP_GEMM_CASE(256, A_K, B_TMA_MN)
+  SOUP_GEMM_CASE(128, A_K, B_TMA_MN)
+  SOUP_GEMM_CASE(64, A_K, B_TMA_MN)
+  SOUP_GEMM_CASE(64, A_MN, B_TMA_K)
+  SOUP_GEMM_CASE(48, A_MN, B_TMA_K)
+  SOUP_GEMM_CASE(32, A_MN, B_TMA_K)
+  SOUP_GEMM_CASE(16, A_MN, B_TMA_K)
+#undef SOUP_GEMM_CASE
+  return fail(SOUP_ERR_SHAPE, "gemm: no kernel for BN=%d a_major=%d b_mode=%d (M=%d N=%d K=%d)", bn,
+              d.a_major, d.b_mode, d.M, d.N, d.K);
 }
 
 }  // namespace
@@ -780,7 +1156,7 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
   for (int i = 0; i < 4; ++i) { ka.seg_end[i] = d.seg_end[i]; ka.seg_row[i] = d.seg_row[i]; }
   ka.pair_off = d.pair_off;
   ka.epi = d.epi;
-  ka.out_kind = d.out_kind; ka.out = d.out; ka.ldo = d.ldo; ka.out2 = d.out2;
+  ka.out_kind = d.out_kind; ka.out = d.out; ka.ldo = d.ldo; ka.out2 = d.out2; ka.out_lo = d.out_lo;
   ka.resid = d.resid; ka.resid_f32 = d.resid_f32; ka.ldr = d.ldr; ka.alpha = d.alpha;
   ka.scale_amax = d.scale_amax;
   ka.aux16 = d.aux16; ka.ld_aux = d.ld_aux; ka.swiglu_I = d.swiglu_I;
@@ -799,52 +1175,36 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
   ka.err = device_error_word();
   SOUP_CHECK(ka.err != nullptr, SOUP_ERR_CUDA, "device error word unavailable");
 
-  if (d.tf32) {
-    SOUP_CHECK(d.b_mode == B_TMA_K && d.tail_ksteps == 0 && d.pair_off == 0 && d.epi == EPI_STORE && bn <= 64,
-               SOUP_ERR_SHAPE, "gemm: tf32 mode supports skinny (N <= 64) K-major-B GEMMs without tail");
-#define SOUP_GEMM_TF(BN_, AM_) \
-  if (bn == BN_ && d.a_major == AM_) return launch<BN_, AM_, B_TMA_K, true>(d, ka, st);
-    SOUP_GEMM_TF(64, A_K) SOUP_GEMM_TF(48, A_K) SOUP_GEMM_TF(32, A_K) SOUP_GEMM_TF(16, A_K)
-    SOUP_GEMM_TF(64, A_MN) SOUP_GEMM_TF(48, A_MN) SOUP_GEMM_TF(32, A_MN) SOUP_GEMM_TF(16, A_MN)
-#undef SOUP_GEMM_TF
-    return fail(SOUP_ERR_SHAPE, "gemm: no tf32 kernel for BN=%d", bn);
+  if (d.split_ws && d.split_ws_bytes > 0 && !nf4 && d.epi == EPI_STORE && d.tail_ksteps == 0 &&
+      !d.resid && !d.resid_f32 && d.pair_off == 0 && d.rope_cols == 0 &&
+      (d.out_kind == OUT_BF16_T || d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T || d.out_kind == OUT_BF16) &&
+      d.N % 4 == 0 && soup_aligned(d.split_ws, 16)) {
+    const int sms = sm_count();
+    const int tiles = ((d.M + BM - 1) / BM) * ((d.N + bn - 1) / bn);
+    int splits = std::min(8, std::min(ka.num_kb / 2, (sms + tiles - 1) / tiles));
+    while (splits > 1 && (size_t)splits * d.M * d.N * 4 > d.split_ws_bytes) --splits;
+    if (splits > 1) {
+      KArgs kz = ka;
+      kz.kb_split = (ka.num_kb + splits - 1) / splits;
+      splits = (ka.num_kb + kz.kb_split - 1) / kz.kb_split;
+      kz.out = d.split_ws;
+      kz.out_kind = OUT_F32;
+      kz.ldo = d.N;
+      kz.out2 = nullptr;
+      kz.out_lo = nullptr;
+      kz.alpha = 1.f;
+      kz.scale_amax = nullptr;
+      kz.vec_ok = 1;
+      SOUP_TRY(dispatch(d, kz, bn, st));
+      const size_t total = (size_t)d.M * d.N;
+      const int blocks = (int)std::min<size_t>((total + 255) / 256, (size_t)sms * 8);
+      splitk_reduce_kernel<<<blocks, 256, 0, st>>>(d.split_ws, splits, d.M, d.N, d.out_kind, d.out, d.out2,
+                                                   d.out_lo, d.ldo, d.alpha, d.scale_amax);
+      SOUP_LAUNCH_CHECK();
+      return SOUP_OK;
+    }
   }
-  if (d.A_lo.ptr) {
-    SOUP_CHECK(d.a_major == A_K && !d.tf32 && (bn == 256 || bn == 128) && d.A_lo.rows == d.A.rows &&
-                   d.A_lo.cols == d.A.cols,
-               SOUP_ERR_SHAPE, "gemm: dual-A needs a K-major bf16 A, N tile 128/256 and matching hi/lo shapes");
-#define SOUP_GEMM_DUAL(BN_, BMD_) \
-  if (bn == BN_ && d.b_mode == BMD_) return launch<BN_, A_K, BMD_, false, true>(d, ka, st);
-    SOUP_GEMM_DUAL(256, B_NF4_K) SOUP_GEMM_DUAL(128, B_NF4_K) SOUP_GEMM_DUAL(256, B_NF4_MN)
-    SOUP_GEMM_DUAL(128, B_NF4_MN) SOUP_GEMM_DUAL(256, B_TMA_K) SOUP_GEMM_DUAL(128, B_TMA_K)
-    SOUP_GEMM_DUAL(256, B_TMA_MN) SOUP_GEMM_DUAL(128, B_TMA_MN)
-#undef SOUP_GEMM_DUAL
-    return fail(SOUP_ERR_SHAPE, "gemm: no dual-A kernel for BN=%d b_mode=%d", bn, d.b_mode);
-  }
-#define SOUP_GEMM_CASE(BN_, AM_, BMD_) \
-  if (bn == BN_ && d.a_major == AM_ && d.b_mode == BMD_) return launch<BN_, AM_, BMD_>(d, ka, st);
-  SOUP_GEMM_CASE(256, A_K, B_NF4_K)
-  SOUP_GEMM_CASE(128, A_K, B_NF4_K)
-  SOUP_GEMM_CASE(64, A_K, B_NF4_K)
-  SOUP_GEMM_CASE(256, A_K, B_NF4_MN)
-  SOUP_GEMM_CASE(128, A_K, B_NF4_MN)
-  SOUP_GEMM_CASE(64, A_K, B_NF4_MN)
-  SOUP_GEMM_CASE(256, A_K, B_TMA_K)
-  SOUP_GEMM_CASE(128, A_K, B_TMA_K)
-  SOUP_GEMM_CASE(64, A_K, B_TMA_K)
-  SOUP_GEMM_CASE(48, A_K, B_TMA_K)
-  SOUP_GEMM_CASE(32, A_K, B_TMA_K)
-  SOUP_GEMM_CASE(16, A_K, B_TMA_K)
-  SOUP_GEMM_CASE(256, A_K, B_TMA_MN)
-  SOUP_GEMM_CASE(128, A_K, B_TMA_MN)
-  SOUP_GEMM_CASE(64, A_K, B_TMA_MN)
-  SOUP_GEMM_CASE(64, A_MN, B_TMA_K)
-  SOUP_GEMM_CASE(48, A_MN, B_TMA_K)
-  SOUP_GEMM_CASE(32, A_MN, B_TMA_K)
-  SOUP_GEMM_CASE(16, A_MN, B_TMA_K)
-#undef SOUP_GEMM_CASE
-  return fail(SOUP_ERR_SHAPE, "gemm: no kernel for BN=%d a_major=%d b_mode=%d (M=%d N=%d K=%d)", bn,
-              d.a_major, d.b_mode, d.M, d.N, d.K);
+  return dispatch(d, ka, bn, st);
 }
 
 }  // namespace soup

@@ -69,6 +69,8 @@ struct GemmDesc {
   int out_kind = OUT_BF16;
   void* out = nullptr;
   float* out2 = nullptr;            // OUT_BF16_T only: also the unrounded fp32 values, same layout
+  uint16_t* out_lo = nullptr;       // OUT_BF16_T and EPI_SWIGLU_BWD: also the rounding residual
+                                    // bf16(v - bf16(v)), same layout
   int64_t ldo = 0;
   const uint16_t* resid = nullptr;  // bf16 [M, N] row stride ldr (row-major outputs)
   const float* resid_f32 = nullptr; // fp32 [M, N] row stride ldr (row-major outputs)
@@ -87,6 +89,13 @@ struct GemmDesc {
   const float* rope_cos = nullptr;
   const float* rope_sin = nullptr;
   int bn = 0;               // N tile (0 = pick)
+  // Optional split-K for skinny GEMMs (N <= 64, TMA operands, plain store
+  // epilogue): when a workspace is given and the M x N tiles alone cannot
+  // fill the GPU, the K range is cut into up to 8 slices whose fp32 partial
+  // products land in split_ws ([slices, M, N]); a second kernel sums them
+  // in slice order (deterministic) and applies the epilogue.
+  float* split_ws = nullptr;
+  size_t split_ws_bytes = 0;
 };
 
 soup_status gemm(const GemmDesc& d, cudaStream_t stream);

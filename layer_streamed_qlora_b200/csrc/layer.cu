@@ -38,6 +38,9 @@ struct WS {
   size_t x1_32, dqkv32, u32, g32, A32, Bt32;  // fp32 operands of the q/k/v LoRA-gradient GEMMs (tf32)
   size_t x1_lo, dh2_lo;                       // bf16 rounding residuals (dual-A GEMM inputs)
   size_t attn32, uo32, go32, Ao32;            // fp32 operands of the o LoRA-gradient GEMMs (tf32)
+  size_t splitk, splitk_bytes;                // fp32 partial products of split-K LoRA GEMMs
+  size_t u_gu_lo, g_d_lo, u_d32;     // MLP LoRA-gradient operands beyond bf16 (residuals, fp32)
+  size_t x2_32, Agu32, g_gu32, d_gu_lo;
   size_t total;
 };
 
@@ -95,6 +98,15 @@ WS layout(const Dims& m) {
   w.uo32 = take(r * ldT * 4);
   w.go32 = take(r * ldT * 4);
   w.Ao32 = take(r * (size_t)m.o_in * 4);
+  w.splitk_bytes = 8 * T * 64 * 4;
+  w.splitk = take(w.splitk_bytes);
+  w.u_gu_lo = take(2 * r * ldT * 2);
+  w.g_d_lo = take(r * ldT * 2);
+  w.u_d32 = take(r * ldT * 4);
+  w.x2_32 = take(T * H * 4);
+  w.Agu32 = take(2 * r * H * 4);
+  w.g_gu32 = take(2 * r * ldT * 4);
+  w.d_gu_lo = take(T * 2 * I * 2);
   w.total = o;
   return w;
 }
@@ -179,22 +191,39 @@ soup_status proj_fwd(const soup_weight* W, const uint16_t* x, int T, const uint1
   return gemm(g, st);
 }
 
+// Split-K workspace handed to the skinny LoRA GEMMs.
+struct SplitWS {
+  float* p = nullptr;
+  size_t bytes = 0;
+};
+void use_split(GemmDesc& g, const SplitWS& sw) {
+  g.split_ws = sw.p;
+  g.split_ws_bytes = sw.bytes;
+}
+
 // u' = bf16(s * x A^T), transposed [rows, ldT]
+// (optionally also the fp32 values u32 and the rounding residual ulo)
 soup_status lora_down(const uint16_t* x, int T, int K, const uint16_t* A, int rows, float s, uint16_t* u,
-                      int64_t ldT, cudaStream_t st) {
+                      int64_t ldT, cudaStream_t st, const SplitWS& sw, float* u32 = nullptr,
+                      uint16_t* ulo = nullptr) {
   GemmDesc g;
   g.M = T; g.N = rows; g.K = K;
   g.A = Mat{x, T, K, K};
   g.b_mode = B_TMA_K;
   g.B = Mat{A, rows, K, K};
   g.out_kind = OUT_BF16_T; g.out = u; g.ldo = ldT; g.alpha = s;
+  g.out2 = u32; g.out_lo = ulo;
+  use_split(g, sw);
   return gemm(g, st);
 }
 
 // g' = bf16(s * dy B) for one adapter segment: dy = columns [c0, c0+n) of a
 // [T, ld] buffer, B [n, r]; writes rows of a transposed [*, ldT] buffer.
+// (optionally with dy's rounding residual dy_lo as a second A, and the fp32
+// values g32 and residual glo as extra outputs)
 soup_status lora_g(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t* Bl, int r, float s, uint16_t* Bt,
-                   uint16_t* gout, int64_t ldT, cudaStream_t st) {
+                   uint16_t* gout, int64_t ldT, cudaStream_t st, const SplitWS& sw, uint16_t* glo = nullptr,
+                   const uint16_t* dy_lo = nullptr, float* g32 = nullptr) {
   SOUP_TRY(transpose_bf16(Bl, n, r, Bt, st));
   GemmDesc g;
   g.M = T; g.N = r; g.K = n;
@@ -202,12 +231,16 @@ soup_status lora_g(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t*
   g.b_mode = B_TMA_K;
   g.B = Mat{Bt, r, n, n};
   g.out_kind = OUT_BF16_T; g.out = gout; g.ldo = ldT; g.alpha = s;
+  g.out_lo = glo;
+  g.out2 = g32;
+  if (dy_lo) g.A_lo = Mat{dy_lo, T, n, ld};
+  use_split(g, sw);
   return gemm(g, st);
 }
 
 // dB [n, r] = dy_seg^T u_seg^T : dy = columns of a [T, ld] buffer.
 soup_status lora_dB(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t* u, int r, int64_t ldT, float* dB,
-                    cudaStream_t st) {
+                    cudaStream_t st, const SplitWS& sw) {
   GemmDesc g;
   g.M = n; g.N = r; g.K = T;
   g.a_major = A_MN;
@@ -215,12 +248,13 @@ soup_status lora_dB(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t
   g.b_mode = B_TMA_K;
   g.B = Mat{u, r, T, ldT};
   g.out_kind = OUT_F32; g.out = dB; g.ldo = r;
+  use_split(g, sw);
   return gemm(g, st);
 }
 
 // dA [rows, K] = g'^T x  (computed transposed: M = K, N = rows)
 soup_status lora_dA(const uint16_t* x, int T, int K, const uint16_t* gt, int rows, int64_t ldT, float* dA,
-                    cudaStream_t st) {
+                    cudaStream_t st, const SplitWS& sw) {
   GemmDesc g;
   g.M = K; g.N = rows; g.K = T;
   g.a_major = A_MN;
@@ -228,6 +262,38 @@ soup_status lora_dA(const uint16_t* x, int T, int K, const uint16_t* gt, int row
   g.b_mode = B_TMA_K;
   g.B = Mat{gt, rows, T, ldT};
   g.out_kind = OUT_F32_T; g.out = dA; g.ldo = K;
+  use_split(g, sw);
+  return gemm(g, st);
+}
+
+// dA [rows, K] = (g' + g_lo)^T x, with g' and its rounding residual g_lo
+// stored transposed [rows, ldT] (a K-major A of M = rows) and x [T, K] the
+// MN-major B: two bf16 MMAs per k-step give an fp32-accurate g.
+soup_status lora_dA_dual(const uint16_t* gt, const uint16_t* gt_lo, int rows, int64_t ldT, const uint16_t* x, int T,
+                         int K, float* dA, cudaStream_t st, const SplitWS& sw) {
+  GemmDesc g;
+  g.M = rows; g.N = K; g.K = T;
+  g.A = Mat{gt, rows, T, ldT};
+  g.A_lo = Mat{gt_lo, rows, T, ldT};
+  g.b_mode = B_TMA_MN;
+  g.B = Mat{x, T, K, K};
+  g.out_kind = OUT_F32; g.out = dA; g.ldo = K;
+  use_split(g, sw);
+  return gemm(g, st);
+}
+
+// dB [n, r] = dy_seg^T (u' + u_lo)^T, computed as (u' + u_lo) dy_seg = dB^T
+// (M = r) and stored transposed; dy = columns [c0, c0+n) of a [T, ld] buffer.
+soup_status lora_dB_dual(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t* ut, const uint16_t* ut_lo,
+                         int r, int64_t ldT, float* dB, cudaStream_t st, const SplitWS& sw) {
+  GemmDesc g;
+  g.M = r; g.N = n; g.K = T;
+  g.A = Mat{ut, r, T, ldT};
+  g.A_lo = Mat{ut_lo, r, T, ldT};
+  g.b_mode = B_TMA_MN;
+  g.B = Mat{dy, T, n, ld};
+  g.out_kind = OUT_F32_T; g.out = dB; g.ldo = r;
+  use_split(g, sw);
   return gemm(g, st);
 }
 
@@ -235,7 +301,7 @@ soup_status lora_dA(const uint16_t* x, int T, int K, const uint16_t* gt, int row
 // u = s x A^T (bf16 copy u' for the tail, fp32 copy for dB), g = s dy B
 // (bf16 copy g' for the tail, fp32 copy for dA), dA = g^T x, dB = dy^T u.
 soup_status lora_down_tf32(const float* x, int T, int K, const float* A32, int rows, float s, uint16_t* u,
-                           float* u32, int64_t ldT, cudaStream_t st) {
+                           float* u32, int64_t ldT, cudaStream_t st, const SplitWS& sw, uint16_t* ulo = nullptr) {
   GemmDesc g;
   g.tf32 = true;
   g.M = T; g.N = rows; g.K = K;
@@ -243,11 +309,14 @@ soup_status lora_down_tf32(const float* x, int T, int K, const float* A32, int r
   g.b_mode = B_TMA_K;
   g.B = Mat{A32, rows, K, K};
   g.out_kind = OUT_BF16_T; g.out = u; g.out2 = u32; g.ldo = ldT; g.alpha = s;
+  g.out_lo = ulo;
+  use_split(g, sw);
   return gemm(g, st);
 }
 
 soup_status lora_g_tf32(const float* dy, int64_t ld, int T, int n, const uint16_t* Bl, int r, float s, float* Bt32,
-                        uint16_t* gout, float* g32, int64_t ldT, cudaStream_t st) {
+                        uint16_t* gout, float* g32, int64_t ldT, cudaStream_t st, const SplitWS& sw,
+                        uint16_t* glo = nullptr) {
   SOUP_TRY(transpose_bf16_f32(Bl, n, r, Bt32, st));
   GemmDesc g;
   g.tf32 = true;
@@ -256,11 +325,13 @@ soup_status lora_g_tf32(const float* dy, int64_t ld, int T, int n, const uint16_
   g.b_mode = B_TMA_K;
   g.B = Mat{Bt32, r, n, n};
   g.out_kind = OUT_BF16_T; g.out = gout; g.out2 = g32; g.ldo = ldT; g.alpha = s;
+  g.out_lo = glo;
+  use_split(g, sw);
   return gemm(g, st);
 }
 
 soup_status lora_dB_tf32(const float* dy, int64_t ld, int T, int n, const float* u32, int r, int64_t ldT, float* dB,
-                         cudaStream_t st) {
+                         cudaStream_t st, const SplitWS& sw) {
   GemmDesc g;
   g.tf32 = true;
   g.M = n; g.N = r; g.K = T;
@@ -269,11 +340,12 @@ soup_status lora_dB_tf32(const float* dy, int64_t ld, int T, int n, const float*
   g.b_mode = B_TMA_K;
   g.B = Mat{u32, r, T, ldT};
   g.out_kind = OUT_F32; g.out = dB; g.ldo = r;
+  use_split(g, sw);
   return gemm(g, st);
 }
 
 soup_status lora_dA_tf32(const float* x, int T, int K, const float* g32, int rows, int64_t ldT, float* dA,
-                         cudaStream_t st) {
+                         cudaStream_t st, const SplitWS& sw) {
   GemmDesc g;
   g.tf32 = true;
   g.M = K; g.N = rows; g.K = T;
@@ -282,6 +354,7 @@ soup_status lora_dA_tf32(const float* x, int T, int K, const float* g32, int row
   g.b_mode = B_TMA_K;
   g.B = Mat{g32, rows, T, ldT};
   g.out_kind = OUT_F32_T; g.out = dA; g.ldo = K;
+  use_split(g, sw);
   return gemm(g, st);
 }
 
@@ -290,9 +363,10 @@ soup_status lora_dA_tf32(const float* x, int T, int K, const float* g32, int row
 soup_status proj_bwd(const soup_weight* W, const uint16_t* dy, int T, const uint16_t* gt, int64_t ldT, int g_rows,
                      const uint16_t* Al, bool on, uint16_t* dx, cudaStream_t st, int out_kind = OUT_BF16,
                      int swiglu_I = 0, uint16_t* aux16 = nullptr, const unsigned int* scale_amax = nullptr,
-                     const uint16_t* dy_lo = nullptr) {
+                     const uint16_t* dy_lo = nullptr, uint16_t* out_lo = nullptr) {
   GemmDesc g;
   g.scale_amax = scale_amax;
+  g.out_lo = out_lo;
   if (dy_lo) g.A_lo = Mat{dy_lo, T, W->out_features, W->out_features};
   g.M = T; g.N = (int)W->in_features; g.K = (int)W->out_features;
   g.A = Mat{dy, T, W->out_features, W->out_features};
@@ -319,6 +393,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
                     const WS& ws, char* base, const uint16_t* h_in, uint16_t* h_out, bool on, bool recompute,
                     cudaStream_t st) {
   const int T = m.T, r = m.r;
+  const SplitWS SW{PF(splitk), ws.splitk_bytes};
   SOUP_TRY(rope_table(m.S, m.d, (double)c->theta, PF(cosb), PF(sinb), st));
   SOUP_TRY(rmsnorm_fwd(h_in, nullptr, W->norm1, T, m.H, c->eps, P(x1), PF(rinv1), st, on ? PF(x1_32) : nullptr,
                        recompute ? P(x1_lo) : nullptr));
@@ -326,7 +401,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     // q/k/v adapters: u from the fp32 normalised input (tf32 tensor cores); the
     // tail consumes its bf16 copy, the dB GEMM its fp32 copy
     SOUP_TRY(bf16_to_f32(L->A_qkv, (size_t)3 * r * m.H, PF(A32), st));
-    SOUP_TRY(lora_down_tf32(PF(x1_32), T, m.H, PF(A32), 3 * r, m.s, P(u_qkv), PF(u32), m.ldT, st));
+    SOUP_TRY(lora_down_tf32(PF(x1_32), T, m.H, PF(A32), 3 * r, m.s, P(u_qkv), PF(u32), m.ldT, st, SW));
   }
   {
     const int se[3] = {m.Hq * m.d, (m.Hq + m.Hkv) * m.d, m.qkv_w};
@@ -346,7 +421,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
                          recompute ? P(attn16) : nullptr, on ? PF(attn32) : nullptr));
   if (on) {
     SOUP_TRY(bf16_to_f32(L->A_o, (size_t)r * m.o_in, PF(Ao32), st));
-    SOUP_TRY(lora_down_tf32(PF(attn32), T, m.o_in, PF(Ao32), r, m.s, P(u_o), PF(uo32), m.ldT, st));
+    SOUP_TRY(lora_down_tf32(PF(attn32), T, m.o_in, PF(Ao32), r, m.s, P(u_o), PF(uo32), m.ldT, st, SW));
   }
   {
     const int se[1] = {m.H};
@@ -357,8 +432,12 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     SOUP_TRY(proj_fwd(&W->o, P(attn), T, P(u_o), m.ldT, r, L ? L->B_o : nullptr, r, 1, se, sr, on,
                       reinterpret_cast<uint16_t*>(PF(h2)), st, o));
   }
-  SOUP_TRY(rmsnorm_fwd(nullptr, PF(h2), W->norm2, T, m.H, c->eps, P(x2), PF(rinv2), st));
-  if (on) SOUP_TRY(lora_down(P(x2), T, m.H, L->A_gu, 2 * r, m.s, P(u_gu), m.ldT, st));
+  SOUP_TRY(rmsnorm_fwd(nullptr, PF(h2), W->norm2, T, m.H, c->eps, P(x2), PF(rinv2), st, on ? PF(x2_32) : nullptr));
+  if (on) {
+    // u_gu from the unrounded x2 (tf32), with its rounding residual for dB
+    SOUP_TRY(bf16_to_f32(L->A_gu, (size_t)2 * r * m.H, PF(Agu32), st));
+    SOUP_TRY(lora_down_tf32(PF(x2_32), T, m.H, PF(Agu32), 2 * r, m.s, P(u_gu), nullptr, m.ldT, st, SW, P(u_gu_lo)));
+  }
   {
     const int se[1] = {2 * m.I};
     const int sr[1] = {0};
@@ -368,7 +447,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     SOUP_TRY(proj_fwd(&W->gate_up, P(x2), T, P(u_gu), m.ldT, 2 * r, L ? L->B_gu : nullptr, r, 1, se, sr, on,
                       P(act), st, o));
   }
-  if (on) SOUP_TRY(lora_down(P(act), T, m.I, L->A_down, r, m.s, P(u_d), m.ldT, st));
+  if (on) SOUP_TRY(lora_down(P(act), T, m.I, L->A_down, r, m.s, P(u_d), m.ldT, st, SW, PF(u_d32)));
   if (!recompute) {
     const int se[1] = {m.H};
     const int sr[1] = {0};
@@ -427,6 +506,7 @@ extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const
              "soup_decoder_layer_bwd: workspace %zu < %zu bytes or misaligned", workspace_bytes, ws.total);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(workspace);
+  const SplitWS SW{PF(splitk), ws.splitk_bytes};
   const int T = m.T, r = m.r, H = m.H, I = m.I;
   const int64_t ldT = m.ldT;
 
@@ -434,26 +514,31 @@ extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const
 
   // ---- MLP block
   SOUP_TRY(f32_to_bf16(dh_out, (size_t)T * H, P(dh_b), st));
-  if (on) SOUP_TRY(lora_g(P(dh_b), H, T, H, L->B_down, r, m.s, P(Bt), P(g_d), ldT, st));
+  // LoRA gradients of the MLP: g_down from the fp32 dh (tf32), the others
+  // from hi + lo (rounding residual) operand pairs, so no operand of a
+  // LoRA-gradient GEMM carries more than the bf16 rounding of d_gu
+  if (on)
+    SOUP_TRY(lora_g_tf32(dh_out, H, T, H, L->B_down, r, m.s, PF(Bt32), P(g_d), nullptr, ldT, st, SW, P(g_d_lo)));
   // d_gu = SwiGLU backward of (dh W_down + g' A_down), fused in the epilogue
   SOUP_TRY(proj_bwd(&W->down, P(dh_b), T, P(g_d), ldT, r, on ? L->A_down : nullptr, on, P(d_gu), st, OUT_BF16, I,
-                    P(gu16)));
+                    P(gu16), nullptr, nullptr, on ? P(d_gu_lo) : nullptr));
   if (on) {
-    SOUP_TRY(lora_dB(P(dh_b), H, T, H, P(u_d), r, ldT, G->dB_down, st));
-    SOUP_TRY(lora_dA(P(act), T, I, P(g_d), r, ldT, G->dA_down, st));
+    SOUP_TRY(lora_dB_tf32(dh_out, H, T, H, PF(u_d32), r, ldT, G->dB_down, st, SW));
+    SOUP_TRY(lora_dA_dual(P(g_d), P(g_d_lo), r, ldT, P(act), T, I, G->dA_down, st, SW));
   }
   uint16_t* d_gu = P(d_gu);
   if (on) {
     for (int sg = 0; sg < 2; ++sg)
       SOUP_TRY(lora_g(d_gu + (size_t)sg * I, 2 * I, T, I, L->B_gu + (size_t)sg * I * r, r, m.s, P(Bt),
-                      P(g_gu) + (size_t)sg * r * ldT, ldT, st));
+                      P(g_gu) + (size_t)sg * r * ldT, ldT, st, SW, nullptr, P(d_gu_lo) + (size_t)sg * I,
+                      PF(g_gu32) + (size_t)sg * r * ldT));
   }
   SOUP_TRY(proj_bwd(&W->gate_up, d_gu, T, P(g_gu), ldT, 2 * r, on ? L->A_gu : nullptr, on, P(dx2), st));
   if (on) {
     for (int sg = 0; sg < 2; ++sg)
-      SOUP_TRY(lora_dB(d_gu + (size_t)sg * I, 2 * I, T, I, P(u_gu) + (size_t)sg * r * ldT, r, ldT,
-                       G->dB_gu + (size_t)sg * I * r, st));
-    SOUP_TRY(lora_dA(P(x2), T, H, P(g_gu), 2 * r, ldT, G->dA_gu, st));
+      SOUP_TRY(lora_dB_dual(d_gu + (size_t)sg * I, 2 * I, T, I, P(u_gu) + (size_t)sg * r * ldT,
+                            P(u_gu_lo) + (size_t)sg * r * ldT, r, ldT, G->dB_gu + (size_t)sg * I * r, st, SW));
+    SOUP_TRY(lora_dA_tf32(PF(x2_32), T, H, PF(g_gu32), 2 * r, ldT, G->dA_gu, st, SW));
   }
   unsigned int* gamax = reinterpret_cast<unsigned int*>(base + ws.gamax);
   SOUP_CUDA_TRY(cudaMemsetAsync(gamax, 0, sizeof(unsigned int), st));
@@ -461,14 +546,14 @@ extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const
                        P(dh2_lo)));
 
   // ---- attention block
-  if (on) SOUP_TRY(lora_g_tf32(PF(dh2), H, T, H, L->B_o, r, m.s, PF(Bt32), P(g_o), PF(go32), ldT, st));
+  if (on) SOUP_TRY(lora_g_tf32(PF(dh2), H, T, H, L->B_o, r, m.s, PF(Bt32), P(g_o), PF(go32), ldT, st, SW));
   // dO for the attention backward: from the fp32-accurate dh2 (hi + lo parts),
   // stored fp16 scaled by a power of two derived from max |dh2|
   SOUP_TRY(proj_bwd(&W->o, P(dh2_b), T, P(g_o), ldT, r, on ? L->A_o : nullptr, on, P(d_attn), st, OUT_F16, 0,
                     nullptr, gamax, P(dh2_lo)));
   if (on) {
-    SOUP_TRY(lora_dB_tf32(PF(dh2), H, T, H, PF(uo32), r, ldT, G->dB_o, st));
-    SOUP_TRY(lora_dA_tf32(PF(attn32), T, m.o_in, PF(go32), r, ldT, G->dA_o, st));
+    SOUP_TRY(lora_dB_tf32(PF(dh2), H, T, H, PF(uo32), r, ldT, G->dB_o, st, SW));
+    SOUP_TRY(lora_dA_tf32(PF(attn32), T, m.o_in, PF(go32), r, ldT, G->dA_o, st, SW));
   }
   SOUP_TRY(attn_rowdot(P(d_attn), P(attn16), T, m.Hq, PF(D), st));
   // dq and dk leave the attention backward already rotated back (inverse RoPE in its epilogues)
@@ -479,14 +564,14 @@ extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const
   if (on) {
     for (int sg = 0; sg < 3; ++sg)
       SOUP_TRY(lora_g_tf32(PF(dqkv32) + seg_c[sg], m.qkv_w, T, seg_n[sg], L->B_qkv + (size_t)seg_c[sg] * r, r, m.s,
-                           PF(Bt32), P(g_qkv) + (size_t)sg * r * ldT, PF(g32) + (size_t)sg * r * ldT, ldT, st));
+                           PF(Bt32), P(g_qkv) + (size_t)sg * r * ldT, PF(g32) + (size_t)sg * r * ldT, ldT, st, SW));
   }
   SOUP_TRY(proj_bwd(&W->qkv, P(d_qkv), T, P(g_qkv), ldT, 3 * r, on ? L->A_qkv : nullptr, on, P(dx1), st));
   if (on) {
     for (int sg = 0; sg < 3; ++sg)
       SOUP_TRY(lora_dB_tf32(PF(dqkv32) + seg_c[sg], m.qkv_w, T, seg_n[sg], PF(u32) + (size_t)sg * r * ldT, r, ldT,
-                            G->dB_qkv + (size_t)seg_c[sg] * r, st));
-    SOUP_TRY(lora_dA_tf32(PF(x1_32), T, H, PF(g32), 3 * r, ldT, G->dA_qkv, st));
+                            G->dB_qkv + (size_t)seg_c[sg] * r, st, SW));
+    SOUP_TRY(lora_dA_tf32(PF(x1_32), T, H, PF(g32), 3 * r, ldT, G->dA_qkv, st, SW));
   }
   SOUP_TRY(rmsnorm_bwd(h_in, nullptr, W->norm1, PF(rinv1), P(dx1), PF(dh2), T, H, dh_in, nullptr, st));
   return SOUP_OK;

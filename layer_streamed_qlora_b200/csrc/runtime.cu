@@ -27,6 +27,7 @@ struct ProfRec {
   double flops, bytes;
 };
 bool g_prof = false;
+int g_prof_mask = 0;
 std::vector<ProfRec> g_prof_recs;
 size_t g_prof_used = 0;
 int g_prof_open = -1;
@@ -74,7 +75,7 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 bool profiling() { return g_prof; }
 
 void profile_begin(cudaStream_t st, int cls, double flops, double bytes) {
-  if (!g_prof) return;
+  if (!g_prof || !(g_prof_mask & (1 << cls))) return;
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_prof_used == g_prof_recs.size()) {
     ProfRec r;
@@ -125,9 +126,10 @@ extern "C" soup_status soup_device_error(int32_t* code_out) {
 
 extern "C" int64_t soup_launch_count(void) { return g_launches.load(); }
 
-extern "C" soup_status soup_profile_enable(int32_t on) {
+extern "C" soup_status soup_profile_enable(int32_t class_mask) {
   std::lock_guard<std::mutex> lk(g_mu);
-  g_prof = on != 0;
+  g_prof = class_mask != 0;
+  g_prof_mask = class_mask;
   g_prof_used = 0;
   g_prof_open = -1;
   return SOUP_OK;
