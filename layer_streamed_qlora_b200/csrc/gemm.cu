@@ -286,13 +286,14 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
   }
   if (NF4 && threadIdx.x >= 64) {
     if constexpr (CG == 2) {
+      // entry b of every lane: (c[b >> 4], c[b & 15]); b is warp-uniform
       float2* lut2 = reinterpret_cast<float2*>(smem_raw);
       for (int i = threadIdx.x - 64; i < 256 * 32; i += 256) {
         const int b = i >> 5;
-        lut2[i] = make_float2(__uint_as_float(nf4_code_bits(b >> 4)), __uint_as_float(nf4_code_bits(b & 15)));
+        lut2[i] = make_float2(__uint_as_float(c_nf4_bits[b >> 4]), __uint_as_float(c_nf4_bits[b & 15]));
       }
     } else {
-      for (int i = threadIdx.x - 64; i < 16 * 32; i += 256) lut[i] = __uint_as_float(nf4_code_bits(i >> 5));
+      for (int i = threadIdx.x - 64; i < 16 * 32; i += 256) lut[i] = __uint_as_float(c_nf4_bits[i >> 5]);
     }
   }
   if (warp == 1) {
@@ -324,6 +325,17 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     // transaction bytes of both land on the even CTA's full barrier.
     if (lane == 0) {
       const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(full), 0);
+      for (int ip = 0; ip < 12 && ip < num_kb; ++ip) {  // warm L2 with the first stages' codes
+        if (!B_MN) {
+          const int r0 = paired ? (rank == 0 ? nb : args.pair_off + nb) : n0 + (int)rank * 128;
+          ptx::tma_prefetch_l2_2d(&tmB, ip * 32, r0);
+          if ((ip & 3) == 0) ptx::tma_prefetch_l2_2d(&tmA2, ip, r0);
+        } else {
+          const int c0 = n0 + (int)rank * 128;
+          ptx::tma_prefetch_l2_2d(&tmB, c0 / 2, ip * BK);
+          ptx::tma_prefetch_l2_2d(&tmA2, (c0 / 64) & ~3, ip * BK);
+        }
+      }
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -341,18 +353,30 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
         if (!tail) {
           ptx::tma_load_2d_pair(a, &tmA, bar, it * BKE, m0);
           // this CTA's codes and absmax for the stage (tmB: codes bytes,
-          // tmA2: absmax fp32; boxes out of range read as zeros)
+          // tmA2: absmax fp32; boxes out of range read as zeros), and an L2
+          // prefetch of those of stage it + PF, so that a slot refill, issued
+          // only when the slot frees, waits for L2 rather than DRAM
           uint8_t* c = sC + s * C::C_STAGE;
           uint8_t* sc = sS + s * C::S_STAGE;
+          constexpr int PF = 12;
+          const int ip = it + PF;
           ptx::mbar_arrive_expect_tx(&cfull[s], (uint32_t)(C::C_STAGE + (B_MN ? 1024 : 2048)));
           if (!B_MN) {
             const int r0 = paired ? (rank == 0 ? nb : args.pair_off + nb) : n0 + (int)rank * 128;
             ptx::tma_load_2d(c, &tmB, &cfull[s], it * 32, r0);
             ptx::tma_load_2d(sc, &tmA2, &cfull[s], it & ~3, r0);
+            if (ip < num_kb) {
+              ptx::tma_prefetch_l2_2d(&tmB, ip * 32, r0);
+              if ((ip & 3) == 0) ptx::tma_prefetch_l2_2d(&tmA2, ip, r0);
+            }
           } else {
             const int c0 = n0 + (int)rank * 128;
             ptx::tma_load_2d(c, &tmB, &cfull[s], c0 / 2, it * BK);
             ptx::tma_load_2d(sc, &tmA2, &cfull[s], (c0 / 64) & ~3, it * BK);
+            if (ip < num_kb) {
+              ptx::tma_prefetch_l2_2d(&tmB, c0 / 2, ip * BK);
+              ptx::tma_prefetch_l2_2d(&tmA2, (c0 / 64) & ~3, ip * BK);
+            }
           }
         } else {
           ptx::tma_load_2d_pair(a, &tmTA, bar, m0, tail_row);
