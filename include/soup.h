@@ -285,8 +285,10 @@ soup_status soup_stream_plan_free(soup_plan* plan);
 /* Enqueues the copy of `item` (a layer index, SOUP_ITEM_EMBED or
  * SOUP_ITEM_HEAD) into a free slot on the plan's copy stream; the copy first
  * waits (on the device) until the compute stream released the slot's
- * previous item.  Refuses when every slot of the kind holds an unreleased
- * item or the item is already held. */
+ * previous item.  Copies of 8 MiB or more are split in two halves, the
+ * second on a second copy stream (a second DMA engine), joined back before
+ * the item is marked ready.  Refuses when every slot of the kind holds an
+ * unreleased item or the item is already held. */
 soup_status soup_stream_prefetch(soup_plan* plan, int32_t item);
 
 /* Makes `compute_stream` wait (on the device) until the item's copy is done

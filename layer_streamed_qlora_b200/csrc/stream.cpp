@@ -29,6 +29,12 @@ struct soup_plan {
   char* arena = nullptr;      // n_buffers * layer_bytes + vocab_bytes
   size_t arena_bytes = 0;
   cudaStream_t copy = nullptr;
+  // A second copy stream takes half of every large copy: on some hosts one
+  // DMA engine moves ~35 GB/s over PCIe Gen5 while two together reach the
+  // link's ~55 GB/s.  fork/join order it after `copy`'s waits and before
+  // the slot's ready event.
+  cudaStream_t copy2 = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
   struct Slot {
     char* dev = nullptr;
     size_t bytes = 0;
@@ -113,6 +119,11 @@ extern "C" soup_status soup_stream_plan(const soup_stream_desc* d, soup_plan** o
   p->arena_bytes = arena;
   e = cudaStreamCreateWithFlags(&p->copy, cudaStreamNonBlocking);
   if (e != cudaSuccess) return cleanup(fail(SOUP_ERR_CUDA, "soup_stream_plan: copy stream: %s", cudaGetErrorString(e)));
+  e = cudaStreamCreateWithFlags(&p->copy2, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cleanup(fail(SOUP_ERR_CUDA, "soup_stream_plan: copy stream: %s", cudaGetErrorString(e)));
+  if (cudaEventCreateWithFlags(&p->fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&p->join, cudaEventDisableTiming) != cudaSuccess)
+    return cleanup(fail(SOUP_ERR_CUDA, "soup_stream_plan: event creation failed"));
   p->slots.resize(p->n_buffers + 1);
   for (int s = 0; s <= p->n_buffers; ++s) {
     auto& sl = p->slots[s];
@@ -129,6 +140,9 @@ extern "C" soup_status soup_stream_plan(const soup_stream_desc* d, soup_plan** o
 extern "C" soup_status soup_stream_plan_free(soup_plan* p) {
   if (!p) return SOUP_OK;
   if (p->copy) cudaStreamSynchronize(p->copy);
+  if (p->copy2) cudaStreamSynchronize(p->copy2);
+  if (p->fork) cudaEventDestroy(p->fork);
+  if (p->join) cudaEventDestroy(p->join);
   for (auto& sl : p->slots) {
     if (sl.ready) cudaEventDestroy(sl.ready);
     if (sl.free_) cudaEventDestroy(sl.free_);
@@ -142,6 +156,7 @@ extern "C" soup_status soup_stream_plan_free(soup_plan* p) {
     cudaEventDestroy(pr.second);
   }
   if (p->copy) cudaStreamDestroy(p->copy);
+  if (p->copy2) cudaStreamDestroy(p->copy2);
   if (p->arena) cudaFree(p->arena);
   delete p;
   return SOUP_OK;
@@ -192,7 +207,19 @@ extern "C" soup_status soup_stream_prefetch(soup_plan* p, int32_t item) {
   }
   auto& ce = p->copy_events[p->copy_used++];
   SOUP_CUDA_TRY(cudaEventRecord(ce.first, p->copy));
-  SOUP_CUDA_TRY(cudaMemcpyAsync(sl.dev, src, bytes, cudaMemcpyHostToDevice, p->copy));
+  if (bytes >= (8u << 20)) {
+    // second half on the second copy stream, after the same waits
+    const size_t half = (bytes / 2) & ~(size_t)255;
+    SOUP_CUDA_TRY(cudaEventRecord(p->fork, p->copy));
+    SOUP_CUDA_TRY(cudaStreamWaitEvent(p->copy2, p->fork, 0));
+    SOUP_CUDA_TRY(cudaMemcpyAsync(sl.dev, src, half, cudaMemcpyHostToDevice, p->copy));
+    SOUP_CUDA_TRY(cudaMemcpyAsync(sl.dev + half, static_cast<const char*>(src) + half, bytes - half,
+                                  cudaMemcpyHostToDevice, p->copy2));
+    SOUP_CUDA_TRY(cudaEventRecord(p->join, p->copy2));
+    SOUP_CUDA_TRY(cudaStreamWaitEvent(p->copy, p->join, 0));
+  } else {
+    SOUP_CUDA_TRY(cudaMemcpyAsync(sl.dev, src, bytes, cudaMemcpyHostToDevice, p->copy));
+  }
   SOUP_CUDA_TRY(cudaEventRecord(sl.ready, p->copy));
   SOUP_CUDA_TRY(cudaEventRecord(ce.second, p->copy));
   sl.item = item;
