@@ -66,19 +66,24 @@ def peaks():
 
 
 def gemm_traffic():
-    """Per-launch DRAM bytes of the dominant kernel from a committed ncu
-    summary, if it was taken on the current GEMM source (else None)."""
-    p = os.path.join(ROOT, "profiles", "gemm_nf4_traffic.json")
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summary (lines "key: value"), if it was taken on the current GEMM source
+    (else None)."""
+    p = os.path.join(ROOT, "profiles", "gemm_nf4_fwd_traffic.md")
     src = os.path.join(ROOT, "layer_streamed_qlora_b200", "csrc", "gemm.cu")
     if not os.path.exists(p):
         return None
+    d = {}
     with open(p) as f:
-        d = json.load(f)
+        for line in f:
+            k, sep, v = line.strip().lstrip("-* ").partition(": ")
+            if sep and k in ("gemm_cu_sha256", "bytes_per_launch"):
+                d[k] = v.strip().strip("`")
     with open(src, "rb") as f:
         h = hashlib.sha256(f.read()).hexdigest()
-    if d.get("gemm_cu_sha256") != h:
+    if d.get("gemm_cu_sha256") != h or "bytes_per_launch" not in d:
         return None
-    return d
+    return {"bytes_per_launch": float(d["bytes_per_launch"])}
 
 
 class ClockSampler:
@@ -200,6 +205,49 @@ def run_reference(args, w, name):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+# Launch mix of the forward fused NF4 GEMM per layer and step: the forward
+# pass runs q|k|v, o, gate|up and down; the recompute runs o and gate|up
+# again (its q|k|v GEMM takes a hi + lo A pair: another kernel).
+PROBE_WEIGHTS = {"qkv": 1, "o": 2, "gate_up": 2, "down": 1}
+
+
+def probe_shapes(w):
+    H, I = w["hidden"], w["intermediate"]
+    qkv = (w["n_q_heads"] + 2 * w["n_kv_heads"]) * w["head_dim"]
+    return {"qkv": (qkv, H), "o": (H, w["n_q_heads"] * w["head_dim"]), "gate_up": (2 * I, H), "down": (H, I)}
+
+
+def run_probe_gemm(w):
+    """One forward fused NF4 GEMM per projection shape of the workload's layer
+    at its token count (random NF4 weights, LoRA r), each after one warm-up
+    launch, in the order of PROBE_WEIGHTS: an ncu capture of the fused GEMM
+    kernel with -s 1 -c 1 per shape (or -c 8 for all) reads DRAM traffic per launch."""
+    import torch
+
+    from layer_streamed_qlora_b200 import _lib as L
+    T, r = w["batch"] * w["seq"], w["rank"]
+    g = torch.Generator(device="cuda").manual_seed(7)
+    for name, (N, K) in probe_shapes(w).items():
+        W = torch.randn(N, K, device="cuda", generator=g) * 0.02
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+        absmax = torch.empty((N, K // 64), dtype=torch.float32, device="cuda")
+        flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+        L.soup_nf4_quantize(W, codes, absmax, flag)
+        del W
+        wt = L.weight_nf4(codes, absmax, N, K)
+        x = torch.randn(T, K, device="cuda", generator=g).bfloat16()
+        A = (torch.randn(r, K, device="cuda", generator=g) * 0.02).bfloat16()
+        Bm = (torch.randn(N, r, device="cuda", generator=g) * 0.02).bfloat16()
+        y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+        u = torch.empty(r, T, dtype=torch.bfloat16, device="cuda")
+        for _ in range(2):
+            L.soup_lora_linear_fwd(wt, A, Bm, r, w["alpha"] / r, x, T, y, u)
+        torch.cuda.synchronize()
+        print(f"probe {name}: N={N} K={K} T={T}", flush=True)
+    print(json.dumps({"probe": "fused NF4 forward GEMMs", "weights": PROBE_WEIGHTS}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -210,6 +258,8 @@ def main():
     ap.add_argument("--buffers", type=int, default=0, help="override stream_buffers (2..8)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (diagnostics only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--probe-gemm", action="store_true",
+                    help="run each forward fused NF4 GEMM shape of one layer twice and exit (for an ncu capture)")
     args = ap.parse_args()
     w = dict(WORKLOADS[args.workload])
     if args.buffers:
@@ -218,6 +268,8 @@ def main():
         w["n_layers"] = args.layers
     if args.impl == "reference":
         return run_reference(args, w, args.workload)
+    if args.probe_gemm:
+        return run_probe_gemm(w)
 
     import torch
     import torch.distributed as dist
@@ -269,13 +321,17 @@ def main():
     torch.cuda.reset_peak_memory_stats()
     clocks = ClockSampler(local)
     clocks.start()
-    L.profile_enable(0b0011)  # event-time only the dominant kernel (the fused NF4 GEMMs) in the timed region
+    L.profile_enable(0b00001)  # event-time only the dominant kernel (the fused NF4 forward GEMM) in the timed region
     n0 = L.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e0.record(st)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        if i == 0:  # NVTX range: lets an ncu launch list capture exactly one step
+            torch.cuda.nvtx.range_push("soup_step")
         step()
+        if i == 0:
+            torch.cuda.nvtx.range_pop()
     e1.record(st)
     torch.cuda.synchronize()
     if world > 1:
@@ -287,7 +343,7 @@ def main():
     sstats = model.plan.stats()
     clk = clocks.stop()
     # per-class breakdown of every GEMM from one extra, separately profiled step
-    L.profile_enable(0b1111)
+    L.profile_enable(0b11111)
     step()
     torch.cuda.synchronize()
     prof_all = L.profile_read()

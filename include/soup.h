@@ -63,7 +63,8 @@ int64_t soup_launch_count(void);
  * soup_profile_read synchronises those events and sums them per class:
  * 0 = fused NF4-decode GEMM (forward, W), 1 = fused NF4-decode GEMM
  * (backward, W^T), 2 = other GEMMs with N > 64, 3 = skinny LoRA GEMMs
- * (N <= 64).  Enabling resets the records; class_mask 0 disables. */
+ * (N <= 64), 4 = fused NF4-decode GEMMs with a hi + lo A pair (either
+ * direction).  Enabling resets the records; class_mask 0 disables. */
 typedef struct soup_gemm_profile {
   int64_t launches;
   double total_ms;

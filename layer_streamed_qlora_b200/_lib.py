@@ -70,7 +70,7 @@ class GemmProfile(ctypes.Structure):
                 ("bytes", ctypes.c_double)]
 
 
-GEMM_CLASSES = ("nf4_fwd", "nf4_bwd", "bf16", "lora_skinny")
+GEMM_CLASSES = ("nf4_fwd", "nf4_bwd", "bf16", "lora_skinny", "nf4_dual")
 
 SOUP_ITEM_EMBED = -1
 SOUP_ITEM_HEAD = -2

@@ -1030,7 +1030,8 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
   if (profiling()) {
     // algorithmic work: 2 M N K (+ 2 M N r for the LoRA tail); bytes: the
     // operands read once and the output written once
-    const int cls = BMD == B_NF4_K ? GC_NF4_FWD : (BMD == B_NF4_MN ? GC_NF4_BWD : (d.N <= 64 ? GC_SKINNY : GC_BF16));
+    const int cls = (DUAL && BMD >= B_NF4_K) ? GC_NF4_DUAL
+                    : BMD == B_NF4_K ? GC_NF4_FWD : (BMD == B_NF4_MN ? GC_NF4_BWD : (d.N <= 64 ? GC_SKINNY : GC_BF16));
     const double tail_k = d.tail_ksteps > 0 ? (double)d.tailA.rows : 0.0;
     const double flops = 2.0 * d.M * d.N * ((double)d.K * (DUAL ? 2 : 1) + (paired ? 16.0 : tail_k));
     const double wbytes = (BMD >= B_NF4_K) ? (double)d.N * d.K * (0.5 + 4.0 / 64) : (double)d.N * d.K * 2;

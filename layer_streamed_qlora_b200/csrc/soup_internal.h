@@ -34,7 +34,7 @@ void count_launch();
 
 // Optional CUDA-event timing of GEMM launches, by class, on the launching
 // stream (enabled through soup_profile_enable).
-enum GemmClass : int { GC_NF4_FWD = 0, GC_NF4_BWD = 1, GC_BF16 = 2, GC_SKINNY = 3, GC_N = 4 };
+enum GemmClass : int { GC_NF4_FWD = 0, GC_NF4_BWD = 1, GC_BF16 = 2, GC_SKINNY = 3, GC_NF4_DUAL = 4, GC_N = 5 };
 bool profiling();
 void profile_begin(cudaStream_t st, int cls, double flops, double bytes);
 void profile_end(cudaStream_t st);
