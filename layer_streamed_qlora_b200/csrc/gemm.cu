@@ -54,9 +54,11 @@ struct Cfg {
   static constexpr int S_STAGE = CG == 2 ? 2048 : 0;
   static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   static constexpr int BAR_BYTES = 256;
-  // CTA pairs: byte-indexed NF4 table (256 code pairs x 32 lanes x float2)
-  // at the start of shared memory; single CTAs: nibble table after the barriers
-  static constexpr int LUT_BYTES = CG == 2 ? 65536 : 16 * 32 * 4;
+  // CTA pairs: byte-indexed NF4 table (256 code pairs x 32 lanes x float2;
+  // x 16 half-warp lanes when two A tiles per stage leave no room) at the
+  // start of shared memory; single CTAs: nibble table after the barriers
+  static constexpr int LUT_LANES = DUAL ? 16 : 32;
+  static constexpr int LUT_BYTES = CG == 2 ? 256 * LUT_LANES * 8 : 16 * 32 * 4;
   static constexpr int STAGE_BYTES = A_STAGE + B_STAGE + C_STAGE + S_STAGE;
   static constexpr int STAGE_BUDGET = CG == 2 ? (232448 - 1024 - BAR_BYTES - LUT_BYTES) : 196608;
   static constexpr int STAGES = (STAGE_BUDGET / STAGE_BYTES) > 8 ? 8 : (STAGE_BUDGET / STAGE_BYTES);
@@ -171,15 +173,20 @@ __device__ __forceinline__ uint4 decode8(uint32_t w, const float* lut_lane, floa
 }
 
 // Same result from the byte-indexed table of the pair kernels: entry b of
-// lane l (byte offset b*256 + l*8) holds the codebook values of the two
-// codes packed in byte b (high nibble first); one byte permute forms the
-// offset, one 8-byte shared load fetches both values, one packed multiply
-// scales them, and the products are rounded exactly as above.
-__device__ __forceinline__ uint4 decode8_pairs(uint32_t w, const uint8_t* lut_bytes, uint32_t lane8, float am) {
+// lane l holds the codebook values of the two codes packed in byte b (high
+// nibble first), at byte offset b*256 + l*8 (LANES = 32; lane_b = l*8) or, in
+// the half-size table, b*128 + (l % 16)*8 (LANES = 16; lane_b = (l % 16)*16,
+// the offset halved after the permute), so that the lanes reading one 8-byte
+// wavefront hit distinct banks.  One byte permute forms the offset, one
+// 8-byte shared load fetches both values, one packed multiply scales them,
+// and the products are rounded exactly as above.
+template <int LANES>
+__device__ __forceinline__ uint4 decode8_pairs(uint32_t w, const uint8_t* lut_bytes, uint32_t lane_b, float am) {
   uint32_t o[4];
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
-    const uint32_t off = __byte_perm(w, lane8, 0x5504u | ((uint32_t)p << 4));
+    uint32_t off = __byte_perm(w, lane_b, 0x5504u | ((uint32_t)p << 4));
+    if (LANES == 16) off >>= 1;
     const float2 c = *reinterpret_cast<const float2*>(lut_bytes + off);
     const float2 f = ptx::mul_f32x2(c, am);
     o[p] = pack_bf16x2(f.x, f.y);
@@ -214,10 +221,11 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmTA,
                 const __grid_constant__ CUtensorMap tmTB, const __grid_constant__ CUtensorMap tmA2,
+                const __grid_constant__ CUtensorMap tmA3,
                 const KArgs args) {
   using C = Cfg<BN, DUAL, CG>;
   static_assert(!DUAL || (AMJ == A_K && !TF), "dual-A: K-major bf16 A only");
-  static_assert(CG == 1 || (BN == 256 && AMJ == A_K && BMD >= B_NF4_K && !TF && !DUAL),
+  static_assert(CG == 1 || (BN == 256 && AMJ == A_K && BMD >= B_NF4_K && !TF),
                 "CTA pairs: NF4 B, K-major bf16 A, 256-wide tiles");
   constexpr bool NF4 = BMD >= B_NF4_K;
   constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
@@ -278,6 +286,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmA);
     if (DUAL || CG == 2) ptx::prefetch_tmap(&tmA2);
+    if (DUAL && CG == 2) ptx::prefetch_tmap(&tmA3);
     if (!NF4 || CG == 2) ptx::prefetch_tmap(&tmB);
     if (args.tail_ksteps > 0) {
       ptx::prefetch_tmap(&tmTA);
@@ -286,10 +295,10 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
   }
   if (NF4 && threadIdx.x >= 64) {
     if constexpr (CG == 2) {
-      // entry b of every lane: (c[b >> 4], c[b & 15]); b is warp-uniform
+      // entry b of every lane: (c[b >> 4], c[b & 15])
       float2* lut2 = reinterpret_cast<float2*>(smem_raw);
-      for (int i = threadIdx.x - 64; i < 256 * 32; i += 256) {
-        const int b = i >> 5;
+      for (int i = threadIdx.x - 64; i < 256 * C::LUT_LANES; i += 256) {
+        const int b = i / C::LUT_LANES;
         lut2[i] = make_float2(__uint_as_float(c_nf4_bits[b >> 4]), __uint_as_float(c_nf4_bits[b & 15]));
       }
     } else {
@@ -347,11 +356,13 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
         uint8_t* a = sA + s * C::A_STAGE;
         uint8_t* b = sB + s * C::B_STAGE;
         const bool tail = it >= num_kb;
-        const uint32_t bytes = tail ? (uint32_t)(A_STAGE_BYTES + C::B_STAGE) : (uint32_t)A_STAGE_BYTES;
+        const uint32_t bytes = tail ? (uint32_t)(A_STAGE_BYTES + C::B_STAGE) : (uint32_t)C::A_STAGE;
         if (rank == 0) ptx::mbar_arrive_expect_tx(&full[s], 2 * bytes);
         const uint32_t bar = full0 + s * 8;
         if (!tail) {
           ptx::tma_load_2d_pair(a, &tmA, bar, it * BKE, m0);
+          // hi + lo A pair: the rounding residual tile (tmA3) beside it
+          if (DUAL) ptx::tma_load_2d_pair(a + A_STAGE_BYTES, &tmA3, bar, it * BKE, m0);
           // this CTA's codes and absmax for the stage (tmB: codes bytes,
           // tmA2: absmax fp32; boxes out of range read as zeros), and an L2
           // prefetch of those of stage it + PF, so that a slot refill, issued
@@ -430,6 +441,9 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
             const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k * KSTEP_MN, CHUNK_BYTES, 1024)
                                      : ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
             ptx::mma_bf16_pair(tmem, ad, bd, tail ? idesc_tail : idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+            if (DUAL && !tail)  // lo part of A against the same B tile
+              ptx::mma_bf16_pair(tmem, ptx::smem_desc_sw128(a_base + A_STAGE_BYTES + k * 32, 16, 1024), bd, idesc_main,
+                                 1u);
           }
         }
         ptx::mma_commit_pair(&empty[s], 3);
@@ -559,7 +573,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
       // per stage (one absmax), codes of stage it+1 prefetched in registers.
       // Arrivals go to the even CTA's full barrier.
       const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(full), 0);
-      const uint32_t lane8 = (uint32_t)lane * 8u;
+      const uint32_t lane_b = C::LUT_LANES == 32 ? (uint32_t)lane * 8u : (uint32_t)(lane & 15) * 16u;
       const uint8_t* lutb = smem_raw;
       // thread -> (shared row of the B stage, first 16-byte unit, chunk),
       // its 16 code bytes within the staged codes tile, and its absmax
@@ -607,7 +621,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
           const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const uint4 v = valid ? decode8_pairs(ws[u], lutb, lane8, am) : make_uint4(0, 0, 0, 0);
+            const uint4 v = valid ? decode8_pairs<C::LUT_LANES>(ws[u], lutb, lane_b, am) : make_uint4(0, 0, 0, 0);
             st_shared_v4(b + (((unit0 + u) ^ (srow & 7)) << 4), v);
           }
           ptx::fence_proxy_async_smem();
@@ -985,9 +999,10 @@ constexpr int CU_DT_U8 = 0;  // CU_TENSOR_MAP_DATA_TYPE_UINT8
 template <int BN, int AMJ, int BMD, bool TF = false, bool DUAL = false, int CG = 1>
 soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
   using C = Cfg<BN, DUAL, CG>;
-  CUtensorMap mA, mB, mTA, mTB, mA2;
+  CUtensorMap mA, mB, mTA, mTB, mA2, mA3;
   memset(&mA2, 0, sizeof(mA2));
-  if (DUAL) SOUP_TRY(make_map(&mA2, d.A_lo, 64, 128, "A (lo part)"));
+  memset(&mA3, 0, sizeof(mA3));
+  if (DUAL) SOUP_TRY(make_map(CG == 2 ? &mA3 : &mA2, d.A_lo, 64, 128, "A (lo part)"));
   memset(&mA, 0, sizeof(mA));
   memset(&mB, 0, sizeof(mB));
   memset(&mTA, 0, sizeof(mTA));
@@ -1053,9 +1068,9 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    SOUP_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, mA, mB, mTA, mTB, mA2, ka));
+    SOUP_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, mA, mB, mTA, mTB, mA2, mA3, ka));
   } else {
-    kern<<<grid, NT, C::SMEM, st>>>(mA, mB, mTA, mTB, mA2, ka);
+    kern<<<grid, NT, C::SMEM, st>>>(mA, mB, mTA, mTB, mA2, mA3, ka);
   }
   SOUP_LAUNCH_CHECK();
   profile_end(st);
@@ -1091,7 +1106,14 @@ soup_status dispatch(const GemmDesc& d, const KArgs& ka, int bn, cudaStream_t st
 #undef SOUP_GEMM_TF
     return fail(SOUP_ERR_SHAPE, "gemm: no tf32 kernel for BN=%d", bn);
   }
+  // NF4 B with 256-wide tiles: CTA pairs (half the decode per CTA)
+  const bool pair_ok = nf4 && bn == 256 && d.a_major == A_K && soup_aligned(d.absmax, 16) &&
+                       (d.b_mode == B_NF4_K ? d.K % 256 == 0 : d.N % 256 == 0);
   if (d.A_lo.ptr) {
+    if (pair_ok && d.A_lo.rows == d.A.rows && d.A_lo.cols == d.A.cols) {
+      if (d.b_mode == B_NF4_K) return launch<256, A_K, B_NF4_K, false, true, 2>(d, ka, st);
+      return launch<256, A_K, B_NF4_MN, false, true, 2>(d, ka, st);
+    }
     SOUP_CHECK(d.a_major == A_K && !d.tf32 && (bn == 256 || bn == 128 || (bn <= 32 && d.b_mode == B_TMA_K)) &&
                    d.A_lo.rows == d.A.rows &&
                    d.A_lo.cols == d.A.cols,
@@ -1106,9 +1128,6 @@ soup_status dispatch(const GemmDesc& d, const KArgs& ka, int bn, cudaStream_t st
 #undef SOUP_GEMM_DUAL
     return fail(SOUP_ERR_SHAPE, "gemm: no dual-A kernel for BN=%d b_mode=%d", bn, d.b_mode);
   }
-  // NF4 B with 256-wide tiles: CTA pairs (half the decode per CTA)
-  const bool pair_ok = nf4 && bn == 256 && d.a_major == A_K && soup_aligned(d.absmax, 16) &&
-                       (d.b_mode == B_NF4_K ? d.K % 256 == 0 : d.N % 256 == 0);
   if (pair_ok) {
     if (d.b_mode == B_NF4_K) return launch<256, A_K, B_NF4_K, false, false, 2>(d, ka, st);
     return launch<256, A_K, B_NF4_MN, false, false, 2>(d, ka, st);
