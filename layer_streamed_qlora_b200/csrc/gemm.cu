@@ -216,6 +216,176 @@ __device__ __forceinline__ void load_codes(const uint8_t* src, uint32_t (&w)[NWO
   }
 }
 
+// Epilogue of one accumulator tile: the warp owns TMEM lanes 32q..32q+31
+// (output rows m0 + 32q + lane) of the accumulator at column `tacc`, and its
+// 16-column chunks ch0, ch0 + chs, ...
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uint32_t tacc, int m0, int n0, int nb,
+                                              int q, int lane, int ch0, int chs) {
+  const uint32_t trow = tacc + ((uint32_t)(q * 32) << 16);
+  const int row = m0 + q * 32 + lane;
+  const bool row_ok = row < args.M;
+  constexpr int NCH = BN / 16;
+  const float alpha =
+      args.scale_amax ? args.alpha * grad_scale_from_amax(__uint_as_float(*args.scale_amax)) : args.alpha;
+  const bool vec = args.vec_ok != 0;
+  if (args.epi == EPI_SWIGLU) {
+    // paired gate|up tile: chunk c (gate) pairs with c + NCH/2 (up); both
+    // owned by this warp (NCH/2 is even)
+    const int I = args.swiglu_I;
+    for (int ch = ch0; ch < NCH / 2; ch += chs) {
+      uint32_t vg[16], vu[16];
+      ptx::tmem_ld16(trow + ch * 16, vg);
+      ptx::tmem_ld16(trow + (ch + NCH / 2) * 16, vu);
+      ptx::tmem_ld_wait();
+      const int n = nb + ch * 16;
+      if (!row_ok || n >= I) continue;
+      float a[16], gg[16], uu[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        gg[i] = __uint_as_float(vg[i]) * alpha;
+        uu[i] = __uint_as_float(vu[i]) * alpha;
+        a[i] = gg[i] * sigmoid_f(gg[i]) * uu[i];
+      }
+      store_row16(outp, OUT_BF16, args.ldo, row, n, I, a, vec);
+      if (args.aux16) {
+        store_row16(args.aux16, OUT_F16, args.ld_aux, row, n, I, gg, vec);
+        store_row16(args.aux16 + I, OUT_F16, args.ld_aux, row, n, I, uu, vec);
+      }
+    }
+  } else if ((BN >= 128) && args.rope_cols > 0 && n0 < args.rope_cols) {
+    // RoPE (q/k heads of the fused QKV projection): the pair (i, i + 64)
+    // of a 128-wide head lives in chunks c and c + 4 of the head, which
+    // the same warp owns; rotate the fp32 accumulators, then round once.
+    for (int ch = ch0; ch < NCH; ch += chs) {
+      if ((ch & 7) >= 4) continue;
+      uint32_t v0[16], v1[16];
+      ptx::tmem_ld16(trow + ch * 16, v0);
+      ptx::tmem_ld16(trow + (ch + 4) * 16, v1);
+      ptx::tmem_ld_wait();
+      const int n = n0 + ch * 16;
+      if (!row_ok || n >= args.N) continue;
+      const int pos = row % args.rope_S;
+      const float* cs = args.rope_cos + (size_t)pos * 64 + (ch & 7) * 16;
+      const float* sn = args.rope_sin + (size_t)pos * 64 + (ch & 7) * 16;
+      float a[16], b[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float x0 = __uint_as_float(v0[i]) * alpha, x1 = __uint_as_float(v1[i]) * alpha;
+        const float c = __ldg(cs + i), sv = __ldg(sn + i);
+        a[i] = x0 * c - x1 * sv;
+        b[i] = x1 * c + x0 * sv;
+      }
+      store_row16(outp, args.out_kind, args.ldo, row, n, args.N, a, vec);
+      store_row16(outp, args.out_kind, args.ldo, row, n + 64, args.N, b, vec);
+    }
+  } else {
+    for (int ch = ch0; ch < NCH; ch += chs) {
+      uint32_t v[16];
+      ptx::tmem_ld16(trow + ch * 16, v);
+      ptx::tmem_ld_wait();
+      const int n = n0 + ch * 16;
+      if (!row_ok || n >= args.N) continue;
+      float f[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * alpha;
+      const bool full16 = vec && (n + 16 <= args.N);
+      if (args.epi == EPI_SWIGLU_BWD) {
+        // f = dL/d(act); g, u from the forward (fp16); out = [dL/dg | dL/du] bf16
+        const int I = args.swiglu_I;
+        uint16_t gb[16], ub[16];
+        const uint16_t* gp = args.aux16 + (size_t)row * args.ld_aux + n;
+        if (full16) {
+          load16_u16(gp, gb);
+          load16_u16(gp + I, ub);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            gb[i] = (n + i < args.N) ? gp[i] : 0;
+            ub[i] = (n + i < args.N) ? gp[I + i] : 0;
+          }
+        }
+        float dg[16], du[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float g = f16_to_f32(gb[i]), u = f16_to_f32(ub[i]);
+          const float sg = sigmoid_f(g);
+          dg[i] = f[i] * u * sg * (1.0f + g * (1.0f - sg));
+          du[i] = f[i] * g * sg;
+        }
+        store_row16(outp, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
+        store_row16(static_cast<uint16_t*>(outp) + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
+        if (args.out_lo) {  // rounding residuals of both halves, same layout
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            dg[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(dg[i], 0.f) & 0xFFFF));
+            du[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(du[i], 0.f) & 0xFFFF));
+          }
+          store_row16(args.out_lo, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
+          store_row16(args.out_lo + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
+        }
+        continue;
+      }
+      if (args.out_kind == OUT_BF16_T || args.out_kind == OUT_F32_T) {
+        if (args.out_kind == OUT_BF16_T) {
+          uint16_t* o = static_cast<uint16_t*>(outp);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (n + i < args.N)
+              o[(size_t)(n + i) * args.ldo + row] = static_cast<uint16_t>(pack_bf16x2(f[i], 0.f) & 0xFFFF);
+          if (args.out2) {  // the same values unrounded, fp32, same layout
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (n + i < args.N) args.out2[(size_t)(n + i) * args.ldo + row] = f[i];
+          }
+          if (args.out_lo) {  // rounding residual: hi + lo carries ~16 significant bits
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (n + i < args.N) {
+                const uint16_t hb = static_cast<uint16_t>(pack_bf16x2(f[i], 0.f) & 0xFFFF);
+                args.out_lo[(size_t)(n + i) * args.ldo + row] =
+                    static_cast<uint16_t>(pack_bf16x2(f[i] - bf16_to_f32(hb), 0.f) & 0xFFFF);
+              }
+          }
+        } else {
+          float* o = static_cast<float*>(outp);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (n + i < args.N) o[(size_t)(n + i) * args.ldo + row] = f[i];
+        }
+        continue;
+      }
+      if (args.resid) {
+        const uint16_t* r = args.resid + (size_t)row * args.ldr + n;
+        if (full16) {
+          uint16_t rb[16];
+          load16_u16(r, rb);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) f[i] += bf16_to_f32(rb[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (n + i < args.N) f[i] += bf16_to_f32(r[i]);
+        }
+      } else if (args.resid_f32) {
+        const float* r = args.resid_f32 + (size_t)row * args.ldr + n;
+        if (full16) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 x = reinterpret_cast<const float4*>(r)[i];
+            f[4 * i] += x.x; f[4 * i + 1] += x.y; f[4 * i + 2] += x.z; f[4 * i + 3] += x.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (n + i < args.N) f[i] += r[i];
+        }
+      }
+      store_row16(outp, args.out_kind, args.ldo, row, n, args.N, f, vec);
+    }
+  }
+}
+
 template <int BN, int AMJ, int BMD, bool TF, bool DUAL, int CG>
 __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -736,169 +906,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
       *abort_flag = 1;
     } else {
       ptx::tc_fence_after();
-      const int row = m0 + q * 32 + lane;
-      const bool row_ok = row < args.M;
-      constexpr int NCH = BN / 16;
-      const float alpha =
-          args.scale_amax ? args.alpha * grad_scale_from_amax(__uint_as_float(*args.scale_amax)) : args.alpha;
-      const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-      const int ch0 = NEPI == 8 ? ew / 4 : 0, chs = NEPI == 8 ? 2 : 1;
-      const bool vec = args.vec_ok != 0;
-      if (args.epi == EPI_SWIGLU) {
-        // paired gate|up tile: chunk c (gate) pairs with c + NCH/2 (up); both
-        // owned by this warp (NCH/2 is even)
-        const int I = args.swiglu_I;
-        for (int ch = ch0; ch < NCH / 2; ch += chs) {
-          uint32_t vg[16], vu[16];
-          ptx::tmem_ld16(trow + ch * 16, vg);
-          ptx::tmem_ld16(trow + (ch + NCH / 2) * 16, vu);
-          ptx::tmem_ld_wait();
-          const int n = nb + ch * 16;
-          if (!row_ok || n >= I) continue;
-          float a[16], gg[16], uu[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            gg[i] = __uint_as_float(vg[i]) * alpha;
-            uu[i] = __uint_as_float(vu[i]) * alpha;
-            a[i] = gg[i] * sigmoid_f(gg[i]) * uu[i];
-          }
-          store_row16(outp, OUT_BF16, args.ldo, row, n, I, a, vec);
-          if (args.aux16) {
-            store_row16(args.aux16, OUT_F16, args.ld_aux, row, n, I, gg, vec);
-            store_row16(args.aux16 + I, OUT_F16, args.ld_aux, row, n, I, uu, vec);
-          }
-        }
-      } else if ((BN >= 128) && args.rope_cols > 0 && n0 < args.rope_cols) {
-        // RoPE (q/k heads of the fused QKV projection): the pair (i, i + 64)
-        // of a 128-wide head lives in chunks c and c + 4 of the head, which
-        // the same warp owns; rotate the fp32 accumulators, then round once.
-        for (int ch = ch0; ch < NCH; ch += chs) {
-          if ((ch & 7) >= 4) continue;
-          uint32_t v0[16], v1[16];
-          ptx::tmem_ld16(trow + ch * 16, v0);
-          ptx::tmem_ld16(trow + (ch + 4) * 16, v1);
-          ptx::tmem_ld_wait();
-          const int n = n0 + ch * 16;
-          if (!row_ok || n >= args.N) continue;
-          const int pos = row % args.rope_S;
-          const float* cs = args.rope_cos + (size_t)pos * 64 + (ch & 7) * 16;
-          const float* sn = args.rope_sin + (size_t)pos * 64 + (ch & 7) * 16;
-          float a[16], b[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float x0 = __uint_as_float(v0[i]) * alpha, x1 = __uint_as_float(v1[i]) * alpha;
-            const float c = __ldg(cs + i), sv = __ldg(sn + i);
-            a[i] = x0 * c - x1 * sv;
-            b[i] = x1 * c + x0 * sv;
-          }
-          store_row16(outp, args.out_kind, args.ldo, row, n, args.N, a, vec);
-          store_row16(outp, args.out_kind, args.ldo, row, n + 64, args.N, b, vec);
-        }
-      } else {
-        for (int ch = ch0; ch < NCH; ch += chs) {
-          uint32_t v[16];
-          ptx::tmem_ld16(trow + ch * 16, v);
-          ptx::tmem_ld_wait();
-          const int n = n0 + ch * 16;
-          if (!row_ok || n >= args.N) continue;
-          float f[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * alpha;
-          const bool full16 = vec && (n + 16 <= args.N);
-          if (args.epi == EPI_SWIGLU_BWD) {
-            // f = dL/d(act); g, u from the forward (fp16); out = [dL/dg | dL/du] bf16
-            const int I = args.swiglu_I;
-            uint16_t gb[16], ub[16];
-            const uint16_t* gp = args.aux16 + (size_t)row * args.ld_aux + n;
-            if (full16) {
-              load16_u16(gp, gb);
-              load16_u16(gp + I, ub);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                gb[i] = (n + i < args.N) ? gp[i] : 0;
-                ub[i] = (n + i < args.N) ? gp[I + i] : 0;
-              }
-            }
-            float dg[16], du[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g = f16_to_f32(gb[i]), u = f16_to_f32(ub[i]);
-              const float sg = sigmoid_f(g);
-              dg[i] = f[i] * u * sg * (1.0f + g * (1.0f - sg));
-              du[i] = f[i] * g * sg;
-            }
-            store_row16(outp, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
-            store_row16(static_cast<uint16_t*>(outp) + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
-            if (args.out_lo) {  // rounding residuals of both halves, same layout
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                dg[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(dg[i], 0.f) & 0xFFFF));
-                du[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(du[i], 0.f) & 0xFFFF));
-              }
-              store_row16(args.out_lo, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
-              store_row16(args.out_lo + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
-            }
-            continue;
-          }
-          if (args.out_kind == OUT_BF16_T || args.out_kind == OUT_F32_T) {
-            if (args.out_kind == OUT_BF16_T) {
-              uint16_t* o = static_cast<uint16_t*>(outp);
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (n + i < args.N)
-                  o[(size_t)(n + i) * args.ldo + row] = static_cast<uint16_t>(pack_bf16x2(f[i], 0.f) & 0xFFFF);
-              if (args.out2) {  // the same values unrounded, fp32, same layout
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                  if (n + i < args.N) args.out2[(size_t)(n + i) * args.ldo + row] = f[i];
-              }
-              if (args.out_lo) {  // rounding residual: hi + lo carries ~16 significant bits
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                  if (n + i < args.N) {
-                    const uint16_t hb = static_cast<uint16_t>(pack_bf16x2(f[i], 0.f) & 0xFFFF);
-                    args.out_lo[(size_t)(n + i) * args.ldo + row] =
-                        static_cast<uint16_t>(pack_bf16x2(f[i] - bf16_to_f32(hb), 0.f) & 0xFFFF);
-                  }
-              }
-            } else {
-              float* o = static_cast<float*>(outp);
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (n + i < args.N) o[(size_t)(n + i) * args.ldo + row] = f[i];
-            }
-            continue;
-          }
-          if (args.resid) {
-            const uint16_t* r = args.resid + (size_t)row * args.ldr + n;
-            if (full16) {
-              uint16_t rb[16];
-              load16_u16(r, rb);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) f[i] += bf16_to_f32(rb[i]);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (n + i < args.N) f[i] += bf16_to_f32(r[i]);
-            }
-          } else if (args.resid_f32) {
-            const float* r = args.resid_f32 + (size_t)row * args.ldr + n;
-            if (full16) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float4 x = reinterpret_cast<const float4*>(r)[i];
-                f[4 * i] += x.x; f[4 * i + 1] += x.y; f[4 * i + 2] += x.z; f[4 * i + 3] += x.w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (n + i < args.N) f[i] += r[i];
-            }
-          }
-          store_row16(outp, args.out_kind, args.ldo, row, n, args.N, f, vec);
-        }
-      }
+      epilogue_tile<BN>(args, outp, tmem, m0, n0, nb, q, lane, NEPI == 8 ? ew / 4 : 0, NEPI == 8 ? 2 : 1);
     }
   }
 
@@ -917,6 +925,328 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     ptx::tc_fence_after();
     if constexpr (CG == 2) ptx::tmem_dealloc_pair(tmem, C::TMEM_COLS);
     else ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Persistent form of the CTA-pair NF4 GEMM: each pair loops over 256x256
+// output tiles (t = pair, pair + pairs, ...; M tiles fastest) with two
+// accumulators in tensor memory (2 x 256 columns), so that 4 epilogue warps
+// drain tile i while the MMA warp already accumulates tile i + 1.  Roles:
+// warp 0 TMA producer, warp 1 TMEM owner + MMA issuer (even CTA), warps 2..9
+// NF4 decode, warps 10..13 epilogue.  The shared-memory ring, decode, tail
+// K-block and epilogues are those of gemm_kernel with CTA pairs; the stage
+// counter runs on across tiles and the decode table is built once.
+constexpr int PERSIST_THREADS = 32 * 14;
+
+struct PairTile {
+  int m0, n0, nb, tail_row;
+};
+
+__device__ __forceinline__ PairTile pair_tile(const KArgs& args, int t, int mtiles, uint32_t rank) {
+  constexpr int BN = 256;
+  PairTile p;
+  const int mt = t % mtiles, nt = t / mtiles;
+  p.m0 = mt * 256 + (int)rank * 128;
+  const bool paired = args.pair_off > 0;
+  p.nb = paired ? nt * (BN / 2) : nt * BN;
+  p.n0 = p.nb;
+  int tr = args.seg_row[0];
+  if (args.nseg > 1 && p.n0 >= args.seg_end[0]) tr = args.seg_row[1];
+  if (args.nseg > 2 && p.n0 >= args.seg_end[1]) tr = args.seg_row[2];
+  if (args.nseg > 3 && p.n0 >= args.seg_end[2]) tr = args.seg_row[3];
+  p.tail_row = paired ? 0 : tr;
+  return p;
+}
+
+template <int BMD, bool DUAL>
+__global__ void __launch_bounds__(PERSIST_THREADS, 1)
+    gemm_pair_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmTA, const __grid_constant__ CUtensorMap tmTB,
+                         const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmA3,
+                         const KArgs args, int mtiles, int ntiles_total) {
+  constexpr int BN = 256;
+  using C = Cfg<BN, DUAL, 2>;
+  constexpr bool B_MN = BMD == B_NF4_MN;
+  constexpr int STAGES = C::STAGES;
+  constexpr int KSTEP_MN = 16 * 128;
+  constexpr int CHUNK_BYTES = 64 * 128;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw + C::LUT_BYTES) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::A_STAGE;
+  uint8_t* sC = sB + STAGES * C::B_STAGE;
+  uint8_t* sS = sC + STAGES * C::C_STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sS + STAGES * C::S_STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* cfull = empty + STAGES;
+  uint64_t* acc_full = cfull + STAGES;   // [2] MMA of a tile done (both CTAs, multicast commit)
+  uint64_t* acc_empty = acc_full + 2;    // [2] even CTA: both CTAs' epilogues drained the buffer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_kb = args.num_kb;
+  const int n_iters = num_kb + (args.tail_ksteps > 0 ? 1 : 0);
+  const bool paired = args.pair_off > 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1 + 16);
+      ptx::mbar_init(&empty[s], 1);
+      ptx::mbar_init(&cfull[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&acc_full[b], 1);
+      ptx::mbar_init(&acc_empty[b], 8);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+    ptx::prefetch_tmap(&tmA2);
+    if (DUAL) ptx::prefetch_tmap(&tmA3);
+    if (args.tail_ksteps > 0) {
+      ptx::prefetch_tmap(&tmTA);
+      ptx::prefetch_tmap(&tmTB);
+    }
+  }
+  if (warp >= 2 && warp < 10) {
+    float2* lut2 = reinterpret_cast<float2*>(smem_raw);
+    for (int i = threadIdx.x - 64; i < 256 * C::LUT_LANES; i += 256) {
+      const int b = i / C::LUT_LANES;
+      lut2[i] = make_float2(__uint_as_float(c_nf4_bits[b >> 4]), __uint_as_float(c_nf4_bits[b & 15]));
+    }
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(tmem_slot, 512);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  ptx::cluster_sync();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(full), 0);
+      int gi = 0;
+      bool ok = true;
+      for (int t = pair; t < ntiles_total && ok; t += npairs) {
+        const PairTile tl = pair_tile(args, t, mtiles, rank);
+        const int r0 = paired ? (rank == 0 ? tl.nb : args.pair_off + tl.nb) : tl.n0 + (int)rank * 128;
+        const int c0 = tl.n0 + (int)rank * 128;
+        for (int it = 0; it < n_iters; ++it, ++gi) {
+          const int s = gi % STAGES;
+          const uint32_t ph = (gi / STAGES) & 1;
+          if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+            atomicOr(args.err, 1);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* a = sA + s * C::A_STAGE;
+          uint8_t* b = sB + s * C::B_STAGE;
+          const bool tail = it >= num_kb;
+          const uint32_t bytes = tail ? (uint32_t)(A_STAGE_BYTES + C::B_STAGE) : (uint32_t)C::A_STAGE;
+          if (rank == 0) ptx::mbar_arrive_expect_tx(&full[s], 2 * bytes);
+          const uint32_t bar = full0 + s * 8;
+          if (!tail) {
+            ptx::tma_load_2d_pair(a, &tmA, bar, it * BK, tl.m0);
+            if (DUAL) ptx::tma_load_2d_pair(a + A_STAGE_BYTES, &tmA3, bar, it * BK, tl.m0);
+            uint8_t* c = sC + s * C::C_STAGE;
+            uint8_t* sc = sS + s * C::S_STAGE;
+            const int ip = it + 12;
+            ptx::mbar_arrive_expect_tx(&cfull[s], (uint32_t)(C::C_STAGE + (B_MN ? 1024 : 2048)));
+            if (!B_MN) {
+              ptx::tma_load_2d(c, &tmB, &cfull[s], it * 32, r0);
+              ptx::tma_load_2d(sc, &tmA2, &cfull[s], it & ~3, r0);
+              if (ip < num_kb) {
+                ptx::tma_prefetch_l2_2d(&tmB, ip * 32, r0);
+                if ((ip & 3) == 0) ptx::tma_prefetch_l2_2d(&tmA2, ip, r0);
+              }
+            } else {
+              ptx::tma_load_2d(c, &tmB, &cfull[s], c0 / 2, it * BK);
+              ptx::tma_load_2d(sc, &tmA2, &cfull[s], (c0 / 64) & ~3, it * BK);
+              if (ip < num_kb) {
+                ptx::tma_prefetch_l2_2d(&tmB, c0 / 2, ip * BK);
+                ptx::tma_prefetch_l2_2d(&tmA2, (c0 / 64) & ~3, ip * BK);
+              }
+            }
+          } else {
+            ptx::mbar_arrive(&cfull[s]);  // keeps cfull's phase in step with the slot's uses
+            ptx::tma_load_2d_pair(a, &tmTA, bar, tl.m0, tl.tail_row);
+            ptx::tma_load_2d_pair(a + 8192, &tmTA, bar, tl.m0 + 64, tl.tail_row);
+            if (!B_MN) {
+              if (paired) {
+                ptx::tma_load_2d_pair(b, &tmTB, bar, 0, tl.nb + (int)rank * 64);
+                ptx::tma_load_2d_pair(b + 8192, &tmTB, bar, 0, args.pair_off + tl.nb + (int)rank * 64);
+              } else {
+                ptx::tma_load_2d_pair(b, &tmTB, bar, 0, tl.n0 + (int)rank * 128);
+              }
+            } else {
+              ptx::tma_load_2d_pair(b, &tmTB, bar, c0, 0);
+              ptx::tma_load_2d_pair(b + 8192, &tmTB, bar, c0 + 64, 0);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------- MMA issuer (even CTA of the pair)
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc_main = ptx::idesc_bf16(2 * BM, BN, 0, B_MN ? 1 : 0);
+      constexpr uint32_t idesc_tail = ptx::idesc_bf16(2 * BM, BN, 1, B_MN ? 1 : 0);
+      constexpr uint32_t idesc_half = ptx::idesc_bf16(2 * BM, BN / 2, 1, B_MN ? 1 : 0);
+      int gi = 0, lt = 0;
+      bool ok = true;
+      for (int t = pair; t < ntiles_total && ok; t += npairs, ++lt) {
+        const int ab = lt & 1;
+        if (!ptx::mbar_wait_bounded(&acc_empty[ab], ((lt >> 1) & 1) ^ 1, abort_flag)) {
+          atomicOr(args.err, 1);
+          *abort_flag = 1;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t tacc = tmem + (uint32_t)(ab * BN);
+        for (int it = 0; it < n_iters; ++it, ++gi) {
+          const int s = gi % STAGES;
+          const uint32_t ph = (gi / STAGES) & 1;
+          if (!ptx::mbar_wait_bounded(&full[s], ph, abort_flag)) {
+            atomicOr(args.err, 1);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a_base = ptx::smem_u32(sA + s * C::A_STAGE);
+          const uint32_t b_base = ptx::smem_u32(sB + s * C::B_STAGE);
+          const bool tail = it >= num_kb;
+          if (tail && paired) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const uint64_t ad = ptx::smem_desc_sw128(a_base + hf * 2048, 8192, 1024);
+              const uint64_t bd = ptx::smem_desc_sw128(b_base + hf * 8192, 16, 1024);
+              ptx::mma_bf16_pair(tacc + hf * (BN / 2), ad, bd, idesc_half, 1u);
+            }
+          } else {
+            const int nk = tail ? args.tail_ksteps : 4;
+            for (int k = 0; k < nk; ++k) {
+              const uint64_t ad = tail ? ptx::smem_desc_sw128(a_base + k * KSTEP_MN, CHUNK_BYTES, 1024)
+                                       : ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
+              const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k * KSTEP_MN, CHUNK_BYTES, 1024)
+                                       : ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
+              ptx::mma_bf16_pair(tacc, ad, bd, tail ? idesc_tail : idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+              if (DUAL && !tail)
+                ptx::mma_bf16_pair(tacc, ptx::smem_desc_sw128(a_base + A_STAGE_BYTES + k * 32, 16, 1024), bd,
+                                   idesc_main, 1u);
+            }
+          }
+          ptx::mma_commit_pair(&empty[s], 3);
+        }
+        if (ok) ptx::mma_commit_pair(&acc_full[ab], 3);
+      }
+    }
+  } else if (warp < 10) {
+    // ----------------------------------------------------- NF4 decode warps
+    const int td = threadIdx.x - 64;
+    const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(full), 0);
+    const uint32_t lane_b = C::LUT_LANES == 32 ? (uint32_t)lane * 8u : (uint32_t)(lane & 15) * 16u;
+    const uint8_t* lutb = smem_raw;
+    int gi = 0;
+    bool ok = true;
+    for (int t = pair; t < ntiles_total && ok; t += npairs) {
+      const PairTile tl = pair_tile(args, t, mtiles, rank);
+      int srow, unit0, chunk, coff, soff;
+      bool valid;
+      if constexpr (BMD == B_NF4_K) {
+        const int row = td >> 1, h = td & 1;
+        const int n = paired ? (rank == 0 ? tl.nb + row : args.pair_off + tl.nb + row) : tl.n0 + (int)rank * 128 + row;
+        valid = n < args.N;
+        srow = row;
+        unit0 = h * 4;
+        chunk = 0;
+        coff = row * 32 + h * 16;
+        soff = row * 4;
+      } else {
+        const int q = td & 3, kr = td >> 2;
+        const int col = tl.n0 + (int)rank * 128 + q * 32;
+        valid = col < args.N;
+        srow = kr;
+        unit0 = (q & 1) * 4;
+        chunk = q >> 1;
+        coff = kr * 64 + q * 16;
+        soff = kr * 4 + ((tl.n0 + (int)rank * 128) / 64 & 3) + (q >> 1);
+      }
+      uint8_t* const drow = sB + chunk * 8192 + srow * 128;
+      for (int it = 0; it < n_iters; ++it, ++gi) {
+        const int s = gi % STAGES;
+        const uint32_t ph = (gi / STAGES) & 1;
+        // cfull completes once per use of the slot (the tail stage arrives without bytes)
+        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag) ||
+            !ptx::mbar_wait_bounded(&cfull[s], ph, abort_flag)) {
+          atomicOr(args.err, 1);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        if (it < num_kb) {
+          const uint4 w = *reinterpret_cast<const uint4*>(sC + s * C::C_STAGE + coff);
+          const float am =
+              reinterpret_cast<const float*>(sS + s * C::S_STAGE)[soff + (BMD == B_NF4_K ? (it & 3) : 0)];
+          uint8_t* b = drow + s * C::B_STAGE;
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 v = valid ? decode8_pairs<C::LUT_LANES>(ws[u], lutb, lane_b, am) : make_uint4(0, 0, 0, 0);
+            st_shared_v4(b + (((unit0 + u) ^ (srow & 7)) << 4), v);
+          }
+          ptx::fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(full0 + s * 8);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // warps 10..13 own TMEM lane quadrants 2, 3, 0, 1; each drains all 256
+    // columns of its 32 rows, then frees the buffer on the even CTA
+    const int q = warp & 3;
+    const uint32_t acc_empty0 = ptx::mapa_shared(ptx::smem_u32(acc_empty), 0);
+    int lt = 0;
+    for (int t = pair; t < ntiles_total; t += npairs, ++lt) {
+      const PairTile tl = pair_tile(args, t, mtiles, rank);
+      const int ab = lt & 1;
+      if (!ptx::mbar_wait_bounded(&acc_full[ab], (lt >> 1) & 1, abort_flag)) {
+        atomicOr(args.err, 1);
+        *abort_flag = 1;
+        break;
+      }
+      ptx::tc_fence_after();
+      epilogue_tile<BN>(args, args.out, tmem + (uint32_t)(ab * BN), tl.m0, tl.n0, tl.nb, q, lane, 0, 1);
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(acc_empty0 + ab * 8);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000LL) {
+    }
+    __syncthreads();
+  }
+  ptx::cluster_sync();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -996,8 +1326,9 @@ soup_status make_plain_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_
 }
 constexpr int CU_DT_U8 = 0;  // CU_TENSOR_MAP_DATA_TYPE_UINT8
 
-template <int BN, int AMJ, int BMD, bool TF = false, bool DUAL = false, int CG = 1>
+template <int BN, int AMJ, int BMD, bool TF = false, bool DUAL = false, int CG = 1, bool PERSIST = false>
 soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
+  static_assert(!PERSIST || (CG == 2 && BN == 256 && AMJ == A_K && BMD >= B_NF4_K && !TF), "persistent: NF4 pairs");
   using C = Cfg<BN, DUAL, CG>;
   CUtensorMap mA, mB, mTA, mTB, mA2, mA3;
   memset(&mA2, 0, sizeof(mA2));
@@ -1031,6 +1362,49 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
     // it; paired gate|up tiles: one half of the pair's half)
     if (!B_MN) SOUP_TRY(make_map(&mTB, d.tailB, 64, (paired ? BN / 2 : BN) / CG, "tail B"));
     else SOUP_TRY(make_map(&mTB, d.tailB, 64, 64, "tail B (MN-major)"));
+  }
+  if constexpr (PERSIST) {
+    auto kp = gemm_pair_persistent<BMD, DUAL>;
+    static int max_pairs = 0;  // per instantiation: co-resident CTA pairs
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.blockDim = dim3(PERSIST_THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    if (max_pairs == 0) {
+      SOUP_CUDA_TRY(cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+      cfg.gridDim = dim3(2 * (sm_count() / 2));
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, kp, &cfg) != cudaSuccess || nc <= 0) {
+        cudaGetLastError();
+        nc = sm_count() / 2;
+      }
+      max_pairs = nc;
+    }
+    const int mtiles = (d.M + 2 * BM - 1) / (2 * BM);
+    const int ntiles = paired ? d.pair_off / (BN / 2) : (d.N + BN - 1) / BN;
+    const int total = mtiles * ntiles;
+    const int npairs = std::min(total, max_pairs);
+    cfg.gridDim = dim3(2 * npairs);
+    if (profiling()) {
+      const int cls = DUAL ? GC_NF4_DUAL : (BMD == B_NF4_K ? GC_NF4_FWD : GC_NF4_BWD);
+      const double tail_k = d.tail_ksteps > 0 ? (double)d.tailA.rows : 0.0;
+      const double flops = 2.0 * d.M * d.N * ((double)d.K * (DUAL ? 2 : 1) + (paired ? 16.0 : tail_k));
+      const double bytes = (double)d.M * d.K * 2 + (double)d.N * d.K * (0.5 + 4.0 / 64) +
+                           (double)d.M * d.N * ((d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T) ? 4 : 2);
+      profile_begin(st, cls, flops, bytes);
+    }
+    SOUP_CUDA_TRY(cudaLaunchKernelEx(&cfg, kp, mA, mB, mTA, mTB, mA2, mA3, ka, mtiles, total));
+    SOUP_LAUNCH_CHECK();
+    profile_end(st);
+    return SOUP_OK;
   }
   auto kern = gemm_kernel<BN, AMJ, BMD, TF, DUAL, CG>;
   static bool attr_set = false;  // per instantiation
@@ -1111,6 +1485,10 @@ soup_status dispatch(const GemmDesc& d, const KArgs& ka, int bn, cudaStream_t st
                        (d.b_mode == B_NF4_K ? d.K % 256 == 0 : d.N % 256 == 0);
   if (d.A_lo.ptr) {
     if (pair_ok && d.A_lo.rows == d.A.rows && d.A_lo.cols == d.A.cols) {
+      if (d.persistent) {
+        if (d.b_mode == B_NF4_K) return launch<256, A_K, B_NF4_K, false, true, 2, true>(d, ka, st);
+        return launch<256, A_K, B_NF4_MN, false, true, 2, true>(d, ka, st);
+      }
       if (d.b_mode == B_NF4_K) return launch<256, A_K, B_NF4_K, false, true, 2>(d, ka, st);
       return launch<256, A_K, B_NF4_MN, false, true, 2>(d, ka, st);
     }
@@ -1129,6 +1507,10 @@ soup_status dispatch(const GemmDesc& d, const KArgs& ka, int bn, cudaStream_t st
     return fail(SOUP_ERR_SHAPE, "gemm: no dual-A kernel for BN=%d b_mode=%d", bn, d.b_mode);
   }
   if (pair_ok) {
+    if (d.persistent) {
+      if (d.b_mode == B_NF4_K) return launch<256, A_K, B_NF4_K, false, false, 2, true>(d, ka, st);
+      return launch<256, A_K, B_NF4_MN, false, false, 2, true>(d, ka, st);
+    }
     if (d.b_mode == B_NF4_K) return launch<256, A_K, B_NF4_K, false, false, 2>(d, ka, st);
     return launch<256, A_K, B_NF4_MN, false, false, 2>(d, ka, st);
   }

@@ -89,6 +89,10 @@ struct GemmDesc {
   const float* rope_cos = nullptr;
   const float* rope_sin = nullptr;
   int bn = 0;               // N tile (0 = pick)
+  // NF4 GEMMs on CTA pairs: persistent tile loop with two accumulators (the
+  // epilogue of one tile overlaps the next tile's main loop) or one tile
+  // per pair
+  bool persistent = true;
   // Optional split-K for skinny GEMMs (N <= 64, TMA operands, plain store
   // epilogue): when a workspace is given and the M x N tiles alone cannot
   // fill the GPU, the K range is cut into up to 8 slices whose fp32 partial
