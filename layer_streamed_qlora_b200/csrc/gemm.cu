@@ -930,13 +930,13 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
 
 // Persistent form of the CTA-pair NF4 GEMM: each pair loops over 256x256
 // output tiles (t = pair, pair + pairs, ...; M tiles fastest) with two
-// accumulators in tensor memory (2 x 256 columns), so that 4 epilogue warps
+// accumulators in tensor memory (2 x 256 columns), so that 8 epilogue warps
 // drain tile i while the MMA warp already accumulates tile i + 1.  Roles:
 // warp 0 TMA producer, warp 1 TMEM owner + MMA issuer (even CTA), warps 2..9
-// NF4 decode, warps 10..13 epilogue.  The shared-memory ring, decode, tail
+// NF4 decode, warps 10..17 epilogue (two per TMEM lane quadrant).  The shared-memory ring, decode, tail
 // K-block and epilogues are those of gemm_kernel with CTA pairs; the stage
 // counter runs on across tiles and the decode table is built once.
-constexpr int PERSIST_THREADS = 32 * 14;
+constexpr int PERSIST_THREADS = 32 * 18;
 
 struct PairTile {
   int m0, n0, nb, tail_row;
@@ -1002,7 +1002,7 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&acc_full[b], 1);
-      ptx::mbar_init(&acc_empty[b], 8);
+      ptx::mbar_init(&acc_empty[b], 16);
     }
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -1214,9 +1214,10 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // warps 10..13 own TMEM lane quadrants 2, 3, 0, 1; each drains all 256
-    // columns of its 32 rows, then frees the buffer on the even CTA
-    const int q = warp & 3;
+    // warps 10..17 own TMEM lane quadrants 2, 3, 0, 1 (twice); each drains
+    // every other 16-column chunk of its 32 rows, then frees the buffer on
+    // the even CTA
+    const int q = warp & 3, ew = warp - 10;
     const uint32_t acc_empty0 = ptx::mapa_shared(ptx::smem_u32(acc_empty), 0);
     int lt = 0;
     for (int t = pair; t < ntiles_total; t += npairs, ++lt) {
@@ -1228,7 +1229,7 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
-      epilogue_tile<BN>(args, args.out, tmem + (uint32_t)(ab * BN), tl.m0, tl.n0, tl.nb, q, lane, 0, 1);
+      epilogue_tile<BN>(args, args.out, tmem + (uint32_t)(ab * BN), tl.m0, tl.n0, tl.nb, q, lane, ew / 4, 2);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(acc_empty0 + ab * 8);
