@@ -299,17 +299,13 @@ def main():
     model.set_ids(ids_host)
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
-    flat = None
-    if world > 1:
-        flat_numel = sum(v.numel() for gd in model.grads for v in gd.values())
-        flat = torch.empty(flat_numel, dtype=torch.float32, device="cuda")
+    from layer_streamed_qlora_b200 import dp
 
     def step():
         loss = model.sft_step() if w["task"] == "sft" else model.dpo_step(w["prompt"], w["beta"])
-        if world > 1:
-            # data parallel: the one exchange of the step, the LoRA gradients
-            torch.cat([v.reshape(-1) for gd in model.grads for v in gd.values()], out=flat)
-            dist.all_reduce(flat)
+        # data parallel: the one exchange of the step, the LoRA gradients
+        # averaged in place (a no-op on one rank)
+        dp.allreduce_mean_(model.grad_flat)
         return loss
 
     for _ in range(max(3, args.warmup)):

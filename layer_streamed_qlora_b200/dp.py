@@ -1,0 +1,53 @@
+"""Data parallelism for the streamed LoRA step.
+
+One process per GPU: every rank streams its own copy of the frozen base over
+its own host link and runs its own micro-batch through the whole step; the
+LoRA gradients, the only trained state, are averaged across ranks once per
+step.  They live in one flat fp32 buffer (each factor a 256-byte-aligned view
+into it), so the exchange is a single in-place all-reduce of that buffer.
+"""
+from __future__ import annotations
+
+import torch
+
+ALIGN = 64  # elements (256 bytes)
+
+
+def flat_layout(shapes):
+    """Offsets (in elements) of tensors of the given shapes packed in order,
+    each starting on a 256-byte boundary, and the total length."""
+    offs, n = [], 0
+    for sh in shapes:
+        offs.append(n)
+        size = 1
+        for d in sh:
+            size *= int(d)
+        n += (size + ALIGN - 1) // ALIGN * ALIGN
+    return offs, n
+
+
+def flat_views(shapes, device, dtype=torch.float32):
+    """A zeroed flat buffer and one contiguous view per shape (see flat_layout)."""
+    offs, n = flat_layout(shapes)
+    flat = torch.zeros(max(n, 1), dtype=dtype, device=device)
+    views = []
+    for o, sh in zip(offs, shapes):
+        size = 1
+        for d in sh:
+            size *= int(d)
+        views.append(flat[o:o + size].view(sh))
+    return flat, views
+
+
+def allreduce_mean_(flat: torch.Tensor, group=None) -> torch.Tensor:
+    """Average `flat` over the process group in place: one all-reduce (sum)
+    and one scale by 1/world.  A no-op when torch.distributed is not
+    initialised or the group has a single rank."""
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized():
+        return flat
+    world = dist.get_world_size(group)
+    if world > 1:
+        dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+        flat.mul_(1.0 / world)
+    return flat

@@ -22,6 +22,7 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib as L
+from . import dp
 
 ITEM_EMBED, ITEM_HEAD = L.SOUP_ITEM_EMBED, L.SOUP_ITEM_HEAD
 PROJS = ("q", "k", "v", "o", "gate", "up", "down")
@@ -186,8 +187,12 @@ class StreamedLoRAModel:
         before = torch.cuda.memory_allocated()
         self.final_norm = weights.final_norm().contiguous()
         self.lora = [{k: v.contiguous() for k, v in weights.lora(l).items()} for l in range(cfg.n_layers)]
-        self.grads = [{"d" + k: torch.zeros(v.shape, dtype=torch.float32, device="cuda") for k, v in lo.items()}
-                      for lo in self.lora]
+        # LoRA gradients: fp32 views into one flat buffer (the data-parallel
+        # exchange all-reduces that buffer in place; see dp.py)
+        keys = [list(lo.keys()) for lo in self.lora]
+        self.grad_flat, views = dp.flat_views([lo[k].shape for lo, ks in zip(self.lora, keys) for k in ks], "cuda")
+        it = iter(views)
+        self.grads = [{"d" + k: next(it) for k in ks} for ks in keys]
         self.lora_s = [L.layer_lora(lo) for lo in self.lora]
         self.grads_s = [L.layer_grads(g) for g in self.grads]
         self.ckpt = torch.empty((cfg.n_layers + 1, T, cfg.hidden), dtype=torch.bfloat16, device="cuda")

@@ -1,0 +1,91 @@
+"""Data-parallel exchange of the LoRA gradients on two CPU ranks (gloo).
+
+The flat-buffer layout must be identical on every rank and the in-place
+all-reduce must leave every rank with the mean of the ranks' gradients in
+every view.  CPU only: the same code path runs over NCCL on GPUs.
+"""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from layer_streamed_qlora_b200 import dp
+
+SHAPES = [(16, 4096), (6144, 16), (16, 4096), (4096, 16), (32, 4096), (28672, 16), (16, 14336), (4096, 16),
+          (3, 5)]
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        flat, views = dp.flat_views(SHAPES, "cpu")
+        g = torch.Generator().manual_seed(100 + rank)
+        vals = []
+        for v in views:
+            v.copy_(torch.randn(v.shape, generator=g))
+            vals.append(v.clone())
+        dp.allreduce_mean_(flat)
+        # numpy copies: plain pickles (tensors would travel as shared-memory handles)
+        q.put((rank, [v.numpy().copy() for v in views], [v.numpy() for v in vals], dp.flat_layout(SHAPES),
+               flat.numpy().copy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_flat_layout_alignment():
+    offs, n = dp.flat_layout(SHAPES)
+    assert all(o % 64 == 0 for o in offs)
+    assert n >= sum(a * b for a, b in SHAPES)
+    flat, views = dp.flat_views(SHAPES, "cpu")
+    for v, sh in zip(views, SHAPES):
+        assert tuple(v.shape) == sh and v.is_contiguous() and (v.data_ptr() - flat.data_ptr()) % 256 == 0
+
+
+def test_allreduce_mean_single_process_is_noop():
+    flat, _ = dp.flat_views([(4, 4)], "cpu")
+    flat.fill_(3.0)
+    dp.allreduce_mean_(flat)
+    assert torch.all(flat == 3.0)
+
+
+@pytest.mark.timeout(120)
+def test_two_rank_gradient_average():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        rank, after, before, layout, gap = q.get(timeout=100)
+        res[rank] = (after, before, layout, gap)
+    for p in procs:
+        p.join(timeout=30)
+        assert p.exitcode == 0
+    assert res[0][2] == res[1][2]  # same layout on every rank
+    for i in range(len(SHAPES)):
+        mean = (res[0][1][i] + res[1][1][i]) / 2
+        for r in range(world):
+            torch.testing.assert_close(torch.from_numpy(res[r][0][i]), torch.from_numpy(mean), rtol=1e-6, atol=1e-6)
+    # the alignment padding between views stays zero
+    offs, n = dp.flat_layout(SHAPES)
+    for r in range(world):
+        pad = torch.ones(n, dtype=torch.bool)
+        for o, (a, b) in zip(offs, SHAPES):
+            pad[o:o + a * b] = False
+        assert torch.all(torch.from_numpy(res[r][3])[pad] == 0)
