@@ -147,3 +147,20 @@ def lora_params(shape: LayerShape, seed: int, layer: int = 0, std: float = 0.02,
 def uniform_ids(seed: int, name: str, shape, vocab: int) -> np.ndarray:
     g = rng_for(seed, name)
     return g.integers(0, vocab, size=shape, dtype=np.int64).astype(np.int32)
+
+
+def nf4_stored_blocks(seed: int, name: str, out_f: int, in_f: int, w_std: float = 0.02):
+    """Stored NF4 weights drawn directly (no quantisation step), shaped like
+    the NF4 codes of N(0, w_std) weights: the two extreme levels (+-1, the
+    block's absmax element) with probability 1/128 each, the 14 inner levels
+    equally likely (NF4 levels are equiprobable quantiles), two independent
+    codes per byte (high nibble first); a per-64-block absmax of the size the
+    largest of 64 N(0, w_std) draws has (w_std x U[2.0, 3.2]).  Returns
+    (uint8 [out_f, in_f/2], float32 [out_f, in_f/64])."""
+    g = rng_for(seed, name)
+    p = np.full(16, (1.0 - 2.0 / 128) / 14)
+    p[0] = p[15] = 1.0 / 128
+    codes = g.choice(16, size=(out_f, in_f), p=p).astype(np.uint8)
+    packed = (codes[:, 0::2] << 4) | codes[:, 1::2]
+    absmax = (w_std * (2.0 + 1.2 * g.random((out_f, in_f // 64)))).astype(np.float32)
+    return packed.astype(np.uint8), absmax

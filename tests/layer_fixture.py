@@ -40,6 +40,15 @@ class DevLayer:
                 self.keep += [codes, absmax]
                 structs[name] = L.weight_nf4(codes, absmax, *W32.shape)
                 deq = onf4.dequant_bf16(*onf4.quantize(W32)).astype(np.float64)
+            elif kind == "nf4_stored":
+                # stored NF4 weights drawn directly (full-size layers: the
+                # oracle only dequantises, no fp64 quantisation of 218 M weights)
+                packed, am = ss.nf4_stored_blocks(seed, f"{layer}.{name}.nf4", *W32.shape)
+                codes = torch.from_numpy(packed).cuda()
+                absmax = torch.from_numpy(am).cuda()
+                self.keep += [codes, absmax]
+                structs[name] = L.weight_nf4(codes, absmax, *W32.shape)
+                deq = onf4.dequant_bf16(packed, am).astype(np.float64)
             else:
                 deq = onf4.round_to_bf16(W32).astype(np.float64)
                 wb = dev_bf16(deq)
