@@ -14,10 +14,6 @@ namespace soup {
 namespace {
 
 __device__ __forceinline__ float b2f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
-__device__ __forceinline__ uint16_t f2b(float f) {
-  __nv_bfloat16 h = __float2bfloat16_rn(f);
-  return *reinterpret_cast<uint16_t*>(&h);
-}
 __device__ __forceinline__ void unpack8(const uint4 v, float* f) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll

@@ -238,34 +238,6 @@ soup_status lora_g(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t*
   return gemm(g, st);
 }
 
-// dB [n, r] = dy_seg^T u_seg^T : dy = columns of a [T, ld] buffer.
-soup_status lora_dB(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t* u, int r, int64_t ldT, float* dB,
-                    cudaStream_t st, const SplitWS& sw) {
-  GemmDesc g;
-  g.M = n; g.N = r; g.K = T;
-  g.a_major = A_MN;
-  g.A = Mat{dy, T, n, ld};
-  g.b_mode = B_TMA_K;
-  g.B = Mat{u, r, T, ldT};
-  g.out_kind = OUT_F32; g.out = dB; g.ldo = r;
-  use_split(g, sw);
-  return gemm(g, st);
-}
-
-// dA [rows, K] = g'^T x  (computed transposed: M = K, N = rows)
-soup_status lora_dA(const uint16_t* x, int T, int K, const uint16_t* gt, int rows, int64_t ldT, float* dA,
-                    cudaStream_t st, const SplitWS& sw) {
-  GemmDesc g;
-  g.M = K; g.N = rows; g.K = T;
-  g.a_major = A_MN;
-  g.A = Mat{x, T, K, K};
-  g.b_mode = B_TMA_K;
-  g.B = Mat{gt, rows, T, ldT};
-  g.out_kind = OUT_F32_T; g.out = dA; g.ldo = K;
-  use_split(g, sw);
-  return gemm(g, st);
-}
-
 // dA [rows, K] = (g' + g_lo)^T x, with g' and its rounding residual g_lo
 // stored transposed [rows, ldT] (a K-major A of M = rows) and x [T, K] the
 // MN-major B: two bf16 MMAs per k-step give an fp32-accurate g.
