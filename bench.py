@@ -388,6 +388,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "global_batch": B * world, "seq_len": S, "layers": cfg.n_layers,
                    "base": cfg.kind, "stream_buffers": w["buffers"], "device_cap_gb": w["cap_gb"],
+                   "device_cap_bytes": cap,
+                   "kept_qkv_layers": 0 if model.keep is None else int(model.keep.shape[0]),
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (the streamed base, >4 GB per step)"},
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": ids_host.numel() * 4,

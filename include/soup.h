@@ -237,6 +237,27 @@ soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const soup_layer
                                    const soup_layer_grads* grads, int32_t adapters_on,
                                    void* workspace, size_t workspace_bytes, void* stream);
 
+/* Selective keep of the layer's q|k|v between its two reads (the pages'
+ * forward read and recompute read of every layer; deep dive, section "How
+ * layer streaming works"): the forward pass, which waits on its copy stream
+ * anyway, computes q|k|v from the fp32-accurate normalised input (the same
+ * values the recompute would produce) and leaves them in qkv_keep; the
+ * backward then skips its q|k|v GEMM.  Results are bit-identical to the
+ * fwd + recompute pair above.  qkv_keep: fp16 [T, (Hq + 2 Hkv) * head_dim],
+ * soup_decoder_layer_keep_bytes bytes, 16-byte aligned, owned by the caller
+ * and kept untouched between the two calls of the same layer. */
+size_t soup_decoder_layer_keep_bytes(const soup_layer_cfg* cfg, int64_t batch, int64_t seq);
+soup_status soup_decoder_layer_fwd_keep(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                        const soup_layer_cfg* cfg, const uint16_t* h_in, int64_t batch,
+                                        int64_t seq, uint16_t* h_out, int32_t adapters_on, uint16_t* qkv_keep,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+soup_status soup_decoder_layer_bwd_kept(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                        const soup_layer_cfg* cfg, const uint16_t* h_in,
+                                        const float* dh_out, int64_t batch, int64_t seq, float* dh_in,
+                                        const soup_layer_grads* grads, int32_t adapters_on,
+                                        const uint16_t* qkv_kept, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
 /* ------------------------------------------------------- layer streaming ---
  * The frozen base lives in pinned host RAM as one blob per decoder layer
  * (Soup pages, "how layer streaming works": per-layer shards in page-locked

@@ -361,14 +361,18 @@ soup_status proj_bwd(const soup_weight* W, const uint16_t* dy, int T, const uint
 
 // Forward through the layer; with `keep_down_out` false the final down GEMM
 // (whose output the backward pass does not need) is skipped.
+// keep (forward pass only): also compute q|k|v with the hi + lo A pair and
+// leave them (fp16, [T, qkv_w]) in `keep` for the backward; kept (recompute
+// only): q|k|v of this layer kept by the forward pass, whose GEMM is skipped.
 soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const soup_layer_cfg* c, const Dims& m,
                     const WS& ws, char* base, const uint16_t* h_in, uint16_t* h_out, bool on, bool recompute,
-                    cudaStream_t st) {
+                    cudaStream_t st, uint16_t* keep = nullptr, const uint16_t* kept = nullptr) {
   const int T = m.T, r = m.r;
   const SplitWS SW{PF(splitk), ws.splitk_bytes};
   SOUP_TRY(rope_table(m.S, m.d, (double)c->theta, PF(cosb), PF(sinb), st));
+  const bool precise_qkv = (recompute && !kept) || keep;  // q|k|v from the hi + lo x1 pair
   SOUP_TRY(rmsnorm_fwd(h_in, nullptr, W->norm1, T, m.H, c->eps, P(x1), PF(rinv1), st, on ? PF(x1_32) : nullptr,
-                       recompute ? P(x1_lo) : nullptr));
+                       precise_qkv ? P(x1_lo) : nullptr));
   if (on) {
     // q/k/v adapters: u from the fp32 normalised input (tf32 tensor cores); the
     // tail consumes its bf16 copy, the dB GEMM its fp32 copy
@@ -385,11 +389,13 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     // for the backward, q/k/v from an fp32-accurate x1 (hi + lo parts): the
     // attention backward amplifies the bf16 rounding of x1 into the q/k/v
     // adapter gradients
-    if (recompute) o.x_lo = P(x1_lo);
-    SOUP_TRY(proj_fwd(&W->qkv, P(x1), T, P(u_qkv), m.ldT, 3 * r, L ? L->B_qkv : nullptr, r, 3, se, sr, on, P(qkv),
-                      st, o));
+    if (precise_qkv) o.x_lo = P(x1_lo);
+    if (!kept)
+      SOUP_TRY(proj_fwd(&W->qkv, P(x1), T, P(u_qkv), m.ldT, 3 * r, L ? L->B_qkv : nullptr, r, 3, se, sr, on,
+                        keep ? keep : P(qkv), st, o));
   }
-  SOUP_TRY(attention_fwd(P(qkv), m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(attn), PF(lse), st,
+  const uint16_t* qkvp = kept ? kept : (keep ? keep : P(qkv));
+  SOUP_TRY(attention_fwd(qkvp, m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(attn), PF(lse), st,
                          recompute ? P(attn16) : nullptr, on ? PF(attn32) : nullptr));
   if (on) {
     SOUP_TRY(bf16_to_f32(L->A_o, (size_t)r * m.o_in, PF(Ao32), st));
@@ -442,10 +448,16 @@ extern "C" size_t soup_decoder_layer_workspace(const soup_layer_cfg* cfg, int64_
   return layout(m).total;
 }
 
-extern "C" soup_status soup_decoder_layer_fwd(const soup_layer_weights* W, const soup_layer_lora* lora,
-                                              const soup_layer_cfg* cfg, const uint16_t* h_in, int64_t batch,
-                                              int64_t seq, uint16_t* h_out, int32_t adapters_on, void* workspace,
-                                              size_t workspace_bytes, void* stream) {
+extern "C" size_t soup_decoder_layer_keep_bytes(const soup_layer_cfg* cfg, int64_t batch, int64_t seq) {
+  Dims m;
+  if (make_dims(cfg, batch, seq, &m) != SOUP_OK) return 0;
+  return (size_t)m.T * m.qkv_w * 2;
+}
+
+static soup_status layer_fwd_impl(const soup_layer_weights* W, const soup_layer_lora* lora, const soup_layer_cfg* cfg,
+                                  const uint16_t* h_in, int64_t batch, int64_t seq, uint16_t* h_out,
+                                  int32_t adapters_on, void* workspace, size_t workspace_bytes, void* stream,
+                                  uint16_t* keep) {
   Dims m;
   SOUP_TRY(make_dims(cfg, batch, seq, &m));
   SOUP_TRY(check_weights(W, m));
@@ -457,14 +469,32 @@ extern "C" soup_status soup_decoder_layer_fwd(const soup_layer_weights* W, const
   SOUP_CHECK(workspace_bytes >= ws.total && soup_aligned(workspace, 256), SOUP_ERR_INVALID_ARG,
              "soup_decoder_layer_fwd: workspace %zu < %zu bytes or misaligned", workspace_bytes, ws.total);
   return forward(W, lora, cfg, m, ws, static_cast<char*>(workspace), h_in, h_out, adapters_on != 0, false,
-                 static_cast<cudaStream_t>(stream));
+                 static_cast<cudaStream_t>(stream), keep);
 }
 
-extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const soup_layer_lora* L,
-                                              const soup_layer_cfg* cfg, const uint16_t* h_in, const float* dh_out,
-                                              int64_t batch, int64_t seq, float* dh_in,
-                                              const soup_layer_grads* G, int32_t adapters_on, void* workspace,
+extern "C" soup_status soup_decoder_layer_fwd(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                              const soup_layer_cfg* cfg, const uint16_t* h_in, int64_t batch,
+                                              int64_t seq, uint16_t* h_out, int32_t adapters_on, void* workspace,
                                               size_t workspace_bytes, void* stream) {
+  return layer_fwd_impl(W, lora, cfg, h_in, batch, seq, h_out, adapters_on, workspace, workspace_bytes, stream,
+                        nullptr);
+}
+
+extern "C" soup_status soup_decoder_layer_fwd_keep(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                                   const soup_layer_cfg* cfg, const uint16_t* h_in, int64_t batch,
+                                                   int64_t seq, uint16_t* h_out, int32_t adapters_on,
+                                                   uint16_t* qkv_keep, void* workspace, size_t workspace_bytes,
+                                                   void* stream) {
+  SOUP_CHECK(qkv_keep && soup_aligned(qkv_keep, 16), SOUP_ERR_INVALID_ARG,
+             "soup_decoder_layer_fwd_keep: null or misaligned keep buffer");
+  return layer_fwd_impl(W, lora, cfg, h_in, batch, seq, h_out, adapters_on, workspace, workspace_bytes, stream,
+                        qkv_keep);
+}
+
+static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_lora* L, const soup_layer_cfg* cfg,
+                                  const uint16_t* h_in, const float* dh_out, int64_t batch, int64_t seq, float* dh_in,
+                                  const soup_layer_grads* G, int32_t adapters_on, void* workspace,
+                                  size_t workspace_bytes, void* stream, const uint16_t* kept) {
   Dims m;
   SOUP_TRY(make_dims(cfg, batch, seq, &m));
   SOUP_TRY(check_weights(W, m));
@@ -482,7 +512,8 @@ extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const
   const int T = m.T, r = m.r, H = m.H, I = m.I;
   const int64_t ldT = m.ldT;
 
-  SOUP_TRY(forward(W, L, cfg, m, ws, base, h_in, nullptr, on, true, st));
+  SOUP_TRY(forward(W, L, cfg, m, ws, base, h_in, nullptr, on, true, st, nullptr, kept));
+  const uint16_t* qkvp = kept ? kept : P(qkv);
 
   // ---- MLP block
   SOUP_TRY(f32_to_bf16(dh_out, (size_t)T * H, P(dh_b), st));
@@ -529,7 +560,7 @@ extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const
   }
   SOUP_TRY(attn_rowdot(P(d_attn), P(attn16), T, m.Hq, PF(D), st));
   // dq and dk leave the attention backward already rotated back (inverse RoPE in its epilogues)
-  SOUP_TRY(attention_bwd(P(qkv), m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(d_attn), PF(lse), PF(D), P(d_qkv), PF(cosb),
+  SOUP_TRY(attention_bwd(qkvp, m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(d_attn), PF(lse), PF(D), P(d_qkv), PF(cosb),
                          PF(sinb), gamax, st, on ? PF(dqkv32) : nullptr));
   const int seg_n[3] = {m.Hq * m.d, m.Hkv * m.d, m.Hkv * m.d};
   const int seg_c[3] = {0, m.Hq * m.d, (m.Hq + m.Hkv) * m.d};
@@ -594,4 +625,25 @@ extern "C" soup_status soup_layer_blob_views(const soup_layer_cfg* cfg, int32_t 
   o += align256((size_t)m.H * 2);
   out->norm2 = reinterpret_cast<const uint16_t*>(b + o);
   return SOUP_OK;
+}
+
+extern "C" soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const soup_layer_lora* L,
+                                              const soup_layer_cfg* cfg, const uint16_t* h_in, const float* dh_out,
+                                              int64_t batch, int64_t seq, float* dh_in,
+                                              const soup_layer_grads* G, int32_t adapters_on, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  return layer_bwd_impl(W, L, cfg, h_in, dh_out, batch, seq, dh_in, G, adapters_on, workspace, workspace_bytes,
+                        stream, nullptr);
+}
+
+extern "C" soup_status soup_decoder_layer_bwd_kept(const soup_layer_weights* W, const soup_layer_lora* L,
+                                                   const soup_layer_cfg* cfg, const uint16_t* h_in,
+                                                   const float* dh_out, int64_t batch, int64_t seq, float* dh_in,
+                                                   const soup_layer_grads* G, int32_t adapters_on,
+                                                   const uint16_t* qkv_kept, void* workspace,
+                                                   size_t workspace_bytes, void* stream) {
+  SOUP_CHECK(qkv_kept && soup_aligned(qkv_kept, 16), SOUP_ERR_INVALID_ARG,
+             "soup_decoder_layer_bwd_kept: null or misaligned kept buffer");
+  return layer_bwd_impl(W, L, cfg, h_in, dh_out, batch, seq, dh_in, G, adapters_on, workspace, workspace_bytes,
+                        stream, qkv_kept);
 }

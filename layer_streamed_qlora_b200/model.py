@@ -125,12 +125,31 @@ class StreamedLoRAModel:
         weights = weights or SyntheticWeights(cfg, seed)
         self._build_blobs(weights)
         self._alloc(weights)
+        # q|k|v of every layer kept from the forward pass for the backward
+        # (skips the backward's q|k|v GEMM; identical results), when the
+        # device cap still admits the plan with it
+        # (layers 0 .. n_keep-1: as many as fit)
+        per = L.soup_decoder_layer_keep_bytes(self.lcfg, batch, seq)
+        n_keep = cfg.n_layers
+        while n_keep > 0 and not self._plan_fits(device_cap_bytes, self.reserve_bytes + n_keep * per):
+            n_keep -= 1
+        self.keep = None
+        if per and n_keep:
+            self.keep = torch.empty((n_keep, per // 2), dtype=torch.float16, device="cuda")
+            self.reserve_bytes += n_keep * per
         self.plan = L.Plan(self.host_layers, self.blob_bytes, n_buffers, self.vocab_bytes, self.host_embed,
                            self.host_head, device_cap_bytes, self.reserve_bytes)
         self._views = {}
         # When set to a dict, the backward pass stores dL/d(layer input) of
         # every layer in it (index l = input of layer l, n_layers = head output).
         self.capture_dh = None
+
+    def _plan_fits(self, cap: int, reserve: int) -> bool:
+        """Whether soup_stream_plan would admit this model with `reserve`
+        bytes of other device memory (slots + vocab slot + reserve <= cap)."""
+        if not cap:
+            return True
+        return self.n_buffers * self.blob_bytes + self.vocab_bytes + reserve <= cap
 
     # ------------------------------------------------------------ shard build
     def _build_blobs(self, weights):
@@ -235,8 +254,12 @@ class StreamedLoRAModel:
             P.prefetch(l)
         for l in range(nl):
             base = P.wait(l)
-            L.soup_decoder_layer_fwd(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.batch, self.seq,
-                                     self.ckpt[l + 1], adapters_on, self.ws)
+            if adapters_on and self.keep is not None and l < self.keep.shape[0]:
+                L.soup_decoder_layer_fwd_keep(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.batch,
+                                              self.seq, self.ckpt[l + 1], adapters_on, self.keep[l], self.ws)
+            else:
+                L.soup_decoder_layer_fwd(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.batch,
+                                         self.seq, self.ckpt[l + 1], adapters_on, self.ws)
             P.release(l)
             if l + N < nl:
                 P.prefetch(l + N)
@@ -258,8 +281,13 @@ class StreamedLoRAModel:
             if self.capture_dh is not None:  # inspection hook for layer-by-layer checks
                 self.capture_dh[l + 1] = self.dh.clone()
             base = P.wait(l)
-            L.soup_decoder_layer_bwd(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.dh, self.batch,
-                                     self.seq, self.dh, self.grads_s[l], 1, self.ws)
+            if self.keep is not None and l < self.keep.shape[0]:
+                L.soup_decoder_layer_bwd_kept(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.dh,
+                                              self.batch, self.seq, self.dh, self.grads_s[l], 1, self.keep[l],
+                                              self.ws)
+            else:
+                L.soup_decoder_layer_bwd(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.dh,
+                                         self.batch, self.seq, self.dh, self.grads_s[l], 1, self.ws)
             P.release(l)
             if l - N >= 0:
                 P.prefetch(l - N)

@@ -92,3 +92,34 @@ def test_layer_backward_is_deterministic():
     assert np.array_equal(o1, o2) and np.array_equal(d1, d2)
     for k in g1:
         assert torch.equal(g1[k], dl.grads_t[k]), k
+
+
+@pytest.mark.parametrize("kind", ["nf4", "bf16"])
+def test_kept_qkv_backward_is_bit_identical(kind):
+    """fwd_keep + bwd_kept (q|k|v kept from the forward pass, the backward's
+    q|k|v GEMM skipped) gives exactly the gradients and dh_in of fwd + the
+    recompute backward, and a forward output within the oracle tolerance."""
+    shape = SMALL
+    B, S = 2, 130
+    T = B * S
+    dl = DevLayer(L, shape, seed=6, kind=kind)
+    h, dh = inputs(shape, B, S, seed=7)
+    o1, d1 = run_layer(dl, h, dh, B, S)
+    g1 = {k: v.clone() for k, v in dl.grads_t.items()}
+    ws = torch.empty(L.soup_decoder_layer_workspace(dl.cfg, B, S), dtype=torch.uint8, device="cuda")
+    keep = torch.empty(L.soup_decoder_layer_keep_bytes(dl.cfg, B, S) // 2, dtype=torch.float16, device="cuda")
+    hd = dev_bf16(h.reshape(T, -1))
+    out = torch.empty_like(hd)
+    L.soup_decoder_layer_fwd_keep(dl.W, dl.lora, dl.cfg, hd, B, S, out, 1, keep, ws)
+    dho = dev_f32(dh.reshape(T, -1))
+    dhi = torch.empty_like(dho)
+    for v in dl.grads_t.values():
+        v.zero_()
+    L.soup_decoder_layer_bwd_kept(dl.W, dl.lora, dl.cfg, hd, dho, B, S, dhi, dl.grads, 1, keep, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(dhi).reshape(h.shape), d1)
+    for k in g1:
+        assert torch.equal(g1[k], dl.grads_t[k]), k
+    ref, _ = layer_fwd(h, dl.Wd, dl.lora_np, shape)
+    assert_close(host(out).reshape(h.shape), ref, "h_out (q|k|v from the hi + lo input)")
+    assert_close(host(out).reshape(h.shape), o1, "h_out vs plain forward", rel=5e-3, maxrel=1e-2)
