@@ -205,10 +205,11 @@ def run_reference(args, w, name):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-# Launch mix of the forward fused NF4 GEMM per layer and step: the forward
-# pass runs q|k|v, o, gate|up and down; the recompute runs o and gate|up
-# again (its q|k|v GEMM takes a hi + lo A pair: another kernel).
-PROBE_WEIGHTS = {"qkv": 1, "o": 2, "gate_up": 2, "down": 1}
+# Launch mix of the forward fused NF4 GEMM (one A operand) per layer and
+# step: the forward pass runs o, gate|up and down, the recompute o and
+# gate|up again; q|k|v (kept from the forward pass) takes a hi + lo A pair,
+# another kernel.
+PROBE_WEIGHTS = {"qkv": 0, "o": 2, "gate_up": 2, "down": 1}
 
 
 def probe_shapes(w):
