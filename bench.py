@@ -180,22 +180,33 @@ def cpu_baseline(w, tokens=256):
                       f"({t:.2f} s), projected to the {w['n_layers']}-layer stack (head excluded)"}
 
 
+def bench_config(w, name, world, kept_layers=None):
+    cfg = {"workload": name, "global_batch": w["batch"] * world, "seq_len": w["seq"], "layers": w["n_layers"],
+           "base": w["kind"], "stream_buffers": w["buffers"], "device_cap_gb": w["cap_gb"],
+           "device_cap_bytes": int(w["cap_gb"] * (1 << 30)),
+           "parallelism": f"dp{world}" if world > 1 else "single",
+           "l2": "inputs larger than L2 (the streamed base, >4 GB per step)"}
+    if kept_layers is not None:
+        cfg["kept_qkv_layers"] = kept_layers
+    return cfg
+
+
 def run_reference(args, w, name):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    for _ in range(args.warmup and 1):
-        pass
-    per = []
     tokens = 256
+    for _ in range(args.warmup):  # untimed warm-up samples
+        oracle_sample_seconds(w, tokens)
+    per = []
     for _ in range(args.steps):
         per.append(oracle_sample_seconds(w, tokens))
     t = statistics.median(per)
     value = tokens / (t * w["n_layers"])
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0, "steps": args.steps,
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t * w["n_layers"] * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": name, "global_batch": w["batch"], "seq_len": w["seq"], "layers": w["n_layers"]},
+            "config": bench_config(w, name, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                              "sample": f"per step: one decoder layer fwd+bwd on 1x{tokens} tokens, fp64 numpy, "
                                        f"projected to {w['n_layers']} layers"},
@@ -387,12 +398,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "global_batch": B * world, "seq_len": S, "layers": cfg.n_layers,
-                   "base": cfg.kind, "stream_buffers": w["buffers"], "device_cap_gb": w["cap_gb"],
-                   "device_cap_bytes": cap,
-                   "kept_qkv_layers": 0 if model.keep is None else int(model.keep.shape[0]),
-                   "parallelism": f"dp{world}" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (the streamed base, >4 GB per step)"},
+        "config": bench_config(w, args.workload, world, 0 if model.keep is None else int(model.keep.shape[0])),
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": ids_host.numel() * 4,
                 "d2h_bytes_per_step": 4},
         "gpu_launches": launches,
