@@ -329,7 +329,10 @@ def main():
     torch.cuda.reset_peak_memory_stats()
     clocks = ClockSampler(local)
     clocks.start()
-    L.profile_enable(0b00001)  # event-time only the dominant kernel (the fused NF4 forward GEMM) in the timed region
+    # event-time only the dominant kernel class in the timed region: the fused
+    # NF4 forward GEMM, or the bf16 GEMMs of an un-quantised base
+    dom_mask = 0b00001 if cfg.kind == "nf4" else 0b00100
+    L.profile_enable(dom_mask)
     n0 = L.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -380,7 +383,7 @@ def main():
     dom_name, dom = max(((k, v) for k, v in prof.items() if v["launches"]), key=lambda kv: kv[1]["total_ms"])
     achieved = dom["flops"] / (dom["total_ms"] / 1e3) / 1e12 if dom["total_ms"] > 0 else 0.0
     peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
-    tr = gemm_traffic()
+    tr = gemm_traffic() if dom_name == "nf4_fwd" else None
     roofline = {"bound": "tensor", "kernel": f"gemm {dom_name}", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak if peak else None,
                 "traffic": tr.get("bytes_per_launch") if tr else None,
