@@ -1,3 +1,4 @@
+#include <algorithm>
 // Memory-bound kernels of the decoder layer: RMSNorm forward/backward, the
 // RoPE angle table, the attention-backward row dot D = rowsum(dO * O), and
 // dtype conversions.  (RoPE itself is applied in the QKV GEMM epilogue and in
@@ -282,6 +283,56 @@ soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t s
 soup_status bf16_to_f32(const uint16_t* in, size_t n, float* out, cudaStream_t st) {
   SOUP_CHECK(n % 8 == 0, SOUP_ERR_SHAPE, "bf16_to_f32: n %% 8");
   bf16_to_f32_kernel<<<grid_for(n / 8, 256), 256, 0, st>>>(in, n, out);
+  SOUP_LAUNCH_CHECK();
+  return SOUP_OK;
+}
+
+
+namespace {
+struct PrepArgs {
+  PrepJobs jobs;
+  long long start[5];  // prefix sums of the jobs' output element counts
+};
+
+__global__ void lora_prep_kernel(const PrepArgs a) {
+  const long long total = a.start[a.jobs.njobs];
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    int k = 0;
+    while (k + 1 < a.jobs.njobs && idx >= a.start[k + 1]) ++k;
+    const PrepJob& J = a.jobs.job[k];
+    const long long i = idx - a.start[k];
+    if (J.kind == PREP_COPY_F32) {
+      static_cast<float*>(J.out)[i] = b2f(J.in[i]);
+    } else {
+      const int R = (int)(i / J.N), n = (int)(i % J.N);
+      const int s = R / J.r, j = R % J.r;
+      int seg = 0;
+      while (seg + 1 < J.nseg && n >= J.seg_end[seg]) ++seg;
+      const uint16_t v = seg == s ? J.in[(size_t)n * J.r + j] : static_cast<uint16_t>(0);
+      if (J.out_bf16) static_cast<uint16_t*>(J.out)[i] = v;
+      else static_cast<float*>(J.out)[i] = b2f(v);
+    }
+  }
+}
+}  // namespace
+
+soup_status lora_prep(const PrepJobs& jobs, cudaStream_t st) {
+  SOUP_CHECK(jobs.njobs >= 1 && jobs.njobs <= 4, SOUP_ERR_INVALID_ARG, "lora_prep: %d jobs", jobs.njobs);
+  PrepArgs a;
+  a.jobs = jobs;
+  a.start[0] = 0;
+  for (int k = 0; k < jobs.njobs; ++k) {
+    const PrepJob& J = jobs.job[k];
+    SOUP_CHECK(J.in && J.out, SOUP_ERR_INVALID_ARG, "lora_prep: null job pointer");
+    const long long n = J.kind == PREP_COPY_F32 ? (long long)J.rows * J.cols : (long long)J.nseg * J.r * J.N;
+    SOUP_CHECK(n > 0 && (J.kind == PREP_COPY_F32 || (J.r > 0 && J.nseg >= 1 && J.nseg <= 3)), SOUP_ERR_SHAPE,
+               "lora_prep: bad job %d", k);
+    a.start[k + 1] = a.start[k] + n;
+  }
+  const long long total = a.start[jobs.njobs];
+  const int blocks = (int)std::min<long long>((total + 255) / 256, (long long)sm_count() * 8);
+  lora_prep_kernel<<<blocks, 256, 0, st>>>(a);
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
 }

@@ -29,6 +29,28 @@ soup_status attn_rowdot(const uint16_t* dO, const uint16_t* O, int T, int Hq, fl
 soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t st);
 soup_status bf16_to_f32(const uint16_t* in, size_t n, float* out, cudaStream_t st);
 
+// LoRA operand preparation in one launch (up to 4 jobs):
+//   PREP_COPY_F32:   out[i] = fp32(in[i]), i < rows * cols (in and out [rows, cols])
+//   PREP_BLOCKDIAG_T: in = B [N, r] (rows grouped in nseg segments ending at
+//     seg_end[]), out [nseg * r, N] = the block-diagonal transpose: row
+//     s*r + j, column n holds B[n, j] when n lies in segment s, else 0
+//     (fp32, or bf16 with out_bf16)
+enum PrepKind : int { PREP_COPY_F32 = 0, PREP_BLOCKDIAG_T = 1 };
+struct PrepJob {
+  int kind = PREP_COPY_F32;
+  int out_bf16 = 0;
+  const uint16_t* in = nullptr;
+  void* out = nullptr;
+  int rows = 0, cols = 0;  // PREP_COPY_F32
+  int N = 0, r = 0, nseg = 1;
+  int seg_end[3] = {0, 0, 0};
+};
+struct PrepJobs {
+  int njobs = 0;
+  PrepJob job[4];
+};
+soup_status lora_prep(const PrepJobs& jobs, cudaStream_t st);
+
 // Causal GQA flash attention, head_dim 128.  qkv [T, ld] (fp16) holds q heads
 // at columns [0, Hq*128), k heads at [Hq*128, (Hq+Hkv)*128), v after them;
 // T = Bsz * S tokens, batch-major.  out [T, Hq*128] bf16; lse [Hq, T] (log2

@@ -34,13 +34,14 @@ struct Dims {
 // Workspace layout (byte offsets, each 256-aligned).
 struct WS {
   size_t x1, rinv1, qkv, attn, lse, h2, x2, rinv2, gu16, act, u_qkv, u_o, u_gu, u_d, cosb, sinb;
-  size_t dh_b, g_d, g_gu, g_o, g_qkv, Bt, d_gu, dx2, dh2, dh2_b, d_attn, D, d_qkv, dx1, attn16, gamax;
-  size_t x1_32, dqkv32, u32, g32, A32, Bt32;  // fp32 operands of the q/k/v LoRA-gradient GEMMs (tf32)
+  size_t dh_b, g_d, g_gu, g_o, g_qkv, d_gu, dx2, dh2, dh2_b, d_attn, D, d_qkv, dx1, attn16, gamax;
+  size_t x1_32, dqkv32, u32, g32, A32;  // fp32 operands of the q/k/v LoRA-gradient GEMMs (tf32)
   size_t x1_lo, dh2_lo;                       // bf16 rounding residuals (dual-A GEMM inputs)
   size_t attn32, uo32, go32, Ao32;            // fp32 operands of the o LoRA-gradient GEMMs (tf32)
   size_t splitk, splitk_bytes;                // fp32 partial products of split-K LoRA GEMMs
   size_t u_gu_lo, g_d_lo, u_d32;     // MLP LoRA-gradient operands beyond bf16 (residuals, fp32)
   size_t x2_32, Agu32, g_gu32, d_gu_lo;
+  size_t Bt_down32, Bt_o32, Bbd_qkv32, Bbd_gu;  // B factors prepared for the g GEMMs (transposed, block-diagonal)
   size_t total;
 };
 
@@ -75,7 +76,6 @@ WS layout(const Dims& m) {
   w.g_o = take(r * ldT * 2);
   w.g_qkv = take(3 * r * ldT * 2);
   size_t max_out = std::max<size_t>(std::max<size_t>(H, I), (size_t)m.qkv_w);
-  w.Bt = take(max_out * r * 2);
   w.d_gu = take(T * 2 * I * 2);
   w.dx2 = take(T * H * 2);
   w.dh2 = take(T * H * 4);
@@ -91,7 +91,6 @@ WS layout(const Dims& m) {
   w.u32 = take(3 * r * ldT * 4);
   w.g32 = take(3 * r * ldT * 4);
   w.A32 = take(3 * r * H * 4);
-  w.Bt32 = take(max_out * r * 4);
   w.x1_lo = take(T * H * 2);
   w.dh2_lo = take(T * H * 2);
   w.attn32 = take(T * m.o_in * 4);
@@ -107,6 +106,10 @@ WS layout(const Dims& m) {
   w.Agu32 = take(2 * r * H * 4);
   w.g_gu32 = take(2 * r * ldT * 4);
   w.d_gu_lo = take(T * 2 * I * 2);
+  w.Bt_down32 = take(r * H * 4);
+  w.Bt_o32 = take(r * H * 4);
+  w.Bbd_qkv32 = take(3 * r * (size_t)m.qkv_w * 4);
+  w.Bbd_gu = take(2 * r * 2 * I * 2);
   w.total = o;
   return w;
 }
@@ -217,23 +220,22 @@ soup_status lora_down(const uint16_t* x, int T, int K, const uint16_t* A, int ro
   return gemm(g, st);
 }
 
-// g' = bf16(s * dy B) for one adapter segment: dy = columns [c0, c0+n) of a
-// [T, ld] buffer, B [n, r]; writes rows of a transposed [*, ldT] buffer.
-// (optionally with dy's rounding residual dy_lo as a second A, and the fp32
-// values g32 and residual glo as extra outputs)
-soup_status lora_g(const uint16_t* dy, int64_t ld, int T, int n, const uint16_t* Bl, int r, float s, uint16_t* Bt,
-                   uint16_t* gout, int64_t ldT, cudaStream_t st, const SplitWS& sw, uint16_t* glo = nullptr,
-                   const uint16_t* dy_lo = nullptr, float* g32 = nullptr) {
-  SOUP_TRY(transpose_bf16(Bl, n, r, Bt, st));
+
+// g' = bf16(s * dy Bt^T) with a prepared Bt [rows, n] (transposed, possibly
+// block-diagonal over segments of dy's columns): one GEMM for all segments;
+// optionally dy's residual dy_lo (a second A), and the fp32 values g32 and
+// residual glo as extra outputs.  tf32: dy, Bt fp32.
+soup_status lora_g_prepared(const void* dy, const void* dy_lo, int64_t ld, int T, int n, const void* Bt, int rows,
+                            float s, bool tf32, uint16_t* gout, float* g32, uint16_t* glo, int64_t ldT,
+                            cudaStream_t st, const SplitWS& sw) {
   GemmDesc g;
-  g.M = T; g.N = r; g.K = n;
+  g.tf32 = tf32;
+  g.M = T; g.N = rows; g.K = n;
   g.A = Mat{dy, T, n, ld};
-  g.b_mode = B_TMA_K;
-  g.B = Mat{Bt, r, n, n};
-  g.out_kind = OUT_BF16_T; g.out = gout; g.ldo = ldT; g.alpha = s;
-  g.out_lo = glo;
-  g.out2 = g32;
   if (dy_lo) g.A_lo = Mat{dy_lo, T, n, ld};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{Bt, rows, n, n};
+  g.out_kind = OUT_BF16_T; g.out = gout; g.out2 = g32; g.out_lo = glo; g.ldo = ldT; g.alpha = s;
   use_split(g, sw);
   return gemm(g, st);
 }
@@ -269,9 +271,8 @@ soup_status lora_dB_dual(const uint16_t* dy, int64_t ld, int T, int n, const uin
   return gemm(g, st);
 }
 
-// tf32 variants of the LoRA GEMMs of the q/k/v group, on fp32 operands:
-// u = s x A^T (bf16 copy u' for the tail, fp32 copy for dB), g = s dy B
-// (bf16 copy g' for the tail, fp32 copy for dA), dA = g^T x, dB = dy^T u.
+// tf32 variants of the LoRA GEMMs on fp32 operands: u = s x A^T (bf16 copy
+// u' for the tail, fp32 copy for dB), dA = g^T x, dB = dy^T u.
 soup_status lora_down_tf32(const float* x, int T, int K, const float* A32, int rows, float s, uint16_t* u,
                            float* u32, int64_t ldT, cudaStream_t st, const SplitWS& sw, uint16_t* ulo = nullptr) {
   GemmDesc g;
@@ -286,21 +287,6 @@ soup_status lora_down_tf32(const float* x, int T, int K, const float* A32, int r
   return gemm(g, st);
 }
 
-soup_status lora_g_tf32(const float* dy, int64_t ld, int T, int n, const uint16_t* Bl, int r, float s, float* Bt32,
-                        uint16_t* gout, float* g32, int64_t ldT, cudaStream_t st, const SplitWS& sw,
-                        uint16_t* glo = nullptr) {
-  SOUP_TRY(transpose_bf16_f32(Bl, n, r, Bt32, st));
-  GemmDesc g;
-  g.tf32 = true;
-  g.M = T; g.N = r; g.K = n;
-  g.A = Mat{dy, T, n, ld};
-  g.b_mode = B_TMA_K;
-  g.B = Mat{Bt32, r, n, n};
-  g.out_kind = OUT_BF16_T; g.out = gout; g.out2 = g32; g.ldo = ldT; g.alpha = s;
-  g.out_lo = glo;
-  use_split(g, sw);
-  return gemm(g, st);
-}
 
 soup_status lora_dB_tf32(const float* dy, int64_t ld, int T, int n, const float* u32, int r, int64_t ldT, float* dB,
                          cudaStream_t st, const SplitWS& sw) {
@@ -376,7 +362,13 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
   if (on) {
     // q/k/v adapters: u from the fp32 normalised input (tf32 tensor cores); the
     // tail consumes its bf16 copy, the dB GEMM its fp32 copy
-    SOUP_TRY(bf16_to_f32(L->A_qkv, (size_t)3 * r * m.H, PF(A32), st));
+    // fp32 copies of the three A factors (tf32 operands), one launch
+    PrepJobs pj;
+    pj.njobs = 3;
+    pj.job[0].in = L->A_qkv; pj.job[0].out = PF(A32); pj.job[0].rows = 3 * r; pj.job[0].cols = m.H;
+    pj.job[1].in = L->A_o; pj.job[1].out = PF(Ao32); pj.job[1].rows = r; pj.job[1].cols = m.o_in;
+    pj.job[2].in = L->A_gu; pj.job[2].out = PF(Agu32); pj.job[2].rows = 2 * r; pj.job[2].cols = m.H;
+    SOUP_TRY(lora_prep(pj, st));
     SOUP_TRY(lora_down_tf32(PF(x1_32), T, m.H, PF(A32), 3 * r, m.s, P(u_qkv), PF(u32), m.ldT, st, SW));
   }
   {
@@ -398,7 +390,6 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
   SOUP_TRY(attention_fwd(qkvp, m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(attn), PF(lse), st,
                          recompute ? P(attn16) : nullptr, on ? PF(attn32) : nullptr));
   if (on) {
-    SOUP_TRY(bf16_to_f32(L->A_o, (size_t)r * m.o_in, PF(Ao32), st));
     SOUP_TRY(lora_down_tf32(PF(attn32), T, m.o_in, PF(Ao32), r, m.s, P(u_o), PF(uo32), m.ldT, st, SW));
   }
   {
@@ -413,7 +404,6 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
   SOUP_TRY(rmsnorm_fwd(nullptr, PF(h2), W->norm2, T, m.H, c->eps, P(x2), PF(rinv2), st, on ? PF(x2_32) : nullptr));
   if (on) {
     // u_gu from the unrounded x2 (tf32), with its rounding residual for dB
-    SOUP_TRY(bf16_to_f32(L->A_gu, (size_t)2 * r * m.H, PF(Agu32), st));
     SOUP_TRY(lora_down_tf32(PF(x2_32), T, m.H, PF(Agu32), 2 * r, m.s, P(u_gu), nullptr, m.ldT, st, SW, P(u_gu_lo)));
   }
   {
@@ -515,13 +505,33 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
   SOUP_TRY(forward(W, L, cfg, m, ws, base, h_in, nullptr, on, true, st, nullptr, kept));
   const uint16_t* qkvp = kept ? kept : P(qkv);
 
+  // ---- B factors for the g GEMMs, one launch: B_down^T and B_o^T (fp32),
+  // block-diagonal transposes of B_qkv (fp32, 3 segments) and B_gu (bf16,
+  // 2 segments), so each g = s dy B is one GEMM over all its segments
+  if (on) {
+    PrepJobs pj;
+    pj.njobs = 4;
+    PrepJob& a = pj.job[0];
+    a.kind = PREP_BLOCKDIAG_T; a.in = L->B_down; a.out = PF(Bt_down32); a.N = H; a.r = r;
+    PrepJob& b = pj.job[1];
+    b.kind = PREP_BLOCKDIAG_T; b.in = L->B_o; b.out = PF(Bt_o32); b.N = H; b.r = r;
+    PrepJob& c = pj.job[2];
+    c.kind = PREP_BLOCKDIAG_T; c.in = L->B_qkv; c.out = PF(Bbd_qkv32); c.N = m.qkv_w; c.r = r; c.nseg = 3;
+    c.seg_end[0] = m.Hq * m.d; c.seg_end[1] = (m.Hq + m.Hkv) * m.d; c.seg_end[2] = m.qkv_w;
+    PrepJob& d = pj.job[3];
+    d.kind = PREP_BLOCKDIAG_T; d.out_bf16 = 1; d.in = L->B_gu; d.out = P(Bbd_gu); d.N = 2 * I; d.r = r; d.nseg = 2;
+    d.seg_end[0] = I; d.seg_end[1] = 2 * I;
+    SOUP_TRY(lora_prep(pj, st));
+  }
+
   // ---- MLP block
   SOUP_TRY(f32_to_bf16(dh_out, (size_t)T * H, P(dh_b), st));
   // LoRA gradients of the MLP: g_down from the fp32 dh (tf32), the others
   // from hi + lo (rounding residual) operand pairs, so no operand of a
   // LoRA-gradient GEMM carries more than the bf16 rounding of d_gu
   if (on)
-    SOUP_TRY(lora_g_tf32(dh_out, H, T, H, L->B_down, r, m.s, PF(Bt32), P(g_d), nullptr, ldT, st, SW, P(g_d_lo)));
+    SOUP_TRY(lora_g_prepared(dh_out, nullptr, H, T, H, PF(Bt_down32), r, m.s, true, P(g_d), nullptr, P(g_d_lo), ldT,
+                             st, SW));
   // d_gu = SwiGLU backward of (dh W_down + g' A_down), fused in the epilogue
   SOUP_TRY(proj_bwd(&W->down, P(dh_b), T, P(g_d), ldT, r, on ? L->A_down : nullptr, on, P(d_gu), st, OUT_BF16, I,
                     P(gu16), nullptr, nullptr, on ? P(d_gu_lo) : nullptr));
@@ -530,12 +540,9 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
     SOUP_TRY(lora_dA_dual(P(g_d), P(g_d_lo), r, ldT, P(act), T, I, G->dA_down, st, SW));
   }
   uint16_t* d_gu = P(d_gu);
-  if (on) {
-    for (int sg = 0; sg < 2; ++sg)
-      SOUP_TRY(lora_g(d_gu + (size_t)sg * I, 2 * I, T, I, L->B_gu + (size_t)sg * I * r, r, m.s, P(Bt),
-                      P(g_gu) + (size_t)sg * r * ldT, ldT, st, SW, nullptr, P(d_gu_lo) + (size_t)sg * I,
-                      PF(g_gu32) + (size_t)sg * r * ldT));
-  }
+  if (on)  // g_gate | g_up in one GEMM (block-diagonal B_gu^T), d_gu hi + lo
+    SOUP_TRY(lora_g_prepared(d_gu, P(d_gu_lo), 2 * I, T, 2 * I, P(Bbd_gu), 2 * r, m.s, false, P(g_gu), PF(g_gu32),
+                             nullptr, ldT, st, SW));
   SOUP_TRY(proj_bwd(&W->gate_up, d_gu, T, P(g_gu), ldT, 2 * r, on ? L->A_gu : nullptr, on, P(dx2), st));
   if (on) {
     for (int sg = 0; sg < 2; ++sg)
@@ -549,7 +556,9 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
                        P(dh2_lo)));
 
   // ---- attention block
-  if (on) SOUP_TRY(lora_g_tf32(PF(dh2), H, T, H, L->B_o, r, m.s, PF(Bt32), P(g_o), PF(go32), ldT, st, SW));
+  if (on)
+    SOUP_TRY(lora_g_prepared(PF(dh2), nullptr, H, T, H, PF(Bt_o32), r, m.s, true, P(g_o), PF(go32), nullptr, ldT, st,
+                             SW));
   // dO for the attention backward: from the fp32-accurate dh2 (hi + lo parts),
   // stored fp16 scaled by a power of two derived from max |dh2|
   SOUP_TRY(proj_bwd(&W->o, P(dh2_b), T, P(g_o), ldT, r, on ? L->A_o : nullptr, on, P(d_attn), st, OUT_F16, 0,
@@ -564,11 +573,9 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
                          PF(sinb), gamax, st, on ? PF(dqkv32) : nullptr));
   const int seg_n[3] = {m.Hq * m.d, m.Hkv * m.d, m.Hkv * m.d};
   const int seg_c[3] = {0, m.Hq * m.d, (m.Hq + m.Hkv) * m.d};
-  if (on) {
-    for (int sg = 0; sg < 3; ++sg)
-      SOUP_TRY(lora_g_tf32(PF(dqkv32) + seg_c[sg], m.qkv_w, T, seg_n[sg], L->B_qkv + (size_t)seg_c[sg] * r, r, m.s,
-                           PF(Bt32), P(g_qkv) + (size_t)sg * r * ldT, PF(g32) + (size_t)sg * r * ldT, ldT, st, SW));
-  }
+  if (on)  // g_q | g_k | g_v in one GEMM (block-diagonal B_qkv^T)
+    SOUP_TRY(lora_g_prepared(PF(dqkv32), nullptr, m.qkv_w, T, m.qkv_w, PF(Bbd_qkv32), 3 * r, m.s, true, P(g_qkv),
+                             PF(g32), nullptr, ldT, st, SW));
   SOUP_TRY(proj_bwd(&W->qkv, P(d_qkv), T, P(g_qkv), ldT, 3 * r, on ? L->A_qkv : nullptr, on, P(dx1), st));
   if (on) {
     for (int sg = 0; sg < 3; ++sg)
