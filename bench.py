@@ -33,6 +33,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -90,11 +91,10 @@ class ClockSampler:
     def __init__(self, dev):
         self.dev = dev
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{dev}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"soup_bench_clocks_{os.getpid()}_{dev}.csv")
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,"

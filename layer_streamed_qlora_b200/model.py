@@ -108,6 +108,18 @@ class SyntheticWeights:
         return {k: _randn(s, _seed(self.seed, l, k), 0.02).to(torch.bfloat16) for k, s in shapes.items()}
 
 
+def kept_layer_count(n_layers: int, per_layer: int, arena: int, reserve: int, cap: int) -> int:
+    """How many layers' q|k|v (per_layer bytes each) can be kept while
+    soup_stream_plan still admits the model: arena (slots + vocab slot) +
+    reserve + kept <= cap; all layers without a cap."""
+    if per_layer <= 0:
+        return 0
+    if not cap:
+        return n_layers
+    room = cap - arena - reserve
+    return max(0, min(n_layers, room // per_layer))
+
+
 class StreamedLoRAModel:
     """Frozen base in pinned host blobs + a soup_plan slot ring + resident LoRA.
 
@@ -130,9 +142,8 @@ class StreamedLoRAModel:
         # device cap still admits the plan with it
         # (layers 0 .. n_keep-1: as many as fit)
         per = L.soup_decoder_layer_keep_bytes(self.lcfg, batch, seq)
-        n_keep = cfg.n_layers
-        while n_keep > 0 and not self._plan_fits(device_cap_bytes, self.reserve_bytes + n_keep * per):
-            n_keep -= 1
+        n_keep = kept_layer_count(cfg.n_layers, per, self.n_buffers * self.blob_bytes + self.vocab_bytes,
+                                  self.reserve_bytes, device_cap_bytes)
         self.keep = None
         if per and n_keep:
             self.keep = torch.empty((n_keep, per // 2), dtype=torch.float16, device="cuda")
@@ -143,13 +154,6 @@ class StreamedLoRAModel:
         # When set to a dict, the backward pass stores dL/d(layer input) of
         # every layer in it (index l = input of layer l, n_layers = head output).
         self.capture_dh = None
-
-    def _plan_fits(self, cap: int, reserve: int) -> bool:
-        """Whether soup_stream_plan would admit this model with `reserve`
-        bytes of other device memory (slots + vocab slot + reserve <= cap)."""
-        if not cap:
-            return True
-        return self.n_buffers * self.blob_bytes + self.vocab_bytes + reserve <= cap
 
     # ------------------------------------------------------------ shard build
     def _build_blobs(self, weights):

@@ -13,7 +13,7 @@ Qwen2.5 shape of the workloads:
   a   = silu(LoRA_gate(x2)) * LoRA_up(x2)
   out = h2 + LoRA_down(a)
 
-Readings (the pages are silent; listed in the design doc): RMSNorm
+Readings (where the pages are silent): RMSNorm
 y = x / sqrt(mean(x^2) + eps) * w with frozen w; RoPE is the rotate-half form
 pairing (i, i + d/2) with inv_freq_i = theta^(-2i/d), no frequency rescaling,
 positions restarting at 0 in every sequence; attention scale 1/sqrt(d), causal

@@ -5,7 +5,7 @@ Follows the pages' ``quantization: 4bit`` (NF4) frozen base (Soup pages,
 NF4) with the data type defined by QLoRA (Dettmers et al. 2023, section 3,
 "4-bit NormalFloat quantization"; the 16 values are the ones listed in that
 paper's appendix on the NF4 data type).  The pages do not print the
-codebook; the readings below are this build's and are listed in the design doc.
+codebook; the readings below fill what they leave open.
 
 Readings
   * block = 64 consecutive elements along the input dimension of a row;

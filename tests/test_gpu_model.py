@@ -4,7 +4,7 @@ reduced depth and width, plus the pages' bit-exactness protocol: streamed runs
 (stream_buffers 2, 4, 8 and an all-resident ring) give the same bits.
 
 Deep stacks compound bf16 rounding layer after layer, so (reading of the
-comparison protocol, listed in the design doc) every layer is checked against the
+comparison protocol) every layer is checked against the
 oracle fed the GPU's own bf16 layer input and fp32 upstream gradient, the head
 against the oracle on the GPU's final hidden state, and the DPO loss against
 the DPO formula on the GPU's own sequence sums, each within relative Frobenius

@@ -63,3 +63,16 @@ def test_blob_layout_sizes_match_the_shapes():
     assert v.norm2 + 4096 * 2 <= nf4
     cq = L.layer_cfg(ss.QWEN3B_LAYER)
     assert abs(L.soup_layer_blob_bytes(cq, L.SOUP_WEIGHT_BF16) - 154_148_864) < 10 * 256
+
+
+def test_kept_layer_count_respects_the_device_cap():
+    from layer_streamed_qlora_b200.model import kept_layer_count
+    per = 25_165_824  # q|k|v of an 8B layer at 2048 tokens, fp16
+    arena = 2 * 122_700_000 + 1_050_700_000
+    assert kept_layer_count(32, per, arena, 2_000_000_000, 0) == 32          # no cap: every layer
+    assert kept_layer_count(32, per, arena, 2_000_000_000, 1 << 32) == 32    # 4 GiB: all fit
+    k = kept_layer_count(32, per, arena, 2_000_000_000, 4_000_000_000)       # 4e9 bytes: some
+    assert 0 < k < 32 and arena + 2_000_000_000 + k * per <= 4_000_000_000
+    assert arena + 2_000_000_000 + (k + 1) * per > 4_000_000_000
+    assert kept_layer_count(32, per, arena, 3_000_000_000, 4_000_000_000) == 0  # no room
+    assert kept_layer_count(32, 0, arena, 0, 0) == 0
