@@ -137,12 +137,14 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_sample_seconds(w, tokens=256, reps=1):
     """Times the CPU oracle (fp64 numpy) on one decoder layer of the workload's
-    shape: forward + backward for `tokens` tokens of one sequence.  Weights are
-    random fp64 (their preparation is not timed)."""
+    shape: forward + backward for `tokens` tokens of one sequence, then the
+    AdamW step over that layer's LoRA factors.  Weights are random fp64 (their
+    preparation is not timed).  Returns (layer seconds, AdamW seconds)."""
     import numpy as np
 
     import soup_synth as ss
     from oracle.layer import layer_bwd, layer_fwd
+    from oracle.optim import adamw_step
     shape = ss.LayerShape(hidden=w["hidden"], n_q_heads=w["n_q_heads"], n_kv_heads=w["n_kv_heads"],
                           head_dim=w["head_dim"], intermediate=w["intermediate"], rank=w["rank"], alpha=w["alpha"])
     g = np.random.default_rng(0)
@@ -153,15 +155,29 @@ def oracle_sample_seconds(w, tokens=256, reps=1):
     for p in ss.PROJ_NAMES:
         o, i = shape.proj_shape(p)
         lora[p] = (g.standard_normal((shape.rank, i)) * 0.02, g.standard_normal((o, shape.rank)) * 0.02)
+    moments = {p: [(np.zeros_like(a), np.zeros_like(a)) for a in lora[p]] for p in ss.PROJ_NAMES}
     h = g.standard_normal((1, tokens, shape.hidden))
     dh = g.standard_normal(h.shape)
-    times = []
+    times, adam = [], []
     for _ in range(reps):
         t0 = time.perf_counter()
         _, cache = layer_fwd(h, W, lora, shape)
-        layer_bwd(cache, W, lora, shape, dh)
-        times.append(time.perf_counter() - t0)
-    return min(times)
+        _, grads = layer_bwd(cache, W, lora, shape, dh)
+        t1 = time.perf_counter()
+        for p in ss.PROJ_NAMES:
+            for j in range(2):
+                m, v = moments[p][j]
+                adamw_step(lora[p][j], grads[p][j], m, v, 1, 5e-4)
+        times.append(t1 - t0)
+        adam.append(time.perf_counter() - t1)
+    return min(times), min(adam)
+
+
+def oracle_seconds_per_token(w, t_layer, t_adam, tokens):
+    """Oracle time per token of the whole stack: the layer sample covers
+    `tokens` tokens, the AdamW step one optimiser step of the workload's
+    batch * seq tokens."""
+    return (t_layer / tokens + t_adam / (w["batch"] * w["seq"])) * w["n_layers"]
 
 
 def blas_threads():
@@ -173,11 +189,12 @@ def blas_threads():
 
 
 def cpu_baseline(w, tokens=256):
-    t = oracle_sample_seconds(w, tokens)
-    per_token_stack = t * w["n_layers"] / tokens
+    t, ta = oracle_sample_seconds(w, tokens)
+    per_token_stack = oracle_seconds_per_token(w, t, ta, tokens)
     return {"value": 1.0 / per_token_stack, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"one {w['hidden']}-hidden decoder layer, fwd+bwd on 1x{tokens} tokens in fp64 numpy "
-                      f"({t:.2f} s), projected to the {w['n_layers']}-layer stack (head excluded)"}
+            "sample": f"one {w['hidden']}-hidden decoder layer, fwd+bwd on 1x{tokens} tokens ({t:.2f} s) and the "
+                      f"AdamW step of its LoRA factors ({ta:.3f} s, per {w['batch'] * w['seq']}-token step) in "
+                      f"fp64 numpy, projected to the {w['n_layers']}-layer stack (head excluded)"}
 
 
 def bench_config(w, name, world, kept_layers=None):
@@ -185,7 +202,8 @@ def bench_config(w, name, world, kept_layers=None):
            "base": w["kind"], "stream_buffers": w["buffers"], "device_cap_gb": w["cap_gb"],
            "device_cap_bytes": int(w["cap_gb"] * (1 << 30)),
            "parallelism": f"dp{world}" if world > 1 else "single",
-           "l2": "inputs larger than L2 (the streamed base, >4 GB per step)"}
+           "l2": "inputs larger than L2 (the streamed base, >4 GB per step)",
+           "optimizer": "AdamW on the LoRA adapters every step (lr 5e-4, fp32 master + moments)"}
     if kept_layers is not None:
         cfg["kept_qkv_layers"] = kept_layers
     return cfg
@@ -200,16 +218,18 @@ def run_reference(args, w, name):
         oracle_sample_seconds(w, tokens)
     per = []
     for _ in range(args.steps):
-        per.append(oracle_sample_seconds(w, tokens))
-    t = statistics.median(per)
-    value = tokens / (t * w["n_layers"])
+        t, ta = oracle_sample_seconds(w, tokens)
+        per.append(oracle_seconds_per_token(w, t, ta, tokens))
+    per_token = statistics.median(per)
+    value = 1.0 / per_token
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": t * w["n_layers"] * 1e3, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": per_token * tokens * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": bench_config(w, name, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"per step: one decoder layer fwd+bwd on 1x{tokens} tokens, fp64 numpy, "
-                                       f"projected to {w['n_layers']} layers"},
+                             "sample": f"per step: one decoder layer fwd+bwd on 1x{tokens} tokens and the AdamW "
+                                       f"step of its LoRA factors, fp64 numpy, projected to {w['n_layers']} "
+                                       f"layers"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -316,8 +336,10 @@ def main():
     def step():
         loss = model.sft_step() if w["task"] == "sft" else model.dpo_step(w["prompt"], w["beta"])
         # data parallel: the one exchange of the step, the LoRA gradients
-        # averaged in place (a no-op on one rank)
-        dp.allreduce_mean_(model.grad_flat)
+        # summed in place (a no-op on one rank); the optimiser step takes the
+        # mean's 1/world as its gradient scale
+        world_ = dp.allreduce_sum_(model.grad_flat)
+        model.optimizer_step(grad_scale=1.0 / world_)
         return loss
 
     for _ in range(max(3, args.warmup)):

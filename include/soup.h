@@ -387,6 +387,35 @@ soup_status soup_dpo_loss(const float* logp_policy, const float* logp_ref, int64
                           int64_t prompt_len, float beta, float* loss, float* seq_sums, float* coef,
                           void* stream);
 
+/* ---------------------------------------------------------------- AdamW ---
+ * One AdamW step over the LoRA adapters, which stay resident in device memory
+ * with their gradients and optimiser state while the base streams (Soup
+ * pages, "how layer streaming works").  AdamW is Adam with decoupled weight
+ * decay (Loshchilov & Hutter, "Decoupled Weight Decay Regularization", ICLR
+ * 2019), the decay folded into the learning rate.  For i < n, with
+ * g = grad_scale * grad[i]:
+ *   theta <- theta * (1 - lr * weight_decay)
+ *   m     <- beta1 * m + (1 - beta1) * g
+ *   v     <- beta2 * v + (1 - beta2) * g^2
+ *   theta <- theta - (lr / (1 - beta1^t)) * m / (sqrt(v) / sqrt(1 - beta2^t) + eps)
+ * theta (the fp32 master copy), m, v: fp32 [n], updated in place.  grad:
+ * fp32 [n], read, then set to zero when zero_grad != 0 (a backward pass that
+ * accumulates can then run straight into it).  theta_bf16 (optional, NULL to
+ * skip): bf16 [n] <- round-to-nearest-even of the new theta, the working copy
+ * the GEMMs read.  t >= 1 is this step's index; the bias corrections are
+ * formed on the host in double.  grad_scale multiplies the incoming gradient
+ * (1/world when it arrives as a data-parallel sum).  nonfinite_dev (optional):
+ * a device int32 set to 1 when a gradient element is NaN or Inf (the update
+ * is still applied; the call never clears it).
+ * Errors: SOUP_ERR_ALIGN unless theta, grad, m, v are 16-byte and theta_bf16
+ * 8-byte aligned; SOUP_ERR_INVALID_ARG for t < 1, a beta outside [0, 1),
+ * eps <= 0, or a negative lr / weight_decay.  n = 0 is a no-op.  One kernel
+ * launch, asynchronous on `stream`; the caller owns every buffer. */
+soup_status soup_adamw_step(float* theta, uint16_t* theta_bf16, float* grad, float* m, float* v, int64_t n,
+                            float lr, float beta1, float beta2, float eps, float weight_decay,
+                            float grad_scale, int64_t t, int32_t zero_grad, int32_t* nonfinite_dev,
+                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -129,6 +129,8 @@ _SIGS = {
     "soup_ce_loss": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
     "soup_dpo_loss": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_float, c_void_p, c_void_p,
                                 c_void_p, c_void_p]),
+    "soup_adamw_step": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_float, c_float,
+                                  c_float, c_float, c_float, c_float, c_int64, c_int32, c_void_p, c_void_p]),
 }
 
 _lib = None
@@ -383,3 +385,15 @@ def soup_ce_loss(logp, batch, seq, loss, coef, stream=None):
 def soup_dpo_loss(logp_policy, logp_ref, pairs, seq, prompt_len, beta, loss, seq_sums, coef, stream=None):
     _check("soup_dpo_loss", lib().soup_dpo_loss(_p(logp_policy), _p(logp_ref), pairs, seq, prompt_len, beta,
                                                 _p(loss), _p(seq_sums), _p(coef), _stream(stream)))
+
+
+def soup_adamw_step(theta, theta_bf16, grad, m, v, lr, beta1, beta2, eps, weight_decay, grad_scale, t,
+                    zero_grad=True, nonfinite=None, stream=None):
+    """One AdamW step over flat fp32 buffers (theta, grad, m, v of equal
+    length; theta_bf16 the bf16 working copy or None)."""
+    n = theta.numel()
+    for x in (grad, m, v) + (() if theta_bf16 is None else (theta_bf16,)):
+        assert x.numel() == n and x.is_contiguous()
+    _check("soup_adamw_step", lib().soup_adamw_step(_p(theta), _p(theta_bf16), _p(grad), _p(m), _p(v), n, lr, beta1,
+                                                    beta2, eps, weight_decay, grad_scale, t, 1 if zero_grad else 0,
+                                                    _p(nonfinite), _stream(stream)))

@@ -3,19 +3,22 @@
 One process per GPU: every rank streams its own copy of the frozen base over
 its own host link and runs its own micro-batch through the whole step; the
 LoRA gradients, the only trained state, are averaged across ranks once per
-step.  They live in one flat fp32 buffer (each factor a 256-byte-aligned view
-into it), so the exchange is a single in-place all-reduce of that buffer.
+step.  They live in one flat fp32 buffer (each factor a view into it that
+starts on a 512-byte boundary, 256 bytes for the bf16 working copies laid out
+the same way), so the exchange is a single in-place all-reduce of that buffer;
+the 1/world of the mean can be left to the optimiser step (its gradient
+scale), which reads the buffer anyway.
 """
 from __future__ import annotations
 
 import torch
 
-ALIGN = 64  # elements (256 bytes)
+ALIGN = 128  # elements (512 bytes of fp32, 256 of bf16)
 
 
 def flat_layout(shapes):
     """Offsets (in elements) of tensors of the given shapes packed in order,
-    each starting on a 256-byte boundary, and the total length."""
+    each starting on a multiple of ALIGN elements, and the total length."""
     offs, n = [], 0
     for sh in shapes:
         offs.append(n)
@@ -51,3 +54,17 @@ def allreduce_mean_(flat: torch.Tensor, group=None) -> torch.Tensor:
         dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
         flat.mul_(1.0 / world)
     return flat
+
+
+def allreduce_sum_(flat: torch.Tensor, group=None) -> int:
+    """Sum `flat` over the process group in place (one all-reduce) and return
+    the group's size, so that the caller can fold the 1/world of the mean into
+    its next pass over the buffer.  Returns 1 without touching `flat` when
+    torch.distributed is not initialised or the group has a single rank."""
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized():
+        return 1
+    world = dist.get_world_size(group)
+    if world > 1:
+        dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    return world

@@ -6,13 +6,14 @@ into per-layer shards held in pinned host RAM; a ring of `stream_buffers`
 stream works on the previous layer; the vocab-sized embed_tokens / lm_head
 share one slot; every layer is read once for the forward pass and once more
 for the checkpoint-recompute backward (layers still resident in the ring at
-the turn-around are not copied again); only the LoRA adapters (and their
-gradients) live in VRAM permanently.
+the turn-around are not copied again); only the LoRA adapters, their
+gradients and their AdamW state live in VRAM permanently.
 
 This module is host-side orchestration only: device memory comes from
 PyTorch, and every operation of the step (NF4 quantisation of the shards,
-embedding, the decoder layers forward and backward, the chunked output head
-and the losses) runs in the CUDA library through its C ABI (``_lib``).
+embedding, the decoder layers forward and backward, the chunked output head,
+the losses and the AdamW update) runs in the CUDA library through its C ABI
+(``_lib``).
 """
 from __future__ import annotations
 
@@ -108,6 +109,18 @@ class SyntheticWeights:
         return {k: _randn(s, _seed(self.seed, l, k), 0.02).to(torch.bfloat16) for k, s in shapes.items()}
 
 
+@dataclass(frozen=True)
+class AdamW:
+    """AdamW hyperparameters for the adapters.  The Soup pages' run sets only
+    the learning rate (5e-4); the rest are the defaults of the Trainer those
+    pages run on (betas 0.9 / 0.999, eps 1e-8, no weight decay)."""
+    lr: float = 5e-4
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    weight_decay: float = 0.0
+
+
 def kept_layer_count(n_layers: int, per_layer: int, arena: int, reserve: int, cap: int) -> int:
     """How many layers' q|k|v (per_layer bytes each) can be kept while
     soup_stream_plan still admits the model: arena (slots + vocab slot) +
@@ -129,8 +142,9 @@ class StreamedLoRAModel:
     """
 
     def __init__(self, cfg: ModelConfig, batch: int, seq: int, n_buffers: int = 2, device_cap_bytes: int = 0,
-                 head_chunk: int = 256, weights=None, seed: int = 0):
+                 head_chunk: int = 256, weights=None, seed: int = 0, adamw: AdamW | None = None):
         self.cfg, self.batch, self.seq, self.n_buffers = cfg, batch, seq, n_buffers
+        self.adamw = adamw or AdamW()
         self.T = batch * seq
         self.head_chunk = head_chunk
         self.lcfg = cfg.layer_cfg()
@@ -209,13 +223,29 @@ class StreamedLoRAModel:
         cfg, T = self.cfg, self.T
         before = torch.cuda.memory_allocated()
         self.final_norm = weights.final_norm().contiguous()
-        self.lora = [{k: v.contiguous() for k, v in weights.lora(l).items()} for l in range(cfg.n_layers)]
-        # LoRA gradients: fp32 views into one flat buffer (the data-parallel
-        # exchange all-reduces that buffer in place; see dp.py)
-        keys = [list(lo.keys()) for lo in self.lora]
-        self.grad_flat, views = dp.flat_views([lo[k].shape for lo, ks in zip(self.lora, keys) for k in ks], "cuda")
+        # LoRA factors (bf16, what the GEMMs read), their gradients (fp32),
+        # and the AdamW state (fp32 master copy, first and second moments):
+        # five flat buffers with one layout, each factor a view, so that the
+        # data-parallel exchange is one all-reduce and the optimiser step one
+        # launch over the whole adapter set (see dp.py)
+        init = [weights.lora(l) for l in range(cfg.n_layers)]
+        keys = [list(lo.keys()) for lo in init]
+        shapes = [lo[k].shape for lo, ks in zip(init, keys) for k in ks]
+        self.lora_flat, lviews = dp.flat_views(shapes, "cuda", torch.bfloat16)
+        it = iter(lviews)
+        self.lora = [{k: next(it) for k in ks} for ks in keys]
+        for lo, src in zip(self.lora, init):
+            for k, v in lo.items():
+                v.copy_(src[k])
+        del init
+        self.grad_flat, views = dp.flat_views(shapes, "cuda")
         it = iter(views)
         self.grads = [{"d" + k: next(it) for k in ks} for ks in keys]
+        self.master_flat = self.lora_flat.float()
+        self.adam_m = torch.zeros_like(self.grad_flat)
+        self.adam_v = torch.zeros_like(self.grad_flat)
+        self.adam_t = 0
+        self.nonfinite = torch.zeros(1, dtype=torch.int32, device="cuda")
         self.lora_s = [L.layer_lora(lo) for lo in self.lora]
         self.grads_s = [L.layer_grads(g) for g in self.grads]
         self.ckpt = torch.empty((cfg.n_layers + 1, T, cfg.hidden), dtype=torch.bfloat16, device="cuda")
@@ -329,6 +359,19 @@ class StreamedLoRAModel:
         self._head(self.coef, self.logp, self.dh)
         self._backward_layers()
         return self.loss
+
+    def optimizer_step(self, grad_scale: float = 1.0):
+        """AdamW on every LoRA factor: one kernel launch over the flat buffers
+        updates the fp32 master copy and the moments, rewrites the bf16 factors
+        the next step's GEMMs read, and clears the gradients (the backward pass
+        accumulates into them).  grad_scale multiplies the gradients (1/world
+        after a data-parallel sum).  A non-finite gradient sets
+        self.nonfinite (device) to 1."""
+        o = self.adamw
+        self.adam_t += 1
+        L.soup_adamw_step(self.master_flat, self.lora_flat, self.grad_flat, self.adam_m, self.adam_v, o.lr,
+                          o.beta1, o.beta2, o.eps, o.weight_decay, grad_scale, self.adam_t, zero_grad=True,
+                          nonfinite=self.nonfinite)
 
     def forward_logprobs(self, adapters_on=True):
         """Forward only (no grads): per-token log-probs into self.logp."""

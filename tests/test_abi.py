@@ -57,3 +57,27 @@ def test_library_is_sm100a_only(libpath):
         pytest.skip("cuobjdump unavailable")
     arches = set(re.findall(r"sm_(\d+a?)", out.stdout))
     assert arches == {"100a"}, arches
+
+
+def test_adamw_refuses_bad_arguments_on_the_host(libpath):
+    """soup_adamw_step's argument checks run on the host before any CUDA
+    call: the step index, the hyperparameter ranges and the alignment of
+    every buffer.  The pointers below are never dereferenced."""
+    from layer_streamed_qlora_b200 import _lib
+    f = _lib.lib().soup_adamw_step
+    P = ctypes.c_void_p
+    ok = [P(0x10000), P(0x20000), P(0x30000), P(0x40000), P(0x50000)]  # theta, bf16, grad, m, v
+
+    def call(ptrs=ok, n=1024, lr=1e-3, b1=0.9, b2=0.999, eps=1e-8, wd=0.0, t=1):
+        return f(*ptrs, n, lr, b1, b2, eps, wd, 1.0, t, 1, None, None)
+
+    INVALID, SHAPE, ALIGN = 1, 2, 3
+    assert call(t=0) == INVALID
+    assert call(b1=1.0) == INVALID and call(b2=-0.1) == INVALID
+    assert call(eps=0.0) == INVALID and call(lr=-1e-3) == INVALID and call(wd=-0.1) == INVALID
+    assert call(n=-1) == SHAPE
+    assert call(n=0) == 0  # nothing to do, nothing launched
+    assert call(ptrs=[ok[0], ok[1], P(0x30004), ok[3], ok[4]]) == ALIGN  # grad not 16-byte aligned
+    assert call(ptrs=[ok[0], P(0x20004), ok[2], ok[3], ok[4]]) == ALIGN  # bf16 copy not 8-byte aligned
+    assert call(ptrs=[None] + ok[1:]) == INVALID
+    assert b"soup_adamw_step" in _lib.lib().soup_last_error()

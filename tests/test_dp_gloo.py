@@ -37,21 +37,36 @@ def _rank_main(rank, world, port, q):
         for v in views:
             v.copy_(torch.randn(v.shape, generator=g))
             vals.append(v.clone())
+        summed = flat.clone()
         dp.allreduce_mean_(flat)
+        world_seen = dp.allreduce_sum_(summed)
         # numpy copies: plain pickles (tensors would travel as shared-memory handles)
         q.put((rank, [v.numpy().copy() for v in views], [v.numpy() for v in vals], dp.flat_layout(SHAPES),
-               flat.numpy().copy()))
+               flat.numpy().copy(), summed.numpy().copy(), world_seen))
     finally:
         dist.destroy_process_group()
 
 
 def test_flat_layout_alignment():
     offs, n = dp.flat_layout(SHAPES)
-    assert all(o % 64 == 0 for o in offs)
+    assert all(o % dp.ALIGN == 0 for o in offs) and dp.ALIGN % 128 == 0
     assert n >= sum(a * b for a, b in SHAPES)
+    # fp32 views (gradients, AdamW state) on 512-byte and bf16 views (the
+    # factors the GEMMs read) on 256-byte boundaries, at the same offsets
     flat, views = dp.flat_views(SHAPES, "cpu")
-    for v, sh in zip(views, SHAPES):
-        assert tuple(v.shape) == sh and v.is_contiguous() and (v.data_ptr() - flat.data_ptr()) % 256 == 0
+    flat16, views16 = dp.flat_views(SHAPES, "cpu", torch.bfloat16)
+    assert flat16.numel() == flat.numel()
+    for v, w, sh in zip(views, views16, SHAPES):
+        assert tuple(v.shape) == sh and v.is_contiguous() and (v.data_ptr() - flat.data_ptr()) % 512 == 0
+        assert tuple(w.shape) == sh and w.is_contiguous() and (w.data_ptr() - flat16.data_ptr()) % 256 == 0
+        assert (w.data_ptr() - flat16.data_ptr()) // 2 == (v.data_ptr() - flat.data_ptr()) // 4
+
+
+def test_allreduce_sum_single_process_is_noop():
+    flat, _ = dp.flat_views([(4, 4)], "cpu")
+    flat.fill_(3.0)
+    assert dp.allreduce_sum_(flat) == 1
+    assert torch.all(flat == 3.0)
 
 
 def test_allreduce_mean_single_process_is_noop():
@@ -72,8 +87,8 @@ def test_two_rank_gradient_average():
         p.start()
     res = {}
     for _ in range(world):
-        rank, after, before, layout, gap = q.get(timeout=100)
-        res[rank] = (after, before, layout, gap)
+        rank, after, before, layout, gap, summed, world_seen = q.get(timeout=100)
+        res[rank] = (after, before, layout, gap, summed, world_seen)
     for p in procs:
         p.join(timeout=30)
         assert p.exitcode == 0
@@ -82,8 +97,13 @@ def test_two_rank_gradient_average():
         mean = (res[0][1][i] + res[1][1][i]) / 2
         for r in range(world):
             torch.testing.assert_close(torch.from_numpy(res[r][0][i]), torch.from_numpy(mean), rtol=1e-6, atol=1e-6)
-    # the alignment padding between views stays zero
+    # the sum variant leaves the 1/world to the caller and reports world
     offs, n = dp.flat_layout(SHAPES)
+    for r in range(world):
+        assert res[r][5] == world
+        torch.testing.assert_close(torch.from_numpy(res[r][4]), torch.from_numpy(res[r][3]) * world, rtol=1e-6,
+                                   atol=1e-6)
+    # the alignment padding between views stays zero
     for r in range(world):
         pad = torch.ones(n, dtype=torch.bool)
         for o, (a, b) in zip(offs, SHAPES):
