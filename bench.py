@@ -323,7 +323,7 @@ def main():
     cap = int(w["cap_gb"] * (1 << 30))
     torch.cuda.reset_peak_memory_stats()
     t_build = time.time()
-    model = StreamedLoRAModel(cfg, B, S, n_buffers=w["buffers"], device_cap_bytes=cap, seed=0)
+    model = StreamedLoRAModel(cfg, B, S, n_buffers=w["buffers"], device_cap_bytes=cap, seed=0, task=w["task"])
     t_build = time.time() - t_build
     g = torch.Generator().manual_seed(1000 + rank)
     ids_host = torch.randint(0, cfg.vocab, (B, S), generator=g, dtype=torch.int32).pin_memory()

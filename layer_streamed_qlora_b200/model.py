@@ -142,9 +142,13 @@ class StreamedLoRAModel:
     """
 
     def __init__(self, cfg: ModelConfig, batch: int, seq: int, n_buffers: int = 2, device_cap_bytes: int = 0,
-                 head_chunk: int = 256, weights=None, seed: int = 0, adamw: AdamW | None = None):
+                 head_chunk: int = 256, weights=None, seed: int = 0, adamw: AdamW | None = None,
+                 task: str = "sft"):
         self.cfg, self.batch, self.seq, self.n_buffers = cfg, batch, seq, n_buffers
         self.adamw = adamw or AdamW()
+        if task not in ("sft", "dpo"):
+            raise ValueError(f"task must be 'sft' or 'dpo', not {task!r}")
+        self.task = task
         self.T = batch * seq
         self.head_chunk = head_chunk
         self.lcfg = cfg.layer_cfg()
@@ -260,6 +264,11 @@ class StreamedLoRAModel:
         self.loss = torch.zeros(1, dtype=torch.float32, device="cuda")
         self.seq_sums = torch.zeros(4 * max(1, self.batch // 2), dtype=torch.float32, device="cuda")
         self.ids = torch.empty((self.batch, self.seq), dtype=torch.int32, device="cuda")
+        # DPO: running hidden state of the adapters-off reference pass, which
+        # shares each layer visit with the policy's forward pass (ping-pong)
+        self.h_ref = None
+        if self.task == "dpo":
+            self.h_ref = torch.empty((2, T, cfg.hidden), dtype=torch.bfloat16, device="cuda")
         self.reserve_bytes = torch.cuda.memory_allocated() - before
 
     def views(self, base: int) -> L.LayerWeights:
@@ -298,11 +307,37 @@ class StreamedLoRAModel:
             if l + N < nl:
                 P.prefetch(l + N)
 
-    def _head(self, coef, logp, dh):
+    def _forward_layers_shared(self):
+        """One visit per layer serves both forward passes of a DPO step: the
+        reference (adapters off) runs from ckpt[0] through the h_ref ping-pong
+        buffers, the policy (adapters on) through the checkpoints, on the same
+        resident copy of the layer.  Same calls on the same inputs as the two
+        separate passes, so the same bits, with one layer read fewer."""
+        P, N, nl = self.plan, self.n_buffers, self.cfg.n_layers
+        for l in range(min(N, nl)):
+            P.prefetch(l)
+        for l in range(nl):
+            base = P.wait(l)
+            w = self.views(base)
+            h_in = self.ckpt[0] if l == 0 else self.h_ref[(l - 1) % 2]
+            L.soup_decoder_layer_fwd(w, self.lora_s[l], self.lcfg, h_in, self.batch, self.seq, self.h_ref[l % 2],
+                                     False, self.ws)
+            if self.keep is not None and l < self.keep.shape[0]:
+                L.soup_decoder_layer_fwd_keep(w, self.lora_s[l], self.lcfg, self.ckpt[l], self.batch, self.seq,
+                                              self.ckpt[l + 1], True, self.keep[l], self.ws)
+            else:
+                L.soup_decoder_layer_fwd(w, self.lora_s[l], self.lcfg, self.ckpt[l], self.batch, self.seq,
+                                         self.ckpt[l + 1], True, self.ws)
+            P.release(l)
+            if l + N < nl:
+                P.prefetch(l + N)
+
+    def _head(self, coef, logp, dh, h=None):
         P = self.plan
         P.prefetch(self.head_item)
         E = P.wait(self.head_item)
-        L.soup_head_fwd_bwd(self.ckpt[self.cfg.n_layers], self.final_norm, E, self.cfg.vocab, self.cfg.hidden,
+        h = self.ckpt[self.cfg.n_layers] if h is None else h
+        L.soup_head_fwd_bwd(h, self.final_norm, E, self.cfg.vocab, self.cfg.hidden,
                             self.ids, self.batch, self.seq, self.cfg.eps, self.head_chunk, coef, logp, dh,
                             self.head_ws)
         P.release(self.head_item)
@@ -347,12 +382,19 @@ class StreamedLoRAModel:
     def dpo_step(self, prompt_len: int, beta: float):
         """One DPO step on self.ids ([2P, seq]: rows 2p chosen, 2p+1 rejected):
         reference pass with adapters off over the same streamed base, policy
-        pass with adapters on, DPO loss, backward through the policy."""
+        pass with adapters on, DPO loss, backward through the policy.  A model
+        built with task="dpo" runs both forward passes in one visit per layer
+        (two layer reads per step instead of three); otherwise they are two
+        streamed passes."""
         pairs = self.batch // 2
         self._embed()
-        self._forward_layers(False)
-        self._head(None, self.logp_ref, None)
-        self._forward_layers(True)
+        if self.h_ref is not None:
+            self._forward_layers_shared()
+            self._head(None, self.logp_ref, None, h=self.h_ref[(self.cfg.n_layers - 1) % 2])
+        else:
+            self._forward_layers(False)
+            self._head(None, self.logp_ref, None)
+            self._forward_layers(True)
         self._head(None, self.logp, None)
         L.soup_dpo_loss(self.logp, self.logp_ref, pairs, self.seq, prompt_len, beta, self.loss, self.seq_sums,
                         self.coef)

@@ -43,9 +43,9 @@ def small_cfg(kind="nf4", tied=False, n_layers=3):
                          alpha=32.0, vocab=512, n_layers=n_layers, kind=kind, tied=tied)
 
 
-def build(cfg, B, S, n_buffers=2, seed=0, chunk=48):
+def build(cfg, B, S, n_buffers=2, seed=0, chunk=48, task="sft"):
     w = NumpyWeights(cfg, seed)
-    m = M.StreamedLoRAModel(cfg, B, S, n_buffers=n_buffers, weights=w, head_chunk=chunk)
+    m = M.StreamedLoRAModel(cfg, B, S, n_buffers=n_buffers, weights=w, head_chunk=chunk, task=task)
     return m, w
 
 
@@ -169,3 +169,35 @@ def test_dpo_step_matches_oracle():
             assert_close(got[p][0], grads[l][p][0], f"e2e L{l} dA_{p}", rel=2e-2, maxrel=5e-2)
             assert_close(got[p][1], grads[l][p][1], f"e2e L{l} dB_{p}", rel=2e-2, maxrel=5e-2)
     m.close()
+
+
+def _dpo_ids(cfg, pairs, P_len, C_len, seed=10):
+    rows = []
+    for p in range(pairs):
+        prompt = ss.uniform_ids(seed + p, "prompt", (P_len,), cfg.vocab)
+        for which in ("chosen", "rejected"):
+            rows.append(np.concatenate([prompt, ss.uniform_ids(seed + p, which, (C_len,), cfg.vocab)]))
+    return np.stack(rows)
+
+
+def test_dpo_shared_visit_equals_two_passes_bit_exact():
+    """task="dpo" runs the reference and the policy forward pass in one visit
+    per layer: the same bits as the two separate streamed passes, with fewer
+    layer copies."""
+    cfg = small_cfg("nf4", False, n_layers=4)
+    pairs, P_len, C_len = 2, 24, 24
+    ids = _dpo_ids(cfg, pairs, P_len, C_len)
+    out = {}
+    for task in ("sft", "dpo"):  # "sft": a model without the shared-visit buffers
+        m, _ = build(cfg, 2 * pairs, P_len + C_len, seed=5, task=task)
+        set_ids(m, ids)
+        m.plan.reset_stats()
+        loss = m.dpo_step(P_len, 0.1).clone()
+        torch.cuda.synchronize()
+        out[task] = (loss, m.logp.clone(), m.logp_ref.clone(), m.seq_sums.clone(), m.grad_flat.clone(),
+                     m.plan.stats()["copies"])
+        m.close()
+    a, b = out["sft"], out["dpo"]
+    for x, y, name in zip(a[:5], b[:5], ("loss", "logp", "logp_ref", "seq_sums", "grads")):
+        assert torch.equal(x, y), name
+    assert b[5] < a[5], (a[5], b[5])
