@@ -289,6 +289,10 @@ def main():
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
     ap.add_argument("--buffers", type=int, default=0, help="override stream_buffers (2..8)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (diagnostics only)")
+    ap.add_argument("--source", default="ram", choices=["ram", "disk"],
+                    help="stream_source: layer shards in pinned RAM, or files read ahead from disk")
+    ap.add_argument("--shard-dir", default="", help="directory for the disk tier's shard files (default: a temp dir)")
+    ap.add_argument("--read-ahead", type=int, default=2, help="stream_read_ahead for the disk tier (1..8)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--probe-gemm", action="store_true",
                     help="run each forward fused NF4 GEMM shape of one layer twice and exit (for an ncu capture)")
@@ -323,7 +327,12 @@ def main():
     cap = int(w["cap_gb"] * (1 << 30))
     torch.cuda.reset_peak_memory_stats()
     t_build = time.time()
-    model = StreamedLoRAModel(cfg, B, S, n_buffers=w["buffers"], device_cap_bytes=cap, seed=0, task=w["task"])
+    shard_dir = None
+    if args.source == "disk":
+        import tempfile
+        shard_dir = args.shard_dir or tempfile.mkdtemp(prefix="soup_shards_")
+    model = StreamedLoRAModel(cfg, B, S, n_buffers=w["buffers"], device_cap_bytes=cap, seed=0, task=w["task"],
+                              stream_source=args.source, shard_dir=shard_dir, read_ahead=args.read_ahead)
     t_build = time.time() - t_build
     g = torch.Generator().manual_seed(1000 + rank)
     ids_host = torch.randint(0, cfg.vocab, (B, S), generator=g, dtype=torch.int32).pin_memory()
@@ -423,7 +432,9 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": bench_config(w, args.workload, world, 0 if model.keep is None else int(model.keep.shape[0])),
+        "config": dict(bench_config(w, args.workload, world, 0 if model.keep is None else int(model.keep.shape[0])),
+                       stream_source=args.source,
+                       **({"read_ahead": args.read_ahead} if args.source == "disk" else {})),
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": ids_host.numel() * 4,
                 "d2h_bytes_per_step": 4},
         "gpu_launches": launches,
@@ -436,6 +447,7 @@ def main():
                    "copy_ms_per_step": copy_ms, "stall_ms_per_step": sstats["stall_ms"] / args.steps,
                    "stall_frac": (sstats["stall_ms"] / args.steps) / ms},
         "gemm_tflops_per_step": step_flops / (ms / 1e3) / 1e12,
+        "disk": model.disk.stats() if model.disk is not None else None,
         "peak_device_bytes": torch.cuda.max_memory_allocated() + sstats["arena_bytes"],
         "build_s": t_build,
         "loss": float(loss_host.item()),
@@ -445,6 +457,9 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     model.close()
+    if shard_dir and not args.shard_dir:
+        import shutil
+        shutil.rmtree(shard_dir, ignore_errors=True)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:

@@ -44,6 +44,7 @@ typedef int32_t soup_status;
 #define SOUP_ERR_OOM_PLAN 5    /* a stream plan does not fit the device cap */
 #define SOUP_ERR_TIMEOUT 6     /* a host wait or a kernel's bounded wait expired */
 #define SOUP_ERR_CUDA 7        /* a CUDA runtime call failed */
+#define SOUP_ERR_IO 8          /* a shard file could not be opened or read */
 
 /* Message describing the last failure on the calling thread ("" if none). */
 const char* soup_last_error(void);
@@ -278,7 +279,8 @@ typedef struct soup_plan soup_plan; /* opaque */
 typedef struct soup_stream_desc {
   int32_t n_layers;
   size_t layer_bytes;              /* bytes of one layer blob (multiple of 256) */
-  const void* const* host_layers;  /* n_layers pinned host blobs */
+  const void* const* host_layers;  /* n_layers pinned host blobs, or NULL when every layer copy
+                                      comes from soup_stream_prefetch_from (disk tier) */
   size_t vocab_bytes;              /* bytes of the vocab slot (0: none; multiple of 256) */
   const void* host_embed;          /* pinned host embed_tokens blob (vocab_bytes) or NULL */
   const void* host_head;           /* pinned host lm_head blob or NULL (tied: same as embed) */
@@ -313,6 +315,20 @@ soup_status soup_stream_plan_free(soup_plan* plan);
  * unreleased item or the item is already held. */
 soup_status soup_stream_prefetch(soup_plan* plan, int32_t item);
 
+/* As soup_stream_prefetch for a layer, but the copy reads `host_src` (a
+ * page-locked buffer of layer_bytes, e.g. a disk-tier staging buffer) and,
+ * when copy_done_event (a cudaEvent_t) is not NULL, records it on the copy
+ * stream once the copy has finished reading host_src.  A layer still
+ * resident in a released slot is reused as by soup_stream_prefetch (no copy,
+ * the event is not recorded).  Layers of a plan made without host_layers
+ * can only be brought in this way. */
+soup_status soup_stream_prefetch_from(soup_plan* plan, int32_t layer, const void* host_src,
+                                      void* copy_done_event);
+
+/* *resident <- 1 if a slot holds `item` (a prefetch of it makes no copy;
+ * while it is still held, a prefetch refuses), else 0.  Host only. */
+soup_status soup_stream_resident(soup_plan* plan, int32_t item, int32_t* resident);
+
 /* Makes `compute_stream` wait (on the device) until the item's copy is done
  * and returns the slot's device address in *slot_dev. */
 soup_status soup_stream_wait(soup_plan* plan, int32_t item, void* compute_stream, void** slot_dev);
@@ -337,6 +353,62 @@ void* soup_stream_copy_stream(soup_plan* plan);
  * `event` (a cudaEvent_t). */
 soup_status soup_stream_debug_fail_next_copy(soup_plan* plan);
 soup_status soup_stream_debug_gate_next_copy(soup_plan* plan, void* event);
+
+/* ------------------------------------------------------------ disk tier ---
+ * The pages' `stream_source: disk` with `stream_read_ahead` (1..8): the
+ * frozen base's per-layer shards are files (one per layer, layer_bytes each,
+ * the blob layout below), read ahead into `read_ahead` host staging buffers
+ * by `io_threads` threads, each read cut into 8 MiB requests (Soup pages,
+ * "how layer streaming works" and the streaming configuration keys).
+ * The reader follows a cyclic layer visit order (soup_disk_schedule: one
+ * training step's visits, e.g. 0..L-1 then L-1..0) and replays the plan's
+ * slot ring (n_slots = stream_buffers, least recently used first) over it, so
+ * it reads only the visits that need a copy.  A consumer that visits layers
+ * in that order calls, for a layer that soup_stream_resident reports absent:
+ * soup_disk_acquire -> soup_stream_prefetch_from(host, event) ->
+ * soup_disk_release.  A staging buffer is refilled only after its
+ * copy-done event has completed.  Visits the consumer passes over are
+ * dropped (stats.skipped); a layer acquired out of order resynchronises the
+ * reader on its next visit: results never depend on the schedule.
+ * flags: SOUP_DISK_PINNED: page-locked staging buffers (cudaHostAlloc) and
+ * one CUDA event per buffer for the copy hand-off (needs a device); without
+ * it, plain page-aligned host memory and no CUDA call at all (host-side use
+ * and tests).  SOUP_DISK_DIRECT: O_DIRECT reads (no page-cache copy), per
+ * file, where the file system accepts them (else buffered reads).
+ * Errors: SOUP_ERR_IO (a file cannot be opened or read; a read error is
+ * reported by the acquire of that visit), SOUP_ERR_SHAPE (a file's size is
+ * not layer_bytes), SOUP_ERR_TIMEOUT (acquire waited timeout_ms), and
+ * SOUP_ERR_INVALID_ARG (out-of-range arguments, a layer not in the
+ * schedule, a layer acquired twice or released without being held). */
+#define SOUP_DISK_PINNED 1
+#define SOUP_DISK_DIRECT 2
+
+typedef struct soup_disk soup_disk; /* opaque */
+
+typedef struct soup_disk_stats_t {
+  int64_t reads;       /* staging buffers filled with a visit that was then acquired or is waiting */
+  int64_t skipped;     /* visits read (or being read) and then passed over */
+  int64_t acquires;
+  uint64_t bytes_read;
+  double read_ms;      /* sum over reads of the time from start to last byte (reads overlap) */
+  double wait_ms;      /* total time acquire calls waited */
+  int32_t direct_files;/* shards read with O_DIRECT */
+} soup_disk_stats_t;
+
+soup_status soup_disk_open(const char* const* paths, int32_t n_layers, size_t layer_bytes, int32_t read_ahead,
+                           int32_t n_slots, int32_t io_threads, int32_t flags, soup_disk** out);
+soup_status soup_disk_close(soup_disk* disk);
+/* Sets the cyclic visit order (layer indices, each < n_layers) and restarts
+ * the reader on it; refused while a staging buffer is held. */
+soup_status soup_disk_schedule(soup_disk* disk, const int32_t* order, int32_t n);
+/* Waits (at most timeout_ms) for the staging buffer of `layer`'s next copied
+ * visit; *host <- its address (layer_bytes valid), *copy_done_event <- the
+ * buffer's cudaEvent_t (NULL without SOUP_DISK_PINNED).  The buffer is held
+ * until soup_disk_release. */
+soup_status soup_disk_acquire(soup_disk* disk, int32_t layer, int32_t timeout_ms, const void** host,
+                              void** copy_done_event);
+soup_status soup_disk_release(soup_disk* disk, int32_t layer);
+soup_status soup_disk_stats(soup_disk* disk, soup_disk_stats_t* out);
 
 /* Layer blob layout (host arithmetic, no device access).  NF4 blob: qkv
  * codes | qkv absmax | o codes | o absmax | gate_up codes | gate_up absmax |

@@ -65,6 +65,14 @@ class StreamStats(ctypes.Structure):
                 ("waits", c_int64), ("stall_ms", ctypes.c_double), ("copy_ms", ctypes.c_double)]
 
 
+class DiskStats(ctypes.Structure):
+    _fields_ = [("reads", c_int64), ("skipped", c_int64), ("acquires", c_int64), ("bytes_read", ctypes.c_uint64),
+                ("read_ms", ctypes.c_double), ("wait_ms", ctypes.c_double), ("direct_files", c_int32)]
+
+
+SOUP_DISK_PINNED, SOUP_DISK_DIRECT = 1, 2
+
+
 class GemmProfile(ctypes.Structure):
     _fields_ = [("launches", c_int64), ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
                 ("bytes", ctypes.c_double)]
@@ -112,6 +120,15 @@ _SIGS = {
     "soup_stream_plan": (c_int32, [ctypes.POINTER(StreamDesc), ctypes.POINTER(c_void_p)]),
     "soup_stream_plan_free": (c_int32, [c_void_p]),
     "soup_stream_prefetch": (c_int32, [c_void_p, c_int32]),
+    "soup_stream_prefetch_from": (c_int32, [c_void_p, c_int32, c_void_p, c_void_p]),
+    "soup_stream_resident": (c_int32, [c_void_p, c_int32, ctypes.POINTER(c_int32)]),
+    "soup_disk_open": (c_int32, [ctypes.POINTER(ctypes.c_char_p), c_int32, c_size_t, c_int32, c_int32, c_int32,
+                                 c_int32, ctypes.POINTER(c_void_p)]),
+    "soup_disk_close": (c_int32, [c_void_p]),
+    "soup_disk_schedule": (c_int32, [c_void_p, ctypes.POINTER(c_int32), c_int32]),
+    "soup_disk_acquire": (c_int32, [c_void_p, c_int32, c_int32, ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p)]),
+    "soup_disk_release": (c_int32, [c_void_p, c_int32]),
+    "soup_disk_stats": (c_int32, [c_void_p, ctypes.POINTER(DiskStats)]),
     "soup_stream_wait": (c_int32, [c_void_p, c_int32, c_void_p, ctypes.POINTER(c_void_p)]),
     "soup_stream_wait_host": (c_int32, [c_void_p, c_int32, c_int32]),
     "soup_stream_release": (c_int32, [c_void_p, c_int32, c_void_p]),
@@ -297,10 +314,19 @@ class Plan:
     """Owns a soup_plan (slot arena + copy stream)."""
 
     def __init__(self, host_layers, layer_bytes, n_buffers, vocab_bytes=0, host_embed=None, host_head=None,
-                 device_cap_bytes=0, reserve_bytes=0):
-        self._arr = (c_void_p * len(host_layers))(*[t.data_ptr() for t in host_layers])
+                 device_cap_bytes=0, reserve_bytes=0, n_layers=None):
+        """host_layers: pinned host blobs, one per layer, or None (then
+        n_layers gives the count and every layer copy comes through
+        prefetch_from, e.g. from a Disk reader)."""
+        if host_layers is None:
+            n = int(n_layers)
+            arr = None
+        else:
+            n = len(host_layers)
+            self._arr = (c_void_p * n)(*[t.data_ptr() for t in host_layers])
+            arr = ctypes.cast(self._arr, ctypes.POINTER(c_void_p))
         self._keep = (host_layers, host_embed, host_head)
-        d = StreamDesc(len(host_layers), layer_bytes, ctypes.cast(self._arr, ctypes.POINTER(c_void_p)), vocab_bytes,
+        d = StreamDesc(n, layer_bytes, arr, vocab_bytes,
                        host_embed.data_ptr() if host_embed is not None else None,
                        host_head.data_ptr() if host_head is not None else None, n_buffers, device_cap_bytes,
                        reserve_bytes)
@@ -321,6 +347,15 @@ class Plan:
 
     def prefetch(self, item):
         _check("soup_stream_prefetch", lib().soup_stream_prefetch(self.h, item))
+
+    def prefetch_from(self, layer, host_ptr: int, copy_done_event=None):
+        _check("soup_stream_prefetch_from", lib().soup_stream_prefetch_from(self.h, layer, c_void_p(host_ptr),
+                                                                            c_void_p(copy_done_event)))
+
+    def resident(self, item) -> bool:
+        r = c_int32(0)
+        _check("soup_stream_resident", lib().soup_stream_resident(self.h, item, ctypes.byref(r)))
+        return bool(r.value)
 
     def wait(self, item, stream=None) -> int:
         p = c_void_p()
@@ -397,3 +432,47 @@ def soup_adamw_step(theta, theta_bf16, grad, m, v, lr, beta1, beta2, eps, weight
     _check("soup_adamw_step", lib().soup_adamw_step(_p(theta), _p(theta_bf16), _p(grad), _p(m), _p(v), n, lr, beta1,
                                                     beta2, eps, weight_decay, grad_scale, t, 1 if zero_grad else 0,
                                                     _p(nonfinite), _stream(stream)))
+
+
+class Disk:
+    """Owns a soup_disk reader: per-layer shard files read ahead into
+    `read_ahead` staging buffers along a cyclic layer visit schedule."""
+
+    def __init__(self, paths, layer_bytes, read_ahead=2, n_slots=2, io_threads=4, pinned=True, direct=True):
+        self._paths = (ctypes.c_char_p * len(paths))(*[os.fsencode(p) for p in paths])
+        flags = (SOUP_DISK_PINNED if pinned else 0) | (SOUP_DISK_DIRECT if direct else 0)
+        h = c_void_p()
+        _check("soup_disk_open", lib().soup_disk_open(self._paths, len(paths), layer_bytes, read_ahead, n_slots,
+                                                      io_threads, flags, ctypes.byref(h)))
+        self.h = h
+        self.layer_bytes = layer_bytes
+
+    def schedule(self, order):
+        arr = (c_int32 * len(order))(*order)
+        _check("soup_disk_schedule", lib().soup_disk_schedule(self.h, arr, len(order)))
+
+    def acquire(self, layer, timeout_ms=60000):
+        """Returns (host address, copy-done cudaEvent_t or None)."""
+        host, ev = c_void_p(), c_void_p()
+        _check("soup_disk_acquire", lib().soup_disk_acquire(self.h, layer, timeout_ms, ctypes.byref(host),
+                                                            ctypes.byref(ev)))
+        return host.value, ev.value
+
+    def release(self, layer):
+        _check("soup_disk_release", lib().soup_disk_release(self.h, layer))
+
+    def stats(self) -> dict:
+        s = DiskStats()
+        _check("soup_disk_stats", lib().soup_disk_stats(self.h, ctypes.byref(s)))
+        return {k: getattr(s, k) for k, _ in DiskStats._fields_}
+
+    def close(self):
+        if self.h:
+            lib().soup_disk_close(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -88,12 +88,14 @@ extern "C" soup_status soup_stream_plan(const soup_stream_desc* d, soup_plan** o
   *out = nullptr;
   SOUP_CHECK(d->n_buffers >= 2 && d->n_buffers <= 8, SOUP_ERR_INVALID_ARG,
              "soup_stream_plan: stream_buffers must be in [2, 8] (got %d)", d->n_buffers);
-  SOUP_CHECK(d->n_layers >= 1 && d->host_layers, SOUP_ERR_INVALID_ARG, "soup_stream_plan: no layers");
+  SOUP_CHECK(d->n_layers >= 1, SOUP_ERR_INVALID_ARG, "soup_stream_plan: no layers");
   SOUP_CHECK(d->layer_bytes > 0 && d->layer_bytes % 256 == 0, SOUP_ERR_ALIGN,
              "soup_stream_plan: layer_bytes must be a positive multiple of 256");
   SOUP_CHECK(d->vocab_bytes % 256 == 0, SOUP_ERR_ALIGN, "soup_stream_plan: vocab_bytes must be a multiple of 256");
-  for (int i = 0; i < d->n_layers; ++i)
-    SOUP_CHECK(d->host_layers[i] != nullptr, SOUP_ERR_INVALID_ARG, "soup_stream_plan: host layer %d is null", i);
+  // host_layers == NULL: every layer copy comes from soup_stream_prefetch_from (disk tier)
+  if (d->host_layers)
+    for (int i = 0; i < d->n_layers; ++i)
+      SOUP_CHECK(d->host_layers[i] != nullptr, SOUP_ERR_INVALID_ARG, "soup_stream_plan: host layer %d is null", i);
   const size_t arena = (size_t)d->n_buffers * d->layer_bytes + d->vocab_bytes;
   if (d->device_cap_bytes > 0) {
     const size_t need = arena + d->reserve_bytes;
@@ -105,7 +107,10 @@ extern "C" soup_status soup_stream_plan(const soup_stream_desc* d, soup_plan** o
   p->n_layers = d->n_layers;
   p->layer_bytes = d->layer_bytes;
   p->vocab_bytes = d->vocab_bytes;
-  p->host_layers.assign(d->host_layers, d->host_layers + d->n_layers);
+  if (d->host_layers)
+    p->host_layers.assign(d->host_layers, d->host_layers + d->n_layers);
+  else
+    p->host_layers.assign(d->n_layers, nullptr);
   p->host_embed = d->host_embed;
   p->host_head = d->host_head;
   p->n_buffers = d->n_buffers;
@@ -162,7 +167,11 @@ extern "C" soup_status soup_stream_plan_free(soup_plan* p) {
   return SOUP_OK;
 }
 
-extern "C" soup_status soup_stream_prefetch(soup_plan* p, int32_t item) {
+namespace {
+
+// src_override: the host bytes of a layer (else the plan's own host copy);
+// done: recorded on the copy stream after the copy (may be null).
+soup_status prefetch_impl(soup_plan* p, int32_t item, const void* src_override, cudaEvent_t done) {
   using namespace soup;
   SOUP_TRY(check_item(p, item));
   int s = slot_of(p, item);
@@ -188,7 +197,12 @@ extern "C" soup_status soup_stream_prefetch(soup_plan* p, int32_t item) {
                "soup_stream_prefetch: the vocab slot holds item %d, not released", p->slots[s].item);
   }
   auto& sl = p->slots[s];
-  const void* src = item >= 0 ? p->host_layers[item] : (item == SOUP_ITEM_EMBED ? p->host_embed : p->host_head);
+  const void* src = src_override ? src_override
+                                  : (item >= 0 ? p->host_layers[item]
+                                               : (item == SOUP_ITEM_EMBED ? p->host_embed : p->host_head));
+  SOUP_CHECK(src, SOUP_ERR_INVALID_ARG,
+             "soup_stream_prefetch: the plan holds no host copy of layer %d (bring it with soup_stream_prefetch_from)",
+             item);
   const size_t bytes = item >= 0 ? p->layer_bytes : p->vocab_bytes;
   if (p->fail_next_copy) {
     p->fail_next_copy = false;
@@ -221,11 +235,34 @@ extern "C" soup_status soup_stream_prefetch(soup_plan* p, int32_t item) {
     SOUP_CUDA_TRY(cudaMemcpyAsync(sl.dev, src, bytes, cudaMemcpyHostToDevice, p->copy));
   }
   SOUP_CUDA_TRY(cudaEventRecord(sl.ready, p->copy));
+  if (done) SOUP_CUDA_TRY(cudaEventRecord(done, p->copy));
   SOUP_CUDA_TRY(cudaEventRecord(ce.second, p->copy));
   sl.item = item;
   sl.pinned = true;
   ++p->copies;
   p->bytes_copied += bytes;
+  return SOUP_OK;
+}
+
+}  // namespace
+
+extern "C" soup_status soup_stream_prefetch(soup_plan* p, int32_t item) {
+  return prefetch_impl(p, item, nullptr, nullptr);
+}
+
+extern "C" soup_status soup_stream_prefetch_from(soup_plan* p, int32_t layer, const void* host_src,
+                                                 void* copy_done_event) {
+  using namespace soup;
+  SOUP_CHECK(layer >= 0 && host_src, SOUP_ERR_INVALID_ARG,
+             "soup_stream_prefetch_from: needs a layer index and a host source");
+  return prefetch_impl(p, layer, host_src, static_cast<cudaEvent_t>(copy_done_event));
+}
+
+extern "C" soup_status soup_stream_resident(soup_plan* p, int32_t item, int32_t* resident) {
+  using namespace soup;
+  SOUP_TRY(check_item(p, item));
+  SOUP_CHECK(resident, SOUP_ERR_INVALID_ARG, "soup_stream_resident: null out");
+  *resident = slot_of(p, item) >= 0 ? 1 : 0;
   return SOUP_OK;
 }
 

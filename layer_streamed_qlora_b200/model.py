@@ -9,6 +9,10 @@ for the checkpoint-recompute backward (layers still resident in the ring at
 the turn-around are not copied again); only the LoRA adapters, their
 gradients and their AdamW state live in VRAM permanently.
 
+With ``stream_source="disk"`` (the pages' disk tier) the per-layer shards are
+files instead, read ahead into ``read_ahead`` page-locked staging buffers by
+the library's shard reader and copied from there.
+
 This module is host-side orchestration only: device memory comes from
 PyTorch, and every operation of the step (NF4 quantisation of the shards,
 embedding, the decoder layers forward and backward, the chunked output head,
@@ -17,6 +21,7 @@ the losses and the AdamW update) runs in the CUDA library through its C ABI
 """
 from __future__ import annotations
 
+import os
 import zlib
 from dataclasses import dataclass
 
@@ -143,8 +148,15 @@ class StreamedLoRAModel:
 
     def __init__(self, cfg: ModelConfig, batch: int, seq: int, n_buffers: int = 2, device_cap_bytes: int = 0,
                  head_chunk: int = 256, weights=None, seed: int = 0, adamw: AdamW | None = None,
-                 task: str = "sft"):
+                 task: str = "sft", stream_source: str = "ram", shard_dir: str | None = None,
+                 read_ahead: int = 2, io_threads: int = 4):
         self.cfg, self.batch, self.seq, self.n_buffers = cfg, batch, seq, n_buffers
+        if stream_source not in ("ram", "disk"):
+            raise ValueError(f"stream_source must be 'ram' or 'disk', not {stream_source!r}")
+        if stream_source == "disk" and not shard_dir:
+            raise ValueError("stream_source='disk' needs a shard_dir for the per-layer shard files")
+        self.stream_source, self.shard_dir = stream_source, shard_dir
+        self.disk = None
         self.adamw = adamw or AdamW()
         if task not in ("sft", "dpo"):
             raise ValueError(f"task must be 'sft' or 'dpo', not {task!r}")
@@ -167,7 +179,16 @@ class StreamedLoRAModel:
             self.keep = torch.empty((n_keep, per // 2), dtype=torch.float16, device="cuda")
             self.reserve_bytes += n_keep * per
         self.plan = L.Plan(self.host_layers, self.blob_bytes, n_buffers, self.vocab_bytes, self.host_embed,
-                           self.host_head, device_cap_bytes, self.reserve_bytes)
+                           self.host_head, device_cap_bytes, self.reserve_bytes, n_layers=cfg.n_layers)
+        if stream_source == "disk":
+            # the pages' disk tier: shards read ahead from files into
+            # read_ahead page-locked staging buffers along the step's visit
+            # order (forward 0..L-1, backward L-1..0; a task="dpo" model's
+            # shared visits follow the same order)
+            self.disk = L.Disk(self.shard_paths, self.blob_bytes, read_ahead=read_ahead, n_slots=n_buffers,
+                               io_threads=io_threads, pinned=True, direct=True)
+            nl = cfg.n_layers
+            self.disk.schedule(list(range(nl)) + list(range(nl - 1, -1, -1)))
         self._views = {}
         # When set to a dict, the backward pass stores dL/d(layer input) of
         # every layer in it (index l = input of layer l, n_layers = head output).
@@ -188,7 +209,12 @@ class StreamedLoRAModel:
             off = ptr - base
             return staging[off:off + nbytes]
 
-        self.host_layers = []
+        disk = self.stream_source == "disk"
+        self.host_layers = None if disk else []
+        self.shard_paths = []
+        if disk:
+            os.makedirs(self.shard_dir, exist_ok=True)
+            hb = torch.empty(self.blob_bytes, dtype=torch.uint8, pin_memory=True)
         for l in range(cfg.n_layers):
             w = weights.layer(l)
             for name in ("qkv", "o", "gate_up", "down"):
@@ -205,9 +231,15 @@ class StreamedLoRAModel:
                     region(sw.w, n * 2).view(torch.bfloat16).copy_(W.reshape(-1).to(torch.bfloat16))
             region(v.norm1, cfg.hidden * 2).view(torch.bfloat16).copy_(w["norm1"].reshape(-1))
             region(v.norm2, cfg.hidden * 2).view(torch.bfloat16).copy_(w["norm2"].reshape(-1))
-            hb = torch.empty(self.blob_bytes, dtype=torch.uint8, pin_memory=True)
-            hb.copy_(staging)
-            self.host_layers.append(hb)
+            if disk:  # one shard file per layer, the blob's bytes
+                hb.copy_(staging)
+                path = os.path.join(self.shard_dir, f"layer_{l:03d}.bin")
+                hb.numpy().tofile(path)
+                self.shard_paths.append(path)
+            else:
+                hb = torch.empty(self.blob_bytes, dtype=torch.uint8, pin_memory=True)
+                hb.copy_(staging)
+                self.host_layers.append(hb)
             del w
         del staging
         V, H = cfg.vocab, cfg.hidden
@@ -290,11 +322,24 @@ class StreamedLoRAModel:
         the vocab slot is left to the lm_head."""
         L.soup_embed(self.host_embed.data_ptr(), self.cfg.vocab, self.cfg.hidden, self.ids, self.T, self.ckpt[0])
 
+    def _prefetch(self, l):
+        """Brings layer l into a slot: from its pinned host blob, or with the
+        disk tier from the reader's staging buffer (a layer still resident in
+        a slot makes no copy either way)."""
+        if self.disk is None or self.plan.resident(l):
+            self.plan.prefetch(l)
+            return
+        host, ev = self.disk.acquire(l)
+        try:
+            self.plan.prefetch_from(l, host, ev)
+        finally:
+            self.disk.release(l)
+
     def _forward_layers(self, adapters_on: bool):
         """ckpt[0] -> ckpt[L], saving every layer input (the checkpoints)."""
         P, N, nl = self.plan, self.n_buffers, self.cfg.n_layers
         for l in range(min(N, nl)):
-            P.prefetch(l)
+            self._prefetch(l)
         for l in range(nl):
             base = P.wait(l)
             if adapters_on and self.keep is not None and l < self.keep.shape[0]:
@@ -305,7 +350,7 @@ class StreamedLoRAModel:
                                          self.seq, self.ckpt[l + 1], adapters_on, self.ws)
             P.release(l)
             if l + N < nl:
-                P.prefetch(l + N)
+                self._prefetch(l + N)
 
     def _forward_layers_shared(self):
         """One visit per layer serves both forward passes of a DPO step: the
@@ -315,7 +360,7 @@ class StreamedLoRAModel:
         separate passes, so the same bits, with one layer read fewer."""
         P, N, nl = self.plan, self.n_buffers, self.cfg.n_layers
         for l in range(min(N, nl)):
-            P.prefetch(l)
+            self._prefetch(l)
         for l in range(nl):
             base = P.wait(l)
             w = self.views(base)
@@ -330,7 +375,7 @@ class StreamedLoRAModel:
                                          self.ckpt[l + 1], True, self.ws)
             P.release(l)
             if l + N < nl:
-                P.prefetch(l + N)
+                self._prefetch(l + N)
 
     def _head(self, coef, logp, dh, h=None):
         P = self.plan
@@ -345,7 +390,7 @@ class StreamedLoRAModel:
     def _backward_layers(self):
         P, N, nl = self.plan, self.n_buffers, self.cfg.n_layers
         for l in range(nl - 1, max(nl - 1 - N, -1), -1):
-            P.prefetch(l)  # the layers still resident from the forward pass are reused, not copied
+            self._prefetch(l)  # the layers still resident from the forward pass are reused, not copied
         for l in range(nl - 1, -1, -1):
             if self.capture_dh is not None:  # inspection hook for layer-by-layer checks
                 self.capture_dh[l + 1] = self.dh.clone()
@@ -359,7 +404,7 @@ class StreamedLoRAModel:
                                          self.batch, self.seq, self.dh, self.grads_s[l], 1, self.ws)
             P.release(l)
             if l - N >= 0:
-                P.prefetch(l - N)
+                self._prefetch(l - N)
         if self.capture_dh is not None:
             self.capture_dh[0] = self.dh.clone()
 
@@ -424,5 +469,8 @@ class StreamedLoRAModel:
 
     def close(self):
         if getattr(self, "plan", None) is not None:
-            self.plan.free()
+            self.plan.free()  # synchronises the copy streams first
             self.plan = None
+        if getattr(self, "disk", None) is not None:
+            self.disk.close()  # staging buffers: no copy reads them any more
+            self.disk = None

@@ -76,3 +76,14 @@ def test_kept_layer_count_respects_the_device_cap():
     assert arena + 2_000_000_000 + (k + 1) * per > 4_000_000_000
     assert kept_layer_count(32, per, arena, 3_000_000_000, 4_000_000_000) == 0  # no room
     assert kept_layer_count(32, 0, arena, 0, 0) == 0
+
+
+def test_plan_without_host_layers_passes_validation():
+    # the disk tier's plan holds no host copies of the layers (they arrive
+    # through soup_stream_prefetch_from); validation accepts a NULL array.
+    # Without a GPU the arena allocation that follows fails with SOUP_ERR_CUDA.
+    d = L.StreamDesc(4, 1 << 20, None, 0, None, None, 2, 0, 0)
+    st, h = _plan_status(d)
+    if st == 0:
+        L.lib().soup_stream_plan_free(h)
+    assert st in (0, 7), L.lib().soup_last_error()
