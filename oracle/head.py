@@ -13,6 +13,10 @@
   where pi_* / ref_* are the summed next-token log-probabilities of the
   chosen / rejected continuation tokens under the policy (adapters on) and the
   reference (adapters off).  Prompt positions are masked out.
+* SimPO and ORPO, the reference-free preference losses the pages name as the
+  ones without DPO's extra reference reads ("memory-free reference model"):
+  SimPO (Meng, Xia & Chen 2024) and ORPO (Hong, Lee & Thorne 2024), both on
+  length-normalised continuation log-likelihoods (see their functions).
 fp64 throughout.
 """
 from __future__ import annotations
@@ -91,3 +95,47 @@ def dpo_loss(pi_c, pi_r, ref_c, ref_r, beta):
     loss = float(np.sum(np.logaddexp(0.0, -z))) / P
     dz = -(0.5 * (1.0 - np.tanh(0.5 * z))) / P        # d/dz softplus(-z) = -sigmoid(-z)
     return loss, beta * dz, -beta * dz
+
+
+def _sigmoid_neg(z):
+    """sigmoid(-z), computed without overflow."""
+    return 0.5 * (1.0 - np.tanh(0.5 * z))
+
+
+def _log1mexp(m):
+    """log(1 - exp(m)) for m < 0 (Maechler's two-branch form, accurate on both
+    sides of m = -log 2)."""
+    m = np.asarray(m, np.float64)
+    return np.where(m > -np.log(2.0), np.log(-np.expm1(m)), np.log1p(-np.exp(m)))
+
+
+def simpo_loss(pi_c, pi_r, n_c, n_r, beta, gamma):
+    """SimPO over P pairs: with the length-normalised sequence log-likelihoods
+    m = pi / n (pi the summed continuation log-probs, n the continuation
+    length),
+      L = -(1/P) sum_p log sigmoid(beta (m_c - m_r) - gamma).
+    Returns (loss, dL/dpi_c [P], dL/dpi_r [P])."""
+    pi_c, pi_r = np.asarray(pi_c, np.float64), np.asarray(pi_r, np.float64)
+    z = beta * (pi_c / n_c - pi_r / n_r) - gamma
+    P = z.shape[0]
+    loss = float(np.sum(np.logaddexp(0.0, -z))) / P
+    dz = -_sigmoid_neg(z) / P
+    return loss, beta * dz / n_c, -beta * dz / n_r
+
+
+def orpo_loss(pi_c, pi_r, n_c, n_r, lam):
+    """ORPO over P pairs: the chosen continuation's mean token NLL plus lam
+    times the odds-ratio term.  With m = pi / n the length-normalised
+    log-likelihood, odds(y) = exp(m) / (1 - exp(m)), so
+    log odds = m - log(1 - exp(m)), and
+      L = (1/P) sum_p [ -m_c - lam log sigmoid(log odds_c - log odds_r) ].
+    Returns (loss, dL/dpi_c [P], dL/dpi_r [P]); d(log odds)/dm = 1 / (1 - exp(m))."""
+    pi_c, pi_r = np.asarray(pi_c, np.float64), np.asarray(pi_r, np.float64)
+    m_c, m_r = pi_c / n_c, pi_r / n_r
+    z = (m_c - _log1mexp(m_c)) - (m_r - _log1mexp(m_r))
+    P = z.shape[0]
+    loss = (float(np.sum(-m_c)) + lam * float(np.sum(np.logaddexp(0.0, -z)))) / P
+    s = _sigmoid_neg(z)
+    dm_c = (-1.0 - lam * s / -np.expm1(m_c)) / P
+    dm_r = (lam * s / -np.expm1(m_r)) / P
+    return loss, dm_c / n_c, dm_r / n_r

@@ -1,4 +1,4 @@
-"""The whole LoRA-adapted stack for one SFT or DPO step
+"""The whole LoRA-adapted stack for one SFT, DPO, SimPO or ORPO step
 (oracle; test infrastructure only).
 
 Streaming (one layer in VRAM at a time, each layer read for the forward pass
@@ -12,7 +12,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .head import ce_loss, dpo_loss, embed, token_logprobs, token_logprobs_bwd
+from .head import ce_loss, dpo_loss, embed, orpo_loss, simpo_loss, token_logprobs, token_logprobs_bwd
 from .layer import layer_bwd, layer_fwd
 
 
@@ -66,9 +66,35 @@ def dpo_step(params, ids, shape, prompt_len, beta):
     ref, _ = seq_logprob_sums(params, ids, shape, prompt_len, adapters_on=False)
     pol, (h, caches, hc, m) = seq_logprob_sums(params, ids, shape, prompt_len, adapters_on=True)
     loss, dc, dr = dpo_loss(pol[0::2], pol[1::2], ref[0::2], ref[1::2], beta)
+    grads, ex = _policy_backward(params, ids, shape, (h, caches, hc, m), dc, dr)
+    return loss, grads, dict(ex, policy=pol, reference=ref)
+
+
+def _policy_backward(params, ids, shape, fwd, dc, dr):
+    """Backward from dL/d(sequence sums) (chosen rows 2p, rejected 2p+1)
+    through the continuation mask, the head and the stack."""
+    h, caches, hc, m = fwd
     dseq = np.empty(ids.shape[0])
     dseq[0::2], dseq[1::2] = dc, dr
     dlogp = dseq[:, None] * m[None, :]
     dh = token_logprobs_bwd(hc, params["final_norm"], params["head"], ids, dlogp)
     grads, _, layer_dout = stack_bwd(params, caches, shape, dh)
-    return loss, grads, dict(policy=pol, reference=ref, dh_top=dh, layer_dout=layer_dout)
+    return grads, dict(dh_top=dh, layer_dout=layer_dout)
+
+
+def simpo_step(params, ids, shape, prompt_len, beta, gamma):
+    """Reference-free: one policy pass.  ids as for dpo_step; every row has
+    S - prompt_len continuation targets."""
+    pol, fwd = seq_logprob_sums(params, ids, shape, prompt_len, adapters_on=True)
+    n = float(fwd[3].sum())
+    loss, dc, dr = simpo_loss(pol[0::2], pol[1::2], n, n, beta, gamma)
+    grads, ex = _policy_backward(params, ids, shape, fwd, dc, dr)
+    return loss, grads, dict(ex, policy=pol)
+
+
+def orpo_step(params, ids, shape, prompt_len, lam):
+    pol, fwd = seq_logprob_sums(params, ids, shape, prompt_len, adapters_on=True)
+    n = float(fwd[3].sum())
+    loss, dc, dr = orpo_loss(pol[0::2], pol[1::2], n, n, lam)
+    grads, ex = _policy_backward(params, ids, shape, fwd, dc, dr)
+    return loss, grads, dict(ex, policy=pol)
