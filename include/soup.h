@@ -459,6 +459,27 @@ soup_status soup_dpo_loss(const float* logp_policy, const float* logp_ref, int64
                           int64_t prompt_len, float beta, float* loss, float* seq_sums, float* coef,
                           void* stream);
 
+/* Reference-free preference losses (the pages name ORPO and SimPO as the
+ * methods without DPO's reference reads: "memory-free reference model").
+ * logp [2*pairs, seq-1] holds the policy's next-token log-probs; rows 2p /
+ * 2p+1 are the chosen / rejected sequence of pair p, sharing a prompt of
+ * prompt_len tokens, so each row has n = seq - max(prompt_len, 1)
+ * continuation targets (positions j with j + 1 >= prompt_len).  With s a
+ * row's summed continuation log-probs and m = s / n:
+ *   SimPO (Meng, Xia & Chen 2024):
+ *     L = -(1/P) sum_p log sigmoid(beta (m_c - m_r) - gamma)
+ *   ORPO (Hong, Lee & Thorne 2024), lo = m - log(1 - exp(m)) the log odds:
+ *     L = (1/P) sum_p [ -m_c - lam log sigmoid(lo_c - lo_r) ]
+ * *loss (device float) <- L; seq_sums (optional, [2*pairs]) <- s per row;
+ * coef [2*pairs, seq-1] <- dL/dlogp (0 on prompt positions).  One kernel
+ * launch; SOUP_ERR_SHAPE unless 1 <= pairs <= 2048, seq >= 2 and
+ * 0 <= prompt_len < seq.  A row whose mean log-likelihood is 0 (probability
+ * 1) has infinite log odds: ORPO is then not finite. */
+soup_status soup_simpo_loss(const float* logp, int64_t pairs, int64_t seq, int64_t prompt_len, float beta,
+                            float gamma, float* loss, float* seq_sums, float* coef, void* stream);
+soup_status soup_orpo_loss(const float* logp, int64_t pairs, int64_t seq, int64_t prompt_len, float lam,
+                           float* loss, float* seq_sums, float* coef, void* stream);
+
 /* ---------------------------------------------------------------- AdamW ---
  * One AdamW step over the LoRA adapters, which stay resident in device memory
  * with their gradients and optimiser state while the base streams (Soup

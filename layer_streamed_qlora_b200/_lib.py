@@ -146,6 +146,10 @@ _SIGS = {
     "soup_ce_loss": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
     "soup_dpo_loss": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_float, c_void_p, c_void_p,
                                 c_void_p, c_void_p]),
+    "soup_simpo_loss": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_float, c_float, c_void_p, c_void_p,
+                                  c_void_p, c_void_p]),
+    "soup_orpo_loss": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_float, c_void_p, c_void_p, c_void_p,
+                                 c_void_p]),
     "soup_adamw_step": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_float, c_float,
                                   c_float, c_float, c_float, c_float, c_int64, c_int32, c_void_p, c_void_p]),
 }
@@ -420,6 +424,16 @@ def soup_ce_loss(logp, batch, seq, loss, coef, stream=None):
 def soup_dpo_loss(logp_policy, logp_ref, pairs, seq, prompt_len, beta, loss, seq_sums, coef, stream=None):
     _check("soup_dpo_loss", lib().soup_dpo_loss(_p(logp_policy), _p(logp_ref), pairs, seq, prompt_len, beta,
                                                 _p(loss), _p(seq_sums), _p(coef), _stream(stream)))
+
+
+def soup_simpo_loss(logp, pairs, seq, prompt_len, beta, gamma, loss, seq_sums, coef, stream=None):
+    _check("soup_simpo_loss", lib().soup_simpo_loss(_p(logp), pairs, seq, prompt_len, beta, gamma, _p(loss),
+                                                    _p(seq_sums), _p(coef), _stream(stream)))
+
+
+def soup_orpo_loss(logp, pairs, seq, prompt_len, lam, loss, seq_sums, coef, stream=None):
+    _check("soup_orpo_loss", lib().soup_orpo_loss(_p(logp), pairs, seq, prompt_len, lam, _p(loss), _p(seq_sums),
+                                                  _p(coef), _stream(stream)))
 
 
 def soup_adamw_step(theta, theta_bf16, grad, m, v, lr, beta1, beta2, eps, weight_decay, grad_scale, t,

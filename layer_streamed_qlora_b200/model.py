@@ -447,6 +447,30 @@ class StreamedLoRAModel:
         self._backward_layers()
         return self.loss
 
+    def _preference_step(self, loss_fn):
+        """Reference-free preference step: one policy pass (two layer reads
+        per step, as for SFT), the loss and dL/dlogp from the sequence sums,
+        then the head's backward and the recompute backward."""
+        self._embed()
+        self._forward_layers(True)
+        self._head(None, self.logp, None)
+        loss_fn()
+        self._head(self.coef, self.logp, self.dh)
+        self._backward_layers()
+        return self.loss
+
+    def simpo_step(self, prompt_len: int, beta: float = 2.0, gamma: float = 1.0):
+        """One SimPO step on self.ids (rows 2p chosen, 2p+1 rejected)."""
+        pairs = self.batch // 2
+        return self._preference_step(lambda: L.soup_simpo_loss(self.logp, pairs, self.seq, prompt_len, beta, gamma,
+                                                               self.loss, self.seq_sums, self.coef))
+
+    def orpo_step(self, prompt_len: int, lam: float = 0.1):
+        """One ORPO step on self.ids (rows 2p chosen, 2p+1 rejected)."""
+        pairs = self.batch // 2
+        return self._preference_step(lambda: L.soup_orpo_loss(self.logp, pairs, self.seq, prompt_len, lam,
+                                                              self.loss, self.seq_sums, self.coef))
+
     def optimizer_step(self, grad_scale: float = 1.0):
         """AdamW on every LoRA factor: one kernel launch over the flat buffers
         updates the fp32 master copy and the moments, rewrites the bf16 factors
