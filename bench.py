@@ -52,6 +52,14 @@ WORKLOADS = {
     "llama8b-nf4-stream-dpo": dict(hidden=4096, n_q_heads=32, n_kv_heads=8, head_dim=128, intermediate=14336,
                                    rank=16, alpha=32.0, vocab=128256, n_layers=32, kind="nf4", tied=False,
                                    batch=8, seq=512, buffers=2, cap_gb=0.0, task="dpo", prompt=256, beta=0.1),
+    # the reference-free preference losses on the same stream and pairs
+    "llama8b-nf4-stream-simpo": dict(hidden=4096, n_q_heads=32, n_kv_heads=8, head_dim=128, intermediate=14336,
+                                     rank=16, alpha=32.0, vocab=128256, n_layers=32, kind="nf4", tied=False,
+                                     batch=8, seq=512, buffers=2, cap_gb=0.0, task="simpo", prompt=256, beta=2.0,
+                                     gamma=1.0),
+    "llama8b-nf4-stream-orpo": dict(hidden=4096, n_q_heads=32, n_kv_heads=8, head_dim=128, intermediate=14336,
+                                    rank=16, alpha=32.0, vocab=128256, n_layers=32, kind="nf4", tied=False,
+                                    batch=8, seq=512, buffers=2, cap_gb=0.0, task="orpo", prompt=256, lam=0.1),
 }
 DEFAULT = "llama8b-nf4-stream-sft"
 METRIC = "train tokens/s, 8B-shape NF4 streamed LoRA, 1 B200; fused GEMM % bf16 peak"
@@ -343,7 +351,15 @@ def main():
     from layer_streamed_qlora_b200 import dp
 
     def step():
-        loss = model.sft_step() if w["task"] == "sft" else model.dpo_step(w["prompt"], w["beta"])
+        task = w["task"]
+        if task == "sft":
+            loss = model.sft_step()
+        elif task == "dpo":
+            loss = model.dpo_step(w["prompt"], w["beta"])
+        elif task == "simpo":
+            loss = model.simpo_step(w["prompt"], w["beta"], w["gamma"])
+        else:
+            loss = model.orpo_step(w["prompt"], w["lam"])
         # data parallel: the one exchange of the step, the LoRA gradients
         # summed in place (a no-op on one rank); the optimiser step takes the
         # mean's 1/world as its gradient scale

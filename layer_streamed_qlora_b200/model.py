@@ -158,8 +158,8 @@ class StreamedLoRAModel:
         self.stream_source, self.shard_dir = stream_source, shard_dir
         self.disk = None
         self.adamw = adamw or AdamW()
-        if task not in ("sft", "dpo"):
-            raise ValueError(f"task must be 'sft' or 'dpo', not {task!r}")
+        if task not in ("sft", "dpo", "simpo", "orpo"):
+            raise ValueError(f"task must be 'sft', 'dpo', 'simpo' or 'orpo', not {task!r}")
         self.task = task
         self.T = batch * seq
         self.head_chunk = head_chunk
