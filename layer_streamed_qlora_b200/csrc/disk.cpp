@@ -148,9 +148,10 @@ void pump(soup_disk* d) {
       }
       if (++scanned >= n) {  // every layer stays resident: no copies after the first cycle
         d->exhausted = true;
-        return;
+        break;
       }
     }
+    if (layer < 0) break;  // exhausted; the reads queued above still need the wake-up below
     b.state = B_READING;
     b.pos = d->next_read - 1;
     b.layer = layer;

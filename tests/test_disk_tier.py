@@ -10,6 +10,7 @@ wasted, and keep handing out correct bytes when the consumer strays from the
 schedule."""
 import ctypes
 import os
+import time
 
 import numpy as np
 import pytest
@@ -45,7 +46,7 @@ def _consume(disk, data, visits, n_slots):
         if l in ring:
             ring.remove(l)
         else:
-            host, ev = disk.acquire(l, timeout_ms=20000)
+            host, ev = disk.acquire(l, timeout_ms=5000)
             assert ev is None
             assert ctypes.string_at(host, LAYER_BYTES) == data[l], f"layer {l}: wrong bytes"
             disk.release(l)
@@ -109,13 +110,18 @@ def test_consumer_off_schedule_still_gets_the_right_bytes(shards):
         disk.close()
 
 
-def test_every_layer_fits_the_ring(shards):
+@pytest.mark.parametrize("read_ahead,n_slots", [(2, 4), (8, 8)])
+def test_every_layer_fits_the_ring(shards, read_ahead, n_slots):
+    # (8, 8): more staging buffers than copied visits, so the reader runs out
+    # of visits to read in the same pass that queues the first reads; those
+    # reads must still start
     paths, data = shards
-    disk = _open(paths[:3], 2, 4)
+    disk = _open(paths[:3], read_ahead, n_slots)
     try:
         order = _sft_order(3)
+        time.sleep(0.2)  # let the I/O threads go idle first: the queued reads must wake them
         disk.schedule(order)
-        assert _consume(disk, data, order * 4, 4) == 3  # read once, resident afterwards
+        assert _consume(disk, data, order * 4, n_slots) == 3  # read once, resident afterwards
         assert disk.stats()["reads"] == 3
     finally:
         disk.close()
