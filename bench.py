@@ -145,8 +145,9 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_sample_seconds(w, tokens=256, reps=1):
     """Times the CPU oracle (fp64 numpy) on one decoder layer of the workload's
-    shape: forward + backward for `tokens` tokens of one sequence, then the
-    AdamW step over that layer's LoRA factors.  Weights are random fp64 (their
+    shape: forward + backward for `tokens` tokens of one sequence (plus the
+    adapters-off reference forward for DPO), then the AdamW step over that
+    layer's LoRA factors.  Weights are random fp64 (their
     preparation is not timed).  Returns (layer seconds, AdamW seconds)."""
     import numpy as np
 
@@ -169,6 +170,8 @@ def oracle_sample_seconds(w, tokens=256, reps=1):
     times, adam = [], []
     for _ in range(reps):
         t0 = time.perf_counter()
+        if w.get("task") == "dpo":  # the adapters-off reference pass of a DPO step
+            layer_fwd(h, W, lora, shape, False)
         _, cache = layer_fwd(h, W, lora, shape)
         _, grads = layer_bwd(cache, W, lora, shape, dh)
         t1 = time.perf_counter()
