@@ -9,6 +9,12 @@
  * backward pass re-reads and recomputes the layer and produces
  * dL/dx = W^T dL/dy plus the adapter terms, and dA, dB, while W stays frozen.
  *
+ * Sections below: status and profiling; NF4 quantisation; the LoRA linear
+ * layer; the decoder layer (forward, recompute backward, kept q|k|v); the
+ * stream plan (slot ring, copies, waits); the disk tier (shard files read
+ * ahead into staging buffers); layer blob layout; embedding, output head,
+ * cross-entropy and DPO; SimPO and ORPO; the AdamW step on the adapters.
+ *
  * Conventions for every entry point
  *  - Every function returns a soup_status; SOUP_OK (0) on success.  On failure
  *    soup_last_error() returns a message for the calling thread.  Nothing
@@ -16,7 +22,8 @@
  *    is out of range is refused.
  *  - Pointers named *_dev, and all tensor pointers unless stated otherwise,
  *    are CUDA device pointers owned by the caller.  The library allocates no
- *    device memory except the slot arena of soup_stream_plan.
+ *    device memory except the slot arena of soup_stream_plan (and the
+ *    disk tier's page-locked host staging buffers, in soup_disk_open).
  *  - "bf16" tensors are passed as uint16_t bit patterns (IEEE bfloat16).
  *  - Matrices are row-major.  [R, C] means R rows of C contiguous elements.
  *  - `stream` is a cudaStream_t passed as void*; work is enqueued on it and
