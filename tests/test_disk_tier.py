@@ -212,3 +212,47 @@ def test_read_error_is_reported_by_the_acquire(shards, tmp_path):
         disk.release(2)
     finally:
         disk.close()
+
+
+def test_randomized_settings_orders_and_idle_threads(tmp_path):
+    # seeded random read-ahead / slot / thread counts, O_DIRECT on or off,
+    # I/O threads idle or not when the schedule arrives, and consumers that
+    # stray from the schedule: every acquired buffer must hold its layer
+    import random
+    lb = (8 << 20) + 4352  # two requests, the second ragged
+    rng = np.random.default_rng(21)
+    paths, marks = [], []
+    for l in range(7):
+        b = rng.integers(0, 256, lb, dtype=np.uint8)
+        p = tmp_path / f"r{l}.bin"
+        b.tofile(p)
+        paths.append(str(p))
+        marks.append((b[:64].tobytes(), b[lb // 2:lb // 2 + 64].tobytes(), b[-64:].tobytes()))
+    n = len(paths)
+    order = _sft_order(n)
+    for trial in range(24):
+        rnd = random.Random(trial)
+        ra, ns, io = rnd.randint(1, 8), rnd.randint(2, 8), rnd.randint(1, 8)
+        disk = L.Disk(paths, lb, read_ahead=ra, n_slots=ns, io_threads=io, pinned=False, direct=bool(trial % 2))
+        try:
+            if trial % 3 == 0:
+                time.sleep(0.02)
+            disk.schedule(order)
+            visits = order * 3
+            if trial % 4 == 1:
+                visits = visits[:9] + rnd.sample(range(n), n) + visits[9:]
+            ring = []
+            for l in visits:
+                if l in ring:
+                    ring.remove(l)
+                else:
+                    host, _ = disk.acquire(l, timeout_ms=5000)
+                    got = (ctypes.string_at(host, 64), ctypes.string_at(host + lb // 2, 64),
+                           ctypes.string_at(host + lb - 64, 64))
+                    assert got == marks[l], (trial, l)
+                    disk.release(l)
+                ring.append(l)
+                if len(ring) > ns:
+                    ring.pop(0)
+        finally:
+            disk.close()
