@@ -203,7 +203,8 @@ def cpu_baseline(w, tokens=256):
     t, ta = oracle_sample_seconds(w, tokens)
     per_token_stack = oracle_seconds_per_token(w, t, ta, tokens)
     return {"value": 1.0 / per_token_stack, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"one {w['hidden']}-hidden decoder layer, fwd+bwd on 1x{tokens} tokens ({t:.2f} s) and the "
+            "sample": f"one {w['hidden']}-hidden decoder layer, "
+                      f"{'reference fwd + ' if w.get('task') == 'dpo' else ''}fwd+bwd on 1x{tokens} tokens ({t:.2f} s) and the "
                       f"AdamW step of its LoRA factors ({ta:.3f} s, per {w['batch'] * w['seq']}-token step) in "
                       f"fp64 numpy, projected to the {w['n_layers']}-layer stack (head excluded)"}
 
@@ -238,7 +239,9 @@ def run_reference(args, w, name):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": bench_config(w, name, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"per step: one decoder layer fwd+bwd on 1x{tokens} tokens and the AdamW "
+                             "sample": f"per step: one decoder layer "
+                                       f"{'reference fwd + ' if w.get('task') == 'dpo' else ''}fwd+bwd on 1x{tokens} "
+                                       f"tokens and the AdamW "
                                        f"step of its LoRA factors, fp64 numpy, projected to {w['n_layers']} "
                                        f"layers"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
