@@ -2,17 +2,22 @@
 
 The flat-buffer layout must be identical on every rank and the in-place
 all-reduce must leave every rank with the mean of the ranks' gradients in
-every view.  CPU only: the same code path runs over NCCL on GPUs.
+every view (or the sum, for the variant that leaves the 1/world to the
+optimiser step); an AdamW step with grad_scale = 1/world after the sum must
+leave every rank with the parameters of one step on the mean gradient.  CPU
+only: the same code path runs over NCCL on GPUs.
 """
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
 from layer_streamed_qlora_b200 import dp
+from oracle.optim import adamw_step
 
 SHAPES = [(16, 4096), (6144, 16), (16, 4096), (4096, 16), (32, 4096), (28672, 16), (16, 14336), (4096, 16),
           (3, 5)]
@@ -40,9 +45,15 @@ def _rank_main(rank, world, port, q):
         summed = flat.clone()
         dp.allreduce_mean_(flat)
         world_seen = dp.allreduce_sum_(summed)
+        # the training step's exchange: a sum, then the optimiser step with
+        # grad_scale = 1/world on parameters that start equal on every rank
+        theta0 = np.linspace(-0.05, 0.05, summed.numel())
+        z = np.zeros(summed.numel())
+        theta1, _, _ = adamw_step(theta0, summed.numpy().astype(np.float64), z, z, 1, 5e-4,
+                                  grad_scale=1.0 / world_seen)
         # numpy copies: plain pickles (tensors would travel as shared-memory handles)
         q.put((rank, [v.numpy().copy() for v in views], [v.numpy() for v in vals], dp.flat_layout(SHAPES),
-               flat.numpy().copy(), summed.numpy().copy(), world_seen))
+               flat.numpy().copy(), summed.numpy().copy(), world_seen, theta1))
     finally:
         dist.destroy_process_group()
 
@@ -87,8 +98,8 @@ def test_two_rank_gradient_average():
         p.start()
     res = {}
     for _ in range(world):
-        rank, after, before, layout, gap, summed, world_seen = q.get(timeout=100)
-        res[rank] = (after, before, layout, gap, summed, world_seen)
+        rank, after, before, layout, gap, summed, world_seen, theta1 = q.get(timeout=100)
+        res[rank] = (after, before, layout, gap, summed, world_seen, theta1)
     for p in procs:
         p.join(timeout=30)
         assert p.exitcode == 0
@@ -103,6 +114,13 @@ def test_two_rank_gradient_average():
         assert res[r][5] == world
         torch.testing.assert_close(torch.from_numpy(res[r][4]), torch.from_numpy(res[r][3]) * world, rtol=1e-6,
                                    atol=1e-6)
+    # after the optimiser step every rank holds the same parameters: those of
+    # one AdamW step on the mean gradient
+    assert np.array_equal(res[0][6], res[1][6])
+    mean_flat = (res[0][4] / world).astype(np.float64)
+    z = np.zeros(mean_flat.size)
+    ref, _, _ = adamw_step(np.linspace(-0.05, 0.05, mean_flat.size), mean_flat, z, z, 1, 5e-4)
+    np.testing.assert_allclose(res[0][6], ref, rtol=1e-12, atol=1e-15)
     # the alignment padding between views stays zero
     for r in range(world):
         pad = torch.ones(n, dtype=torch.bool)
