@@ -87,3 +87,13 @@ def test_plan_without_host_layers_passes_validation():
     if st == 0:
         L.lib().soup_stream_plan_free(h)
     assert st in (0, 7), L.lib().soup_last_error()
+
+
+def test_model_refuses_unknown_settings_before_touching_the_gpu():
+    # refuse, never ignore: checked before any allocation
+    from layer_streamed_qlora_b200.model import ModelConfig, StreamedLoRAModel
+    cfg = ModelConfig(hidden=512, n_q_heads=4, n_kv_heads=2, head_dim=128, intermediate=1024, rank=16, alpha=32.0,
+                      vocab=512, n_layers=2)
+    for kw in ({"stream_source": "nvme"}, {"stream_source": "disk"}, {"task": "kto"}):
+        with pytest.raises(ValueError):
+            StreamedLoRAModel(cfg, 2, 16, **kw)
