@@ -126,6 +126,31 @@ class AdamW:
     weight_decay: float = 0.0
 
 
+def device_bytes_lower_bound(cfg: ModelConfig, batch: int, seq: int, n_buffers: int, head_chunk: int) -> int:
+    """Device bytes a streamed model needs at least, from the library's host
+    size queries: the slot arena (n_buffers layer blobs + the vocab slot),
+    the layer checkpoints [L+1, T, H] bf16, the layer and head workspaces."""
+    lcfg = cfg.layer_cfg()
+    blob = L.soup_layer_blob_bytes(lcfg, cfg.weight_kind)
+    vocab = (cfg.vocab * cfg.hidden * 2 + 255) // 256 * 256
+    T = batch * seq
+    return (n_buffers * blob + vocab + (cfg.n_layers + 1) * T * cfg.hidden * 2 +
+            L.soup_decoder_layer_workspace(lcfg, batch, seq) +
+            L.soup_head_workspace(cfg.vocab, cfg.hidden, batch, seq, head_chunk))
+
+
+def precheck_device_bytes(cfg, batch, seq, n_buffers, head_chunk, cap):
+    """Refuses, before any shard is built or any device memory is taken, a
+    model whose lower-bound device need exceeds the cap (the stream plan makes
+    the exact check once the model's own allocations are known)."""
+    if not cap:
+        return
+    need = device_bytes_lower_bound(cfg, batch, seq, n_buffers, head_chunk)
+    if need > cap:
+        raise ValueError(f"the streamed model needs at least {need} device bytes ({n_buffers} slots, the vocab slot, "
+                         f"checkpoints and workspaces) > device cap {cap}")
+
+
 def kept_layer_count(n_layers: int, per_layer: int, arena: int, reserve: int, cap: int) -> int:
     """How many layers' q|k|v (per_layer bytes each) can be kept while
     soup_stream_plan still admits the model: arena (slots + vocab slot) +
@@ -164,6 +189,7 @@ class StreamedLoRAModel:
         self.T = batch * seq
         self.head_chunk = head_chunk
         self.lcfg = cfg.layer_cfg()
+        precheck_device_bytes(cfg, batch, seq, n_buffers, head_chunk, device_cap_bytes)
         weights = weights or SyntheticWeights(cfg, seed)
         self._build_blobs(weights)
         self._alloc(weights)

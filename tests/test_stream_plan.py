@@ -97,3 +97,14 @@ def test_model_refuses_unknown_settings_before_touching_the_gpu():
     for kw in ({"stream_source": "nvme"}, {"stream_source": "disk"}, {"task": "kto"}):
         with pytest.raises(ValueError):
             StreamedLoRAModel(cfg, 2, 16, **kw)
+
+
+def test_model_precheck_refuses_a_cap_below_the_lower_bound_before_any_work():
+    from layer_streamed_qlora_b200.model import ModelConfig, StreamedLoRAModel, device_bytes_lower_bound
+    cfg = ModelConfig(hidden=4096, n_q_heads=32, n_kv_heads=8, head_dim=128, intermediate=14336, rank=16,
+                      alpha=32.0, vocab=128256, n_layers=32)
+    lb = device_bytes_lower_bound(cfg, 4, 512, 2, 256)
+    # 2 slots x 122.7 MB + the 1050.7 MB vocab slot + 33 checkpoints x 16.8 MB + workspaces
+    assert 2 * 122_699_776 + 1_050_673_152 + 33 * 2048 * 4096 * 2 < lb < 4 << 30
+    with pytest.raises(ValueError, match="device cap"):
+        StreamedLoRAModel(cfg, 4, 512, n_buffers=2, device_cap_bytes=1 << 30)  # refused at once, no GPU needed
