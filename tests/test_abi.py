@@ -81,3 +81,15 @@ def test_adamw_refuses_bad_arguments_on_the_host(libpath):
     assert call(ptrs=[ok[0], P(0x20004), ok[2], ok[3], ok[4]]) == ALIGN  # bf16 copy not 8-byte aligned
     assert call(ptrs=[None] + ok[1:]) == INVALID
     assert b"soup_adamw_step" in _lib.lib().soup_last_error()
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/soup.h declares a C ABI: a C99 translation unit that includes
+    it and takes the address of every declared function compiles with gcc."""
+    names = _declared()
+    src = tmp_path / "abi.c"
+    body = "\n".join(f"  (void)&{n};" for n in names)
+    src.write_text(f'#include "soup.h"\nint main(void) {{\n{body}\n  return 0;\n}}\n')
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-I", os.path.join(ROOT, "include"),
+                        str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
