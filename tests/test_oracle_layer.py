@@ -153,3 +153,70 @@ def test_B_zero_and_adapters_off_reproduce_base_exactly():
     assert np.array_equal(off, zero)
     on, _ = layer_fwd(h, W, lora, shape)
     assert not np.allclose(on, off)
+
+
+# ----------------------------------------------------------------------------- constants pinned by closed forms
+# Each test below fails if the oracle's RoPE exponent, attention scale or
+# RMSNorm epsilon placement is changed: the expected values are computed from
+# scalar closed forms (math module), not by re-running the oracle's formula.
+import math
+
+
+def test_rope_frequencies_at_position_one_closed_form():
+    """The 8B layer (theta 5e5, head_dim 128): at position 1, pair i turns by
+    exactly theta^(-2i/128) radians, so pair 0 turns by 1 rad and the last
+    pair (i = 63) by 5e5^(-126/128).  A rotated unit vector e_i reads
+    (cos a_i, sin a_i) in components (i, i + 64)."""
+    d, theta = 128, 5e5
+    assert ss.LLAMA8B_LAYER.theta == 5e5 and ss.LLAMA8B_LAYER.head_dim == d
+    cos, sin = L.rope_tables(2, d, theta)
+    for i, angle in ((0, 1.0), (32, 5e5 ** -0.5), (63, 5e5 ** (-126.0 / 128.0))):
+        e = np.zeros((1, 2, 1, d))
+        e[0, 1, 0, i] = 1.0
+        r = L.rope_fwd(e, cos, sin)[0, 1, 0]
+        assert abs(r[i] - math.cos(angle)) < 1e-15, (i, r[i], math.cos(angle))
+        assert abs(r[i + 64] - math.sin(angle)) < 1e-15, (i, r[i + 64], math.sin(angle))
+        others = np.delete(r, [i, i + 64])
+        assert np.all(others == 0.0)
+    # the second component of a pair turns the other way: e_{i+64} -> (-sin a, cos a)
+    e = np.zeros((1, 2, 1, d))
+    e[0, 1, 0, 64] = 1.0
+    r = L.rope_fwd(e, cos, sin)[0, 1, 0]
+    assert abs(r[0] + math.sin(1.0)) < 1e-15 and abs(r[64] - math.cos(1.0)) < 1e-15
+    # position p turns pair 0 by p rad (not p * anything else)
+    cos7, sin7 = L.rope_tables(8, d, theta)
+    assert abs(cos7[7, 0] - math.cos(7.0)) < 1e-15 and abs(sin7[7, 0] - math.sin(7.0)) < 1e-15
+
+
+def test_attention_scale_two_token_closed_form():
+    """head_dim 128, two tokens with k0 = 0 and q1 . k1 = c: the second query's
+    softmax weights are 1 / (1 + e^(c/sqrt(128))) on v0 and
+    e^(c/sqrt(128)) / (1 + e^(c/sqrt(128))) on v1."""
+    d, c = 128, 3.0
+    g = np.random.default_rng(11)
+    q = np.zeros((1, 2, 1, d)); k = np.zeros((1, 2, 1, d)); v = np.zeros((1, 2, 1, d))
+    q[0, 1, 0] = g.standard_normal(d)
+    k1 = g.standard_normal(d)
+    k1 *= c / float(q[0, 1, 0] @ k1)               # q1 . k1 = c exactly up to rounding
+    k[0, 1, 0] = k1
+    v[0, 0, 0, 0] = 1.0                            # v0 = e_0, v1 = e_1
+    v[0, 1, 0, 1] = 1.0
+    out, _ = L.attention_fwd(q, k, v)
+    z = math.exp(c / math.sqrt(128.0))
+    assert abs(out[0, 1, 0, 0] - 1.0 / (1.0 + z)) < 1e-13
+    assert abs(out[0, 1, 0, 1] - z / (1.0 + z)) < 1e-13
+    assert np.all(out[0, 1, 0, 2:] == 0.0)
+
+
+def test_rmsnorm_eps_inside_the_root_constant_row():
+    """A constant row c with eps > 0 normalises to w * c / sqrt(c^2 + eps)
+    (eps added to the mean square, inside the square root)."""
+    eps = 1e-5
+    w = np.array([0.5, 2.0, -1.5, 1.0])
+    for c in (0.01, -0.003, 2.0):
+        x = np.full((1, 4), c)
+        y, rinv = L.rmsnorm_fwd(x, w, eps)
+        expect = c / math.sqrt(c * c + eps)
+        np.testing.assert_allclose(y[0], w * expect, rtol=1e-14, atol=0)
+        assert abs(rinv[0, 0] - 1.0 / math.sqrt(c * c + eps)) <= 1e-14 / math.sqrt(c * c + eps)
+    assert ss.LLAMA8B_LAYER.eps == 1e-5
