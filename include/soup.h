@@ -62,22 +62,42 @@ const char* soup_last_error(void);
  * Returns SOUP_OK, or SOUP_ERR_CUDA if the read itself failed. */
 soup_status soup_device_error(int32_t* code_out);
 
+/* Test of the kernels' bounded waits, with no fault and no hang: computes
+ * C[M, N] (fp32, row-major) = A[M, K] B[N, K]^T (bf16, row-major, device
+ * pointers) with the one-CTA tcgen05 GEMM engine, whose mbarrier waits give
+ * up after wait_limit_cycles SM clock cycles (0 = the default, ~2 s).  With
+ * skip_producer_arrivals != 0 the engine's TMA producer issues nothing and
+ * never arrives, so the MMA warp's wait runs out: the CTA records code 1 in
+ * the device error word (soup_device_error), issues no tensor-core work,
+ * frees its tensor memory and returns; C is left unwritten and the context
+ * stays usable.  Sizes in (0, 4096], K % 8 == 0, N % 4 == 0.  Async on
+ * `stream`. */
+soup_status soup_debug_gemm_bounded_wait(const uint16_t* A, const uint16_t* B, int64_t M, int64_t N, int64_t K,
+                                         float* C, int64_t wait_limit_cycles, int32_t skip_producer_arrivals,
+                                         void* stream);
+
 /* Number of kernels this library has launched in this process. */
 int64_t soup_launch_count(void);
 
-/* Optional timing of the tensor-core GEMM launches: while enabled, every GEMM
- * launch of a class in class_mask (bit c = class c) is bracketed by CUDA
- * events recorded on its own stream and tagged with its algorithmic work.
- * soup_profile_read synchronises those events and sums them per class:
+/* Optional timing of kernel launches: while enabled, every launch of a class
+ * in class_mask (bit c = class c) is bracketed by CUDA events recorded on its
+ * own stream and tagged with its algorithmic work.  soup_profile_read
+ * synchronises those events and sums them per class:
  * 0 = fused NF4-decode GEMM (forward, W), 1 = fused NF4-decode GEMM
  * (backward, W^T), 2 = other GEMMs with N > 64, 3 = skinny LoRA GEMMs
  * (N <= 64), 4 = fused NF4-decode GEMMs with a hi + lo A pair (either
- * direction).  Enabling resets the records; class_mask 0 disables. */
+ * direction), 5 = attention (forward and backward kernels; flops 4 B Hq d
+ * S(S+1)/2 forward, 2.5x that backward), 6 = RMSNorm forward / backward,
+ * 7 = split-K reductions, 8 = other elementwise kernels (RoPE tables, LoRA
+ * operand preparation, conversions, attention row dots, embedding gather),
+ * 9 = cross-entropy rows of the output head, 10 = AdamW.  Classes 6..10
+ * carry algorithmic bytes (each operand read once, each output written
+ * once) and no flops.  Enabling resets the records; class_mask 0 disables. */
 typedef struct soup_gemm_profile {
   int64_t launches;
   double total_ms;
-  double flops;  /* 2 M N (K + r_tail) summed over launches */
-  double bytes;  /* A read once + B (NF4 packed or bf16) + output written once */
+  double flops;  /* GEMMs: 2 M N (K + r_tail) summed over launches; attention as above */
+  double bytes;  /* operands read once + outputs written once */
 } soup_gemm_profile;
 soup_status soup_profile_enable(int32_t class_mask);
 soup_status soup_profile_read(soup_gemm_profile* out, int32_t n_classes);
@@ -164,14 +184,19 @@ soup_status soup_lora_linear_bwd(const soup_weight* W, const uint16_t* A, const 
  *  - Sizes whose scratch, soup_lora_linear_bwd_workspace(T, r, out), exceeds
  *    that maximum are refused with SOUP_ERR_SHAPE and a message (nothing runs).
  *  - The first call on each device does a one-time set-up (it looks up the
- *    array's device address with that device current); make that first call
- *    before any stream capture.
+ *    array's device address with that device current and caches it with the
+ *    device's context; a call in a new context, e.g. after cudaDeviceReset,
+ *    looks it up again); make that first call before any stream capture.
  *  - Every call shares the one array and it keeps the last call's contents:
  *    calls that overlap on the GPU (different streams, or different host
  *    threads on one device) race and corrupt each other's results; serialise
  *    them.  No part of the scratch has to start at zero.
  *  - Never calls cudaMalloc, cudaFree or any allocating routine. */
 size_t soup_lora_linear_bwd_noalloc_max_scratch(void);
+/* Device bytes the library holds in module-static arrays (the scratch above)
+ * on every device that loads it: memory outside any allocator, to be counted
+ * against a device budget. */
+size_t soup_static_device_bytes(void);
 soup_status soup_lora_linear_bwd_noalloc(const soup_weight* W, const uint16_t* A, const uint16_t* B,
                                          int32_t r, float scale, const uint16_t* x,
                                          const uint16_t* u_save, const uint16_t* dy, int64_t T,
@@ -348,12 +373,19 @@ soup_status soup_stream_wait_host(soup_plan* plan, int32_t item, int32_t timeout
 soup_status soup_stream_release(soup_plan* plan, int32_t item, void* compute_stream);
 
 /* Copy/stall statistics since the plan was made or last reset (synchronises
- * the copy stream and the recorded events). */
+ * the copy stream and the recorded events).  The timing events form two
+ * fixed rings of 256 (start, end) pairs (one for copies, one for waits):
+ * an entry's elapsed time is folded into a running total before the entry
+ * is reused, so a run of any length holds a bounded number of events. */
 soup_status soup_stream_stats(soup_plan* plan, soup_stream_stats_t* out);
 soup_status soup_stream_stats_reset(soup_plan* plan);
 
 /* The plan's copy stream (cudaStream_t as void*). */
 void* soup_stream_copy_stream(soup_plan* plan);
+
+/* Number of CUDA events the plan holds for its statistics (at most 1024;
+ * -1 for a NULL plan).  Host only. */
+int64_t soup_stream_debug_timing_events(soup_plan* plan);
 
 /* Fault-injection hooks for tests (host side only): the next prefetch fails
  * with SOUP_ERR_CUDA without copying; or the next copy first waits on

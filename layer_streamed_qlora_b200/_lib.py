@@ -79,6 +79,11 @@ class GemmProfile(ctypes.Structure):
 
 
 GEMM_CLASSES = ("nf4_fwd", "nf4_bwd", "bf16", "lora_skinny", "nf4_dual")
+# every class soup_profile_enable can time, in bit order: the GEMM classes,
+# then attention (flops) and the memory-bound kernels (algorithmic bytes)
+PROFILE_CLASSES = GEMM_CLASSES + ("attention", "rmsnorm", "splitk_reduce", "elementwise", "ce_rows", "adamw")
+HBM_CLASSES = ("rmsnorm", "splitk_reduce", "elementwise", "ce_rows", "adamw")
+PROFILE_ALL = (1 << len(PROFILE_CLASSES)) - 1
 
 SOUP_ITEM_EMBED = -1
 SOUP_ITEM_HEAD = -2
@@ -135,6 +140,10 @@ _SIGS = {
     "soup_stream_stats": (c_int32, [c_void_p, ctypes.POINTER(StreamStats)]),
     "soup_stream_stats_reset": (c_int32, [c_void_p]),
     "soup_stream_copy_stream": (c_void_p, [c_void_p]),
+    "soup_stream_debug_timing_events": (c_int64, [c_void_p]),
+    "soup_static_device_bytes": (c_size_t, []),
+    "soup_debug_gemm_bounded_wait": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64,
+                                               c_int32, c_void_p]),
     "soup_stream_debug_fail_next_copy": (c_int32, [c_void_p]),
     "soup_stream_debug_gate_next_copy": (c_int32, [c_void_p, c_void_p]),
     "soup_layer_blob_bytes": (c_size_t, [ctypes.POINTER(LayerCfg), c_int32]),
@@ -197,14 +206,30 @@ def launch_count() -> int:
 
 
 def profile_enable(class_mask: int):
-    """class_mask bit c enables timing of GEMM class c (GEMM_CLASSES order); 0 disables."""
+    """class_mask bit c enables timing of kernel class c (PROFILE_CLASSES order); 0 disables."""
     _check("soup_profile_enable", lib().soup_profile_enable(int(class_mask)))
 
 
 def profile_read() -> dict:
-    arr = (GemmProfile * len(GEMM_CLASSES))()
-    _check("soup_profile_read", lib().soup_profile_read(arr, len(GEMM_CLASSES)))
-    return {name: {k: getattr(arr[i], k) for k, _ in GemmProfile._fields_} for i, name in enumerate(GEMM_CLASSES)}
+    arr = (GemmProfile * len(PROFILE_CLASSES))()
+    _check("soup_profile_read", lib().soup_profile_read(arr, len(PROFILE_CLASSES)))
+    return {name: {k: getattr(arr[i], k) for k, _ in GemmProfile._fields_} for i, name in enumerate(PROFILE_CLASSES)}
+
+
+def soup_debug_gemm_bounded_wait(A, B, C, wait_limit_cycles=0, skip_producer_arrivals=False, stream=None):
+    """C = A B^T (A [M, K], B [N, K] bf16; C [M, N] fp32) on the one-CTA GEMM
+    engine with a caller-set mbarrier wait limit; with skip_producer_arrivals
+    the producer never arrives and the kernel's wait runs out (device error 1)."""
+    M, K = A.shape
+    N = B.shape[0]
+    _check("soup_debug_gemm_bounded_wait", lib().soup_debug_gemm_bounded_wait(
+        _p(A), _p(B), M, N, K, _p(C), int(wait_limit_cycles), 1 if skip_producer_arrivals else 0, _stream(stream)))
+
+
+def static_device_bytes() -> int:
+    """Device bytes the library holds in module-static arrays on every device
+    that loads it (held until process exit, outside any allocator)."""
+    return int(lib().soup_static_device_bytes())
 
 
 # ---------------------------------------------------------------- NF4
@@ -382,6 +407,9 @@ class Plan:
 
     def copy_stream_handle(self) -> int:
         return lib().soup_stream_copy_stream(self.h)
+
+    def timing_events(self) -> int:
+        return int(lib().soup_stream_debug_timing_events(self.h))
 
     def debug_fail_next_copy(self):
         _check("soup_stream_debug_fail_next_copy", lib().soup_stream_debug_fail_next_copy(self.h))

@@ -528,8 +528,11 @@ soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
   SOUP_TRY(attn_init());
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   dim3 grid((S + 63) / 64, Hq, Bsz);
+  const double fl = 4.0 * Bsz * Hq * (double)HD * ((double)S * (S + 1) / 2);
+  profile_begin(st, GC_ATTN, fl, 0.0);
   attn_fwd_kernel<<<grid, 128, FWD_SMEM, st>>>(qkv, ld, S, Hq, Hkv, out, lse, scale_log2, out16, out32);
   SOUP_LAUNCH_CHECK();
+  profile_end(st);
   return SOUP_OK;
 }
 
@@ -540,6 +543,8 @@ soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
   SOUP_TRY(attn_init());
   const float scale = 1.0f / sqrtf((float)HD);
   const float scale_log2 = 1.4426950408889634f * scale;
+  const double fl = 2.5 * 4.0 * Bsz * Hq * (double)HD * ((double)S * (S + 1) / 2);
+  profile_begin(st, GC_ATTN, fl, 0.0);
   dim3 g1((S + 63) / 64, Hkv, Bsz);
   attn_bwd_dkdv_kernel<<<g1, 128, DKDV_SMEM, st>>>(qkv, ld, S, Hq, Hkv, dout, lse, D, dqkv, scale_log2, scale,
                                                    rope_cos, rope_sin, amax, dqkv32);
@@ -548,6 +553,7 @@ soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
   attn_bwd_dq_kernel<<<g2, 128, DQ_SMEM, st>>>(qkv, ld, S, Hq, Hkv, dout, lse, D, dqkv, scale_log2, scale,
                                                rope_cos, rope_sin, amax, dqkv32);
   SOUP_LAUNCH_CHECK();
+  profile_end(st);
   return SOUP_OK;
 }
 

@@ -229,8 +229,12 @@ unsigned grid_for(size_t work, int threads) {
 soup_status rmsnorm_fwd(const uint16_t* x, const float* x_f32, const uint16_t* w, int T, int H, float eps,
                         uint16_t* y, float* rinv, cudaStream_t st, float* y32, uint16_t* ylo) {
   SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
+  const double n = (double)T * H;
+  profile_begin(st, GC_RMSNORM, 0.0,
+                n * (x_f32 ? 4 : 2) + H * 2.0 + n * 2 + T * 4.0 + (y32 ? n * 4 : 0.0) + (ylo ? n * 2 : 0.0));
   rmsnorm_fwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, T, H, eps, y, rinv, y32, ylo);
   SOUP_LAUNCH_CHECK();
+  profile_end(st);
   return SOUP_OK;
 }
 
@@ -238,9 +242,14 @@ soup_status rmsnorm_bwd(const uint16_t* x, const float* x_f32, const uint16_t* w
                         const uint16_t* dy, const float* dres, int T, int H, float* dh, uint16_t* dh_bf16,
                         cudaStream_t st, unsigned int* amax, uint16_t* dh_lo) {
   SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
+  const double n = (double)T * H;
+  profile_begin(st, GC_RMSNORM, 0.0,
+                n * (x_f32 ? 4 : 2) + H * 2.0 + T * 4.0 + n * 2 + (dres ? n * 4 : 0.0) + n * 4 +
+                    (dh_bf16 ? n * 2 : 0.0) + (dh_lo ? n * 2 : 0.0));
   rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, rinv, dy, nullptr, dres, T, H, dh, dh_bf16, amax,
                                                   dh_lo);
   SOUP_LAUNCH_CHECK();
+  profile_end(st);
   return SOUP_OK;
 }
 
@@ -262,21 +271,27 @@ soup_status transpose_bf16_f32(const uint16_t* in, int rows, int cols, float* ou
 
 soup_status rope_table(int S, int head_dim, double theta, float* cosb, float* sinb, cudaStream_t st) {
   const int n = S * head_dim / 2;
+  profile_begin(st, GC_ELEM, 0.0, n * 8.0);
   rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(S, head_dim / 2, theta, cosb, sinb);
   SOUP_LAUNCH_CHECK();
+  profile_end(st);
   return SOUP_OK;
 }
 
 soup_status attn_rowdot(const uint16_t* dO, const uint16_t* O, int T, int Hq, float* D, cudaStream_t st) {
+  profile_begin(st, GC_ELEM, 0.0, (double)T * Hq * (128 * 2 * 2 + 4));
   attn_rowdot_kernel<<<(T * Hq + 7) / 8, 256, 0, st>>>(dO, O, T, Hq, D);
   SOUP_LAUNCH_CHECK();
+  profile_end(st);
   return SOUP_OK;
 }
 
 soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t st) {
   SOUP_CHECK(n % 8 == 0, SOUP_ERR_SHAPE, "f32_to_bf16: n %% 8");
+  profile_begin(st, GC_ELEM, 0.0, n * 6.0);
   f32_to_bf16_kernel<<<grid_for(n / 8, 256), 256, 0, st>>>(in, n, out);
   SOUP_LAUNCH_CHECK();
+  profile_end(st);
   return SOUP_OK;
 }
 
@@ -332,8 +347,16 @@ soup_status lora_prep(const PrepJobs& jobs, cudaStream_t st) {
   }
   const long long total = a.start[jobs.njobs];
   const int blocks = (int)std::min<long long>((total + 255) / 256, (long long)sm_count() * 8);
+  double bytes = 0;  // each output element written once, each input element read once
+  for (int k = 0; k < jobs.njobs; ++k) {
+    const PrepJob& J = jobs.job[k];
+    const double outs = (double)(a.start[k + 1] - a.start[k]);
+    bytes += J.kind == PREP_COPY_F32 ? outs * 6.0 : outs * (J.out_bf16 ? 2 : 4) + (double)J.N * J.r * 2;
+  }
+  profile_begin(st, GC_ELEM, 0.0, bytes);
   lora_prep_kernel<<<blocks, 256, 0, st>>>(a);
   SOUP_LAUNCH_CHECK();
+  profile_end(st);
   return SOUP_OK;
 }
 

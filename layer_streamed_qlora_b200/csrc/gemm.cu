@@ -91,6 +91,8 @@ struct KArgs {
   const float* rope_cos;
   const float* rope_sin;
   int* err;
+  long long wait_limit;  // clock cycles a bounded mbarrier wait may take before it gives up
+  int skip_producer;     // test hook (one-CTA kernel): the TMA producer issues nothing and never arrives
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -518,7 +520,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.wait_limit)) {
           atomicOr(args.err, 1);
           *abort_flag = 1;
           break;
@@ -586,7 +588,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (!ptx::mbar_wait_bounded(&full[s], ph, abort_flag)) {
+        if (!ptx::mbar_wait_bounded(&full[s], ph, abort_flag, args.wait_limit)) {
           atomicOr(args.err, 1);
           *abort_flag = 1;
           ok = false;
@@ -622,11 +624,11 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (lane == 0 && !args.skip_producer) {
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.wait_limit)) {
           atomicOr(args.err, 1);
           *abort_flag = 1;
           break;
@@ -686,7 +688,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (!ptx::mbar_wait_bounded(&full[s], ph, abort_flag)) {
+        if (!ptx::mbar_wait_bounded(&full[s], ph, abort_flag, args.wait_limit)) {
           atomicOr(args.err, 1);
           *abort_flag = 1;
           ok = false;
@@ -773,13 +775,13 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
       for (int it = 0; it < n_iters; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+        if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.wait_limit)) {
           atomicOr(args.err, 1);
           *abort_flag = 1;
           break;
         }
         if (it < num_kb) {
-          if (!ptx::mbar_wait_bounded(&cfull[s], ph, abort_flag)) {
+          if (!ptx::mbar_wait_bounded(&cfull[s], ph, abort_flag, args.wait_limit)) {
             atomicOr(args.err, 1);
             *abort_flag = 1;
             break;
@@ -831,7 +833,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
             load_codes(src + (size_t)(it + 1) * 32, wn);
             amn = __ldg(amp + it + 1);
           }
-          if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+          if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.wait_limit)) {
             atomicOr(args.err, 1);
             *abort_flag = 1;
             break;
@@ -876,7 +878,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
             load_codes(src + (size_t)(it + 1) * cstep, wn);
             amn = __ldg(amp + (size_t)(it + 1) * astep);
           }
-          if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+          if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.wait_limit)) {
             atomicOr(args.err, 1);
             *abort_flag = 1;
             break;
@@ -1592,6 +1594,8 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
               (!d.resid || (soup_aligned(d.resid, 16) && (d.ldr * 2) % 16 == 0)) &&
               (!d.resid_f32 || (soup_aligned(d.resid_f32, 16) && (d.ldr * 4) % 16 == 0)) &&
               (!d.aux16 || (soup_aligned(d.aux16, 16) && (d.ld_aux * 2) % 16 == 0 && (d.swiglu_I % 8) == 0));
+  ka.wait_limit = d.wait_limit > 0 ? d.wait_limit : 4000000000LL;
+  ka.skip_producer = d.debug_skip_producer;
   ka.rope_cols = d.rope_cols; ka.rope_S = d.rope_S;
   ka.rope_cos = d.rope_cos; ka.rope_sin = d.rope_sin;
   if (d.rope_cols > 0) {
@@ -1625,9 +1629,13 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
       SOUP_TRY(dispatch(d, kz, bn, st));
       const size_t total = (size_t)d.M * d.N;
       const int blocks = (int)std::min<size_t>((total + 255) / 256, (size_t)sms * 8);
+      const int oes = (d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T) ? 4 : 2;
+      profile_begin(st, GC_SPLITK, 0.0,
+                    (double)total * (4.0 * splits + oes + (d.out2 ? 4 : 0) + (d.out_lo ? 2 : 0)));
       splitk_reduce_kernel<<<blocks, 256, 0, st>>>(d.split_ws, splits, d.M, d.N, d.out_kind, d.out, d.out2,
                                                    d.out_lo, d.ldo, d.alpha, d.scale_amax);
       SOUP_LAUNCH_CHECK();
+      profile_end(st);
       return SOUP_OK;
     }
   }
@@ -1635,3 +1643,23 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
 }
 
 }  // namespace soup
+
+using namespace soup;
+
+extern "C" soup_status soup_debug_gemm_bounded_wait(const uint16_t* A, const uint16_t* B, int64_t M, int64_t N,
+                                                    int64_t K, float* C, int64_t wait_limit_cycles,
+                                                    int32_t skip_producer_arrivals, void* stream) {
+  SOUP_CHECK(A && B && C, SOUP_ERR_INVALID_ARG, "soup_debug_gemm_bounded_wait: null pointer");
+  SOUP_CHECK(M > 0 && N > 0 && K > 0 && M <= 4096 && N <= 4096 && K <= 4096 && K % 8 == 0 && N % 4 == 0,
+             SOUP_ERR_SHAPE, "soup_debug_gemm_bounded_wait: sizes must be in (0, 4096], K %% 8 == 0, N %% 4 == 0");
+  SOUP_CHECK(wait_limit_cycles >= 0, SOUP_ERR_INVALID_ARG, "soup_debug_gemm_bounded_wait: negative wait limit");
+  GemmDesc g;  // bf16 K-major operands: the one-CTA engine, no split-K
+  g.M = (int)M; g.N = (int)N; g.K = (int)K;
+  g.A = Mat{A, M, K, K};
+  g.b_mode = B_TMA_K;
+  g.B = Mat{B, N, K, K};
+  g.out_kind = OUT_F32; g.out = C; g.ldo = N;
+  g.wait_limit = wait_limit_cycles;
+  g.debug_skip_producer = skip_producer_arrivals ? 1 : 0;
+  return gemm(g, static_cast<cudaStream_t>(stream));
+}

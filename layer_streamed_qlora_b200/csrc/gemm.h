@@ -100,6 +100,12 @@ struct GemmDesc {
   // in slice order (deterministic) and applies the epilogue.
   float* split_ws = nullptr;
   size_t split_ws_bytes = 0;
+  // Clock cycles a bounded mbarrier wait in the kernel may take before the
+  // CTA records an error and winds down (0 = the default, ~2 s).
+  long long wait_limit = 0;
+  // Test hook, honoured by the one-CTA engine only: the TMA producer issues
+  // no loads and never arrives, so the MMA warp's bounded wait runs out.
+  int debug_skip_producer = 0;
 };
 
 soup_status gemm(const GemmDesc& d, cudaStream_t stream);

@@ -180,9 +180,11 @@ extern "C" soup_status soup_embed(const uint16_t* E, int64_t V, int64_t H, const
   SOUP_CHECK(soup_aligned(E, 16) && soup_aligned(h, 16), SOUP_ERR_ALIGN, "soup_embed: alignment");
   int* err = device_error_word();
   SOUP_CHECK(err, SOUP_ERR_CUDA, "device error word unavailable");
+  profile_begin(static_cast<cudaStream_t>(stream), GC_ELEM, 0.0, (double)T * (H * 4.0 + 4.0));
   embed_kernel<<<(unsigned)((T + 7) / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(E, V, (int)H, ids, (int)T, h,
                                                                                         err);
   SOUP_LAUNCH_CHECK();
+  profile_end(static_cast<cudaStream_t>(stream));
   return SOUP_OK;
 }
 
@@ -221,8 +223,10 @@ extern "C" soup_status soup_head_fwd_bwd(const uint16_t* h, const uint16_t* w_fi
     g.B = Mat{E, V, H, H};
     g.out_kind = OUT_F32; g.out = logits; g.ldo = V;
     SOUP_TRY(gemm(g, st));
+    profile_begin(st, GC_CE, 0.0, (double)c * V * (4.0 + (coef ? 2.0 : 0.0)) + c * 12.0);
     ce_rows_kernel<<<c, 1024, 0, st>>>(logits, V, ids, (int)t0, (int)seq, coef, logp, coef ? dlog : nullptr);
     SOUP_LAUNCH_CHECK();
+    profile_end(st);
     if (coef) {
       GemmDesc g2;  // dxn[t0:t0+c] = dlogits E
       g2.M = c; g2.N = (int)H; g2.K = (int)V;

@@ -195,29 +195,57 @@ static __device__ __align__(256) uint8_t g_lora_noalloc_scratch[SOUP_NOALLOC_SCR
 
 namespace {
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {nullptr};
+// Per device: the context the address was looked up in, and the address.
+struct NoallocAddr {
+  void* ctx = nullptr;
+  void* ptr = nullptr;
+};
+NoallocAddr g_noalloc[64];
+
+typedef int (*CtxGetCurrentFn)(void** ctx);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(f);
+  }();
+  return fn;
+}
 
 // Device address of the scratch array on the current device.  Host code may
 // not pass the array's name to a kernel (that is a host-side stand-in, not a
-// device address), so it is looked up once per device, with that device
-// current, and cached.
+// device address), so it is looked up with the device current, on the
+// device's first call, and cached together with the context it belongs to: a
+// call made in a new context (after cudaDeviceReset, say, which unloads the
+// module and with it the array) looks the address up again, and so does every
+// call while the thread has no current context to compare with.
 soup_status noalloc_scratch(void** out) {
   int dev = 0;
   SOUP_CUDA_TRY(cudaGetDevice(&dev));
   SOUP_CHECK(dev >= 0 && dev < 64, SOUP_ERR_INVALID_ARG, "soup_lora_linear_bwd_noalloc: device %d out of range", dev);
+  void* ctx = nullptr;
+  CtxGetCurrentFn get = ctx_get_current();
+  const bool known_ctx = get && get(&ctx) == 0 && ctx != nullptr;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocAddr& c = g_noalloc[dev];
+  if (!known_ctx || c.ptr == nullptr || c.ctx != ctx) {
     void* p = nullptr;
     SOUP_CUDA_TRY(cudaGetSymbolAddress(&p, g_lora_noalloc_scratch));
     SOUP_CHECK(p != nullptr && soup_aligned(p, 256), SOUP_ERR_CUDA, "soup_lora_linear_bwd_noalloc: bad scratch address");
-    g_noalloc_ptr[dev] = p;
+    c.ptr = p;
+    c.ctx = known_ctx ? ctx : nullptr;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = c.ptr;
   return SOUP_OK;
 }
 }  // namespace
 
 extern "C" size_t soup_lora_linear_bwd_noalloc_max_scratch(void) { return SOUP_NOALLOC_SCRATCH_BYTES; }
+
+extern "C" size_t soup_static_device_bytes(void) { return SOUP_NOALLOC_SCRATCH_BYTES; }
 
 extern "C" soup_status soup_lora_linear_bwd_noalloc(const soup_weight* W, const uint16_t* A, const uint16_t* B,
                                                     int32_t r, float scale, const uint16_t* x,

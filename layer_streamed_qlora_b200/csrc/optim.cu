@@ -135,9 +135,14 @@ extern "C" soup_status soup_adamw_step(float* theta, uint16_t* theta_bf16, float
   const int64_t cap = (int64_t)sm_count() * 8;  // 8 resident 256-thread blocks per SM
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;  // the scalar tail runs in block 0
+  // algorithmic bytes: theta, g, m, v read (16 B); theta, m, v written (12 B),
+  // g cleared (4 B) and the bf16 copy (2 B) when asked
+  profile_begin(static_cast<cudaStream_t>(stream), GC_ADAMW, 0.0,
+                (double)n * (28.0 + (zero_grad ? 4.0 : 0.0) + (theta_bf16 ? 2.0 : 0.0)));
   adamw_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<float4*>(theta), reinterpret_cast<uint2*>(theta_bf16), reinterpret_cast<float4*>(grad),
       reinterpret_cast<float4*>(m), reinterpret_cast<float4*>(v), n4, n, a, nonfinite_dev);
   SOUP_LAUNCH_CHECK();
+  profile_end(static_cast<cudaStream_t>(stream));
   return SOUP_OK;
 }

@@ -32,9 +32,13 @@ int sm_count();
 // through SOUP_LAUNCH_CHECK).
 void count_launch();
 
-// Optional CUDA-event timing of GEMM launches, by class, on the launching
-// stream (enabled through soup_profile_enable).
-enum GemmClass : int { GC_NF4_FWD = 0, GC_NF4_BWD = 1, GC_BF16 = 2, GC_SKINNY = 3, GC_NF4_DUAL = 4, GC_N = 5 };
+// Optional CUDA-event timing of kernel launches, by class, on the launching
+// stream (enabled through soup_profile_enable): the GEMM classes, attention,
+// and the memory-bound kernels tagged with their algorithmic bytes.
+enum GemmClass : int {
+  GC_NF4_FWD = 0, GC_NF4_BWD = 1, GC_BF16 = 2, GC_SKINNY = 3, GC_NF4_DUAL = 4,
+  GC_ATTN = 5, GC_RMSNORM = 6, GC_SPLITK = 7, GC_ELEM = 8, GC_CE = 9, GC_ADAMW = 10, GC_N = 11
+};
 bool profiling();
 void profile_begin(cudaStream_t st, int cls, double flops, double bytes);
 void profile_end(cudaStream_t st);

@@ -18,6 +18,64 @@
 
 #include "soup_internal.h"
 
+namespace {
+// Timing events of the stream's statistics, as a fixed ring: each prefetch
+// or wait records one (start, end) pair.  Before an entry is reused, its
+// elapsed time is folded into a running total, so a long training run holds
+// at most kTimedCap event pairs per ring however many steps it takes.
+struct TimedRing {
+  static constexpr size_t kCap = 256;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> ev;
+  size_t recorded = 0;     // pairs recorded since the last reset
+  double folded_ms = 0.0;  // elapsed time of the pairs already overwritten
+  // Next pair to record into; folds the previous lap's pair of this entry.
+  soup_status next(std::pair<cudaEvent_t, cudaEvent_t>** out) {
+    const size_t i = recorded % kCap;
+    if (i == ev.size()) {
+      cudaEvent_t a, b;
+      SOUP_CUDA_TRY(cudaEventCreate(&a));
+      if (cudaEventCreate(&b) != cudaSuccess) {
+        cudaEventDestroy(a);
+        return soup::fail(SOUP_ERR_CUDA, "timing event creation failed");
+      }
+      ev.emplace_back(a, b);
+    } else {
+      SOUP_CUDA_TRY(cudaEventSynchronize(ev[i].second));
+      float ms = 0.f;
+      SOUP_CUDA_TRY(cudaEventElapsedTime(&ms, ev[i].first, ev[i].second));
+      folded_ms += ms;
+    }
+    ++recorded;
+    *out = &ev[i];
+    return SOUP_OK;
+  }
+  // Total elapsed time of every pair recorded since the last reset.
+  soup_status total_ms(double* out) const {
+    double t = folded_ms;
+    const size_t live = std::min(recorded, ev.size());
+    for (size_t i = 0; i < live; ++i) {
+      SOUP_CUDA_TRY(cudaEventSynchronize(ev[i].second));
+      float ms = 0.f;
+      SOUP_CUDA_TRY(cudaEventElapsedTime(&ms, ev[i].first, ev[i].second));
+      t += ms;
+    }
+    *out = t;
+    return SOUP_OK;
+  }
+  void reset() {
+    recorded = 0;
+    folded_ms = 0.0;
+  }
+  void destroy() {
+    for (auto& pr : ev) {
+      cudaEventDestroy(pr.first);
+      cudaEventDestroy(pr.second);
+    }
+    ev.clear();
+  }
+};
+}  // namespace
+
 struct soup_plan {
   int n_layers = 0;
   size_t layer_bytes = 0, vocab_bytes = 0;
@@ -50,10 +108,8 @@ struct soup_plan {
   // statistics
   long long copies = 0, reuses = 0;
   size_t bytes_copied = 0;
-  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> stall_events;  // (before wait, after wait) on compute
-  size_t stall_used = 0;
-  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> copy_events;  // (start, end) of each copy on the copy stream
-  size_t copy_used = 0;
+  TimedRing stall_events;  // (before wait, after wait) on the compute stream
+  TimedRing copy_events;   // (start, end) of each copy on the copy stream
   bool fail_next_copy = false;
   cudaEvent_t gate = nullptr;   // test hook: the next copy waits on this event
 };
@@ -152,14 +208,8 @@ extern "C" soup_status soup_stream_plan_free(soup_plan* p) {
     if (sl.ready) cudaEventDestroy(sl.ready);
     if (sl.free_) cudaEventDestroy(sl.free_);
   }
-  for (auto& pr : p->stall_events) {
-    cudaEventDestroy(pr.first);
-    cudaEventDestroy(pr.second);
-  }
-  for (auto& pr : p->copy_events) {
-    cudaEventDestroy(pr.first);
-    cudaEventDestroy(pr.second);
-  }
+  p->stall_events.destroy();
+  p->copy_events.destroy();
   if (p->copy) cudaStreamDestroy(p->copy);
   if (p->copy2) cudaStreamDestroy(p->copy2);
   if (p->arena) cudaFree(p->arena);
@@ -213,13 +263,9 @@ soup_status prefetch_impl(soup_plan* p, int32_t item, const void* src_override, 
     SOUP_CUDA_TRY(cudaStreamWaitEvent(p->copy, p->gate, 0));
     p->gate = nullptr;
   }
-  if (p->copy_used == p->copy_events.size()) {
-    cudaEvent_t a, b;
-    SOUP_CUDA_TRY(cudaEventCreate(&a));
-    SOUP_CUDA_TRY(cudaEventCreate(&b));
-    p->copy_events.emplace_back(a, b);
-  }
-  auto& ce = p->copy_events[p->copy_used++];
+  std::pair<cudaEvent_t, cudaEvent_t>* cep = nullptr;
+  SOUP_TRY(p->copy_events.next(&cep));
+  auto& ce = *cep;
   SOUP_CUDA_TRY(cudaEventRecord(ce.first, p->copy));
   if (bytes >= (8u << 20)) {
     // second half on the second copy stream, after the same waits
@@ -274,13 +320,9 @@ extern "C" soup_status soup_stream_wait(soup_plan* p, int32_t item, void* comput
   SOUP_CHECK(s >= 0 && p->slots[s].pinned, SOUP_ERR_INVALID_ARG, "soup_stream_wait: item %d was not prefetched",
              item);
   cudaStream_t cs = static_cast<cudaStream_t>(compute_stream);
-  if (p->stall_used == p->stall_events.size()) {
-    cudaEvent_t a, b;
-    SOUP_CUDA_TRY(cudaEventCreate(&a));
-    SOUP_CUDA_TRY(cudaEventCreate(&b));
-    p->stall_events.emplace_back(a, b);
-  }
-  auto& pr = p->stall_events[p->stall_used++];
+  std::pair<cudaEvent_t, cudaEvent_t>* prp = nullptr;
+  SOUP_TRY(p->stall_events.next(&prp));
+  auto& pr = *prp;
   SOUP_CUDA_TRY(cudaEventRecord(pr.first, cs));
   SOUP_CUDA_TRY(cudaStreamWaitEvent(cs, p->slots[s].ready, 0));
   SOUP_CUDA_TRY(cudaEventRecord(pr.second, cs));
@@ -328,21 +370,11 @@ extern "C" soup_status soup_stream_stats(soup_plan* p, soup_stream_stats_t* out)
   out->reuses = p->reuses;
   out->bytes_copied = p->bytes_copied;
   out->arena_bytes = p->arena_bytes;
-  double stall = 0;
-  for (size_t i = 0; i < p->stall_used; ++i) {
-    SOUP_CUDA_TRY(cudaEventSynchronize(p->stall_events[i].second));
-    float ms = 0;
-    SOUP_CUDA_TRY(cudaEventElapsedTime(&ms, p->stall_events[i].first, p->stall_events[i].second));
-    stall += ms;
-  }
-  out->waits = (int64_t)p->stall_used;
+  double stall = 0, cms = 0;
+  SOUP_TRY(p->stall_events.total_ms(&stall));
+  SOUP_TRY(p->copy_events.total_ms(&cms));
+  out->waits = (int64_t)p->stall_events.recorded;
   out->stall_ms = stall;
-  double cms = 0;
-  for (size_t i = 0; i < p->copy_used; ++i) {
-    float ms = 0;
-    SOUP_CUDA_TRY(cudaEventElapsedTime(&ms, p->copy_events[i].first, p->copy_events[i].second));
-    cms += ms;
-  }
   out->copy_ms = cms;
   return SOUP_OK;
 }
@@ -352,8 +384,8 @@ extern "C" soup_status soup_stream_stats_reset(soup_plan* p) {
   SOUP_CUDA_TRY(cudaStreamSynchronize(p->copy));
   p->copies = p->reuses = 0;
   p->bytes_copied = 0;
-  p->stall_used = 0;
-  p->copy_used = 0;
+  p->stall_events.reset();
+  p->copy_events.reset();
   return SOUP_OK;
 }
 
@@ -370,3 +402,7 @@ extern "C" soup_status soup_stream_debug_gate_next_copy(soup_plan* p, void* even
 }
 
 extern "C" void* soup_stream_copy_stream(soup_plan* p) { return p ? p->copy : nullptr; }
+
+extern "C" int64_t soup_stream_debug_timing_events(soup_plan* p) {
+  return p ? (int64_t)(2 * (p->stall_events.ev.size() + p->copy_events.ev.size())) : -1;
+}

@@ -129,14 +129,15 @@ class AdamW:
 def device_bytes_lower_bound(cfg: ModelConfig, batch: int, seq: int, n_buffers: int, head_chunk: int) -> int:
     """Device bytes a streamed model needs at least, from the library's host
     size queries: the slot arena (n_buffers layer blobs + the vocab slot),
-    the layer checkpoints [L+1, T, H] bf16, the layer and head workspaces."""
+    the layer checkpoints [L+1, T, H] bf16, the layer and head workspaces,
+    and the library's module-static device arrays."""
     lcfg = cfg.layer_cfg()
     blob = L.soup_layer_blob_bytes(lcfg, cfg.weight_kind)
     vocab = (cfg.vocab * cfg.hidden * 2 + 255) // 256 * 256
     T = batch * seq
     return (n_buffers * blob + vocab + (cfg.n_layers + 1) * T * cfg.hidden * 2 +
             L.soup_decoder_layer_workspace(lcfg, batch, seq) +
-            L.soup_head_workspace(cfg.vocab, cfg.hidden, batch, seq, head_chunk))
+            L.soup_head_workspace(cfg.vocab, cfg.hidden, batch, seq, head_chunk) + L.static_device_bytes())
 
 
 def precheck_device_bytes(cfg, batch, seq, n_buffers, head_chunk, cap):
@@ -327,7 +328,10 @@ class StreamedLoRAModel:
         self.h_ref = None
         if self.task == "dpo":
             self.h_ref = torch.empty((2, T, cfg.hidden), dtype=torch.bfloat16, device="cuda")
-        self.reserve_bytes = torch.cuda.memory_allocated() - before
+        # what the model holds besides the slot arena: its own tensors and the
+        # library's module-static device arrays (held on every device that
+        # loads the library, outside torch's allocator)
+        self.reserve_bytes = torch.cuda.memory_allocated() - before + L.static_device_bytes()
 
     def views(self, base: int) -> L.LayerWeights:
         w = self._views.get(base)

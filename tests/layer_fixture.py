@@ -21,7 +21,7 @@ def quantize_dev(L, W32):
 class DevLayer:
     """Device tensors of one layer + the ctypes structs pointing at them."""
 
-    def __init__(self, L, shape, seed=0, layer=0, kind="nf4", zero_B=False, lora_std=0.02):
+    def __init__(self, L, shape, seed=0, layer=0, kind="nf4", zero_B=False, lora_std=0.02, check_codes=False):
         self.shape = shape
         Wf = ss.layer_weights_f32(shape, seed, layer)
         lo = ss.lora_params(shape, seed, layer, std=lora_std, zero_B=zero_B)
@@ -36,10 +36,17 @@ class DevLayer:
         self.W_oracle = {}
         for name, W32 in fused.items():
             if kind == "nf4":
+                # the GPU quantises the fp32 weights; the oracle quantises the
+                # same weights itself (no oracle input comes from the GPU)
                 codes, absmax = quantize_dev(L, W32)
                 self.keep += [codes, absmax]
                 structs[name] = L.weight_nf4(codes, absmax, *W32.shape)
-                deq = onf4.dequant_bf16(*onf4.quantize(W32)).astype(np.float64)
+                packed, am = onf4.quantize(W32)
+                if check_codes:
+                    assert np.array_equal(codes.cpu().numpy(), packed), f"{name}: NF4 codes differ"
+                    assert np.array_equal(absmax.cpu().numpy(), am), f"{name}: absmax differs"
+                deq = onf4.dequant_bf16(packed, am).astype(np.float64)
+                del packed, am
             elif kind == "nf4_stored":
                 # stored NF4 weights drawn directly (full-size layers: the
                 # oracle only dequantises, no fp64 quantisation of 218 M weights)

@@ -62,6 +62,26 @@ def test_workloads_and_config(bench):
 def test_oracle_projection(bench):
     w = dict(bench.WORKLOADS[bench.DEFAULT])
     # a layer sample of 256 tokens taking 2 s and an AdamW step of 0.5 s per
-    # 2048-token step, over 32 layers
-    per_tok = bench.oracle_seconds_per_token(w, 2.0, 0.5, 256)
-    assert per_tok == pytest.approx((2.0 / 256 + 0.5 / 2048) * 32, rel=1e-12)
+    # 2048-token step, over 32 layers; a head sample of 64 tokens over 1/8 of
+    # the vocabulary taking 0.25 s
+    per_tok = bench.oracle_seconds_per_token(w, 2.0, 0.5, 0.25, 256)
+    assert bench.HEAD_SAMPLE_TOKENS == 64 and bench.HEAD_VOCAB_FRACTION == 8
+    assert per_tok == pytest.approx((2.0 / 256 + 0.5 / 2048) * 32 + 0.25 * 8 / 64, rel=1e-12)
+
+
+def test_gpus_n_spawns_n_ranks_itself():
+    """`bench.py --gpus 2` without a launcher starts two ranks itself (RANK /
+    WORLD_SIZE / MASTER_* set for each), which join one process group; here
+    with the gloo backend and the launcher check only (no GPU)."""
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dist-check",
+                          "--backend", "gloo"], env=env, capture_output=True, text=True, timeout=240)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout  # rank 0 alone prints
+    d = lines[0]
+    assert d["n_gpus"] == 2 and d["ranks_joined"] == 2 and d["rank_sum"] == 3.0 and d["backend"] == "gloo"

@@ -123,3 +123,36 @@ def test_kept_qkv_backward_is_bit_identical(kind):
     ref, _ = layer_fwd(h, dl.Wd, dl.lora_np, shape)
     assert_close(host(out).reshape(h.shape), ref, "h_out (q|k|v from the hi + lo input)")
     assert_close(host(out).reshape(h.shape), o1, "h_out vs plain forward", rel=5e-3, maxrel=1e-2)
+
+
+@pytest.mark.parametrize("h_scale,norm_scale,dh_scale", [
+    (32.0, 1.0, 1.0),          # large residual stream (power of two: still bf16-exact)
+    (1.0, 4.0, 1.0),           # large normalised activations: q/k/v and g/u (fp16 inside the layer) x4
+    (1.0, 1.0, 2.0 ** -14),    # tiny upstream gradient: dO would underflow fp16 without its scale
+    (1.0, 1.0, 2.0 ** 10),     # large upstream gradient
+])
+def test_layer_holds_range(h_scale, norm_scale, dh_scale):
+    """Scaled hidden states, RMSNorm weights and upstream gradients (the
+    magnitudes real checkpoints produce, which the N(0, 1) inputs of the
+    other tests do not reach): the same oracle tolerances hold, so the fp16
+    q/k/v, g/u and scaled-dO paths keep their range."""
+    shape = SMALL
+    B, S = 2, 100
+    dl = DevLayer(L, shape, seed=8, kind="nf4")
+    if norm_scale != 1.0:
+        dl.norm1.mul_(norm_scale)  # powers of two: exact in bf16
+        dl.norm2.mul_(norm_scale)
+        dl.Wd["norm1"] = dl.Wd["norm1"] * norm_scale
+        dl.Wd["norm2"] = dl.Wd["norm2"] * norm_scale
+    h, dh = inputs(shape, B, S, seed=9)
+    h, dh = h * h_scale, dh * dh_scale
+    out, dhi = run_layer(dl, h, dh, B, S)
+    ref, cache = layer_fwd(h, dl.Wd, dl.lora_np, shape)
+    dref, gref = layer_bwd(cache, dl.Wd, dl.lora_np, shape, dh)
+    tag = f"x{h_scale}/{norm_scale}/{dh_scale}"
+    assert_close(out, ref, f"h_out {tag}")
+    assert_close(dhi, dref, f"dh_in {tag}")
+    got = dl.split_grads()
+    for p in ss.PROJ_NAMES:
+        assert_close(got[p][0], gref[p][0], f"dA_{p} {tag}")
+        assert_close(got[p][1], gref[p][1], f"dB_{p} {tag}")

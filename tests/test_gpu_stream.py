@@ -107,3 +107,57 @@ def test_injected_copy_failure_is_a_status():
     plan.prefetch(0)  # the next one works
     plan.wait_host(0, 10000)
     plan.free()
+
+
+def test_timing_events_stay_bounded_and_totals_survive_the_ring():
+    """1,200 prefetch / wait / release cycles (more than four laps of the
+    256-entry timing rings): the plan holds at most 1,024 events, and the
+    statistics still count every copy and wait, with totals no smaller
+    than those of the first 200 cycles."""
+    nb = 1 << 12
+    blobs = _blobs(3, nb)
+    plan = L.Plan(blobs, nb, 2)
+    n = 1200
+    for i in range(n):
+        item = i % 3
+        plan.prefetch(item)
+        plan.wait(item)
+        plan.release(item)
+        if i == 199:
+            torch.cuda.synchronize()
+            early = plan.stats()
+    torch.cuda.synchronize()
+    s = plan.stats()
+    assert plan.timing_events() <= 1024
+    assert s["copies"] + s["reuses"] == n and s["waits"] == n
+    assert s["bytes_copied"] == s["copies"] * nb
+    assert s["copy_ms"] >= early["copy_ms"] and s["stall_ms"] >= early["stall_ms"]
+    plan.reset_stats()
+    assert plan.stats()["waits"] == 0 and plan.stats()["copy_ms"] == 0.0
+    plan.free()
+
+
+def test_gemm_bounded_wait_runs_out_and_the_context_survives():
+    """The producer of a one-CTA tcgen05 GEMM is told to skip its arrivals and
+    the kernel's mbarrier waits are limited to 2e6 SM cycles (~1 ms): the MMA
+    warp's wait runs out, the kernel records code 1 in the device error word
+    and returns (no MMA, tensor memory freed, output untouched).  The same
+    device then runs the GEMM normally, and it matches a float64 reference."""
+    g = torch.Generator(device="cuda").manual_seed(3)
+    M, N, K = 256, 128, 192
+    A = torch.randn(M, K, device="cuda", generator=g).bfloat16()
+    B = torch.randn(N, K, device="cuda", generator=g).bfloat16()
+    C = torch.full((M, N), 7.0, device="cuda")
+    assert L.device_error() == 0
+    t0 = time.time()
+    L.soup_debug_gemm_bounded_wait(A, B, C, wait_limit_cycles=2_000_000, skip_producer_arrivals=True)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 5.0
+    assert L.device_error() == 1
+    assert torch.all(C == 7.0)  # nothing was written
+    L.soup_debug_gemm_bounded_wait(A, B, C, wait_limit_cycles=2_000_000, skip_producer_arrivals=False)
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    ref = A.double() @ B.double().T
+    err = (C.double() - ref).norm() / ref.norm()
+    assert err < 1e-4, float(err)

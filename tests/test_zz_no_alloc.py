@@ -83,3 +83,40 @@ def test_noalloc_refuses_sizes_beyond_its_scratch(L):
     assert "static maximum" in str(e.value)
     torch.cuda.synchronize()
     assert torch.isnan(dA).all()  # nothing ran
+
+
+def _free_bytes():
+    free, _ = torch.cuda.mem_get_info()
+    return free
+
+
+def test_noalloc_allocates_nothing_and_fills_its_whole_scratch(L):
+    """A size whose scratch is exactly the static maximum (r = 16, out = 64,
+    a ragged T with round_up8(T) * r * 2 + the B^T part = 8 MiB): the second
+    call leaves the device's free memory and torch's allocated bytes
+    unchanged, and both calls match the workspace path."""
+    cap = L.soup_lora_linear_bwd_noalloc_max_scratch()
+    r, n_out, n_in = 16, 64, 128
+    T = (cap - 256 * ((r * n_out * 2 + 255) // 256)) // (2 * r) - 5  # ragged: round_up8(T) lands on the limit
+    need = L.soup_lora_linear_bwd_workspace(T, r, n_out)
+    assert cap - 256 < need <= cap, (T, need, cap)
+    t, T, n_in, n_out, r = _problem(L, T=T, n_in=n_in, n_out=n_out, r=r, seed=12)
+    dx0, dA0, dB0 = _outs(T, n_in, n_out, r)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    L.soup_lora_linear_bwd(t["W"], t["A"], t["B"], r, 2.0, t["x"], t["u"], t["dy"], T, dx0, dA0, dB0, ws)
+    torch.cuda.synchronize()
+    ref = (host(dx0), host(dA0), host(dB0))
+    del ws, dx0, dA0, dB0
+    outs = [_outs(T, n_in, n_out, r) for _ in range(2)]
+    for call in range(2):
+        dx, dA, dB = outs[call]
+        torch.cuda.synchronize()
+        free0, alloc0 = _free_bytes(), torch.cuda.memory_allocated()
+        L.soup_lora_linear_bwd_noalloc(t["W"], t["A"], t["B"], r, 2.0, t["x"], t["u"], t["dy"], T, dx, dA, dB)
+        torch.cuda.synchronize()
+        if call == 1:  # the first call may load the library's module (and its static array)
+            assert _free_bytes() == free0, "the allocation-free backward changed the device's free memory"
+            assert torch.cuda.memory_allocated() == alloc0
+        for name, got, want in zip(("dx", "dA", "dB"), (host(dx), host(dA), host(dB)), ref):
+            assert_close(got, want, f"near-limit call {call}: {name}")
+    assert L.device_error() == 0
