@@ -202,6 +202,32 @@ soup_status soup_lora_linear_bwd_noalloc(const soup_weight* W, const uint16_t* A
                                          const uint16_t* u_save, const uint16_t* dy, int64_t T,
                                          uint16_t* dx, float* dA, float* dB, void* stream);
 
+/* ------------------------------------------------------------- attention ---
+ * The decoder layer's causal GQA attention on its own (Soup pages, "how layer
+ * streaming works": the layer the stream feeds; the attention itself is the
+ * Llama-3.1-8B layer's: causal within each sequence, kv head = q head /
+ * (n_q_heads / n_kv_heads), scale 1/sqrt(128)).  head_dim is 128.
+ * qkv: [batch * seq, ld] fp16 (ld >= (n_q + 2 n_kv) * 128, ld % 8 == 0, base
+ * 16-byte aligned): q heads at columns [0, 128 n_q), k heads after them, then
+ * v heads; tokens batch-major (sequence b is rows [b*seq, (b+1)*seq)); q and k
+ * as they enter the dot products (after RoPE).
+ * soup_attention_fwd: out [batch*seq, 128 n_q] bf16, out16 (may be NULL) the
+ * same values in fp16, lse [n_q, batch*seq] fp32 = log2 of each row's softmax
+ * denominator including the row maximum (log2 units).
+ * soup_attention_bwd: from the forward's out16 and lse and dout [batch*seq,
+ * 128 n_q] fp16, writes D [n_q, batch*seq] (rowsum(dout * out), a buffer the
+ * caller provides) and dq, dk, dv (bf16) into dqkv at qkv's layout (dq
+ * includes the 1/sqrt(128) scale; row stride ld), and the same values in fp32
+ * into dqkv32 when it is not NULL.  Both run on the tensor cores (tcgen05,
+ * accumulators in tensor memory), are deterministic, and are async on
+ * `stream`.  Refusals: SOUP_ERR_SHAPE (bad sizes, n_q % n_kv != 0),
+ * SOUP_ERR_ALIGN. */
+soup_status soup_attention_fwd(const uint16_t* qkv, int64_t ld, int64_t batch, int64_t seq, int32_t n_q_heads,
+                               int32_t n_kv_heads, uint16_t* out, uint16_t* out16, float* lse, void* stream);
+soup_status soup_attention_bwd(const uint16_t* qkv, int64_t ld, int64_t batch, int64_t seq, int32_t n_q_heads,
+                               int32_t n_kv_heads, const uint16_t* out16, const uint16_t* dout, const float* lse,
+                               float* D, uint16_t* dqkv, float* dqkv32, void* stream);
+
 /* --------------------------------------------------------- decoder layer ---
  * One Llama-style decoder layer with LoRA on all seven projections (the unit
  * the pages stream "one decoder layer at a time"; Soup pages, "layer

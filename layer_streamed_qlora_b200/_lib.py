@@ -142,6 +142,10 @@ _SIGS = {
     "soup_stream_copy_stream": (c_void_p, [c_void_p]),
     "soup_stream_debug_timing_events": (c_int64, [c_void_p]),
     "soup_static_device_bytes": (c_size_t, []),
+    "soup_attention_fwd": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_int32, c_int32, c_void_p, c_void_p,
+                                     c_void_p, c_void_p]),
+    "soup_attention_bwd": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_int32, c_int32, c_void_p, c_void_p,
+                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "soup_debug_gemm_bounded_wait": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64,
                                                c_int32, c_void_p]),
     "soup_stream_debug_fail_next_copy": (c_int32, [c_void_p]),
@@ -224,6 +228,19 @@ def soup_debug_gemm_bounded_wait(A, B, C, wait_limit_cycles=0, skip_producer_arr
     N = B.shape[0]
     _check("soup_debug_gemm_bounded_wait", lib().soup_debug_gemm_bounded_wait(
         _p(A), _p(B), M, N, K, _p(C), int(wait_limit_cycles), 1 if skip_producer_arrivals else 0, _stream(stream)))
+
+
+def soup_attention_fwd(qkv, batch, seq, n_q, n_kv, out, out16, lse, stream=None):
+    """Causal GQA attention forward on the q|k|v rows (fp16 [batch*seq, ld])."""
+    _check("soup_attention_fwd", lib().soup_attention_fwd(_p(qkv), qkv.shape[1], batch, seq, n_q, n_kv, _p(out),
+                                                          _p(out16), _p(lse), _stream(stream)))
+
+
+def soup_attention_bwd(qkv, batch, seq, n_q, n_kv, out16, dout, lse, D, dqkv, dqkv32=None, stream=None):
+    """Backward of soup_attention_fwd: dq|dk|dv into dqkv (bf16, qkv's layout)."""
+    _check("soup_attention_bwd", lib().soup_attention_bwd(_p(qkv), qkv.shape[1], batch, seq, n_q, n_kv, _p(out16),
+                                                          _p(dout), _p(lse), _p(D), _p(dqkv), _p(dqkv32),
+                                                          _stream(stream)))
 
 
 def static_device_bytes() -> int:

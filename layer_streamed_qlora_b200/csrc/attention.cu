@@ -1,521 +1,917 @@
-// Causal GQA attention (head_dim 128) for the decoder layer: flash-style
-// forward with online softmax, and a two-pass backward that needs no atomics
-// (pass 1: dK, dV per key block, summing the q heads of the group in a fixed
-// order; pass 2: dQ per query block), so every run gives the same bits.
+// Causal GQA attention (head_dim 128) of the decoder layer on the fifth-
+// generation tensor cores: tcgen05.mma with the accumulators in tensor memory,
+// operand tiles brought into 128-byte-swizzled shared memory by TMA (no
+// cluster multicast), warp-specialised CTAs (one TMA thread, one MMA thread,
+// four softmax / epilogue warps, one query or key row per thread).
 //
-// Tensor-core path: warp-level mma.sync m16n8k16 with fp16 operands and fp32
-// accumulation, ldmatrix operand loads from padded shared-memory tiles;
-// softmax in fp32 in the log2 domain; the saved log-sum-exp is in log2 units.
+//   forward   per (128-query tile, q head): S_j = Q K_j^T into tensor memory,
+//             online softmax in fp32 (log2 domain) from a two-pass read of the
+//             row (max, then 2^(s - m) and the row sum), P_j in fp16 into
+//             shared memory, O_j = P_j V_j into a fresh tensor-memory
+//             accumulator, folded into the row's fp32 running output in
+//             registers with the online-softmax correction.  S and O are
+//             double-buffered in tensor memory (4 x 128 columns), so the
+//             tensor cores compute S_{j+1} and O_j while the softmax warps
+//             work on block j.
+//   backward  two passes, no atomics (every run gives the same bits):
+//             pass 1 per (128-key block, kv head): for each q head of the group
+//             and each 64-query tile at or after the block, S^T = K Q^T and
+//             dP^T = V dO^T (tensor memory), P^T = 2^(S^T scale - L) and
+//             dS^T = P^T (dP^T - D) in fp16 into shared memory, then
+//             dV += P^T dO and dK += dS^T Q accumulated in tensor memory;
+//             pass 2 per (128-query tile, q head): S = Q K^T, dP = dO V^T per
+//             64-key block, dS into shared memory, dQ += dS K in tensor memory.
+//             Q, dO (pass 1) and K (pass 2) tiles serve both as K-major and as
+//             MN-major operands of the same shared-memory bytes.
+//
 // Inputs q, k, v and dO are fp16 (the projections write them in fp16: same
-// 16-bit traffic as bf16 with 8x finer rounding for these O(1) values), the
-// probabilities P and dS enter the MMAs as fp16; outputs (attention output,
-// dq, dk, dv) are bf16, the operand type of the projection GEMMs.
+// 16-bit traffic as bf16 with 8x finer rounding for these O(1) values), P and
+// dS enter the MMAs as fp16, accumulation is fp32; the saved log-sum-exp is
+// in log2 units.  Outputs (attention output, dq, dk, dv) are bf16, with
+// optional fp16 / fp32 copies.  Every mbarrier wait is bounded: on expiry the
+// CTA records code 2 in the device error word, stops issuing work, lets copies
+// and MMAs in flight land, frees its tensor memory and returns.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "elementwise.h"
 #include "gscale.cuh"
+#include "ptx.cuh"
 
 namespace soup {
 namespace {
 
-constexpr int HD = 128;   // head dim
-constexpr int LDS = 136;  // padded smem row (elements): conflict-free ldmatrix
+constexpr int HD = 128;          // head dim
+constexpr int ERR_ATTN_WAIT = 2;  // device error code: a bounded wait of an attention kernel expired
 
-__device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(su32(p)));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(su32(p)));
-}
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t packbf(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ uint32_t packh(float lo, float hi) {
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(dst)), "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
+__device__ __forceinline__ uint32_t pack_b2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// One 16-byte unit (8 16-bit values) of row r of a K-major 128-byte-swizzled
+// tile (rows of 128 bytes; unit u of row r stored at unit u ^ (r % 8)).
+__device__ __forceinline__ void st_unit(uint8_t* tile, int r, int u, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  *reinterpret_cast<uint4*>(tile + r * 128 + ((u ^ (r & 7)) << 4)) = make_uint4(a, b, c, d);
 }
-
-// Loads `rows` rows of a head (128 bf16 each) starting at token row `r0` of
-// sequence-local index `s0` (rows with s0 + r >= S are zero-filled).
-__device__ __forceinline__ void load_tile(uint16_t* dst, const uint16_t* base, int ld, int col, int r0, int s0,
-                                          int S, int rows, int tid, int nthr) {
-  for (int idx = tid; idx < rows * 16; idx += nthr) {
-    const int r = idx >> 4, c = (idx & 15) * 8;
-    const bool ok = (s0 + r) < S;
-    const uint16_t* src = base + (size_t)(ok ? r0 + r : r0) * ld + col + c;
-    cp_async16(dst + r * LDS + c, src, ok);
-  }
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+// K-major operand descriptor: 128-byte rows, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return ptx::smem_desc_sw128(saddr, 16, 1024); }
+// MN-major operand descriptor: 64-element MN chunks `chunk` bytes apart.
+__device__ __forceinline__ uint64_t mndesc(uint32_t saddr, uint32_t chunk) {
+  return ptx::smem_desc_sw128(saddr, chunk, 1024);
 }
 
-// A fragment (16x16) address for this lane from a row-major tile.
-__device__ __forceinline__ const uint16_t* a_addr(const uint16_t* tile, int row0, int col0, int lane) {
-  const int mi = lane >> 3, ri = lane & 7;
-  return tile + (row0 + (mi & 1) * 8 + ri) * LDS + col0 + (mi >> 1) * 8;
-}
-// Two B fragments (n-tiles n0, n0+8; k16) from a tile stored [n][k] (non-trans).
-__device__ __forceinline__ const uint16_t* bn_addr(const uint16_t* tile, int n0, int k0, int lane) {
-  const int mi = lane >> 3, ri = lane & 7;
-  return tile + (n0 + (mi >> 1) * 8 + ri) * LDS + k0 + (mi & 1) * 8;
-}
-// Two B fragments (n-tiles n0, n0+8; k16) from a tile stored [k][n] (trans).
-__device__ __forceinline__ const uint16_t* bk_addr(const uint16_t* tile, int k0, int n0, int lane) {
-  const int mi = lane >> 3, ri = lane & 7;
-  return tile + (k0 + (mi & 1) * 8 + ri) * LDS + n0 + (mi >> 1) * 8;
-}
+struct AttnArgs {
+  int S, Hq, Hkv, T;
+  float scale_log2;  // log2(e) / sqrt(head_dim)
+  float scale;       // 1 / sqrt(head_dim)
+  // forward
+  uint16_t* out;
+  float* lse;
+  uint16_t* out16;
+  float* out32;
+  // backward
+  const float* L;  // [Hq, T] log2-domain log-sum-exp of the forward pass
+  const float* D;  // [Hq, T] rowsum(dO * O)
+  uint16_t* dqkv;  // [T, ld] bf16
+  float* dqkv32;   // [T, ld] fp32 or null
+  int ld;
+  const float* rcos;  // [S, 64] or null: rotate dq / dk back
+  const float* rsin;
+  const unsigned int* amax;  // dO's power-of-two gradient scale, or null
+  int* err;
+  long long wait_limit;
+};
 
+#define ATTN_WAIT(bar, parity)                                                   \
+  (ptx::mbar_wait_bounded((bar), (parity), abort_flag, a.wait_limit) ||          \
+   (atomicOr(a.err, ERR_ATTN_WAIT), *abort_flag = 1, false))
 
-// Stores one row (this lane's 16 x 2 columns of a 128-wide head) scaled by
-// `scale`, rotating pairs (i, i+64) back by the position's angle when tables
-// are given: (a, b) -> (a c + b s, b c - a s).
-__device__ __forceinline__ void store_row_rot(uint16_t* p, const float (&acc)[16][4], int e0, float scale,
-                                              const float* cosr, const float* sinr, int t4, float* p32 = nullptr) {
-#pragma unroll
-  for (int dt = 0; dt < 8; ++dt) {
-    float a0 = acc[dt][e0] * scale, a1 = acc[dt][e0 + 1] * scale;
-    float b0 = acc[dt + 8][e0] * scale, b1 = acc[dt + 8][e0 + 1] * scale;
-    if (cosr) {
-      const int c = dt * 8 + 2 * t4;
-      const float c0 = cosr[c], c1 = cosr[c + 1], s0 = sinr[c], s1 = sinr[c + 1];
-      const float ra0 = a0 * c0 + b0 * s0, rb0 = b0 * c0 - a0 * s0;
-      const float ra1 = a1 * c1 + b1 * s1, rb1 = b1 * c1 - a1 * s1;
-      a0 = ra0; a1 = ra1; b0 = rb0; b1 = rb1;
-    }
-    *reinterpret_cast<uint32_t*>(p + dt * 8 + 2 * t4) = packbf(a0, a1);
-    *reinterpret_cast<uint32_t*>(p + 64 + dt * 8 + 2 * t4) = packbf(b0, b1);
-    if (p32) {
-      *reinterpret_cast<float2*>(p32 + dt * 8 + 2 * t4) = make_float2(a0, a1);
-      *reinterpret_cast<float2*>(p32 + 64 + dt * 8 + 2 * t4) = make_float2(b0, b1);
-    }
-  }
-}
-
-// ------------------------------------------------------------------ forward
-__global__ void __launch_bounds__(128) attn_fwd_kernel(const uint16_t* __restrict__ qkv, int ld, int S, int Hq,
-                                                        int Hkv, uint16_t* __restrict__ out,
-                                                        float* __restrict__ lse, float scale_log2,
-                                                        uint16_t* __restrict__ out16, float* __restrict__ out32) {
-  extern __shared__ __align__(16) uint16_t sm[];
-  uint16_t* Qs = sm;
-  uint16_t* Ks = Qs + 64 * LDS;   // 2 buffers
-  uint16_t* Vs = Ks + 2 * 64 * LDS;
-  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g4 = lane >> 2, t4 = lane & 3;
-  const int T = gridDim.z * S;
-  const int grp = Hq / Hkv, kvh = h / grp;
-  const int qcol = h * HD, kcol = (Hq + kvh) * HD, vcol = (Hq + Hkv + kvh) * HD;
-  const int row0 = b * S;
-  load_tile(Qs, qkv, ld, qcol, row0 + qb * 64, qb * 64, S, 64, tid, 128);
-  load_tile(Ks, qkv, ld, kcol, row0, 0, S, 64, tid, 128);
-  load_tile(Vs, qkv, ld, vcol, row0, 0, S, 64, tid, 128);
-  cp_commit();
-  cp_wait<0>();
+// Tail of every attention kernel: all threads meet, a CTA that gave up lets
+// copies and MMAs in flight land (~1 ms, bounded), then warp 1 frees the
+// tensor memory.
+__device__ __forceinline__ void attn_teardown(volatile int* abort_flag, int warp, uint32_t tmem) {
+  ptx::tc_fence_before();
   __syncthreads();
-  uint32_t qf[8][4];
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) ldsm_x4(qf[kk], a_addr(Qs, warp * 16, kk * 16, lane));
-  float o[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  const int qr0 = qb * 64 + warp * 16 + g4, qr1 = qr0 + 8;
-  const int nkb = qb + 1;
-  for (int j = 0; j < nkb; ++j) {
-    if (j + 1 < nkb) {
-      load_tile(Ks + ((j + 1) & 1) * 64 * LDS, qkv, ld, kcol, row0 + (j + 1) * 64, (j + 1) * 64, S, 64, tid, 128);
-      load_tile(Vs + ((j + 1) & 1) * 64 * LDS, qkv, ld, vcol, row0 + (j + 1) * 64, (j + 1) * 64, S, 64, tid, 128);
-      cp_commit();
-      cp_wait<1>();
-    } else {
-      cp_wait<0>();
-    }
-    __syncthreads();
-    const uint16_t* Kb = Ks + (j & 1) * 64 * LDS;
-    const uint16_t* Vb = Vs + (j & 1) * 64 * LDS;
-    float s[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-      for (int nt2 = 0; nt2 < 4; ++nt2) {
-        uint32_t bf[4];
-        ldsm_x4(bf, bn_addr(Kb, nt2 * 16, kk * 16, lane));
-        mma16816(s[2 * nt2], qf[kk], bf[0], bf[1]);
-        mma16816(s[2 * nt2 + 1], qf[kk], bf[2], bf[3]);
-      }
-    }
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = j * 64 + nt * 8 + 2 * t4 + (e & 1);
-        const int qr = (e < 2) ? qr0 : qr1;
-        float v = s[nt][e] * scale_log2;
-        if (key > qr || key >= S) v = -INFINITY;
-        s[nt][e] = v;
-      }
-      mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
-      mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float c0 = (mn0 == -INFINITY) ? 1.f : exp2f(m0 - mn0);
-    const float c1 = (mn1 == -INFINITY) ? 1.f : exp2f(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    float sum0 = 0.f, sum1 = 0.f;
-    uint32_t pa[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const float p0 = (s[nt][0] == -INFINITY) ? 0.f : exp2f(s[nt][0] - mn0);
-      const float p1 = (s[nt][1] == -INFINITY) ? 0.f : exp2f(s[nt][1] - mn0);
-      const float p2 = (s[nt][2] == -INFINITY) ? 0.f : exp2f(s[nt][2] - mn1);
-      const float p3 = (s[nt][3] == -INFINITY) ? 0.f : exp2f(s[nt][3] - mn1);
-      sum0 += p0 + p1;
-      sum1 += p2 + p3;
-      pa[nt >> 1][(nt & 1) * 2 + 0] = packh(p0, p1);
-      pa[nt >> 1][(nt & 1) * 2 + 1] = packh(p2, p3);
-    }
-    l0 = l0 * c0 + sum0;
-    l1 = l1 * c1 + sum1;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      o[i][0] *= c0; o[i][1] *= c0; o[i][2] *= c1; o[i][3] *= c1;
-    }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-      for (int dt2 = 0; dt2 < 8; ++dt2) {
-        uint32_t bf[4];
-        ldsm_x4_t(bf, bk_addr(Vb, kk * 16, dt2 * 16, lane));
-        mma16816(o[2 * dt2], pa[kk], bf[0], bf[1]);
-        mma16816(o[2 * dt2 + 1], pa[kk], bf[2], bf[3]);
-      }
+  if (*abort_flag) {
+    const long long t0 = clock64();
+    while (clock64() - t0 < 2000000LL) {
     }
     __syncthreads();
   }
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  const float i0 = 1.f / l0, i1 = 1.f / l1;
-  const int ldo = Hq * HD;
-  if (qr0 < S) {
-    const size_t off = (size_t)(row0 + qr0) * ldo + h * HD;
-#pragma unroll
-    for (int dt = 0; dt < 16; ++dt) {
-      *reinterpret_cast<uint32_t*>(out + off + dt * 8 + 2 * t4) = packbf(o[dt][0] * i0, o[dt][1] * i0);
-      if (out16) *reinterpret_cast<uint32_t*>(out16 + off + dt * 8 + 2 * t4) = packh(o[dt][0] * i0, o[dt][1] * i0);
-      if (out32) *reinterpret_cast<float2*>(out32 + off + dt * 8 + 2 * t4) = make_float2(o[dt][0] * i0, o[dt][1] * i0);
-    }
-    if (t4 == 0) lse[(size_t)h * T + row0 + qr0] = m0 + log2f(l0);
-  }
-  if (qr1 < S) {
-    const size_t off = (size_t)(row0 + qr1) * ldo + h * HD;
-#pragma unroll
-    for (int dt = 0; dt < 16; ++dt) {
-      *reinterpret_cast<uint32_t*>(out + off + dt * 8 + 2 * t4) = packbf(o[dt][2] * i1, o[dt][3] * i1);
-      if (out16) *reinterpret_cast<uint32_t*>(out16 + off + dt * 8 + 2 * t4) = packh(o[dt][2] * i1, o[dt][3] * i1);
-      if (out32) *reinterpret_cast<float2*>(out32 + off + dt * 8 + 2 * t4) = make_float2(o[dt][2] * i1, o[dt][3] * i1);
-    }
-    if (t4 == 0) lse[(size_t)h * T + row0 + qr1] = m1 + log2f(l1);
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
   }
 }
 
-// --------------------------------------------------- backward pass 1: dK, dV
-// CTA = 64 keys (4 warps x 16) of one kv head; loops over the group's q heads
-// and over query blocks of 32 at or after the key block.
-__global__ void __launch_bounds__(128) attn_bwd_dkdv_kernel(const uint16_t* __restrict__ qkv, int ld, int S, int Hq,
-                                                             int Hkv, const uint16_t* __restrict__ dout,
-                                                             const float* __restrict__ lse,
-                                                             const float* __restrict__ Dd,
-                                                             uint16_t* __restrict__ dqkv, float scale_log2,
-                                                             float scale, const float* __restrict__ rcos,
-                                                             const float* __restrict__ rsin,
-                                                             const unsigned int* __restrict__ amax,
-                                                             float* __restrict__ dqkv32) {
-  extern __shared__ __align__(16) uint16_t sm[];
-  uint16_t* Ks = sm;
-  uint16_t* Vs = Ks + 64 * LDS;
-  uint16_t* Qs = Vs + 64 * LDS;        // 2 x 32 rows
-  uint16_t* Os = Qs + 2 * 32 * LDS;    // dO, 2 x 32 rows
-  float* Ls = reinterpret_cast<float*>(Os + 2 * 32 * LDS);  // 2 x 32
-  float* Ds = Ls + 64;                                       // 2 x 32
-  const int kb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g4 = lane >> 2, t4 = lane & 3;
-  const int T = gridDim.z * S;
-  const int grp = Hq / Hkv;
-  const int kcol = (Hq + kvh) * HD, vcol = (Hq + Hkv + kvh) * HD;
+// Rotates the pair (i, i + 64) of a 128-wide head back by the position's
+// angle: (a, b) -> (a c + b s, b c - a s).
+__device__ __forceinline__ void rope_back(float& x0, float& x1, float c, float s) {
+  const float a = x0 * c + x1 * s, b = x1 * c - x0 * s;
+  x0 = a;
+  x1 = b;
+}
+
+// ====================================================================== forward
+// Shared memory: Q tile (2 chunks x 16 KB), 2 K|V stages (64 KB each), 2 P
+// buffers (32 KB each), barriers, the partial row sums.  Warps: 0 TMA, 1 MMA,
+// 2..9 softmax (two per row).
+constexpr int F_Q = 0, F_KV = 32768, F_P = F_KV + 2 * 65536, F_BAR = F_P + 2 * 32768;
+constexpr int F_SMEM = F_BAR + 256 + 1024 + 1024;
+
+__global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CUtensorMap tm, const AttnArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + F_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 3;
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_free = bars + 7;
+  uint64_t* p_full = bars + 9;
+  uint64_t* p_empty = bars + 11;
+  uint64_t* o_full = bars + 13;
+  uint64_t* o_free = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* lsum = reinterpret_cast<float*>(sm + F_BAR + 256);  // [2][128] partial row sums
+
+  const int S = a.S;
+  const int nqt = (S + 127) / 128;
+  const int qb = nqt - 1 - (int)blockIdx.x;  // the longest rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (a.Hq / a.Hkv);
   const int row0 = b * S;
-  const int ldo = Hq * HD;
-  load_tile(Ks, qkv, ld, kcol, row0 + kb * 64, kb * 64, S, 64, tid, 128);
-  load_tile(Vs, qkv, ld, vcol, row0 + kb * 64, kb * 64, S, 64, tid, 128);
-  cp_commit();
-  const int qb_first = (kb * 64) / 32;
-  const int nqb = (S + 31) / 32;
-  const int per_head = nqb - qb_first;
+  const int nkb = qb + 1;
+  const int qcol = h * HD, kcol = (a.Hq + g) * HD, vcol = (a.Hq + a.Hkv + g) * HD;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&kv_full[i], 1);
+      ptx::mbar_init(&kv_empty[i], 1);
+      ptx::mbar_init(&s_full[i], 1);
+      ptx::mbar_init(&s_free[i], 8);
+      ptx::mbar_init(&p_full[i], 8);
+      ptx::mbar_init(&p_empty[i], 1);
+      ptx::mbar_init(&o_full[i], 1);
+      ptx::mbar_init(&o_free[i], 8);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tm);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;  // columns: S[0] 0, S[1] 128, O[0] 256, O[1] 384
+  bool ok = true;
+  float o[64];  // softmax warps: this thread's 64 output columns, unnormalised
+  float m = -INFINITY;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      const int qrow = row0 + qb * 128;
+      ptx::mbar_arrive_expect_tx(q_full, 32768);
+      ptx::tma_load_2d(sm + F_Q, &tm, q_full, qcol, qrow);
+      ptx::tma_load_2d(sm + F_Q + 16384, &tm, q_full, qcol + 64, qrow);
+      for (int j = 0; j < nkb; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!ATTN_WAIT(&kv_empty[s], ph ^ 1)) break;
+        uint8_t* kv = sm + F_KV + s * 65536;
+        const int r = row0 + j * 128;
+        ptx::mbar_arrive_expect_tx(&kv_full[s], 65536);
+        ptx::tma_load_2d(kv, &tm, &kv_full[s], kcol, r);
+        ptx::tma_load_2d(kv + 16384, &tm, &kv_full[s], kcol + 64, r);
+        ptx::tma_load_2d(kv + 32768, &tm, &kv_full[s], vcol, r);
+        ptx::tma_load_2d(kv + 49152, &tm, &kv_full[s], vcol + 64, r);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_s = ptx::idesc_fmt(128, 128, 0, 0, 0u);  // fp16 A, B; fp32 D
+      constexpr uint32_t id_o = ptx::idesc_fmt(128, 128, 0, 1, 0u);  // V: MN-major B
+      const uint32_t qa = ptx::smem_u32(sm + F_Q);
+      const bool go = ATTN_WAIT(q_full, 0);
+      for (int jj = 0; go && jj <= nkb; ++jj) {
+        if (jj < nkb) {  // S_jj = Q K_jj^T
+          const int s = jj & 1;
+          const uint32_t ph = (jj >> 1) & 1;
+          if (!ATTN_WAIT(&kv_full[s], ph) || !ATTN_WAIT(&s_free[s], ph ^ 1)) break;
+          ptx::tc_fence_after();
+          const uint32_t ka = ptx::smem_u32(sm + F_KV + s * 65536);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            ptx::mma_bf16(tmem + s * 128, kdesc(qa + (k >> 2) * 16384 + (k & 3) * 32),
+                          kdesc(ka + (k >> 2) * 16384 + (k & 3) * 32), id_s, k > 0 ? 1u : 0u);
+          ptx::mma_commit(&s_full[s]);
+        }
+        if (jj >= 1) {  // O_j = P_j V_j, j = jj - 1
+          const int j = jj - 1, s = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          if (!ATTN_WAIT(&p_full[s], ph) || !ATTN_WAIT(&o_free[s], ph ^ 1)) break;
+          ptx::tc_fence_after();
+          const uint32_t pa = ptx::smem_u32(sm + F_P + s * 32768);
+          const uint32_t va = ptx::smem_u32(sm + F_KV + s * 65536 + 32768);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            ptx::mma_bf16(tmem + 256 + s * 128, kdesc(pa + (k >> 2) * 16384 + (k & 3) * 32), mndesc(va + k * 2048, 16384),
+                          id_o, k > 0 ? 1u : 0u);
+          ptx::mma_commit(&o_full[s]);
+          ptx::mma_commit(&kv_empty[s]);
+          ptx::mma_commit(&p_empty[s]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------- softmax warps: two per row (64 columns each)
+    // Both warps of a pair read the whole row of S for its maximum (the same
+    // values in the same order, so the same maximum), then each computes P
+    // and folds O for its half of the columns, with a partial row sum.
+    const int quad = warp & 3, half = (warp - 2) >> 2;
+    const int row = quad * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    const int qi = qb * 128 + row;  // query position in the sequence
+    const float sl2 = a.scale_log2;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) o[i] = 0.f;
+    float l = 0.f, m_o = -INFINITY, m_pend = -INFINITY;
+    auto fold_o = [&](int jo, float mj) -> bool {
+      const int s = jo & 1;
+      const uint32_t ph = (jo >> 1) & 1;
+      if (!ATTN_WAIT(&o_full[s], ph)) return false;
+      ptx::tc_fence_after();
+      const float alpha = exp2f(m_o - mj);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tl + 256 + s * 128 + half * 64 + c * 32, v);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha, __uint_as_float(v[i]));
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&o_free[s]);
+      m_o = mj;
+      return true;
+    };
+    for (int j = 0; j < nkb; ++j) {
+      const int s = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      if (!ATTN_WAIT(&s_full[s], ph)) { ok = false; break; }
+      ptx::tc_fence_after();
+      const int key0 = j * 128;
+      const bool edge = key0 + 127 > qi || key0 + 128 > S;  // some key of the block is masked for this row
+      // pass 1: the row's maximum over the block
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tl + s * 128 + c * 32, v);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int key = key0 + c * 32 + i;
+          float x = __uint_as_float(v[i]) * sl2;
+          if (edge && (key > qi || key >= S)) x = -INFINITY;
+          mx = fmaxf(mx, x);
+        }
+      }
+      const float m_new = fmaxf(m, mx);
+      // pass 2 (this warp's 64 keys): p = 2^(x - m_new) (0 where masked),
+      // partial row sum, P in fp16
+      if (!ATTN_WAIT(&p_empty[s], ph ^ 1)) { ok = false; break; }
+      uint8_t* P = sm + F_P + s * 32768 + half * 16384;  // keys 0..63 | 64..127
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tl + s * 128 + half * 64 + c * 32, v);
+        ptx::tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int key = key0 + half * 64 + c * 32 + i;
+          float x0 = __uint_as_float(v[i]) * sl2, x1 = __uint_as_float(v[i + 1]) * sl2;
+          if (edge) {
+            if (key > qi || key >= S) x0 = -INFINITY;
+            if (key + 1 > qi || key + 1 >= S) x1 = -INFINITY;
+          }
+          const float p0 = exp2f(x0 - m_new), p1 = exp2f(x1 - m_new);
+          sum += p0 + p1;
+          pk[i >> 1] = pack_h2(p0, p1);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          st_unit(P, row, c * 4 + u, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+      }
+      ptx::tc_fence_before();
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(&s_free[s]);
+        ptx::mbar_arrive(&p_full[s]);
+      }
+      l = l * exp2f(m - m_new) + sum;
+      m = m_new;
+      if (j >= 1 && !fold_o(j - 1, m_pend)) { ok = false; break; }
+      m_pend = m_new;
+    }
+    if (ok) ok = fold_o(nkb - 1, m_pend);
+    lsum[half * 128 + row] = l;
+  }
+  // the two partial row sums meet here; then each softmax thread stores its
+  // 64 output columns (and half 0 the log-sum-exp)
+  __syncthreads();
+  if (warp >= 2 && ok) {
+    const int quad = warp & 3, half = (warp - 2) >> 2;
+    const int row = quad * 32 + lane;
+    const int qi = qb * 128 + row;
+    if (qi < S) {
+      const float l = lsum[row] + lsum[128 + row];
+      const float inv = 1.f / l;
+      const size_t off = (size_t)(row0 + qi) * (a.Hq * HD) + h * HD + half * 64;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float f[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = o[u * 8 + i] * inv;
+        reinterpret_cast<uint4*>(a.out + off)[u] =
+            make_uint4(pack_b2(f[0], f[1]), pack_b2(f[2], f[3]), pack_b2(f[4], f[5]), pack_b2(f[6], f[7]));
+        if (a.out16)
+          reinterpret_cast<uint4*>(a.out16 + off)[u] =
+              make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
+        if (a.out32) {
+          reinterpret_cast<float4*>(a.out32 + off)[2 * u] = make_float4(f[0], f[1], f[2], f[3]);
+          reinterpret_cast<float4*>(a.out32 + off)[2 * u + 1] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+      }
+      if (half == 0) a.lse[(size_t)h * a.T + row0 + qi] = m + log2f(l);
+    }
+  }
+  attn_teardown(abort_flag, warp, tmem);
+}
+
+// ================================================ backward pass 1: dK and dV
+// Shared memory: K and V of the block (32 KB each, K-major, 128 rows), NS
+// stages of (Q tile | dO tile) (64 rows: 16 KB each) with their L and D
+// values, 2 P^T and 2 dS^T buffers ([128 keys, 64 queries] fp16, 16 KB each).
+constexpr int B1_NS = 3;
+constexpr int B1_K = 0, B1_V = 32768, B1_ST = 65536;
+constexpr int B1_STAGE = 32768;
+constexpr int B1_P = B1_ST + B1_NS * B1_STAGE;  // 2 x 16 KB
+constexpr int B1_DS = B1_P + 2 * 16384;         // 2 x 16 KB
+constexpr int B1_LD = B1_DS + 2 * 16384;        // NS x (64 L + 64 D) floats
+constexpr int B1_BAR = B1_LD + B1_NS * 512;
+constexpr int B1_SMEM = B1_BAR + 256 + 1024;
+
+__global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tm128,
+                                                           const __grid_constant__ CUtensorMap tm64,
+                                                           const __grid_constant__ CUtensorMap tmdo64,
+                                                           const AttnArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + B1_BAR);
+  uint64_t* kv_full = bars;               // 1
+  uint64_t* full = bars + 1;              // [NS]
+  uint64_t* empty = full + B1_NS;         // [NS]
+  uint64_t* st_full = empty + B1_NS;      // [2]
+  uint64_t* st_free = st_full + 2;        // [2]
+  uint64_t* p_full = st_free + 2;         // [2]
+  uint64_t* p_empty = p_full + 2;         // [2]
+  uint64_t* acc_full = p_empty + 2;       // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int S = a.S;
+  const int kb = blockIdx.x;  // key block: the first ones have the most query tiles
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int grp = a.Hq / a.Hkv;
+  const int row0 = b * S;
+  const int kcol = (a.Hq + g) * HD, vcol = (a.Hq + a.Hkv + g) * HD;
+  const int qt0 = 2 * kb;                 // first 64-query tile at or after the block
+  const int nqt = (S + 63) / 64;
+  const int per_head = nqt - qt0;
   const int n_it = per_head * grp;
-  auto issue = [&](int it, int buf) {
-    const int hh = it / per_head, qb2 = qb_first + it % per_head;
-    const int h = kvh * grp + hh;
-    load_tile(Qs + buf * 32 * LDS, qkv, ld, h * HD, row0 + qb2 * 32, qb2 * 32, S, 32, tid, 128);
-    load_tile(Os + buf * 32 * LDS, dout, ldo, h * HD, row0 + qb2 * 32, qb2 * 32, S, 32, tid, 128);
-    if (tid < 32) {
-      const int q = qb2 * 32 + tid;
-      Ls[buf * 32 + tid] = (q < S) ? lse[(size_t)h * T + row0 + q] : 0.f;
-      Ds[buf * 32 + tid] = (q < S) ? Dd[(size_t)h * T + row0 + q] : 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(kv_full, 1);
+    for (int i = 0; i < B1_NS; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], 1);
     }
-  };
-  float dk[16][4], dv[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    dk[i][0] = dk[i][1] = dk[i][2] = dk[i][3] = 0.f;
-    dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&st_full[i], 1);
+      ptx::mbar_init(&st_free[i], 4);
+      ptx::mbar_init(&p_full[i], 4);
+      ptx::mbar_init(&p_empty[i], 1);
+    }
+    ptx::mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tm128);
+    ptx::prefetch_tmap(&tm64);
+    ptx::prefetch_tmap(&tmdo64);
   }
-  const int key0 = kb * 64 + warp * 16 + g4, key1 = key0 + 8;
-  if (n_it > 0) issue(0, 0);
-  cp_commit();
-  for (int it = 0; it < n_it; ++it) {
-    const int buf = it & 1;
-    if (it + 1 < n_it) {
-      __syncthreads();  // everyone done with buffer buf^1 (iteration it-1)
-      issue(it + 1, buf ^ 1);
-      cp_commit();
-      cp_wait<1>();
-    } else {
-      cp_wait<0>();
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  // columns: S^T[0] 0, S^T[1] 64, dP^T[0] 128, dP^T[1] 192, dV 256, dK 384
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------- TMA producer (whole warp)
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx(kv_full, 65536);
+      const int r = row0 + kb * 128;
+      ptx::tma_load_2d(sm + B1_K, &tm128, kv_full, kcol, r);
+      ptx::tma_load_2d(sm + B1_K + 16384, &tm128, kv_full, kcol + 64, r);
+      ptx::tma_load_2d(sm + B1_V, &tm128, kv_full, vcol, r);
+      ptx::tma_load_2d(sm + B1_V + 16384, &tm128, kv_full, vcol + 64, r);
     }
-    __syncthreads();
-    const int qb2 = qb_first + it % per_head;
-    const uint16_t* Qb = Qs + buf * 32 * LDS;
-    const uint16_t* Ob = Os + buf * 32 * LDS;
-    const float* Lb = Ls + buf * 32;
-    const float* Db = Ds + buf * 32;
-    // S^T = K Q^T and dP^T = V dO^T  (16 keys x 32 queries)
-    float st[4][4], dpt[4][4];
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % B1_NS;
+      const uint32_t ph = (it / B1_NS) & 1;
+      int okw = 1;
+      if (lane == 0) okw = ATTN_WAIT(&empty[s], ph ^ 1) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+      const int hh = it / per_head, qt = qt0 + it % per_head;
+      const int h = g * grp + hh;
+      const int q0 = qt * 64;
+      // this tile's L and D (the softmax warps read them after the stage's full barrier)
+      float* LD = reinterpret_cast<float*>(sm + B1_LD + s * 512);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      st[i][0] = st[i][1] = st[i][2] = st[i][3] = 0.f;
-      dpt[i][0] = dpt[i][1] = dpt[i][2] = dpt[i][3] = 0.f;
-    }
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      uint32_t ka[4], va[4];
-      ldsm_x4(ka, a_addr(Ks, warp * 16, kk * 16, lane));
-      ldsm_x4(va, a_addr(Vs, warp * 16, kk * 16, lane));
-#pragma unroll
-      for (int nt2 = 0; nt2 < 2; ++nt2) {
-        uint32_t bq[4], bo[4];
-        ldsm_x4(bq, bn_addr(Qb, nt2 * 16, kk * 16, lane));
-        ldsm_x4(bo, bn_addr(Ob, nt2 * 16, kk * 16, lane));
-        mma16816(st[2 * nt2], ka, bq[0], bq[1]);
-        mma16816(st[2 * nt2 + 1], ka, bq[2], bq[3]);
-        mma16816(dpt[2 * nt2], va, bo[0], bo[1]);
-        mma16816(dpt[2 * nt2 + 1], va, bo[2], bo[3]);
+      for (int i = lane; i < 64; i += 32) {
+        const bool in = q0 + i < S;
+        LD[i] = in ? a.L[(size_t)h * a.T + row0 + q0 + i] : 0.f;
+        LD[64 + i] = in ? a.D[(size_t)h * a.T + row0 + q0 + i] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        uint8_t* st = sm + B1_ST + s * B1_STAGE;
+        ptx::mbar_arrive_expect_tx(&full[s], 32768);
+        ptx::tma_load_2d(st, &tm64, &full[s], h * HD, row0 + q0);            // Q
+        ptx::tma_load_2d(st + 8192, &tm64, &full[s], h * HD + 64, row0 + q0);
+        ptx::tma_load_2d(st + 16384, &tmdo64, &full[s], h * HD, row0 + q0);  // dO
+        ptx::tma_load_2d(st + 24576, &tmdo64, &full[s], h * HD + 64, row0 + q0);
       }
     }
-    uint32_t pa[2][4], da[2][4];
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_st = ptx::idesc_fmt(128, 64, 0, 0, 0u);    // S^T, dP^T: [128 keys, 64 queries]
+      constexpr uint32_t id_acc = ptx::idesc_fmt(128, 128, 0, 1, 0u);  // dV, dK: B (dO, Q) MN-major
+      const uint32_t ka = ptx::smem_u32(sm + B1_K), va = ptx::smem_u32(sm + B1_V);
+      bool ok = ATTN_WAIT(kv_full, 0);
+      for (int jj = 0; ok && jj <= n_it; ++jj) {
+        if (jj < n_it) {
+          const int s = jj % B1_NS, bb = jj & 1;
+          const uint32_t ph = (jj / B1_NS) & 1, pb = (jj >> 1) & 1;
+          if (!ATTN_WAIT(&full[s], ph) || !ATTN_WAIT(&st_free[bb], pb ^ 1)) break;
+          ptx::tc_fence_after();
+          const uint32_t qa = ptx::smem_u32(sm + B1_ST + s * B1_STAGE), oa = qa + 16384;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      float p[4], ds[4];
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+            ptx::mma_bf16(tmem + bb * 64, kdesc(ka + (k >> 2) * 16384 + (k & 3) * 32), kdesc(qa + off), id_st,
+                          k > 0 ? 1u : 0u);
+          }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int ql = nt * 8 + 2 * t4 + (e & 1);
-        const int q = qb2 * 32 + ql;
-        const int key = (e < 2) ? key0 : key1;
-        const bool ok = (q >= key) && (q < S) && (key < S);
-        p[e] = ok ? exp2f(st[nt][e] * scale_log2 - Lb[ql]) : 0.f;
-        ds[e] = p[e] * (dpt[nt][e] - Db[ql]);
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+            ptx::mma_bf16(tmem + 128 + bb * 64, kdesc(va + (k >> 2) * 16384 + (k & 3) * 32), kdesc(oa + off), id_st,
+                          k > 0 ? 1u : 0u);
+          }
+          ptx::mma_commit(&st_full[bb]);
+        }
+        if (jj >= 1) {  // dV += P^T dO, dK += dS^T Q for iteration it = jj - 1
+          const int it = jj - 1, s = it % B1_NS, bb = it & 1;
+          const uint32_t pb = (it >> 1) & 1;
+          if (!ATTN_WAIT(&p_full[bb], pb)) break;
+          ptx::tc_fence_after();
+          const uint32_t qa = ptx::smem_u32(sm + B1_ST + s * B1_STAGE), oa = qa + 16384;
+          const uint32_t pa = ptx::smem_u32(sm + B1_P + bb * 16384), da = ptx::smem_u32(sm + B1_DS + bb * 16384);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            ptx::mma_bf16(tmem + 256, kdesc(pa + k * 32), mndesc(oa + k * 2048, 8192), id_acc,
+                          (it > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            ptx::mma_bf16(tmem + 384, kdesc(da + k * 32), mndesc(qa + k * 2048, 8192), id_acc,
+                          (it > 0 || k > 0) ? 1u : 0u);
+          ptx::mma_commit(&p_empty[bb]);
+          ptx::mma_commit(&empty[s]);
+        }
       }
-      pa[nt >> 1][(nt & 1) * 2 + 0] = packh(p[0], p[1]);
-      pa[nt >> 1][(nt & 1) * 2 + 1] = packh(p[2], p[3]);
-      da[nt >> 1][(nt & 1) * 2 + 0] = packh(ds[0], ds[1]);
-      da[nt >> 1][(nt & 1) * 2 + 1] = packh(ds[2], ds[3]);
+      if (ok && n_it > 0) ptx::mma_commit(acc_full);
     }
-    // dV += P^T dO ; dK += dS^T Q
+  } else {
+    // ------------------------------------ elementwise warps (one key row each)
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    const int key = kb * 128 + row;
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % B1_NS, bb = it & 1;
+      const uint32_t pb = (it >> 1) & 1;
+      const int q0 = (qt0 + it % per_head) * 64;
+      // the stage's full barrier also publishes the L and D values the
+      // producer warp stored next to the tiles (it cannot move on to the
+      // stage's next use before these warps release this iteration)
+      if (!ATTN_WAIT(&full[s], (it / B1_NS) & 1) || !ATTN_WAIT(&st_full[bb], pb)) { ok = false; break; }
+      ptx::tc_fence_after();
+      const float* LD = reinterpret_cast<const float*>(sm + B1_LD + s * 512);
+      if (!ATTN_WAIT(&p_empty[bb], pb ^ 1)) { ok = false; break; }
+      uint8_t* P = sm + B1_P + bb * 16384;
+      uint8_t* DS = sm + B1_DS + bb * 16384;
+      const bool edge = q0 < key || q0 + 64 > S || key >= S;  // some query of the tile is masked for this key
 #pragma unroll
-    for (int kq = 0; kq < 2; ++kq) {
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[32], dv[32];
+        ptx::tmem_ld32(tl + bb * 64 + c * 32, sv);
+        ptx::tmem_ld32(tl + 128 + bb * 64 + c * 32, dv);
+        ptx::tmem_ld_wait();
+        uint32_t pk[16], dk[16];
 #pragma unroll
-      for (int dt2 = 0; dt2 < 8; ++dt2) {
-        uint32_t bo[4], bq[4];
-        ldsm_x4_t(bo, bk_addr(Ob, kq * 16, dt2 * 16, lane));
-        ldsm_x4_t(bq, bk_addr(Qb, kq * 16, dt2 * 16, lane));
-        mma16816(dv[2 * dt2], pa[kq], bo[0], bo[1]);
-        mma16816(dv[2 * dt2 + 1], pa[kq], bo[2], bo[3]);
-        mma16816(dk[2 * dt2], da[kq], bq[0], bq[1]);
-        mma16816(dk[2 * dt2 + 1], da[kq], bq[2], bq[3]);
+        for (int i = 0; i < 32; i += 2) {
+          float p[2], d[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int qi = c * 32 + i + e;
+            const int q = q0 + qi;
+            float x = __uint_as_float(sv[i + e]) * sl2 - LD[qi];
+            if (edge && (q < key || q >= S || key >= S)) x = -INFINITY;
+            p[e] = exp2f(x);
+            d[e] = p[e] * (__uint_as_float(dv[i + e]) - LD[64 + qi]);
+          }
+          pk[i >> 1] = pack_h2(p[0], p[1]);
+          dk[i >> 1] = pack_h2(d[0], d[1]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          st_unit(P, row, c * 4 + u, pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          st_unit(DS, row, c * 4 + u, dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(&st_free[bb]);
+        ptx::mbar_arrive(&p_full[bb]);
+      }
+    }
+    // epilogue: dK (x scale, RoPE back) and dV from tensor memory, unscaled
+    if (ok && n_it > 0 && ATTN_WAIT(acc_full, 0)) {
+      ptx::tc_fence_after();
+      const float unscale = a.amax ? 1.f / grad_scale_from_amax(__uint_as_float(*a.amax)) : 1.f;
+      const bool in = key < S;
+      const size_t r = (size_t)(row0 + key) * a.ld;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+        const uint32_t col0 = which ? 384 : 256;
+        const float mul = which ? a.scale * unscale : unscale;
+        const int dcol = which ? kcol : vcol;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {  // pairs (c*32 + i, c*32 + i + 64)
+          uint32_t v0[32], v1[32];
+          ptx::tmem_ld32(tl + col0 + c * 32, v0);
+          ptx::tmem_ld32(tl + col0 + 64 + c * 32, v1);
+          ptx::tmem_ld_wait();
+          float f0[32], f1[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            f0[i] = __uint_as_float(v0[i]) * mul;
+            f1[i] = __uint_as_float(v1[i]) * mul;
+          }
+          if (which && a.rcos && in) {
+            const float* cs = a.rcos + (size_t)key * 64 + c * 32;
+            const float* sn = a.rsin + (size_t)key * 64 + c * 32;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rope_back(f0[i], f1[i], __ldg(cs + i), __ldg(sn + i));
+          }
+          if (in) {
+            uint16_t* o0 = a.dqkv + r + dcol + c * 32;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              reinterpret_cast<uint4*>(o0)[u] =
+                  make_uint4(pack_b2(f0[8 * u], f0[8 * u + 1]), pack_b2(f0[8 * u + 2], f0[8 * u + 3]),
+                             pack_b2(f0[8 * u + 4], f0[8 * u + 5]), pack_b2(f0[8 * u + 6], f0[8 * u + 7]));
+              reinterpret_cast<uint4*>(o0 + 64)[u] =
+                  make_uint4(pack_b2(f1[8 * u], f1[8 * u + 1]), pack_b2(f1[8 * u + 2], f1[8 * u + 3]),
+                             pack_b2(f1[8 * u + 4], f1[8 * u + 5]), pack_b2(f1[8 * u + 6], f1[8 * u + 7]));
+            }
+            if (a.dqkv32) {
+              float* p0 = a.dqkv32 + r + dcol + c * 32;
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                reinterpret_cast<float4*>(p0)[u] = make_float4(f0[4 * u], f0[4 * u + 1], f0[4 * u + 2], f0[4 * u + 3]);
+                reinterpret_cast<float4*>(p0 + 64)[u] =
+                    make_float4(f1[4 * u], f1[4 * u + 1], f1[4 * u + 2], f1[4 * u + 3]);
+              }
+            }
+          }
+        }
       }
     }
   }
-  // dO carried the power-of-two gradient scale: undo it (exact)
-  const float unscale = amax ? 1.f / grad_scale_from_amax(__uint_as_float(*amax)) : 1.f;
-  if (key0 < S) {
-    const size_t r = (size_t)(row0 + key0) * ld;
-    store_row_rot(dqkv + r + kcol, dk, 0, scale * unscale, rcos ? rcos + (size_t)key0 * 64 : nullptr,
-                  rsin ? rsin + (size_t)key0 * 64 : nullptr, t4, dqkv32 ? dqkv32 + r + kcol : nullptr);
-    store_row_rot(dqkv + r + vcol, dv, 0, unscale, nullptr, nullptr, t4, dqkv32 ? dqkv32 + r + vcol : nullptr);
-  }
-  if (key1 < S) {
-    const size_t r = (size_t)(row0 + key1) * ld;
-    store_row_rot(dqkv + r + kcol, dk, 2, scale * unscale, rcos ? rcos + (size_t)key1 * 64 : nullptr,
-                  rsin ? rsin + (size_t)key1 * 64 : nullptr, t4, dqkv32 ? dqkv32 + r + kcol : nullptr);
-    store_row_rot(dqkv + r + vcol, dv, 2, unscale, nullptr, nullptr, t4, dqkv32 ? dqkv32 + r + vcol : nullptr);
-  }
+  attn_teardown(abort_flag, warp, tmem);
 }
 
-// ------------------------------------------------------- backward pass 2: dQ
-__global__ void __launch_bounds__(128) attn_bwd_dq_kernel(const uint16_t* __restrict__ qkv, int ld, int S, int Hq,
-                                                           int Hkv, const uint16_t* __restrict__ dout,
-                                                           const float* __restrict__ lse,
-                                                           const float* __restrict__ Dd,
-                                                           uint16_t* __restrict__ dqkv, float scale_log2,
-                                                           float scale, const float* __restrict__ rcos,
-                                                           const float* __restrict__ rsin,
-                                                           const unsigned int* __restrict__ amax,
-                                                           float* __restrict__ dqkv32) {
-  extern __shared__ __align__(16) uint16_t sm[];
-  uint16_t* Qs = sm;
-  uint16_t* Os = Qs + 64 * LDS;
-  uint16_t* Ks = Os + 64 * LDS;  // 2 buffers
-  uint16_t* Vs = Ks + 2 * 64 * LDS;
-  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g4 = lane >> 2, t4 = lane & 3;
-  const int T = gridDim.z * S;
-  const int grp = Hq / Hkv, kvh = h / grp;
-  const int kcol = (Hq + kvh) * HD, vcol = (Hq + Hkv + kvh) * HD;
+// ======================================================= backward pass 2: dQ
+// Shared memory: Q and dO of the tile (32 KB each, 128 rows), NS stages of
+// (K block | V block) (64 rows: 16 KB each), 2 dS buffers ([128 queries, 64
+// keys] fp16, 16 KB each).
+constexpr int B2_NS = 3;
+constexpr int B2_Q = 0, B2_O = 32768, B2_ST = 65536;
+constexpr int B2_STAGE = 32768;
+constexpr int B2_DS = B2_ST + B2_NS * B2_STAGE;
+constexpr int B2_BAR = B2_DS + 2 * 16384;
+constexpr int B2_SMEM = B2_BAR + 256 + 1024;
+
+__global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tm128,
+                                                         const __grid_constant__ CUtensorMap tm64,
+                                                         const __grid_constant__ CUtensorMap tmdo128,
+                                                         const AttnArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + B2_BAR);
+  uint64_t* qo_full = bars;               // 1
+  uint64_t* full = bars + 1;              // [NS]
+  uint64_t* empty = full + B2_NS;         // [NS]
+  uint64_t* st_full = empty + B2_NS;      // [2]
+  uint64_t* st_free = st_full + 2;        // [2]
+  uint64_t* ds_full = st_free + 2;        // [2]
+  uint64_t* ds_empty = ds_full + 2;       // [2]
+  uint64_t* acc_full = ds_empty + 2;      // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int S = a.S;
+  const int nqt = (S + 127) / 128;
+  const int qb = nqt - 1 - (int)blockIdx.x;  // the longest rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (a.Hq / a.Hkv);
   const int row0 = b * S;
-  const int ldo = Hq * HD;
-  load_tile(Qs, qkv, ld, h * HD, row0 + qb * 64, qb * 64, S, 64, tid, 128);
-  load_tile(Os, dout, ldo, h * HD, row0 + qb * 64, qb * 64, S, 64, tid, 128);
-  load_tile(Ks, qkv, ld, kcol, row0, 0, S, 64, tid, 128);
-  load_tile(Vs, qkv, ld, vcol, row0, 0, S, 64, tid, 128);
-  cp_commit();
-  const int qr0 = qb * 64 + warp * 16 + g4, qr1 = qr0 + 8;
-  const float L0 = (qr0 < S) ? lse[(size_t)h * T + row0 + qr0] : 0.f;
-  const float L1 = (qr1 < S) ? lse[(size_t)h * T + row0 + qr1] : 0.f;
-  const float D0 = (qr0 < S) ? Dd[(size_t)h * T + row0 + qr0] : 0.f;
-  const float D1 = (qr1 < S) ? Dd[(size_t)h * T + row0 + qr1] : 0.f;
-  float dq[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
-  const int nkb = qb + 1;
-  for (int j = 0; j < nkb; ++j) {
-    if (j + 1 < nkb) {
-      load_tile(Ks + ((j + 1) & 1) * 64 * LDS, qkv, ld, kcol, row0 + (j + 1) * 64, (j + 1) * 64, S, 64, tid, 128);
-      load_tile(Vs + ((j + 1) & 1) * 64 * LDS, qkv, ld, vcol, row0 + (j + 1) * 64, (j + 1) * 64, S, 64, tid, 128);
-      cp_commit();
-      cp_wait<1>();
-    } else {
-      cp_wait<0>();
+  const int kcol = (a.Hq + g) * HD, vcol = (a.Hq + a.Hkv + g) * HD;
+  const int n_it = min(2 * qb + 2, (S + 63) / 64);  // 64-key blocks up to the diagonal and the sequence end
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(qo_full, 1);
+    for (int i = 0; i < B2_NS; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], 1);
     }
-    __syncthreads();
-    const uint16_t* Kb = Ks + (j & 1) * 64 * LDS;
-    const uint16_t* Vb = Vs + (j & 1) * 64 * LDS;
-    float s[8][4], dp[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-      dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&st_full[i], 1);
+      ptx::mbar_init(&st_free[i], 4);
+      ptx::mbar_init(&ds_full[i], 4);
+      ptx::mbar_init(&ds_empty[i], 1);
     }
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      uint32_t qa[4], oa[4];
-      ldsm_x4(qa, a_addr(Qs, warp * 16, kk * 16, lane));
-      ldsm_x4(oa, a_addr(Os, warp * 16, kk * 16, lane));
-#pragma unroll
-      for (int nt2 = 0; nt2 < 4; ++nt2) {
-        uint32_t bk[4], bv[4];
-        ldsm_x4(bk, bn_addr(Kb, nt2 * 16, kk * 16, lane));
-        ldsm_x4(bv, bn_addr(Vb, nt2 * 16, kk * 16, lane));
-        mma16816(s[2 * nt2], qa, bk[0], bk[1]);
-        mma16816(s[2 * nt2 + 1], qa, bk[2], bk[3]);
-        mma16816(dp[2 * nt2], oa, bv[0], bv[1]);
-        mma16816(dp[2 * nt2 + 1], oa, bv[2], bv[3]);
+    ptx::mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tm128);
+    ptx::prefetch_tmap(&tm64);
+    ptx::prefetch_tmap(&tmdo128);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  // columns: S[0] 0, S[1] 64, dP[0] 128, dP[1] 192, dQ 256
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int qrow = row0 + qb * 128;
+      ptx::mbar_arrive_expect_tx(qo_full, 65536);
+      ptx::tma_load_2d(sm + B2_Q, &tm128, qo_full, h * HD, qrow);
+      ptx::tma_load_2d(sm + B2_Q + 16384, &tm128, qo_full, h * HD + 64, qrow);
+      ptx::tma_load_2d(sm + B2_O, &tmdo128, qo_full, h * HD, qrow);
+      ptx::tma_load_2d(sm + B2_O + 16384, &tmdo128, qo_full, h * HD + 64, qrow);
+      for (int j = 0; j < n_it; ++j) {
+        const int s = j % B2_NS;
+        const uint32_t ph = (j / B2_NS) & 1;
+        if (!ATTN_WAIT(&empty[s], ph ^ 1)) break;
+        uint8_t* st = sm + B2_ST + s * B2_STAGE;
+        const int r = row0 + j * 64;
+        ptx::mbar_arrive_expect_tx(&full[s], 32768);
+        ptx::tma_load_2d(st, &tm64, &full[s], kcol, r);
+        ptx::tma_load_2d(st + 8192, &tm64, &full[s], kcol + 64, r);
+        ptx::tma_load_2d(st + 16384, &tm64, &full[s], vcol, r);
+        ptx::tma_load_2d(st + 24576, &tm64, &full[s], vcol + 64, r);
       }
     }
-    uint32_t da[4][4];
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = ptx::idesc_fmt(128, 64, 0, 0, 0u);    // S, dP: [128 queries, 64 keys]
+      constexpr uint32_t id_q = ptx::idesc_fmt(128, 128, 0, 1, 0u);   // dQ: B (K) MN-major
+      const uint32_t qa = ptx::smem_u32(sm + B2_Q), oa = ptx::smem_u32(sm + B2_O);
+      bool ok = ATTN_WAIT(qo_full, 0);
+      for (int jj = 0; ok && jj <= n_it; ++jj) {
+        if (jj < n_it) {
+          const int s = jj % B2_NS, bb = jj & 1;
+          const uint32_t ph = (jj / B2_NS) & 1, pb = (jj >> 1) & 1;
+          if (!ATTN_WAIT(&full[s], ph) || !ATTN_WAIT(&st_free[bb], pb ^ 1)) break;
+          ptx::tc_fence_after();
+          const uint32_t ka = ptx::smem_u32(sm + B2_ST + s * B2_STAGE), va = ka + 16384;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      float ds[4];
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+            ptx::mma_bf16(tmem + bb * 64, kdesc(qa + (k >> 2) * 16384 + (k & 3) * 32), kdesc(ka + off), id_s,
+                          k > 0 ? 1u : 0u);
+          }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = j * 64 + nt * 8 + 2 * t4 + (e & 1);
-        const int qr = (e < 2) ? qr0 : qr1;
-        const bool ok = (key <= qr) && (key < S) && (qr < S);
-        const float p = ok ? exp2f(s[nt][e] * scale_log2 - ((e < 2) ? L0 : L1)) : 0.f;
-        ds[e] = p * (dp[nt][e] - ((e < 2) ? D0 : D1));
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t off = (k >> 2) * 8192 + (k & 3) * 32;
+            ptx::mma_bf16(tmem + 128 + bb * 64, kdesc(oa + (k >> 2) * 16384 + (k & 3) * 32), kdesc(va + off), id_s,
+                          k > 0 ? 1u : 0u);
+          }
+          ptx::mma_commit(&st_full[bb]);
+        }
+        if (jj >= 1) {  // dQ += dS_j K_j, j = jj - 1
+          const int j = jj - 1, s = j % B2_NS, bb = j & 1;
+          const uint32_t pb = (j >> 1) & 1;
+          if (!ATTN_WAIT(&ds_full[bb], pb)) break;
+          ptx::tc_fence_after();
+          const uint32_t ka = ptx::smem_u32(sm + B2_ST + s * B2_STAGE);
+          const uint32_t da = ptx::smem_u32(sm + B2_DS + bb * 16384);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            ptx::mma_bf16(tmem + 256, kdesc(da + k * 32), mndesc(ka + k * 2048, 8192), id_q,
+                          (j > 0 || k > 0) ? 1u : 0u);
+          ptx::mma_commit(&ds_empty[bb]);
+          ptx::mma_commit(&empty[s]);
+        }
       }
-      da[nt >> 1][(nt & 1) * 2 + 0] = packh(ds[0], ds[1]);
-      da[nt >> 1][(nt & 1) * 2 + 1] = packh(ds[2], ds[3]);
+      if (ok) ptx::mma_commit(acc_full);
     }
+  } else {
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    const int qi = qb * 128 + row;
+    const bool qin = qi < S;
+    const float Lr = qin ? a.L[(size_t)h * a.T + row0 + qi] : 0.f;
+    const float Dr = qin ? a.D[(size_t)h * a.T + row0 + qi] : 0.f;
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    for (int j = 0; j < n_it; ++j) {
+      const int bb = j & 1;
+      const uint32_t pb = (j >> 1) & 1;
+      const int key0 = j * 64;
+      if (!ATTN_WAIT(&st_full[bb], pb)) { ok = false; break; }
+      ptx::tc_fence_after();
+      if (!ATTN_WAIT(&ds_empty[bb], pb ^ 1)) { ok = false; break; }
+      uint8_t* DS = sm + B2_DS + bb * 16384;
+      const bool edge = key0 + 63 > qi || key0 + 64 > S || !qin;
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[32], dv[32];
+        ptx::tmem_ld32(tl + bb * 64 + c * 32, sv);
+        ptx::tmem_ld32(tl + 128 + bb * 64 + c * 32, dv);
+        ptx::tmem_ld_wait();
+        uint32_t dk[16];
 #pragma unroll
-      for (int dt2 = 0; dt2 < 8; ++dt2) {
-        uint32_t bk[4];
-        ldsm_x4_t(bk, bk_addr(Kb, kk * 16, dt2 * 16, lane));
-        mma16816(dq[2 * dt2], da[kk], bk[0], bk[1]);
-        mma16816(dq[2 * dt2 + 1], da[kk], bk[2], bk[3]);
+        for (int i = 0; i < 32; i += 2) {
+          float d[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int key = key0 + c * 32 + i + e;
+            float x = __uint_as_float(sv[i + e]) * sl2 - Lr;
+            if (edge && (key > qi || key >= S || !qin)) x = -INFINITY;
+            const float p = exp2f(x);
+            d[e] = p * (__uint_as_float(dv[i + e]) - Dr);
+          }
+          dk[i >> 1] = pack_h2(d[0], d[1]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) st_unit(DS, row, c * 4 + u, dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+      }
+      ptx::tc_fence_before();
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(&st_free[bb]);
+        ptx::mbar_arrive(&ds_full[bb]);
       }
     }
-    __syncthreads();
+    if (ok && ATTN_WAIT(acc_full, 0)) {
+      ptx::tc_fence_after();
+      const float unscale = a.amax ? 1.f / grad_scale_from_amax(__uint_as_float(*a.amax)) : 1.f;
+      const float mul = a.scale * unscale;
+      const size_t r = (size_t)(row0 + qi) * a.ld + h * HD;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v0[32], v1[32];
+        ptx::tmem_ld32(tl + 256 + c * 32, v0);
+        ptx::tmem_ld32(tl + 256 + 64 + c * 32, v1);
+        ptx::tmem_ld_wait();
+        float f0[32], f1[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          f0[i] = __uint_as_float(v0[i]) * mul;
+          f1[i] = __uint_as_float(v1[i]) * mul;
+        }
+        if (qin) {
+          if (a.rcos) {
+            const float* cs = a.rcos + (size_t)qi * 64 + c * 32;
+            const float* sn = a.rsin + (size_t)qi * 64 + c * 32;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rope_back(f0[i], f1[i], __ldg(cs + i), __ldg(sn + i));
+          }
+          uint16_t* o0 = a.dqkv + r + c * 32;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            reinterpret_cast<uint4*>(o0)[u] =
+                make_uint4(pack_b2(f0[8 * u], f0[8 * u + 1]), pack_b2(f0[8 * u + 2], f0[8 * u + 3]),
+                           pack_b2(f0[8 * u + 4], f0[8 * u + 5]), pack_b2(f0[8 * u + 6], f0[8 * u + 7]));
+            reinterpret_cast<uint4*>(o0 + 64)[u] =
+                make_uint4(pack_b2(f1[8 * u], f1[8 * u + 1]), pack_b2(f1[8 * u + 2], f1[8 * u + 3]),
+                           pack_b2(f1[8 * u + 4], f1[8 * u + 5]), pack_b2(f1[8 * u + 6], f1[8 * u + 7]));
+          }
+          if (a.dqkv32) {
+            float* p0 = a.dqkv32 + r + c * 32;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              reinterpret_cast<float4*>(p0)[u] = make_float4(f0[4 * u], f0[4 * u + 1], f0[4 * u + 2], f0[4 * u + 3]);
+              reinterpret_cast<float4*>(p0 + 64)[u] = make_float4(f1[4 * u], f1[4 * u + 1], f1[4 * u + 2], f1[4 * u + 3]);
+            }
+          }
+        }
+      }
+    }
   }
-  const float unscale = amax ? 1.f / grad_scale_from_amax(__uint_as_float(*amax)) : 1.f;
-  if (qr0 < S) {
-    const size_t r = (size_t)(row0 + qr0) * ld + h * HD;
-    store_row_rot(dqkv + r, dq, 0, scale * unscale, rcos ? rcos + (size_t)qr0 * 64 : nullptr,
-                  rsin ? rsin + (size_t)qr0 * 64 : nullptr, t4, dqkv32 ? dqkv32 + r : nullptr);
-  }
-  if (qr1 < S) {
-    const size_t r = (size_t)(row0 + qr1) * ld + h * HD;
-    store_row_rot(dqkv + r, dq, 2, scale * unscale, rcos ? rcos + (size_t)qr1 * 64 : nullptr,
-                  rsin ? rsin + (size_t)qr1 * 64 : nullptr, t4, dqkv32 ? dqkv32 + r : nullptr);
-  }
+  attn_teardown(abort_flag, warp, tmem);
 }
 
-constexpr int FWD_SMEM = 5 * 64 * LDS * 2;
-constexpr int DKDV_SMEM = (2 * 64 + 4 * 32) * LDS * 2 + 4 * 32 * 4;
-constexpr int DQ_SMEM = 6 * 64 * LDS * 2;
+#undef ATTN_WAIT
+
+// 2-D fp16 tensor map over [rows, cols] (row stride ld elements), box of
+// 64 columns (128 bytes) x box_rows rows, 128-byte swizzle.
+soup_status fp16_map(CUtensorMap* m, const uint16_t* p, int64_t rows, int64_t cols, int64_t ld, uint32_t box_rows,
+                     const char* what) {
+  SOUP_CHECK(p && rows > 0 && cols > 0, SOUP_ERR_INVALID_ARG, "attention: %s is empty", what);
+  SOUP_CHECK(soup_aligned(p, 16) && (ld * 2) % 16 == 0, SOUP_ERR_ALIGN, "attention: %s base / row stride alignment",
+             what);
+  EncodeTiledFn enc = encode_tiled();
+  SOUP_CHECK(enc != nullptr, SOUP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const uint64_t gdim[2] = {(uint64_t)cols, (uint64_t)rows};
+  const uint64_t gstride[1] = {(uint64_t)(ld * 2)};
+  const uint32_t box[2] = {64, box_rows};
+  const uint32_t estr[2] = {1, 1};
+  const int r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(p), gdim, gstride, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  SOUP_CHECK(r == 0, SOUP_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with %d", what, r);
+  return SOUP_OK;
+}
 
 soup_status attn_init() {
   static bool init = false;
   if (!init) {
-    SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FWD_SMEM));
-    SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DKDV_SMEM));
-    SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DQ_SMEM));
+    SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM));
+    SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, B1_SMEM));
+    SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, B2_SMEM));
     init = true;
   }
+  return SOUP_OK;
+}
+
+soup_status attn_check(int ld, int Bsz, int S, int Hq, int Hkv) {
+  SOUP_CHECK(Hkv > 0 && Hq % Hkv == 0 && S > 0 && Bsz > 0, SOUP_ERR_SHAPE, "attention: bad heads/shape");
+  SOUP_CHECK(ld >= (Hq + 2 * Hkv) * HD && ld % 8 == 0, SOUP_ERR_SHAPE, "attention: row stride %d", ld);
+  SOUP_CHECK((int64_t)Bsz * S < (1LL << 31), SOUP_ERR_SHAPE, "attention: too many tokens");
   return SOUP_OK;
 }
 
@@ -523,14 +919,27 @@ soup_status attn_init() {
 
 soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, uint16_t* out, float* lse,
                           cudaStream_t st, uint16_t* out16, float* out32) {
-  SOUP_CHECK(Hq % Hkv == 0 && S > 0 && Bsz > 0, SOUP_ERR_SHAPE, "attention: bad heads/shape");
-  SOUP_CHECK(ld % 8 == 0 && soup_aligned(qkv, 16) && soup_aligned(out, 16), SOUP_ERR_ALIGN, "attention: alignment");
+  SOUP_TRY(attn_check(ld, Bsz, S, Hq, Hkv));
+  SOUP_CHECK(soup_aligned(qkv, 16) && soup_aligned(out, 16) && (!out16 || soup_aligned(out16, 16)) &&
+                 (!out32 || soup_aligned(out32, 16)) && lse,
+             SOUP_ERR_ALIGN, "attention: alignment");
   SOUP_TRY(attn_init());
-  const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
-  dim3 grid((S + 63) / 64, Hq, Bsz);
+  const int T = Bsz * S;
+  CUtensorMap tm;
+  SOUP_TRY(fp16_map(&tm, qkv, T, (Hq + 2 * Hkv) * HD, ld, 128, "q|k|v"));
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.T = T;
+  a.scale = 1.0f / sqrtf((float)HD);
+  a.scale_log2 = 1.4426950408889634f * a.scale;
+  a.out = out; a.lse = lse; a.out16 = out16; a.out32 = out32;
+  a.err = device_error_word();
+  SOUP_CHECK(a.err, SOUP_ERR_CUDA, "device error word unavailable");
+  a.wait_limit = 4000000000LL;
   const double fl = 4.0 * Bsz * Hq * (double)HD * ((double)S * (S + 1) / 2);
   profile_begin(st, GC_ATTN, fl, 0.0);
-  attn_fwd_kernel<<<grid, 128, FWD_SMEM, st>>>(qkv, ld, S, Hq, Hkv, out, lse, scale_log2, out16, out32);
+  dim3 grid((S + 127) / 128, Hq, Bsz);
+  attn_fwd_tc<<<grid, 320, F_SMEM, st>>>(tm, a);
   SOUP_LAUNCH_CHECK();
   profile_end(st);
   return SOUP_OK;
@@ -539,22 +948,63 @@ soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
 soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, const uint16_t* dout,
                           const float* lse, const float* D, uint16_t* dqkv, const float* rope_cos,
                           const float* rope_sin, const unsigned int* amax, cudaStream_t st, float* dqkv32) {
-  SOUP_CHECK(Hq % Hkv == 0 && S > 0 && Bsz > 0, SOUP_ERR_SHAPE, "attention: bad heads/shape");
+  SOUP_TRY(attn_check(ld, Bsz, S, Hq, Hkv));
+  SOUP_CHECK(soup_aligned(qkv, 16) && soup_aligned(dout, 16) && soup_aligned(dqkv, 16) &&
+                 (!dqkv32 || soup_aligned(dqkv32, 16)) && lse && D,
+             SOUP_ERR_ALIGN, "attention backward: alignment");
+  SOUP_CHECK(!rope_cos == !rope_sin, SOUP_ERR_INVALID_ARG, "attention backward: RoPE tables go together");
   SOUP_TRY(attn_init());
-  const float scale = 1.0f / sqrtf((float)HD);
-  const float scale_log2 = 1.4426950408889634f * scale;
+  const int T = Bsz * S;
+  CUtensorMap tm128, tm64, tmdo64, tmdo128;
+  SOUP_TRY(fp16_map(&tm128, qkv, T, (Hq + 2 * Hkv) * HD, ld, 128, "q|k|v"));
+  SOUP_TRY(fp16_map(&tm64, qkv, T, (Hq + 2 * Hkv) * HD, ld, 64, "q|k|v"));
+  SOUP_TRY(fp16_map(&tmdo64, dout, T, Hq * HD, Hq * HD, 64, "dO"));
+  SOUP_TRY(fp16_map(&tmdo128, dout, T, Hq * HD, Hq * HD, 128, "dO"));
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.T = T;
+  a.scale = 1.0f / sqrtf((float)HD);
+  a.scale_log2 = 1.4426950408889634f * a.scale;
+  a.L = lse; a.D = D; a.dqkv = dqkv; a.dqkv32 = dqkv32; a.ld = ld;
+  a.rcos = rope_cos; a.rsin = rope_sin; a.amax = amax;
+  a.err = device_error_word();
+  SOUP_CHECK(a.err, SOUP_ERR_CUDA, "device error word unavailable");
+  a.wait_limit = 4000000000LL;
   const double fl = 2.5 * 4.0 * Bsz * Hq * (double)HD * ((double)S * (S + 1) / 2);
   profile_begin(st, GC_ATTN, fl, 0.0);
-  dim3 g1((S + 63) / 64, Hkv, Bsz);
-  attn_bwd_dkdv_kernel<<<g1, 128, DKDV_SMEM, st>>>(qkv, ld, S, Hq, Hkv, dout, lse, D, dqkv, scale_log2, scale,
-                                                   rope_cos, rope_sin, amax, dqkv32);
+  dim3 g1((S + 127) / 128, Hkv, Bsz);
+  attn_bwd_dkdv_tc<<<g1, 192, B1_SMEM, st>>>(tm128, tm64, tmdo64, a);
   SOUP_LAUNCH_CHECK();
-  dim3 g2((S + 63) / 64, Hq, Bsz);
-  attn_bwd_dq_kernel<<<g2, 128, DQ_SMEM, st>>>(qkv, ld, S, Hq, Hkv, dout, lse, D, dqkv, scale_log2, scale,
-                                               rope_cos, rope_sin, amax, dqkv32);
+  dim3 g2((S + 127) / 128, Hq, Bsz);
+  attn_bwd_dq_tc<<<g2, 192, B2_SMEM, st>>>(tm128, tm64, tmdo128, a);
   SOUP_LAUNCH_CHECK();
   profile_end(st);
   return SOUP_OK;
 }
 
 }  // namespace soup
+
+using namespace soup;
+
+extern "C" soup_status soup_attention_fwd(const uint16_t* qkv, int64_t ld, int64_t batch, int64_t seq, int32_t n_q_heads,
+                                          int32_t n_kv_heads, uint16_t* out, uint16_t* out16, float* lse,
+                                          void* stream) {
+  SOUP_CHECK(qkv && out && lse, SOUP_ERR_INVALID_ARG, "soup_attention_fwd: null pointer");
+  SOUP_CHECK(batch > 0 && seq > 0 && batch * seq < (1LL << 31) && ld > 0 && ld < (1LL << 31), SOUP_ERR_SHAPE,
+             "soup_attention_fwd: bad shape");
+  return attention_fwd(qkv, (int)ld, (int)batch, (int)seq, n_q_heads, n_kv_heads, out, lse,
+                       static_cast<cudaStream_t>(stream), out16, nullptr);
+}
+
+extern "C" soup_status soup_attention_bwd(const uint16_t* qkv, int64_t ld, int64_t batch, int64_t seq,
+                                          int32_t n_q_heads, int32_t n_kv_heads, const uint16_t* out16,
+                                          const uint16_t* dout, const float* lse, float* D, uint16_t* dqkv,
+                                          float* dqkv32, void* stream) {
+  SOUP_CHECK(qkv && out16 && dout && lse && D && dqkv, SOUP_ERR_INVALID_ARG, "soup_attention_bwd: null pointer");
+  SOUP_CHECK(batch > 0 && seq > 0 && batch * seq < (1LL << 31) && ld > 0 && ld < (1LL << 31), SOUP_ERR_SHAPE,
+             "soup_attention_bwd: bad shape");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SOUP_TRY(attn_rowdot(dout, out16, (int)(batch * seq), n_q_heads, D, st));
+  return attention_bwd(qkv, (int)ld, (int)batch, (int)seq, n_q_heads, n_kv_heads, dout, lse, D, dqkv, nullptr,
+                       nullptr, nullptr, st, dqkv32);
+}

@@ -220,6 +220,11 @@ class StreamedLoRAModel:
         # When set to a dict, the backward pass stores dL/d(layer input) of
         # every layer in it (index l = input of layer l, n_layers = head output).
         self.capture_dh = None
+        # the shard build's temporaries (fp32 weights, the staging blob) are
+        # freed; hand their cached blocks back so that the device holds what
+        # the model uses, not what building it once needed
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
 
     # ------------------------------------------------------------ shard build
     def _build_blobs(self, weights):

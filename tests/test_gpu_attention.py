@@ -1,0 +1,114 @@
+"""The causal GQA attention kernels (tcgen05, accumulators in tensor memory)
+through the C ABI against the oracle's attention (fp64, plain softmax):
+output, log-sum-exp, dq, dk, dv within relative Frobenius 5e-3 and
+max|diff| 1e-2 max|ref|, on shapes that span several 128-row tiles with
+ragged tails, a one-token sequence, GQA groups of 1, 2 and 4, and several
+sequences per batch.  The inputs are fp16-exact, so both sides see the same
+numbers; the backward is deterministic (same bits twice)."""
+import numpy as np
+import pytest
+import torch
+
+import soup_synth as ss
+from oracle import layer as OL
+from tests.gpu_util import assert_close, host
+
+pytestmark = pytest.mark.gpu
+HD = 128
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from layer_streamed_qlora_b200 import _lib as lib
+    lib.lib()
+    yield lib
+    assert lib.device_error() == 0
+
+
+def f16_values(a):
+    return np.asarray(a, np.float32).astype(np.float16).astype(np.float64)
+
+
+def run_case(L, B, S, Hq, Hkv, seed, qscale=1.0, pad_cols=0):
+    T = B * S
+    ld = (Hq + 2 * Hkv) * HD + pad_cols
+    qkv = f16_values(ss.normal_f32(seed, "attn.qkv", (T, ld)) * np.float32(qscale))
+    dout = f16_values(ss.normal_f32(seed, "attn.dout", (T, Hq * HD)))
+    qkv_d = torch.from_numpy(qkv.astype(np.float16)).cuda()
+    dout_d = torch.from_numpy(dout.astype(np.float16)).cuda()
+    out = torch.empty((T, Hq * HD), dtype=torch.bfloat16, device="cuda")
+    out16 = torch.empty((T, Hq * HD), dtype=torch.float16, device="cuda")
+    lse = torch.empty((Hq, T), dtype=torch.float32, device="cuda")
+    L.soup_attention_fwd(qkv_d, B, S, Hq, Hkv, out, out16, lse)
+    D = torch.empty((Hq, T), dtype=torch.float32, device="cuda")
+    dqkv = torch.zeros((T, ld), dtype=torch.bfloat16, device="cuda")
+    dqkv32 = torch.zeros((T, ld), dtype=torch.float32, device="cuda")
+    L.soup_attention_bwd(qkv_d, B, S, Hq, Hkv, out16, dout_d, lse, D, dqkv, dqkv32)
+    torch.cuda.synchronize()
+    got = dict(out=host(out), lse=host(lse), dqkv=host(dqkv), dqkv32=host(dqkv32))
+    # oracle on the same fp16-exact values
+    q = qkv[:, :Hq * HD].reshape(B, S, Hq, HD)
+    k = qkv[:, Hq * HD:(Hq + Hkv) * HD].reshape(B, S, Hkv, HD)
+    v = qkv[:, (Hq + Hkv) * HD:(Hq + 2 * Hkv) * HD].reshape(B, S, Hkv, HD)
+    ref, probs = OL.attention_fwd(q, k, v)
+    dq, dk, dv = OL.attention_bwd(q, k, v, probs, dout.reshape(B, S, Hq, HD))
+    # log2 of each row's softmax denominator (with the row maximum)
+    sc = 1.0 / np.sqrt(HD)
+    lse_ref = np.empty((Hq, T))
+    for b in range(B):
+        for h in range(Hq):
+            z = (q[b, :, h] @ k[b, :, h // (Hq // Hkv)].T) * sc
+            z[np.triu(np.ones((S, S), bool), 1)] = -np.inf
+            mx = z.max(axis=1)
+            lse_ref[h, b * S:(b + 1) * S] = (mx + np.log(np.exp(z - mx[:, None]).sum(axis=1))) / np.log(2.0)
+    return got, dict(out=ref.reshape(T, Hq * HD), lse=lse_ref, dq=dq.reshape(T, -1), dk=dk.reshape(T, -1),
+                     dv=dv.reshape(T, -1)), (qkv_d, dout_d, out16, lse, D, dqkv, ld)
+
+
+CASES = [
+    (2, 100, 4, 2),    # ragged single tile per sequence, GQA group 2
+    (1, 256, 4, 1),    # two full tiles, one kv head for four q heads
+    (3, 130, 8, 2),    # a full tile and a 2-row tail, three sequences
+    (1, 1, 2, 2),      # one token: the output is v
+    (2, 384, 2, 2),    # three tiles, no grouping
+    (1, 517, 8, 2),    # five tiles with a 5-row tail
+]
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv", CASES)
+def test_attention_matches_oracle(L, B, S, Hq, Hkv):
+    got, ref, _ = run_case(L, B, S, Hq, Hkv, seed=B * 1000 + S)
+    assert_close(got["out"], ref["out"], f"out B{B} S{S}")
+    assert np.max(np.abs(got["lse"] - ref["lse"])) < 2e-3, np.max(np.abs(got["lse"] - ref["lse"]))
+    qo, ko = Hq * HD, (Hq + Hkv) * HD
+    for name, g32, gbf in (("dq", got["dqkv32"][:, :qo], got["dqkv"][:, :qo]),
+                           ("dk", got["dqkv32"][:, qo:ko], got["dqkv"][:, qo:ko]),
+                           ("dv", got["dqkv32"][:, ko:ko + Hkv * HD], got["dqkv"][:, ko:ko + Hkv * HD])):
+        if not np.any(ref[name]):
+            # one token: the softmax is the constant 1, so dq = dk = 0 exactly;
+            # the kernel's dP - D cancels to rounding level (D comes from the
+            # fp16 output, dP from the MMA)
+            assert np.max(np.abs(g32)) < 1e-5 and np.max(np.abs(gbf)) < 1e-5, name
+            continue
+        assert_close(g32, ref[name], f"{name} (fp32) B{B} S{S}")
+        assert_close(gbf, ref[name], f"{name} (bf16) B{B} S{S}")
+
+
+def test_attention_large_logits_and_row_stride(L):
+    """q, k scaled x4 (logits ~16x sharper) and a row stride with 8 extra
+    columns: the same tolerances hold and the extra columns stay untouched."""
+    got, ref, _ = run_case(L, 2, 200, 4, 2, seed=77, qscale=2.0, pad_cols=8)
+    assert_close(got["out"], ref["out"], "out (sharp)")
+    qo = 4 * HD
+    assert_close(got["dqkv32"][:, :qo], ref["dq"], "dq (sharp)")
+    assert np.all(got["dqkv"][:, -8:] == 0.0)
+
+
+def test_attention_backward_is_deterministic(L):
+    got, _, (qkv_d, dout_d, out16, lse, D, dqkv, ld) = run_case(L, 2, 300, 8, 2, seed=5)
+    first = dqkv.clone()
+    L.soup_attention_bwd(qkv_d, 2, 300, 8, 2, out16, dout_d, lse, D, dqkv)
+    torch.cuda.synchronize()
+    assert torch.equal(first, dqkv)
