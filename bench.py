@@ -325,6 +325,47 @@ def run_probe_gemm(w):
     return 0
 
 
+def run_probe_attention(w, reps=20):
+    """Times the attention kernels alone (soup_attention_fwd / _bwd, CUDA
+    events on the launching stream, after warm-up) at the workload's shape and
+    at one 2048-token sequence, random fp16 q|k|v and dO; prints one JSON
+    line per shape with TFLOP/s (algorithmic: 4 B Hq d S(S+1)/2 forward, 2.5x
+    that backward)."""
+    import torch
+
+    from layer_streamed_qlora_b200 import _lib as L
+    Hq, Hkv, d = w["n_q_heads"], w["n_kv_heads"], w["head_dim"]
+    g = torch.Generator(device="cuda").manual_seed(11)
+    for B, S in ((w["batch"], w["seq"]), (1, 2048)):
+        T = B * S
+        qkv = torch.randn(T, (Hq + 2 * Hkv) * d, device="cuda", generator=g).half()
+        dout = torch.randn(T, Hq * d, device="cuda", generator=g).half()
+        out = torch.empty(T, Hq * d, device="cuda", dtype=torch.bfloat16)
+        out16 = torch.empty(T, Hq * d, device="cuda", dtype=torch.float16)
+        lse = torch.empty(Hq, T, device="cuda")
+        D = torch.empty(Hq, T, device="cuda")
+        dqkv = torch.empty(T, (Hq + 2 * Hkv) * d, device="cuda", dtype=torch.bfloat16)
+        fl = 4.0 * B * Hq * d * S * (S + 1) / 2
+        res = {"probe": "attention", "batch": B, "seq": S, "n_q_heads": Hq, "n_kv_heads": Hkv}
+        for name, fn, flops in (("fwd", lambda: L.soup_attention_fwd(qkv, B, S, Hq, Hkv, out, out16, lse), fl),
+                                ("bwd", lambda: L.soup_attention_bwd(qkv, B, S, Hq, Hkv, out16, dout, lse, D, dqkv),
+                                 2.5 * fl)):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            res[name] = {"ms": ms, "TFLOP/s": flops / (ms / 1e3) / 1e12}
+        print(json.dumps(res), flush=True)
+    assert L.device_error() == 0
+    return 0
+
+
 def spawn_ranks(args):
     """`--gpus N` without a launcher: starts N copies of this command, one
     process per GPU with RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* set (the
@@ -417,6 +458,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--probe-gemm", action="store_true",
                     help="run each forward fused NF4 GEMM shape of one layer twice and exit (for an ncu capture)")
+    ap.add_argument("--probe-attention", action="store_true",
+                    help="time the attention kernels alone at the workload's shape and at seq 2048, and exit")
     ap.add_argument("--dist-check", action="store_true",
                     help="only join the process group of --gpus ranks and report them (launcher check)")
     ap.add_argument("--backend", default="nccl", choices=["nccl", "gloo"],
@@ -435,6 +478,8 @@ def main():
         return run_dist_check(args)
     if args.probe_gemm:
         return run_probe_gemm(w)
+    if args.probe_attention:
+        return run_probe_attention(w)
 
     import torch
     import torch.distributed as dist

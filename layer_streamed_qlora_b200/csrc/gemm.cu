@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(32 * (2 + (BMD >= B_NF4_K ? 8 : 4)), 1)
   const int num_kb = args.kb_split > 0 ? min(args.kb_split, args.num_kb - kz) : args.num_kb;
   const int n_iters = num_kb + (args.tail_ksteps > 0 ? 1 : 0);
   void* const outp = args.kb_split > 0 ? static_cast<void*>(static_cast<float*>(args.out) +
-                                                           (size_t)blockIdx.z * args.M * args.ldo)
+                                                           (size_t)blockIdx.z * args.M * args.N)
                                        : args.out;
 
   if (threadIdx.x == 0) {
@@ -1254,7 +1254,8 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
 }
 
 // Split-K epilogue: out = alpha * sum over slices (in slice order) of the
-// fp32 partial products ws[z, M, N], stored as the GEMM's own epilogue would.
+// fp32 partial products ws[z] ([M, N], or [N, M] for a transposed output),
+// stored as the GEMM's own epilogue would.
 __global__ void splitk_reduce_kernel(const float* __restrict__ ws, int splits, int M, int N, int out_kind,
                                      void* out, float* out2, uint16_t* out_lo, long long ldo, float alpha,
                                      const unsigned int* scale_amax) {
@@ -1266,7 +1267,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ ws, int splits, i
     const int m = tr ? (int)(idx % M) : (int)(idx / N);
     const int n = tr ? (int)(idx / M) : (int)(idx % N);
     float acc = 0.f;
-    for (int z = 0; z < splits; ++z) acc += ws[z * plane + (size_t)m * N + n];
+    const size_t pi = tr ? (size_t)n * M + m : (size_t)m * N + n;  // planes are [N, M] for transposed outputs
+    for (int z = 0; z < splits; ++z) acc += ws[z * plane + pi];
     const float v = acc * a;
     const size_t o = tr ? (size_t)n * ldo + m : (size_t)m * ldo + n;
     if (out_kind == OUT_F32 || out_kind == OUT_F32_T) {
@@ -1618,9 +1620,13 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
       KArgs kz = ka;
       kz.kb_split = (ka.num_kb + splits - 1) / splits;
       splits = (ka.num_kb + kz.kb_split - 1) / kz.kb_split;
+      // partial planes in the output's own orientation ([M, N], or [N, M]
+      // for transposed outputs), so that the reduction reads and writes
+      // consecutive addresses with consecutive threads
+      const bool tr = d.out_kind == OUT_BF16_T || d.out_kind == OUT_F32_T;
       kz.out = d.split_ws;
-      kz.out_kind = OUT_F32;
-      kz.ldo = d.N;
+      kz.out_kind = tr ? OUT_F32_T : OUT_F32;
+      kz.ldo = tr ? d.M : d.N;
       kz.out2 = nullptr;
       kz.out_lo = nullptr;
       kz.alpha = 1.f;

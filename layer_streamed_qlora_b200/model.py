@@ -192,8 +192,13 @@ class StreamedLoRAModel:
         self.lcfg = cfg.layer_cfg()
         precheck_device_bytes(cfg, batch, seq, n_buffers, head_chunk, device_cap_bytes)
         weights = weights or SyntheticWeights(cfg, seed)
-        self._build_blobs(weights)
+        # the model's resident tensors first, the shard build's temporaries
+        # after them: freed temporaries then leave whole cached segments that
+        # empty_cache() can hand back (no resident tensor pins them)
         self._alloc(weights)
+        self._build_blobs(weights)
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
         # q|k|v of every layer kept from the forward pass for the backward
         # (skips the backward's q|k|v GEMM; identical results), when the
         # device cap still admits the plan with it
