@@ -41,24 +41,26 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
 
-template <int BN, bool DUAL = false, int CG = 1>
+template <int BN, bool DUAL = false, int CG = 1, bool NF4B = true>
 struct Cfg {
   // DUAL: each stage holds two A tiles (the hi and lo bf16 parts of a more
   // precise A), multiplied against the same B tile.  CG = 2: the tile is
   // shared by a CTA pair (M = 256 over the pair, each CTA holds half of B).
+  // NF4B (CTA pairs): B is decoded from NF4 codes; otherwise bf16 B tiles
+  // come straight from TMA and there is no decode table.
   static constexpr int A_STAGE = A_STAGE_BYTES * (DUAL ? 2 : 1);
   static constexpr int B_STAGE = (BN / CG) * BK * 2;
-  // CTA pairs also stage the packed codes (128 rows x 32 bytes, or 64 k-rows
-  // x 64 bytes) and a 4-block-wide absmax box per stage through TMA
-  static constexpr int C_STAGE = CG == 2 ? 4096 : 0;
-  static constexpr int S_STAGE = CG == 2 ? 2048 : 0;
+  // NF4 CTA pairs also stage the packed codes (128 rows x 32 bytes, or 64
+  // k-rows x 64 bytes) and a 4-block-wide absmax box per stage through TMA
+  static constexpr int C_STAGE = (CG == 2 && NF4B) ? 4096 : 0;
+  static constexpr int S_STAGE = (CG == 2 && NF4B) ? 2048 : 0;
   static constexpr int TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   static constexpr int BAR_BYTES = 256;
   // CTA pairs: byte-indexed NF4 table (256 code pairs x 32 lanes x float2;
   // x 16 half-warp lanes when two A tiles per stage leave no room) at the
   // start of shared memory; single CTAs: nibble table after the barriers
   static constexpr int LUT_LANES = DUAL ? 16 : 32;
-  static constexpr int LUT_BYTES = CG == 2 ? 256 * LUT_LANES * 8 : 16 * 32 * 4;
+  static constexpr int LUT_BYTES = CG == 2 ? (NF4B ? 256 * LUT_LANES * 8 : 0) : 16 * 32 * 4;
   static constexpr int STAGE_BYTES = A_STAGE + B_STAGE + C_STAGE + S_STAGE;
   static constexpr int STAGE_BUDGET = CG == 2 ? (232448 - 1024 - BAR_BYTES - LUT_BYTES) : 196608;
   static constexpr int STAGES = (STAGE_BUDGET / STAGE_BYTES) > 8 ? 8 : (STAGE_BUDGET / STAGE_BYTES);
@@ -967,8 +969,9 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
                          const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmA3,
                          const KArgs args, int mtiles, int ntiles_total) {
   constexpr int BN = 256;
-  using C = Cfg<BN, DUAL, 2>;
-  constexpr bool B_MN = BMD == B_NF4_MN;
+  constexpr bool NF4 = BMD >= B_NF4_K;  // else bf16 B tiles by TMA, no decode
+  using C = Cfg<BN, DUAL, 2, NF4>;
+  constexpr bool B_MN = BMD == B_NF4_MN || BMD == B_TMA_MN;
   constexpr int STAGES = C::STAGES;
   constexpr int KSTEP_MN = 16 * 128;
   constexpr int CHUNK_BYTES = 64 * 128;
@@ -998,7 +1001,7 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&full[s], 1 + 16);
+      ptx::mbar_init(&full[s], NF4 ? 1 + 16 : 1);
       ptx::mbar_init(&empty[s], 1);
       ptx::mbar_init(&cfull[s], 1);
     }
@@ -1010,14 +1013,14 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmA);
     ptx::prefetch_tmap(&tmB);
-    ptx::prefetch_tmap(&tmA2);
+    if (NF4) ptx::prefetch_tmap(&tmA2);
     if (DUAL) ptx::prefetch_tmap(&tmA3);
     if (args.tail_ksteps > 0) {
       ptx::prefetch_tmap(&tmTA);
       ptx::prefetch_tmap(&tmTB);
     }
   }
-  if (warp >= 2 && warp < 10) {
+  if (NF4 && warp >= 2 && warp < 10) {
     float2* lut2 = reinterpret_cast<float2*>(smem_raw);
     for (int i = threadIdx.x - 64; i < 256 * C::LUT_LANES; i += 256) {
       const int b = i / C::LUT_LANES;
@@ -1055,12 +1058,24 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
           uint8_t* a = sA + s * C::A_STAGE;
           uint8_t* b = sB + s * C::B_STAGE;
           const bool tail = it >= num_kb;
-          const uint32_t bytes = tail ? (uint32_t)(A_STAGE_BYTES + C::B_STAGE) : (uint32_t)C::A_STAGE;
+          const uint32_t bytes = tail ? (uint32_t)(A_STAGE_BYTES + C::B_STAGE)
+                                      : (uint32_t)(C::A_STAGE + (NF4 ? 0 : C::B_STAGE));
           if (rank == 0) ptx::mbar_arrive_expect_tx(&full[s], 2 * bytes);
           const uint32_t bar = full0 + s * 8;
           if (!tail) {
             ptx::tma_load_2d_pair(a, &tmA, bar, it * BK, tl.m0);
             if (DUAL) ptx::tma_load_2d_pair(a + A_STAGE_BYTES, &tmA3, bar, it * BK, tl.m0);
+            if constexpr (!NF4) {
+              // bf16 B: this CTA's 128 rows (K-major; paired tiles: its half
+              // of the pair) or 128 columns as two 64-wide chunks (MN-major)
+              if constexpr (!B_MN) {
+                ptx::tma_load_2d_pair(b, &tmB, bar, it * BK, r0);
+              } else {
+                ptx::tma_load_2d_pair(b, &tmB, bar, c0, it * BK);
+                ptx::tma_load_2d_pair(b + 8192, &tmB, bar, c0 + 64, it * BK);
+              }
+              continue;
+            }
             uint8_t* c = sC + s * C::C_STAGE;
             uint8_t* sc = sS + s * C::S_STAGE;
             const int ip = it + 12;
@@ -1081,7 +1096,7 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
               }
             }
           } else {
-            ptx::mbar_arrive(&cfull[s]);  // keeps cfull's phase in step with the slot's uses
+            if (NF4) ptx::mbar_arrive(&cfull[s]);  // keeps cfull's phase in step with the slot's uses
             ptx::tma_load_2d_pair(a, &tmTA, bar, tl.m0, tl.tail_row);
             ptx::tma_load_2d_pair(a + 8192, &tmTA, bar, tl.m0 + 64, tl.tail_row);
             if (!B_MN) {
@@ -1156,6 +1171,8 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
     }
   } else if (warp < 10) {
     // ----------------------------------------------------- NF4 decode warps
+    // (bf16 B: the TMA brings the B tiles, these warps have nothing to do)
+    if constexpr (NF4) {
     const int td = threadIdx.x - 64;
     const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(full), 0);
     const uint32_t lane_b = C::LUT_LANES == 32 ? (uint32_t)lane * 8u : (uint32_t)(lane & 15) * 16u;
@@ -1213,6 +1230,7 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive_cluster(full0 + s * 8);
       }
+    }
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -1333,8 +1351,8 @@ constexpr int CU_DT_U8 = 0;  // CU_TENSOR_MAP_DATA_TYPE_UINT8
 
 template <int BN, int AMJ, int BMD, bool TF = false, bool DUAL = false, int CG = 1, bool PERSIST = false>
 soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
-  static_assert(!PERSIST || (CG == 2 && BN == 256 && AMJ == A_K && BMD >= B_NF4_K && !TF), "persistent: NF4 pairs");
-  using C = Cfg<BN, DUAL, CG>;
+  static_assert(!PERSIST || (CG == 2 && BN == 256 && AMJ == A_K && !TF), "persistent: CTA pairs, K-major A");
+  using C = Cfg<BN, DUAL, CG, (CG == 1 || BMD >= B_NF4_K)>;
   CUtensorMap mA, mB, mTA, mTB, mA2, mA3;
   memset(&mA2, 0, sizeof(mA2));
   memset(&mA3, 0, sizeof(mA3));
@@ -1348,9 +1366,11 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
   if (AMJ == A_K) SOUP_TRY(make_map(&mA, d.A, EW, 128, "A", TF));
   else SOUP_TRY(make_map(&mA, d.A, EW, EW, "A (MN-major)", TF, TF ? CU_SWIZZLE_128B_ATOM_32B : CU_SWIZZLE_128B));
   constexpr bool B_MN = (BMD == B_TMA_MN || BMD == B_NF4_MN);
-  if (BMD == B_TMA_K) SOUP_TRY(make_map(&mB, d.B, EW, paired ? BN / 2 : BN, "B", TF));
+  // K-major B boxes: the tile's rows (CTA pairs: this CTA's 128 of them;
+  // paired gate|up tiles: one half of the pair's rows)
+  if (BMD == B_TMA_K) SOUP_TRY(make_map(&mB, d.B, EW, CG == 2 ? 128 : (paired ? BN / 2 : BN), "B", TF));
   if (BMD == B_TMA_MN) SOUP_TRY(make_map(&mB, d.B, 64, 64, "B (MN-major)"));
-  if (CG == 2) {
+  if (CG == 2 && BMD >= B_NF4_K) {
     // codes and absmax staged per stage: K-major 128 rows x 32 bytes and a
     // 128 x 4 absmax box; transposed 64 k-rows x 64 bytes and a 64 x 4 box
     if (BMD == B_NF4_K) {
@@ -1399,10 +1419,12 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
     const int npairs = std::min(total, max_pairs);
     cfg.gridDim = dim3(2 * npairs);
     if (profiling()) {
-      const int cls = DUAL ? GC_NF4_DUAL : (BMD == B_NF4_K ? GC_NF4_FWD : GC_NF4_BWD);
+      const int cls = BMD < B_NF4_K ? GC_BF16
+                                    : (DUAL ? GC_NF4_DUAL : (BMD == B_NF4_K ? GC_NF4_FWD : GC_NF4_BWD));
       const double tail_k = d.tail_ksteps > 0 ? (double)d.tailA.rows : 0.0;
       const double flops = 2.0 * d.M * d.N * ((double)d.K * (DUAL ? 2 : 1) + (paired ? 16.0 : tail_k));
-      const double bytes = (double)d.M * d.K * 2 + (double)d.N * d.K * (0.5 + 4.0 / 64) +
+      const double wbytes = BMD >= B_NF4_K ? (double)d.N * d.K * (0.5 + 4.0 / 64) : (double)d.N * d.K * 2;
+      const double bytes = (double)d.M * d.K * 2 + wbytes +
                            (double)d.M * d.N * ((d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T) ? 4 : 2);
       profile_begin(st, cls, flops, bytes);
     }
@@ -1410,7 +1432,7 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
     SOUP_LAUNCH_CHECK();
     profile_end(st);
     return SOUP_OK;
-  }
+  } else {
   auto kern = gemm_kernel<BN, AMJ, BMD, TF, DUAL, CG>;
   static bool attr_set = false;  // per instantiation
   if (!attr_set) {
@@ -1454,6 +1476,7 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
   SOUP_LAUNCH_CHECK();
   profile_end(st);
   return SOUP_OK;
+  }
 }
 
 int pick_bn(const GemmDesc& d) {
@@ -1484,6 +1507,13 @@ soup_status dispatch(const GemmDesc& d, const KArgs& ka, int bn, cudaStream_t st
     SOUP_GEMM_TF(64, A_MN) SOUP_GEMM_TF(48, A_MN) SOUP_GEMM_TF(32, A_MN) SOUP_GEMM_TF(16, A_MN)
 #undef SOUP_GEMM_TF
     return fail(SOUP_ERR_SHAPE, "gemm: no tf32 kernel for BN=%d", bn);
+  }
+  // bf16 B with 256-wide tiles and at least one 256-row M tile: the
+  // persistent CTA-pair engine with TMA-fed B (no split-K, single A)
+  if (!nf4 && !d.A_lo.ptr && bn == 256 && d.a_major == A_K && d.M >= 256 && ka.kb_split == 0 && d.persistent &&
+      (d.b_mode == B_TMA_K || (d.b_mode == B_TMA_MN && d.N % 256 == 0))) {
+    if (d.b_mode == B_TMA_K) return launch<256, A_K, B_TMA_K, false, false, 2, true>(d, ka, st);
+    return launch<256, A_K, B_TMA_MN, false, false, 2, true>(d, ka, st);
   }
   // NF4 B with 256-wide tiles: CTA pairs (half the decode per CTA)
   const bool pair_ok = nf4 && bn == 256 && d.a_major == A_K && soup_aligned(d.absmax, 16) &&

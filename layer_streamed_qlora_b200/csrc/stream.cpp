@@ -39,7 +39,8 @@ struct TimedRing {
         return soup::fail(SOUP_ERR_CUDA, "timing event creation failed");
       }
       ev.emplace_back(a, b);
-    } else {
+    } else if (recorded >= kCap) {
+      // this entry holds a pair recorded since the last reset (a lap ago)
       SOUP_CUDA_TRY(cudaEventSynchronize(ev[i].second));
       float ms = 0.f;
       SOUP_CUDA_TRY(cudaEventElapsedTime(&ms, ev[i].first, ev[i].second));
@@ -49,10 +50,11 @@ struct TimedRing {
     *out = &ev[i];
     return SOUP_OK;
   }
-  // Total elapsed time of every pair recorded since the last reset.
+  // Total elapsed time of every pair recorded since the last reset (entries
+  // [0, min(recorded, kCap)) hold this lap's pairs; older ones are folded).
   soup_status total_ms(double* out) const {
     double t = folded_ms;
-    const size_t live = std::min(recorded, ev.size());
+    const size_t live = std::min(recorded, kCap);
     for (size_t i = 0; i < live; ++i) {
       SOUP_CUDA_TRY(cudaEventSynchronize(ev[i].second));
       float ms = 0.f;

@@ -137,6 +137,33 @@ def test_timing_events_stay_bounded_and_totals_survive_the_ring():
     plan.free()
 
 
+def test_timing_totals_after_a_reset_count_only_new_pairs():
+    """After soup_stream_stats_reset the rings still hold a lap of older
+    event pairs; the totals of the next few copies must not include them:
+    20 copies of 1 MiB after the reset take about 20/600 of the 600 copies
+    before it (the copies are identical), not twice that."""
+    nb = 1 << 20
+    plan = L.Plan(_blobs(3, nb), nb, 2)
+
+    def cycles(n):
+        for i in range(n):
+            item = i % 3
+            plan.prefetch(item)
+            plan.wait(item)
+            plan.release(item)
+        torch.cuda.synchronize()
+
+    cycles(600)
+    before = plan.stats()
+    plan.reset_stats()
+    cycles(20)
+    after = plan.stats()
+    assert after["copies"] == 20 and after["waits"] == 20
+    expect = before["copy_ms"] * 20 / 600
+    assert 0.5 * expect <= after["copy_ms"] <= 1.6 * expect, (after["copy_ms"], expect)
+    plan.free()
+
+
 def test_gemm_bounded_wait_runs_out_and_the_context_survives():
     """The producer of a one-CTA tcgen05 GEMM is told to skip its arrivals and
     the kernel's mbarrier waits are limited to 2e6 SM cycles (~1 ms): the MMA
