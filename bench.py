@@ -235,7 +235,7 @@ def cpu_baseline(w, tokens=256):
             "sample": _sample_text(w, tokens, t, ta, th)}
 
 
-def bench_config(w, name, world, kept_layers=None):
+def bench_config(w, name, world, kept_layers=None, saved_layers=None, recompute=None):
     cfg = {"workload": name, "global_batch": w["batch"] * world, "seq_len": w["seq"], "layers": w["n_layers"],
            "base": w["kind"], "stream_buffers": w["buffers"], "device_cap_gb": w["cap_gb"],
            "device_cap_bytes": int(w["cap_gb"] * (1 << 30)),
@@ -244,6 +244,10 @@ def bench_config(w, name, world, kept_layers=None):
            "optimizer": "AdamW on the LoRA adapters every step (lr 5e-4, fp32 master + moments)"}
     if kept_layers is not None:
         cfg["kept_qkv_layers"] = kept_layers
+    if saved_layers is not None:
+        cfg["saved_layers"] = saved_layers
+    if recompute is not None:
+        cfg["stream_recompute"] = recompute
     return cfg
 
 
@@ -455,6 +459,9 @@ def main():
                     help="stream_source: layer shards in pinned RAM, or files read ahead from disk")
     ap.add_argument("--shard-dir", default="", help="directory for the disk tier's shard files (default: a temp dir)")
     ap.add_argument("--read-ahead", type=int, default=2, help="stream_read_ahead for the disk tier (1..8)")
+    ap.add_argument("--recompute", default="auto", choices=["auto", "recompute", "keep"],
+                    help="stream_recompute: keep activations for the backward as the cap admits (auto), keep none, "
+                         "or keep every layer's")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--probe-gemm", action="store_true",
                     help="run each forward fused NF4 GEMM shape of one layer twice and exit (for an ncu capture)")
@@ -510,7 +517,8 @@ def main():
         import tempfile
         shard_dir = args.shard_dir or tempfile.mkdtemp(prefix="soup_shards_")
     model = StreamedLoRAModel(cfg, B, S, n_buffers=w["buffers"], device_cap_bytes=cap, seed=0, task=w["task"],
-                              stream_source=args.source, shard_dir=shard_dir, read_ahead=args.read_ahead)
+                              stream_source=args.source, shard_dir=shard_dir, read_ahead=args.read_ahead,
+                              stream_recompute=args.recompute)
     t_build = time.time() - t_build
     g = torch.Generator().manual_seed(1000 + rank)
     ids_host = torch.randint(0, cfg.vocab, (B, S), generator=g, dtype=torch.int32).pin_memory()
@@ -652,7 +660,8 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(bench_config(w, args.workload, world, 0 if model.keep is None else int(model.keep.shape[0])),
+        "config": dict(bench_config(w, args.workload, world, sum(1 for k in model.keep_plan if k == "qkv"),
+                                    sum(1 for k in model.keep_plan if k == "saved"), args.recompute),
                        stream_source=args.source,
                        **({"read_ahead": args.read_ahead} if args.source == "disk" else {})),
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": ids_host.numel() * 4,

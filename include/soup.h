@@ -317,6 +317,30 @@ soup_status soup_decoder_layer_bwd_kept(const soup_layer_weights* W, const soup_
                                         const uint16_t* qkv_kept, void* workspace, size_t workspace_bytes,
                                         void* stream);
 
+/* Keep-activations form (the pages' `stream_recompute` key: keep the
+ * layer's activations instead of recomputing them; Soup pages, the streaming
+ * configuration keys).  soup_decoder_layer_fwd_save runs the forward pass and
+ * leaves every intermediate the backward reads (the normalised inputs, q|k|v
+ * from the hi + lo input, the attention output and log-sum-exp, the mid
+ * residual, the SwiGLU inputs and output, the LoRA down-projections, ...) in
+ * `saved`, soup_decoder_layer_saved_bytes bytes, 256-byte aligned, owned by
+ * the caller and left untouched until soup_decoder_layer_bwd_saved of the
+ * same layer, which then runs no forward recompute at all (the layer is still
+ * read a second time: the backward needs W^T).  Results are bit-identical to
+ * the soup_decoder_layer_fwd_keep / soup_decoder_layer_bwd_kept pair (same
+ * kernels on the same values).  The workspace is the same as for the other
+ * forms. */
+size_t soup_decoder_layer_saved_bytes(const soup_layer_cfg* cfg, int64_t batch, int64_t seq);
+soup_status soup_decoder_layer_fwd_save(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                        const soup_layer_cfg* cfg, const uint16_t* h_in, int64_t batch,
+                                        int64_t seq, uint16_t* h_out, int32_t adapters_on, void* saved,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+soup_status soup_decoder_layer_bwd_saved(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                         const soup_layer_cfg* cfg, const uint16_t* h_in,
+                                         const float* dh_out, int64_t batch, int64_t seq, float* dh_in,
+                                         const soup_layer_grads* grads, int32_t adapters_on, const void* saved,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------- layer streaming ---
  * The frozen base lives in pinned host RAM as one blob per decoder layer
  * (Soup pages, "how layer streaming works": per-layer shards in page-locked

@@ -122,6 +122,14 @@ _SIGS = {
                                               ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_int64, c_int64,
                                               c_void_p, ctypes.POINTER(LayerGrads), c_int32, c_void_p, c_void_p,
                                               c_size_t, c_void_p]),
+    "soup_decoder_layer_saved_bytes": (c_size_t, [ctypes.POINTER(LayerCfg), c_int64, c_int64]),
+    "soup_decoder_layer_fwd_save": (c_int32, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerLora),
+                                              ctypes.POINTER(LayerCfg), c_void_p, c_int64, c_int64, c_void_p,
+                                              c_int32, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "soup_decoder_layer_bwd_saved": (c_int32, [ctypes.POINTER(LayerWeights), ctypes.POINTER(LayerLora),
+                                               ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_int64, c_int64,
+                                               c_void_p, ctypes.POINTER(LayerGrads), c_int32, c_void_p, c_void_p,
+                                               c_size_t, c_void_p]),
     "soup_stream_plan": (c_int32, [ctypes.POINTER(StreamDesc), ctypes.POINTER(c_void_p)]),
     "soup_stream_plan_free": (c_int32, [c_void_p]),
     "soup_stream_prefetch": (c_int32, [c_void_p, c_int32]),
@@ -353,6 +361,27 @@ def soup_decoder_layer_bwd_kept(W: LayerWeights, lora, cfg: LayerCfg, h_in, dh_o
     _check("soup_decoder_layer_bwd_kept", lib().soup_decoder_layer_bwd_kept(
         ctypes.byref(W), lp, ctypes.byref(cfg), _p(h_in), _p(dh_out), batch, seq, _p(dh_in), gp, int(adapters_on),
         _p(qkv_kept), _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def soup_decoder_layer_saved_bytes(cfg: LayerCfg, batch, seq) -> int:
+    return int(lib().soup_decoder_layer_saved_bytes(ctypes.byref(cfg), batch, seq))
+
+
+def soup_decoder_layer_fwd_save(W: LayerWeights, lora, cfg: LayerCfg, h_in, batch, seq, h_out, adapters_on, saved,
+                                workspace, stream=None):
+    lp = ctypes.byref(lora) if lora is not None else None
+    _check("soup_decoder_layer_fwd_save", lib().soup_decoder_layer_fwd_save(
+        ctypes.byref(W), lp, ctypes.byref(cfg), _p(h_in), batch, seq, _p(h_out), int(adapters_on), _p(saved),
+        _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def soup_decoder_layer_bwd_saved(W: LayerWeights, lora, cfg: LayerCfg, h_in, dh_out, batch, seq, dh_in, grads,
+                                 adapters_on, saved, workspace, stream=None):
+    lp = ctypes.byref(lora) if lora is not None else None
+    gp = ctypes.byref(grads) if grads is not None else None
+    _check("soup_decoder_layer_bwd_saved", lib().soup_decoder_layer_bwd_saved(
+        ctypes.byref(W), lp, ctypes.byref(cfg), _p(h_in), _p(dh_out), batch, seq, _p(dh_in), gp, int(adapters_on),
+        _p(saved), _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 # ---------------------------------------------------------------- streaming

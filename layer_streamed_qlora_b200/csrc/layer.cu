@@ -42,6 +42,7 @@ struct WS {
   size_t u_gu_lo, g_d_lo, u_d32;     // MLP LoRA-gradient operands beyond bf16 (residuals, fp32)
   size_t x2_32, Agu32, g_gu32, d_gu_lo;
   size_t Bt_down32, Bt_o32, Bbd_qkv32, Bbd_gu;  // B factors prepared for the g GEMMs (transposed, block-diagonal)
+  size_t fwd_bytes;  // [0, fwd_bytes): the fields the forward pass leaves for the backward
   size_t total;
 };
 
@@ -54,6 +55,8 @@ WS layout(const Dims& m) {
     return at;
   };
   const size_t T = m.T, H = m.H, I = m.I, r = m.r, ldT = m.ldT;
+  // ---- fields the forward pass computes and the backward reads (the part a
+  // saved layer keeps): offsets [0, fwd_bytes)
   w.x1 = take(T * H * 2);
   w.rinv1 = take(T * 4);
   w.qkv = take(T * m.qkv_w * 2);  // fp16
@@ -70,12 +73,25 @@ WS layout(const Dims& m) {
   w.u_d = take(r * ldT * 2);
   w.cosb = take((size_t)m.S * (m.d / 2) * 4);
   w.sinb = take((size_t)m.S * (m.d / 2) * 4);
+  w.attn16 = take(T * m.o_in * 2);  // fp16 copy of the attention output (for D = rowsum(dO * O))
+  w.x1_32 = take(T * H * 4);
+  w.u32 = take(3 * r * ldT * 4);
+  w.A32 = take(3 * r * H * 4);
+  w.x1_lo = take(T * H * 2);
+  w.attn32 = take(T * m.o_in * 4);
+  w.uo32 = take(r * ldT * 4);
+  w.Ao32 = take(r * (size_t)m.o_in * 4);
+  w.u_gu_lo = take(2 * r * ldT * 2);
+  w.u_d32 = take(r * ldT * 4);
+  w.x2_32 = take(T * H * 4);
+  w.Agu32 = take(2 * r * H * 4);
+  w.fwd_bytes = o;
+  // ---- backward-only fields and scratch
   w.dh_b = take(T * H * 2);
   w.g_d = take(r * ldT * 2);
   w.g_gu = take(2 * r * ldT * 2);
   w.g_o = take(r * ldT * 2);
   w.g_qkv = take(3 * r * ldT * 2);
-  size_t max_out = std::max<size_t>(std::max<size_t>(H, I), (size_t)m.qkv_w);
   w.d_gu = take(T * 2 * I * 2);
   w.dx2 = take(T * H * 2);
   w.dh2 = take(T * H * 4);
@@ -84,26 +100,14 @@ WS layout(const Dims& m) {
   w.D = take((size_t)m.Hq * T * 4);
   w.d_qkv = take(T * m.qkv_w * 2);
   w.dx1 = take(T * H * 2);
-  w.attn16 = take(T * m.o_in * 2);  // fp16 copy of the attention output (for D = rowsum(dO * O))
   w.gamax = take(4);                // max |dh2| bit pattern (gradient scale of dO)
-  w.x1_32 = take(T * H * 4);
   w.dqkv32 = take(T * m.qkv_w * 4);
-  w.u32 = take(3 * r * ldT * 4);
   w.g32 = take(3 * r * ldT * 4);
-  w.A32 = take(3 * r * H * 4);
-  w.x1_lo = take(T * H * 2);
   w.dh2_lo = take(T * H * 2);
-  w.attn32 = take(T * m.o_in * 4);
-  w.uo32 = take(r * ldT * 4);
   w.go32 = take(r * ldT * 4);
-  w.Ao32 = take(r * (size_t)m.o_in * 4);
   w.splitk_bytes = 8 * T * 64 * 4;
   w.splitk = take(w.splitk_bytes);
-  w.u_gu_lo = take(2 * r * ldT * 2);
   w.g_d_lo = take(r * ldT * 2);
-  w.u_d32 = take(r * ldT * 4);
-  w.x2_32 = take(T * H * 4);
-  w.Agu32 = take(2 * r * H * 4);
   w.g_gu32 = take(2 * r * ldT * 4);
   w.d_gu_lo = take(T * 2 * I * 2);
   w.Bt_down32 = take(r * H * 4);
@@ -148,8 +152,12 @@ soup_status check_weights(const soup_layer_weights* W, const Dims& m) {
   return SOUP_OK;
 }
 
-#define P(off) (reinterpret_cast<uint16_t*>(base + ws.off))
-#define PF(off) (reinterpret_cast<float*>(base + ws.off))
+// Field addresses: the forward pass's fields [0, fwd_bytes) live at `fb` (the
+// layer workspace itself, or a saved layer's own region), the backward-only
+// fields and scratch at `base` (the layer workspace).
+#define FIELD(off) ((ws.off) < ws.fwd_bytes ? fb + (ws.off) : base + (ws.off))
+#define P(off) (reinterpret_cast<uint16_t*>(FIELD(off)))
+#define PF(off) (reinterpret_cast<float*>(FIELD(off)))
 
 // y = x W^T (+ tail u B^T) (+ resid) into out [T, N]
 struct ProjOpts {
@@ -345,18 +353,21 @@ soup_status proj_bwd(const soup_weight* W, const uint16_t* dy, int T, const uint
   return gemm(g, st);
 }
 
-// Forward through the layer; with `keep_down_out` false the final down GEMM
-// (whose output the backward pass does not need) is skipped.
+// Forward through the layer.  save: also produce what only the backward
+// reads (fp16 g | u for the SwiGLU backward, the fp16 attention output for
+// D, q|k|v from the hi + lo x1 pair); want_out: run the final down GEMM
+// (the recompute inside the backward does not need its output).  The
+// forward fields go to `fb` (FIELD), scratch to `base`.
 // keep (forward pass only): also compute q|k|v with the hi + lo A pair and
 // leave them (fp16, [T, qkv_w]) in `keep` for the backward; kept (recompute
 // only): q|k|v of this layer kept by the forward pass, whose GEMM is skipped.
 soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const soup_layer_cfg* c, const Dims& m,
-                    const WS& ws, char* base, const uint16_t* h_in, uint16_t* h_out, bool on, bool recompute,
-                    cudaStream_t st, uint16_t* keep = nullptr, const uint16_t* kept = nullptr) {
+                    const WS& ws, char* base, char* fb, const uint16_t* h_in, uint16_t* h_out, bool on, bool save,
+                    bool want_out, cudaStream_t st, uint16_t* keep = nullptr, const uint16_t* kept = nullptr) {
   const int T = m.T, r = m.r;
   const SplitWS SW{PF(splitk), ws.splitk_bytes};
   SOUP_TRY(rope_table(m.S, m.d, (double)c->theta, PF(cosb), PF(sinb), st));
-  const bool precise_qkv = (recompute && !kept) || keep;  // q|k|v from the hi + lo x1 pair
+  const bool precise_qkv = (save && !kept) || keep;  // q|k|v from the hi + lo x1 pair
   SOUP_TRY(rmsnorm_fwd(h_in, nullptr, W->norm1, T, m.H, c->eps, P(x1), PF(rinv1), st, on ? PF(x1_32) : nullptr,
                        precise_qkv ? P(x1_lo) : nullptr));
   if (on) {
@@ -388,7 +399,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
   }
   const uint16_t* qkvp = kept ? kept : (keep ? keep : P(qkv));
   SOUP_TRY(attention_fwd(qkvp, m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(attn), PF(lse), st,
-                         recompute ? P(attn16) : nullptr, on ? PF(attn32) : nullptr));
+                         save ? P(attn16) : nullptr, on ? PF(attn32) : nullptr));
   if (on) {
     SOUP_TRY(lora_down_tf32(PF(attn32), T, m.o_in, PF(Ao32), r, m.s, P(u_o), PF(uo32), m.ldT, st, SW));
   }
@@ -411,12 +422,12 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     const int sr[1] = {0};
     ProjOpts o;
     o.swiglu_I = m.I;
-    o.aux16 = recompute ? P(gu16) : nullptr;  // g | u are needed only by the backward
+    o.aux16 = save ? P(gu16) : nullptr;  // g | u are needed only by the backward
     SOUP_TRY(proj_fwd(&W->gate_up, P(x2), T, P(u_gu), m.ldT, 2 * r, L ? L->B_gu : nullptr, r, 1, se, sr, on,
                       P(act), st, o));
   }
   if (on) SOUP_TRY(lora_down(P(act), T, m.I, L->A_down, r, m.s, P(u_d), m.ldT, st, SW, PF(u_d32)));
-  if (!recompute) {
+  if (want_out) {
     const int se[1] = {m.H};
     const int sr[1] = {0};
     ProjOpts o;
@@ -438,6 +449,12 @@ extern "C" size_t soup_decoder_layer_workspace(const soup_layer_cfg* cfg, int64_
   return layout(m).total;
 }
 
+extern "C" size_t soup_decoder_layer_saved_bytes(const soup_layer_cfg* cfg, int64_t batch, int64_t seq) {
+  Dims m;
+  if (make_dims(cfg, batch, seq, &m) != SOUP_OK) return 0;
+  return layout(m).fwd_bytes;
+}
+
 extern "C" size_t soup_decoder_layer_keep_bytes(const soup_layer_cfg* cfg, int64_t batch, int64_t seq) {
   Dims m;
   if (make_dims(cfg, batch, seq, &m) != SOUP_OK) return 0;
@@ -447,7 +464,7 @@ extern "C" size_t soup_decoder_layer_keep_bytes(const soup_layer_cfg* cfg, int64
 static soup_status layer_fwd_impl(const soup_layer_weights* W, const soup_layer_lora* lora, const soup_layer_cfg* cfg,
                                   const uint16_t* h_in, int64_t batch, int64_t seq, uint16_t* h_out,
                                   int32_t adapters_on, void* workspace, size_t workspace_bytes, void* stream,
-                                  uint16_t* keep) {
+                                  uint16_t* keep, void* saved = nullptr) {
   Dims m;
   SOUP_TRY(make_dims(cfg, batch, seq, &m));
   SOUP_TRY(check_weights(W, m));
@@ -458,7 +475,13 @@ static soup_status layer_fwd_impl(const soup_layer_weights* W, const soup_layer_
   const WS ws = layout(m);
   SOUP_CHECK(workspace_bytes >= ws.total && soup_aligned(workspace, 256), SOUP_ERR_INVALID_ARG,
              "soup_decoder_layer_fwd: workspace %zu < %zu bytes or misaligned", workspace_bytes, ws.total);
-  return forward(W, lora, cfg, m, ws, static_cast<char*>(workspace), h_in, h_out, adapters_on != 0, false,
+  char* base = static_cast<char*>(workspace);
+  if (saved) {  // everything the backward reads stays in the layer's saved region
+    SOUP_CHECK(soup_aligned(saved, 256), SOUP_ERR_ALIGN, "soup_decoder_layer_fwd_save: saved region not 256-byte aligned");
+    return forward(W, lora, cfg, m, ws, base, static_cast<char*>(saved), h_in, h_out, adapters_on != 0, true, true,
+                   static_cast<cudaStream_t>(stream));
+  }
+  return forward(W, lora, cfg, m, ws, base, base, h_in, h_out, adapters_on != 0, false, true,
                  static_cast<cudaStream_t>(stream), keep);
 }
 
@@ -481,10 +504,20 @@ extern "C" soup_status soup_decoder_layer_fwd_keep(const soup_layer_weights* W, 
                         qkv_keep);
 }
 
+extern "C" soup_status soup_decoder_layer_fwd_save(const soup_layer_weights* W, const soup_layer_lora* lora,
+                                                   const soup_layer_cfg* cfg, const uint16_t* h_in, int64_t batch,
+                                                   int64_t seq, uint16_t* h_out, int32_t adapters_on, void* saved,
+                                                   void* workspace, size_t workspace_bytes, void* stream) {
+  SOUP_CHECK(saved, SOUP_ERR_INVALID_ARG, "soup_decoder_layer_fwd_save: null saved region");
+  return layer_fwd_impl(W, lora, cfg, h_in, batch, seq, h_out, adapters_on, workspace, workspace_bytes, stream,
+                        nullptr, saved);
+}
+
 static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_lora* L, const soup_layer_cfg* cfg,
                                   const uint16_t* h_in, const float* dh_out, int64_t batch, int64_t seq, float* dh_in,
                                   const soup_layer_grads* G, int32_t adapters_on, void* workspace,
-                                  size_t workspace_bytes, void* stream, const uint16_t* kept) {
+                                  size_t workspace_bytes, void* stream, const uint16_t* kept,
+                                  const void* saved = nullptr) {
   Dims m;
   SOUP_TRY(make_dims(cfg, batch, seq, &m));
   SOUP_TRY(check_weights(W, m));
@@ -498,11 +531,19 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
              "soup_decoder_layer_bwd: workspace %zu < %zu bytes or misaligned", workspace_bytes, ws.total);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(workspace);
+  char* fb = base;  // forward fields (below: or the saved region)
   const SplitWS SW{PF(splitk), ws.splitk_bytes};
   const int T = m.T, r = m.r, H = m.H, I = m.I;
   const int64_t ldT = m.ldT;
 
-  SOUP_TRY(forward(W, L, cfg, m, ws, base, h_in, nullptr, on, true, st, nullptr, kept));
+  // forward fields: recomputed into the workspace (the layer was read again
+  // for this), or what a saved forward pass left in the layer's own region
+  if (saved) {
+    SOUP_CHECK(soup_aligned(saved, 256), SOUP_ERR_ALIGN, "soup_decoder_layer_bwd_saved: saved region not 256-byte aligned");
+    fb = static_cast<char*>(const_cast<void*>(saved));
+  } else {
+    SOUP_TRY(forward(W, L, cfg, m, ws, base, fb, h_in, nullptr, on, true, false, st, nullptr, kept));
+  }
   const uint16_t* qkvp = kept ? kept : P(qkv);
 
   // ---- B factors for the g GEMMs, one launch: B_down^T and B_o^T (fp32),
@@ -653,4 +694,14 @@ extern "C" soup_status soup_decoder_layer_bwd_kept(const soup_layer_weights* W, 
              "soup_decoder_layer_bwd_kept: null or misaligned kept buffer");
   return layer_bwd_impl(W, L, cfg, h_in, dh_out, batch, seq, dh_in, G, adapters_on, workspace, workspace_bytes,
                         stream, qkv_kept);
+}
+
+extern "C" soup_status soup_decoder_layer_bwd_saved(const soup_layer_weights* W, const soup_layer_lora* L,
+                                                    const soup_layer_cfg* cfg, const uint16_t* h_in,
+                                                    const float* dh_out, int64_t batch, int64_t seq, float* dh_in,
+                                                    const soup_layer_grads* G, int32_t adapters_on, const void* saved,
+                                                    void* workspace, size_t workspace_bytes, void* stream) {
+  SOUP_CHECK(saved, SOUP_ERR_INVALID_ARG, "soup_decoder_layer_bwd_saved: null saved region");
+  return layer_bwd_impl(W, L, cfg, h_in, dh_out, batch, seq, dh_in, G, adapters_on, workspace, workspace_bytes,
+                        stream, nullptr, saved);
 }

@@ -164,6 +164,43 @@ def kept_layer_count(n_layers: int, per_layer: int, arena: int, reserve: int, ca
     return max(0, min(n_layers, room // per_layer))
 
 
+STREAM_RECOMPUTE = ("auto", "recompute", "keep")
+
+
+def plan_keep(n_layers: int, qkv_bytes: int, saved_bytes: int, arena: int, reserve: int, cap: int,
+              mode: str = "auto") -> list:
+    """Per-layer plan of what the forward pass keeps for the backward (the
+    pages' `stream_recompute` key): "saved" (every intermediate: no forward
+    recompute in the backward), "qkv" (q|k|v only: the backward skips its
+    q|k|v GEMM) or None (full recompute), such that the slot arena, the
+    model's own device bytes (reserve) and the kept bytes fit a nonzero cap.
+
+    recompute: keep nothing.  keep: every layer saved, or ValueError when
+    that does not fit.  auto: q|k|v first for as many layers as fit (it saves
+    the most recompute time per byte), then, when every layer keeps q|k|v
+    and room is left, upgrade layers (from the first) to saved ones."""
+    if mode not in STREAM_RECOMPUTE:
+        raise ValueError(f"stream_recompute must be one of {STREAM_RECOMPUTE}, not {mode!r}")
+    if mode == "recompute" or n_layers <= 0:
+        return [None] * max(0, n_layers)
+    room = (cap - arena - reserve) if cap else None
+    if mode == "keep":
+        need = n_layers * saved_bytes
+        if room is not None and need > room:
+            raise ValueError(f"stream_recompute='keep' needs {need} device bytes for {n_layers} saved layers, "
+                             f"{max(0, room)} left under the device cap {cap}")
+        return ["saved"] * n_layers
+    if room is None:
+        return ["saved"] * n_layers
+    n_qkv = 0 if qkv_bytes <= 0 else max(0, min(n_layers, room // qkv_bytes))
+    plan = ["qkv"] * n_qkv + [None] * (n_layers - n_qkv)
+    if n_qkv == n_layers and saved_bytes > qkv_bytes:
+        extra = room - n_layers * qkv_bytes
+        for l in range(min(n_layers, max(0, extra) // (saved_bytes - qkv_bytes))):
+            plan[l] = "saved"
+    return plan
+
+
 class StreamedLoRAModel:
     """Frozen base in pinned host blobs + a soup_plan slot ring + resident LoRA.
 
@@ -175,13 +212,16 @@ class StreamedLoRAModel:
     def __init__(self, cfg: ModelConfig, batch: int, seq: int, n_buffers: int = 2, device_cap_bytes: int = 0,
                  head_chunk: int = 256, weights=None, seed: int = 0, adamw: AdamW | None = None,
                  task: str = "sft", stream_source: str = "ram", shard_dir: str | None = None,
-                 read_ahead: int = 2, io_threads: int = 4):
+                 read_ahead: int = 2, io_threads: int = 4, stream_recompute: str = "auto"):
         self.cfg, self.batch, self.seq, self.n_buffers = cfg, batch, seq, n_buffers
         if stream_source not in ("ram", "disk"):
             raise ValueError(f"stream_source must be 'ram' or 'disk', not {stream_source!r}")
         if stream_source == "disk" and not shard_dir:
             raise ValueError("stream_source='disk' needs a shard_dir for the per-layer shard files")
         self.stream_source, self.shard_dir = stream_source, shard_dir
+        if stream_recompute not in STREAM_RECOMPUTE:
+            raise ValueError(f"stream_recompute must be one of {STREAM_RECOMPUTE}, not {stream_recompute!r}")
+        self.stream_recompute = stream_recompute
         self.disk = None
         self.adamw = adamw or AdamW()
         if task not in ("sft", "dpo", "simpo", "orpo"):
@@ -199,17 +239,29 @@ class StreamedLoRAModel:
         self._build_blobs(weights)
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
-        # q|k|v of every layer kept from the forward pass for the backward
-        # (skips the backward's q|k|v GEMM; identical results), when the
-        # device cap still admits the plan with it
-        # (layers 0 .. n_keep-1: as many as fit)
+        # what each layer's forward pass keeps for its backward (identical
+        # results either way): every intermediate ("saved": no recompute),
+        # q|k|v ("qkv": the backward skips its q|k|v GEMM) or nothing, as the
+        # device cap admits (stream_recompute)
         per = L.soup_decoder_layer_keep_bytes(self.lcfg, batch, seq)
-        n_keep = kept_layer_count(cfg.n_layers, per, self.n_buffers * self.blob_bytes + self.vocab_bytes,
-                                  self.reserve_bytes, device_cap_bytes)
-        self.keep = None
-        if per and n_keep:
+        per_saved = L.soup_decoder_layer_saved_bytes(self.lcfg, batch, seq)
+        self.keep_plan = plan_keep(cfg.n_layers, per, per_saved, self.n_buffers * self.blob_bytes + self.vocab_bytes,
+                                   self.reserve_bytes, device_cap_bytes, stream_recompute)
+        n_keep = sum(1 for k in self.keep_plan if k == "qkv")
+        n_saved = sum(1 for k in self.keep_plan if k == "saved")
+        self.keep, self.saved = None, None
+        self.keep_row, self.saved_row = {}, {}
+        if n_keep:
             self.keep = torch.empty((n_keep, per // 2), dtype=torch.float16, device="cuda")
             self.reserve_bytes += n_keep * per
+        if n_saved:
+            self.saved = torch.empty((n_saved, per_saved), dtype=torch.uint8, device="cuda")
+            self.reserve_bytes += n_saved * per_saved
+        for l, k in enumerate(self.keep_plan):
+            if k == "qkv":
+                self.keep_row[l] = len(self.keep_row)
+            elif k == "saved":
+                self.saved_row[l] = len(self.saved_row)
         self.plan = L.Plan(self.host_layers, self.blob_bytes, n_buffers, self.vocab_bytes, self.host_embed,
                            self.host_head, device_cap_bytes, self.reserve_bytes, n_layers=cfg.n_layers)
         if stream_source == "disk":
@@ -325,8 +377,13 @@ class StreamedLoRAModel:
         self.dh = torch.empty((T, cfg.hidden), dtype=torch.float32, device="cuda")
         self.ws = torch.empty(L.soup_decoder_layer_workspace(self.lcfg, self.batch, self.seq), dtype=torch.uint8,
                               device="cuda")
-        self.head_ws = torch.empty(L.soup_head_workspace(cfg.vocab, cfg.hidden, self.batch, self.seq,
-                                                         self.head_chunk), dtype=torch.uint8, device="cuda")
+        # the output head runs between the layer passes, never during a layer
+        # call: its workspace shares the layer workspace's memory
+        head_bytes = L.soup_head_workspace(cfg.vocab, cfg.hidden, self.batch, self.seq, self.head_chunk)
+        if head_bytes <= self.ws.numel():
+            self.head_ws = self.ws[:head_bytes]
+        else:
+            self.head_ws = torch.empty(head_bytes, dtype=torch.uint8, device="cuda")
         self.logp = torch.empty((self.batch, self.seq - 1), dtype=torch.float32, device="cuda")
         self.logp_ref = torch.empty_like(self.logp)
         self.coef = torch.empty_like(self.logp)
@@ -382,9 +439,8 @@ class StreamedLoRAModel:
             self._prefetch(l)
         for l in range(nl):
             base = P.wait(l)
-            if adapters_on and self.keep is not None and l < self.keep.shape[0]:
-                L.soup_decoder_layer_fwd_keep(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.batch,
-                                              self.seq, self.ckpt[l + 1], adapters_on, self.keep[l], self.ws)
+            if adapters_on:
+                self._policy_fwd(l, self.views(base))
             else:
                 L.soup_decoder_layer_fwd(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.batch,
                                          self.seq, self.ckpt[l + 1], adapters_on, self.ws)
@@ -407,15 +463,24 @@ class StreamedLoRAModel:
             h_in = self.ckpt[0] if l == 0 else self.h_ref[(l - 1) % 2]
             L.soup_decoder_layer_fwd(w, self.lora_s[l], self.lcfg, h_in, self.batch, self.seq, self.h_ref[l % 2],
                                      False, self.ws)
-            if self.keep is not None and l < self.keep.shape[0]:
-                L.soup_decoder_layer_fwd_keep(w, self.lora_s[l], self.lcfg, self.ckpt[l], self.batch, self.seq,
-                                              self.ckpt[l + 1], True, self.keep[l], self.ws)
-            else:
-                L.soup_decoder_layer_fwd(w, self.lora_s[l], self.lcfg, self.ckpt[l], self.batch, self.seq,
-                                         self.ckpt[l + 1], True, self.ws)
+            self._policy_fwd(l, w)
             P.release(l)
             if l + N < nl:
                 self._prefetch(l + N)
+
+    def _policy_fwd(self, l, w):
+        """Layer l's forward pass with the adapters on, keeping what the keep
+        plan says for its backward."""
+        k = self.keep_plan[l]
+        if k == "saved":
+            L.soup_decoder_layer_fwd_save(w, self.lora_s[l], self.lcfg, self.ckpt[l], self.batch, self.seq,
+                                          self.ckpt[l + 1], True, self.saved[self.saved_row[l]], self.ws)
+        elif k == "qkv":
+            L.soup_decoder_layer_fwd_keep(w, self.lora_s[l], self.lcfg, self.ckpt[l], self.batch, self.seq,
+                                          self.ckpt[l + 1], True, self.keep[self.keep_row[l]], self.ws)
+        else:
+            L.soup_decoder_layer_fwd(w, self.lora_s[l], self.lcfg, self.ckpt[l], self.batch, self.seq,
+                                     self.ckpt[l + 1], True, self.ws)
 
     def _head(self, coef, logp, dh, h=None):
         P = self.plan
@@ -435,10 +500,15 @@ class StreamedLoRAModel:
             if self.capture_dh is not None:  # inspection hook for layer-by-layer checks
                 self.capture_dh[l + 1] = self.dh.clone()
             base = P.wait(l)
-            if self.keep is not None and l < self.keep.shape[0]:
+            k = self.keep_plan[l]
+            if k == "saved":
+                L.soup_decoder_layer_bwd_saved(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.dh,
+                                               self.batch, self.seq, self.dh, self.grads_s[l], 1,
+                                               self.saved[self.saved_row[l]], self.ws)
+            elif k == "qkv":
                 L.soup_decoder_layer_bwd_kept(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.dh,
-                                              self.batch, self.seq, self.dh, self.grads_s[l], 1, self.keep[l],
-                                              self.ws)
+                                              self.batch, self.seq, self.dh, self.grads_s[l], 1,
+                                              self.keep[self.keep_row[l]], self.ws)
             else:
                 L.soup_decoder_layer_bwd(self.views(base), self.lora_s[l], self.lcfg, self.ckpt[l], self.dh,
                                          self.batch, self.seq, self.dh, self.grads_s[l], 1, self.ws)

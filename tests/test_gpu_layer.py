@@ -156,3 +156,39 @@ def test_layer_holds_range(h_scale, norm_scale, dh_scale):
     for p in ss.PROJ_NAMES:
         assert_close(got[p][0], gref[p][0], f"dA_{p} {tag}")
         assert_close(got[p][1], gref[p][1], f"dB_{p} {tag}")
+
+
+@pytest.mark.parametrize("kind", ["nf4", "bf16"])
+def test_saved_layer_backward_is_bit_identical_to_kept(kind):
+    """fwd_save + bwd_saved (every intermediate kept, no forward recompute in
+    the backward) gives the bits of fwd_keep + bwd_kept (q|k|v kept, the rest
+    recomputed): h_out, dh_in and every LoRA gradient."""
+    shape = SMALL
+    B, S = 2, 130
+    T = B * S
+    dl = DevLayer(L, shape, seed=6, kind=kind)
+    h, dh = inputs(shape, B, S, seed=7)
+    ws = torch.empty(L.soup_decoder_layer_workspace(dl.cfg, B, S), dtype=torch.uint8, device="cuda")
+    hd = dev_bf16(h.reshape(T, -1))
+    dho = dev_f32(dh.reshape(T, -1))
+    keep = torch.empty(L.soup_decoder_layer_keep_bytes(dl.cfg, B, S) // 2, dtype=torch.float16, device="cuda")
+    out_k = torch.empty_like(hd)
+    dhi_k = torch.empty_like(dho)
+    L.soup_decoder_layer_fwd_keep(dl.W, dl.lora, dl.cfg, hd, B, S, out_k, 1, keep, ws)
+    L.soup_decoder_layer_bwd_kept(dl.W, dl.lora, dl.cfg, hd, dho, B, S, dhi_k, dl.grads, 1, keep, ws)
+    torch.cuda.synchronize()
+    g_k = {k: v.clone() for k, v in dl.grads_t.items()}
+    for v in dl.grads_t.values():
+        v.zero_()
+    saved = torch.empty(L.soup_decoder_layer_saved_bytes(dl.cfg, B, S), dtype=torch.uint8, device="cuda")
+    assert saved.numel() < ws.numel()
+    out_s = torch.empty_like(hd)
+    dhi_s = torch.empty_like(dho)
+    L.soup_decoder_layer_fwd_save(dl.W, dl.lora, dl.cfg, hd, B, S, out_s, 1, saved, ws)
+    ws.fill_(0xFF)  # nothing the backward reads may come from the workspace of the forward call
+    L.soup_decoder_layer_bwd_saved(dl.W, dl.lora, dl.cfg, hd, dho, B, S, dhi_s, dl.grads, 1, saved, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out_s, out_k)
+    assert torch.equal(dhi_s, dhi_k)
+    for k in g_k:
+        assert torch.equal(g_k[k], dl.grads_t[k]), k

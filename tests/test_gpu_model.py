@@ -43,9 +43,10 @@ def small_cfg(kind="nf4", tied=False, n_layers=3):
                          alpha=32.0, vocab=512, n_layers=n_layers, kind=kind, tied=tied)
 
 
-def build(cfg, B, S, n_buffers=2, seed=0, chunk=48, task="sft"):
+def build(cfg, B, S, n_buffers=2, seed=0, chunk=48, task="sft", recompute="auto"):
     w = NumpyWeights(cfg, seed)
-    m = M.StreamedLoRAModel(cfg, B, S, n_buffers=n_buffers, weights=w, head_chunk=chunk, task=task)
+    m = M.StreamedLoRAModel(cfg, B, S, n_buffers=n_buffers, weights=w, head_chunk=chunk, task=task,
+                            stream_recompute=recompute)
     return m, w
 
 
@@ -72,11 +73,15 @@ def check_layers_on_gpu_inputs(m, w, cfg):
             assert_close(got[p][1], grads[p][1], f"L{l} dB_{p}")
 
 
-@pytest.mark.parametrize("kind,tied", [("nf4", False), ("bf16", True)])
-def test_sft_step_matches_oracle(kind, tied):
+@pytest.mark.parametrize("kind,tied,recompute", [("nf4", False, "auto"), ("bf16", True, "auto"),
+                                                ("nf4", False, "recompute")])
+def test_sft_step_matches_oracle(kind, tied, recompute):
+    """recompute="auto" (uncapped): every layer keeps its activations (no
+    forward recompute in the backward); "recompute": none kept."""
     cfg = small_cfg(kind, tied)
     B, S = 2, 64
-    m, w = build(cfg, B, S)
+    m, w = build(cfg, B, S, recompute=recompute)
+    assert m.keep_plan == (["saved"] * cfg.n_layers if recompute == "auto" else [None] * cfg.n_layers)
     m.capture_dh = {}
     ids = ss.uniform_ids(1, "ids", (B, S), cfg.vocab)
     set_ids(m, ids)

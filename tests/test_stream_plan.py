@@ -108,3 +108,29 @@ def test_model_precheck_refuses_a_cap_below_the_lower_bound_before_any_work():
     assert 2 * 122_699_776 + 1_050_673_152 + 33 * 2048 * 4096 * 2 < lb < 4 << 30
     with pytest.raises(ValueError, match="device cap"):
         StreamedLoRAModel(cfg, 4, 512, n_buffers=2, device_cap_bytes=1 << 30)  # refused at once, no GPU needed
+
+
+def test_keep_plan_modes_and_the_cap():
+    from layer_streamed_qlora_b200.model import plan_keep
+    qkv, saved = 25_165_824, 455_000_000
+    arena, reserve = 1_296_000_000, 2_500_000_000
+    # no cap: auto keeps everything
+    assert plan_keep(32, qkv, saved, arena, reserve, 0) == ["saved"] * 32
+    assert plan_keep(32, qkv, saved, arena, reserve, 0, "recompute") == [None] * 32
+    assert plan_keep(32, qkv, saved, arena, reserve, 0, "keep") == ["saved"] * 32
+    # 4 GiB: q|k|v for the layers that fit, nothing saved
+    cap = 1 << 32
+    p = plan_keep(32, qkv, saved, arena, reserve, cap)
+    k = p.count("qkv")
+    assert 0 < k < 32 and p.count("saved") == 0 and p[:k] == ["qkv"] * k
+    assert arena + reserve + k * qkv <= cap < arena + reserve + (k + 1) * qkv
+    # room for every q|k|v and two upgrades: the first two layers are saved
+    cap2 = arena + reserve + 32 * qkv + 2 * (saved - qkv) + 1000
+    p2 = plan_keep(32, qkv, saved, arena, reserve, cap2)
+    assert p2[:2] == ["saved", "saved"] and p2[2:] == ["qkv"] * 30
+    assert arena + reserve + 2 * saved + 30 * qkv <= cap2
+    # keep refuses a cap that cannot hold every saved layer; unknown modes refused
+    with pytest.raises(ValueError):
+        plan_keep(32, qkv, saved, arena, reserve, cap, "keep")
+    with pytest.raises(ValueError):
+        plan_keep(32, qkv, saved, arena, reserve, cap, "sometimes")
