@@ -462,6 +462,9 @@ def main():
     ap.add_argument("--recompute", default="auto", choices=["auto", "recompute", "keep"],
                     help="stream_recompute: keep activations for the backward as the cap admits (auto), keep none, "
                          "or keep every layer's")
+    ap.add_argument("--no-prompt-dedup", action="store_true",
+                    help="preference workloads: lay out both sequences of a pair in full instead of storing and "
+                         "computing their shared prompt once")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--probe-gemm", action="store_true",
                     help="run each forward fused NF4 GEMM shape of one layer twice and exit (for an ncu capture)")
@@ -518,10 +521,14 @@ def main():
         shard_dir = args.shard_dir or tempfile.mkdtemp(prefix="soup_shards_")
     model = StreamedLoRAModel(cfg, B, S, n_buffers=w["buffers"], device_cap_bytes=cap, seed=0, task=w["task"],
                               stream_source=args.source, shard_dir=shard_dir, read_ahead=args.read_ahead,
-                              stream_recompute=args.recompute)
+                              stream_recompute=args.recompute,
+                              prompt_dedup=0 if (w["task"] == "sft" or args.no_prompt_dedup) else w["prompt"])
     t_build = time.time() - t_build
     g = torch.Generator().manual_seed(1000 + rank)
-    ids_host = torch.randint(0, cfg.vocab, (B, S), generator=g, dtype=torch.int32).pin_memory()
+    ids_host = torch.randint(0, cfg.vocab, (B, S), generator=g, dtype=torch.int32)
+    if w["task"] != "sft":  # preference pairs: rows 2p, 2p+1 share their prompt
+        ids_host[1::2, :w["prompt"]] = ids_host[0::2, :w["prompt"]]
+    ids_host = ids_host.pin_memory()
     loss_host = torch.zeros(1, dtype=torch.float32).pin_memory()
     model.set_ids(ids_host)
     torch.cuda.synchronize()
@@ -662,6 +669,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(bench_config(w, args.workload, world, sum(1 for k in model.keep_plan if k == "qkv"),
                                     sum(1 for k in model.keep_plan if k == "saved"), args.recompute),
+                       token_rows_per_step=model.T, prompt_dedup=model.prompt_dedup,
                        stream_source=args.source,
                        **({"read_ahead": args.read_ahead} if args.source == "disk" else {})),
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": ids_host.numel() * 4,

@@ -207,26 +207,36 @@ soup_status soup_lora_linear_bwd_noalloc(const soup_weight* W, const uint16_t* A
  * streaming works": the layer the stream feeds; the attention itself is the
  * Llama-3.1-8B layer's: causal within each sequence, kv head = q head /
  * (n_q_heads / n_kv_heads), scale 1/sqrt(128)).  head_dim is 128.
- * qkv: [batch * seq, ld] fp16 (ld >= (n_q + 2 n_kv) * 128, ld % 8 == 0, base
- * 16-byte aligned): q heads at columns [0, 128 n_q), k heads after them, then
- * v heads; tokens batch-major (sequence b is rows [b*seq, (b+1)*seq)); q and k
- * as they enter the dot products (after RoPE).
- * soup_attention_fwd: out [batch*seq, 128 n_q] bf16, out16 (may be NULL) the
- * same values in fp16, lse [n_q, batch*seq] fp32 = log2 of each row's softmax
- * denominator including the row maximum (log2 units).
- * soup_attention_bwd: from the forward's out16 and lse and dout [batch*seq,
- * 128 n_q] fp16, writes D [n_q, batch*seq] (rowsum(dout * out), a buffer the
- * caller provides) and dq, dk, dv (bf16) into dqkv at qkv's layout (dq
- * includes the 1/sqrt(128) scale; row stride ld), and the same values in fp32
- * into dqkv32 when it is not NULL.  Both run on the tensor cores (tcgen05,
- * accumulators in tensor memory), are deterministic, and are async on
- * `stream`.  Refusals: SOUP_ERR_SHAPE (bad sizes, n_q % n_kv != 0),
- * SOUP_ERR_ALIGN. */
+ * Token layout: `batch` sequences of `seq` tokens.  prefix_share <= 1: each
+ * sequence is its own `seq` rows (sequence b = rows [b*seq, (b+1)*seq)).
+ * prefix_share = G > 1: consecutive groups of G sequences share their first
+ * prefix_len tokens (a positive multiple of 128, < seq), stored once: a
+ * group's rows are [prefix | continuation of its sequence 0 | ... | of its
+ * sequence G-1], G * (seq - prefix_len) + prefix_len rows per group (the
+ * preference pairs of a DPO step with one prompt); the prefix's own queries
+ * belong to sequence 0 of the group; dk, dv of a prefix row sum the
+ * contributions of every sequence of the group.  T = number of rows.
+ * qkv: [T, ld] fp16 (ld >= (n_q + 2 n_kv) * 128, ld % 8 == 0, base 16-byte
+ * aligned): q heads at columns [0, 128 n_q), k heads after them, then v heads;
+ * q and k as they enter the dot products (after RoPE).
+ * soup_attention_fwd: out [T, 128 n_q] bf16, out16 (may be NULL) the same
+ * values in fp16, lse [n_q, T] fp32 = log2 of each row's softmax denominator
+ * including the row maximum (log2 units).
+ * soup_attention_bwd: from the forward's out16 and lse and dout [T, 128 n_q]
+ * fp16, writes D [n_q, T] (rowsum(dout * out), a buffer the caller provides)
+ * and dq, dk, dv (bf16) into dqkv at qkv's layout (dq includes the
+ * 1/sqrt(128) scale; row stride ld), and the same values in fp32 into dqkv32
+ * when it is not NULL.  Both run on the tensor cores (tcgen05, accumulators
+ * in tensor memory), are deterministic, and are async on `stream`.
+ * Refusals: SOUP_ERR_SHAPE (bad sizes, n_q % n_kv != 0, a prefix layout that
+ * does not fit), SOUP_ERR_ALIGN. */
 soup_status soup_attention_fwd(const uint16_t* qkv, int64_t ld, int64_t batch, int64_t seq, int32_t n_q_heads,
-                               int32_t n_kv_heads, uint16_t* out, uint16_t* out16, float* lse, void* stream);
+                               int32_t n_kv_heads, int32_t prefix_share, int64_t prefix_len, uint16_t* out,
+                               uint16_t* out16, float* lse, void* stream);
 soup_status soup_attention_bwd(const uint16_t* qkv, int64_t ld, int64_t batch, int64_t seq, int32_t n_q_heads,
-                               int32_t n_kv_heads, const uint16_t* out16, const uint16_t* dout, const float* lse,
-                               float* D, uint16_t* dqkv, float* dqkv32, void* stream);
+                               int32_t n_kv_heads, int32_t prefix_share, int64_t prefix_len, const uint16_t* out16,
+                               const uint16_t* dout, const float* lse, float* D, uint16_t* dqkv, float* dqkv32,
+                               void* stream);
 
 /* --------------------------------------------------------- decoder layer ---
  * One Llama-style decoder layer with LoRA on all seven projections (the unit
@@ -250,6 +260,16 @@ typedef struct soup_layer_cfg {
   float alpha;           /* LoRA scale s = alpha / r */
   float eps;             /* RMSNorm epsilon */
   float theta;           /* RoPE base */
+  /* Token layout of the layer calls' `batch` sequences of `seq` tokens.
+   * prefix_share <= 1: sequence b is token rows [b*seq, (b+1)*seq).
+   * prefix_share = G > 1: consecutive groups of G sequences share their
+   * first prefix_len tokens (a positive multiple of 128, < seq), stored once
+   * per group as [prefix | continuation of sequence 0 | ... | of sequence
+   * G-1]: a preference pair's prompt is computed once (G = 2).  Every
+   * activation buffer of the layer calls then holds
+   * batch / G * (prefix_len + G * (seq - prefix_len)) rows. */
+  int32_t prefix_share;
+  int32_t prefix_len;
 } soup_layer_cfg;
 
 /* The frozen base of one layer (all NF4 or all bf16), as it sits in a device
@@ -527,6 +547,20 @@ soup_status soup_head_fwd_bwd(const uint16_t* h, const uint16_t* w_final, const 
                               int64_t H, const int32_t* ids, int64_t batch, int64_t seq, float eps,
                               int32_t chunk, const float* coef, float* logp, float* dh, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/* Row gather: dst[i] = src[idx[i]] for i < n, rows of row_bytes bytes (a
+ * multiple of 4; device pointers).  Used to lay out a preference batch's
+ * tokens with the shared prompt stored once and to collect the rows the
+ * output head reads.  Async on `stream`. */
+soup_status soup_gather_rows(const void* src, int64_t row_bytes, const int32_t* idx, int64_t n, void* dst,
+                             void* stream);
+/* Row sums in a fixed order: dst[d] = sum over k in [start[d], start[d+1]) of
+ * src[src_idx[k]] (fp32 rows of H values; an empty range gives zeros), for
+ * d < n_dst.  Scatters the head's dL/dh back to the token rows, adding the
+ * contributions of both sequences of a pair at their shared prompt row
+ * (deterministic).  Async on `stream`. */
+soup_status soup_sum_rows_f32(const float* src, int64_t H, const int32_t* src_idx, const int32_t* start,
+                              int64_t n_dst, float* dst, void* stream);
 
 /* Mean next-token cross-entropy over batch*(seq-1) targets into *loss (a
  * device float; optional, then logp may be NULL); coef (optional) <-

@@ -37,7 +37,7 @@ class SoupWeight(ctypes.Structure):
 class LayerCfg(ctypes.Structure):
     _fields_ = [("hidden", c_int32), ("n_q_heads", c_int32), ("n_kv_heads", c_int32), ("head_dim", c_int32),
                 ("intermediate", c_int32), ("rank", c_int32), ("alpha", c_float), ("eps", c_float),
-                ("theta", c_float)]
+                ("theta", c_float), ("prefix_share", c_int32), ("prefix_len", c_int32)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -150,10 +150,12 @@ _SIGS = {
     "soup_stream_copy_stream": (c_void_p, [c_void_p]),
     "soup_stream_debug_timing_events": (c_int64, [c_void_p]),
     "soup_static_device_bytes": (c_size_t, []),
-    "soup_attention_fwd": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_int32, c_int32, c_void_p, c_void_p,
-                                     c_void_p, c_void_p]),
-    "soup_attention_bwd": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_int32, c_int32, c_void_p, c_void_p,
-                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "soup_gather_rows": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_void_p, c_void_p]),
+    "soup_sum_rows_f32": (c_int32, [c_void_p, c_int64, c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
+    "soup_attention_fwd": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_int32, c_int32, c_int32, c_int64,
+                                     c_void_p, c_void_p, c_void_p, c_void_p]),
+    "soup_attention_bwd": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_int32, c_int32, c_int32, c_int64,
+                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "soup_debug_gemm_bounded_wait": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64,
                                                c_int32, c_void_p]),
     "soup_stream_debug_fail_next_copy": (c_int32, [c_void_p]),
@@ -238,17 +240,35 @@ def soup_debug_gemm_bounded_wait(A, B, C, wait_limit_cycles=0, skip_producer_arr
         _p(A), _p(B), M, N, K, _p(C), int(wait_limit_cycles), 1 if skip_producer_arrivals else 0, _stream(stream)))
 
 
-def soup_attention_fwd(qkv, batch, seq, n_q, n_kv, out, out16, lse, stream=None):
-    """Causal GQA attention forward on the q|k|v rows (fp16 [batch*seq, ld])."""
-    _check("soup_attention_fwd", lib().soup_attention_fwd(_p(qkv), qkv.shape[1], batch, seq, n_q, n_kv, _p(out),
-                                                          _p(out16), _p(lse), _stream(stream)))
-
-
-def soup_attention_bwd(qkv, batch, seq, n_q, n_kv, out16, dout, lse, D, dqkv, dqkv32=None, stream=None):
-    """Backward of soup_attention_fwd: dq|dk|dv into dqkv (bf16, qkv's layout)."""
-    _check("soup_attention_bwd", lib().soup_attention_bwd(_p(qkv), qkv.shape[1], batch, seq, n_q, n_kv, _p(out16),
-                                                          _p(dout), _p(lse), _p(D), _p(dqkv), _p(dqkv32),
+def soup_attention_fwd(qkv, batch, seq, n_q, n_kv, out, out16, lse, prefix_share=1, prefix_len=0, stream=None):
+    """Causal GQA attention forward on the q|k|v rows (fp16 [T, ld]); groups of
+    prefix_share sequences may share a prefix of prefix_len tokens stored once."""
+    _check("soup_attention_fwd", lib().soup_attention_fwd(_p(qkv), qkv.shape[1], batch, seq, n_q, n_kv,
+                                                          prefix_share, prefix_len, _p(out), _p(out16), _p(lse),
                                                           _stream(stream)))
+
+
+def soup_attention_bwd(qkv, batch, seq, n_q, n_kv, out16, dout, lse, D, dqkv, dqkv32=None, prefix_share=1,
+                       prefix_len=0, stream=None):
+    """Backward of soup_attention_fwd: dq|dk|dv into dqkv (bf16, qkv's layout)."""
+    _check("soup_attention_bwd", lib().soup_attention_bwd(_p(qkv), qkv.shape[1], batch, seq, n_q, n_kv,
+                                                          prefix_share, prefix_len, _p(out16), _p(dout), _p(lse),
+                                                          _p(D), _p(dqkv), _p(dqkv32), _stream(stream)))
+
+
+def soup_gather_rows(src, idx, dst, stream=None):
+    """dst[i] = src[idx[i]] row by row (src, dst: device tensors of equal row size)."""
+    n = idx.numel()
+    rb = dst.numel() * dst.element_size() // max(1, n)
+    _check("soup_gather_rows", lib().soup_gather_rows(_p(src), rb, _p(idx), n, _p(dst), _stream(stream)))
+
+
+def soup_sum_rows_f32(src, src_idx, start, dst, stream=None):
+    """dst[d] = sum of src rows src_idx[start[d]:start[d+1]] (fp32 [*, H])."""
+    H = dst.shape[-1]
+    n_dst = dst.numel() // H
+    _check("soup_sum_rows_f32", lib().soup_sum_rows_f32(_p(src), H, _p(src_idx), _p(start), n_dst, _p(dst),
+                                                        _stream(stream)))
 
 
 def static_device_bytes() -> int:

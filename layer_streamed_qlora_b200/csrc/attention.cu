@@ -69,7 +69,12 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t saddr, uint32_t chunk) {
 }
 
 struct AttnArgs {
-  int S, Hq, Hkv, T;
+  int S, Hq, Hkv, T;  // S: tokens per sequence; T: token rows in memory
+  // Sequences come in groups of G that share their first Lp positions,
+  // stored once: a group's rows are [prefix | continuation of sequence 0 |
+  // ... | continuation of sequence G-1] (G = 1, Lp = 0: sequence v is rows
+  // [v S, (v + 1) S)).  Queries of the shared prefix belong to sequence 0.
+  int G, Lp;
   float scale_log2;  // log2(e) / sqrt(head_dim)
   float scale;       // 1 / sqrt(head_dim)
   // forward
@@ -89,6 +94,13 @@ struct AttnArgs {
   int* err;
   long long wait_limit;
 };
+
+// Physical token row of position t of sequence v.
+__device__ __forceinline__ int vrow(const AttnArgs& a, int v, int t) {
+  const int Lc = a.S - a.Lp;
+  const int g = v / a.G, i = v - g * a.G;
+  return g * (a.Lp + a.G * Lc) + (t < a.Lp ? t : a.Lp + i * Lc + (t - a.Lp));
+}
 
 #define ATTN_WAIT(bar, parity)                                                   \
   (ptx::mbar_wait_bounded((bar), (parity), abort_flag, a.wait_limit) ||          \
@@ -147,9 +159,9 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
   const int S = a.S;
   const int nqt = (S + 127) / 128;
   const int qb = nqt - 1 - (int)blockIdx.x;  // the longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.y, v = blockIdx.z;  // q head, sequence
+  if (v % a.G != 0 && qb * 128 < a.Lp) return;  // shared-prefix queries: sequence 0 of the group computes them
   const int g = h / (a.Hq / a.Hkv);
-  const int row0 = b * S;
   const int nkb = qb + 1;
   const int qcol = h * HD, kcol = (a.Hq + g) * HD, vcol = (a.Hq + a.Hkv + g) * HD;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -185,7 +197,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
   if (warp == 0) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
-      const int qrow = row0 + qb * 128;
+      const int qrow = vrow(a, v, qb * 128);
       ptx::mbar_arrive_expect_tx(q_full, 32768);
       ptx::tma_load_2d(sm + F_Q, &tm, q_full, qcol, qrow);
       ptx::tma_load_2d(sm + F_Q + 16384, &tm, q_full, qcol + 64, qrow);
@@ -194,7 +206,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
         const uint32_t ph = (j >> 1) & 1;
         if (!ATTN_WAIT(&kv_empty[s], ph ^ 1)) break;
         uint8_t* kv = sm + F_KV + s * 65536;
-        const int r = row0 + j * 128;
+        const int r = vrow(a, v, j * 128);
         ptx::mbar_arrive_expect_tx(&kv_full[s], 65536);
         ptx::tma_load_2d(kv, &tm, &kv_full[s], kcol, r);
         ptx::tma_load_2d(kv + 16384, &tm, &kv_full[s], kcol + 64, r);
@@ -347,7 +359,8 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
     if (qi < S) {
       const float l = lsum[row] + lsum[128 + row];
       const float inv = 1.f / l;
-      const size_t off = (size_t)(row0 + qi) * (a.Hq * HD) + h * HD + half * 64;
+      const int prow = vrow(a, v, qi);
+      const size_t off = (size_t)prow * (a.Hq * HD) + h * HD + half * 64;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         float f[8];
@@ -363,7 +376,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
           reinterpret_cast<float4*>(a.out32 + off)[2 * u + 1] = make_float4(f[4], f[5], f[6], f[7]);
         }
       }
-      if (half == 0) a.lse[(size_t)h * a.T + row0 + qi] = m + log2f(l);
+      if (half == 0) a.lse[(size_t)h * a.T + prow] = m + log2f(l);
     }
   }
   attn_teardown(abort_flag, warp, tmem);
@@ -401,15 +414,37 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int S = a.S;
-  const int kb = blockIdx.x;  // key block: the first ones have the most query tiles
-  const int g = blockIdx.y, b = blockIdx.z;
+  // physical key block pb of sequence group gq: a block of the shared prefix
+  // (every sequence of the group attends to it) or a continuation block of
+  // one sequence; the first blocks have the most query tiles
+  const int g = blockIdx.y, gq = blockIdx.z;
+  const int nb_pre = a.Lp / 128, nbc = (S - a.Lp + 127) / 128;
+  const int pb = blockIdx.x;
+  const bool prefix = pb < nb_pre;
+  const int own = prefix ? 0 : (pb - nb_pre) / nbc;            // sequence of the group owning the block
+  const int kb = prefix ? pb : nb_pre + (pb - nb_pre) % nbc;    // block index within the sequence
+  const int v0 = gq * a.G + own;
   const int grp = a.Hq / a.Hkv;
-  const int row0 = b * S;
   const int kcol = (a.Hq + g) * HD, vcol = (a.Hq + a.Hkv + g) * HD;
-  const int qt0 = 2 * kb;                 // first 64-query tile at or after the block
   const int nqt = (S + 63) / 64;
-  const int per_head = nqt - qt0;
-  const int n_it = per_head * grp;
+  // work items (sequence of the group, q head of the kv group, 64-query
+  // tile): the owner's tiles from the block on; for a prefix block also the
+  // other sequences' continuation tiles
+  const int per0 = nqt - 2 * kb, perR = nqt - a.Lp / 64;
+  const int seg0 = grp * per0;
+  const int n_it = seg0 + (prefix ? (a.G - 1) * grp * perR : 0);
+  auto item = [&](int it, int& vseq, int& hh, int& qt) {
+    if (it < seg0) {
+      vseq = v0;
+      hh = it / per0;
+      qt = 2 * kb + it % per0;
+    } else {
+      const int r = it - seg0, segR = grp * perR;
+      vseq = gq * a.G + 1 + r / segR;
+      hh = (r % segR) / perR;
+      qt = a.Lp / 64 + (r % segR) % perR;
+    }
+  };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -445,7 +480,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
     // ---------------------------------------------- TMA producer (whole warp)
     if (lane == 0) {
       ptx::mbar_arrive_expect_tx(kv_full, 65536);
-      const int r = row0 + kb * 128;
+      const int r = vrow(a, v0, kb * 128);
       ptx::tma_load_2d(sm + B1_K, &tm128, kv_full, kcol, r);
       ptx::tma_load_2d(sm + B1_K + 16384, &tm128, kv_full, kcol + 64, r);
       ptx::tma_load_2d(sm + B1_V, &tm128, kv_full, vcol, r);
@@ -458,25 +493,27 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
       if (lane == 0) okw = ATTN_WAIT(&empty[s], ph ^ 1) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
-      const int hh = it / per_head, qt = qt0 + it % per_head;
+      int vs, hh, qt;
+      item(it, vs, hh, qt);
       const int h = g * grp + hh;
       const int q0 = qt * 64;
+      const int qrow0 = vrow(a, vs, q0);
       // this tile's L and D (the softmax warps read them after the stage's full barrier)
       float* LD = reinterpret_cast<float*>(sm + B1_LD + s * 512);
 #pragma unroll
       for (int i = lane; i < 64; i += 32) {
         const bool in = q0 + i < S;
-        LD[i] = in ? a.L[(size_t)h * a.T + row0 + q0 + i] : 0.f;
-        LD[64 + i] = in ? a.D[(size_t)h * a.T + row0 + q0 + i] : 0.f;
+        LD[i] = in ? a.L[(size_t)h * a.T + qrow0 + i] : 0.f;
+        LD[64 + i] = in ? a.D[(size_t)h * a.T + qrow0 + i] : 0.f;
       }
       __syncwarp();
       if (lane == 0) {
         uint8_t* st = sm + B1_ST + s * B1_STAGE;
         ptx::mbar_arrive_expect_tx(&full[s], 32768);
-        ptx::tma_load_2d(st, &tm64, &full[s], h * HD, row0 + q0);            // Q
-        ptx::tma_load_2d(st + 8192, &tm64, &full[s], h * HD + 64, row0 + q0);
-        ptx::tma_load_2d(st + 16384, &tmdo64, &full[s], h * HD, row0 + q0);  // dO
-        ptx::tma_load_2d(st + 24576, &tmdo64, &full[s], h * HD + 64, row0 + q0);
+        ptx::tma_load_2d(st, &tm64, &full[s], h * HD, qrow0);            // Q
+        ptx::tma_load_2d(st + 8192, &tm64, &full[s], h * HD + 64, qrow0);
+        ptx::tma_load_2d(st + 16384, &tmdo64, &full[s], h * HD, qrow0);  // dO
+        ptx::tma_load_2d(st + 24576, &tmdo64, &full[s], h * HD + 64, qrow0);
       }
     }
   } else if (warp == 1) {
@@ -539,7 +576,9 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
     for (int it = 0; it < n_it; ++it) {
       const int s = it % B1_NS, bb = it & 1;
       const uint32_t pb = (it >> 1) & 1;
-      const int q0 = (qt0 + it % per_head) * 64;
+      int vs, hh, qt;
+      item(it, vs, hh, qt);
+      const int q0 = qt * 64;
       // the stage's full barrier also publishes the L and D values the
       // producer warp stored next to the tiles (it cannot move on to the
       // stage's next use before these warps release this iteration)
@@ -591,7 +630,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
       ptx::tc_fence_after();
       const float unscale = a.amax ? 1.f / grad_scale_from_amax(__uint_as_float(*a.amax)) : 1.f;
       const bool in = key < S;
-      const size_t r = (size_t)(row0 + key) * a.ld;
+      const size_t r = (size_t)(in ? vrow(a, v0, key) : 0) * a.ld;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
         const uint32_t col0 = which ? 384 : 256;
@@ -675,9 +714,9 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
   const int S = a.S;
   const int nqt = (S + 127) / 128;
   const int qb = nqt - 1 - (int)blockIdx.x;  // the longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.y, v = blockIdx.z;  // q head, sequence
+  if (v % a.G != 0 && qb * 128 < a.Lp) return;  // shared-prefix queries: sequence 0 of the group
   const int g = h / (a.Hq / a.Hkv);
-  const int row0 = b * S;
   const int kcol = (a.Hq + g) * HD, vcol = (a.Hq + a.Hkv + g) * HD;
   const int n_it = min(2 * qb + 2, (S + 63) / 64);  // 64-key blocks up to the diagonal and the sequence end
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -713,7 +752,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
 
   if (warp == 0) {
     if (lane == 0) {
-      const int qrow = row0 + qb * 128;
+      const int qrow = vrow(a, v, qb * 128);
       ptx::mbar_arrive_expect_tx(qo_full, 65536);
       ptx::tma_load_2d(sm + B2_Q, &tm128, qo_full, h * HD, qrow);
       ptx::tma_load_2d(sm + B2_Q + 16384, &tm128, qo_full, h * HD + 64, qrow);
@@ -724,7 +763,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
         const uint32_t ph = (j / B2_NS) & 1;
         if (!ATTN_WAIT(&empty[s], ph ^ 1)) break;
         uint8_t* st = sm + B2_ST + s * B2_STAGE;
-        const int r = row0 + j * 64;
+        const int r = vrow(a, v, j * 64);
         ptx::mbar_arrive_expect_tx(&full[s], 32768);
         ptx::tma_load_2d(st, &tm64, &full[s], kcol, r);
         ptx::tma_load_2d(st + 8192, &tm64, &full[s], kcol + 64, r);
@@ -782,8 +821,9 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const int qi = qb * 128 + row;
     const bool qin = qi < S;
-    const float Lr = qin ? a.L[(size_t)h * a.T + row0 + qi] : 0.f;
-    const float Dr = qin ? a.D[(size_t)h * a.T + row0 + qi] : 0.f;
+    const int prow = qin ? vrow(a, v, qi) : 0;
+    const float Lr = qin ? a.L[(size_t)h * a.T + prow] : 0.f;
+    const float Dr = qin ? a.D[(size_t)h * a.T + prow] : 0.f;
     const float sl2 = a.scale_log2;
     bool ok = true;
     for (int j = 0; j < n_it; ++j) {
@@ -830,7 +870,7 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
       ptx::tc_fence_after();
       const float unscale = a.amax ? 1.f / grad_scale_from_amax(__uint_as_float(*a.amax)) : 1.f;
       const float mul = a.scale * unscale;
-      const size_t r = (size_t)(row0 + qi) * a.ld + h * HD;
+      const size_t r = (size_t)prow * a.ld + h * HD;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t v0[32], v1[32];
@@ -908,28 +948,34 @@ soup_status attn_init() {
   return SOUP_OK;
 }
 
-soup_status attn_check(int ld, int Bsz, int S, int Hq, int Hkv) {
+soup_status attn_check(int ld, int Bsz, int S, int Hq, int Hkv, int G, int Lp) {
   SOUP_CHECK(Hkv > 0 && Hq % Hkv == 0 && S > 0 && Bsz > 0, SOUP_ERR_SHAPE, "attention: bad heads/shape");
   SOUP_CHECK(ld >= (Hq + 2 * Hkv) * HD && ld % 8 == 0, SOUP_ERR_SHAPE, "attention: row stride %d", ld);
   SOUP_CHECK((int64_t)Bsz * S < (1LL << 31), SOUP_ERR_SHAPE, "attention: too many tokens");
+  SOUP_CHECK(G >= 1 && Bsz % G == 0 && (G == 1 ? Lp == 0 : (Lp > 0 && Lp < S && Lp % 128 == 0)), SOUP_ERR_SHAPE,
+             "attention: prefix sharing needs groups of G sequences dividing the batch and a shared prefix that is "
+             "a positive multiple of 128 shorter than the sequence (G=%d, prefix %d, seq %d)", G, Lp, S);
   return SOUP_OK;
 }
+
+// Token rows of Bsz sequences of S tokens in groups of G sharing Lp.
+int attn_rows(int Bsz, int S, int G, int Lp) { return (Bsz / G) * (Lp + G * (S - Lp)); }
 
 }  // namespace
 
 soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, uint16_t* out, float* lse,
-                          cudaStream_t st, uint16_t* out16, float* out32) {
-  SOUP_TRY(attn_check(ld, Bsz, S, Hq, Hkv));
+                          cudaStream_t st, uint16_t* out16, float* out32, int G, int Lp) {
+  SOUP_TRY(attn_check(ld, Bsz, S, Hq, Hkv, G, Lp));
   SOUP_CHECK(soup_aligned(qkv, 16) && soup_aligned(out, 16) && (!out16 || soup_aligned(out16, 16)) &&
                  (!out32 || soup_aligned(out32, 16)) && lse,
              SOUP_ERR_ALIGN, "attention: alignment");
   SOUP_TRY(attn_init());
-  const int T = Bsz * S;
+  const int T = attn_rows(Bsz, S, G, Lp);
   CUtensorMap tm;
   SOUP_TRY(fp16_map(&tm, qkv, T, (Hq + 2 * Hkv) * HD, ld, 128, "q|k|v"));
   AttnArgs a;
   memset(&a, 0, sizeof(a));
-  a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.T = T;
+  a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.T = T; a.G = G; a.Lp = Lp;
   a.scale = 1.0f / sqrtf((float)HD);
   a.scale_log2 = 1.4426950408889634f * a.scale;
   a.out = out; a.lse = lse; a.out16 = out16; a.out32 = out32;
@@ -947,14 +993,15 @@ soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
 
 soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, const uint16_t* dout,
                           const float* lse, const float* D, uint16_t* dqkv, const float* rope_cos,
-                          const float* rope_sin, const unsigned int* amax, cudaStream_t st, float* dqkv32) {
-  SOUP_TRY(attn_check(ld, Bsz, S, Hq, Hkv));
+                          const float* rope_sin, const unsigned int* amax, cudaStream_t st, float* dqkv32, int G,
+                          int Lp) {
+  SOUP_TRY(attn_check(ld, Bsz, S, Hq, Hkv, G, Lp));
   SOUP_CHECK(soup_aligned(qkv, 16) && soup_aligned(dout, 16) && soup_aligned(dqkv, 16) &&
                  (!dqkv32 || soup_aligned(dqkv32, 16)) && lse && D,
              SOUP_ERR_ALIGN, "attention backward: alignment");
   SOUP_CHECK(!rope_cos == !rope_sin, SOUP_ERR_INVALID_ARG, "attention backward: RoPE tables go together");
   SOUP_TRY(attn_init());
-  const int T = Bsz * S;
+  const int T = attn_rows(Bsz, S, G, Lp);
   CUtensorMap tm128, tm64, tmdo64, tmdo128;
   SOUP_TRY(fp16_map(&tm128, qkv, T, (Hq + 2 * Hkv) * HD, ld, 128, "q|k|v"));
   SOUP_TRY(fp16_map(&tm64, qkv, T, (Hq + 2 * Hkv) * HD, ld, 64, "q|k|v"));
@@ -962,7 +1009,7 @@ soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
   SOUP_TRY(fp16_map(&tmdo128, dout, T, Hq * HD, Hq * HD, 128, "dO"));
   AttnArgs a;
   memset(&a, 0, sizeof(a));
-  a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.T = T;
+  a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.T = T; a.G = G; a.Lp = Lp;
   a.scale = 1.0f / sqrtf((float)HD);
   a.scale_log2 = 1.4426950408889634f * a.scale;
   a.L = lse; a.D = D; a.dqkv = dqkv; a.dqkv32 = dqkv32; a.ld = ld;
@@ -972,7 +1019,7 @@ soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
   a.wait_limit = 4000000000LL;
   const double fl = 2.5 * 4.0 * Bsz * Hq * (double)HD * ((double)S * (S + 1) / 2);
   profile_begin(st, GC_ATTN, fl, 0.0);
-  dim3 g1((S + 127) / 128, Hkv, Bsz);
+  dim3 g1(Lp / 128 + G * ((S - Lp + 127) / 128), Hkv, Bsz / G);
   attn_bwd_dkdv_tc<<<g1, 192, B1_SMEM, st>>>(tm128, tm64, tmdo64, a);
   SOUP_LAUNCH_CHECK();
   dim3 g2((S + 127) / 128, Hq, Bsz);
@@ -987,24 +1034,31 @@ soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
 using namespace soup;
 
 extern "C" soup_status soup_attention_fwd(const uint16_t* qkv, int64_t ld, int64_t batch, int64_t seq, int32_t n_q_heads,
-                                          int32_t n_kv_heads, uint16_t* out, uint16_t* out16, float* lse,
-                                          void* stream) {
+                                          int32_t n_kv_heads, int32_t prefix_share, int64_t prefix_len, uint16_t* out,
+                                          uint16_t* out16, float* lse, void* stream) {
   SOUP_CHECK(qkv && out && lse, SOUP_ERR_INVALID_ARG, "soup_attention_fwd: null pointer");
   SOUP_CHECK(batch > 0 && seq > 0 && batch * seq < (1LL << 31) && ld > 0 && ld < (1LL << 31), SOUP_ERR_SHAPE,
              "soup_attention_fwd: bad shape");
+  SOUP_CHECK(prefix_len >= 0 && prefix_len < seq, SOUP_ERR_SHAPE, "soup_attention_fwd: prefix length");
+  const int G = prefix_share > 1 ? prefix_share : 1;
   return attention_fwd(qkv, (int)ld, (int)batch, (int)seq, n_q_heads, n_kv_heads, out, lse,
-                       static_cast<cudaStream_t>(stream), out16, nullptr);
+                       static_cast<cudaStream_t>(stream), out16, nullptr, G, G > 1 ? (int)prefix_len : 0);
 }
 
 extern "C" soup_status soup_attention_bwd(const uint16_t* qkv, int64_t ld, int64_t batch, int64_t seq,
-                                          int32_t n_q_heads, int32_t n_kv_heads, const uint16_t* out16,
+                                          int32_t n_q_heads, int32_t n_kv_heads, int32_t prefix_share,
+                                          int64_t prefix_len, const uint16_t* out16,
                                           const uint16_t* dout, const float* lse, float* D, uint16_t* dqkv,
                                           float* dqkv32, void* stream) {
   SOUP_CHECK(qkv && out16 && dout && lse && D && dqkv, SOUP_ERR_INVALID_ARG, "soup_attention_bwd: null pointer");
   SOUP_CHECK(batch > 0 && seq > 0 && batch * seq < (1LL << 31) && ld > 0 && ld < (1LL << 31), SOUP_ERR_SHAPE,
              "soup_attention_bwd: bad shape");
+  SOUP_CHECK(prefix_len >= 0 && prefix_len < seq, SOUP_ERR_SHAPE, "soup_attention_bwd: prefix length");
+  const int G = prefix_share > 1 ? prefix_share : 1;
+  const int Lp = G > 1 ? (int)prefix_len : 0;
+  SOUP_TRY(attn_check((int)ld, (int)batch, (int)seq, n_q_heads, n_kv_heads, G, Lp));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  SOUP_TRY(attn_rowdot(dout, out16, (int)(batch * seq), n_q_heads, D, st));
+  SOUP_TRY(attn_rowdot(dout, out16, attn_rows((int)batch, (int)seq, G, Lp), n_q_heads, D, st));
   return attention_bwd(qkv, (int)ld, (int)batch, (int)seq, n_q_heads, n_kv_heads, dout, lse, D, dqkv, nullptr,
-                       nullptr, nullptr, st, dqkv32);
+                       nullptr, nullptr, st, dqkv32, G, Lp);
 }

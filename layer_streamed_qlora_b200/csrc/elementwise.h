@@ -56,8 +56,12 @@ soup_status lora_prep(const PrepJobs& jobs, cudaStream_t st);
 // T = Bsz * S tokens, batch-major.  out [T, Hq*128] bf16; lse [Hq, T] (log2
 // units); out16 (optional) [T, Hq*128] fp16 copy of the output, out32
 // (optional) an fp32 copy.
+// Sequences may come in groups of G sharing their first Lp tokens (Lp a
+// multiple of 128), stored once per group as [prefix | continuation of each
+// sequence]; T = Bsz / G * (Lp + G * (S - Lp)) token rows.
 soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, uint16_t* out,
-                          float* lse, cudaStream_t st, uint16_t* out16 = nullptr, float* out32 = nullptr);
+                          float* lse, cudaStream_t st, uint16_t* out16 = nullptr, float* out32 = nullptr, int G = 1,
+                          int Lp = 0);
 // Backward: dout [T, Hq*128] fp16; D [Hq, T] = rowsum(dout * out); dqkv bf16; writes dq, dk,
 // dv into dqkv [T, ld] at the same column layout as qkv.  q and k in qkv are
 // post-RoPE; when rope_cos/rope_sin ([S, 64]) are given, dq and dk are
@@ -68,6 +72,6 @@ soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
 soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, int Hkv, const uint16_t* dout,
                           const float* lse, const float* D, uint16_t* dqkv, const float* rope_cos,
                           const float* rope_sin, const unsigned int* amax, cudaStream_t st,
-                          float* dqkv32 = nullptr);
+                          float* dqkv32 = nullptr, int G = 1, int Lp = 0);
 
 }  // namespace soup

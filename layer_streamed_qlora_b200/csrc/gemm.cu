@@ -89,7 +89,7 @@ struct KArgs {
   long long ld_aux;
   int swiglu_I;
   int vec_ok;
-  int rope_cols, rope_S;
+  int rope_cols, rope_S, rope_Lp, rope_G;
   const float* rope_cos;
   const float* rope_sin;
   int* err;
@@ -269,7 +269,12 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
       ptx::tmem_ld_wait();
       const int n = n0 + ch * 16;
       if (!row_ok || n >= args.N) continue;
-      const int pos = row % args.rope_S;
+      int pos = row % args.rope_S;
+      if (args.rope_G > 1) {  // shared-prefix layout: position within the row's sequence
+        const int lc = args.rope_S - args.rope_Lp;
+        const int r = row % (args.rope_Lp + args.rope_G * lc);
+        pos = r < args.rope_Lp ? r : args.rope_Lp + (r - args.rope_Lp) % lc;
+      }
       const float* cs = args.rope_cos + (size_t)pos * 64 + (ch & 7) * 16;
       const float* sn = args.rope_sin + (size_t)pos * 64 + (ch & 7) * 16;
       float a[16], b[16];
@@ -1629,6 +1634,8 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
   ka.wait_limit = d.wait_limit > 0 ? d.wait_limit : 4000000000LL;
   ka.skip_producer = d.debug_skip_producer;
   ka.rope_cols = d.rope_cols; ka.rope_S = d.rope_S;
+  ka.rope_Lp = d.rope_group > 1 ? d.rope_prefix : 0;
+  ka.rope_G = d.rope_group > 1 ? d.rope_group : 1;
   ka.rope_cos = d.rope_cos; ka.rope_sin = d.rope_sin;
   if (d.rope_cols > 0) {
     SOUP_CHECK((d.out_kind == OUT_BF16 || d.out_kind == OUT_F16) && !d.resid && !d.resid_f32 && d.rope_cos &&

@@ -88,6 +88,11 @@ struct GemmDesc {
   int rope_cols = 0, rope_S = 0;
   const float* rope_cos = nullptr;
   const float* rope_sin = nullptr;
+  // Rows in groups of rope_group sequences sharing their first rope_prefix
+  // positions (stored once: [prefix | continuation of each sequence]): the
+  // position of a row is then its position within its sequence (rope_S =
+  // the sequence length).  rope_group <= 1: position = row % rope_S.
+  int rope_prefix = 0, rope_group = 1;
   int bn = 0;               // N tile (0 = pick)
   // NF4 GEMMs on CTA pairs: persistent tile loop with two accumulators (the
   // epilogue of one tile overlaps the next tile's main loop) or one tile

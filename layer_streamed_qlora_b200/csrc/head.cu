@@ -271,3 +271,73 @@ extern "C" soup_status soup_dpo_loss(const float* logp_policy, const float* logp
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
 }
+
+namespace soup {
+namespace {
+
+// One warp per output row: 16-byte words when the row and both bases allow,
+// else 4-byte words.
+__global__ void gather_rows_kernel(const uint8_t* __restrict__ src, int64_t row_bytes, const int32_t* __restrict__ idx,
+                                   int64_t n, uint8_t* __restrict__ dst, int vec16) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n;
+       r += (int64_t)gridDim.x * (blockDim.x >> 5)) {
+    const uint8_t* s = src + (int64_t)idx[r] * row_bytes;
+    uint8_t* d = dst + r * row_bytes;
+    if (vec16) {
+      for (int64_t w = lane; w < row_bytes / 16; w += 32)
+        reinterpret_cast<uint4*>(d)[w] = reinterpret_cast<const uint4*>(s)[w];
+    } else {
+      for (int64_t w = lane; w < row_bytes / 4; w += 32)
+        reinterpret_cast<uint32_t*>(d)[w] = reinterpret_cast<const uint32_t*>(s)[w];
+    }
+  }
+}
+
+// dst[d] = sum over k in [start[d], start[d+1]) of src[src_idx[k]], in k order.
+__global__ void sum_rows_kernel(const float* __restrict__ src, int64_t H, const int32_t* __restrict__ src_idx,
+                                const int32_t* __restrict__ start, int64_t n_dst, float* __restrict__ dst) {
+  for (int64_t d = blockIdx.x; d < n_dst; d += gridDim.x) {
+    const int k0 = start[d], k1 = start[d + 1];
+    for (int64_t c = threadIdx.x; c < H; c += blockDim.x) {
+      float acc = 0.f;
+      for (int k = k0; k < k1; ++k) acc += src[(int64_t)src_idx[k] * H + c];
+      dst[d * H + c] = acc;
+    }
+  }
+}
+
+}  // namespace
+}  // namespace soup
+
+extern "C" soup_status soup_gather_rows(const void* src, int64_t row_bytes, const int32_t* idx, int64_t n, void* dst,
+                                        void* stream) {
+  SOUP_CHECK(src && idx && dst, SOUP_ERR_INVALID_ARG, "soup_gather_rows: null pointer");
+  SOUP_CHECK(row_bytes > 0 && row_bytes % 4 == 0 && n >= 0, SOUP_ERR_SHAPE, "soup_gather_rows: rows of %lld bytes",
+             (long long)row_bytes);
+  SOUP_CHECK(soup_aligned(src, 4) && soup_aligned(dst, 4), SOUP_ERR_ALIGN, "soup_gather_rows: alignment");
+  if (n == 0) return SOUP_OK;
+  const int vec16 = row_bytes % 16 == 0 && soup_aligned(src, 16) && soup_aligned(dst, 16);
+  const unsigned blocks = (unsigned)std::min<int64_t>((n + 7) / 8, (int64_t)sm_count() * 8);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  profile_begin(st, GC_ELEM, 0.0, 2.0 * n * row_bytes + 4.0 * n);
+  gather_rows_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint8_t*>(src), row_bytes, idx, n,
+                                             static_cast<uint8_t*>(dst), vec16);
+  SOUP_LAUNCH_CHECK();
+  profile_end(st);
+  return SOUP_OK;
+}
+
+extern "C" soup_status soup_sum_rows_f32(const float* src, int64_t H, const int32_t* src_idx, const int32_t* start,
+                                         int64_t n_dst, float* dst, void* stream) {
+  SOUP_CHECK(src && src_idx && start && dst, SOUP_ERR_INVALID_ARG, "soup_sum_rows_f32: null pointer");
+  SOUP_CHECK(H > 0 && n_dst >= 0, SOUP_ERR_SHAPE, "soup_sum_rows_f32: bad shape");
+  if (n_dst == 0) return SOUP_OK;
+  const unsigned blocks = (unsigned)std::min<int64_t>(n_dst, (int64_t)sm_count() * 16);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  profile_begin(st, GC_ELEM, 0.0, 8.0 * n_dst * H);
+  sum_rows_kernel<<<blocks, 256, 0, st>>>(src, H, src_idx, start, n_dst, dst);
+  SOUP_LAUNCH_CHECK();
+  profile_end(st);
+  return SOUP_OK;
+}

@@ -27,6 +27,7 @@ namespace {
 
 struct Dims {
   int T, S, B, H, Hq, Hkv, d, I, r, qkv_w, o_in;
+  int G, Lp;  // groups of G sequences sharing Lp prefix tokens (G = 1: none); T = token rows
   int64_t ldT;
   float s;
 };
@@ -129,7 +130,15 @@ soup_status make_dims(const soup_layer_cfg* c, int64_t batch, int64_t seq, Dims*
              "decoder layer: intermediate must be a multiple of 128");
   SOUP_CHECK(batch >= 1 && seq >= 1 && batch * seq < (1 << 24), SOUP_ERR_SHAPE, "decoder layer: batch/seq");
   SOUP_CHECK(c->eps >= 0.f && c->theta > 0.f, SOUP_ERR_INVALID_ARG, "decoder layer: eps/theta");
-  m->B = (int)batch; m->S = (int)seq; m->T = (int)(batch * seq);
+  const int G = c->prefix_share > 1 ? c->prefix_share : 1;
+  const int Lp = G > 1 ? c->prefix_len : 0;
+  SOUP_CHECK(G == 1 || (batch % G == 0 && Lp > 0 && Lp < seq && Lp % 128 == 0), SOUP_ERR_SHAPE,
+             "decoder layer: prefix sharing needs groups of %d sequences dividing the batch (%lld) and a shared "
+             "prefix that is a positive multiple of 128 shorter than the sequence (%d of %lld)", G, (long long)batch,
+             Lp, (long long)seq);
+  m->G = G; m->Lp = Lp;
+  m->B = (int)batch; m->S = (int)seq;
+  m->T = (int)((batch / G) * (Lp + G * (seq - Lp)));
   m->H = c->hidden; m->Hq = c->n_q_heads; m->Hkv = c->n_kv_heads; m->d = c->head_dim;
   m->I = c->intermediate; m->r = c->rank;
   m->qkv_w = (m->Hq + 2 * m->Hkv) * m->d;
@@ -167,6 +176,7 @@ struct ProjOpts {
   int rope_cols = 0, rope_S = 0;
   const float* rope_cos = nullptr;
   const float* rope_sin = nullptr;
+  int rope_prefix = 0, rope_group = 1;
   int swiglu_I = 0;          // > 0: paired gate|up tiles with the SwiGLU epilogue
   uint16_t* aux16 = nullptr; // SwiGLU: fp16 g | u output (may be null)
   const uint16_t* x_lo = nullptr;  // dual-A: bf16 rounding residual of x
@@ -190,6 +200,7 @@ soup_status proj_fwd(const soup_weight* W, const uint16_t* x, int T, const uint1
   g.out_kind = o.out_kind; g.out = out; g.ldo = W->out_features;
   g.resid = o.resid; g.resid_f32 = o.resid_f32; g.ldr = W->out_features;
   g.rope_cols = o.rope_cols; g.rope_S = o.rope_S; g.rope_cos = o.rope_cos; g.rope_sin = o.rope_sin;
+  g.rope_prefix = o.rope_prefix; g.rope_group = o.rope_group;
   if (o.swiglu_I > 0) {
     g.pair_off = o.swiglu_I;
     g.nseg = 1;
@@ -389,6 +400,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     o.out_kind = OUT_F16;  // q, k, v feed only the attention kernels
     o.rope_cols = (m.Hq + m.Hkv) * m.d;
     o.rope_S = m.S; o.rope_cos = PF(cosb); o.rope_sin = PF(sinb);
+    o.rope_prefix = m.Lp; o.rope_group = m.G;
     // for the backward, q/k/v from an fp32-accurate x1 (hi + lo parts): the
     // attention backward amplifies the bf16 rounding of x1 into the q/k/v
     // adapter gradients
@@ -399,7 +411,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
   }
   const uint16_t* qkvp = kept ? kept : (keep ? keep : P(qkv));
   SOUP_TRY(attention_fwd(qkvp, m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(attn), PF(lse), st,
-                         save ? P(attn16) : nullptr, on ? PF(attn32) : nullptr));
+                         save ? P(attn16) : nullptr, on ? PF(attn32) : nullptr, m.G, m.Lp));
   if (on) {
     SOUP_TRY(lora_down_tf32(PF(attn32), T, m.o_in, PF(Ao32), r, m.s, P(u_o), PF(uo32), m.ldT, st, SW));
   }
@@ -611,7 +623,7 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
   SOUP_TRY(attn_rowdot(P(d_attn), P(attn16), T, m.Hq, PF(D), st));
   // dq and dk leave the attention backward already rotated back (inverse RoPE in its epilogues)
   SOUP_TRY(attention_bwd(qkvp, m.qkv_w, m.B, m.S, m.Hq, m.Hkv, P(d_attn), PF(lse), PF(D), P(d_qkv), PF(cosb),
-                         PF(sinb), gamax, st, on ? PF(dqkv32) : nullptr));
+                         PF(sinb), gamax, st, on ? PF(dqkv32) : nullptr, m.G, m.Lp));
   const int seg_n[3] = {m.Hq * m.d, m.Hkv * m.d, m.Hkv * m.d};
   const int seg_c[3] = {0, m.Hq * m.d, (m.Hq + m.Hkv) * m.d};
   if (on)  // g_q | g_k | g_v in one GEMM (block-diagonal B_qkv^T)
@@ -643,8 +655,12 @@ extern "C" size_t soup_layer_blob_bytes(const soup_layer_cfg* cfg, int32_t kind)
 
 extern "C" soup_status soup_layer_blob_views(const soup_layer_cfg* cfg, int32_t kind, const void* base,
                                              soup_layer_weights* out) {
+  SOUP_CHECK(cfg, SOUP_ERR_INVALID_ARG, "soup_layer_blob_views: null cfg");
+  soup_layer_cfg one = *cfg;  // the blob does not depend on the token layout
+  one.prefix_share = 0;
+  one.prefix_len = 0;
   Dims m;
-  SOUP_TRY(make_dims(cfg, 1, 1, &m));
+  SOUP_TRY(make_dims(&one, 1, 1, &m));
   SOUP_CHECK(out, SOUP_ERR_INVALID_ARG, "soup_layer_blob_views: null out");
   SOUP_CHECK(kind == SOUP_WEIGHT_NF4 || kind == SOUP_WEIGHT_BF16, SOUP_ERR_INVALID_ARG, "bad weight kind %d", kind);
   SOUP_CHECK(soup_aligned(base, 256), SOUP_ERR_ALIGN, "soup_layer_blob_views: base not 256-byte aligned");

@@ -58,9 +58,12 @@ class ModelConfig:
     def o_in(self):
         return self.n_q_heads * self.head_dim
 
-    def layer_cfg(self) -> L.LayerCfg:
+    def layer_cfg(self, prompt_share: int = 0) -> L.LayerCfg:
+        """The layer calls' configuration; prompt_share > 0: pairs of
+        sequences share their first prompt_share tokens, stored once."""
         return L.LayerCfg(self.hidden, self.n_q_heads, self.n_kv_heads, self.head_dim, self.intermediate,
-                          self.rank, float(self.alpha), float(self.eps), float(self.theta))
+                          self.rank, float(self.alpha), float(self.eps), float(self.theta),
+                          2 if prompt_share else 0, int(prompt_share))
 
     @property
     def weight_kind(self):
@@ -126,27 +129,77 @@ class AdamW:
     weight_decay: float = 0.0
 
 
-def device_bytes_lower_bound(cfg: ModelConfig, batch: int, seq: int, n_buffers: int, head_chunk: int) -> int:
+def token_rows(batch: int, seq: int, prompt_share: int = 0) -> int:
+    """Token rows of `batch` sequences of `seq` tokens; with prompt_share,
+    pairs share their first prompt_share tokens, stored once."""
+    if not prompt_share:
+        return batch * seq
+    return (batch // 2) * (prompt_share + 2 * (seq - prompt_share))
+
+
+def prompt_dedup_indices(batch: int, seq: int, prompt: int):
+    """Index arrays (int32 numpy) of the shared-prompt layout of a preference
+    batch (rows 2p chosen, 2p+1 rejected, sharing their first `prompt`
+    tokens; the pair's token rows are [prompt | chosen continuation |
+    rejected continuation]):
+      phys      [token rows]: each token row's position in the flat ids [batch * seq]
+                (prompt rows: the chosen sequence's);
+      head_rows [batch * (seq - prompt + 1)]: for each sequence v and
+                j = 0 .. seq - prompt, the token row of position prompt - 1 + j
+                (the positions whose next-token log-probs cover the continuation);
+      head_ids  [same]: the flat ids position of that (v, position);
+      start, src: for each token row d, the head rows reading it are
+                src[start[d]:start[d + 1]] (in increasing order)."""
+    import numpy as np
+    Lp, Lc = prompt, seq - prompt
+    span = Lp + 2 * Lc
+
+    def row(v, t):
+        p, i = divmod(v, 2)
+        return p * span + (t if t < Lp else Lp + i * Lc + (t - Lp))
+
+    T = (batch // 2) * span
+    phys = np.empty(T, np.int32)
+    for v in range(batch):
+        for t in range(seq):
+            if v % 2 == 0 or t >= Lp:
+                phys[row(v, t)] = v * seq + t
+    hl = Lc + 1
+    head_rows = np.array([row(v, Lp - 1 + j) for v in range(batch) for j in range(hl)], np.int32)
+    head_ids = np.array([v * seq + Lp - 1 + j for v in range(batch) for j in range(hl)], np.int32)
+    readers = [[] for _ in range(T)]
+    for h, d in enumerate(head_rows):
+        readers[d].append(h)
+    start = np.zeros(T + 1, np.int32)
+    start[1:] = np.cumsum([len(r) for r in readers])
+    src = np.array([h for r in readers for h in r], np.int32)
+    return phys, head_rows, head_ids, start, src
+
+
+def device_bytes_lower_bound(cfg: ModelConfig, batch: int, seq: int, n_buffers: int, head_chunk: int,
+                             prompt_share: int = 0) -> int:
     """Device bytes a streamed model needs at least, from the library's host
     size queries: the slot arena (n_buffers layer blobs + the vocab slot),
-    the layer checkpoints [L+1, T, H] bf16, the layer and head workspaces,
-    and the library's module-static device arrays."""
-    lcfg = cfg.layer_cfg()
+    the layer checkpoints [L+1, T, H] bf16, the layer workspace (which the
+    head's shares when it is the larger), and the library's module-static
+    device arrays."""
+    lcfg = cfg.layer_cfg(prompt_share)
     blob = L.soup_layer_blob_bytes(lcfg, cfg.weight_kind)
     vocab = (cfg.vocab * cfg.hidden * 2 + 255) // 256 * 256
-    T = batch * seq
+    T = token_rows(batch, seq, prompt_share)
+    head_seq = seq - prompt_share + 1 if prompt_share else seq
     return (n_buffers * blob + vocab + (cfg.n_layers + 1) * T * cfg.hidden * 2 +
-            L.soup_decoder_layer_workspace(lcfg, batch, seq) +
-            L.soup_head_workspace(cfg.vocab, cfg.hidden, batch, seq, head_chunk) + L.static_device_bytes())
+            max(L.soup_decoder_layer_workspace(lcfg, batch, seq),
+                L.soup_head_workspace(cfg.vocab, cfg.hidden, batch, head_seq, head_chunk)) + L.static_device_bytes())
 
 
-def precheck_device_bytes(cfg, batch, seq, n_buffers, head_chunk, cap):
+def precheck_device_bytes(cfg, batch, seq, n_buffers, head_chunk, cap, prompt_share=0):
     """Refuses, before any shard is built or any device memory is taken, a
     model whose lower-bound device need exceeds the cap (the stream plan makes
     the exact check once the model's own allocations are known)."""
     if not cap:
         return
-    need = device_bytes_lower_bound(cfg, batch, seq, n_buffers, head_chunk)
+    need = device_bytes_lower_bound(cfg, batch, seq, n_buffers, head_chunk, prompt_share)
     if need > cap:
         raise ValueError(f"the streamed model needs at least {need} device bytes ({n_buffers} slots, the vocab slot, "
                          f"checkpoints and workspaces) > device cap {cap}")
@@ -212,7 +265,7 @@ class StreamedLoRAModel:
     def __init__(self, cfg: ModelConfig, batch: int, seq: int, n_buffers: int = 2, device_cap_bytes: int = 0,
                  head_chunk: int = 256, weights=None, seed: int = 0, adamw: AdamW | None = None,
                  task: str = "sft", stream_source: str = "ram", shard_dir: str | None = None,
-                 read_ahead: int = 2, io_threads: int = 4, stream_recompute: str = "auto"):
+                 read_ahead: int = 2, io_threads: int = 4, stream_recompute: str = "auto", prompt_dedup: int = 0):
         self.cfg, self.batch, self.seq, self.n_buffers = cfg, batch, seq, n_buffers
         if stream_source not in ("ram", "disk"):
             raise ValueError(f"stream_source must be 'ram' or 'disk', not {stream_source!r}")
@@ -227,10 +280,22 @@ class StreamedLoRAModel:
         if task not in ("sft", "dpo", "simpo", "orpo"):
             raise ValueError(f"task must be 'sft', 'dpo', 'simpo' or 'orpo', not {task!r}")
         self.task = task
-        self.T = batch * seq
+        # preference pairs with one prompt: the prompt's tokens are stored and
+        # computed once per pair (prompt_dedup = the shared prompt length)
+        if prompt_dedup:
+            if task not in ("dpo", "simpo", "orpo"):
+                raise ValueError("prompt_dedup applies to the preference tasks (pairs sharing a prompt)")
+            if batch % 2 or not (0 < prompt_dedup < seq) or prompt_dedup % 128:
+                raise ValueError(f"prompt_dedup needs an even batch and a shared prompt that is a positive multiple "
+                                 f"of 128 shorter than the sequence (batch {batch}, prompt {prompt_dedup}, seq {seq})")
+        self.prompt_dedup = int(prompt_dedup)
+        self.T = token_rows(batch, seq, self.prompt_dedup)
+        # the output head reads, per sequence, head_seq consecutive positions
+        # (with a shared prompt: the last prompt position and the continuation)
+        self.head_seq = seq - self.prompt_dedup + 1 if self.prompt_dedup else seq
         self.head_chunk = head_chunk
-        self.lcfg = cfg.layer_cfg()
-        precheck_device_bytes(cfg, batch, seq, n_buffers, head_chunk, device_cap_bytes)
+        self.lcfg = cfg.layer_cfg(self.prompt_dedup)
+        precheck_device_bytes(cfg, batch, seq, n_buffers, head_chunk, device_cap_bytes, self.prompt_dedup)
         weights = weights or SyntheticWeights(cfg, seed)
         # the model's resident tensors first, the shard build's temporaries
         # after them: freed temporaries then leave whole cached segments that
@@ -379,17 +444,28 @@ class StreamedLoRAModel:
                               device="cuda")
         # the output head runs between the layer passes, never during a layer
         # call: its workspace shares the layer workspace's memory
-        head_bytes = L.soup_head_workspace(cfg.vocab, cfg.hidden, self.batch, self.seq, self.head_chunk)
+        head_bytes = L.soup_head_workspace(cfg.vocab, cfg.hidden, self.batch, self.head_seq, self.head_chunk)
         if head_bytes <= self.ws.numel():
             self.head_ws = self.ws[:head_bytes]
         else:
             self.head_ws = torch.empty(head_bytes, dtype=torch.uint8, device="cuda")
-        self.logp = torch.empty((self.batch, self.seq - 1), dtype=torch.float32, device="cuda")
+        self.logp = torch.empty((self.batch, self.head_seq - 1), dtype=torch.float32, device="cuda")
         self.logp_ref = torch.empty_like(self.logp)
         self.coef = torch.empty_like(self.logp)
         self.loss = torch.zeros(1, dtype=torch.float32, device="cuda")
         self.seq_sums = torch.zeros(4 * max(1, self.batch // 2), dtype=torch.float32, device="cuda")
         self.ids = torch.empty((self.batch, self.seq), dtype=torch.int32, device="cuda")
+        self.ids_tok = self.ids  # ids of the token rows (the shared-prompt layout: gathered)
+        self.ids_head = self.ids  # targets of the rows the head reads
+        if self.prompt_dedup:
+            phys, hrows, hids, start, src = prompt_dedup_indices(self.batch, self.seq, self.prompt_dedup)
+            dev = lambda a: torch.from_numpy(a).to("cuda")
+            self.dd_phys, self.dd_head_rows, self.dd_head_ids = dev(phys), dev(hrows), dev(hids)
+            self.dd_start, self.dd_src = dev(start), dev(src)
+            self.ids_tok = torch.empty(self.T, dtype=torch.int32, device="cuda")
+            self.ids_head = torch.empty((self.batch, self.head_seq), dtype=torch.int32, device="cuda")
+            self.h_head = torch.empty((self.batch * self.head_seq, cfg.hidden), dtype=torch.bfloat16, device="cuda")
+            self.dh_head = torch.empty((self.batch * self.head_seq, cfg.hidden), dtype=torch.float32, device="cuda")
         # DPO: running hidden state of the adapters-off reference pass, which
         # shares each layer visit with the policy's forward pass (ping-pong)
         self.h_ref = None
@@ -417,7 +493,7 @@ class StreamedLoRAModel:
         from the pinned host matrix (mapped into the device address space), so
         only the batch's rows cross the host link, not the whole vocab matrix;
         the vocab slot is left to the lm_head."""
-        L.soup_embed(self.host_embed.data_ptr(), self.cfg.vocab, self.cfg.hidden, self.ids, self.T, self.ckpt[0])
+        L.soup_embed(self.host_embed.data_ptr(), self.cfg.vocab, self.cfg.hidden, self.ids_tok, self.T, self.ckpt[0])
 
     def _prefetch(self, l):
         """Brings layer l into a slot: from its pinned host blob, or with the
@@ -487,9 +563,20 @@ class StreamedLoRAModel:
         P.prefetch(self.head_item)
         E = P.wait(self.head_item)
         h = self.ckpt[self.cfg.n_layers] if h is None else h
-        L.soup_head_fwd_bwd(h, self.final_norm, E, self.cfg.vocab, self.cfg.hidden,
-                            self.ids, self.batch, self.seq, self.cfg.eps, self.head_chunk, coef, logp, dh,
-                            self.head_ws)
+        if self.prompt_dedup:
+            # the rows whose log-probs cover each sequence's continuation (the
+            # shared last prompt row read once per sequence of the pair), and
+            # their dL/dh summed back onto the token rows in a fixed order
+            L.soup_gather_rows(h, self.dd_head_rows, self.h_head)
+            L.soup_head_fwd_bwd(self.h_head, self.final_norm, E, self.cfg.vocab, self.cfg.hidden, self.ids_head,
+                                self.batch, self.head_seq, self.cfg.eps, self.head_chunk, coef, logp,
+                                None if dh is None else self.dh_head, self.head_ws)
+            if dh is not None:
+                L.soup_sum_rows_f32(self.dh_head, self.dd_src, self.dd_start, dh)
+        else:
+            L.soup_head_fwd_bwd(h, self.final_norm, E, self.cfg.vocab, self.cfg.hidden,
+                                self.ids, self.batch, self.seq, self.cfg.eps, self.head_chunk, coef, logp, dh,
+                                self.head_ws)
         P.release(self.head_item)
 
     def _backward_layers(self):
@@ -522,6 +609,9 @@ class StreamedLoRAModel:
     def set_ids(self, ids_host):
         """Copies a step's token ids [batch, seq] (pinned int32 host tensor) to the device."""
         self.ids.copy_(ids_host, non_blocking=True)
+        if self.prompt_dedup:  # token rows of the shared-prompt layout, and the head's targets
+            L.soup_gather_rows(self.ids, self.dd_phys, self.ids_tok)
+            L.soup_gather_rows(self.ids, self.dd_head_ids, self.ids_head)
 
     def sft_step(self):
         """One SFT step on self.ids: next-token CE; leaves LoRA grads in self.grads
@@ -551,11 +641,21 @@ class StreamedLoRAModel:
             self._head(None, self.logp_ref, None)
             self._forward_layers(True)
         self._head(None, self.logp, None)
-        L.soup_dpo_loss(self.logp, self.logp_ref, pairs, self.seq, prompt_len, beta, self.loss, self.seq_sums,
-                        self.coef)
+        hs, pl = self._loss_layout(prompt_len)
+        L.soup_dpo_loss(self.logp, self.logp_ref, pairs, hs, pl, beta, self.loss, self.seq_sums, self.coef)
         self._head(self.coef, self.logp, self.dh)
         self._backward_layers()
         return self.loss
+
+    def _loss_layout(self, prompt_len):
+        """(sequence length, prompt length) of the head's log-probs as the
+        preference losses see them: the whole sequences, or with a shared
+        prompt stored once only the rows that predict the continuation."""
+        if not self.prompt_dedup:
+            return self.seq, prompt_len
+        if prompt_len != self.prompt_dedup:
+            raise ValueError(f"this model shares a {self.prompt_dedup}-token prompt, not {prompt_len}")
+        return self.head_seq, 1
 
     def _preference_step(self, loss_fn):
         """Reference-free preference step: one policy pass (two layer reads
@@ -572,13 +672,15 @@ class StreamedLoRAModel:
     def simpo_step(self, prompt_len: int, beta: float = 2.0, gamma: float = 1.0):
         """One SimPO step on self.ids (rows 2p chosen, 2p+1 rejected)."""
         pairs = self.batch // 2
-        return self._preference_step(lambda: L.soup_simpo_loss(self.logp, pairs, self.seq, prompt_len, beta, gamma,
+        hs, pl = self._loss_layout(prompt_len)
+        return self._preference_step(lambda: L.soup_simpo_loss(self.logp, pairs, hs, pl, beta, gamma,
                                                                self.loss, self.seq_sums, self.coef))
 
     def orpo_step(self, prompt_len: int, lam: float = 0.1):
         """One ORPO step on self.ids (rows 2p chosen, 2p+1 rejected)."""
         pairs = self.batch // 2
-        return self._preference_step(lambda: L.soup_orpo_loss(self.logp, pairs, self.seq, prompt_len, lam,
+        hs, pl = self._loss_layout(prompt_len)
+        return self._preference_step(lambda: L.soup_orpo_loss(self.logp, pairs, hs, pl, lam,
                                                               self.loss, self.seq_sums, self.coef))
 
     def optimizer_step(self, grad_scale: float = 1.0):

@@ -112,3 +112,56 @@ def test_attention_backward_is_deterministic(L):
     L.soup_attention_bwd(qkv_d, 2, 300, 8, 2, out16, dout_d, lse, D, dqkv)
     torch.cuda.synchronize()
     assert torch.equal(first, dqkv)
+
+
+def test_attention_with_a_shared_prefix_matches_oracle(L):
+    """Two groups of G = 2 sequences (preference pairs) sharing a 256-token
+    prefix stored once, with 100-token continuations (ragged): each
+    sequence's output equals the oracle's attention over that sequence
+    expanded (prefix + its own continuation); the prefix's gradients sum the
+    contributions of both sequences of its group (its queries belong to the
+    group's first sequence, whose output the prefix rows hold)."""
+    G, P, Lp, Lc, Hq, Hkv = 2, 2, 256, 100, 8, 2
+    S = Lp + Lc
+    span = Lp + G * Lc
+    T = P * span
+    ld = (Hq + 2 * Hkv) * HD
+    qkv = f16_values(ss.normal_f32(31, "attn.share.qkv", (T, ld)))
+    dout = f16_values(ss.normal_f32(31, "attn.share.dout", (T, Hq * HD)))
+    qkv_d = torch.from_numpy(qkv.astype(np.float16)).cuda()
+    dout_d = torch.from_numpy(dout.astype(np.float16)).cuda()
+    out = torch.empty((T, Hq * HD), dtype=torch.bfloat16, device="cuda")
+    out16 = torch.empty((T, Hq * HD), dtype=torch.float16, device="cuda")
+    lse = torch.empty((Hq, T), dtype=torch.float32, device="cuda")
+    L.soup_attention_fwd(qkv_d, P * G, S, Hq, Hkv, out, out16, lse, prefix_share=G, prefix_len=Lp)
+    D = torch.empty((Hq, T), dtype=torch.float32, device="cuda")
+    dqkv32 = torch.zeros((T, ld), dtype=torch.float32, device="cuda")
+    dqkv = torch.zeros((T, ld), dtype=torch.bfloat16, device="cuda")
+    L.soup_attention_bwd(qkv_d, P * G, S, Hq, Hkv, out16, dout_d, lse, D, dqkv, dqkv32, prefix_share=G, prefix_len=Lp)
+    torch.cuda.synchronize()
+    got_out, got_d = host(out), host(dqkv32)
+    ref_out = np.zeros((T, Hq * HD))
+    ref_d = np.zeros((T, ld))
+    for p in range(P):
+        base = p * span
+        for i in range(G):
+            rows = np.concatenate([np.arange(base, base + Lp), np.arange(base + Lp + i * Lc, base + Lp + (i + 1) * Lc)])
+            x = qkv[rows]
+            q = x[:, :Hq * HD].reshape(1, S, Hq, HD)
+            k = x[:, Hq * HD:(Hq + Hkv) * HD].reshape(1, S, Hkv, HD)
+            v = x[:, (Hq + Hkv) * HD:(Hq + 2 * Hkv) * HD].reshape(1, S, Hkv, HD)
+            o, probs = OL.attention_fwd(q, k, v)
+            do = dout[rows].copy()
+            if i > 0:
+                do[:Lp] = 0.0  # the prefix's outputs are the first sequence's
+            dq, dk, dv = OL.attention_bwd(q, k, v, probs, do.reshape(1, S, Hq, HD))
+            own = rows if i == 0 else rows[Lp:]
+            sl = slice(0, S) if i == 0 else slice(Lp, S)
+            ref_out[own] = o.reshape(S, -1)[sl]
+            grads = np.concatenate([dq.reshape(S, -1), dk.reshape(S, -1), dv.reshape(S, -1)], axis=1)
+            ref_d[rows] += grads  # prefix rows: dk, dv from every sequence (dq of a later one is 0)
+    assert_close(got_out, ref_out, "out (shared prefix)")
+    qo, ko = Hq * HD, (Hq + Hkv) * HD
+    assert_close(got_d[:, :qo], ref_d[:, :qo], "dq (shared prefix)")
+    assert_close(got_d[:, qo:ko], ref_d[:, qo:ko], "dk (shared prefix)")
+    assert_close(got_d[:, ko:], ref_d[:, ko:], "dv (shared prefix)")

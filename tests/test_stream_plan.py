@@ -134,3 +134,40 @@ def test_keep_plan_modes_and_the_cap():
         plan_keep(32, qkv, saved, arena, reserve, cap, "keep")
     with pytest.raises(ValueError):
         plan_keep(32, qkv, saved, arena, reserve, cap, "sometimes")
+
+
+def test_prompt_dedup_indices_brute_force():
+    """The shared-prompt layout's index arrays against a direct construction:
+    pairs (2p chosen, 2p+1 rejected) whose prompts are equal, laid out as
+    [prompt | chosen continuation | rejected continuation]."""
+    import numpy as np
+
+    from layer_streamed_qlora_b200.model import prompt_dedup_indices, token_rows
+    B, S, Lp = 6, 11, 4
+    Lc = S - Lp
+    rng = np.random.default_rng(0)
+    ids = rng.integers(0, 1000, size=(B, S))
+    ids[1::2, :Lp] = ids[0::2, :Lp]  # each pair shares its prompt
+    phys, hrows, hids, start, src = prompt_dedup_indices(B, S, Lp)
+    T = token_rows(B, S, Lp)
+    assert T == (B // 2) * (Lp + 2 * Lc) == phys.size
+    flat = ids.reshape(-1)
+    tok = flat[phys]
+    expect = np.concatenate([np.concatenate([ids[2 * p, :Lp], ids[2 * p, Lp:], ids[2 * p + 1, Lp:]])
+                             for p in range(B // 2)])
+    assert np.array_equal(tok, expect)
+    # the head reads, per sequence, positions Lp-1 .. S-1 of that sequence
+    assert hrows.size == B * (Lc + 1) and np.array_equal(flat[hids], ids[:, Lp - 1:].reshape(-1))
+    for v in range(B):
+        for j in range(Lc + 1):
+            t = Lp - 1 + j
+            assert tok[hrows[v * (Lc + 1) + j]] == ids[v, t]
+    # the CSR lists every head row once, under the token row it reads
+    assert start[0] == 0 and start[-1] == hrows.size and np.array_equal(np.sort(src), np.arange(hrows.size))
+    for d in range(T):
+        for h in src[start[d]:start[d + 1]]:
+            assert hrows[h] == d
+    # the last prompt row of each pair is read by both sequences
+    for p in range(B // 2):
+        d = p * (Lp + 2 * Lc) + Lp - 1
+        assert start[d + 1] - start[d] == 2
