@@ -57,8 +57,10 @@ typedef int32_t soup_status;
 const char* soup_last_error(void);
 
 /* Reads and clears the device error word of the current device (synchronises
- * the device).  *code_out = 0 when no kernel reported a problem; otherwise a
- * nonzero code (1 = a bounded wait on an mbarrier expired in a GEMM).
+ * the device).  *code_out = 0 when no kernel reported a problem; otherwise
+ * the OR of the codes the kernels recorded: 1 = a bounded wait on an mbarrier
+ * expired in a GEMM, 2 = a token id outside the vocabulary in soup_embed (its
+ * row is written as zeros), 4 = a bounded wait expired in an attention kernel.
  * Returns SOUP_OK, or SOUP_ERR_CUDA if the read itself failed. */
 soup_status soup_device_error(int32_t* code_out);
 

@@ -29,7 +29,7 @@
 // dS enter the MMAs as fp16, accumulation is fp32; the saved log-sum-exp is
 // in log2 units.  Outputs (attention output, dq, dk, dv) are bf16, with
 // optional fp16 / fp32 copies.  Every mbarrier wait is bounded: on expiry the
-// CTA records code 2 in the device error word, stops issuing work, lets copies
+// CTA records code 4 in the device error word, stops issuing work, lets copies
 // and MMAs in flight land, frees its tensor memory and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -43,7 +43,7 @@ namespace soup {
 namespace {
 
 constexpr int HD = 128;          // head dim
-constexpr int ERR_ATTN_WAIT = 2;  // device error code: a bounded wait of an attention kernel expired
+constexpr int ERR_ATTN_WAIT = 4;  // device error code: a bounded wait of an attention kernel expired
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);

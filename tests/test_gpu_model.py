@@ -51,7 +51,8 @@ def build(cfg, B, S, n_buffers=2, seed=0, chunk=48, task="sft", recompute="auto"
 
 
 def set_ids(m, ids):
-    m.ids.copy_(torch.from_numpy(ids.astype(np.int32)))
+    m.set_ids(torch.from_numpy(ids.astype(np.int32)))  # the model also lays out the shared-prompt rows
+    torch.cuda.synchronize()
 
 
 def check_layers_on_gpu_inputs(m, w, cfg):
