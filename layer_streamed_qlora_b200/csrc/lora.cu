@@ -193,55 +193,6 @@ extern "C" soup_status soup_lora_linear_bwd(const soup_weight* W, const uint16_t
 #define SOUP_NOALLOC_SCRATCH_BYTES (8u << 20)
 static __device__ __align__(256) uint8_t g_lora_noalloc_scratch[SOUP_NOALLOC_SCRATCH_BYTES];
 
-namespace {
-std::mutex g_noalloc_mu;
-// Per device: the context the address was looked up in, and the address.
-struct NoallocAddr {
-  void* ctx = nullptr;
-  void* ptr = nullptr;
-};
-NoallocAddr g_noalloc[64];
-
-typedef int (*CtxGetCurrentFn)(void** ctx);
-CtxGetCurrentFn ctx_get_current() {
-  static CtxGetCurrentFn fn = [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      f = nullptr;
-    return reinterpret_cast<CtxGetCurrentFn>(f);
-  }();
-  return fn;
-}
-
-// Device address of the scratch array on the current device.  Host code may
-// not pass the array's name to a kernel (that is a host-side stand-in, not a
-// device address), so it is looked up with the device current, on the
-// device's first call, and cached together with the context it belongs to: a
-// call made in a new context (after cudaDeviceReset, say, which unloads the
-// module and with it the array) looks the address up again, and so does every
-// call while the thread has no current context to compare with.
-soup_status noalloc_scratch(void** out) {
-  int dev = 0;
-  SOUP_CUDA_TRY(cudaGetDevice(&dev));
-  SOUP_CHECK(dev >= 0 && dev < 64, SOUP_ERR_INVALID_ARG, "soup_lora_linear_bwd_noalloc: device %d out of range", dev);
-  void* ctx = nullptr;
-  CtxGetCurrentFn get = ctx_get_current();
-  const bool known_ctx = get && get(&ctx) == 0 && ctx != nullptr;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  NoallocAddr& c = g_noalloc[dev];
-  if (!known_ctx || c.ptr == nullptr || c.ctx != ctx) {
-    void* p = nullptr;
-    SOUP_CUDA_TRY(cudaGetSymbolAddress(&p, g_lora_noalloc_scratch));
-    SOUP_CHECK(p != nullptr && soup_aligned(p, 256), SOUP_ERR_CUDA, "soup_lora_linear_bwd_noalloc: bad scratch address");
-    c.ptr = p;
-    c.ctx = known_ctx ? ctx : nullptr;
-  }
-  *out = c.ptr;
-  return SOUP_OK;
-}
-}  // namespace
 
 extern "C" size_t soup_lora_linear_bwd_noalloc_max_scratch(void) { return SOUP_NOALLOC_SCRATCH_BYTES; }
 
@@ -260,7 +211,7 @@ extern "C" soup_status soup_lora_linear_bwd_noalloc(const soup_weight* W, const 
              "static maximum of %u bytes; use soup_lora_linear_bwd with a workspace",
              (long long)T, r, (long long)W->out_features, need, SOUP_NOALLOC_SCRATCH_BYTES);
   void* ws = nullptr;
-  SOUP_TRY(noalloc_scratch(&ws));
+  SOUP_TRY(static_symbol_address(SYM_NOALLOC_SCRATCH, reinterpret_cast<const void*>(g_lora_noalloc_scratch), &ws));
   // Every byte of the scratch that this call reads it first writes (the
   // transpose fills B^T, the GEMM fills g' for columns [0, T), the only ones
   // read), so nothing left by an earlier call needs clearing.

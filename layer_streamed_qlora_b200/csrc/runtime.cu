@@ -13,9 +13,8 @@ namespace {
 thread_local char g_last_error[1024] = "";
 
 // Written by kernels when one of their bounded waits expires (nonzero code).
-__device__ int g_soup_device_error = 0;
+__device__ __align__(256) int g_soup_device_error = 0;
 
-int* g_err_ptr[64] = {nullptr};
 std::mutex g_mu;
 soup::EncodeTiledFn g_encode = nullptr;
 bool g_encode_tried = false;
@@ -45,16 +44,54 @@ soup_status fail(soup_status st, const char* fmt, ...) {
 
 void clear_error() { g_last_error[0] = 0; }
 
-int* device_error_word() {
+namespace {
+typedef int (*CtxGetCurrentFn)(void** ctx);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(f);
+  }();
+  return fn;
+}
+// Per (array, device): the context the address was looked up in, and the address.
+struct SymAddr {
+  void* ctx = nullptr;
+  void* ptr = nullptr;
+};
+SymAddr g_sym[SYM_N][64];
+std::mutex g_sym_mu;
+}  // namespace
+
+soup_status static_symbol_address(int which, const void* symbol, void** out) {
+  SOUP_CHECK(which >= 0 && which < SYM_N && symbol && out, SOUP_ERR_INVALID_ARG, "static_symbol_address: bad argument");
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_err_ptr[dev]) {
+  SOUP_CUDA_TRY(cudaGetDevice(&dev));
+  SOUP_CHECK(dev >= 0 && dev < 64, SOUP_ERR_INVALID_ARG, "device %d out of range", dev);
+  void* ctx = nullptr;
+  CtxGetCurrentFn get = ctx_get_current();
+  const bool known_ctx = get && get(&ctx) == 0 && ctx != nullptr;
+  std::lock_guard<std::mutex> lk(g_sym_mu);
+  SymAddr& c = g_sym[which][dev];
+  if (!known_ctx || c.ptr == nullptr || c.ctx != ctx) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_soup_device_error) != cudaSuccess) return nullptr;
-    g_err_ptr[dev] = static_cast<int*>(p);
+    SOUP_CUDA_TRY(cudaGetSymbolAddress(&p, symbol));
+    SOUP_CHECK(p != nullptr && soup_aligned(p, 256), SOUP_ERR_CUDA, "static array %d: bad device address", which);
+    c.ptr = p;
+    c.ctx = known_ctx ? ctx : nullptr;
   }
-  return g_err_ptr[dev];
+  *out = c.ptr;
+  return SOUP_OK;
+}
+
+int* device_error_word() {
+  void* p = nullptr;
+  if (static_symbol_address(SYM_DEVICE_ERROR, reinterpret_cast<const void*>(&g_soup_device_error), &p) != SOUP_OK)
+    return nullptr;
+  return static_cast<int*>(p);
 }
 
 EncodeTiledFn encode_tiled() {

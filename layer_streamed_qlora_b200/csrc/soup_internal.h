@@ -19,6 +19,17 @@ void clear_error();
 // waits expired; read by soup_device_error()).
 int* device_error_word();
 
+// Device address, on the current device, of one of the library's
+// module-static __device__ arrays.  Host code may not pass such an array's
+// name to a kernel (that is a host-side stand-in, not a device address), so
+// it is looked up with the device current and cached together with the CUDA
+// context it belongs to: a call in a new context (after cudaDeviceReset,
+// say, which unloads the module and its arrays) looks it up again, and so
+// does every call while the thread has no current context to compare with.
+enum StaticSym : int { SYM_DEVICE_ERROR = 0, SYM_NOALLOC_SCRATCH = 1, SYM_N = 2 };
+soup_status static_symbol_address(int which, const void* symbol, void** out);
+
+
 // cuTensorMapEncodeTiled resolved through the runtime's driver entry point.
 typedef int (*EncodeTiledFn)(void* tmap, int dtype, uint32_t rank, void* gaddr,
                              const uint64_t* gdim, const uint64_t* gstride,

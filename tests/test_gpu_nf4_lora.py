@@ -154,21 +154,25 @@ def test_lora_linear_tiles_and_ragged_tail():
         assert_close(g[k], ref, k)
 
 
-def test_fused_nf4_equals_dequant_then_bf16_gemm_bit_exact():
-    W, x, A, B, dy, r, s = _c1(seed=5, T=256, n_in=1024, n_out=1024, r=16, alpha=32.0)
+# (T, in, out): one-pair-per-M-tile decode (1 M tile of 256), and decode
+# shared by groups of 4 (ragged last M tile) and 8 CTA pairs, forward (W)
+# and backward (W^T) layouts
+@pytest.mark.parametrize("T,n_in,n_out", [(256, 1024, 1024), (1000, 1024, 768), (2048, 2048, 1536)])
+def test_fused_nf4_equals_dequant_then_bf16_gemm_bit_exact(T, n_in, n_out):
+    W, x, A, B, dy, r, s = _c1(seed=5, T=T, n_in=n_in, n_out=n_out, r=16, alpha=32.0)
     g_nf4 = run_gpu_lora(W, x, A, B, dy, r, s, "nf4")
     # bf16 path on exactly the dequantised weights
-    T, n_in = x.shape
     wb = dev_bf16(g_nf4["deq"])
     Wd = L.weight_bf16(wb)
     xd, Ad, Bd, dyd = dev_bf16(x), dev_bf16(A), dev_bf16(B), dev_bf16(dy)
-    y = torch.empty((T, 1024), dtype=torch.bfloat16, device="cuda")
-    u = torch.zeros((r, T), dtype=torch.bfloat16, device="cuda")
+    ldT = (T + 7) // 8 * 8
+    y = torch.empty((T, n_out), dtype=torch.bfloat16, device="cuda")
+    u = torch.zeros((r, ldT), dtype=torch.bfloat16, device="cuda")
     L.soup_lora_linear_fwd(Wd, Ad, Bd, r, s, xd, T, y, u)
     dx = torch.empty((T, n_in), dtype=torch.bfloat16, device="cuda")
     dA = torch.empty((r, n_in), dtype=torch.float32, device="cuda")
-    dB = torch.empty((1024, r), dtype=torch.float32, device="cuda")
-    ws = torch.empty(L.soup_lora_linear_bwd_workspace(T, r, 1024), dtype=torch.uint8, device="cuda")
+    dB = torch.empty((n_out, r), dtype=torch.float32, device="cuda")
+    ws = torch.empty(L.soup_lora_linear_bwd_workspace(T, r, n_out), dtype=torch.uint8, device="cuda")
     L.soup_lora_linear_bwd(Wd, Ad, Bd, r, s, xd, u, dyd, T, dx, dA, dB, ws)
     torch.cuda.synchronize()
     assert np.array_equal(host(y), g_nf4["y"])
