@@ -58,6 +58,15 @@ __device__ __forceinline__ uint32_t pack_b2(float lo, float hi) {
 __device__ __forceinline__ void st_unit(uint8_t* tile, int r, int u, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   *reinterpret_cast<uint4*>(tile + r * 128 + ((u ^ (r & 7)) << 4)) = make_uint4(a, b, c, d);
 }
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32: relative error
+// about 2^-22, results below 2^-126 flushed to zero).  Every argument here is
+// a scaled score minus a running maximum or log-sum-exp (<= 0 up to
+// rounding), or -inf for a masked key, whose power is 0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
 }
@@ -269,7 +278,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
       const uint32_t ph = (jo >> 1) & 1;
       if (!ATTN_WAIT(&o_full[s], ph)) return false;
       ptx::tc_fence_after();
-      const float alpha = exp2f(m_o - mj);
+      const float alpha = ex2(m_o - mj);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
@@ -291,22 +300,26 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
       ptx::tc_fence_after();
       const int key0 = j * 128;
       const bool edge = key0 + 127 > qi || key0 + 128 > S;  // some key of the block is masked for this row
-      // pass 1: the row's maximum over the block
+      // pass 1: the row's maximum over the block, of the raw scores (the
+      // scale is positive: it multiplies the maximum once)
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
         ptx::tmem_ld32(tl + s * 128 + c * 32, v);
         ptx::tmem_ld_wait();
+        if (edge) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int key = key0 + c * 32 + i;
-          float x = __uint_as_float(v[i]) * sl2;
-          if (edge && (key > qi || key >= S)) x = -INFINITY;
-          mx = fmaxf(mx, x);
+          for (int i = 0; i < 32; ++i) {
+            const int key = key0 + c * 32 + i;
+            if (key <= qi && key < S) mx = fmaxf(mx, __uint_as_float(v[i]));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(v[i]));
         }
       }
-      const float m_new = fmaxf(m, mx);
+      const float m_new = fmaxf(m, mx * sl2);
       // pass 2 (this warp's 64 keys): p = 2^(x - m_new) (0 where masked),
       // partial row sum, P in fp16
       if (!ATTN_WAIT(&p_empty[s], ph ^ 1)) { ok = false; break; }
@@ -321,12 +334,13 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
           const int key = key0 + half * 64 + c * 32 + i;
-          float x0 = __uint_as_float(v[i]) * sl2, x1 = __uint_as_float(v[i + 1]) * sl2;
+          // one FMA per exponent argument: x * scale - m
+          float x0 = fmaf(__uint_as_float(v[i]), sl2, -m_new), x1 = fmaf(__uint_as_float(v[i + 1]), sl2, -m_new);
           if (edge) {
             if (key > qi || key >= S) x0 = -INFINITY;
             if (key + 1 > qi || key + 1 >= S) x1 = -INFINITY;
           }
-          const float p0 = exp2f(x0 - m_new), p1 = exp2f(x1 - m_new);
+          const float p0 = ex2(x0), p1 = ex2(x1);
           sum += p0 + p1;
           pk[i >> 1] = pack_h2(p0, p1);
         }
@@ -341,7 +355,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
         ptx::mbar_arrive(&s_free[s]);
         ptx::mbar_arrive(&p_full[s]);
       }
-      l = l * exp2f(m - m_new) + sum;
+      l = l * ex2(m - m_new) + sum;
       m = m_new;
       if (j >= 1 && !fold_o(j - 1, m_pend)) { ok = false; break; }
       m_pend = m_new;
@@ -603,9 +617,9 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
           for (int e = 0; e < 2; ++e) {
             const int qi = c * 32 + i + e;
             const int q = q0 + qi;
-            float x = __uint_as_float(sv[i + e]) * sl2 - LD[qi];
+            float x = fmaf(__uint_as_float(sv[i + e]), sl2, -LD[qi]);
             if (edge && (q < key || q >= S || key >= S)) x = -INFINITY;
-            p[e] = exp2f(x);
+            p[e] = ex2(x);
             d[e] = p[e] * (__uint_as_float(dv[i + e]) - LD[64 + qi]);
           }
           pk[i >> 1] = pack_h2(p[0], p[1]);
@@ -848,9 +862,9 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int key = key0 + c * 32 + i + e;
-            float x = __uint_as_float(sv[i + e]) * sl2 - Lr;
+            float x = fmaf(__uint_as_float(sv[i + e]), sl2, -Lr);
             if (edge && (key > qi || key >= S || !qin)) x = -INFINITY;
-            const float p = exp2f(x);
+            const float p = ex2(x);
             d[e] = p * (__uint_as_float(dv[i + e]) - Dr);
           }
           dk[i >> 1] = pack_h2(d[0], d[1]);
