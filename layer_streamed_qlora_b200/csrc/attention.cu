@@ -2,7 +2,8 @@
 // generation tensor cores: tcgen05.mma with the accumulators in tensor memory,
 // operand tiles brought into 128-byte-swizzled shared memory by TMA (no
 // cluster multicast), warp-specialised CTAs (one TMA thread, one MMA thread,
-// four softmax / epilogue warps, one query or key row per thread).
+// eight softmax / elementwise warps: two per query or key row, each taking
+// half of the row's columns).
 //
 //   forward   per (128-query tile, q head): S_j = Q K_j^T into tensor memory,
 //             online softmax in fp32 (log2 domain) from a two-pass read of the
@@ -13,7 +14,8 @@
 //             double-buffered in tensor memory (4 x 128 columns), so the
 //             tensor cores compute S_{j+1} and O_j while the softmax warps
 //             work on block j.
-//   backward  two passes, no atomics (every run gives the same bits):
+//   backward  two passes in one launch, no atomics (every run gives the same
+//             bits):
 //             pass 1 per (128-key block, kv head): for each q head of the group
 //             and each 64-query tile at or after the block, S^T = K Q^T and
 //             dP^T = V dO^T (tensor memory), P^T = 2^(S^T scale - L) and
@@ -21,6 +23,8 @@
 //             dV += P^T dO and dK += dS^T Q accumulated in tensor memory;
 //             pass 2 per (128-query tile, q head): S = Q K^T, dP = dO V^T per
 //             64-key block, dS into shared memory, dQ += dS K in tensor memory.
+//             The passes write disjoint outputs, so their CTAs share the grid
+//             (heaviest pass-1 key blocks first, then pass-2 query tiles).
 //             Q, dO (pass 1) and K (pass 2) tiles serve both as K-major and as
 //             MN-major operands of the same shared-memory bytes.
 //
@@ -409,10 +413,10 @@ constexpr int B1_LD = B1_DS + 2 * 16384;        // NS x (64 L + 64 D) floats
 constexpr int B1_BAR = B1_LD + B1_NS * 512;
 constexpr int B1_SMEM = B1_BAR + 256 + 1024;
 
-__global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant__ CUtensorMap tm128,
-                                                           const __grid_constant__ CUtensorMap tm64,
-                                                           const __grid_constant__ CUtensorMap tmdo64,
-                                                           const AttnArgs a) {
+// One CTA of pass 1 (key block bx of sequence group bz, kv head by).
+__device__ __forceinline__ void attn_bwd_dkdv_cta(const CUtensorMap& tm128, const CUtensorMap& tm64,
+                                                  const CUtensorMap& tmdo64, const AttnArgs& a, int bx, int by,
+                                                  int bz) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + B1_BAR);
@@ -431,9 +435,9 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
   // physical key block pb of sequence group gq: a block of the shared prefix
   // (every sequence of the group attends to it) or a continuation block of
   // one sequence; the first blocks have the most query tiles
-  const int g = blockIdx.y, gq = blockIdx.z;
+  const int g = by, gq = bz;
   const int nb_pre = a.Lp / 128, nbc = (S - a.Lp + 127) / 128;
-  const int pb = blockIdx.x;
+  const int pb = bx;
   const bool prefix = pb < nb_pre;
   const int own = prefix ? 0 : (pb - nb_pre) / nbc;            // sequence of the group owning the block
   const int kb = prefix ? pb : nb_pre + (pb - nb_pre) % nbc;    // block index within the sequence
@@ -469,8 +473,8 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&st_full[i], 1);
-      ptx::mbar_init(&st_free[i], 4);
-      ptx::mbar_init(&p_full[i], 4);
+      ptx::mbar_init(&st_free[i], 8);
+      ptx::mbar_init(&p_full[i], 8);
       ptx::mbar_init(&p_empty[i], 1);
     }
     ptx::mbar_init(acc_full, 1);
@@ -580,8 +584,8 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
       if (ok && n_it > 0) ptx::mma_commit(acc_full);
     }
   } else {
-    // ------------------------------------ elementwise warps (one key row each)
-    const int quad = warp & 3;
+    // ---------------- elementwise warps: two per key row, 32 queries each
+    const int quad = warp & 3, half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const int key = kb * 128 + row;
@@ -603,8 +607,8 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
       uint8_t* P = sm + B1_P + bb * 16384;
       uint8_t* DS = sm + B1_DS + bb * 16384;
       const bool edge = q0 < key || q0 + 64 > S || key >= S;  // some query of the tile is masked for this key
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      {
+        const int c = half;  // this warp's 32 queries of the tile
         uint32_t sv[32], dv[32];
         ptx::tmem_ld32(tl + bb * 64 + c * 32, sv);
         ptx::tmem_ld32(tl + 128 + bb * 64 + c * 32, dv);
@@ -639,14 +643,15 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dkdv_tc(const __grid_constant
         ptx::mbar_arrive(&p_full[bb]);
       }
     }
-    // epilogue: dK (x scale, RoPE back) and dV from tensor memory, unscaled
+    // epilogue: dK (x scale, RoPE back) from the second warp of a row, dV
+    // (unscaled) from the first, out of tensor memory
     if (ok && n_it > 0 && ATTN_WAIT(acc_full, 0)) {
       ptx::tc_fence_after();
       const float unscale = a.amax ? 1.f / grad_scale_from_amax(__uint_as_float(*a.amax)) : 1.f;
       const bool in = key < S;
       const size_t r = (size_t)(in ? vrow(a, v0, key) : 0) * a.ld;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+      {
+        const int which = half;  // 0: dV, 1: dK
         const uint32_t col0 = which ? 384 : 256;
         const float mul = which ? a.scale * unscale : unscale;
         const int dcol = which ? kcol : vcol;
@@ -707,10 +712,10 @@ constexpr int B2_DS = B2_ST + B2_NS * B2_STAGE;
 constexpr int B2_BAR = B2_DS + 2 * 16384;
 constexpr int B2_SMEM = B2_BAR + 256 + 1024;
 
-__global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tm128,
-                                                         const __grid_constant__ CUtensorMap tm64,
-                                                         const __grid_constant__ CUtensorMap tmdo128,
-                                                         const AttnArgs a) {
+// One CTA of pass 2 (query tile nqt - 1 - bx of sequence bz, q head by).
+__device__ __forceinline__ void attn_bwd_dq_cta(const CUtensorMap& tm128, const CUtensorMap& tm64,
+                                                const CUtensorMap& tmdo128, const AttnArgs& a, int bx, int by,
+                                                int bz) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + B2_BAR);
@@ -727,8 +732,8 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
 
   const int S = a.S;
   const int nqt = (S + 127) / 128;
-  const int qb = nqt - 1 - (int)blockIdx.x;  // the longest rows first
-  const int h = blockIdx.y, v = blockIdx.z;  // q head, sequence
+  const int qb = nqt - 1 - bx;  // the longest rows first
+  const int h = by, v = bz;     // q head, sequence
   if (v % a.G != 0 && qb * 128 < a.Lp) return;  // shared-prefix queries: sequence 0 of the group
   const int g = h / (a.Hq / a.Hkv);
   const int kcol = (a.Hq + g) * HD, vcol = (a.Hq + a.Hkv + g) * HD;
@@ -743,8 +748,8 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&st_full[i], 1);
-      ptx::mbar_init(&st_free[i], 4);
-      ptx::mbar_init(&ds_full[i], 4);
+      ptx::mbar_init(&st_free[i], 8);
+      ptx::mbar_init(&ds_full[i], 8);
       ptx::mbar_init(&ds_empty[i], 1);
     }
     ptx::mbar_init(acc_full, 1);
@@ -830,7 +835,8 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
       if (ok) ptx::mma_commit(acc_full);
     }
   } else {
-    const int quad = warp & 3;
+    // ---------------- elementwise warps: two per query row, 32 keys each
+    const int quad = warp & 3, half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const int qi = qb * 128 + row;
@@ -849,8 +855,8 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
       if (!ATTN_WAIT(&ds_empty[bb], pb ^ 1)) { ok = false; break; }
       uint8_t* DS = sm + B2_DS + bb * 16384;
       const bool edge = key0 + 63 > qi || key0 + 64 > S || !qin;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      {
+        const int c = half;  // this warp's 32 keys of the block
         uint32_t sv[32], dv[32];
         ptx::tmem_ld32(tl + bb * 64 + c * 32, sv);
         ptx::tmem_ld32(tl + 128 + bb * 64 + c * 32, dv);
@@ -885,8 +891,8 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
       const float unscale = a.amax ? 1.f / grad_scale_from_amax(__uint_as_float(*a.amax)) : 1.f;
       const float mul = a.scale * unscale;
       const size_t r = (size_t)prow * a.ld + h * HD;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      {
+        const int c = half;  // pairs (c*32 + i, c*32 + i + 64)
         uint32_t v0[32], v1[32];
         ptx::tmem_ld32(tl + 256 + c * 32, v0);
         ptx::tmem_ld32(tl + 256 + 64 + c * 32, v1);
@@ -929,6 +935,28 @@ __global__ void __launch_bounds__(192, 1) attn_bwd_dq_tc(const __grid_constant__
   attn_teardown(abort_flag, warp, tmem);
 }
 
+// Both backward passes in one launch (they write disjoint columns of dq|dk|dv
+// and only read the forward's outputs): CTAs [0, n1) are pass-1 key blocks,
+// heaviest (most query tiles) first, the rest pass-2 query tiles, longest
+// first, so the scheduler fills the SMs the uneven causal pass 1 leaves.
+constexpr int B_SMEM = B1_SMEM > B2_SMEM ? B1_SMEM : B2_SMEM;
+__global__ void __launch_bounds__(320, 1) attn_bwd_tc(const __grid_constant__ CUtensorMap tm128,
+                                                      const __grid_constant__ CUtensorMap tm64,
+                                                      const __grid_constant__ CUtensorMap tmdo64,
+                                                      const __grid_constant__ CUtensorMap tmdo128, const AttnArgs a,
+                                                      int x1, int y1, int z1, int y2, int z2) {
+  int i = (int)blockIdx.x;
+  const int n1 = x1 * y1 * z1;
+  if (i < n1) {
+    const int yz = y1 * z1;
+    attn_bwd_dkdv_cta(tm128, tm64, tmdo64, a, i / yz, (i % yz) % y1, (i % yz) / y1);
+  } else {
+    i -= n1;
+    const int yz = y2 * z2;
+    attn_bwd_dq_cta(tm128, tm64, tmdo128, a, i / yz, (i % yz) % y2, (i % yz) / y2);
+  }
+}
+
 #undef ATTN_WAIT
 
 // 2-D fp16 tensor map over [rows, cols] (row stride ld elements), box of
@@ -955,8 +983,7 @@ soup_status attn_init() {
   static bool init = false;
   if (!init) {
     SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, F_SMEM));
-    SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dkdv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, B1_SMEM));
-    SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, B2_SMEM));
+    SOUP_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, B_SMEM));
     init = true;
   }
   return SOUP_OK;
@@ -1033,11 +1060,9 @@ soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
   a.wait_limit = 4000000000LL;
   const double fl = 2.5 * 4.0 * Bsz * Hq * (double)HD * ((double)S * (S + 1) / 2);
   profile_begin(st, GC_ATTN, fl, 0.0);
-  dim3 g1(Lp / 128 + G * ((S - Lp + 127) / 128), Hkv, Bsz / G);
-  attn_bwd_dkdv_tc<<<g1, 192, B1_SMEM, st>>>(tm128, tm64, tmdo64, a);
-  SOUP_LAUNCH_CHECK();
-  dim3 g2((S + 127) / 128, Hq, Bsz);
-  attn_bwd_dq_tc<<<g2, 192, B2_SMEM, st>>>(tm128, tm64, tmdo128, a);
+  const int x1 = Lp / 128 + G * ((S - Lp + 127) / 128), y1 = Hkv, z1 = Bsz / G;  // pass 1
+  const int x2 = (S + 127) / 128, y2 = Hq, z2 = Bsz;                              // pass 2
+  attn_bwd_tc<<<x1 * y1 * z1 + x2 * y2 * z2, 320, B_SMEM, st>>>(tm128, tm64, tmdo64, tmdo128, a, x1, y1, z1, y2, z2);
   SOUP_LAUNCH_CHECK();
   profile_end(st);
   return SOUP_OK;
