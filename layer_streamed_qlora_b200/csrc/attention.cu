@@ -83,6 +83,7 @@ __device__ __forceinline__ uint64_t mndesc(uint32_t saddr, uint32_t chunk) {
 
 struct AttnArgs {
   int S, Hq, Hkv, T;  // S: tokens per sequence; T: token rows in memory
+  int nseq;           // sequences (forward grid)
   // Sequences come in groups of G that share their first Lp positions,
   // stored once: a group's rows are [prefix | continuation of sequence 0 |
   // ... | continuation of sequence G-1] (G = 1, Lp = 0: sequence v is rows
@@ -171,8 +172,10 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
 
   const int S = a.S;
   const int nqt = (S + 127) / 128;
-  const int qb = nqt - 1 - (int)blockIdx.x;  // the longest rows first
-  const int h = blockIdx.y, v = blockIdx.z;  // q head, sequence
+  // one-dimensional grid, query tile outermost: the tiles with the most key
+  // blocks (the last ones) of every head and sequence start first
+  const int hv = (int)blockIdx.x % (a.Hq * a.nseq), qb = nqt - 1 - (int)blockIdx.x / (a.Hq * a.nseq);
+  const int h = hv % a.Hq, v = hv / a.Hq;  // q head, sequence
   if (v % a.G != 0 && qb * 128 < a.Lp) return;  // shared-prefix queries: sequence 0 of the group computes them
   const int g = h / (a.Hq / a.Hkv);
   const int nkb = qb + 1;
@@ -1025,8 +1028,8 @@ soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
   a.wait_limit = 4000000000LL;
   const double fl = 4.0 * Bsz * Hq * (double)HD * ((double)S * (S + 1) / 2);
   profile_begin(st, GC_ATTN, fl, 0.0);
-  dim3 grid((S + 127) / 128, Hq, Bsz);
-  attn_fwd_tc<<<grid, 320, F_SMEM, st>>>(tm, a);
+  a.nseq = Bsz;
+  attn_fwd_tc<<<((S + 127) / 128) * Hq * Bsz, 320, F_SMEM, st>>>(tm, a);
   SOUP_LAUNCH_CHECK();
   profile_end(st);
   return SOUP_OK;
