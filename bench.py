@@ -299,10 +299,12 @@ def probe_shapes(w):
 
 
 def run_probe_gemm(w):
-    """One forward fused NF4 GEMM per projection shape of the workload's layer
-    at its token count (random NF4 weights, LoRA r), each after one warm-up
-    launch, in the order of PROBE_WEIGHTS: an ncu capture of the fused GEMM
-    kernel with -s 1 -c 1 per shape (or -c 8 for all) reads DRAM traffic per launch."""
+    """The fused NF4 GEMMs of each projection shape of the workload's layer at
+    its token count (random NF4 weights, LoRA r), in the order of
+    PROBE_WEIGHTS: per shape a warm-up pass, then one forward (W) and one
+    backward (W^T) launch of the fused kernel; an ncu capture of
+    `gemm_pair_persistent` with -c 16 lists, per shape, warm-up W, warm-up
+    W^T, W, W^T."""
     import torch
 
     from layer_streamed_qlora_b200 import _lib as L
@@ -321,11 +323,18 @@ def run_probe_gemm(w):
         Bm = (torch.randn(N, r, device="cuda", generator=g) * 0.02).bfloat16()
         y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
         u = torch.empty(r, T, dtype=torch.bfloat16, device="cuda")
+        dy = torch.randn(T, N, device="cuda", generator=g).bfloat16()
+        dx = torch.empty(T, K, dtype=torch.bfloat16, device="cuda")
+        dA = torch.empty(r, K, device="cuda")
+        dB = torch.empty(N, r, device="cuda")
+        ws = torch.empty(L.soup_lora_linear_bwd_workspace(T, r, N), dtype=torch.uint8, device="cuda")
         for _ in range(2):
             L.soup_lora_linear_fwd(wt, A, Bm, r, w["alpha"] / r, x, T, y, u)
+            L.soup_lora_linear_bwd(wt, A, Bm, r, w["alpha"] / r, x, u, dy, T, dx, dA, dB, ws)
         torch.cuda.synchronize()
         print(f"probe {name}: N={N} K={K} T={T}", flush=True)
-    print(json.dumps({"probe": "fused NF4 forward GEMMs", "weights": PROBE_WEIGHTS}))
+    assert L.device_error() == 0
+    print(json.dumps({"probe": "fused NF4 GEMMs (W and W^T)", "weights": PROBE_WEIGHTS}))
     return 0
 
 
