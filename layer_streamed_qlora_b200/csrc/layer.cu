@@ -18,6 +18,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "elementwise.h"
 #include "lora_internal.h"
@@ -40,6 +41,7 @@ struct WS {
   size_t x1_lo, dh2_lo;                       // bf16 rounding residuals (dual-A GEMM inputs)
   size_t attn32, uo32, go32, Ao32;            // fp32 operands of the o LoRA-gradient GEMMs (tf32)
   size_t splitk, splitk_bytes;                // fp32 partial products of split-K LoRA GEMMs
+  size_t splitk2;                             // the same for the GEMMs of the side stream (backward)
   size_t u_gu_lo, g_d_lo, u_d32;     // MLP LoRA-gradient operands beyond bf16 (residuals, fp32)
   size_t x2_32, Agu32, g_gu32, d_gu_lo;
   size_t Bt_down32, Bt_o32, Bbd_qkv32, Bbd_gu;  // B factors prepared for the g GEMMs (transposed, block-diagonal)
@@ -108,6 +110,7 @@ WS layout(const Dims& m) {
   w.go32 = take(r * ldT * 4);
   w.splitk_bytes = 8 * T * 64 * 4;
   w.splitk = take(w.splitk_bytes);
+  w.splitk2 = take(w.splitk_bytes);
   w.g_d_lo = take(r * ldT * 2);
   w.g_gu32 = take(2 * r * ldT * 4);
   w.d_gu_lo = take(T * 2 * I * 2);
@@ -372,6 +375,35 @@ soup_status proj_bwd(const soup_weight* W, const uint16_t* dy, int T, const uint
 // keep (forward pass only): also compute q|k|v with the hi + lo A pair and
 // leave them (fp16, [T, qkv_w]) in `keep` for the backward; kept (recompute
 // only): q|k|v of this layer kept by the forward pass, whose GEMM is skipped.
+// The backward's side stream: the LoRA-factor gradients (dA, dB) feed only
+// the optimiser, so they run on a second stream of the device beside the
+// dx chain (on CTAs the big GEMMs' last rounds leave free), joined at the end
+// of the layer.  One stream and six fork / join events per device, created
+// once, again for a new CUDA context.
+struct SideStream {
+  void* ctx = nullptr;
+  cudaStream_t st = nullptr;
+  cudaEvent_t ev[6] = {};
+};
+SideStream g_side[64];
+std::mutex g_side_mu;
+
+soup_status side_stream(SideStream** out) {
+  int dev = 0;
+  SOUP_CUDA_TRY(cudaGetDevice(&dev));
+  SOUP_CHECK(dev >= 0 && dev < 64, SOUP_ERR_INVALID_ARG, "device %d out of range", dev);
+  void* ctx = current_context();
+  std::lock_guard<std::mutex> lk(g_side_mu);
+  SideStream& s = g_side[dev];
+  if (s.st == nullptr || ctx == nullptr || s.ctx != ctx) {
+    SOUP_CUDA_TRY(cudaStreamCreateWithFlags(&s.st, cudaStreamNonBlocking));
+    for (auto& e : s.ev) SOUP_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    s.ctx = ctx;
+  }
+  *out = &s;
+  return SOUP_OK;
+}
+
 soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const soup_layer_cfg* c, const Dims& m,
                     const WS& ws, char* base, char* fb, const uint16_t* h_in, uint16_t* h_out, bool on, bool save,
                     bool want_out, cudaStream_t st, uint16_t* keep = nullptr, const uint16_t* kept = nullptr) {
@@ -577,31 +609,55 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
     SOUP_TRY(lora_prep(pj, st));
   }
 
+  // LoRA-factor gradients go to the side stream: each group waits (event)
+  // for the main-stream step that produced its inputs and is issued after
+  // the next big GEMM, so that GEMM's CTAs are dispatched first
+  SideStream* side = nullptr;
+  if (on) SOUP_TRY(side_stream(&side));
+  const SplitWS SW2{PF(splitk2), ws.splitk_bytes};
+  cudaStream_t s2 = side ? side->st : st;
+  auto mark = [&](int e) -> soup_status {  // the side stream may consume what st has produced so far
+    SOUP_CUDA_TRY(cudaEventRecord(side->ev[e], st));
+    return SOUP_OK;
+  };
+  auto after = [&](int e) -> soup_status {
+    SOUP_CUDA_TRY(cudaStreamWaitEvent(s2, side->ev[e], 0));
+    return SOUP_OK;
+  };
+
   // ---- MLP block
   SOUP_TRY(f32_to_bf16(dh_out, (size_t)T * H, P(dh_b), st));
   // LoRA gradients of the MLP: g_down from the fp32 dh (tf32), the others
   // from hi + lo (rounding residual) operand pairs, so no operand of a
   // LoRA-gradient GEMM carries more than the bf16 rounding of d_gu
-  if (on)
+  if (on) {
     SOUP_TRY(lora_g_prepared(dh_out, nullptr, H, T, H, PF(Bt_down32), r, m.s, true, P(g_d), nullptr, P(g_d_lo), ldT,
                              st, SW));
+    SOUP_TRY(mark(0));
+  }
   // d_gu = SwiGLU backward of (dh W_down + g' A_down), fused in the epilogue
   SOUP_TRY(proj_bwd(&W->down, P(dh_b), T, P(g_d), ldT, r, on ? L->A_down : nullptr, on, P(d_gu), st, OUT_BF16, I,
                     P(gu16), nullptr, nullptr, on ? P(d_gu_lo) : nullptr));
   if (on) {
-    SOUP_TRY(lora_dB_tf32(dh_out, H, T, H, PF(u_d32), r, ldT, G->dB_down, st, SW));
-    SOUP_TRY(lora_dA_dual(P(g_d), P(g_d_lo), r, ldT, P(act), T, I, G->dA_down, st, SW));
+    SOUP_TRY(mark(1));
+    SOUP_TRY(after(0));
+    SOUP_TRY(lora_dB_tf32(dh_out, H, T, H, PF(u_d32), r, ldT, G->dB_down, s2, SW2));
+    SOUP_TRY(lora_dA_dual(P(g_d), P(g_d_lo), r, ldT, P(act), T, I, G->dA_down, s2, SW2));
   }
   uint16_t* d_gu = P(d_gu);
-  if (on)  // g_gate | g_up in one GEMM (block-diagonal B_gu^T), d_gu hi + lo
+  if (on) {  // g_gate | g_up in one GEMM (block-diagonal B_gu^T), d_gu hi + lo
     SOUP_TRY(lora_g_prepared(d_gu, P(d_gu_lo), 2 * I, T, 2 * I, P(Bbd_gu), 2 * r, m.s, false, P(g_gu), PF(g_gu32),
                              nullptr, ldT, st, SW));
+    SOUP_TRY(mark(2));
+  }
   SOUP_TRY(proj_bwd(&W->gate_up, d_gu, T, P(g_gu), ldT, 2 * r, on ? L->A_gu : nullptr, on, P(dx2), st));
   if (on) {
+    SOUP_TRY(after(1));
     for (int sg = 0; sg < 2; ++sg)
       SOUP_TRY(lora_dB_dual(d_gu + (size_t)sg * I, 2 * I, T, I, P(u_gu) + (size_t)sg * r * ldT,
-                            P(u_gu_lo) + (size_t)sg * r * ldT, r, ldT, G->dB_gu + (size_t)sg * I * r, st, SW));
-    SOUP_TRY(lora_dA_tf32(PF(x2_32), T, H, PF(g_gu32), 2 * r, ldT, G->dA_gu, st, SW));
+                            P(u_gu_lo) + (size_t)sg * r * ldT, r, ldT, G->dB_gu + (size_t)sg * I * r, s2, SW2));
+    SOUP_TRY(after(2));
+    SOUP_TRY(lora_dA_tf32(PF(x2_32), T, H, PF(g_gu32), 2 * r, ldT, G->dA_gu, s2, SW2));
   }
   unsigned int* gamax = reinterpret_cast<unsigned int*>(base + ws.gamax);
   SOUP_CUDA_TRY(cudaMemsetAsync(gamax, 0, sizeof(unsigned int), st));
@@ -609,16 +665,19 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
                        P(dh2_lo)));
 
   // ---- attention block
-  if (on)
+  if (on) {
     SOUP_TRY(lora_g_prepared(PF(dh2), nullptr, H, T, H, PF(Bt_o32), r, m.s, true, P(g_o), PF(go32), nullptr, ldT, st,
                              SW));
+    SOUP_TRY(mark(3));
+  }
   // dO for the attention backward: from the fp32-accurate dh2 (hi + lo parts),
   // stored fp16 scaled by a power of two derived from max |dh2|
   SOUP_TRY(proj_bwd(&W->o, P(dh2_b), T, P(g_o), ldT, r, on ? L->A_o : nullptr, on, P(d_attn), st, OUT_F16, 0,
                     nullptr, gamax, P(dh2_lo)));
   if (on) {
-    SOUP_TRY(lora_dB_tf32(PF(dh2), H, T, H, PF(uo32), r, ldT, G->dB_o, st, SW));
-    SOUP_TRY(lora_dA_tf32(PF(attn32), T, m.o_in, PF(go32), r, ldT, G->dA_o, st, SW));
+    SOUP_TRY(after(3));
+    SOUP_TRY(lora_dB_tf32(PF(dh2), H, T, H, PF(uo32), r, ldT, G->dB_o, s2, SW2));
+    SOUP_TRY(lora_dA_tf32(PF(attn32), T, m.o_in, PF(go32), r, ldT, G->dA_o, s2, SW2));
   }
   SOUP_TRY(attn_rowdot(P(d_attn), P(attn16), T, m.Hq, PF(D), st));
   // dq and dk leave the attention backward already rotated back (inverse RoPE in its epilogues)
@@ -626,17 +685,23 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
                          PF(sinb), gamax, st, on ? PF(dqkv32) : nullptr, m.G, m.Lp));
   const int seg_n[3] = {m.Hq * m.d, m.Hkv * m.d, m.Hkv * m.d};
   const int seg_c[3] = {0, m.Hq * m.d, (m.Hq + m.Hkv) * m.d};
-  if (on)  // g_q | g_k | g_v in one GEMM (block-diagonal B_qkv^T)
+  if (on) {  // g_q | g_k | g_v in one GEMM (block-diagonal B_qkv^T)
     SOUP_TRY(lora_g_prepared(PF(dqkv32), nullptr, m.qkv_w, T, m.qkv_w, PF(Bbd_qkv32), 3 * r, m.s, true, P(g_qkv),
                              PF(g32), nullptr, ldT, st, SW));
+    SOUP_TRY(mark(4));
+  }
   SOUP_TRY(proj_bwd(&W->qkv, P(d_qkv), T, P(g_qkv), ldT, 3 * r, on ? L->A_qkv : nullptr, on, P(dx1), st));
   if (on) {
+    SOUP_TRY(after(4));
     for (int sg = 0; sg < 3; ++sg)
       SOUP_TRY(lora_dB_tf32(PF(dqkv32) + seg_c[sg], m.qkv_w, T, seg_n[sg], PF(u32) + (size_t)sg * r * ldT, r, ldT,
-                            G->dB_qkv + (size_t)seg_c[sg] * r, st, SW));
-    SOUP_TRY(lora_dA_tf32(PF(x1_32), T, H, PF(g32), 3 * r, ldT, G->dA_qkv, st, SW));
+                            G->dB_qkv + (size_t)seg_c[sg] * r, s2, SW2));
+    SOUP_TRY(lora_dA_tf32(PF(x1_32), T, H, PF(g32), 3 * r, ldT, G->dA_qkv, s2, SW2));
+    // join: the layer's work is done on st only when the side stream's is
+    SOUP_CUDA_TRY(cudaEventRecord(side->ev[5], s2));
   }
   SOUP_TRY(rmsnorm_bwd(h_in, nullptr, W->norm1, PF(rinv1), P(dx1), PF(dh2), T, H, dh_in, nullptr, st));
+  if (on) SOUP_CUDA_TRY(cudaStreamWaitEvent(st, side->ev[5], 0));
   return SOUP_OK;
 }
 

@@ -66,6 +66,12 @@ SymAddr g_sym[SYM_N][64];
 std::mutex g_sym_mu;
 }  // namespace
 
+void* current_context() {
+  void* ctx = nullptr;
+  CtxGetCurrentFn get = ctx_get_current();
+  return (get && get(&ctx) == 0) ? ctx : nullptr;
+}
+
 soup_status static_symbol_address(int which, const void* symbol, void** out) {
   SOUP_CHECK(which >= 0 && which < SYM_N && symbol && out, SOUP_ERR_INVALID_ARG, "static_symbol_address: bad argument");
   int dev = 0;

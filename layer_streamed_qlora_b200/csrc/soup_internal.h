@@ -26,6 +26,10 @@ int* device_error_word();
 // context it belongs to: a call in a new context (after cudaDeviceReset,
 // say, which unloads the module and its arrays) looks it up again, and so
 // does every call while the thread has no current context to compare with.
+// The calling thread's current CUDA context (null when it has none or the
+// driver entry point is unavailable).
+void* current_context();
+
 enum StaticSym : int { SYM_DEVICE_ERROR = 0, SYM_NOALLOC_SCRATCH = 1, SYM_N = 2 };
 soup_status static_symbol_address(int which, const void* symbol, void** out);
 
