@@ -311,7 +311,11 @@ soup_status soup_decoder_layer_fwd(const soup_layer_weights* W, const soup_layer
 /* Recompute-backward: re-runs the forward from h_in (keeping intermediates),
  * then back-propagates dh_out [T, H] fp32 (gradient w.r.t. h_out) to
  * dh_in [T, H] fp32 and fills the LoRA gradients.  W gets no gradient.
- * dh_in may alias dh_out.  With adapters_on = 0 the grads are not written. */
+ * dh_in may alias dh_out.  With adapters_on = 0 the grads are not written.
+ * The LoRA-factor gradients (dA, dB) run on a library-internal stream of the
+ * device, forked from `stream` by events and joined back into it before the
+ * call returns: to the caller all of the layer's work is ordered on
+ * `stream` as usual (the dA / dB GEMMs overlap the dx chain on the GPU). */
 soup_status soup_decoder_layer_bwd(const soup_layer_weights* W, const soup_layer_lora* lora,
                                    const soup_layer_cfg* cfg, const uint16_t* h_in,
                                    const float* dh_out, int64_t batch, int64_t seq, float* dh_in,
