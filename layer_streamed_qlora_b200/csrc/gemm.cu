@@ -27,6 +27,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "gemm.h"
 #include "nf4_codebook.cuh"
@@ -95,6 +96,18 @@ struct KArgs {
   int* err;
   long long wait_limit;  // clock cycles a bounded mbarrier wait may take before it gives up
   int skip_producer;     // test hook (one-CTA kernel): the TMA producer issues nothing and never arrives
+  // Persistent kernel, last partial round split along K: every pair first
+  // takes sk_full whole tiles (t = pair + j * pairs), then the slice units
+  // u = pair, pair + pairs, ... < sk_units, unit u being k-slice u % sk_k of
+  // leftover tile sk_full * pairs + u / sk_k.  A slice stores its fp32
+  // partial ([256 columns][128 rows] per CTA) in sk_ws; the last slice of a
+  // tile to finish (counted in sk_cnt, tagged with sk_epoch) sums the
+  // tile's partials in slice order and runs the epilogue.  sk_k < 2: whole
+  // tiles only.
+  int sk_full, sk_units, sk_k;
+  float* sk_ws;
+  unsigned long long* sk_cnt;
+  unsigned int sk_epoch;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -223,10 +236,36 @@ __device__ __forceinline__ void load_codes(const uint8_t* src, uint32_t (&w)[NWO
 // Epilogue of one accumulator tile: the warp owns TMEM lanes 32q..32q+31
 // (output rows m0 + 32q + lane) of the accumulator at column `tacc`, and its
 // 16-column chunks ch0, ch0 + chs, ...
+//
+// The accumulator comes from tensor memory, or (split tile: parts != null)
+// is the sum, in slice order, of nparts fp32 partials stored column-major
+// ([256 columns][128 rows] per CTA, slices 2 * 32768 floats apart).
+constexpr int SK_HALF = 256 * 128;  // floats of one CTA's partial
+__device__ __forceinline__ void acc_ld16(uint32_t taddr, int c, uint32_t (&v)[16], const float* parts, int nparts,
+                                         int prow) {
+  if (!parts) {
+    ptx::tmem_ld16(taddr + c, v);
+    ptx::tmem_ld_wait();
+    return;
+  }
+  float a[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a[i] = 0.f;
+  for (int z = 0; z < nparts; ++z) {
+    const float* pz = parts + (size_t)z * 2 * SK_HALF + (size_t)c * 128 + prow;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] += __ldcg(pz + i * 128);
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(a[i]);
+}
+
 template <int BN>
 __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uint32_t tacc, int m0, int n0, int nb,
-                                              int q, int lane, int ch0, int chs) {
+                                              int q, int lane, int ch0, int chs, const float* parts = nullptr,
+                                              int nparts = 0) {
   const uint32_t trow = tacc + ((uint32_t)(q * 32) << 16);
+  const int prow = q * 32 + lane;
   const int row = m0 + q * 32 + lane;
   const bool row_ok = row < args.M;
   constexpr int NCH = BN / 16;
@@ -239,9 +278,8 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
     const int I = args.swiglu_I;
     for (int ch = ch0; ch < NCH / 2; ch += chs) {
       uint32_t vg[16], vu[16];
-      ptx::tmem_ld16(trow + ch * 16, vg);
-      ptx::tmem_ld16(trow + (ch + NCH / 2) * 16, vu);
-      ptx::tmem_ld_wait();
+      acc_ld16(trow, ch * 16, vg, parts, nparts, prow);
+      acc_ld16(trow, (ch + NCH / 2) * 16, vu, parts, nparts, prow);
       const int n = nb + ch * 16;
       if (!row_ok || n >= I) continue;
       float a[16], gg[16], uu[16];
@@ -264,9 +302,8 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
     for (int ch = ch0; ch < NCH; ch += chs) {
       if ((ch & 7) >= 4) continue;
       uint32_t v0[16], v1[16];
-      ptx::tmem_ld16(trow + ch * 16, v0);
-      ptx::tmem_ld16(trow + (ch + 4) * 16, v1);
-      ptx::tmem_ld_wait();
+      acc_ld16(trow, ch * 16, v0, parts, nparts, prow);
+      acc_ld16(trow, (ch + 4) * 16, v1, parts, nparts, prow);
       const int n = n0 + ch * 16;
       if (!row_ok || n >= args.N) continue;
       int pos = row % args.rope_S;
@@ -291,8 +328,7 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
   } else {
     for (int ch = ch0; ch < NCH; ch += chs) {
       uint32_t v[16];
-      ptx::tmem_ld16(trow + ch * 16, v);
-      ptx::tmem_ld_wait();
+      acc_ld16(trow, ch * 16, v, parts, nparts, prow);
       const int n = n0 + ch * 16;
       if (!row_ok || n >= args.N) continue;
       float f[16];
@@ -951,6 +987,33 @@ struct PairTile {
   int m0, n0, nb, tail_row;
 };
 
+// A pair's j-th work item: a whole tile, or (last partial round split along
+// K) k-blocks [kb0, kb1) of a leftover tile; unit >= 0 for a slice.
+struct PairItem {
+  int t, kb0, kb1, unit;
+};
+__device__ __forceinline__ int pair_items(const KArgs& a, int pair, int npairs, int ntiles_total) {
+  if (a.sk_k > 1) return a.sk_full + (pair < a.sk_units ? (a.sk_units - pair + npairs - 1) / npairs : 0);
+  return pair < ntiles_total ? (ntiles_total - pair + npairs - 1) / npairs : 0;
+}
+__device__ __forceinline__ PairItem pair_item(const KArgs& a, int j, int pair, int npairs) {
+  PairItem w;
+  if (a.sk_k > 1 && j >= a.sk_full) {
+    const int u = pair + (j - a.sk_full) * npairs;
+    const int z = u % a.sk_k;
+    w.t = a.sk_full * npairs + u / a.sk_k;
+    w.kb0 = (int)((long long)z * a.num_kb / a.sk_k);
+    w.kb1 = (int)((long long)(z + 1) * a.num_kb / a.sk_k);
+    w.unit = u;
+  } else {
+    w.t = pair + j * npairs;
+    w.kb0 = 0;
+    w.kb1 = a.num_kb;
+    w.unit = -1;
+  }
+  return w;
+}
+
 __device__ __forceinline__ PairTile pair_tile(const KArgs& args, int t, int mtiles, uint32_t rank) {
   constexpr int BN = 256;
   PairTile p;
@@ -993,16 +1056,22 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
   uint64_t* cfull = empty + STAGES;
   uint64_t* acc_full = cfull + STAGES;   // [2] MMA of a tile done (both CTAs, multicast commit)
   uint64_t* acc_empty = acc_full + 2;    // [2] even CTA: both CTAs' epilogues drained the buffer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* sk_done = acc_empty + 2;     // split slice: the 8 epilogue warps stored their partial
+  uint64_t* sk_go = sk_done + 1;         // split slice: whether this CTA sums the tile was decided
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sk_go + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* sk_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = ptx::cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int num_kb = args.num_kb;
-  const int n_iters = num_kb + (args.tail_ksteps > 0 ? 1 : 0);
   const bool paired = args.pair_off > 0;
+  const int nitems = pair_items(args, pair, npairs, ntiles_total);
+  // iterations of an item: its k-blocks, plus the LoRA tail step for the
+  // item that ends the tile's K range
+  auto item_end = [&](const PairItem& w) { return w.kb1 + ((args.tail_ksteps > 0 && w.kb1 == num_kb) ? 1 : 0); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -1014,6 +1083,8 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
       ptx::mbar_init(&acc_full[b], 1);
       ptx::mbar_init(&acc_empty[b], 16);
     }
+    ptx::mbar_init(sk_done, 8);
+    ptx::mbar_init(sk_go, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmA);
@@ -1047,11 +1118,13 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
       const uint32_t full0 = ptx::mapa_shared(ptx::smem_u32(full), 0);
       int gi = 0;
       bool ok = true;
-      for (int t = pair; t < ntiles_total && ok; t += npairs) {
-        const PairTile tl = pair_tile(args, t, mtiles, rank);
+      for (int j = 0; j < nitems && ok; ++j) {
+        const PairItem wi = pair_item(args, j, pair, npairs);
+        const PairTile tl = pair_tile(args, wi.t, mtiles, rank);
         const int r0 = paired ? (rank == 0 ? tl.nb : args.pair_off + tl.nb) : tl.n0 + (int)rank * 128;
         const int c0 = tl.n0 + (int)rank * 128;
-        for (int it = 0; it < n_iters; ++it, ++gi) {
+        const int it_end = item_end(wi);
+        for (int it = wi.kb0; it < it_end; ++it, ++gi) {
           const int s = gi % STAGES;
           const uint32_t ph = (gi / STAGES) & 1;
           if (!ptx::mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
@@ -1127,7 +1200,9 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
       constexpr uint32_t idesc_half = ptx::idesc_bf16(2 * BM, BN / 2, 1, B_MN ? 1 : 0);
       int gi = 0, lt = 0;
       bool ok = true;
-      for (int t = pair; t < ntiles_total && ok; t += npairs, ++lt) {
+      for (int j = 0; j < nitems && ok; ++j, ++lt) {
+        const PairItem wi = pair_item(args, j, pair, npairs);
+        const int it_end = item_end(wi);
         const int ab = lt & 1;
         if (!ptx::mbar_wait_bounded(&acc_empty[ab], ((lt >> 1) & 1) ^ 1, abort_flag)) {
           atomicOr(args.err, 1);
@@ -1136,7 +1211,7 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
         }
         ptx::tc_fence_after();
         const uint32_t tacc = tmem + (uint32_t)(ab * BN);
-        for (int it = 0; it < n_iters; ++it, ++gi) {
+        for (int it = wi.kb0; it < it_end; ++it, ++gi) {
           const int s = gi % STAGES;
           const uint32_t ph = (gi / STAGES) & 1;
           if (!ptx::mbar_wait_bounded(&full[s], ph, abort_flag)) {
@@ -1163,7 +1238,7 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
                                        : ptx::smem_desc_sw128(a_base + k * 32, 16, 1024);
               const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k * KSTEP_MN, CHUNK_BYTES, 1024)
                                        : ptx::smem_desc_sw128(b_base + k * 32, 16, 1024);
-              ptx::mma_bf16_pair(tacc, ad, bd, tail ? idesc_tail : idesc_main, (it > 0 || k > 0) ? 1u : 0u);
+              ptx::mma_bf16_pair(tacc, ad, bd, tail ? idesc_tail : idesc_main, (it > wi.kb0 || k > 0) ? 1u : 0u);
               if (DUAL && !tail)
                 ptx::mma_bf16_pair(tacc, ptx::smem_desc_sw128(a_base + A_STAGE_BYTES + k * 32, 16, 1024), bd,
                                    idesc_main, 1u);
@@ -1184,8 +1259,10 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
     const uint8_t* lutb = smem_raw;
     int gi = 0;
     bool ok = true;
-    for (int t = pair; t < ntiles_total && ok; t += npairs) {
-      const PairTile tl = pair_tile(args, t, mtiles, rank);
+    for (int j = 0; j < nitems && ok; ++j) {
+      const PairItem wi = pair_item(args, j, pair, npairs);
+      const PairTile tl = pair_tile(args, wi.t, mtiles, rank);
+      const int it_end = item_end(wi);
       int srow, unit0, chunk, coff, soff;
       bool valid;
       if constexpr (BMD == B_NF4_K) {
@@ -1208,7 +1285,7 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
         soff = kr * 4 + ((tl.n0 + (int)rank * 128) / 64 & 3) + (q >> 1);
       }
       uint8_t* const drow = sB + chunk * 8192 + srow * 128;
-      for (int it = 0; it < n_iters; ++it, ++gi) {
+      for (int it = wi.kb0; it < it_end; ++it, ++gi) {
         const int s = gi % STAGES;
         const uint32_t ph = (gi / STAGES) & 1;
         // cfull completes once per use of the slot (the tail stage arrives without bytes)
@@ -1244,9 +1321,10 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
     // the even CTA
     const int q = warp & 3, ew = warp - 10;
     const uint32_t acc_empty0 = ptx::mapa_shared(ptx::smem_u32(acc_empty), 0);
-    int lt = 0;
-    for (int t = pair; t < ntiles_total; t += npairs, ++lt) {
-      const PairTile tl = pair_tile(args, t, mtiles, rank);
+    int lt = 0, ns = 0;  // ns: slices handled (phase of sk_done / sk_go)
+    for (int j = 0; j < nitems; ++j, ++lt) {
+      const PairItem wi = pair_item(args, j, pair, npairs);
+      const PairTile tl = pair_tile(args, wi.t, mtiles, rank);
       const int ab = lt & 1;
       if (!ptx::mbar_wait_bounded(&acc_full[ab], (lt >> 1) & 1, abort_flag)) {
         atomicOr(args.err, 1);
@@ -1254,10 +1332,70 @@ __global__ void __launch_bounds__(PERSIST_THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
-      epilogue_tile<BN>(args, args.out, tmem + (uint32_t)(ab * BN), tl.m0, tl.n0, tl.nb, q, lane, ew / 4, 2);
+      const uint32_t tacc = tmem + (uint32_t)(ab * BN);
+      if (wi.unit < 0) {
+        epilogue_tile<BN>(args, args.out, tacc, tl.m0, tl.n0, tl.nb, q, lane, ew / 4, 2);
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(acc_empty0 + ab * 8);
+        continue;
+      }
+      // ---- k-slice of a split tile: store this CTA's partial (column-major),
+      // free the accumulator, count the slice; the last of the tile's slices
+      // to finish sums all of them (slice order) and runs the epilogue
+      const int u0 = wi.unit - wi.unit % args.sk_k;  // the tile's first slice
+      {
+        float* part = args.sk_ws + ((size_t)wi.unit * 2 + rank) * SK_HALF + q * 32 + lane;
+        const uint32_t trow = tacc + ((uint32_t)(q * 32) << 16);
+        for (int ch = ew / 4; ch < BN / 16; ch += 2) {
+          uint32_t v[16];
+          ptx::tmem_ld16(trow + ch * 16, v);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) __stcg(part + (size_t)(ch * 16 + i) * 128, __uint_as_float(v[i]));
+        }
+      }
+      __threadfence();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive_cluster(acc_empty0 + ab * 8);
+      if (lane == 0) {
+        ptx::mbar_arrive_cluster(acc_empty0 + ab * 8);
+        ptx::mbar_arrive(sk_done);
+      }
+      if (ew == 0 && lane == 0) {
+        int last = 0;
+        if (ptx::mbar_wait_bounded(sk_done, (uint32_t)(ns & 1), abort_flag, args.wait_limit)) {
+          // count this CTA's slice on the tile's (epoch-tagged) counter
+          unsigned long long* cnt = args.sk_cnt + (size_t)(wi.unit / args.sk_k) * 2 + rank;
+          unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(cnt), nw;
+          while (true) {
+            nw = (unsigned int)(old >> 32) == args.sk_epoch ? old + 1
+                                                             : (((unsigned long long)args.sk_epoch << 32) | 1ull);
+            const unsigned long long prev = atomicCAS(cnt, old, nw);
+            if (prev == old) break;
+            old = prev;
+          }
+          last = (int)(nw & 0xFFFFFFFFull) == args.sk_k ? 1 : 0;
+          __threadfence();
+        } else {
+          atomicOr(args.err, 1);
+          *abort_flag = 1;
+          last = -1;
+        }
+        *sk_last = last;
+        ptx::mbar_arrive(sk_go);
+      }
+      if (!ptx::mbar_wait_bounded(sk_go, (uint32_t)(ns & 1), abort_flag, args.wait_limit)) {
+        atomicOr(args.err, 1);
+        *abort_flag = 1;
+        break;
+      }
+      ++ns;
+      if (*sk_last == 1) {
+        __threadfence();
+        epilogue_tile<BN>(args, args.out, tacc, tl.m0, tl.n0, tl.nb, q, lane, ew / 4, 2,
+                          args.sk_ws + ((size_t)u0 * 2 + rank) * SK_HALF, args.sk_k);
+      }
     }
   }
 
@@ -1354,6 +1492,37 @@ soup_status make_plain_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_
 }
 constexpr int CU_DT_U8 = 0;  // CU_TENSOR_MAP_DATA_TYPE_UINT8
 
+// Per-device slice counters of the persistent kernel's split last round
+// (one per leftover tile and CTA of the pair, tagged with a launch-unique
+// epoch, so none ever needs clearing).
+constexpr int SK_MAX_TILES = 128;
+__device__ __align__(256) unsigned long long g_sk_cnt[2 * SK_MAX_TILES];
+std::atomic<unsigned int> g_sk_epoch{0};
+
+// The split of the last partial round: leftover tiles L after the full
+// rounds on P pairs are cut into k slices (2 <= k <= 8, >= 64 k-blocks
+// each: a slice pays a pipeline fill, a 128 KB partial store per CTA and
+// its share of the sums) handed round-robin to the pairs; picked to
+// minimise the rounds the leftover then takes, ceil(L k / P) / k of a tile,
+// if that saves at least a tenth of a tile and the partials (L k x 256 KB)
+// fit the scratch.
+int pick_split(int total, int P, int num_kb, size_t scratch_bytes) {
+  const int F = total / P, L = total - F * P;
+  if (L == 0 || L > SK_MAX_TILES) return 0;
+  int best = 0;
+  double best_cost = 0.9;
+  for (int k = 2; k <= 8; ++k) {
+    if (num_kb / k < 64) break;
+    if ((size_t)L * k * 2 * 256 * 128 * sizeof(float) > scratch_bytes) break;
+    const double cost = (double)((L * k + P - 1) / P) / k + 0.01 * k;  // + a little per slice for the sums
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = k;
+    }
+  }
+  return best;
+}
+
 template <int BN, int AMJ, int BMD, bool TF = false, bool DUAL = false, int CG = 1, bool PERSIST = false>
 soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
   static_assert(!PERSIST || (CG == 2 && BN == 256 && AMJ == A_K && !TF), "persistent: CTA pairs, K-major A");
@@ -1421,7 +1590,24 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
     const int mtiles = (d.M + 2 * BM - 1) / (2 * BM);
     const int ntiles = paired ? d.pair_off / (BN / 2) : (d.N + BN - 1) / BN;
     const int total = mtiles * ntiles;
-    const int npairs = std::min(total, max_pairs);
+    int npairs = std::min(total, max_pairs);
+    KArgs kx = ka;
+    kx.sk_k = 0;
+    if (d.sk_scratch && d.sk_scratch_bytes > 0 && soup_aligned(d.sk_scratch, 16)) {
+      const int k = pick_split(total, max_pairs, ka.num_kb, d.sk_scratch_bytes);
+      if (k >= 2) {
+        void* cnt = nullptr;
+        SOUP_TRY(static_symbol_address(SYM_SPLIT_COUNTERS, reinterpret_cast<const void*>(g_sk_cnt), &cnt));
+        const int F = total / max_pairs;
+        kx.sk_full = F;
+        kx.sk_units = (total - F * max_pairs) * k;
+        kx.sk_k = k;
+        kx.sk_ws = static_cast<float*>(d.sk_scratch);
+        kx.sk_cnt = static_cast<unsigned long long*>(cnt);
+        kx.sk_epoch = g_sk_epoch.fetch_add(1) + 1;
+        npairs = F > 0 ? max_pairs : std::min(kx.sk_units, max_pairs);
+      }
+    }
     cfg.gridDim = dim3(2 * npairs);
     if (profiling()) {
       const int cls = BMD < B_NF4_K ? GC_BF16
@@ -1433,7 +1619,7 @@ soup_status launch(const GemmDesc& d, const KArgs& ka, cudaStream_t st) {
                            (double)d.M * d.N * ((d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T) ? 4 : 2);
       profile_begin(st, cls, flops, bytes);
     }
-    SOUP_CUDA_TRY(cudaLaunchKernelEx(&cfg, kp, mA, mB, mTA, mTB, mA2, mA3, ka, mtiles, total));
+    SOUP_CUDA_TRY(cudaLaunchKernelEx(&cfg, kp, mA, mB, mTA, mTB, mA2, mA3, kx, mtiles, total));
     SOUP_LAUNCH_CHECK();
     profile_end(st);
     return SOUP_OK;
@@ -1581,6 +1767,8 @@ soup_status dispatch(const GemmDesc& d, const KArgs& ka, int bn, cudaStream_t st
 }
 
 }  // namespace
+
+size_t gemm_static_device_bytes() { return sizeof(g_sk_cnt); }
 
 soup_status gemm(const GemmDesc& d, cudaStream_t st) {
   SOUP_CHECK(d.M > 0 && d.N > 0 && d.K > 0, SOUP_ERR_SHAPE, "gemm: empty problem %dx%dx%d", d.M, d.N, d.K);

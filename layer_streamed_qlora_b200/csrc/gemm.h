@@ -98,6 +98,11 @@ struct GemmDesc {
   // epilogue of one tile overlaps the next tile's main loop) or one tile
   // per pair
   bool persistent = true;
+  // Persistent kernel: scratch for the fp32 partials of a split last round
+  // of tiles (256 KB per slice; null: whole tiles only).  Device memory
+  // that nothing else uses during the call.
+  void* sk_scratch = nullptr;
+  size_t sk_scratch_bytes = 0;
   // Optional split-K for skinny GEMMs (N <= 64, TMA operands, plain store
   // epilogue): when a workspace is given and the M x N tiles alone cannot
   // fill the GPU, the K range is cut into up to 8 slices whose fp32 partial

@@ -171,6 +171,13 @@ soup_status check_weights(const soup_layer_weights* W, const Dims& m) {
 #define P(off) (reinterpret_cast<uint16_t*>(FIELD(off)))
 #define PF(off) (reinterpret_cast<float*>(FIELD(off)))
 
+// Device memory a big GEMM may use for the partials of its split last
+// round of tiles (nothing else reads or writes it during the call).
+struct Scratch {
+  void* p = nullptr;
+  size_t bytes = 0;
+};
+
 // y = x W^T (+ tail u B^T) (+ resid) into out [T, N]
 struct ProjOpts {
   int out_kind = OUT_BF16;
@@ -183,6 +190,7 @@ struct ProjOpts {
   int swiglu_I = 0;          // > 0: paired gate|up tiles with the SwiGLU epilogue
   uint16_t* aux16 = nullptr; // SwiGLU: fp16 g | u output (may be null)
   const uint16_t* x_lo = nullptr;  // dual-A: bf16 rounding residual of x
+  Scratch sk;
 };
 
 soup_status proj_fwd(const soup_weight* W, const uint16_t* x, int T, const uint16_t* u, int64_t ldT, int u_rows,
@@ -204,6 +212,7 @@ soup_status proj_fwd(const soup_weight* W, const uint16_t* x, int T, const uint1
   g.resid = o.resid; g.resid_f32 = o.resid_f32; g.ldr = W->out_features;
   g.rope_cols = o.rope_cols; g.rope_S = o.rope_S; g.rope_cos = o.rope_cos; g.rope_sin = o.rope_sin;
   g.rope_prefix = o.rope_prefix; g.rope_group = o.rope_group;
+  g.sk_scratch = o.sk.p; g.sk_scratch_bytes = o.sk.bytes;
   if (o.swiglu_I > 0) {
     g.pair_off = o.swiglu_I;
     g.nseg = 1;
@@ -343,8 +352,9 @@ soup_status lora_dA_tf32(const float* x, int T, int K, const float* g32, int row
 soup_status proj_bwd(const soup_weight* W, const uint16_t* dy, int T, const uint16_t* gt, int64_t ldT, int g_rows,
                      const uint16_t* Al, bool on, uint16_t* dx, cudaStream_t st, int out_kind = OUT_BF16,
                      int swiglu_I = 0, uint16_t* aux16 = nullptr, const unsigned int* scale_amax = nullptr,
-                     const uint16_t* dy_lo = nullptr, uint16_t* out_lo = nullptr) {
+                     const uint16_t* dy_lo = nullptr, uint16_t* out_lo = nullptr, Scratch sk = Scratch()) {
   GemmDesc g;
+  g.sk_scratch = sk.p; g.sk_scratch_bytes = sk.bytes;
   g.scale_amax = scale_amax;
   g.out_lo = out_lo;
   if (dy_lo) g.A_lo = Mat{dy_lo, T, W->out_features, W->out_features};
@@ -409,6 +419,9 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
                     bool want_out, cudaStream_t st, uint16_t* keep = nullptr, const uint16_t* kept = nullptr) {
   const int T = m.T, r = m.r;
   const SplitWS SW{PF(splitk), ws.splitk_bytes};
+  // the backward's d_gu residual field is unused during a forward pass or
+  // recompute: the big GEMMs' split last round keeps its partials there
+  const Scratch SK{base + ws.d_gu_lo, (size_t)T * 2 * m.I * 2};
   SOUP_TRY(rope_table(m.S, m.d, (double)c->theta, PF(cosb), PF(sinb), st));
   const bool precise_qkv = (save && !kept) || keep;  // q|k|v from the hi + lo x1 pair
   SOUP_TRY(rmsnorm_fwd(h_in, nullptr, W->norm1, T, m.H, c->eps, P(x1), PF(rinv1), st, on ? PF(x1_32) : nullptr,
@@ -437,6 +450,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     // attention backward amplifies the bf16 rounding of x1 into the q/k/v
     // adapter gradients
     if (precise_qkv) o.x_lo = P(x1_lo);
+    o.sk = SK;
     if (!kept)
       SOUP_TRY(proj_fwd(&W->qkv, P(x1), T, P(u_qkv), m.ldT, 3 * r, L ? L->B_qkv : nullptr, r, 3, se, sr, on,
                         keep ? keep : P(qkv), st, o));
@@ -453,6 +467,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     ProjOpts o;
     o.out_kind = OUT_F32;  // h2 = h + o kept in fp32
     o.resid = h_in;
+    o.sk = SK;
     SOUP_TRY(proj_fwd(&W->o, P(attn), T, P(u_o), m.ldT, r, L ? L->B_o : nullptr, r, 1, se, sr, on,
                       reinterpret_cast<uint16_t*>(PF(h2)), st, o));
   }
@@ -467,6 +482,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     ProjOpts o;
     o.swiglu_I = m.I;
     o.aux16 = save ? P(gu16) : nullptr;  // g | u are needed only by the backward
+    o.sk = SK;
     SOUP_TRY(proj_fwd(&W->gate_up, P(x2), T, P(u_gu), m.ldT, 2 * r, L ? L->B_gu : nullptr, r, 1, se, sr, on,
                       P(act), st, o));
   }
@@ -476,6 +492,7 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     const int sr[1] = {0};
     ProjOpts o;
     o.resid_f32 = PF(h2);
+    o.sk = SK;
     SOUP_TRY(proj_fwd(&W->down, P(act), T, P(u_d), m.ldT, r, L ? L->B_down : nullptr, r, 1, se, sr, on, h_out, st,
                       o));
   }
@@ -636,8 +653,11 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
     SOUP_TRY(mark(0));
   }
   // d_gu = SwiGLU backward of (dh W_down + g' A_down), fused in the epilogue
+  // split-round partials: in dx2 for the down product (it writes d_gu's
+  // residual), then in that residual, which nothing reads after g_gu
+  const Scratch SK_dx2{P(dx2), (size_t)T * H * 2}, SK_lo{P(d_gu_lo), (size_t)T * 2 * I * 2};
   SOUP_TRY(proj_bwd(&W->down, P(dh_b), T, P(g_d), ldT, r, on ? L->A_down : nullptr, on, P(d_gu), st, OUT_BF16, I,
-                    P(gu16), nullptr, nullptr, on ? P(d_gu_lo) : nullptr));
+                    P(gu16), nullptr, nullptr, on ? P(d_gu_lo) : nullptr, SK_dx2));
   if (on) {
     SOUP_TRY(mark(1));
     SOUP_TRY(after(0));
@@ -650,7 +670,8 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
                              nullptr, ldT, st, SW));
     SOUP_TRY(mark(2));
   }
-  SOUP_TRY(proj_bwd(&W->gate_up, d_gu, T, P(g_gu), ldT, 2 * r, on ? L->A_gu : nullptr, on, P(dx2), st));
+  SOUP_TRY(proj_bwd(&W->gate_up, d_gu, T, P(g_gu), ldT, 2 * r, on ? L->A_gu : nullptr, on, P(dx2), st, OUT_BF16, 0,
+                    nullptr, nullptr, nullptr, nullptr, SK_lo));
   if (on) {
     SOUP_TRY(after(1));
     for (int sg = 0; sg < 2; ++sg)
@@ -673,7 +694,7 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
   // dO for the attention backward: from the fp32-accurate dh2 (hi + lo parts),
   // stored fp16 scaled by a power of two derived from max |dh2|
   SOUP_TRY(proj_bwd(&W->o, P(dh2_b), T, P(g_o), ldT, r, on ? L->A_o : nullptr, on, P(d_attn), st, OUT_F16, 0,
-                    nullptr, gamax, P(dh2_lo)));
+                    nullptr, gamax, P(dh2_lo), nullptr, SK_lo));
   if (on) {
     SOUP_TRY(after(3));
     SOUP_TRY(lora_dB_tf32(PF(dh2), H, T, H, PF(uo32), r, ldT, G->dB_o, s2, SW2));
@@ -690,7 +711,8 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
                              PF(g32), nullptr, ldT, st, SW));
     SOUP_TRY(mark(4));
   }
-  SOUP_TRY(proj_bwd(&W->qkv, P(d_qkv), T, P(g_qkv), ldT, 3 * r, on ? L->A_qkv : nullptr, on, P(dx1), st));
+  SOUP_TRY(proj_bwd(&W->qkv, P(d_qkv), T, P(g_qkv), ldT, 3 * r, on ? L->A_qkv : nullptr, on, P(dx1), st, OUT_BF16, 0,
+                    nullptr, nullptr, nullptr, nullptr, SK_lo));
   if (on) {
     SOUP_TRY(after(4));
     for (int sg = 0; sg < 3; ++sg)

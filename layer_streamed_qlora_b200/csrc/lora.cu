@@ -196,7 +196,7 @@ static __device__ __align__(256) uint8_t g_lora_noalloc_scratch[SOUP_NOALLOC_SCR
 
 extern "C" size_t soup_lora_linear_bwd_noalloc_max_scratch(void) { return SOUP_NOALLOC_SCRATCH_BYTES; }
 
-extern "C" size_t soup_static_device_bytes(void) { return SOUP_NOALLOC_SCRATCH_BYTES; }
+extern "C" size_t soup_static_device_bytes(void) { return SOUP_NOALLOC_SCRATCH_BYTES + gemm_static_device_bytes(); }
 
 extern "C" soup_status soup_lora_linear_bwd_noalloc(const soup_weight* W, const uint16_t* A, const uint16_t* B,
                                                     int32_t r, float scale, const uint16_t* x,

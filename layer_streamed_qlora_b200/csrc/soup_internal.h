@@ -30,8 +30,12 @@ int* device_error_word();
 // driver entry point is unavailable).
 void* current_context();
 
-enum StaticSym : int { SYM_DEVICE_ERROR = 0, SYM_NOALLOC_SCRATCH = 1, SYM_N = 2 };
+enum StaticSym : int { SYM_DEVICE_ERROR = 0, SYM_NOALLOC_SCRATCH = 1, SYM_SPLIT_COUNTERS = 2, SYM_N = 3 };
 soup_status static_symbol_address(int which, const void* symbol, void** out);
+
+// Bytes of module-static device arrays held by the GEMM engine (the slice
+// counters of its split last round).
+size_t gemm_static_device_bytes();
 
 
 // cuTensorMapEncodeTiled resolved through the runtime's driver entry point.
