@@ -679,7 +679,7 @@ def main():
         "config": dict(bench_config(w, args.workload, world, sum(1 for k in model.keep_plan if k == "qkv"),
                                     sum(1 for k in model.keep_plan if k == "saved"), args.recompute),
                        token_rows_per_step=model.T, prompt_dedup=model.prompt_dedup,
-                       stream_source=args.source,
+                       head_chunk=model.head_chunk, stream_source=args.source,
                        **({"read_ahead": args.read_ahead} if args.source == "disk" else {})),
         "e2e": {"value": tokens / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": ids_host.numel() * 4,
                 "d2h_bytes_per_step": 4},

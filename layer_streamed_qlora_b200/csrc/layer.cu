@@ -394,6 +394,8 @@ struct SideStream {
   void* ctx = nullptr;
   cudaStream_t st = nullptr;
   cudaEvent_t ev[6] = {};
+  std::mutex issue;  // held while one layer call issues its work: calls from
+                     // several threads then share the side stream in turn
 };
 SideStream g_side[64];
 std::mutex g_side_mu;
@@ -631,6 +633,8 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
   // the next big GEMM, so that GEMM's CTAs are dispatched first
   SideStream* side = nullptr;
   if (on) SOUP_TRY(side_stream(&side));
+  std::unique_lock<std::mutex> issue_lock;
+  if (side) issue_lock = std::unique_lock<std::mutex>(side->issue);
   const SplitWS SW2{PF(splitk2), ws.splitk_bytes};
   cudaStream_t s2 = side ? side->st : st;
   auto mark = [&](int e) -> soup_status {  // the side stream may consume what st has produced so far

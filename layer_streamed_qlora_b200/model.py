@@ -263,7 +263,7 @@ class StreamedLoRAModel:
     """
 
     def __init__(self, cfg: ModelConfig, batch: int, seq: int, n_buffers: int = 2, device_cap_bytes: int = 0,
-                 head_chunk: int = 256, weights=None, seed: int = 0, adamw: AdamW | None = None,
+                 head_chunk="auto", weights=None, seed: int = 0, adamw: AdamW | None = None,
                  task: str = "sft", stream_source: str = "ram", shard_dir: str | None = None,
                  read_ahead: int = 2, io_threads: int = 4, stream_recompute: str = "auto", prompt_dedup: int = 0):
         self.cfg, self.batch, self.seq, self.n_buffers = cfg, batch, seq, n_buffers
@@ -293,9 +293,16 @@ class StreamedLoRAModel:
         # the output head reads, per sequence, head_seq consecutive positions
         # (with a shared prompt: the last prompt position and the continuation)
         self.head_seq = seq - self.prompt_dedup + 1 if self.prompt_dedup else seq
-        self.head_chunk = head_chunk
         self.lcfg = cfg.layer_cfg(self.prompt_dedup)
-        precheck_device_bytes(cfg, batch, seq, n_buffers, head_chunk, device_cap_bytes, self.prompt_dedup)
+        if head_chunk == "auto":
+            # the most token rows per head chunk whose workspace still fits in
+            # the layer workspace (which it shares): fewer, larger logits and
+            # dx GEMMs at no extra device memory
+            lw = L.soup_decoder_layer_workspace(self.lcfg, batch, seq)
+            head_chunk = next((c for c in (1024, 512, 256) if
+                               L.soup_head_workspace(cfg.vocab, cfg.hidden, batch, self.head_seq, c) <= lw), 128)
+        self.head_chunk = int(head_chunk)
+        precheck_device_bytes(cfg, batch, seq, n_buffers, self.head_chunk, device_cap_bytes, self.prompt_dedup)
         weights = weights or SyntheticWeights(cfg, seed)
         # the model's resident tensors first, the shard build's temporaries
         # after them: freed temporaries then leave whole cached segments that

@@ -44,6 +44,16 @@ def test_llama8b_layer_seq2048_matches_oracle(kind):
     torch.cuda.synchronize()
     got_out, got_dh = host(out).reshape(h.shape), host(dhi).reshape(h.shape)
     got = dl.split_grads()
+    # the same backward again gives the same bits (the dA / dB GEMMs on the
+    # side stream, the gate|up W^T product's split last round summed by
+    # whichever slice finishes last: neither may change the result)
+    g1 = {k: v.clone() for k, v in dl.grads_t.items()}
+    dhi2 = torch.empty_like(dho)
+    L.soup_decoder_layer_bwd(dl.W, dl.lora, dl.cfg, hd, dho, B, S, dhi2, dl.grads, 1, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(dhi, dhi2)
+    for k in g1:
+        assert torch.equal(g1[k], dl.grads_t[k]), k
     del ws
     ref, cache = layer_fwd(h, dl.Wd, dl.lora_np, shape)
     assert_close(got_out, ref, "h_out")
