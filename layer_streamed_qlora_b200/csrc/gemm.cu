@@ -125,14 +125,38 @@ __device__ __forceinline__ float f16_to_f32(uint16_t b) {
   return __half2float(__ushort_as_half(b));
 }
 
+// 32-byte global accesses (sm_100 vector width): one instruction moves a
+// row's 16 16-bit values, where two 16-byte ones would each touch the same
+// 32 rows of a warp.  The caller guarantees 32-byte alignment.
+__device__ __forceinline__ void st_global_32B(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+__device__ __forceinline__ void ld_global_32B(const void* p, uint32_t (&w)[8]) {
+  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+               : "l"(p)
+               : "memory");
+}
+
 // Stores 16 consecutive values of one row (row-major 16-bit or fp32 output),
-// vectorised when the whole chunk is in range and aligned.
+// vectorised when the whole chunk is in range and aligned (vec: 0 scalar,
+// 1 16-byte, 2 32-byte accesses).
 __device__ __forceinline__ void store_row16(void* out, int out_kind, long long ldo, int row, int n, int N,
-                                            const float (&f)[16], bool vec) {
+                                            const float (&f)[16], int vec) {
   const bool full = vec && (n + 16 <= N);
   if (out_kind == OUT_F32) {
     float* o = static_cast<float*>(out) + (size_t)row * ldo + n;
-    if (full) {
+    if (full && vec == 2) {
+      uint32_t w[8];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(f[8 * h + i]);
+        st_global_32B(o + 8 * h, w);
+      }
+    } else if (full) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         reinterpret_cast<float4*>(o)[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
@@ -149,8 +173,12 @@ __device__ __forceinline__ void store_row16(void* out, int out_kind, long long l
     uint32_t p[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) p[i] = h ? pack_f16x2(f[2 * i], f[2 * i + 1]) : pack_bf16x2(f[2 * i], f[2 * i + 1]);
-    reinterpret_cast<uint4*>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
-    reinterpret_cast<uint4*>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+    if (vec == 2) {
+      st_global_32B(o, p);
+    } else {
+      reinterpret_cast<uint4*>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
+      reinterpret_cast<uint4*>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+    }
   } else {
 #pragma unroll
     for (int i = 0; i < 16; ++i)
@@ -161,10 +189,28 @@ __device__ __forceinline__ void store_row16(void* out, int out_kind, long long l
   }
 }
 
-__device__ __forceinline__ void load16_u16(const uint16_t* p, uint16_t (&v)[16]) {
-  const uint4 a = *reinterpret_cast<const uint4*>(p);
-  const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+// 16 consecutive 16-bit values as 8 packed words (element 2i in the low half)
+__device__ __forceinline__ void load8_u32(const uint16_t* p, uint32_t (&w)[8], int vec) {
+  if (vec == 2) {
+    ld_global_32B(p, w);
+  } else {
+    const uint4 a = *reinterpret_cast<const uint4*>(p);
+    const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ void load16_u16(const uint16_t* p, uint16_t (&v)[16], int vec) {
+  uint32_t w[8];
+  if (vec == 2) {
+    ld_global_32B(p, w);
+  } else {
+    const uint4 a = *reinterpret_cast<const uint4*>(p);
+    const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     v[2 * i] = static_cast<uint16_t>(w[i] & 0xFFFF);
@@ -271,7 +317,7 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
   constexpr int NCH = BN / 16;
   const float alpha =
       args.scale_amax ? args.alpha * grad_scale_from_amax(__uint_as_float(*args.scale_amax)) : args.alpha;
-  const bool vec = args.vec_ok != 0;
+  const int vec = args.vec_ok;
   if (args.epi == EPI_SWIGLU) {
     // paired gate|up tile: chunk c (gate) pairs with c + NCH/2 (up); both
     // owned by this warp (NCH/2 is even)
@@ -325,6 +371,53 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
       store_row16(outp, args.out_kind, args.ldo, row, n, args.N, a, vec);
       store_row16(outp, args.out_kind, args.ldo, row, n + 64, args.N, b, vec);
     }
+  } else if (args.epi == EPI_SWIGLU_BWD) {
+    // acc = dL/d(act); g, u from the forward (fp16); out = [dL/dg | dL/du]
+    // bf16 (+ rounding residuals)
+    const int I = args.swiglu_I;
+    for (int ch = ch0; ch < NCH; ch += chs) {
+      const int n = n0 + ch * 16;
+      uint32_t v[16];
+      acc_ld16(trow, ch * 16, v, parts, nparts, prow);
+      if (!row_ok || n >= args.N) continue;
+      const bool full16 = vec && (n + 16 <= args.N);
+      uint32_t gw[8], uw[8];  // fp16 pairs (element 2i low)
+      const uint16_t* gp = args.aux16 + (size_t)row * args.ld_aux + n;
+      if (full16) {
+        load8_u32(gp, gw, vec);
+        load8_u32(gp + I, uw, vec);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t g0 = (n + 2 * i < args.N) ? gp[2 * i] : 0, g1 = (n + 2 * i + 1 < args.N) ? gp[2 * i + 1] : 0;
+          const uint32_t u0 = (n + 2 * i < args.N) ? gp[I + 2 * i] : 0,
+                         u1 = (n + 2 * i + 1 < args.N) ? gp[I + 2 * i + 1] : 0;
+          gw[i] = g0 | (g1 << 16);
+          uw[i] = u0 | (u1 << 16);
+        }
+      }
+      float dg[16], du[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float f = __uint_as_float(v[i]) * alpha;
+        const float g = f16_to_f32(static_cast<uint16_t>(gw[i >> 1] >> (16 * (i & 1)))),
+                    u = f16_to_f32(static_cast<uint16_t>(uw[i >> 1] >> (16 * (i & 1))));
+        const float sg = sigmoid_f(g);
+        dg[i] = f * u * sg * (1.0f + g * (1.0f - sg));
+        du[i] = f * g * sg;
+      }
+      store_row16(outp, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
+      store_row16(static_cast<uint16_t*>(outp) + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
+      if (args.out_lo) {  // rounding residuals of both halves, same layout
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          dg[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(dg[i], 0.f) & 0xFFFF));
+          du[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(du[i], 0.f) & 0xFFFF));
+        }
+        store_row16(args.out_lo, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
+        store_row16(args.out_lo + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
+      }
+    }
   } else {
     for (int ch = ch0; ch < NCH; ch += chs) {
       uint32_t v[16];
@@ -335,42 +428,6 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
 #pragma unroll
       for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]) * alpha;
       const bool full16 = vec && (n + 16 <= args.N);
-      if (args.epi == EPI_SWIGLU_BWD) {
-        // f = dL/d(act); g, u from the forward (fp16); out = [dL/dg | dL/du] bf16
-        const int I = args.swiglu_I;
-        uint16_t gb[16], ub[16];
-        const uint16_t* gp = args.aux16 + (size_t)row * args.ld_aux + n;
-        if (full16) {
-          load16_u16(gp, gb);
-          load16_u16(gp + I, ub);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            gb[i] = (n + i < args.N) ? gp[i] : 0;
-            ub[i] = (n + i < args.N) ? gp[I + i] : 0;
-          }
-        }
-        float dg[16], du[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float g = f16_to_f32(gb[i]), u = f16_to_f32(ub[i]);
-          const float sg = sigmoid_f(g);
-          dg[i] = f[i] * u * sg * (1.0f + g * (1.0f - sg));
-          du[i] = f[i] * g * sg;
-        }
-        store_row16(outp, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
-        store_row16(static_cast<uint16_t*>(outp) + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
-        if (args.out_lo) {  // rounding residuals of both halves, same layout
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            dg[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(dg[i], 0.f) & 0xFFFF));
-            du[i] -= bf16_to_f32(static_cast<uint16_t>(pack_bf16x2(du[i], 0.f) & 0xFFFF));
-          }
-          store_row16(args.out_lo, OUT_BF16, args.ldo, row, n, args.N, dg, vec);
-          store_row16(args.out_lo + I, OUT_BF16, args.ldo, row, n, args.N, du, vec);
-        }
-        continue;
-      }
       if (args.out_kind == OUT_BF16_T || args.out_kind == OUT_F32_T) {
         if (args.out_kind == OUT_BF16_T) {
           uint16_t* o = static_cast<uint16_t*>(outp);
@@ -404,7 +461,7 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
         const uint16_t* r = args.resid + (size_t)row * args.ldr + n;
         if (full16) {
           uint16_t rb[16];
-          load16_u16(r, rb);
+          load16_u16(r, rb, vec);
 #pragma unroll
           for (int i = 0; i < 16; ++i) f[i] += bf16_to_f32(rb[i]);
         } else {
@@ -414,7 +471,15 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
         }
       } else if (args.resid_f32) {
         const float* r = args.resid_f32 + (size_t)row * args.ldr + n;
-        if (full16) {
+        if (full16 && vec == 2) {
+          uint32_t w[8];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            ld_global_32B(r + 8 * h, w);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[8 * h + i] += __uint_as_float(w[i]);
+          }
+        } else if (full16) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float4 x = reinterpret_cast<const float4*>(r)[i];
@@ -1815,10 +1880,15 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
   ka.scale_amax = d.scale_amax;
   ka.aux16 = d.aux16; ka.ld_aux = d.ld_aux; ka.swiglu_I = d.swiglu_I;
   const int esz = (d.out_kind == OUT_F32 || d.out_kind == OUT_F32_T) ? 4 : 2;
-  ka.vec_ok = soup_aligned(d.out, 16) && ((d.ldo * esz) % 16 == 0) &&
-              (!d.resid || (soup_aligned(d.resid, 16) && (d.ldr * 2) % 16 == 0)) &&
-              (!d.resid_f32 || (soup_aligned(d.resid_f32, 16) && (d.ldr * 4) % 16 == 0)) &&
-              (!d.aux16 || (soup_aligned(d.aux16, 16) && (d.ld_aux * 2) % 16 == 0 && (d.swiglu_I % 8) == 0));
+  // row-chunk accesses of the epilogue: 32 bytes per instruction where every
+  // row pointer it forms is 32-byte aligned, else 16 bytes, else scalar
+  auto rows_aligned = [&](size_t a) {
+    return soup_aligned(d.out, a) && ((d.ldo * esz) % a == 0) && (!d.out_lo || soup_aligned(d.out_lo, a)) &&
+           (!d.resid || (soup_aligned(d.resid, a) && (d.ldr * 2) % a == 0)) &&
+           (!d.resid_f32 || (soup_aligned(d.resid_f32, a) && (d.ldr * 4) % a == 0)) &&
+           (!d.aux16 || (soup_aligned(d.aux16, a) && (d.ld_aux * 2) % a == 0 && (d.swiglu_I * 2) % a == 0));
+  };
+  ka.vec_ok = rows_aligned(32) ? 2 : (rows_aligned(16) ? 1 : 0);
   ka.wait_limit = d.wait_limit > 0 ? d.wait_limit : 4000000000LL;
   ka.skip_producer = d.debug_skip_producer;
   ka.rope_cols = d.rope_cols; ka.rope_S = d.rope_S;
@@ -1856,7 +1926,7 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
       kz.out_lo = nullptr;
       kz.alpha = 1.f;
       kz.scale_amax = nullptr;
-      kz.vec_ok = 1;
+      kz.vec_ok = (soup_aligned(d.split_ws, 32) && (kz.ldo * 4) % 32 == 0) ? 2 : 1;
       SOUP_TRY(dispatch(d, kz, bn, st));
       const size_t total = (size_t)d.M * d.N;
       const int blocks = (int)std::min<size_t>((total + 255) / 256, (size_t)sms * 8);
