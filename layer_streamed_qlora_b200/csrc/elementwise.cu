@@ -184,7 +184,9 @@ __global__ void attn_rowdot_kernel(const uint16_t* __restrict__ dO, const uint16
   if (lane == 0) D[(size_t)h * T + t] = s;
 }
 
-__global__ void f32_to_bf16_kernel(const float* __restrict__ in, size_t n, uint16_t* __restrict__ out) {
+__global__ void f32_to_bf16_kernel(const float* __restrict__ in, size_t n, uint16_t* __restrict__ out,
+                                   unsigned int* __restrict__ zero_word) {
+  if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0u;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n / 8; i += (size_t)gridDim.x * blockDim.x) {
     const float4 a = reinterpret_cast<const float4*>(in)[2 * i];
     const float4 b = reinterpret_cast<const float4*>(in)[2 * i + 1];
@@ -286,10 +288,10 @@ soup_status attn_rowdot(const uint16_t* dO, const uint16_t* O, int T, int Hq, fl
   return SOUP_OK;
 }
 
-soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t st) {
+soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t st, unsigned int* zero_word) {
   SOUP_CHECK(n % 8 == 0, SOUP_ERR_SHAPE, "f32_to_bf16: n %% 8");
   profile_begin(st, GC_ELEM, 0.0, n * 6.0);
-  f32_to_bf16_kernel<<<grid_for(n / 8, 256), 256, 0, st>>>(in, n, out);
+  f32_to_bf16_kernel<<<grid_for(n / 8, 256), 256, 0, st>>>(in, n, out, zero_word);
   SOUP_LAUNCH_CHECK();
   profile_end(st);
   return SOUP_OK;

@@ -26,7 +26,9 @@ soup_status rope_apply(uint16_t* buf, int T, int S, int ld, int col0, int nh, co
                        bool inverse, cudaStream_t st);
 // D[h, t] = sum_d dO (fp16) * O (fp16)
 soup_status attn_rowdot(const uint16_t* dO, const uint16_t* O, int T, int Hq, float* D, cudaStream_t st);
-soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t st);
+// out = bf16(in) (RNE), n % 8 == 0; zero_word (optional) is set to 0 by the
+// same launch (a counter the next kernels accumulate into).
+soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t st, unsigned int* zero_word = nullptr);
 soup_status bf16_to_f32(const uint16_t* in, size_t n, float* out, cudaStream_t st);
 
 // LoRA operand preparation in one launch (up to 4 jobs):

@@ -647,7 +647,9 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
   };
 
   // ---- MLP block
-  SOUP_TRY(f32_to_bf16(dh_out, (size_t)T * H, P(dh_b), st));
+  // (max |dh2| of the norm2 backward below accumulates into gamax, zeroed here)
+  unsigned int* gamax = reinterpret_cast<unsigned int*>(base + ws.gamax);
+  SOUP_TRY(f32_to_bf16(dh_out, (size_t)T * H, P(dh_b), st, gamax));
   // LoRA gradients of the MLP: g_down from the fp32 dh (tf32), the others
   // from hi + lo (rounding residual) operand pairs, so no operand of a
   // LoRA-gradient GEMM carries more than the bf16 rounding of d_gu
@@ -684,8 +686,6 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
     SOUP_TRY(after(2));
     SOUP_TRY(lora_dA_tf32(PF(x2_32), T, H, PF(g_gu32), 2 * r, ldT, G->dA_gu, s2, SW2));
   }
-  unsigned int* gamax = reinterpret_cast<unsigned int*>(base + ws.gamax);
-  SOUP_CUDA_TRY(cudaMemsetAsync(gamax, 0, sizeof(unsigned int), st));
   SOUP_TRY(rmsnorm_bwd(nullptr, PF(h2), W->norm2, PF(rinv2), P(dx2), dh_out, T, H, PF(dh2), P(dh2_b), st, gamax,
                        P(dh2_lo)));
 
