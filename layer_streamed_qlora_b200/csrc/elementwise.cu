@@ -153,6 +153,95 @@ __global__ void rmsnorm_bwd_kernel(const uint16_t* __restrict__ x, const float* 
   }
 }
 
+// The same backward with one 128-thread CTA per row: every thread loads its
+// (at most CPT) 8-element chunks of x, dy and dres once, up front, and keeps
+// them in registers across the row reduction, so the row streams through
+// memory once with all its loads in flight together.  H / 8 <= 128 * CPT.
+template <int CPT>
+__global__ void __launch_bounds__(128) rmsnorm_bwd_row_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ xf, const uint16_t* __restrict__ w,
+    const float* __restrict__ rinv, const uint16_t* __restrict__ dy, const float* __restrict__ dyf,
+    const float* __restrict__ dres, int T, int H, float* __restrict__ dh, uint16_t* __restrict__ dh_bf16,
+    unsigned int* __restrict__ amax, uint16_t* __restrict__ dh_lo) {
+  __shared__ float red_dot[4], red_max[4];
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int nc = H / 8;
+  const size_t rb = (size_t)row * H;
+  const float r = rinv[row];
+  float a[CPT][8], b[CPT][8], d[CPT][8];
+#pragma unroll
+  for (int k = 0; k < CPT; ++k) {
+    const int c = tid + k * 128;
+    if (c < nc) {
+      const size_t off = rb + (size_t)c * 8;
+      load8(x, xf, off, a[k]);
+      load8(dy, dyf, off, b[k]);
+      if (dres) {
+        const float4 d0 = reinterpret_cast<const float4*>(dres + off)[0];
+        const float4 d1 = reinterpret_cast<const float4*>(dres + off)[1];
+        d[k][0] = d0.x; d[k][1] = d0.y; d[k][2] = d0.z; d[k][3] = d0.w;
+        d[k][4] = d1.x; d[k][5] = d1.y; d[k][6] = d1.z; d[k][7] = d1.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d[k][i] = 0.f;
+      }
+    }
+  }
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  float dot = 0.f;
+#pragma unroll
+  for (int k = 0; k < CPT; ++k) {
+    const int c = tid + k * 128;
+    if (c < nc) {
+      float g[8];
+      unpack8(wr[c], g);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dot += (b[k][i] * g[i]) * (a[k][i] * r);
+    }
+  }
+  dot = warp_sum(dot);
+  if (lane == 0) red_dot[wid] = dot;
+  __syncthreads();
+  dot = ((red_dot[0] + red_dot[1]) + (red_dot[2] + red_dot[3])) / (float)H;
+  float mx = 0.f;
+#pragma unroll
+  for (int k = 0; k < CPT; ++k) {
+    const int c = tid + k * 128;
+    if (c < nc) {
+      float g[8], o[8];
+      unpack8(wr[c], g);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = d[k][i] + r * (b[k][i] * g[i] - (a[k][i] * r) * dot);
+      const size_t base = rb + (size_t)c * 8;
+      reinterpret_cast<float4*>(dh + base)[0] = make_float4(o[0], o[1], o[2], o[3]);
+      reinterpret_cast<float4*>(dh + base)[1] = make_float4(o[4], o[5], o[6], o[7]);
+      if (dh_bf16) {
+        const uint4 hi = pack8(o);
+        reinterpret_cast<uint4*>(dh_bf16 + base)[0] = hi;
+        if (dh_lo) {
+          float oh[8], ol[8];
+          unpack8(hi, oh);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ol[i] = o[i] - oh[i];
+          reinterpret_cast<uint4*>(dh_lo + base)[0] = pack8(ol);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(o[i]));
+    }
+  }
+  if (amax) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) red_max[wid] = mx;
+    __syncthreads();
+    // non-negative floats order like their bit patterns: an integer max is exact and order-independent
+    if (tid == 0)
+      atomicMax(amax, __float_as_uint(fmaxf(fmaxf(red_max[0], red_max[1]), fmaxf(red_max[2], red_max[3]))));
+  }
+}
+
 // cos/sin of pos * theta^(-2i/d), computed in fp64 and rounded to fp32.
 __global__ void rope_table_kernel(int S, int half, double theta, float* __restrict__ cosb, float* __restrict__ sinb) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -248,8 +337,11 @@ soup_status rmsnorm_bwd(const uint16_t* x, const float* x_f32, const uint16_t* w
   profile_begin(st, GC_RMSNORM, 0.0,
                 n * (x_f32 ? 4 : 2) + H * 2.0 + T * 4.0 + n * 2 + (dres ? n * 4 : 0.0) + n * 4 +
                     (dh_bf16 ? n * 2 : 0.0) + (dh_lo ? n * 2 : 0.0));
-  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, rinv, dy, nullptr, dres, T, H, dh, dh_bf16, amax,
-                                                  dh_lo);
+  if (H <= 128 * 8 * 4)
+    rmsnorm_bwd_row_kernel<4><<<T, 128, 0, st>>>(x, x_f32, w, rinv, dy, nullptr, dres, T, H, dh, dh_bf16, amax, dh_lo);
+  else
+    rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, x_f32, w, rinv, dy, nullptr, dres, T, H, dh, dh_bf16, amax,
+                                                    dh_lo);
   SOUP_LAUNCH_CHECK();
   profile_end(st);
   return SOUP_OK;
@@ -258,8 +350,12 @@ soup_status rmsnorm_bwd(const uint16_t* x, const float* x_f32, const uint16_t* w
 soup_status rmsnorm_bwd_f32dy(const uint16_t* x, const uint16_t* w, const float* rinv, const float* dy, int T, int H,
                               float* dh, cudaStream_t st) {
   SOUP_CHECK(H % 256 == 0, SOUP_ERR_SHAPE, "rmsnorm: hidden %d not a multiple of 256", H);
-  rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, nullptr, w, rinv, nullptr, dy, nullptr, T, H, dh, nullptr,
-                                                  nullptr, nullptr);
+  if (H <= 128 * 8 * 4)
+    rmsnorm_bwd_row_kernel<4><<<T, 128, 0, st>>>(x, nullptr, w, rinv, nullptr, dy, nullptr, T, H, dh, nullptr, nullptr,
+                                                 nullptr);
+  else
+    rmsnorm_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(x, nullptr, w, rinv, nullptr, dy, nullptr, T, H, dh, nullptr,
+                                                    nullptr, nullptr);
   SOUP_LAUNCH_CHECK();
   return SOUP_OK;
 }
