@@ -105,6 +105,9 @@ struct AttnArgs {
   const float* rcos;  // [S, 64] or null: rotate dq / dk back
   const float* rsin;
   const unsigned int* amax;  // dO's power-of-two gradient scale, or null
+  // 1: every output pointer (and RoPE table) the epilogues form is 32-byte
+  // aligned, so they move a row's values with 32-byte accesses
+  int v32;
   int* err;
   long long wait_limit;
 };
@@ -135,6 +138,65 @@ __device__ __forceinline__ void attn_teardown(volatile int* abort_flag, int warp
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+// 32 fp32 values -> 32 bf16 (or fp16) at o: 16-byte stores, or 32-byte ones
+// when v32 (o 32-byte aligned).
+template <bool HALF>
+__device__ __forceinline__ void store32_16bit(uint16_t* o, const float (&f)[32], bool v32) {
+  if (v32) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        w[i] = HALF ? pack_h2(f[16 * u + 2 * i], f[16 * u + 2 * i + 1]) : pack_b2(f[16 * u + 2 * i], f[16 * u + 2 * i + 1]);
+      ptx::st_global_32B(o + 16 * u, w);
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        w[i] = HALF ? pack_h2(f[8 * u + 2 * i], f[8 * u + 2 * i + 1]) : pack_b2(f[8 * u + 2 * i], f[8 * u + 2 * i + 1]);
+      reinterpret_cast<uint4*>(o)[u] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+// 32 fp32 values at p: 16-byte stores, or 32-byte ones when v32.
+__device__ __forceinline__ void store32_f32(float* p, const float (&f)[32], bool v32) {
+  if (v32) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(f[8 * u + i]);
+      ptx::st_global_32B(p + 8 * u, w);
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      reinterpret_cast<float4*>(p)[u] = make_float4(f[4 * u], f[4 * u + 1], f[4 * u + 2], f[4 * u + 3]);
+  }
+}
+// 32 consecutive fp32 table values at t (128-byte aligned when v32).
+__device__ __forceinline__ void load32_f32(const float* t, float (&f)[32], bool v32) {
+  if (v32) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t w[8];
+      ptx::ld_global_32B(t + 8 * u, w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[8 * u + i] = __uint_as_float(w[i]);
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(t) + u);
+      f[4 * u] = x.x; f[4 * u + 1] = x.y; f[4 * u + 2] = x.z; f[4 * u + 3] = x.w;
+    }
   }
 }
 
@@ -382,20 +444,15 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_tc(const __grid_constant__ CU
       const float inv = 1.f / l;
       const int prow = vrow(a, v, qi);
       const size_t off = (size_t)prow * (a.Hq * HD) + h * HD + half * 64;
+      const bool v32 = a.v32 != 0;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        float f[8];
+      for (int u = 0; u < 2; ++u) {
+        float f[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) f[i] = o[u * 8 + i] * inv;
-        reinterpret_cast<uint4*>(a.out + off)[u] =
-            make_uint4(pack_b2(f[0], f[1]), pack_b2(f[2], f[3]), pack_b2(f[4], f[5]), pack_b2(f[6], f[7]));
-        if (a.out16)
-          reinterpret_cast<uint4*>(a.out16 + off)[u] =
-              make_uint4(pack_h2(f[0], f[1]), pack_h2(f[2], f[3]), pack_h2(f[4], f[5]), pack_h2(f[6], f[7]));
-        if (a.out32) {
-          reinterpret_cast<float4*>(a.out32 + off)[2 * u] = make_float4(f[0], f[1], f[2], f[3]);
-          reinterpret_cast<float4*>(a.out32 + off)[2 * u + 1] = make_float4(f[4], f[5], f[6], f[7]);
-        }
+        for (int i = 0; i < 32; ++i) f[i] = o[u * 32 + i] * inv;
+        store32_16bit<false>(a.out + off + 32 * u, f, v32);
+        if (a.out16) store32_16bit<true>(a.out16 + off + 32 * u, f, v32);
+        if (a.out32) store32_f32(a.out32 + off + 32 * u, f, v32);
       }
       if (half == 0) a.lse[(size_t)h * a.T + prow] = m + log2f(l);
     }
@@ -670,31 +727,22 @@ __device__ __forceinline__ void attn_bwd_dkdv_cta(const CUtensorMap& tm128, cons
             f0[i] = __uint_as_float(v0[i]) * mul;
             f1[i] = __uint_as_float(v1[i]) * mul;
           }
+          const bool v32 = a.v32 != 0;
           if (which && a.rcos && in) {
-            const float* cs = a.rcos + (size_t)key * 64 + c * 32;
-            const float* sn = a.rsin + (size_t)key * 64 + c * 32;
+            float cs[32], sn[32];
+            load32_f32(a.rcos + (size_t)key * 64 + c * 32, cs, v32);
+            load32_f32(a.rsin + (size_t)key * 64 + c * 32, sn, v32);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) rope_back(f0[i], f1[i], __ldg(cs + i), __ldg(sn + i));
+            for (int i = 0; i < 32; ++i) rope_back(f0[i], f1[i], cs[i], sn[i]);
           }
           if (in) {
             uint16_t* o0 = a.dqkv + r + dcol + c * 32;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              reinterpret_cast<uint4*>(o0)[u] =
-                  make_uint4(pack_b2(f0[8 * u], f0[8 * u + 1]), pack_b2(f0[8 * u + 2], f0[8 * u + 3]),
-                             pack_b2(f0[8 * u + 4], f0[8 * u + 5]), pack_b2(f0[8 * u + 6], f0[8 * u + 7]));
-              reinterpret_cast<uint4*>(o0 + 64)[u] =
-                  make_uint4(pack_b2(f1[8 * u], f1[8 * u + 1]), pack_b2(f1[8 * u + 2], f1[8 * u + 3]),
-                             pack_b2(f1[8 * u + 4], f1[8 * u + 5]), pack_b2(f1[8 * u + 6], f1[8 * u + 7]));
-            }
+            store32_16bit<false>(o0, f0, v32);
+            store32_16bit<false>(o0 + 64, f1, v32);
             if (a.dqkv32) {
               float* p0 = a.dqkv32 + r + dcol + c * 32;
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                reinterpret_cast<float4*>(p0)[u] = make_float4(f0[4 * u], f0[4 * u + 1], f0[4 * u + 2], f0[4 * u + 3]);
-                reinterpret_cast<float4*>(p0 + 64)[u] =
-                    make_float4(f1[4 * u], f1[4 * u + 1], f1[4 * u + 2], f1[4 * u + 3]);
-              }
+              store32_f32(p0, f0, v32);
+              store32_f32(p0 + 64, f1, v32);
             }
           }
         }
@@ -907,29 +955,21 @@ __device__ __forceinline__ void attn_bwd_dq_cta(const CUtensorMap& tm128, const 
           f1[i] = __uint_as_float(v1[i]) * mul;
         }
         if (qin) {
+          const bool v32 = a.v32 != 0;
           if (a.rcos) {
-            const float* cs = a.rcos + (size_t)qi * 64 + c * 32;
-            const float* sn = a.rsin + (size_t)qi * 64 + c * 32;
+            float cs[32], sn[32];
+            load32_f32(a.rcos + (size_t)qi * 64 + c * 32, cs, v32);
+            load32_f32(a.rsin + (size_t)qi * 64 + c * 32, sn, v32);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) rope_back(f0[i], f1[i], __ldg(cs + i), __ldg(sn + i));
+            for (int i = 0; i < 32; ++i) rope_back(f0[i], f1[i], cs[i], sn[i]);
           }
           uint16_t* o0 = a.dqkv + r + c * 32;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            reinterpret_cast<uint4*>(o0)[u] =
-                make_uint4(pack_b2(f0[8 * u], f0[8 * u + 1]), pack_b2(f0[8 * u + 2], f0[8 * u + 3]),
-                           pack_b2(f0[8 * u + 4], f0[8 * u + 5]), pack_b2(f0[8 * u + 6], f0[8 * u + 7]));
-            reinterpret_cast<uint4*>(o0 + 64)[u] =
-                make_uint4(pack_b2(f1[8 * u], f1[8 * u + 1]), pack_b2(f1[8 * u + 2], f1[8 * u + 3]),
-                           pack_b2(f1[8 * u + 4], f1[8 * u + 5]), pack_b2(f1[8 * u + 6], f1[8 * u + 7]));
-          }
+          store32_16bit<false>(o0, f0, v32);
+          store32_16bit<false>(o0 + 64, f1, v32);
           if (a.dqkv32) {
             float* p0 = a.dqkv32 + r + c * 32;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              reinterpret_cast<float4*>(p0)[u] = make_float4(f0[4 * u], f0[4 * u + 1], f0[4 * u + 2], f0[4 * u + 3]);
-              reinterpret_cast<float4*>(p0 + 64)[u] = make_float4(f1[4 * u], f1[4 * u + 1], f1[4 * u + 2], f1[4 * u + 3]);
-            }
+            store32_f32(p0, f0, v32);
+            store32_f32(p0 + 64, f1, v32);
           }
         }
       }
@@ -1023,6 +1063,7 @@ soup_status attention_fwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
   a.scale = 1.0f / sqrtf((float)HD);
   a.scale_log2 = 1.4426950408889634f * a.scale;
   a.out = out; a.lse = lse; a.out16 = out16; a.out32 = out32;
+  a.v32 = soup_aligned(out, 32) && (!out16 || soup_aligned(out16, 32)) && (!out32 || soup_aligned(out32, 32));
   a.err = device_error_word();
   SOUP_CHECK(a.err, SOUP_ERR_CUDA, "device error word unavailable");
   a.wait_limit = 4000000000LL;
@@ -1058,6 +1099,8 @@ soup_status attention_bwd(const uint16_t* qkv, int ld, int Bsz, int S, int Hq, i
   a.scale_log2 = 1.4426950408889634f * a.scale;
   a.L = lse; a.D = D; a.dqkv = dqkv; a.dqkv32 = dqkv32; a.ld = ld;
   a.rcos = rope_cos; a.rsin = rope_sin; a.amax = amax;
+  a.v32 = soup_aligned(dqkv, 32) && (!dqkv32 || soup_aligned(dqkv32, 32)) && (ld * 2) % 32 == 0 &&
+          (!rope_cos || (soup_aligned(rope_cos, 32) && soup_aligned(rope_sin, 32)));
   a.err = device_error_word();
   SOUP_CHECK(a.err, SOUP_ERR_CUDA, "device error word unavailable");
   a.wait_limit = 4000000000LL;

@@ -125,21 +125,6 @@ __device__ __forceinline__ float f16_to_f32(uint16_t b) {
   return __half2float(__ushort_as_half(b));
 }
 
-// 32-byte global accesses (sm_100 vector width): one instruction moves a
-// row's 16 16-bit values, where two 16-byte ones would each touch the same
-// 32 rows of a warp.  The caller guarantees 32-byte alignment.
-__device__ __forceinline__ void st_global_32B(void* p, const uint32_t (&w)[8]) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
-               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-               : "memory");
-}
-__device__ __forceinline__ void ld_global_32B(const void* p, uint32_t (&w)[8]) {
-  asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-               : "l"(p)
-               : "memory");
-}
-
 // Stores 16 consecutive values of one row (row-major 16-bit or fp32 output),
 // vectorised when the whole chunk is in range and aligned (vec: 0 scalar,
 // 1 16-byte, 2 32-byte accesses).
@@ -154,7 +139,7 @@ __device__ __forceinline__ void store_row16(void* out, int out_kind, long long l
       for (int h = 0; h < 2; ++h) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(f[8 * h + i]);
-        st_global_32B(o + 8 * h, w);
+        ptx::st_global_32B(o + 8 * h, w);
       }
     } else if (full) {
 #pragma unroll
@@ -174,7 +159,7 @@ __device__ __forceinline__ void store_row16(void* out, int out_kind, long long l
 #pragma unroll
     for (int i = 0; i < 8; ++i) p[i] = h ? pack_f16x2(f[2 * i], f[2 * i + 1]) : pack_bf16x2(f[2 * i], f[2 * i + 1]);
     if (vec == 2) {
-      st_global_32B(o, p);
+      ptx::st_global_32B(o, p);
     } else {
       reinterpret_cast<uint4*>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
       reinterpret_cast<uint4*>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
@@ -192,7 +177,7 @@ __device__ __forceinline__ void store_row16(void* out, int out_kind, long long l
 // 16 consecutive 16-bit values as 8 packed words (element 2i in the low half)
 __device__ __forceinline__ void load8_u32(const uint16_t* p, uint32_t (&w)[8], int vec) {
   if (vec == 2) {
-    ld_global_32B(p, w);
+    ptx::ld_global_32B(p, w);
   } else {
     const uint4 a = *reinterpret_cast<const uint4*>(p);
     const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
@@ -204,7 +189,7 @@ __device__ __forceinline__ void load8_u32(const uint16_t* p, uint32_t (&w)[8], i
 __device__ __forceinline__ void load16_u16(const uint16_t* p, uint16_t (&v)[16], int vec) {
   uint32_t w[8];
   if (vec == 2) {
-    ld_global_32B(p, w);
+    ptx::ld_global_32B(p, w);
   } else {
     const uint4 a = *reinterpret_cast<const uint4*>(p);
     const uint4 b = *reinterpret_cast<const uint4*>(p + 8);
@@ -475,7 +460,7 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
           uint32_t w[8];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            ld_global_32B(r + 8 * h, w);
+            ptx::ld_global_32B(r + 8 * h, w);
 #pragma unroll
             for (int i = 0; i < 8; ++i) f[8 * h + i] += __uint_as_float(w[i]);
           }
