@@ -418,10 +418,11 @@ __global__ void lora_prep_kernel(const PrepArgs a) {
     if (J.kind == PREP_COPY_F32) {
       static_cast<float*>(J.out)[i] = b2f(J.in[i]);
     } else {
-      const int R = (int)(i / J.N), n = (int)(i % J.N);
-      const int s = R / J.r, j = R % J.r;
+      // 32-bit division: a job has fewer than 2^31 elements (checked on the host)
+      const unsigned R = (unsigned)i / (unsigned)J.N, n = (unsigned)i - R * (unsigned)J.N;
+      const int s = (int)R / J.r, j = (int)R % J.r;
       int seg = 0;
-      while (seg + 1 < J.nseg && n >= J.seg_end[seg]) ++seg;
+      while (seg + 1 < J.nseg && (int)n >= J.seg_end[seg]) ++seg;
       const uint16_t v = seg == s ? J.in[(size_t)n * J.r + j] : static_cast<uint16_t>(0);
       if (J.out_bf16) static_cast<uint16_t*>(J.out)[i] = v;
       else static_cast<float*>(J.out)[i] = b2f(v);
@@ -439,8 +440,8 @@ soup_status lora_prep(const PrepJobs& jobs, cudaStream_t st) {
     const PrepJob& J = jobs.job[k];
     SOUP_CHECK(J.in && J.out, SOUP_ERR_INVALID_ARG, "lora_prep: null job pointer");
     const long long n = J.kind == PREP_COPY_F32 ? (long long)J.rows * J.cols : (long long)J.nseg * J.r * J.N;
-    SOUP_CHECK(n > 0 && (J.kind == PREP_COPY_F32 || (J.r > 0 && J.nseg >= 1 && J.nseg <= 3)), SOUP_ERR_SHAPE,
-               "lora_prep: bad job %d", k);
+    SOUP_CHECK(n > 0 && n < (1LL << 31) && (J.kind == PREP_COPY_F32 || (J.r > 0 && J.nseg >= 1 && J.nseg <= 3)),
+               SOUP_ERR_SHAPE, "lora_prep: bad job %d", k);
     a.start[k + 1] = a.start[k] + n;
   }
   const long long total = a.start[jobs.njobs];

@@ -345,13 +345,31 @@ __device__ __forceinline__ void epilogue_tile(const KArgs& args, void* outp, uin
       }
       const float* cs = args.rope_cos + (size_t)pos * 64 + (ch & 7) * 16;
       const float* sn = args.rope_sin + (size_t)pos * 64 + (ch & 7) * 16;
+      // the position's 16 angles of the chunk, 8 at a time: 32-byte loads
+      // where aligned (each thread owns a row, so scalar loads would touch
+      // 32 rows apiece)
       float a[16], b[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float x0 = __uint_as_float(v0[i]) * alpha, x1 = __uint_as_float(v1[i]) * alpha;
-        const float c = __ldg(cs + i), sv = __ldg(sn + i);
-        a[i] = x0 * c - x1 * sv;
-        b[i] = x1 * c + x0 * sv;
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t cw[8], sw[8];
+        if (vec == 2) {
+          ptx::ld_global_32B(cs + 8 * hh, cw);
+          ptx::ld_global_32B(sn + 8 * hh, sw);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            cw[i] = __float_as_uint(__ldg(cs + 8 * hh + i));
+            sw[i] = __float_as_uint(__ldg(sn + 8 * hh + i));
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int e = 8 * hh + i;
+          const float x0 = __uint_as_float(v0[e]) * alpha, x1 = __uint_as_float(v1[e]) * alpha;
+          const float c = __uint_as_float(cw[i]), sv = __uint_as_float(sw[i]);
+          a[e] = x0 * c - x1 * sv;
+          b[e] = x1 * c + x0 * sv;
+        }
       }
       store_row16(outp, args.out_kind, args.ldo, row, n, args.N, a, vec);
       store_row16(outp, args.out_kind, args.ldo, row, n + 64, args.N, b, vec);
@@ -1871,7 +1889,8 @@ soup_status gemm(const GemmDesc& d, cudaStream_t st) {
     return soup_aligned(d.out, a) && ((d.ldo * esz) % a == 0) && (!d.out_lo || soup_aligned(d.out_lo, a)) &&
            (!d.resid || (soup_aligned(d.resid, a) && (d.ldr * 2) % a == 0)) &&
            (!d.resid_f32 || (soup_aligned(d.resid_f32, a) && (d.ldr * 4) % a == 0)) &&
-           (!d.aux16 || (soup_aligned(d.aux16, a) && (d.ld_aux * 2) % a == 0 && (d.swiglu_I * 2) % a == 0));
+           (!d.aux16 || (soup_aligned(d.aux16, a) && (d.ld_aux * 2) % a == 0 && (d.swiglu_I * 2) % a == 0)) &&
+           (!d.rope_cols || (soup_aligned(d.rope_cos, a) && soup_aligned(d.rope_sin, a)));
   };
   ka.vec_ok = rows_aligned(32) ? 2 : (rows_aligned(16) ? 1 : 0);
   ka.wait_limit = d.wait_limit > 0 ? d.wait_limit : 4000000000LL;
