@@ -160,8 +160,8 @@ HeadWS head_layout(int64_t V, int64_t H, int64_t T, int chunk) {
   w.logits = take((size_t)chunk * V * 4);
   w.dlogits = take((size_t)chunk * V * 2);
   w.dxn = take((size_t)T * H * 4);
-  // dxn = dlogits E has K = V but only (chunk/128)·(H/256) output tiles:
-  // split-K partial products (up to 6 slices)
+  // dxn = dlogits E has K = V but only (chunk/256)·(H/256) output tiles of
+  // the CTA-pair engine: scratch for the fp32 partials of its K slices
   w.splitk_bytes = (size_t)6 * chunk * H * 4;
   w.splitk = take(w.splitk_bytes);
   w.total = o;
@@ -234,8 +234,11 @@ extern "C" soup_status soup_head_fwd_bwd(const uint16_t* h, const uint16_t* w_fi
       g2.b_mode = B_TMA_MN;
       g2.B = Mat{E, V, H, H};
       g2.out_kind = OUT_F32; g2.out = dxn + (size_t)t0 * H; g2.ldo = H;
-      g2.split_ws = reinterpret_cast<float*>(base + ws.splitk);
-      g2.split_ws_bytes = ws.splitk_bytes;
+      // few output tiles, long K: the persistent CTA-pair engine cuts the
+      // tiles into K slices (fp32 partials in this scratch, summed in slice
+      // order by the last slice of each tile)
+      g2.sk_scratch = base + ws.splitk;
+      g2.sk_scratch_bytes = ws.splitk_bytes;
       SOUP_TRY(gemm(g2, st));
     }
   }
