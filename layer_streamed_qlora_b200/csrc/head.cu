@@ -66,12 +66,20 @@ __global__ void __launch_bounds__(1024) ce_rows_kernel(const float* __restrict__
   const bool has_label = s < S - 1;
   const int label = has_label ? ids[t + 1] : -1;
   const float* row = logits + (size_t)i * V;
-  float m = -INFINITY;
-  for (int64_t j = threadIdx.x; j < V; j += blockDim.x) m = fmaxf(m, row[j]);
-  m = block_reduce(m, true, sh);
-  float sum = 0.f;
-  for (int64_t j = threadIdx.x; j < V; j += blockDim.x) sum += expf(row[j] - m);
-  sum = block_reduce(sum, false, sh);
+  // one pass for the row's maximum and its sum of exponentials: each thread
+  // keeps a running maximum and rescales its partial sum when it grows, then
+  // the block combines the (maximum, sum) pairs (V % 8 == 0: float4 loads)
+  float tm = -INFINITY, ts = 0.f;
+  const float4* row4 = reinterpret_cast<const float4*>(row);
+  for (int64_t j = threadIdx.x; j < V / 4; j += blockDim.x) {
+    const float4 x = row4[j];
+    const float mx = fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w));
+    const float mn = fmaxf(tm, mx);
+    ts = ts * expf(tm - mn) + (expf(x.x - mn) + expf(x.y - mn)) + (expf(x.z - mn) + expf(x.w - mn));
+    tm = mn;
+  }
+  const float m = block_reduce(tm, true, sh);
+  float sum = block_reduce(tm == -INFINITY ? 0.f : ts * expf(tm - m), false, sh);
   const float lse = m + logf(sum);
   const bool label_ok = has_label && label >= 0 && label < V;
   if (threadIdx.x == 0 && has_label) logp[(size_t)b * (S - 1) + s] = label_ok ? row[label] - lse : 0.f;
@@ -79,11 +87,19 @@ __global__ void __launch_bounds__(1024) ce_rows_kernel(const float* __restrict__
     const float c = (coef && label_ok) ? coef[(size_t)b * (S - 1) + s] : 0.f;
     uint16_t* drow = dlogits + (size_t)i * V;
     const float inv = 1.0f / sum;
-    for (int64_t j = threadIdx.x; j < V; j += blockDim.x) {
-      const float p = expf(row[j] - m) * inv;
-      const float g = c * ((j == label ? 1.f : 0.f) - p);
-      __nv_bfloat16 hv = __float2bfloat16_rn(g);
-      drow[j] = *reinterpret_cast<uint16_t*>(&hv);
+    for (int64_t j = threadIdx.x; j < V / 4; j += blockDim.x) {
+      const float4 x = row4[j];
+      const float xs[4] = {x.x, x.y, x.z, x.w};
+      uint32_t w[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int64_t j0 = 4 * j + 2 * e;
+        const float g0 = c * ((j0 == label ? 1.f : 0.f) - expf(xs[2 * e] - m) * inv);
+        const float g1 = c * ((j0 + 1 == label ? 1.f : 0.f) - expf(xs[2 * e + 1] - m) * inv);
+        __nv_bfloat162 hv = __floats2bfloat162_rn(g0, g1);
+        w[e] = *reinterpret_cast<uint32_t*>(&hv);
+      }
+      reinterpret_cast<uint2*>(drow)[j] = make_uint2(w[0], w[1]);
     }
   }
 }
