@@ -404,10 +404,11 @@ soup_status bf16_to_f32(const uint16_t* in, size_t n, float* out, cudaStream_t s
 namespace {
 struct PrepArgs {
   PrepJobs jobs;
-  long long start[5];  // prefix sums of the jobs' output element counts
+  long long start[6];  // prefix sums of the jobs' unit counts
 };
 
 __global__ void lora_prep_kernel(const PrepArgs a) {
+  if (a.jobs.zero_word && blockIdx.x == 0 && threadIdx.x == 0) *a.jobs.zero_word = 0u;
   const long long total = a.start[a.jobs.njobs];
   for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
@@ -417,6 +418,17 @@ __global__ void lora_prep_kernel(const PrepArgs a) {
     const long long i = idx - a.start[k];
     if (J.kind == PREP_COPY_F32) {
       static_cast<float*>(J.out)[i] = b2f(J.in[i]);
+    } else if (J.kind == PREP_F32_TO_BF16) {  // unit i: elements 8i .. 8i+7
+      const float4 x0 = reinterpret_cast<const float4*>(J.in32)[2 * i];
+      const float4 x1 = reinterpret_cast<const float4*>(J.in32)[2 * i + 1];
+      const float f[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+      reinterpret_cast<uint4*>(J.out)[i] = pack8(f);
+    } else if (J.kind == PREP_ROPE) {
+      const int pos = (int)(i / J.r), j = (int)(i % J.r);
+      const double inv = pow(J.theta, -(2.0 * j) / (2.0 * J.r));
+      const double ang = (double)pos * inv;
+      static_cast<float*>(J.out)[i] = (float)cos(ang);
+      static_cast<float*>(J.out2)[i] = (float)sin(ang);
     } else {
       // 32-bit division: a job has fewer than 2^31 elements (checked on the host)
       const unsigned R = (unsigned)i / (unsigned)J.N, n = (unsigned)i - R * (unsigned)J.N;
@@ -432,16 +444,33 @@ __global__ void lora_prep_kernel(const PrepArgs a) {
 }  // namespace
 
 soup_status lora_prep(const PrepJobs& jobs, cudaStream_t st) {
-  SOUP_CHECK(jobs.njobs >= 1 && jobs.njobs <= 4, SOUP_ERR_INVALID_ARG, "lora_prep: %d jobs", jobs.njobs);
+  SOUP_CHECK(jobs.njobs >= 1 && jobs.njobs <= 5, SOUP_ERR_INVALID_ARG, "lora_prep: %d jobs", jobs.njobs);
   PrepArgs a;
   a.jobs = jobs;
   a.start[0] = 0;
   for (int k = 0; k < jobs.njobs; ++k) {
     const PrepJob& J = jobs.job[k];
-    SOUP_CHECK(J.in && J.out, SOUP_ERR_INVALID_ARG, "lora_prep: null job pointer");
-    const long long n = J.kind == PREP_COPY_F32 ? (long long)J.rows * J.cols : (long long)J.nseg * J.r * J.N;
-    SOUP_CHECK(n > 0 && n < (1LL << 31) && (J.kind == PREP_COPY_F32 || (J.r > 0 && J.nseg >= 1 && J.nseg <= 3)),
-               SOUP_ERR_SHAPE, "lora_prep: bad job %d", k);
+    long long n = 0;
+    bool ok = false;
+    switch (J.kind) {
+      case PREP_COPY_F32:
+        n = (long long)J.rows * J.cols;
+        ok = J.in && J.out;
+        break;
+      case PREP_BLOCKDIAG_T:
+        n = (long long)J.nseg * J.r * J.N;
+        ok = J.in && J.out && J.r > 0 && J.nseg >= 1 && J.nseg <= 3;
+        break;
+      case PREP_F32_TO_BF16:
+        n = J.n / 8;
+        ok = J.in32 && J.out && J.n % 8 == 0 && soup_aligned(J.in32, 16) && soup_aligned(J.out, 16);
+        break;
+      case PREP_ROPE:
+        n = (long long)J.N * J.r;
+        ok = J.out && J.out2 && J.r > 0 && J.theta > 0.0;
+        break;
+    }
+    SOUP_CHECK(ok && n > 0 && n < (1LL << 31), SOUP_ERR_SHAPE, "lora_prep: bad job %d", k);
     a.start[k + 1] = a.start[k] + n;
   }
   const long long total = a.start[jobs.njobs];
@@ -450,7 +479,10 @@ soup_status lora_prep(const PrepJobs& jobs, cudaStream_t st) {
   for (int k = 0; k < jobs.njobs; ++k) {
     const PrepJob& J = jobs.job[k];
     const double outs = (double)(a.start[k + 1] - a.start[k]);
-    bytes += J.kind == PREP_COPY_F32 ? outs * 6.0 : outs * (J.out_bf16 ? 2 : 4) + (double)J.N * J.r * 2;
+    if (J.kind == PREP_COPY_F32) bytes += outs * 6.0;
+    else if (J.kind == PREP_F32_TO_BF16) bytes += outs * 48.0;  // 8 x (4 in + 2 out)
+    else if (J.kind == PREP_ROPE) bytes += outs * 8.0;
+    else bytes += outs * (J.out_bf16 ? 2 : 4) + (double)J.N * J.r * 2;
   }
   profile_begin(st, GC_ELEM, 0.0, bytes);
   lora_prep_kernel<<<blocks, 256, 0, st>>>(a);

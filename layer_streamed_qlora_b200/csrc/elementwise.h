@@ -31,13 +31,17 @@ soup_status attn_rowdot(const uint16_t* dO, const uint16_t* O, int T, int Hq, fl
 soup_status f32_to_bf16(const float* in, size_t n, uint16_t* out, cudaStream_t st, unsigned int* zero_word = nullptr);
 soup_status bf16_to_f32(const uint16_t* in, size_t n, float* out, cudaStream_t st);
 
-// LoRA operand preparation in one launch (up to 4 jobs):
+// LoRA operand preparation in one launch (up to 5 jobs):
 //   PREP_COPY_F32:   out[i] = fp32(in[i]), i < rows * cols (in and out [rows, cols])
 //   PREP_BLOCKDIAG_T: in = B [N, r] (rows grouped in nseg segments ending at
 //     seg_end[]), out [nseg * r, N] = the block-diagonal transpose: row
 //     s*r + j, column n holds B[n, j] when n lies in segment s, else 0
 //     (fp32, or bf16 with out_bf16)
-enum PrepKind : int { PREP_COPY_F32 = 0, PREP_BLOCKDIAG_T = 1 };
+//   PREP_F32_TO_BF16: out [n] bf16 = RNE(in32 [n] fp32), n % 8 == 0 (the
+//     activation conversion that shares the launch with the factor prep)
+//   PREP_ROPE: out / out2 [N positions, r] fp32 = cos / sin of
+//     pos * theta^(-2j / 2r), computed in fp64 (the same values as rope_table)
+enum PrepKind : int { PREP_COPY_F32 = 0, PREP_BLOCKDIAG_T = 1, PREP_F32_TO_BF16 = 2, PREP_ROPE = 3 };
 struct PrepJob {
   int kind = PREP_COPY_F32;
   int out_bf16 = 0;
@@ -46,10 +50,15 @@ struct PrepJob {
   int rows = 0, cols = 0;  // PREP_COPY_F32
   int N = 0, r = 0, nseg = 1;
   int seg_end[3] = {0, 0, 0};
+  const float* in32 = nullptr;  // PREP_F32_TO_BF16
+  long long n = 0;              // PREP_F32_TO_BF16
+  void* out2 = nullptr;         // PREP_ROPE: the sin table
+  double theta = 0.0;           // PREP_ROPE
 };
 struct PrepJobs {
   int njobs = 0;
-  PrepJob job[4];
+  PrepJob job[5];
+  unsigned int* zero_word = nullptr;  // optional: set to 0 by the same launch
 };
 soup_status lora_prep(const PrepJobs& jobs, cudaStream_t st);
 

@@ -424,20 +424,27 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
   // the backward's d_gu residual field is unused during a forward pass or
   // recompute: the big GEMMs' split last round keeps its partials there
   const Scratch SK{base + ws.d_gu_lo, (size_t)T * 2 * m.I * 2};
-  SOUP_TRY(rope_table(m.S, m.d, (double)c->theta, PF(cosb), PF(sinb), st));
+  // the RoPE table, with adapters on in the same launch as the fp32 copies of
+  // the three A factors (tf32 operands)
+  if (on) {
+    PrepJobs pj;
+    pj.njobs = 4;
+    pj.job[0].in = L->A_qkv; pj.job[0].out = PF(A32); pj.job[0].rows = 3 * r; pj.job[0].cols = m.H;
+    pj.job[1].in = L->A_o; pj.job[1].out = PF(Ao32); pj.job[1].rows = r; pj.job[1].cols = m.o_in;
+    pj.job[2].in = L->A_gu; pj.job[2].out = PF(Agu32); pj.job[2].rows = 2 * r; pj.job[2].cols = m.H;
+    PrepJob& rp = pj.job[3];
+    rp.kind = PREP_ROPE; rp.out = PF(cosb); rp.out2 = PF(sinb); rp.N = m.S; rp.r = m.d / 2;
+    rp.theta = (double)c->theta;
+    SOUP_TRY(lora_prep(pj, st));
+  } else {
+    SOUP_TRY(rope_table(m.S, m.d, (double)c->theta, PF(cosb), PF(sinb), st));
+  }
   const bool precise_qkv = (save && !kept) || keep;  // q|k|v from the hi + lo x1 pair
   SOUP_TRY(rmsnorm_fwd(h_in, nullptr, W->norm1, T, m.H, c->eps, P(x1), PF(rinv1), st, on ? PF(x1_32) : nullptr,
                        precise_qkv ? P(x1_lo) : nullptr));
   if (on) {
     // q/k/v adapters: u from the fp32 normalised input (tf32 tensor cores); the
     // tail consumes its bf16 copy, the dB GEMM its fp32 copy
-    // fp32 copies of the three A factors (tf32 operands), one launch
-    PrepJobs pj;
-    pj.njobs = 3;
-    pj.job[0].in = L->A_qkv; pj.job[0].out = PF(A32); pj.job[0].rows = 3 * r; pj.job[0].cols = m.H;
-    pj.job[1].in = L->A_o; pj.job[1].out = PF(Ao32); pj.job[1].rows = r; pj.job[1].cols = m.o_in;
-    pj.job[2].in = L->A_gu; pj.job[2].out = PF(Agu32); pj.job[2].rows = 2 * r; pj.job[2].cols = m.H;
-    SOUP_TRY(lora_prep(pj, st));
     SOUP_TRY(lora_down_tf32(PF(x1_32), T, m.H, PF(A32), 3 * r, m.s, P(u_qkv), PF(u32), m.ldT, st, SW));
   }
   {
@@ -611,10 +618,16 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
 
   // ---- B factors for the g GEMMs, one launch: B_down^T and B_o^T (fp32),
   // block-diagonal transposes of B_qkv (fp32, 3 segments) and B_gu (bf16,
-  // 2 segments), so each g = s dy B is one GEMM over all its segments
+  // 2 segments), so each g = s dy B is one GEMM over all its segments; the
+  // same launch converts dh_out to bf16 (the down product's A operand) and
+  // zeroes gamax (max |dh2| of the norm2 backward accumulates into it)
+  unsigned int* gamax = reinterpret_cast<unsigned int*>(base + ws.gamax);
   if (on) {
     PrepJobs pj;
-    pj.njobs = 4;
+    pj.njobs = 5;
+    pj.zero_word = gamax;
+    PrepJob& cv = pj.job[4];
+    cv.kind = PREP_F32_TO_BF16; cv.in32 = dh_out; cv.out = P(dh_b); cv.n = (long long)T * H;
     PrepJob& a = pj.job[0];
     a.kind = PREP_BLOCKDIAG_T; a.in = L->B_down; a.out = PF(Bt_down32); a.N = H; a.r = r;
     PrepJob& b = pj.job[1];
@@ -650,9 +663,7 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
   };
 
   // ---- MLP block
-  // (max |dh2| of the norm2 backward below accumulates into gamax, zeroed here)
-  unsigned int* gamax = reinterpret_cast<unsigned int*>(base + ws.gamax);
-  SOUP_TRY(f32_to_bf16(dh_out, (size_t)T * H, P(dh_b), st, gamax));
+  if (!on) SOUP_TRY(f32_to_bf16(dh_out, (size_t)T * H, P(dh_b), st, gamax));
   // LoRA gradients of the MLP: g_down from the fp32 dh (tf32), the others
   // from hi + lo (rounding residual) operand pairs, so no operand of a
   // LoRA-gradient GEMM carries more than the bf16 rounding of d_gu
