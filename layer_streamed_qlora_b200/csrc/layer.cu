@@ -393,7 +393,7 @@ soup_status proj_bwd(const soup_weight* W, const uint16_t* dy, int T, const uint
 struct SideStream {
   void* ctx = nullptr;
   cudaStream_t st = nullptr;
-  cudaEvent_t ev[9] = {};  // 0-4, 7, 8: chain steps the side stream waits for; 5, 6: side-stream milestones
+  cudaEvent_t ev[11] = {};  // 0-4, 7-10: chain steps the side stream waits for; 5, 6: side-stream milestones
   std::mutex issue;  // held while one layer call issues its work: calls from
                      // several threads then share the side stream in turn
 };
@@ -416,9 +416,19 @@ soup_status side_stream(SideStream** out) {
   return SOUP_OK;
 }
 
+// The backward's recompute may hand LoRA down-projections that only the
+// LoRA-factor gradients read (u_qkv of a layer whose q|k|v were kept: no
+// q|k|v GEMM consumes it; u_down: the down product is not recomputed) to the
+// side stream, after an event on the chain marks their input ready.
+struct RecomputeSide {
+  SideStream* side = nullptr;
+  SplitWS sw{nullptr, 0};
+};
+
 soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const soup_layer_cfg* c, const Dims& m,
                     const WS& ws, char* base, char* fb, const uint16_t* h_in, uint16_t* h_out, bool on, bool save,
-                    bool want_out, cudaStream_t st, uint16_t* keep = nullptr, const uint16_t* kept = nullptr) {
+                    bool want_out, cudaStream_t st, uint16_t* keep = nullptr, const uint16_t* kept = nullptr,
+                    const RecomputeSide& rs = RecomputeSide()) {
   const int T = m.T, r = m.r;
   const SplitWS SW{PF(splitk), ws.splitk_bytes};
   // the backward's d_gu residual field is unused during a forward pass or
@@ -445,7 +455,13 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
   if (on) {
     // q/k/v adapters: u from the fp32 normalised input (tf32 tensor cores); the
     // tail consumes its bf16 copy, the dB GEMM its fp32 copy
-    SOUP_TRY(lora_down_tf32(PF(x1_32), T, m.H, PF(A32), 3 * r, m.s, P(u_qkv), PF(u32), m.ldT, st, SW));
+    if (kept && rs.side) {
+      SOUP_CUDA_TRY(cudaEventRecord(rs.side->ev[9], st));
+      SOUP_CUDA_TRY(cudaStreamWaitEvent(rs.side->st, rs.side->ev[9], 0));
+      SOUP_TRY(lora_down_tf32(PF(x1_32), T, m.H, PF(A32), 3 * r, m.s, P(u_qkv), PF(u32), m.ldT, rs.side->st, rs.sw));
+    } else {
+      SOUP_TRY(lora_down_tf32(PF(x1_32), T, m.H, PF(A32), 3 * r, m.s, P(u_qkv), PF(u32), m.ldT, st, SW));
+    }
   }
   {
     const int se[3] = {m.Hq * m.d, (m.Hq + m.Hkv) * m.d, m.qkv_w};
@@ -495,7 +511,15 @@ soup_status forward(const soup_layer_weights* W, const soup_layer_lora* L, const
     SOUP_TRY(proj_fwd(&W->gate_up, P(x2), T, P(u_gu), m.ldT, 2 * r, L ? L->B_gu : nullptr, r, 1, se, sr, on,
                       P(act), st, o));
   }
-  if (on) SOUP_TRY(lora_down(P(act), T, m.I, L->A_down, r, m.s, P(u_d), m.ldT, st, SW, PF(u_d32)));
+  if (on) {
+    if (!want_out && rs.side) {
+      SOUP_CUDA_TRY(cudaEventRecord(rs.side->ev[10], st));
+      SOUP_CUDA_TRY(cudaStreamWaitEvent(rs.side->st, rs.side->ev[10], 0));
+      SOUP_TRY(lora_down(P(act), T, m.I, L->A_down, r, m.s, P(u_d), m.ldT, rs.side->st, rs.sw, PF(u_d32)));
+    } else {
+      SOUP_TRY(lora_down(P(act), T, m.I, L->A_down, r, m.s, P(u_d), m.ldT, st, SW, PF(u_d32)));
+    }
+  }
   if (want_out) {
     const int se[1] = {m.H};
     const int sr[1] = {0};
@@ -606,13 +630,28 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
   const int T = m.T, r = m.r, H = m.H, I = m.I;
   const int64_t ldT = m.ldT;
 
+  // LoRA-factor gradients go to the side stream: each group waits (event)
+  // for the main-stream step that produced its inputs.  The MLP groups are
+  // issued after the next big GEMM; dB_o and dB_qkv, which need only dy and
+  // the forward's u, start beside the skinny g GEMM before the o / q|k|v
+  // dx product (measured: 2 ms less per 32-layer backward than issuing them
+  // after it), so less of the side stream is left when the layer joins it.
+  // The recompute hands it the down-projections only they read.
+  SideStream* side = nullptr;
+  if (on) SOUP_TRY(side_stream(&side));
+  std::unique_lock<std::mutex> issue_lock;
+  if (side) issue_lock = std::unique_lock<std::mutex>(side->issue);
+
   // forward fields: recomputed into the workspace (the layer was read again
   // for this), or what a saved forward pass left in the layer's own region
   if (saved) {
     SOUP_CHECK(soup_aligned(saved, 256), SOUP_ERR_ALIGN, "soup_decoder_layer_bwd_saved: saved region not 256-byte aligned");
     fb = static_cast<char*>(const_cast<void*>(saved));
   } else {
-    SOUP_TRY(forward(W, L, cfg, m, ws, base, fb, h_in, nullptr, on, true, false, st, nullptr, kept));
+    RecomputeSide rs;
+    rs.side = side;
+    rs.sw = SplitWS{PF(splitk2), ws.splitk_bytes};
+    SOUP_TRY(forward(W, L, cfg, m, ws, base, fb, h_in, nullptr, on, true, false, st, nullptr, kept, rs));
   }
   const uint16_t* qkvp = kept ? kept : P(qkv);
 
@@ -641,16 +680,6 @@ static soup_status layer_bwd_impl(const soup_layer_weights* W, const soup_layer_
     SOUP_TRY(lora_prep(pj, st));
   }
 
-  // LoRA-factor gradients go to the side stream: each group waits (event)
-  // for the main-stream step that produced its inputs.  The MLP groups are
-  // issued after the next big GEMM; dB_o and dB_qkv, which need only dy and
-  // the forward's u, start beside the skinny g GEMM before the o / q|k|v
-  // dx product (measured: 2 ms less per 32-layer backward than issuing them
-  // after it), so less of the side stream is left when the layer joins it.
-  SideStream* side = nullptr;
-  if (on) SOUP_TRY(side_stream(&side));
-  std::unique_lock<std::mutex> issue_lock;
-  if (side) issue_lock = std::unique_lock<std::mutex>(side->issue);
   const SplitWS SW2{PF(splitk2), ws.splitk_bytes};
   cudaStream_t s2 = side ? side->st : st;
   auto mark = [&](int e) -> soup_status {  // the side stream may consume what st has produced so far
