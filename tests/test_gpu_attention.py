@@ -165,3 +165,32 @@ def test_attention_with_a_shared_prefix_matches_oracle(L):
     assert_close(got_d[:, :qo], ref_d[:, :qo], "dq (shared prefix)")
     assert_close(got_d[:, qo:ko], ref_d[:, qo:ko], "dk (shared prefix)")
     assert_close(got_d[:, ko:], ref_d[:, ko:], "dv (shared prefix)")
+
+
+def test_attention_16_byte_output_fallback_bit_exact(L):
+    """Outputs 16- but not 32-byte aligned take the epilogues' 16-byte stores
+    instead of their 32-byte ones: the same bits either way."""
+    B, S, Hq, Hkv = 3, 130, 8, 2
+    got, _, (qkv_d, dout_d, out16, lse, D, dqkv, ld) = run_case(L, B, S, Hq, Hkv, seed=21)
+    T = B * S
+
+    def offset_view(shape, dtype):
+        n = shape[0] * shape[1]
+        buf = torch.zeros(n + 32 // torch.tensor([], dtype=dtype).element_size(), dtype=dtype, device="cuda")
+        v = buf[16 // buf.element_size():16 // buf.element_size() + n].view(*shape)
+        assert v.data_ptr() % 32 == 16
+        return v
+
+    out = offset_view((T, Hq * HD), torch.bfloat16)
+    o16 = offset_view((T, Hq * HD), torch.float16)
+    lse2 = torch.empty((Hq, T), dtype=torch.float32, device="cuda")
+    L.soup_attention_fwd(qkv_d, B, S, Hq, Hkv, out, o16, lse2)
+    dq2 = offset_view((T, ld), torch.bfloat16)
+    dq32 = offset_view((T, ld), torch.float32)
+    D2 = torch.empty((Hq, T), dtype=torch.float32, device="cuda")
+    L.soup_attention_bwd(qkv_d, B, S, Hq, Hkv, o16, dout_d, lse2, D2, dq2, dq32)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(out), got["out"])
+    assert np.array_equal(host(lse2), got["lse"])
+    assert np.array_equal(host(dq2), got["dqkv"])
+    assert np.array_equal(host(dq32), got["dqkv32"])

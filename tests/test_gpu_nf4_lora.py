@@ -189,3 +189,31 @@ def test_B_zero_reproduces_frozen_base_exactly():
     assert np.array_equal(g0["y"], g1["y"])
     Wd = g0["deq"].astype(np.float64)
     assert_close(g0["y"], x @ Wd.T, "y(B=0)")
+
+
+def test_epilogue_16_byte_fallback_bit_exact():
+    """Outputs 16- but not 32-byte aligned take the epilogue's 16-byte stores
+    instead of its 32-byte ones: the same bits either way."""
+    T, n_in, n_out = 300, 1024, 768
+    W, x, A, B, dy, r, s = _c1(seed=11, T=T, n_in=n_in, n_out=n_out, r=16, alpha=32.0)
+    g = run_gpu_lora(W, x, A, B, dy, r, s, "nf4")
+    codes, absmax = gpu_quantize(W)
+    Wd = L.weight_nf4(codes, absmax, n_out, n_in)
+    xd, Ad, Bd, dyd = dev_bf16(x), dev_bf16(A), dev_bf16(B), dev_bf16(dy)
+    ldT = (T + 7) // 8 * 8
+    ybuf = torch.empty(T * n_out + 8, dtype=torch.bfloat16, device="cuda")
+    y = ybuf[8:].view(T, n_out)  # 16 bytes past a 512-byte aligned allocation
+    assert y.data_ptr() % 32 == 16
+    u = torch.zeros((r, ldT), dtype=torch.bfloat16, device="cuda")
+    L.soup_lora_linear_fwd(Wd, Ad, Bd, r, s, xd, T, y, u)
+    dxbuf = torch.empty(T * n_in + 8, dtype=torch.bfloat16, device="cuda")
+    dx = dxbuf[8:].view(T, n_in)
+    dA = torch.empty((r, n_in), dtype=torch.float32, device="cuda")
+    dB = torch.empty((n_out, r), dtype=torch.float32, device="cuda")
+    ws = torch.empty(L.soup_lora_linear_bwd_workspace(T, r, n_out), dtype=torch.uint8, device="cuda")
+    L.soup_lora_linear_bwd(Wd, Ad, Bd, r, s, xd, u, dyd, T, dx, dA, dB, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(y), g["y"])
+    assert np.array_equal(host(dx), g["dx"])
+    assert np.array_equal(host(dA), g["dA"])
+    assert np.array_equal(host(dB), g["dB"])
